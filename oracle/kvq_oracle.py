@@ -1,0 +1,319 @@
+"""Plain CPU oracle for the asymmetric 2/4/8-bit KV cache and decode attention.
+
+TEST INFRASTRUCTURE ONLY. This module is a slow, literal restatement of the
+method so that the CUDA library can be checked against it. Only the test
+suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
+may import it; the library itself never does, and it shares no code, table or
+constant with the CUDA sources.
+
+Sources (web pages, cited by title and section):
+
+* "KV1-1.2B" model card, section "Quantization Format: KV1.cpp BQ2_0":
+  the affine quantizer -- scale ``d = fp16(max((max - min) / 3, 1e-6))``,
+  zero ``m = fp16(min)``, code ``q = clamp(round_half_to_even((x - m) / d), 0, 3)``
+  computed in fp32 with the fp16-rounded ``m`` and ``d``; dequantization
+  ``x_hat = q * d + m``; codes packed lowest bits first (``q0 | q1<<2 | ...``);
+  20 bytes per 64 values = 2.5 bits/value. Section "Memory": the per-token and
+  32K-context sizes.
+* "KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV Cache" (README),
+  sections "Overview" and "Example": keys quantized per channel, values per
+  token, 2 or 4 bits (``k_bits``, ``v_bits``), ``group_size``, and a window of
+  ``residual_length`` recent tokens kept in full precision; GQA support
+  (update of 2025.01.18).
+* "Quantize What Counts: More For Keys, Less For Values", section "KV Cache
+  Quantization": independent key and value bit widths, residual length and
+  group size per tensor; bit range up to 8.
+
+Readings taken where the pages are silent (each is listed with its reason in
+the design notes of the repository):
+
+1. The b-bit quantizer generalises the 2-bit rule by replacing 3 with 2^b - 1;
+   the 1e-6 floor on the scale applies at every width.
+2. The zero point is formed from ``min + 0.0`` so that a minimum of -0.0 is
+   stored as +0.0.
+3. Keys are grouped per (KV head, channel) over ``group_k`` consecutive tokens;
+   values per (token, KV head) over ``group_v`` consecutive channels.
+4. The residual window is a ring of exactly R slots. Appending a token to a
+   full ring first quantizes the oldest ``group_k`` tokens of the ring (keys
+   and values together). A multi-token append is the same sequence of
+   single-token appends. ``flush_residual`` quantizes every complete block of
+   ``group_k`` tokens still in the ring.
+5. Decode attention is ``softmax(scale * q K~^T) V~`` over every cached token
+   (no mask: the decode query is the newest position), where K~, V~ are the
+   dequantized values for quantized tokens and the exact stored values for the
+   residual window. Query head h reads KV head ``h // (Hq / Hkv)`` (GQA).
+   A sequence with no cached tokens yields a zero output.
+
+Floating point: the quantizer runs in IEEE fp32 (the precision the KV1 card
+fixes); numpy evaluates each fp32 operation with one rounding and never
+contracts a multiply-add. Attention runs in fp64.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+F32 = np.float32
+F16 = np.float16
+
+# ---------------------------------------------------------------------------
+# Quantizer ("KV1-1.2B", Quantization Format: KV1.cpp BQ2_0)
+# ---------------------------------------------------------------------------
+
+SCALE_FLOOR = F32(1e-6)
+
+
+def fp16_rn(x) -> np.ndarray:
+    """Round fp32 values to fp16, round-to-nearest-even (IEEE binary16)."""
+    return np.asarray(x, dtype=F32).astype(F16)
+
+
+def quantize_groups(x: np.ndarray, bits: int):
+    """Asymmetric min/max quantization of every group along the last axis.
+
+    ``x`` is fp32 with groups along its last axis. Returns ``(codes, d16, m16)``:
+    codes (uint8, same shape as ``x``) and the fp16 scale and zero point of
+    each group (shape ``x.shape[:-1]``).
+
+    Follows the BQ2_0 rule of the KV1 card with 3 replaced by ``2**bits - 1``:
+    ``d = fp16(max((max-min)/(2^b-1), 1e-6))``, ``m = fp16(min)``,
+    ``q = clamp(rint((x - m) / d), 0, 2^b-1)``, all in fp32, using the
+    fp16-rounded ``m`` and ``d``.
+    """
+    assert bits in (2, 4, 8)
+    x = np.asarray(x, dtype=F32)
+    qmax = (1 << bits) - 1
+    mn = x.min(axis=-1)
+    mx = x.max(axis=-1)
+    d = (mx - mn) / F32(qmax)                       # one fp32 division
+    d16 = fp16_rn(np.maximum(d, SCALE_FLOOR))
+    m16 = fp16_rn(mn + F32(0.0))
+    m32 = m16.astype(F32)[..., None]
+    d32 = d16.astype(F32)[..., None]
+    t = (x - m32) / d32                             # fp32 sub, then fp32 div
+    q = np.clip(np.rint(t), 0, qmax).astype(np.uint8)  # rint: ties to even
+    return q, d16, m16
+
+
+def dequantize(codes: np.ndarray, d16: np.ndarray, m16: np.ndarray) -> np.ndarray:
+    """``x_hat = q * d + m`` in fp32: a rounded product, then a rounded sum.
+
+    ``d16``/``m16`` must broadcast against ``codes``.
+    """
+    return codes.astype(F32) * d16.astype(F32) + m16.astype(F32)
+
+
+# ---------------------------------------------------------------------------
+# Bit packing ("KV1-1.2B", BQ2_0 block: q0 | q1<<2 | q2<<4 | q3<<6)
+# ---------------------------------------------------------------------------
+
+
+def pack_codes(codes: np.ndarray, bits: int) -> np.ndarray:
+    """Pack codes along the last axis into uint32 words, lowest bits first.
+
+    Code i of a run of ``32 // bits`` codes sits at bits ``[i*bits, (i+1)*bits)``.
+    """
+    per = 32 // bits
+    c = np.asarray(codes, dtype=np.uint64)
+    assert c.shape[-1] % per == 0
+    c = c.reshape(c.shape[:-1] + (c.shape[-1] // per, per))
+    shifts = (np.arange(per, dtype=np.uint64) * np.uint64(bits))
+    return (c << shifts).sum(axis=-1).astype(np.uint32)
+
+
+def unpack_codes(words: np.ndarray, bits: int) -> np.ndarray:
+    """Inverse of :func:`pack_codes`."""
+    per = 32 // bits
+    w = np.asarray(words, dtype=np.uint64)[..., None]
+    shifts = (np.arange(per, dtype=np.uint64) * np.uint64(bits))
+    c = (w >> shifts) & np.uint64((1 << bits) - 1)
+    return c.reshape(words.shape[:-1] + (words.shape[-1] * per,)).astype(np.uint8)
+
+
+# ---------------------------------------------------------------------------
+# KIVI axes: keys per channel over group_k tokens, values per token over
+# group_v channels ("KIVI" README, Overview)
+# ---------------------------------------------------------------------------
+
+
+def quantize_key_block(k: np.ndarray, bits: int):
+    """Keys of one block: ``k`` is [G, H, D] fp32 (G = group_k tokens).
+
+    Every (head, channel) is one group over the G tokens. Returns
+    codes [G, H, D], d16 [H, D], m16 [H, D].
+    """
+    q, d16, m16 = quantize_groups(np.transpose(k, (1, 2, 0)), bits)
+    return np.transpose(q, (2, 0, 1)), d16, m16
+
+
+def quantize_value_block(v: np.ndarray, bits: int, group_v: int):
+    """Values of one block: ``v`` is [G, H, D] fp32.
+
+    Every (token, head, run of ``group_v`` channels) is one group. Returns
+    codes [G, H, D], d16 [G, H, D/group_v], m16 [G, H, D/group_v].
+    """
+    G, H, D = v.shape
+    assert D % group_v == 0
+    q, d16, m16 = quantize_groups(v.reshape(G, H, D // group_v, group_v), bits)
+    return q.reshape(G, H, D), d16, m16
+
+
+def dequantize_key_block(codes, d16, m16):
+    return dequantize(codes, d16[None, :, :], m16[None, :, :])
+
+
+def dequantize_value_block(codes, d16, m16):
+    G, H, D = codes.shape
+    ng = d16.shape[-1]
+    c = codes.reshape(G, H, ng, D // ng)
+    return dequantize(c, d16[..., None], m16[..., None]).reshape(G, H, D)
+
+
+# Word arrangement of the library's packed block (documented in its header):
+# key words [H, G*bits/32, D] (word w of channel d holds tokens w*32/bits ...),
+# value words [H, G, D*bits/32] (word w of a token holds channels w*32/bits ...).
+
+
+def pack_key_block(codes: np.ndarray, bits: int) -> np.ndarray:
+    """codes [G, H, D] -> uint32 [H, G*bits/32, D], packed along tokens."""
+    words = pack_codes(np.transpose(codes, (1, 2, 0)), bits)   # [H, D, W]
+    return np.ascontiguousarray(np.transpose(words, (0, 2, 1)))
+
+
+def pack_value_block(codes: np.ndarray, bits: int) -> np.ndarray:
+    """codes [G, H, D] -> uint32 [H, G, D*bits/32], packed along channels."""
+    words = pack_codes(codes, bits)                              # [G, H, W]
+    return np.ascontiguousarray(np.transpose(words, (1, 0, 2)))
+
+
+# ---------------------------------------------------------------------------
+# Cache state machine (KIVI README: residual window of recent fp16 tokens)
+# ---------------------------------------------------------------------------
+
+
+class QuantizedBlock:
+    __slots__ = ("kc", "kd", "km", "vc", "vd", "vm")
+
+    def __init__(self, kc, kd, km, vc, vd, vm):
+        self.kc, self.kd, self.km, self.vc, self.vd, self.vm = kc, kd, km, vc, vd, vm
+
+
+class SequenceCache:
+    """KV cache of one sequence in one layer.
+
+    Token values are fp32 arrays holding values exactly representable in the
+    cache's storage type (fp16 or bf16); the ring keeps them unchanged.
+    """
+
+    def __init__(self, num_kv_heads, head_dim, k_bits, v_bits, group_k, group_v, residual):
+        assert residual % group_k == 0 and residual >= group_k
+        self.H, self.D = num_kv_heads, head_dim
+        self.k_bits, self.v_bits = k_bits, v_bits
+        self.group_k, self.group_v, self.residual = group_k, group_v, residual
+        self.blocks: list[QuantizedBlock] = []
+        self.ring_k: list[np.ndarray] = []   # oldest first, each [H, D]
+        self.ring_v: list[np.ndarray] = []
+
+    @property
+    def quantized_tokens(self) -> int:
+        return len(self.blocks) * self.group_k
+
+    @property
+    def residual_tokens(self) -> int:
+        return len(self.ring_k)
+
+    @property
+    def length(self) -> int:
+        return self.quantized_tokens + self.residual_tokens
+
+    def _flush_oldest_block(self):
+        G = self.group_k
+        k = np.stack(self.ring_k[:G]).astype(F32)
+        v = np.stack(self.ring_v[:G]).astype(F32)
+        del self.ring_k[:G]
+        del self.ring_v[:G]
+        kc, kd, km = quantize_key_block(k, self.k_bits)
+        vc, vd, vm = quantize_value_block(v, self.v_bits, self.group_v)
+        self.blocks.append(QuantizedBlock(kc, kd, km, vc, vd, vm))
+
+    def append_token(self, k: np.ndarray, v: np.ndarray):
+        """Append one token ([H, D] each); a full ring first flushes G tokens."""
+        if len(self.ring_k) == self.residual:
+            self._flush_oldest_block()
+        self.ring_k.append(np.asarray(k, dtype=F32).copy())
+        self.ring_v.append(np.asarray(v, dtype=F32).copy())
+
+    def append(self, k: np.ndarray, v: np.ndarray):
+        """Append T tokens ([T, H, D] each) as T single-token appends."""
+        for t in range(k.shape[0]):
+            self.append_token(k[t], v[t])
+
+    def flush_residual(self):
+        """Quantize every complete block of group_k tokens left in the ring."""
+        while len(self.ring_k) >= self.group_k:
+            self._flush_oldest_block()
+
+    def dequantized(self):
+        """(K~, V~) as fp32 [L, H, D]: dequantized blocks, then the ring."""
+        ks, vs = [], []
+        for b in self.blocks:
+            ks.append(dequantize_key_block(b.kc, b.kd, b.km))
+            vs.append(dequantize_value_block(b.vc, b.vd, b.vm))
+        if self.ring_k:
+            ks.append(np.stack(self.ring_k))
+            vs.append(np.stack(self.ring_v))
+        if not ks:
+            z = np.zeros((0, self.H, self.D), F32)
+            return z, z.copy()
+        return np.concatenate(ks).astype(F32), np.concatenate(vs).astype(F32)
+
+
+# ---------------------------------------------------------------------------
+# Decode attention (KIVI README: decoding phase; GQA)
+# ---------------------------------------------------------------------------
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.ndarray:
+    """softmax(scale * q k^T) v for one decode query per head, in fp64.
+
+    q [Hq, D]; k, v [L, Hkv, D]. Query head h uses KV head h // (Hq/Hkv).
+    Returns fp64 [Hq, D]; zeros when L == 0.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    Hq, D = q.shape
+    L, Hkv, _ = k.shape
+    assert Hq % Hkv == 0
+    g = Hq // Hkv
+    out = np.zeros((Hq, D), np.float64)
+    if L == 0:
+        return out
+    for h in range(Hq):
+        kv = h // g
+        s = scale * (k[:, kv, :] @ q[h])
+        p = np.exp(s - s.max())
+        out[h] = (p @ v[:, kv, :]) / p.sum()
+    return out
+
+
+def decode_attention(cache: SequenceCache, q: np.ndarray, scale: float) -> np.ndarray:
+    """Decode attention of one sequence over its quantized blocks and ring."""
+    k, v = cache.dequantized()
+    return attention(q, k, v, scale)
+
+
+# ---------------------------------------------------------------------------
+# Sizes ("KV1-1.2B", Memory; BQ2_0 block = 20 bytes per 64 values)
+# ---------------------------------------------------------------------------
+
+
+def quantized_bytes_per_token(num_kv_heads, head_dim, k_bits, v_bits, group_k, group_v) -> float:
+    """Bytes per cached token over all KV heads of one layer.
+
+    Codes take ``D*(bk+bv)/8`` bytes; each key group (one channel over group_k
+    tokens) and each value group (group_v channels of one token) adds an fp16
+    scale and an fp16 zero point, i.e. 4 bytes.
+    """
+    D = head_dim
+    return num_kv_heads * (D * (k_bits + v_bits) / 8 + 4 * D / group_k + 4 * D / group_v)

@@ -1,0 +1,360 @@
+"""Pins for the CPU oracle: hand-worked cases, closed forms, invariants and an
+independent attention routine. None of these call the CUDA library."""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import kvq_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _bits(h):
+    return int(np.asarray(h, dtype=np.float16).view(np.uint16))
+
+
+# --------------------------------------------------------------------------
+# fp16 rounding and the quantizer (KV1-1.2B card, BQ2_0)
+# --------------------------------------------------------------------------
+
+
+def test_fp16_rne_golden():
+    for c in _load("fp16_rne.json")["cases"]:
+        got = _bits(O.fp16_rn(np.float32(c["x"])))
+        assert got == int(c["bits"], 16), (c, hex(got))
+
+
+def test_quantizer_golden():
+    for c in _load("quantizer_cases.json")["cases"]:
+        x = np.array(c["x"], dtype=np.float32)
+        q, d16, m16 = O.quantize_groups(x, c["bits"])
+        assert q.tolist() == c["codes"], c["name"]
+        assert _bits(d16) == int(c["d16"], 16), (c["name"], hex(_bits(d16)))
+        assert _bits(m16) == int(c["m16"], 16), (c["name"], hex(_bits(m16)))
+        if "xhat" in c:
+            xh = O.dequantize(q, d16, m16)
+            assert xh.tolist() == c["xhat"], c["name"]
+
+
+def test_dequant_golden():
+    for c in _load("quantizer_cases.json")["dequant"]["cases"]:
+        d16 = np.array([int(c["d16"], 16)], np.uint16).view(np.float16)
+        m16 = np.array([int(c["m16"], 16)], np.uint16).view(np.float16)
+        xh = O.dequantize(np.array([c["q"]], np.uint8), d16, m16)
+        assert float(xh[0]) == c["xhat"], c
+
+
+def test_negative_zero_min_bits():
+    # A group whose minimum is -0.0 must store +0.0 whatever the scan order.
+    for x in ([-0.0, 0.0, 3.0], [0.0, -0.0, 3.0], [3.0, -0.0, -0.0]):
+        _, _, m16 = O.quantize_groups(np.array(x, np.float32), 2)
+        assert _bits(m16) == 0x0000
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_error_bound_exact_grid(bits):
+    # min = 0 and max = (2^b-1) * 2^e make m and d exact in fp16: error <= d/2.
+    rng = np.random.default_rng(bits)
+    qmax = (1 << bits) - 1
+    for e in range(-6, 5):
+        d = 2.0 ** e
+        x = rng.uniform(0, qmax * d, size=(64, 32)).astype(np.float32)
+        x[:, 0] = 0.0
+        x[:, 1] = qmax * d
+        q, d16, m16 = O.quantize_groups(x, bits)
+        assert np.all(d16.astype(np.float64) == d) and np.all(m16 == 0)
+        err = np.abs(O.dequantize(q, d16[:, None], m16[:, None]).astype(np.float64) - x)
+        assert err.max() <= d / 2 * (1 + 2 ** -20)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_error_bound_general(bits):
+    rng = np.random.default_rng(10 + bits)
+    qmax = (1 << bits) - 1
+    x = (rng.standard_normal((512, 64)) * np.exp(rng.standard_normal((512, 1)))).astype(np.float32)
+    q, d16, m16 = O.quantize_groups(x, bits)
+    mn = x.min(axis=1).astype(np.float64)
+    d = (x.max(axis=1).astype(np.float64) - mn) / qmax
+    d16f, m16f = d16.astype(np.float64), m16.astype(np.float64)
+    bound = d16f / 2 + np.abs(mn - m16f) + qmax * np.abs(d - d16f) + 4 * np.abs(x).max(axis=1) * 2.0 ** -23
+    xh = O.dequantize(q, d16[:, None], m16[:, None]).astype(np.float64)
+    assert np.all(np.abs(xh - x).max(axis=1) <= bound)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_code_is_nearest_level(bits):
+    # Brute force: the code is the nearest of the 2^b levels m + k d (exact
+    # arithmetic), except within a hair of a midpoint where fp32 rounding of
+    # t may legitimately go either way.
+    rng = np.random.default_rng(20 + bits)
+    qmax = (1 << bits) - 1
+    x = rng.standard_normal((256, 32)).astype(np.float32) * 3
+    q, d16, m16 = O.quantize_groups(x, bits)
+    levels = m16.astype(np.float64)[:, None, None] + d16.astype(np.float64)[:, None, None] * np.arange(qmax + 1)[None, None, :]
+    dist = np.abs(x.astype(np.float64)[:, :, None] - levels)
+    best = dist.argmin(axis=2)
+    t = (x.astype(np.float64) - m16.astype(np.float64)[:, None]) / d16.astype(np.float64)[:, None]
+    near_tie = np.abs(t - np.floor(t) - 0.5) < 1e-4
+    ok = (best == q) | near_tie
+    assert ok.all()
+    assert (np.abs(best.astype(int) - q.astype(int)) <= 1).all()
+
+
+# --------------------------------------------------------------------------
+# Packing (BQ2_0 bit order)
+# --------------------------------------------------------------------------
+
+
+def test_pack_golden():
+    for c in _load("pack_cases.json")["cases"]:
+        w = O.pack_codes(np.array(c["codes"], np.uint8), c["bits"])
+        assert w.tolist() == [int(c["word"], 16)], c
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_pack_roundtrip_and_positions(bits):
+    rng = np.random.default_rng(bits)
+    per = 32 // bits
+    codes = rng.integers(0, 1 << bits, size=(7, 5, per * 3)).astype(np.uint8)
+    words = O.pack_codes(codes, bits)
+    assert words.shape == (7, 5, 3)
+    assert np.array_equal(O.unpack_codes(words, bits), codes)
+    # each code read back with an explicit shift and mask
+    for i in range(per * 3):
+        w = words[..., i // per].astype(np.uint64)
+        assert np.array_equal((w >> np.uint64((i % per) * bits)) & np.uint64((1 << bits) - 1), codes[..., i])
+
+
+def test_block_word_arrangement():
+    # Key words run along tokens for a fixed channel; value words along channels
+    # for a fixed token.
+    G, H, D, b = 32, 2, 32, 2
+    rng = np.random.default_rng(0)
+    codes = rng.integers(0, 4, size=(G, H, D)).astype(np.uint8)
+    kw = O.pack_key_block(codes, b)
+    assert kw.shape == (H, G * b // 32, D)
+    for h, w, d in [(0, 0, 0), (1, 1, 31), (0, 1, 7)]:
+        assert np.array_equal(O.unpack_codes(kw[h, w, d][None], b), codes[w * 16:(w + 1) * 16, h, d])
+    vw = O.pack_value_block(codes, b)
+    assert vw.shape == (H, G, D * b // 32)
+    for h, t, w in [(0, 0, 0), (1, 31, 1), (1, 5, 0)]:
+        assert np.array_equal(O.unpack_codes(vw[h, t, w][None], b), codes[t, h, w * 16:(w + 1) * 16])
+
+
+# --------------------------------------------------------------------------
+# KIVI axes: keys per channel, values per token
+# --------------------------------------------------------------------------
+
+
+def test_key_axis_is_per_channel():
+    # An outlier channel must not degrade the other channels of the same tokens.
+    rng = np.random.default_rng(3)
+    k = rng.standard_normal((64, 2, 16)).astype(np.float32)
+    k[:, :, 5] *= 1000.0
+    codes, d16, m16 = O.quantize_key_block(k, 2)
+    err = np.abs(O.dequantize_key_block(codes, d16, m16) - k)
+    normal = np.delete(err, 5, axis=2)
+    assert normal.max() < 2.0          # ~range/6 of an N(0,1) channel, not ~1000/6
+    assert d16.shape == (2, 16) and codes.shape == k.shape
+
+
+def test_value_axis_is_per_token():
+    rng = np.random.default_rng(4)
+    v = rng.standard_normal((8, 2, 64)).astype(np.float32)
+    v[3] *= 1000.0
+    codes, d16, m16 = O.quantize_value_block(v, 4, 32)
+    err = np.abs(O.dequantize_value_block(codes, d16, m16) - v)
+    assert np.delete(err, 3, axis=0).max() < 0.5
+    assert d16.shape == (8, 2, 2)
+
+
+# --------------------------------------------------------------------------
+# Cache state machine (residual ring, flush of group_k tokens)
+# --------------------------------------------------------------------------
+
+
+def _expected_split(L, R, G):
+    q = 0 if L <= R else G * math.ceil((L - R) / G)
+    return q, L - q
+
+
+@pytest.mark.parametrize("R,G", [(32, 32), (128, 32), (128, 64), (128, 128), (64, 64), (96, 32)])
+def test_state_machine_counts(R, G):
+    H, D = 1, 16
+    c = O.SequenceCache(H, D, 2, 2, G, 16, R)
+    rng = np.random.default_rng(R + G)
+    for L in range(1, 3 * R + 5):
+        c.append_token(rng.standard_normal((H, D)), rng.standard_normal((H, D)))
+        q, n = _expected_split(L, R, G)
+        assert (c.quantized_tokens, c.residual_tokens) == (q, n), L
+        assert c.quantized_tokens % G == 0 and 0 < c.residual_tokens <= R
+
+
+@pytest.mark.parametrize("L,R,G,expect", [(1024, 32, 32, (992, 32)), (4096, 128, 32, (3968, 128)),
+                                          (4352, 128, 32, (4224, 128)), (8192, 128, 64, (8064, 128)),
+                                          (131072, 128, 128, (130944, 128)), (4096, 128, 128, (3968, 128))])
+def test_state_machine_table(L, R, G, expect):
+    assert _expected_split(L, R, G) == expect
+    # and the oracle agrees on a cheap instance (single head, 16 channels)
+    c = O.SequenceCache(1, 16, 2, 2, G, 16, R)
+    z = np.zeros((L, 1, 16), np.float32)
+    c.append(z, z)
+    assert (c.quantized_tokens, c.residual_tokens) == expect
+
+
+def test_ring_and_blocks_hold_the_right_tokens():
+    H, D, G, R = 2, 32, 32, 64
+    rng = np.random.default_rng(7)
+    L = 5 * G + 17
+    k = rng.standard_normal((L, H, D)).astype(np.float32)
+    v = rng.standard_normal((L, H, D)).astype(np.float32)
+    c = O.SequenceCache(H, D, 2, 4, G, 32, R)
+    c.append(k, v)
+    Q = c.quantized_tokens
+    assert np.array_equal(np.stack(c.ring_k), k[Q:]) and np.array_equal(np.stack(c.ring_v), v[Q:])
+    K, V = c.dequantized()
+    assert K.shape == (L, H, D)
+    for j in range(Q // G):
+        blk = slice(j * G, (j + 1) * G)
+        kr = k[blk]
+        rngk = kr.max(axis=0) - kr.min(axis=0)
+        assert np.all(np.abs(K[blk] - kr) <= rngk / 6 * 1.01 + 1e-3)
+        vr = v[blk].reshape(G, H, 1, 32)
+        rngv = (vr.max(axis=3) - vr.min(axis=3))[..., None]
+        assert np.all(np.abs(V[blk].reshape(G, H, 1, 32) - vr) <= rngv / 30 * 1.01 + 1e-3)
+
+
+def test_chunked_append_equals_single_call():
+    H, D, G, R = 2, 32, 32, 64
+    rng = np.random.default_rng(8)
+    L = 300
+    k = rng.standard_normal((L, H, D)).astype(np.float32)
+    v = rng.standard_normal((L, H, D)).astype(np.float32)
+    a = O.SequenceCache(H, D, 2, 2, G, 32, R)
+    a.append(k, v)
+    b = O.SequenceCache(H, D, 2, 2, G, 32, R)
+    pos = 0
+    for n in [1, 63, 2, 100, 1, 1, 132]:
+        b.append(k[pos:pos + n], v[pos:pos + n])
+        pos += n
+    assert pos == L
+    Ka, Va = a.dequantized()
+    Kb, Vb = b.dequantized()
+    assert np.array_equal(Ka, Kb) and np.array_equal(Va, Vb)
+
+
+def test_flush_residual():
+    H, D, G, R = 1, 16, 32, 128
+    c = O.SequenceCache(H, D, 2, 2, G, 16, R)
+    z = np.ones((100, H, D), np.float32)
+    c.append(z, z)
+    assert (c.quantized_tokens, c.residual_tokens) == (0, 100)
+    c.flush_residual()
+    assert (c.quantized_tokens, c.residual_tokens) == (96, 4)
+    c.flush_residual()
+    assert (c.quantized_tokens, c.residual_tokens) == (96, 4)
+
+
+# --------------------------------------------------------------------------
+# Attention: hand example, closed forms, and an independent library routine
+# --------------------------------------------------------------------------
+
+
+def _sdpa(q, k, v, scale):
+    """torch scaled_dot_product_attention in fp64; q [Hq,D], k/v [L,Hkv,D]."""
+    Hq = q.shape[0]
+    Hkv = k.shape[1]
+    kk = torch.from_numpy(np.asarray(k, np.float64)).permute(1, 0, 2).repeat_interleave(Hq // Hkv, 0)
+    vv = torch.from_numpy(np.asarray(v, np.float64)).permute(1, 0, 2).repeat_interleave(Hq // Hkv, 0)
+    qq = torch.from_numpy(np.asarray(q, np.float64))[:, None, :]
+    o = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, scale=scale)
+    return o[:, 0, :].numpy()
+
+
+def test_attention_hand_example():
+    # scores ln3 and 0 -> weights 3/4, 1/4 -> o = 3/4 [4,0] + 1/4 [0,8] = [3,2]
+    q = np.array([[1.0, 0.0]])
+    k = np.array([[[math.log(3.0), 0.0]], [[0.0, 0.0]]])
+    v = np.array([[[4.0, 0.0]], [[0.0, 8.0]]])
+    o = O.attention(q, k, v, 1.0)
+    assert np.allclose(o, [[3.0, 2.0]], atol=1e-14)
+
+
+def test_attention_closed_forms():
+    rng = np.random.default_rng(11)
+    k = rng.standard_normal((50, 2, 8))
+    v = rng.standard_normal((50, 2, 8))
+    o = O.attention(np.zeros((4, 8)), k, v, 0.3)          # uniform weights
+    assert np.allclose(o[0], v[:, 0].mean(0), atol=1e-14) and np.allclose(o[3], v[:, 1].mean(0), atol=1e-14)
+    o1 = O.attention(rng.standard_normal((2, 8)), k[:1], v[:1], 0.3)   # one token
+    assert np.allclose(o1, v[0], atol=1e-15)
+    assert np.array_equal(O.attention(np.ones((2, 8)), k[:0], v[:0], 1.0), np.zeros((2, 8)))
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 2), (32, 8)])
+def test_attention_matches_sdpa(Hq, Hkv):
+    rng = np.random.default_rng(Hq + Hkv)
+    D, L = 16, 77
+    q = rng.standard_normal((Hq, D))
+    k = rng.standard_normal((L, Hkv, D)) * 2
+    v = rng.standard_normal((L, Hkv, D))
+    assert np.abs(O.attention(q, k, v, 0.25) - _sdpa(q, k, v, 0.25)).max() < 1e-12
+
+
+def test_residual_only_cache_is_exact_attention():
+    H, D, G, R = 2, 32, 32, 128
+    rng = np.random.default_rng(12)
+    k = rng.standard_normal((90, H, D)).astype(np.float32)
+    v = rng.standard_normal((90, H, D)).astype(np.float32)
+    c = O.SequenceCache(H, D, 2, 2, G, 32, R)
+    c.append(k, v)
+    assert c.quantized_tokens == 0
+    q = rng.standard_normal((8, D))
+    assert np.abs(O.decode_attention(c, q, D ** -0.5) - _sdpa(q, k, v, D ** -0.5)).max() < 1e-12
+
+
+def test_quantized_cache_attention_matches_sdpa_on_dequantized():
+    H, D, G, R = 2, 64, 32, 64
+    rng = np.random.default_rng(13)
+    L = 333
+    k = rng.standard_normal((L, H, D)).astype(np.float32)
+    v = rng.standard_normal((L, H, D)).astype(np.float32)
+    c = O.SequenceCache(H, D, 2, 4, G, 32, R)
+    c.append(k, v)
+    K, V = c.dequantized()
+    q = rng.standard_normal((8, D))
+    o = O.decode_attention(c, q, D ** -0.5)
+    assert np.abs(o - _sdpa(q, K, V, D ** -0.5)).max() < 1e-12
+    # and the quantized result stays near exact attention on the raw inputs
+    assert np.abs(o - _sdpa(q, k, v, D ** -0.5)).max() < 0.5
+
+
+# --------------------------------------------------------------------------
+# Sizes (KV1-1.2B card, Memory)
+# --------------------------------------------------------------------------
+
+
+def test_kv1_memory_table():
+    t = _load("kv1_memory_table.json")
+    m = t["model"]
+    per_value = O.quantized_bytes_per_token(1, 64, 2, 2, 64, 64) * 8 / 128
+    assert per_value == t["bits_per_value_bq2_0"]
+    for row in t["rows"]:
+        if row["bits"] == 16:
+            per_tok = m["attention_layers"] * m["kv_heads"] * m["head_dim"] * 2 * 2
+        else:
+            per_tok = m["attention_layers"] * O.quantized_bytes_per_token(
+                m["kv_heads"], m["head_dim"], row["bits"], row["bits"], m["group"], m["group"])
+        assert round(per_tok / 1024, 1) == row["per_token_kib"], row
+        assert round(per_tok * 8192 / 2 ** 20) == row["ctx_8k_mib"], row
+        assert round(per_tok * 32768 / 2 ** 20) == row["ctx_32k_mib"], row
