@@ -1,0 +1,422 @@
+// Host side of the C ABI declared in include/kvq.h: argument validation, the
+// arena plan, the host mirror of sequence lengths, the flush planner and the
+// split planner. All device work is enqueued by the launchers of
+// kvq_append.cu and kvq_decode.cu.
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "kvq_append.cuh"
+#include "kvq_decode.cuh"
+
+struct kvq_cache {
+  kvq_config cfg;                 // k_bits / v_bits point at the vectors below
+  std::vector<int8_t> k_bits, v_bits;
+  uint8_t* arena;
+  size_t arena_bytes;
+  int device;
+  // per layer
+  std::vector<int64_t> blocks_off, ring_k_off, ring_v_off, record_bytes;
+  int64_t max_blocks;
+  int64_t lens_off;               // int32 [num_layers][max_batch][2]
+  int64_t ws_o_off, ws_ml_off;    // split partials
+  int32_t slots;                  // partial slots per (sequence, query head)
+  std::vector<int32_t> q_len, n_len;  // host mirror [num_layers][max_batch]
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+kvq_status fail(kvq_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+kvq_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(KVQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool is_group(int g) { return g == 32 || g == 64 || g == 128; }
+bool is_bits(int b) { return b == 2 || b == 4 || b == 8; }
+
+kvq_status validate_config(const kvq_config* c) {
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "config is null");
+  if (c->num_layers < 1 || c->num_layers > KVQ_MAX_LAYERS)
+    return fail(KVQ_ERR_INVALID_ARG, "num_layers %d outside 1..%d", c->num_layers, KVQ_MAX_LAYERS);
+  if (c->max_batch < 1 || c->max_batch > KVQ_MAX_BATCH)
+    return fail(KVQ_ERR_INVALID_ARG, "max_batch %d outside 1..%d", c->max_batch, KVQ_MAX_BATCH);
+  if (c->num_kv_heads < 1 || c->num_q_heads < 1 || c->num_q_heads % c->num_kv_heads != 0)
+    return fail(KVQ_ERR_INVALID_ARG, "num_q_heads %d must be a positive multiple of num_kv_heads %d",
+                c->num_q_heads, c->num_kv_heads);
+  const int g = c->num_q_heads / c->num_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8)
+    return fail(KVQ_ERR_UNSUPPORTED, "query heads per KV head %d not in {1,2,4,8}", g);
+  if (c->head_dim != kvq::kHeadDim)
+    return fail(KVQ_ERR_UNSUPPORTED, "head_dim %d: only %d is built", c->head_dim, kvq::kHeadDim);
+  if (!is_group(c->group_k)) return fail(KVQ_ERR_UNSUPPORTED, "group_k %d not in {32,64,128}", c->group_k);
+  if (!is_group(c->group_v) || c->head_dim % c->group_v != 0)
+    return fail(KVQ_ERR_UNSUPPORTED, "group_v %d not in {32,64,128} or not dividing head_dim", c->group_v);
+  if (c->residual < c->group_k || c->residual % c->group_k != 0)
+    return fail(KVQ_ERR_INVALID_ARG, "residual %d must be a positive multiple of group_k %d", c->residual,
+                c->group_k);
+  if (c->max_tokens < 1) return fail(KVQ_ERR_INVALID_ARG, "max_tokens %d < 1", c->max_tokens);
+  if (c->kv_dtype != KVQ_F16 && c->kv_dtype != KVQ_BF16)
+    return fail(KVQ_ERR_UNSUPPORTED, "kv_dtype %d: only F16 and BF16", c->kv_dtype);
+  if (!c->k_bits || !c->v_bits) return fail(KVQ_ERR_INVALID_ARG, "k_bits / v_bits is null");
+  for (int l = 0; l < c->num_layers; ++l)
+    if (!is_bits(c->k_bits[l]) || !is_bits(c->v_bits[l]))
+      return fail(KVQ_ERR_UNSUPPORTED, "layer %d bits k=%d v=%d not in {2,4,8}", l, c->k_bits[l], c->v_bits[l]);
+  return KVQ_OK;
+}
+
+struct Plan {
+  std::vector<int64_t> blocks_off, ring_k_off, ring_v_off, record_bytes;
+  int64_t max_blocks, lens_off, ws_o_off, ws_ml_off, total;
+  int32_t slots;
+};
+
+Plan make_plan(const kvq_config* c) {
+  using kvq::round_up;
+  Plan p;
+  const int G = c->group_k, D = c->head_dim;
+  const int64_t seqheads = (int64_t)c->max_batch * c->num_kv_heads;
+  p.max_blocks = c->max_tokens / G;
+  int64_t off = 0;
+  for (int l = 0; l < c->num_layers; ++l) {
+    const int kb = c->k_bits[l], vb = c->v_bits[l];
+    const int64_t rec = round_up(kvq::kc_bytes(G, D, kb) + kvq::ksz_bytes(D) + kvq::vc_bytes(G, D, vb) +
+                                     kvq::vsz_bytes(G, D, c->group_v),
+                                 16);
+    p.record_bytes.push_back(rec);
+    p.blocks_off.push_back(off);
+    off = round_up(off + seqheads * p.max_blocks * rec, 256);
+    const int64_t ring = seqheads * c->residual * D * 2;
+    p.ring_k_off.push_back(off);
+    off = round_up(off + ring, 256);
+    p.ring_v_off.push_back(off);
+    off = round_up(off + ring, 256);
+  }
+  p.lens_off = off;
+  off = round_up(off + (int64_t)c->num_layers * c->max_batch * 2 * 4, 256);
+  p.slots = (int32_t)std::min<int64_t>(p.max_blocks, KVQ_MAX_SPLITS) + 1;
+  const int64_t partials = (int64_t)c->max_batch * c->num_q_heads * p.slots;
+  p.ws_o_off = off;
+  off = round_up(off + partials * D * 4, 256);
+  p.ws_ml_off = off;
+  off = round_up(off + partials * 8, 256);
+  p.total = off;
+  return p;
+}
+
+kvq::LayerView layer_view(const kvq_cache* c, int layer) {
+  kvq::LayerView v;
+  const kvq_config& cfg = c->cfg;
+  const int G = cfg.group_k, D = cfg.head_dim;
+  const int kb = c->k_bits[layer], vb = c->v_bits[layer];
+  v.blocks = c->arena + c->blocks_off[layer];
+  v.ring_k = c->arena + c->ring_k_off[layer];
+  v.ring_v = c->arena + c->ring_v_off[layer];
+  v.lens = reinterpret_cast<int32_t*>(c->arena + c->lens_off) + (int64_t)layer * cfg.max_batch * 2;
+  v.record_bytes = c->record_bytes[layer];
+  v.max_blocks = c->max_blocks;
+  v.kc_off = 0;
+  v.ksz_off = (int32_t)kvq::kc_bytes(G, D, kb);
+  v.vc_off = v.ksz_off + (int32_t)kvq::ksz_bytes(D);
+  v.vsz_off = v.vc_off + (int32_t)kvq::vc_bytes(G, D, vb);
+  v.k_bits = kb;
+  v.v_bits = vb;
+  v.num_kv_heads = cfg.num_kv_heads;
+  v.head_dim = D;
+  v.group_k = G;
+  v.group_v = cfg.group_v;
+  v.residual = cfg.residual;
+  v.kv_dtype = cfg.kv_dtype;
+  return v;
+}
+
+kvq_status check_cache_layer(const kvq_cache* c, int layer) {
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "cache is null");
+  if (layer < 0 || layer >= c->cfg.num_layers)
+    return fail(KVQ_ERR_INVALID_ARG, "layer %d outside 0..%d", layer, c->cfg.num_layers - 1);
+  return KVQ_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shared by kvq_append (t_new from the caller) and kvq_flush_residual
+// (t_new = 0, every complete group of the ring flushed).
+kvq_status enqueue_append(kvq_cache* c, int layer, const void* k, const void* v, const int32_t* new_lens,
+                          int batch, bool flush_all, cudaStream_t stream) {
+  const kvq_config& cfg = c->cfg;
+  const int G = cfg.group_k, R = cfg.residual;
+  kvq::AppendParams* p = new (std::nothrow) kvq::AppendParams;
+  if (!p) return fail(KVQ_ERR_INVALID_ARG, "out of host memory");
+  std::memset(p, 0, sizeof *p);
+  p->L = layer_view(c, layer);
+  p->k_in = k;
+  p->v_in = v;
+  p->batch = batch;
+  int32_t* ql = &c->q_len[(size_t)layer * cfg.max_batch];
+  int32_t* nl = &c->n_len[(size_t)layer * cfg.max_batch];
+  int max_flush = 0;
+  int64_t off = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int T = flush_all ? 0 : new_lens[b];
+    int f;
+    if (flush_all) f = nl[b] / G;
+    else f = (nl[b] + T <= R) ? 0 : (nl[b] + T - R + G - 1) / G;
+    p->q_old[b] = ql[b];
+    p->n_old[b] = nl[b];
+    p->t_new[b] = T;
+    p->in_off[b] = (int32_t)off;
+    p->flush[b] = f;
+    off += T;
+    if (f > max_flush) max_flush = f;
+  }
+  cudaError_t e = kvq::launch_append(*p, max_flush, stream);
+  if (e == cudaSuccess) {
+    for (int b = 0; b < batch; ++b) {
+      const int qn = p->q_old[b] + p->flush[b] * G;
+      const int end = p->q_old[b] + p->n_old[b] + p->t_new[b];
+      ql[b] = qn;
+      nl[b] = end - qn;
+    }
+  }
+  delete p;
+  if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KVQ_ERR_CAPACITY: return "sequence capacity exceeded";
+    case KVQ_ERR_WORKSPACE: return "arena too small";
+    case KVQ_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char* kvq_last_error(void) { return g_last_error.c_str(); }
+
+kvq_status kvq_cache_required_bytes(const kvq_config* cfg, size_t* bytes) {
+  g_last_error.clear();
+  kvq_status s = validate_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (!bytes) return fail(KVQ_ERR_INVALID_ARG, "bytes is null");
+  *bytes = (size_t)make_plan(cfg).total;
+  return KVQ_OK;
+}
+
+kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena_bytes, kvq_cache** out) {
+  g_last_error.clear();
+  kvq_status s = validate_config(cfg);
+  if (s != KVQ_OK) return s;
+  if (!out) return fail(KVQ_ERR_INVALID_ARG, "out is null");
+  if (!dev_arena) return fail(KVQ_ERR_INVALID_ARG, "arena is null");
+  if (reinterpret_cast<uintptr_t>(dev_arena) & 255u) return fail(KVQ_ERR_INVALID_ARG, "arena not 256-byte aligned");
+  Plan plan = make_plan(cfg);
+  if ((int64_t)arena_bytes < plan.total)
+    return fail(KVQ_ERR_WORKSPACE, "arena %zu bytes < required %lld", arena_bytes, (long long)plan.total);
+  kvq_cache* c = new (std::nothrow) kvq_cache;
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "out of host memory");
+  c->cfg = *cfg;
+  c->k_bits.assign(cfg->k_bits, cfg->k_bits + cfg->num_layers);
+  c->v_bits.assign(cfg->v_bits, cfg->v_bits + cfg->num_layers);
+  c->cfg.k_bits = c->k_bits.data();
+  c->cfg.v_bits = c->v_bits.data();
+  c->arena = static_cast<uint8_t*>(dev_arena);
+  c->arena_bytes = arena_bytes;
+  c->blocks_off = plan.blocks_off;
+  c->ring_k_off = plan.ring_k_off;
+  c->ring_v_off = plan.ring_v_off;
+  c->record_bytes = plan.record_bytes;
+  c->max_blocks = plan.max_blocks;
+  c->lens_off = plan.lens_off;
+  c->ws_o_off = plan.ws_o_off;
+  c->ws_ml_off = plan.ws_ml_off;
+  c->slots = plan.slots;
+  c->q_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
+  c->n_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
+  cudaError_t e = cudaGetDevice(&c->device);
+  if (e == cudaSuccess) e = cudaMemset(c->arena + c->lens_off, 0, (size_t)cfg->num_layers * cfg->max_batch * 8);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    delete c;
+    return cuda_fail(e, "zeroing the length table");
+  }
+  *out = c;
+  return KVQ_OK;
+}
+
+kvq_status kvq_cache_destroy(kvq_cache* c) {
+  g_last_error.clear();
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "cache is null");
+  delete c;
+  return KVQ_OK;
+}
+
+kvq_status kvq_cache_reset(kvq_cache* c, void* stream) {
+  g_last_error.clear();
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "cache is null");
+  cudaError_t e = cudaMemsetAsync(c->arena + c->lens_off, 0, (size_t)c->cfg.num_layers * c->cfg.max_batch * 8,
+                                  static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "reset");
+  std::fill(c->q_len.begin(), c->q_len.end(), 0);
+  std::fill(c->n_len.begin(), c->n_len.end(), 0);
+  return KVQ_OK;
+}
+
+kvq_status kvq_append(kvq_cache* c, int32_t layer, const void* k, const void* v, const int32_t* new_lens,
+                      int32_t batch, void* stream) {
+  g_last_error.clear();
+  kvq_status s = check_cache_layer(c, layer);
+  if (s != KVQ_OK) return s;
+  if (batch < 0 || batch > c->cfg.max_batch)
+    return fail(KVQ_ERR_INVALID_ARG, "batch %d outside 0..%d", batch, c->cfg.max_batch);
+  if (batch > 0 && !new_lens) return fail(KVQ_ERR_INVALID_ARG, "new_lens is null");
+  int64_t total = 0;
+  for (int b = 0; b < batch; ++b) {
+    if (new_lens[b] < 0) return fail(KVQ_ERR_INVALID_ARG, "new_lens[%d] = %d < 0", b, new_lens[b]);
+    const int64_t L = (int64_t)c->q_len[(size_t)layer * c->cfg.max_batch + b] +
+                      c->n_len[(size_t)layer * c->cfg.max_batch + b] + new_lens[b];
+    if (L > c->cfg.max_tokens)
+      return fail(KVQ_ERR_CAPACITY, "sequence %d would hold %lld tokens > max_tokens %d", b, (long long)L,
+                  c->cfg.max_tokens);
+    total += new_lens[b];
+  }
+  if (total > INT32_MAX) return fail(KVQ_ERR_INVALID_ARG, "more than 2^31-1 tokens in one call");
+  if (total > 0) {
+    if (!k || !v) return fail(KVQ_ERR_INVALID_ARG, "k or v is null");
+    if (!aligned16(k) || !aligned16(v)) return fail(KVQ_ERR_INVALID_ARG, "k and v must be 16-byte aligned");
+  }
+  if (batch == 0) return KVQ_OK;
+  return enqueue_append(c, layer, k, v, new_lens, batch, false, static_cast<cudaStream_t>(stream));
+}
+
+kvq_status kvq_flush_residual(kvq_cache* c, int32_t layer, int32_t batch, void* stream) {
+  g_last_error.clear();
+  kvq_status s = check_cache_layer(c, layer);
+  if (s != KVQ_OK) return s;
+  if (batch < 0 || batch > c->cfg.max_batch)
+    return fail(KVQ_ERR_INVALID_ARG, "batch %d outside 0..%d", batch, c->cfg.max_batch);
+  if (batch == 0) return KVQ_OK;
+  return enqueue_append(c, layer, nullptr, nullptr, nullptr, batch, true, static_cast<cudaStream_t>(stream));
+}
+
+kvq_status kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, void* out, int32_t out_dtype,
+                                float softmax_scale, int32_t batch, void* stream) {
+  g_last_error.clear();
+  kvq_status s = check_cache_layer(c, layer);
+  if (s != KVQ_OK) return s;
+  if (batch < 0 || batch > c->cfg.max_batch)
+    return fail(KVQ_ERR_INVALID_ARG, "batch %d outside 0..%d", batch, c->cfg.max_batch);
+  if (out_dtype != KVQ_F32 && out_dtype != KVQ_F16 && out_dtype != KVQ_BF16)
+    return fail(KVQ_ERR_INVALID_ARG, "out_dtype %d", out_dtype);
+  if (!std::isfinite(softmax_scale)) return fail(KVQ_ERR_INVALID_ARG, "softmax_scale is not finite");
+  if (batch == 0) return KVQ_OK;
+  if (!q || !out) return fail(KVQ_ERR_INVALID_ARG, "q or out is null");
+  if (!aligned16(q) || !aligned16(out)) return fail(KVQ_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+  const kvq_config& cfg = c->cfg;
+  const int G = cfg.group_k;
+  // Split plan: enough quantized splits to give every SM several CTAs.
+  int64_t total_blocks = 0;
+  int max_blk = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int nb = c->q_len[(size_t)layer * cfg.max_batch + b] / G;
+    total_blocks += nb;
+    if (nb > max_blk) max_blk = nb;
+  }
+  const int64_t target_ctas = 148 * 4;
+  int64_t bps = (total_blocks * cfg.num_kv_heads + target_ctas - 1) / target_ctas;
+  if (bps < 1) bps = 1;
+  const int64_t min_bps = (max_blk + (c->slots - 1) - 1) / (c->slots - 1);
+  if (bps < min_bps) bps = min_bps;
+  const int max_splits = (int)((max_blk + bps - 1) / bps);
+  kvq::DecodeParams p;
+  p.L = layer_view(c, layer);
+  p.q = q;
+  p.out = out;
+  p.ws_o = reinterpret_cast<float*>(c->arena + c->ws_o_off);
+  p.ws_ml = reinterpret_cast<float2*>(c->arena + c->ws_ml_off);
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.out_dtype = out_dtype;
+  p.batch = batch;
+  p.num_q_heads = cfg.num_q_heads;
+  p.blocks_per_split = (int32_t)bps;
+  p.slots = c->slots;
+  cudaError_t e = kvq::launch_decode(p, max_splits, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return KVQ_OK;
+}
+
+kvq_status kvq_dequant(kvq_cache* c, int32_t layer, int32_t seq, int32_t t0, int32_t t1, float* k_out,
+                       float* v_out, void* stream) {
+  g_last_error.clear();
+  kvq_status s = check_cache_layer(c, layer);
+  if (s != KVQ_OK) return s;
+  if (seq < 0 || seq >= c->cfg.max_batch) return fail(KVQ_ERR_INVALID_ARG, "seq %d out of range", seq);
+  const size_t i = (size_t)layer * c->cfg.max_batch + seq;
+  const int L = c->q_len[i] + c->n_len[i];
+  if (t0 < 0 || t0 > t1 || t1 > L)
+    return fail(KVQ_ERR_INVALID_ARG, "token range [%d,%d) outside [0,%d]", t0, t1, L);
+  if (t1 == t0) return KVQ_OK;
+  if (!k_out || !v_out) return fail(KVQ_ERR_INVALID_ARG, "k_out or v_out is null");
+  cudaError_t e = kvq::launch_dequant(layer_view(c, layer), seq, t0, t1, k_out, v_out,
+                                      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "dequant launch");
+  return KVQ_OK;
+}
+
+kvq_status kvq_get_layout(const kvq_cache* c, int32_t layer, kvq_layout* out) {
+  g_last_error.clear();
+  kvq_status s = check_cache_layer(c, layer);
+  if (s != KVQ_OK) return s;
+  if (!out) return fail(KVQ_ERR_INVALID_ARG, "out is null");
+  const kvq::LayerView v = layer_view(c, layer);
+  out->blocks = v.blocks;
+  out->record_bytes = v.record_bytes;
+  out->max_blocks = v.max_blocks;
+  out->kc_offset = v.kc_off;
+  out->ksz_offset = v.ksz_off;
+  out->vc_offset = v.vc_off;
+  out->vsz_offset = v.vsz_off;
+  out->ring_k = v.ring_k;
+  out->ring_v = v.ring_v;
+  out->k_bits = v.k_bits;
+  out->v_bits = v.v_bits;
+  return KVQ_OK;
+}
+
+kvq_status kvq_seq_lengths(const kvq_cache* c, int32_t layer, int32_t seq, int32_t* quantized,
+                           int32_t* residual) {
+  g_last_error.clear();
+  kvq_status s = check_cache_layer(c, layer);
+  if (s != KVQ_OK) return s;
+  if (seq < 0 || seq >= c->cfg.max_batch) return fail(KVQ_ERR_INVALID_ARG, "seq %d out of range", seq);
+  if (!quantized || !residual) return fail(KVQ_ERR_INVALID_ARG, "output pointer is null");
+  const size_t i = (size_t)layer * c->cfg.max_batch + seq;
+  *quantized = c->q_len[i];
+  *residual = c->n_len[i];
+  return KVQ_OK;
+}
+
+}  // extern "C"

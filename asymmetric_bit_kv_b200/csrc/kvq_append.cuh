@@ -1,0 +1,28 @@
+// Parameters and launchers of the append / flush / dequantize kernels.
+#pragma once
+
+#include "kvq_internal.cuh"
+
+namespace kvq {
+
+constexpr int kQuantThreads = 128;
+
+// Per-call append plan, passed by value (kernel parameter space up to 32 KB).
+// Lengths are the host mirror's values before the call.
+struct AppendParams {
+  LayerView L;
+  const void* k_in;  // [sum t_new][Hkv][D], kv dtype
+  const void* v_in;
+  int32_t batch;
+  int32_t q_old[KVQ_MAX_BATCH];   // quantized tokens before the call
+  int32_t n_old[KVQ_MAX_BATCH];   // ring tokens before the call
+  int32_t t_new[KVQ_MAX_BATCH];   // tokens appended by the call
+  int32_t in_off[KVQ_MAX_BATCH];  // first input row of each sequence
+  int32_t flush[KVQ_MAX_BATCH];   // G-token blocks quantized by the call
+};
+
+cudaError_t launch_append(const AppendParams& p, int max_flush, cudaStream_t stream);
+cudaError_t launch_dequant(const LayerView& L, int seq, int t0, int t1, float* k_out, float* v_out,
+                           cudaStream_t stream);
+
+}  // namespace kvq

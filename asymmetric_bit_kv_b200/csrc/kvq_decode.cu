@@ -1,0 +1,228 @@
+// Split-KV decode attention over the packed cache, and the log-sum-exp combine.
+//
+// Method: "KIVI" README (decoding over per-channel-quantized keys, per-token-
+// quantized values and the full-precision residual window; GQA update) with
+// the dequantization x_hat = q*d + m of the "KV1-1.2B" card (BQ2_0).
+// The key-side dequantization is folded per block: since every channel of a
+// G-token block has one (scale, zero), q.k_hat = sum_d (q_d s_d) c_d + sum_d q_d z_d,
+// so the per-token work is a dot product of the scaled query with raw codes.
+#include "kvq_decode.cuh"
+
+namespace kvq {
+
+namespace {
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+template <int NG>
+struct SoftmaxState {
+  float m[NG], l[NG], o[NG][4];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int hh = 0; hh < NG; ++hh) {
+      m[hh] = -INFINITY;
+      l[hh] = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) o[hh][c] = 0.f;
+    }
+  }
+  // score in log2 units; v: this lane's 4 channels of the token's value
+  __device__ __forceinline__ void update(int hh, float score, const float* v) {
+    const float mn = fmaxf(m[hh], score);
+    const float alpha = exp2f(m[hh] - mn);
+    const float pe = exp2f(score - mn);
+    l[hh] = l[hh] * alpha + pe;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) o[hh][c] = o[hh][c] * alpha + pe * v[c];
+    m[hh] = mn;
+  }
+};
+
+// One CTA = one split of one (sequence, KV head); 4 warps, each warp walks a
+// quarter of the split's tokens with its own online-softmax state; lane owns
+// channels lane + 32c, c = 0..3.
+template <int NG>
+__global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p) {
+  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const LayerView& L = p.L;
+  const int G = L.group_k, R = L.residual;
+  const int Q = L.lens[2 * b], n = L.lens[2 * b + 1];
+  const int nblk = Q / G;
+  const int bps = p.blocks_per_split;
+  const int S = (nblk + bps - 1) / bps;
+  if (s > S) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int D = kHeadDim;
+
+  __shared__ float sq[NG][D];
+  __shared__ float sqs[NG][D];
+  __shared__ float sbias[4][NG];
+  __shared__ float sm[4][NG], sl[4][NG];
+  __shared__ float so[4][NG][D];
+
+  for (int i = threadIdx.x; i < NG * D; i += blockDim.x) {
+    const int hh = i / D, d = i % D;
+    sq[hh][d] = load_kv(p.q, ((int64_t)b * p.num_q_heads + h * NG + hh) * D + d, L.kv_dtype) * p.scale_log2;
+  }
+  __syncthreads();
+
+  SoftmaxState<NG> st;
+  st.init();
+
+  if (s == 0) {
+    // Residual ring: exact stored values.
+    const int64_t base = ((int64_t)b * L.num_kv_heads + h) * R;
+    for (int i = Q + warp; i < Q + n; i += 4) {
+      const int64_t row = (base + i % R) * D;
+      float kv[4], vv[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        kv[c] = load_kv(L.ring_k, row + lane + 32 * c, L.kv_dtype);
+        vv[c] = load_kv(L.ring_v, row + lane + 32 * c, L.kv_dtype);
+      }
+#pragma unroll
+      for (int hh = 0; hh < NG; ++hh) {
+        float part = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) part += sq[hh][lane + 32 * c] * kv[c];
+        st.update(hh, warp_sum(part), vv);
+      }
+    }
+  } else {
+    const int kb = L.k_bits, vb = L.v_bits, Gv = L.group_v;
+    const int kper = 32 / kb, vper = 32 / vb;
+    const uint32_t kmask = (1u << kb) - 1, vmask = (1u << vb) - 1;
+    const int j0 = (s - 1) * bps, j1 = min(s * bps, nblk);
+    for (int j = j0; j < j1; ++j) {
+      const uint8_t* rec = record_ptr(L, b, h, j);
+      {
+        const int d = threadIdx.x;
+        const __half2 sz = reinterpret_cast<const __half2*>(rec + L.ksz_off)[d];
+        const float sc = __low2float(sz), z = __high2float(sz);
+#pragma unroll
+        for (int hh = 0; hh < NG; ++hh) {
+          sqs[hh][d] = sq[hh][d] * sc;
+          const float bsum = warp_sum(sq[hh][d] * z);
+          if (lane == 0) sbias[warp][hh] = bsum;
+        }
+      }
+      __syncthreads();
+      float bias[NG];
+#pragma unroll
+      for (int hh = 0; hh < NG; ++hh) bias[hh] = sbias[0][hh] + sbias[1][hh] + sbias[2][hh] + sbias[3][hh];
+      const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + L.kc_off);
+      const uint32_t* vc = reinterpret_cast<const uint32_t*>(rec + L.vc_off);
+      const __half2* vsz = reinterpret_cast<const __half2*>(rec + L.vsz_off);
+      for (int t = warp; t < G; t += 4) {
+        float kcode[4], vv[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int d = lane + 32 * c;
+          kcode[c] = (float)((kc[(t / kper) * D + d] >> ((t % kper) * kb)) & kmask);
+          const uint32_t vq = (vc[t * (D / vper) + d / vper] >> ((d % vper) * vb)) & vmask;
+          const __half2 sz = vsz[t * (D / Gv) + d / Gv];
+          vv[c] = (float)vq * __low2float(sz) + __high2float(sz);
+        }
+#pragma unroll
+        for (int hh = 0; hh < NG; ++hh) {
+          float part = 0.f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) part += sqs[hh][lane + 32 * c] * kcode[c];
+          st.update(hh, warp_sum(part) + bias[hh], vv);
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  // Merge the four warps' states and write this split's partial.
+#pragma unroll
+  for (int hh = 0; hh < NG; ++hh) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) so[warp][hh][lane + 32 * c] = st.o[hh][c];
+    if (lane == 0) {
+      sm[warp][hh] = st.m[hh];
+      sl[warp][hh] = st.l[hh];
+    }
+  }
+  __syncthreads();
+  const int d = threadIdx.x;
+#pragma unroll
+  for (int hh = 0; hh < NG; ++hh) {
+    const float M = fmaxf(fmaxf(sm[0][hh], sm[1][hh]), fmaxf(sm[2][hh], sm[3][hh]));
+    float acc = 0.f, lsum = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float f = sm[w][hh] == -INFINITY ? 0.f : exp2f(sm[w][hh] - M);
+        acc += so[w][hh][d] * f;
+        lsum += sl[w][hh] * f;
+      }
+    }
+    const int64_t slot = ((int64_t)b * p.num_q_heads + h * NG + hh) * p.slots + s;
+    p.ws_o[slot * D + d] = acc;
+    if (d == 0) p.ws_ml[slot] = make_float2(M, lsum);
+  }
+}
+
+// grid (Hq, batch); block D threads.
+__global__ void __launch_bounds__(128) combine_kernel(DecodeParams p) {
+  const int hq = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  const LayerView& L = p.L;
+  constexpr int D = kHeadDim;
+  const int nblk = L.lens[2 * b] / L.group_k;
+  const int S = (nblk + p.blocks_per_split - 1) / p.blocks_per_split;
+  const int64_t base = ((int64_t)b * p.num_q_heads + hq) * p.slots;
+  float M = -INFINITY;
+  for (int s = 0; s <= S; ++s) {
+    const float2 ml = p.ws_ml[base + s];
+    if (ml.y > 0.f) M = fmaxf(M, ml.x);
+  }
+  float acc = 0.f, lsum = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s <= S; ++s) {
+      const float2 ml = p.ws_ml[base + s];
+      if (ml.y > 0.f) {
+        const float f = exp2f(ml.x - M);
+        acc += p.ws_o[(base + s) * D + d] * f;
+        lsum += ml.y * f;
+      }
+    }
+  }
+  const float r = lsum > 0.f ? __fdiv_rn(acc, lsum) : 0.f;
+  const int64_t o = ((int64_t)b * p.num_q_heads + hq) * D + d;
+  if (p.out_dtype == KVQ_F32) reinterpret_cast<float*>(p.out)[o] = r;
+  else if (p.out_dtype == KVQ_BF16) reinterpret_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(r);
+  else reinterpret_cast<__half*>(p.out)[o] = __float2half_rn(r);
+}
+
+template <int NG>
+cudaError_t launch_simple(const DecodeParams& p, int max_splits, cudaStream_t stream) {
+  dim3 grid(max_splits + 1, p.L.num_kv_heads, p.batch);
+  decode_split_simple_kernel<NG><<<grid, 128, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeParams& p, int max_splits, cudaStream_t stream) {
+  if (p.batch <= 0) return cudaSuccess;
+  const int g = p.num_q_heads / p.L.num_kv_heads;
+  cudaError_t e;
+  switch (g) {
+    case 1: e = launch_simple<1>(p, max_splits, stream); break;
+    case 2: e = launch_simple<2>(p, max_splits, stream); break;
+    case 4: e = launch_simple<4>(p, max_splits, stream); break;
+    case 8: e = launch_simple<8>(p, max_splits, stream); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  combine_kernel<<<dim3(p.num_q_heads, p.batch), kHeadDim, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

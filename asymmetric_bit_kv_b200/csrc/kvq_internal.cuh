@@ -1,0 +1,79 @@
+// Internal definitions shared by the host entry points and the kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int kHeadDim = 128;  // the decode kernels are specialised for D = 128
+
+// Per-layer view of the packed cache, passed by value to kernels.
+struct LayerView {
+  uint8_t* blocks;        // block records [max_batch][Hkv][max_blocks]
+  void* ring_k;           // [max_batch][Hkv][R][D] kv dtype
+  void* ring_v;
+  int32_t* lens;          // [max_batch][2]: quantized tokens, ring tokens
+  int64_t record_bytes;
+  int64_t max_blocks;
+  int32_t kc_off, ksz_off, vc_off, vsz_off;  // byte offsets inside a record
+  int32_t k_bits, v_bits;
+  int32_t num_kv_heads, head_dim, group_k, group_v, residual;
+  int32_t kv_dtype;       // KVQ_F16 / KVQ_BF16
+};
+
+__host__ __device__ inline int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+// Byte sizes of the four parts of a block record.
+__host__ __device__ inline int64_t kc_bytes(int G, int D, int kb) { return (int64_t)G * kb / 32 * D * 4; }
+__host__ __device__ inline int64_t ksz_bytes(int D) { return (int64_t)D * 4; }
+__host__ __device__ inline int64_t vc_bytes(int G, int D, int vb) { return (int64_t)G * (D * vb / 32) * 4; }
+__host__ __device__ inline int64_t vsz_bytes(int G, int D, int gv) { return (int64_t)G * (D / gv) * 4; }
+
+__device__ __forceinline__ uint8_t* record_ptr(const LayerView& L, int b, int h, int64_t j) {
+  return L.blocks + (((int64_t)b * L.num_kv_heads + h) * L.max_blocks + j) * L.record_bytes;
+}
+
+__device__ __forceinline__ float load_kv(const void* p, int64_t i, int dtype) {
+  if (dtype == KVQ_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+  return __half2float(reinterpret_cast<const __half*>(p)[i]);
+}
+
+// ---------------------------------------------------------------------------
+// The quantizer of the "KV1-1.2B" card (section "Quantization Format: KV1.cpp
+// BQ2_0"), widened from 3 to 2^b - 1 levels. Every operation is an explicitly
+// rounded fp32 intrinsic so the compiler cannot contract or reassociate it;
+// codes, scales and zero points are therefore reproducible bit for bit.
+// ---------------------------------------------------------------------------
+struct GroupParams {
+  __half d16, m16;
+  float d, m;  // fp32 copies of the fp16 values, used for the codes
+};
+
+__device__ __forceinline__ GroupParams group_params(float mn, float mx, int bits) {
+  const float qmax = (float)((1 << bits) - 1);
+  const float d = __fdiv_rn(__fsub_rn(mx, mn), qmax);
+  GroupParams g;
+  g.d16 = __float2half_rn(fmaxf(d, 1e-6f));
+  g.m16 = __float2half_rn(__fadd_rn(mn, 0.0f));  // -0.0 min is stored as +0.0
+  g.d = __half2float(g.d16);
+  g.m = __half2float(g.m16);
+  return g;
+}
+
+__device__ __forceinline__ uint32_t quant_code(float x, const GroupParams& g, int bits) {
+  const float t = __fdiv_rn(__fsub_rn(x, g.m), g.d);
+  const float r = fminf(fmaxf(rintf(t), 0.0f), (float)((1 << bits) - 1));  // rint: ties to even
+  return (uint32_t)r;
+}
+
+// x_hat = q * d + m with two roundings (no fused multiply-add).
+__device__ __forceinline__ float dequant_value(uint32_t q, __half d16, __half m16) {
+  return __fadd_rn(__fmul_rn((float)q, __half2float(d16)), __half2float(m16));
+}
+
+}  // namespace kvq

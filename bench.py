@@ -1,0 +1,494 @@
+"""Decode-step benchmark of the quantized KV cache on B200.
+
+One step = append one new token to every sequence of a batch (quantizing a
+G-token block whenever a ring fills) + decode attention for one query per
+sequence over the whole cache. The workload is the Llama-3-8B-shaped GQA
+layer: batch 32, 32 query / 8 KV heads, head_dim 128, context 8192, bf16
+keys N(0,1) x log-normal channel magnitudes and values N(0,1), keys 2-bit per
+channel in groups of 64 tokens, values 4-bit per token in groups of 64
+channels, residual window 128.
+
+Timing: W warm-up steps, then exactly K steps between barriers and device
+synchronisations, timed with CUDA events on the launching stream; the job
+value is the max over ranks. Each step works on the next of several
+independent cache replicas, so every step streams a different 248 MB cache
+(more than the 126 MB L2) and every replica's context grows only by K/replicas
+tokens. Multi-GPU runs (torchrun) give every rank its own replicas: weak
+scaling, no collective on the data path.
+
+`--impl reference` times the CPU oracle (the plain restatement of the method
+used by the tests) on the host cores instead, on a bounded sample of the same
+workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized-KV decode attention: KV tokens/s and achieved HBM GB/s vs B200 peak"
+UNIT = "KV tokens/s"
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2048)
+    ap.add_argument("--warmup", type=int, default=32)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--replicas", type=int, default=16)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def _dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle baseline (host cores, spawned worker processes)
+# --------------------------------------------------------------------------
+
+def _oracle_worker(conn, unit, ctx):
+    """One unit of the workload -- one (sequence, KV head) with its 4 query
+    heads -- held in the oracle. Prefill is untimed; each 'step' command appends
+    one token and runs decode attention, and replies with the tokens attended."""
+    from threadpoolctl import threadpool_limits
+
+    from asymmetric_bit_kv_b200 import workloads as W
+    from oracle import kvq_oracle as O
+
+    with threadpool_limits(1):
+        wl = W.llama3_8b_gqa()
+        g = wl.num_q_heads // wl.num_kv_heads
+        unit_wl = W.Workload(wl.name, 1, g, 1, wl.head_dim, [ctx], wl.k_bits, wl.v_bits, wl.group_k, wl.group_v,
+                             wl.residual, wl.kv_dtype, wl.key_dist, wl.value_std, wl.seed)
+        extra = 4096
+        k, v = W.generate_tokens(unit_wl, 0, [ctx + extra], seed_offset=7000 + unit)
+        k = k.float().numpy()
+        v = v.float().numpy()
+        c = O.SequenceCache(1, wl.head_dim, wl.k_bits[0], wl.v_bits[0], wl.group_k, wl.group_v, wl.residual)
+        c.append(k[:ctx], v[:ctx])
+        conn.send("ready")
+        i = 0
+        while True:
+            cmd = conn.recv()
+            if cmd != "step":
+                break
+            q = W.generate_queries(unit_wl, 0, 1, step=i)[0].float().numpy()
+            t = ctx + (i % extra)
+            c.append(k[t:t + 1], v[t:t + 1])
+            O.decode_attention(c, q, wl.softmax_scale)
+            i += 1
+            conn.send(c.length)
+    conn.close()
+
+
+class OracleRunner:
+    """`workers` spawned processes, one workload unit each, stepped together."""
+
+    def __init__(self, workers: int, ctx: int = 8192):
+        import multiprocessing as mp
+
+        ctxm = mp.get_context("spawn")
+        self.conns, self.procs = [], []
+        for u in range(workers):
+            a, b = ctxm.Pipe()
+            p = ctxm.Process(target=_oracle_worker, args=(b, u, ctx), daemon=True)
+            p.start()
+            self.conns.append(a)
+            self.procs.append(p)
+        for c in self.conns:
+            assert c.recv() == "ready"
+        self.workers = workers
+        self.ctx = ctx
+
+    def step(self):
+        t0 = time.perf_counter()
+        for c in self.conns:
+            c.send("step")
+        # a unit holds one of the workload's 8 KV heads: count KV tokens
+        # (all heads of a token) as unit tokens / 8
+        toks = sum(c.recv() for c in self.conns) / 8
+        return toks, time.perf_counter() - t0
+
+    def close(self):
+        for c in self.conns:
+            try:
+                c.send("stop")
+            except Exception:
+                pass
+        for p in self.procs:
+            p.join(timeout=10)
+
+    def describe(self, steps):
+        return (f"{self.workers} units of the workload in parallel, one (sequence, KV head) with its 4 query heads "
+                f"each (context {self.ctx}); a step = append one token + fp64 decode attention per unit; "
+                f"{steps} timed steps; KV tokens counted as unit tokens / 8 KV heads")
+
+
+def cpu_oracle_baseline(steps: int = 100, warmup: int = 2):
+    workers = max(1, min(os.cpu_count() or 1, 16))
+    run = OracleRunner(workers)
+    try:
+        for _ in range(warmup):
+            run.step()
+        toks, secs = 0, 0.0
+        for _ in range(steps):
+            t, s = run.step()
+            toks += t
+            secs += s
+    finally:
+        run.close()
+    return {"value": toks / secs, "unit": UNIT, "cores": workers, "kind": "oracle", "sample": run.describe(steps)}
+
+
+# --------------------------------------------------------------------------
+# the library arm
+# --------------------------------------------------------------------------
+
+def run_kvq(a):
+    import torch
+    import torch.distributed as dist
+
+    from asymmetric_bit_kv_b200 import CacheConfig, KVCache
+    from asymmetric_bit_kv_b200 import workloads as W
+    from oracle import kvq_oracle as O  # sizes only (closed-form bytes/token), never on the timed path
+
+    rank, world, local = _dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = W.llama3_8b_gqa()
+    B, Hq, Hkv, D = wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim
+    ctx = wl.context[0]
+    R = a.replicas
+    steps_per_rep = math.ceil((a.warmup + 2 * a.steps) / R) + 2
+    cap = ctx + steps_per_rep + wl.group_k
+    cfg = CacheConfig(1, B, Hq, Hkv, D, cap, wl.group_k, wl.group_v, wl.residual, wl.kv_dtype, wl.k_bits, wl.v_bits)
+    caches = []
+    for r in range(R):
+        c = KVCache(cfg, dev)
+        k, v = W.generate_tokens(wl, 0, [ctx] * B, device=dev, seed_offset=1000 * rank + r)
+        c.append(0, k, v, [ctx] * B)
+        del k, v
+        caches.append(c)
+    torch.cuda.synchronize()
+    n_new = max(a.warmup + a.steps, 1)
+    gen = torch.Generator(device=dev).manual_seed(12345 + rank)
+    pool = 64  # distinct per-step inputs, reused round-robin
+    new_k = torch.randn(pool, B, Hkv, D, generator=gen, device=dev).to(wl.kv_dtype)
+    new_v = torch.randn(pool, B, Hkv, D, generator=gen, device=dev).to(wl.kv_dtype)
+    qs = torch.randn(pool, B, Hq, D, generator=gen, device=dev).to(wl.kv_dtype)
+    out = torch.empty(B, Hq, D, dtype=wl.kv_dtype, device=dev)
+    ones = [1] * B
+    stream = torch.cuda.current_stream()
+    bytes_tok = O.quantized_bytes_per_token(Hkv, D, wl.k_bits[0], wl.v_bits[0], wl.group_k, wl.group_v)
+
+    lengths = [[ctx] * B for _ in range(R)]
+
+    def alg_bytes_and_tokens(r):
+        """Algorithmic bytes read+written by decode attention of replica r (its
+        current lengths): packed cache + residual ring + q + out."""
+        tot, toks = 0.0, 0
+        for b in range(B):
+            qn, n = caches[r].lengths(0, b)
+            tot += qn * bytes_tok + n * Hkv * D * 2 * 2
+            toks += qn + n
+        tot += 2 * B * Hq * D * 2
+        return tot, toks
+
+    def step(i, r, ev=None):
+        caches[r].append(0, new_k[i % pool], new_v[i % pool], ones)
+        if ev is not None:
+            ev[0].record(stream)
+        caches[r].decode_attention(0, qs[i % pool], out, softmax_scale=wl.softmax_scale)
+        if ev is not None:
+            ev[1].record(stream)
+
+    # launches of this library per step: ring write + decode split + combine,
+    # plus one quantize launch on steps where a ring is full (lazy flush)
+    def launches_for(r):
+        q0, n0 = caches[r].lengths(0, 0)
+        return 3 + (1 if n0 == wl.residual else 0)
+
+    for i in range(a.warmup):
+        step(i, i % R)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    # per-step accounting (host mirror, before the step)
+    launches = 0
+    alg_total, tok_total = 0.0, 0
+    dec_events = []
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.1)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(a.steps):
+        r = (a.warmup + i) % R
+        launches += launches_for(r)
+        ab, tk = alg_bytes_and_tokens(r)
+        alg_total += ab
+        tok_total += tk + B  # the decode sees the appended token too
+        ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        step(a.warmup + i, r, ev)
+        dec_events.append(ev)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    dec_ms = sum(x[0].elapsed_time(x[1]) for x in dec_events)
+    # the appended token adds B * Hkv * D * 2 (K, V) * 2 bytes to the residual read
+    alg_total += a.steps * B * Hkv * D * 2 * 2
+    if world > 1:
+        t = torch.tensor([ms, dec_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, dec_ms = float(t[0]), float(t[1])
+    value = tok_total * world / (ms / 1e3)
+    achieved_gbs = alg_total / (dec_ms / 1e3) / 1e9
+
+    # ---- end to end through the public API with host buffers ----
+    e2e_steps = min(a.steps, 512)
+    hk = torch.empty(pool, B, Hkv, D, dtype=wl.kv_dtype).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    hq = torch.empty(pool, B, Hq, D, dtype=wl.kv_dtype).pin_memory()
+    hk.copy_(new_k.cpu())
+    hv.copy_(new_v.cpu())
+    hq.copy_(qs.cpu())
+    hout = torch.empty(B, Hq, D, dtype=wl.kv_dtype).pin_memory()
+    dk = torch.empty(B, Hkv, D, dtype=wl.kv_dtype, device=dev)
+    dv = torch.empty_like(dk)
+    dq = torch.empty(B, Hq, D, dtype=wl.kv_dtype, device=dev)
+    tok_e2e = 0
+    for i in range(e2e_steps):
+        r = (a.warmup + a.steps + i) % R
+        tok_e2e += alg_bytes_and_tokens(r)[1] + B
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for i in range(e2e_steps):
+        r = (a.warmup + a.steps + i) % R
+        j = i % pool
+        dk.copy_(hk[j], non_blocking=True)
+        dv.copy_(hv[j], non_blocking=True)
+        dq.copy_(hq[j], non_blocking=True)
+        caches[r].append(0, dk, dv, ones)
+        caches[r].decode_attention(0, dq, out, softmax_scale=wl.softmax_scale)
+        hout.copy_(out, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    e2e_value = tok_e2e * world / (e2e_ms / 1e3)
+
+    result = None
+    if rank == 0:
+        peak, peak_kind = _peaks()
+        traffic = _committed_traffic()
+        result = {
+            "metric": METRIC,
+            "value": value,
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": a.steps,
+            "warmup": a.warmup,
+            "ms_per_step": ms / a.steps,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic (seeded; Llama-3-8B-shaped layer, no model weights)",
+            "config": {
+                "workload": wl.name,
+                "batch": B, "num_q_heads": Hq, "num_kv_heads": Hkv, "head_dim": D,
+                "context": ctx, "k_bits": wl.k_bits[0], "v_bits": wl.v_bits[0],
+                "group_k": wl.group_k, "group_v": wl.group_v, "residual": wl.residual,
+                "kv_dtype": "bf16", "out_dtype": "bf16",
+                "replicas": R,
+                "mean_context_timed": tok_total / (a.steps * B),
+                "l2": "inputs larger than L2: each step reads a different replica's ~248 MB cache",
+                "parallelism": f"dp{world} (independent replicas per rank)",
+            },
+            "roofline": {
+                "kernel": "decode attention (split-KV kernel + log-sum-exp combine), per call",
+                "bound": "hbm",
+                "achieved": achieved_gbs,
+                "peak": peak,
+                "unit": "GB/s",
+                "frac": achieved_gbs / peak,
+                "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
+                "frac_of_8tbs_nominal": achieved_gbs / 8000.0,
+                "traffic": traffic,
+                "decode_us_per_call": dec_ms / a.steps * 1e3,
+                "alg_bytes_per_call": alg_total / a.steps,
+            },
+            "e2e": {"value": e2e_value, "unit": UNIT,
+                    "h2d_bytes_per_step": int((dk.numel() + dv.numel() + dq.numel()) * 2),
+                    "d2h_bytes_per_step": int(out.numel() * 2), "steps": e2e_steps},
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+    del caches
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def _committed_traffic():
+    """DRAM bytes per launch of the decode kernel from the committed ncu summary, if any."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(p) as f:
+            return json.load(f).get("dram_bytes_per_launch")
+    except Exception:
+        return None
+
+
+def run_reference(a):
+    """The CPU oracle on the host cores, K steps after W warm-up steps; every
+    step is a bounded sample of the workload (one unit per host core)."""
+    rank, world, _ = _dist_env()
+    if rank != 0:
+        return None
+    from asymmetric_bit_kv_b200 import workloads as W
+
+    wl = W.llama3_8b_gqa()
+    workers = max(1, min(os.cpu_count() or 1, 16))
+    t_start = time.perf_counter()
+    run = OracleRunner(workers, wl.context[0])
+    try:
+        for _ in range(a.warmup):
+            run.step()
+        toks, secs = 0, 0.0
+        for _ in range(a.steps):
+            t, s = run.step()
+            toks += t
+            secs += s
+    finally:
+        run.close()
+    value = toks / secs
+    base = {"value": value, "unit": UNIT, "cores": workers, "kind": "oracle", "sample": run.describe(a.steps)}
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": a.steps,
+        "warmup": a.warmup,
+        "ms_per_step": 1e3 * secs / a.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded; Llama-3-8B-shaped layer, no model weights)",
+        "config": {"workload": wl.name, "units_per_step": workers, "context": wl.context[0]},
+        "cpu_baseline": base,
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": time.perf_counter() - t_start,
+    }
+
+
+def main():
+    a = _args()
+    if a.impl == "reference":
+        res = run_reference(a)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    rank, world, _ = _dist_env()
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu = cpu_oracle_baseline()   # spawned before any CUDA work in this process
+    res = run_kvq(a)
+    if res is not None:
+        res["cpu_baseline"] = cpu
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,185 @@
+/*
+ * kvq.h -- C ABI of a B200 (sm_100a) library for an asymmetric 2/4/8-bit
+ * KV cache and decode attention over it.
+ *
+ * The method (web pages, cited by title and section):
+ *  - "KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV Cache" (README),
+ *    sections "Overview" and "Example": keys are quantized per channel and
+ *    values per token, at 2 or 4 bits (k_bits, v_bits) with a group size, and
+ *    the residual_length most recent tokens stay in full precision; the GQA
+ *    update (2025.01.18) adds grouped-query attention.
+ *  - "KV1-1.2B" model card, section "Quantization Format: KV1.cpp BQ2_0":
+ *    the quantizer itself -- in fp32, d = fp16(max((max-min)/(2^b-1), 1e-6)),
+ *    m = fp16(min), q = clamp(round_half_to_even((x - m) / d), 0, 2^b-1) with
+ *    the fp16-rounded m and d, dequantization x_hat = q*d + m, and codes packed
+ *    lowest bits first.
+ *  - "Quantize What Counts: More For Keys, Less For Values", section "KV Cache
+ *    Quantization": key and value bit widths chosen independently and per
+ *    layer (bit range up to 8).
+ *
+ * Ownership. The caller allocates one device arena per cache (size from
+ * kvq_cache_required_bytes) and owns it, every input and output buffer and
+ * every stream. The library never allocates device memory. A kvq_cache handle
+ * is host memory owned by the library (freed by kvq_cache_destroy) and must
+ * not outlive its arena.
+ *
+ * Errors. Every entry point validates its arguments on the host before it
+ * enqueues anything; on failure it returns a negative kvq_status, enqueues no
+ * work and leaves the cache unchanged. kvq_last_error() gives a one-line
+ * reason. KVQ_ERR_CUDA reports a failed launch. Work is asynchronous on the
+ * given stream (a cudaStream_t; NULL = legacy default stream); faults during
+ * execution surface at the caller's next synchronisation, as for any CUDA
+ * kernel. Calls on one cache must be ordered on one stream: they share the
+ * arena's length table and split-partial workspace.
+ *
+ * Threading. A handle is not thread-safe; distinct handles are independent.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kvq_status {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = -1, /* null pointer, bad index, bad shape or size  */
+  KVQ_ERR_UNSUPPORTED = -2, /* valid but not built: bits, dims, dtype      */
+  KVQ_ERR_CAPACITY = -3,    /* a sequence would exceed max_tokens          */
+  KVQ_ERR_WORKSPACE = -4,   /* arena smaller than kvq_cache_required_bytes */
+  KVQ_ERR_CUDA = -5         /* a CUDA launch or call failed                */
+} kvq_status;
+
+typedef enum kvq_dtype { KVQ_F16 = 0, KVQ_BF16 = 1, KVQ_F32 = 2 } kvq_dtype;
+
+#define KVQ_MAX_BATCH 512  /* sequences per cache                        */
+#define KVQ_MAX_LAYERS 512 /* layers per cache                           */
+#define KVQ_MAX_SPLITS 256 /* quantized splits per (sequence, KV head)   */
+
+/* Cache shape. Names follow the KIVI README "Example" (k_bits, v_bits,
+ * group_size, residual_length) with the group size given per tensor as in
+ * "Quantize What Counts" (group_size {"k", "v"}).                          */
+typedef struct kvq_config {
+  int32_t num_layers;   /* 1 .. KVQ_MAX_LAYERS                              */
+  int32_t max_batch;    /* sequences, 1 .. KVQ_MAX_BATCH                    */
+  int32_t num_q_heads;  /* Hq, a multiple of num_kv_heads                   */
+  int32_t num_kv_heads; /* Hkv; Hq/Hkv in {1, 2, 4, 8}                      */
+  int32_t head_dim;     /* D = 128                                          */
+  int32_t max_tokens;   /* per-sequence capacity, quantized + residual      */
+  int32_t group_k;      /* G: tokens per key group (one group per channel);
+                           32, 64 or 128. Flushes move G tokens at a time.  */
+  int32_t group_v;      /* channels per value group (one group per token);
+                           32, 64 or 128, dividing head_dim                 */
+  int32_t residual;     /* R: full-precision ring slots; a multiple of G    */
+  int32_t kv_dtype;     /* KVQ_F16 or KVQ_BF16: keys, values, ring, queries */
+  const int8_t* k_bits; /* host [num_layers], each 2, 4 or 8 (copied)       */
+  const int8_t* v_bits; /* host [num_layers], each 2, 4 or 8 (copied)       */
+} kvq_config;
+
+typedef struct kvq_cache kvq_cache;
+
+/* Where one layer's packed cache lives, for tests and tools that read it.
+ * Block records: for sequence b, KV head h and key block j (tokens
+ * [j*G, (j+1)*G) of that sequence) the record starts at
+ *   blocks + ((b * num_kv_heads + h) * max_blocks + j) * record_bytes
+ * and holds, at the given byte offsets:
+ *   kc  uint32 [G*k_bits/32][D]: word w of channel d packs the codes of
+ *       tokens w*(32/k_bits) + i, i = 0.., code i at bits [i*k_bits, ...)
+ *       (per-channel keys, packed along the token axis);
+ *   ksz half2 [D]: (scale d, zero point m) of each channel's key group;
+ *   vc  uint32 [G][D*v_bits/32]: word w of token t packs the codes of
+ *       channels w*(32/v_bits) + i, code i at bits [i*v_bits, ...)
+ *       (per-token values, packed along head_dim);
+ *   vsz half2 [G][D/group_v]: (scale, zero point) of each value group.
+ * Ring: [max_batch][num_kv_heads][R][D] in kv_dtype; token i of a sequence
+ * (quantized <= i < quantized + residual) sits in slot i % R.              */
+typedef struct kvq_layout {
+  void* blocks;
+  int64_t record_bytes;
+  int64_t max_blocks;
+  int64_t kc_offset, ksz_offset, vc_offset, vsz_offset;
+  void* ring_k;
+  void* ring_v;
+  int32_t k_bits, v_bits;
+} kvq_layout;
+
+/* Device bytes the arena must hold for cfg: all layers' block records and
+ * rings, the length table and the split-partial workspace.                 */
+KVQ_API kvq_status kvq_cache_required_bytes(const kvq_config* cfg, size_t* bytes);
+
+/* Validate cfg and bind a cache to dev_arena (device pointer, 256-byte
+ * aligned, arena_bytes >= required), with the arena's device current. Every
+ * sequence starts empty: the call zeroes the arena's length table and waits
+ * for that to finish before it returns.                                    */
+KVQ_API kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena_bytes,
+                            kvq_cache** out);
+
+/* Free the host handle. Does not touch the arena.                          */
+KVQ_API kvq_status kvq_cache_destroy(kvq_cache* cache);
+
+/* Empty every sequence of every layer (stream-ordered).                    */
+KVQ_API kvq_status kvq_cache_reset(kvq_cache* cache, void* stream);
+
+/* Append new_lens[b] tokens to sequence b of `layer`, b < batch.
+ * k, v: device, token-major [sum(new_lens)][num_kv_heads][head_dim] in
+ * kv_dtype, sequences in order. new_lens: host [batch], each >= 0.
+ * Semantics (KIVI README: residual window of recent full-precision tokens;
+ * KV1 card: each token quantized once when it enters the cache): tokens are
+ * appended one by one; a token that finds the ring full (R tokens) first
+ * causes the oldest G ring tokens to be quantized -- keys per channel over
+ * the G tokens, values per token over group_v channels -- into one block
+ * record. Blocks that a long append would quantize straight away are read
+ * from k, v directly. Fails with KVQ_ERR_CAPACITY if a sequence would exceed
+ * max_tokens.                                                              */
+KVQ_API kvq_status kvq_append(kvq_cache* cache, int32_t layer, const void* k, const void* v,
+                      const int32_t* new_lens, int32_t batch, void* stream);
+
+/* Quantize every complete group of G tokens left in the ring of sequences
+ * 0..batch-1 of `layer`: residual n becomes n % G.                         */
+KVQ_API kvq_status kvq_flush_residual(kvq_cache* cache, int32_t layer, int32_t batch, void* stream);
+
+/* One decode query per sequence: out[b][h] = softmax(scale * q[b][h] K~^T) V~
+ * over all cached tokens of sequence b (no mask), K~/V~ the dequantized
+ * blocks and the exact ring tokens; query head h reads KV head
+ * h / (Hq/Hkv) (GQA). q: device [batch][Hq][D] in kv_dtype. out: device
+ * [batch][Hq][D] in out_dtype (F32, F16 or BF16; round to nearest even).
+ * A sequence with no tokens gives zeros. Uses the arena's workspace.       */
+KVQ_API kvq_status kvq_decode_attention(kvq_cache* cache, int32_t layer, const void* q, void* out,
+                                int32_t out_dtype, float softmax_scale, int32_t batch,
+                                void* stream);
+
+/* Reconstruct tokens [t0, t1) of sequence `seq` as fp32: x_hat = q*d + m
+ * (an fp32 product, then an fp32 sum; KV1 card, BQ2_0) for quantized tokens
+ * and the exact stored value for ring tokens. k_out, v_out: device
+ * [t1-t0][num_kv_heads][head_dim] fp32. 0 <= t0 <= t1 <= sequence length.  */
+KVQ_API kvq_status kvq_dequant(kvq_cache* cache, int32_t layer, int32_t seq, int32_t t0, int32_t t1,
+                       float* k_out, float* v_out, void* stream);
+
+/* Layer layout (see kvq_layout).                                           */
+KVQ_API kvq_status kvq_get_layout(const kvq_cache* cache, int32_t layer, kvq_layout* out);
+
+/* Host mirror of a sequence's lengths: quantized tokens (a multiple of G)
+ * and ring tokens.                                                         */
+KVQ_API kvq_status kvq_seq_lengths(const kvq_cache* cache, int32_t layer, int32_t seq,
+                           int32_t* quantized, int32_t* residual);
+
+/* Static description of a status code.                                     */
+KVQ_API const char* kvq_status_string(kvq_status status);
+
+/* Reason for the last failure on this thread ("" if none).                 */
+KVQ_API const char* kvq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

@@ -1,0 +1,142 @@
+"""Helpers shared by the tests: build a cache and its oracle twin from the same
+inputs, read packed block records back from the device, compare results."""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from asymmetric_bit_kv_b200 import CacheConfig, KVCache
+from oracle import kvq_oracle as O
+
+ATOL = 2e-3       # max-abs error of attention outputs vs the fp64 oracle
+RTOL = 1e-2       # max-rel error, relative to max(|ref|, REL_FLOOR)
+REL_FLOOR = ATOL / RTOL
+
+
+def assert_attention_close(out: np.ndarray, ref: np.ndarray, what: str = ""):
+    out = np.asarray(out, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert out.shape == ref.shape, (out.shape, ref.shape)
+    assert np.isfinite(out).all(), f"{what}: non-finite output"
+    err = np.abs(out - ref)
+    rel = err / np.maximum(np.abs(ref), REL_FLOOR)
+    assert err.max() <= ATOL, f"{what}: max abs err {err.max():.3e} > {ATOL}"
+    assert rel.max() <= RTOL, f"{what}: max rel err {rel.max():.3e} > {RTOL}"
+
+
+def ulp(x: np.ndarray, dtype) -> np.ndarray:
+    """Spacing of `dtype` (torch.float16 / torch.bfloat16) at |x|."""
+    mant = 10 if dtype == torch.float16 else 7
+    emin = -14 if dtype == torch.float16 else -126
+    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** emin)))
+    return 2.0 ** (e - mant)
+
+
+class Twin:
+    """A device cache and one oracle SequenceCache per (layer, sequence)."""
+
+    def __init__(self, cfg: CacheConfig, device="cuda", oracle_seqs=None, oracle_layers=None):
+        self.cfg = cfg
+        self.gpu = KVCache(cfg, device)
+        self.device = device
+        self.oracle_seqs = set(range(cfg.max_batch)) if oracle_seqs is None else set(oracle_seqs)
+        self.oracle_layers = set(range(cfg.num_layers)) if oracle_layers is None else set(oracle_layers)
+        self.ora = {}
+        for layer in self.oracle_layers:
+            for b in self.oracle_seqs:
+                self.ora[(layer, b)] = O.SequenceCache(cfg.num_kv_heads, cfg.head_dim, cfg.k_bits[layer],
+                                                       cfg.v_bits[layer], cfg.group_k, cfg.group_v, cfg.residual)
+
+    def append(self, layer: int, k: torch.Tensor, v: torch.Tensor, new_lens):
+        """k, v: [sum(new_lens), Hkv, D] in the cache dtype (any device)."""
+        self.gpu.append(layer, k.to(self.device), v.to(self.device), new_lens)
+        if layer in self.oracle_layers:
+            off = 0
+            for b, n in enumerate(new_lens):
+                if b in self.oracle_seqs and n > 0:
+                    kk = k[off:off + n].float().cpu().numpy()
+                    vv = v[off:off + n].float().cpu().numpy()
+                    self.ora[(layer, b)].append(kk, vv)
+                off += n
+
+    def flush_residual(self, layer: int, batch: int):
+        self.gpu.flush_residual(layer, batch)
+        for b in range(batch):
+            if (layer, b) in self.ora:
+                self.ora[(layer, b)].flush_residual()
+
+    def check_lengths(self, layer: int, batch: int):
+        for b in range(batch):
+            if (layer, b) in self.ora:
+                o = self.ora[(layer, b)]
+                assert self.gpu.lengths(layer, b) == (o.quantized_tokens, o.residual_tokens), (layer, b)
+
+    def read_records(self, layer: int, b: int, h: int, nblk: int):
+        """Device block records [0, nblk) of (sequence b, KV head h), split into parts."""
+        lay = self.gpu.layout(layer)
+        cfg = self.cfg
+        G, D, Gv = cfg.group_k, cfg.head_dim, cfg.group_v
+        kb, vb = lay.k_bits, lay.v_bits
+        start = lay.blocks - self.gpu.arena.data_ptr() + ((b * cfg.num_kv_heads + h) * lay.max_blocks) * lay.record_bytes
+        raw = self.gpu.arena[start:start + nblk * lay.record_bytes].cpu().numpy().reshape(nblk, lay.record_bytes)
+
+        def part(off, nbytes, dtype, shape):
+            return np.ascontiguousarray(raw[:, off:off + nbytes]).view(dtype).reshape((nblk,) + shape)
+
+        kcw = G * kb // 32
+        vcw = D * vb // 32
+        return {
+            "kc": part(lay.kc_offset, kcw * D * 4, np.uint32, (kcw, D)),
+            "ksz": part(lay.ksz_offset, D * 4, np.float16, (D, 2)),
+            "vc": part(lay.vc_offset, G * vcw * 4, np.uint32, (G, vcw)),
+            "vsz": part(lay.vsz_offset, G * (D // Gv) * 4, np.float16, (G, D // Gv, 2)),
+        }
+
+    def read_ring(self, layer: int, b: int):
+        lay = self.gpu.layout(layer)
+        cfg = self.cfg
+        n = cfg.num_kv_heads * cfg.residual * cfg.head_dim * 2
+        out = []
+        for ptr in (lay.ring_k, lay.ring_v):
+            start = ptr - self.gpu.arena.data_ptr() + b * n
+            raw = self.gpu.arena[start:start + n].cpu()
+            out.append(raw.view(cfg.kv_dtype).float().numpy().reshape(cfg.num_kv_heads, cfg.residual, cfg.head_dim))
+        return out
+
+    def check_codes(self, layer: int, b: int):
+        """Every packed block and ring token of sequence b equals the oracle's, bit for bit."""
+        o = self.ora[(layer, b)]
+        cfg = self.cfg
+        kb, vb = cfg.k_bits[layer], cfg.v_bits[layer]
+        nblk = len(o.blocks)
+        for h in range(cfg.num_kv_heads):
+            if nblk:
+                rec = self.read_records(layer, b, h, nblk)
+                for j, blk in enumerate(o.blocks):
+                    kw = O.pack_key_block(blk.kc, kb)[h]
+                    assert np.array_equal(rec["kc"][j], kw), (layer, b, h, j, "key codes")
+                    assert np.array_equal(rec["ksz"][j][:, 0].view(np.uint16), blk.kd[h].view(np.uint16)), (b, h, j, "key scale")
+                    assert np.array_equal(rec["ksz"][j][:, 1].view(np.uint16), blk.km[h].view(np.uint16)), (b, h, j, "key zero")
+                    vw = O.pack_value_block(blk.vc, vb)[h]
+                    assert np.array_equal(rec["vc"][j], vw), (layer, b, h, j, "value codes")
+                    assert np.array_equal(rec["vsz"][j][..., 0].view(np.uint16), blk.vd[:, h].view(np.uint16)), (b, h, j, "value scale")
+                    assert np.array_equal(rec["vsz"][j][..., 1].view(np.uint16), blk.vm[:, h].view(np.uint16)), (b, h, j, "value zero")
+        if o.residual_tokens:
+            rk, rv = self.read_ring(layer, b)
+            Q = o.quantized_tokens
+            for t in range(o.residual_tokens):
+                slot = (Q + t) % cfg.residual
+                assert np.array_equal(rk[:, slot], o.ring_k[t]), (layer, b, t, "ring key")
+                assert np.array_equal(rv[:, slot], o.ring_v[t]), (layer, b, t, "ring value")
+
+    def check_dequant(self, layer: int, b: int):
+        o = self.ora[(layer, b)]
+        L = o.length
+        k, v = self.gpu.dequant(layer, b, 0, L)
+        K, V = o.dequantized()
+        assert np.array_equal(k.cpu().numpy(), K), (layer, b, "dequant keys")
+        assert np.array_equal(v.cpu().numpy(), V), (layer, b, "dequant values")
+
+    def oracle_decode(self, layer: int, b: int, q_b: np.ndarray, scale: float):
+        return O.decode_attention(self.ora[(layer, b)], q_b, scale)
