@@ -26,7 +26,9 @@ struct kvq_cache {
   int64_t max_blocks;
   int64_t lens_off;               // int32 [num_layers][max_batch][2]
   int64_t ws_o_off, ws_ml_off;    // split partials
+  int64_t err_off;                // int32 device error word
   int32_t slots;                  // partial slots per (sequence, query head)
+  int32_t sm_count;
   std::vector<int32_t> q_len, n_len;  // host mirror [num_layers][max_batch]
 };
 
@@ -83,7 +85,7 @@ kvq_status validate_config(const kvq_config* c) {
 
 struct Plan {
   std::vector<int64_t> blocks_off, ring_k_off, ring_v_off, record_bytes;
-  int64_t max_blocks, lens_off, ws_o_off, ws_ml_off, total;
+  int64_t max_blocks, lens_off, err_off, ws_o_off, ws_ml_off, total;
   int32_t slots;
 };
 
@@ -110,6 +112,8 @@ Plan make_plan(const kvq_config* c) {
   }
   p.lens_off = off;
   off = round_up(off + (int64_t)c->num_layers * c->max_batch * 2 * 4, 256);
+  p.err_off = off;
+  off = round_up(off + 4, 256);
   p.slots = (int32_t)std::min<int64_t>(p.max_blocks, KVQ_MAX_SPLITS) + 1;
   const int64_t partials = (int64_t)c->max_batch * c->num_q_heads * p.slots;
   p.ws_o_off = off;
@@ -253,11 +257,14 @@ kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena
   c->lens_off = plan.lens_off;
   c->ws_o_off = plan.ws_o_off;
   c->ws_ml_off = plan.ws_ml_off;
+  c->err_off = plan.err_off;
   c->slots = plan.slots;
   c->q_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
   c->n_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
   cudaError_t e = cudaGetDevice(&c->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device);
   if (e == cudaSuccess) e = cudaMemset(c->arena + c->lens_off, 0, (size_t)cfg->num_layers * cfg->max_batch * 8);
+  if (e == cudaSuccess) e = cudaMemset(c->arena + c->err_off, 0, 4);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     delete c;
@@ -337,22 +344,40 @@ kvq_status kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, void
   if (!aligned16(q) || !aligned16(out)) return fail(KVQ_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
   const kvq_config& cfg = c->cfg;
   const int G = cfg.group_k;
-  // Split plan: enough quantized splits to give every SM several CTAs.
-  int64_t total_blocks = 0;
+  const kvq::LayerView L = layer_view(c, layer);
+  const bool use_mma = kvq::mma_supported(L);
+  kvq::MmaPlan mp{};
+  int per_sm = 4;
+  if (use_mma) {
+    mp = kvq::make_mma_plan(L);
+    per_sm = kvq::mma_ctas_per_sm(L, mp);
+  }
+  // Split plan: blocks per split chosen to minimise (waves of CTAs) x (blocks
+  // per CTA + a fixed per-CTA overhead), with at most slots-1 splits.
+  std::vector<int> nblk(batch);
   int max_blk = 0;
   for (int b = 0; b < batch; ++b) {
-    const int nb = c->q_len[(size_t)layer * cfg.max_batch + b] / G;
-    total_blocks += nb;
-    if (nb > max_blk) max_blk = nb;
+    nblk[b] = c->q_len[(size_t)layer * cfg.max_batch + b] / G;
+    max_blk = std::max(max_blk, nblk[b]);
   }
-  const int64_t target_ctas = 148 * 4;
-  int64_t bps = (total_blocks * cfg.num_kv_heads + target_ctas - 1) / target_ctas;
-  if (bps < 1) bps = 1;
-  const int64_t min_bps = (max_blk + (c->slots - 1) - 1) / (c->slots - 1);
-  if (bps < min_bps) bps = min_bps;
+  const int64_t slots_gpu = (int64_t)std::max(1, c->sm_count) * per_sm;
+  const int64_t min_bps = std::max<int64_t>(1, (max_blk + (c->slots - 1) - 1) / (c->slots - 1));
+  int64_t bps = std::max<int64_t>(min_bps, max_blk);
+  double best = 1e300;
+  for (int64_t cand = min_bps; cand <= std::max<int64_t>(min_bps, max_blk); ++cand) {
+    int64_t ctas = 0;
+    for (int b = 0; b < batch; ++b) ctas += (nblk[b] + cand - 1) / cand;
+    ctas *= cfg.num_kv_heads;
+    const double waves = (double)((ctas + slots_gpu - 1) / slots_gpu);
+    const double cost = waves * (double)(cand + 2);
+    if (cost < best) {
+      best = cost;
+      bps = cand;
+    }
+  }
   const int max_splits = (int)((max_blk + bps - 1) / bps);
   kvq::DecodeParams p;
-  p.L = layer_view(c, layer);
+  p.L = L;
   p.q = q;
   p.out = out;
   p.ws_o = reinterpret_cast<float*>(c->arena + c->ws_o_off);
@@ -363,6 +388,13 @@ kvq_status kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, void
   p.num_q_heads = cfg.num_q_heads;
   p.blocks_per_split = (int32_t)bps;
   p.slots = c->slots;
+  p.err = reinterpret_cast<int32_t*>(c->arena + c->err_off);
+  if (use_mma) {
+    cudaError_t e = kvq::launch_decode_mma(p, mp, max_splits, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = kvq::launch_combine(p, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    return KVQ_OK;
+  }
   cudaError_t e = kvq::launch_decode(p, max_splits, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return KVQ_OK;
@@ -383,6 +415,17 @@ kvq_status kvq_dequant(kvq_cache* c, int32_t layer, int32_t seq, int32_t t0, int
   cudaError_t e = kvq::launch_dequant(layer_view(c, layer), seq, t0, t1, k_out, v_out,
                                       static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "dequant launch");
+  return KVQ_OK;
+}
+
+kvq_status kvq_device_errors(kvq_cache* c, int32_t* flags) {
+  g_last_error.clear();
+  if (!c || !flags) return fail(KVQ_ERR_INVALID_ARG, "cache or flags is null");
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpy(&v, c->arena + c->err_off, 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && v != 0) e = cudaMemset(c->arena + c->err_off, 0, 4);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  *flags = v;
   return KVQ_OK;
 }
 

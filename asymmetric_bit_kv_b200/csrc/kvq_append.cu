@@ -75,11 +75,12 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_blocks_kernel(AppendPa
     const GroupParams gp = group_params(mn, mx, kb);
     ksz[d] = __halves2half2(gp.d16, gp.m16);
     const int per = 32 / kb;
-    for (int w = 0; w < G / per; ++w) {
+    const int nw = G / per;  // words per channel, stored contiguously
+    for (int w = 0; w < nw; ++w) {
       uint32_t word = 0;
       for (int i = 0; i < per; ++i)
         word |= quant_code(bits_to_float(sk[(w * per + i) * D + d], dt), gp, kb) << (i * kb);
-      kc[w * D + d] = word;
+      kc[d * nw + w] = word;
     }
   }
 
@@ -156,7 +157,7 @@ __global__ void dequant_kernel(LayerView L, int seq, int t0, int n, float* k_out
       const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + L.kc_off);
       const __half2 ksz = reinterpret_cast<const __half2*>(rec + L.ksz_off)[d];
       const int kper = 32 / kb;
-      const uint32_t kq = (kc[(t / kper) * D + d] >> ((t % kper) * kb)) & ((1u << kb) - 1);
+      const uint32_t kq = (kc[d * (G / kper) + t / kper] >> ((t % kper) * kb)) & ((1u << kb) - 1);
       k_out[o] = dequant_value(kq, __low2half(ksz), __high2half(ksz));
       const uint32_t* vc = reinterpret_cast<const uint32_t*>(rec + L.vc_off);
       const int vper = 32 / vb;

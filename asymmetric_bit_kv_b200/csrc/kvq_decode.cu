@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int d = lane + 32 * c;
-          kcode[c] = (float)((kc[(t / kper) * D + d] >> ((t % kper) * kb)) & kmask);
+          kcode[c] = (float)((kc[d * (G / kper) + t / kper] >> ((t % kper) * kb)) & kmask);
           const uint32_t vq = (vc[t * (D / vper) + d / vper] >> ((d % vper) * vb)) & vmask;
           const __half2 sz = vsz[t * (D / Gv) + d / Gv];
           vv[c] = (float)vq * __low2float(sz) + __high2float(sz);
@@ -221,6 +221,11 @@ cudaError_t launch_decode(const DecodeParams& p, int max_splits, cudaStream_t st
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
+  return launch_combine(p, stream);
+}
+
+cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream) {
+  if (p.batch <= 0) return cudaSuccess;
   combine_kernel<<<dim3(p.num_q_heads, p.batch), kHeadDim, 0, stream>>>(p);
   return cudaGetLastError();
 }

@@ -86,6 +86,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kvq_decode_attention": (I32, [P, I32, P, P, I32, F32, I32, P]),
         "kvq_dequant": (I32, [P, I32, I32, I32, I32, P, P, P]),
         "kvq_get_layout": (I32, [P, I32, ctypes.POINTER(kvq_layout)]),
+        "kvq_device_errors": (I32, [P, ctypes.POINTER(I32)]),
         "kvq_seq_lengths": (I32, [P, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32)]),
         "kvq_status_string": (ctypes.c_char_p, [I32]),
         "kvq_last_error": (ctypes.c_char_p, []),
@@ -211,6 +212,12 @@ class KVCache:
         _check(self.lib.kvq_dequant(self.handle, layer, seq, t0, t1, k.data_ptr(), v.data_ptr(), _stream_ptr(stream)),
                "kvq_dequant")
         return k, v
+
+    def device_errors(self) -> int:
+        """Device error flags since the last call (0 = none); synchronises."""
+        f = ctypes.c_int32()
+        _check(self.lib.kvq_device_errors(self.handle, ctypes.byref(f)), "kvq_device_errors")
+        return f.value
 
     def layout(self, layer: int) -> kvq_layout:
         lay = kvq_layout()

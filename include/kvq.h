@@ -92,9 +92,10 @@ typedef struct kvq_cache kvq_cache;
  * [j*G, (j+1)*G) of that sequence) the record starts at
  *   blocks + ((b * num_kv_heads + h) * max_blocks + j) * record_bytes
  * and holds, at the given byte offsets:
- *   kc  uint32 [G*k_bits/32][D]: word w of channel d packs the codes of
+ *   kc  uint32 [D][G*k_bits/32]: word w of channel d packs the codes of
  *       tokens w*(32/k_bits) + i, i = 0.., code i at bits [i*k_bits, ...)
- *       (per-channel keys, packed along the token axis);
+ *       (per-channel keys, packed along the token axis; each channel's
+ *       words are contiguous);
  *   ksz half2 [D]: (scale d, zero point m) of each channel's key group;
  *   vc  uint32 [G][D*v_bits/32]: word w of token t packs the codes of
  *       channels w*(32/v_bits) + i, code i at bits [i*v_bits, ...)
@@ -163,6 +164,12 @@ KVQ_API kvq_status kvq_decode_attention(kvq_cache* cache, int32_t layer, const v
  * [t1-t0][num_kv_heads][head_dim] fp32. 0 <= t0 <= t1 <= sequence length.  */
 KVQ_API kvq_status kvq_dequant(kvq_cache* cache, int32_t layer, int32_t seq, int32_t t0, int32_t t1,
                        float* k_out, float* v_out, void* stream);
+
+/* Device-side failures recorded since the last call, then cleared: bit 0 =
+ * a decode kernel gave up a bounded wait on its copy pipeline (its partial
+ * results are invalid). Synchronous: waits for the device to finish its
+ * work.                                                                   */
+KVQ_API kvq_status kvq_device_errors(kvq_cache* cache, int32_t* flags);
 
 /* Layer layout (see kvq_layout).                                           */
 KVQ_API kvq_status kvq_get_layout(const kvq_cache* cache, int32_t layer, kvq_layout* out);

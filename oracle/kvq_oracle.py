@@ -170,14 +170,13 @@ def dequantize_value_block(codes, d16, m16):
 
 
 # Word arrangement of the library's packed block (documented in its header):
-# key words [H, G*bits/32, D] (word w of channel d holds tokens w*32/bits ...),
+# key words [H, D, G*bits/32] (word w of channel d holds tokens w*32/bits ...),
 # value words [H, G, D*bits/32] (word w of a token holds channels w*32/bits ...).
 
 
 def pack_key_block(codes: np.ndarray, bits: int) -> np.ndarray:
-    """codes [G, H, D] -> uint32 [H, G*bits/32, D], packed along tokens."""
-    words = pack_codes(np.transpose(codes, (1, 2, 0)), bits)   # [H, D, W]
-    return np.ascontiguousarray(np.transpose(words, (0, 2, 1)))
+    """codes [G, H, D] -> uint32 [H, D, G*bits/32], packed along tokens."""
+    return pack_codes(np.transpose(codes, (1, 2, 0)), bits)       # [H, D, W]
 
 
 def pack_value_block(codes: np.ndarray, bits: int) -> np.ndarray:

@@ -87,7 +87,7 @@ class Twin:
         kcw = G * kb // 32
         vcw = D * vb // 32
         return {
-            "kc": part(lay.kc_offset, kcw * D * 4, np.uint32, (kcw, D)),
+            "kc": part(lay.kc_offset, kcw * D * 4, np.uint32, (D, kcw)),
             "ksz": part(lay.ksz_offset, D * 4, np.float16, (D, 2)),
             "vc": part(lay.vc_offset, G * vcw * 4, np.uint32, (G, vcw)),
             "vsz": part(lay.vsz_offset, G * (D // Gv) * 4, np.float16, (G, D // Gv, 2)),

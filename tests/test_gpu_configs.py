@@ -1,0 +1,143 @@
+"""Parity on the five workload shapes at full size.
+
+Every device result that the oracle can afford is compared: all packed codes,
+scales and zero points of the sampled sequences bit for bit, and their decode
+outputs within the attention tolerance. Sequences the oracle does not replay
+are checked through their lengths (the flush rule) and finite outputs.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from asymmetric_bit_kv_b200 import CacheConfig
+from asymmetric_bit_kv_b200 import workloads as W
+from kvq_testutil import Twin, assert_attention_close, ulp
+
+pytestmark = pytest.mark.gpu
+
+
+def _cfg(wl: W.Workload, max_tokens: int, max_batch: int | None = None) -> CacheConfig:
+    return CacheConfig(wl.num_layers, max_batch or wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, max_tokens,
+                       wl.group_k, wl.group_v, wl.residual, wl.kv_dtype, wl.k_bits, wl.v_bits)
+
+
+def _expected_lengths(L, R, G):
+    q = 0 if L <= R else G * -(-(L - R) // G)
+    return q, L - q
+
+
+def _decode_and_check(tw: Twin, wl: W.Workload, layer: int, q: torch.Tensor, seqs, out_dtype=torch.float32):
+    out = tw.gpu.decode_attention(layer, q.cuda(), out_dtype=out_dtype, softmax_scale=wl.softmax_scale)
+    assert tw.gpu.device_errors() == 0
+    out = out.float().cpu().numpy()
+    assert np.isfinite(out).all()
+    qn = q.float().numpy()
+    for b in seqs:
+        ref = tw.oracle_decode(layer, b, qn[b], wl.softmax_scale)
+        if out_dtype == torch.float32:
+            assert_attention_close(out[b], ref, f"layer {layer} seq {b}")
+        else:
+            assert np.all(np.abs(out[b] - ref) <= ulp(ref, out_dtype) / 2 + 2e-3)
+    return out
+
+
+def test_tiny_mha_full():
+    wl = W.tiny_mha()
+    tw = Twin(_cfg(wl, 2048))
+    k, v = W.generate_tokens(wl, 0, wl.context)
+    tw.append(0, k, v, wl.context)
+    tw.check_lengths(0, 1)
+    assert tw.gpu.lengths(0, 0) == (992, 32)
+    tw.check_codes(0, 0)
+    tw.check_dequant(0, 0)
+    q = W.generate_queries(wl, 0, 1)
+    _decode_and_check(tw, wl, 0, q, [0])
+    _decode_and_check(tw, wl, 0, q, [0], out_dtype=torch.float16)
+
+
+def test_llama2_mha_256_decode_steps():
+    wl = W.llama2_7b_mha()
+    steps = wl.extra["decode_steps"]
+    tw = Twin(_cfg(wl, 4096 + steps + 64))
+    B = wl.batch
+    k, v = W.generate_tokens(wl, 0, wl.context)
+    tw.append(0, k, v, wl.context)
+    kn, vn = W.generate_tokens(wl, 0, [steps] * B, seed_offset=1)
+    kn = kn.view(B, steps, wl.num_kv_heads, wl.head_dim)
+    vn = vn.view(B, steps, wl.num_kv_heads, wl.head_dim)
+    check_at = {0, 1, 30, 31, 32, 33, 127, 128, steps - 1}
+    for step in range(steps):
+        tw.append(0, kn[:, step].contiguous(), vn[:, step].contiguous(), [1] * B)
+        if step in check_at:
+            q = W.generate_queries(wl, 0, B, step=step)
+            _decode_and_check(tw, wl, 0, q, range(B))
+    tw.check_lengths(0, B)
+    assert tw.gpu.lengths(0, 0) == _expected_lengths(4096 + steps, wl.residual, wl.group_k)
+    for b in range(B):
+        tw.check_codes(0, b)
+
+
+def test_llama3_gqa_sampled():
+    wl = W.llama3_8b_gqa()
+    sample = [0, 17, 31]
+    tw = Twin(_cfg(wl, 8192 + 64), oracle_seqs=sample)
+    k, v = W.generate_tokens(wl, 0, wl.context)
+    tw.append(0, k, v, wl.context)
+    for b in range(wl.batch):
+        assert tw.gpu.lengths(0, b) == (8064, 128)
+    for b in sample:
+        tw.check_codes(0, b)
+    q = W.generate_queries(wl, 0, wl.batch)
+    _decode_and_check(tw, wl, 0, q, sample)
+    _decode_and_check(tw, wl, 0, q, sample, out_dtype=torch.bfloat16)
+
+
+def test_long_context_and_prefill_chunk():
+    wl = W.long_context_gqa()
+    L = wl.context[0]
+    chunk = wl.extra["prefill_chunk"]
+    tw = Twin(_cfg(wl, L + 64, max_batch=2))
+    k, v = W.generate_tokens(wl, 0, [L])
+    # the long context arrives in a few large appends
+    pos = 0
+    for n in (50000, 1, 70000, L - 120001):
+        tw.append(0, k[pos:pos + n], v[pos:pos + n], [n, 0])
+        pos += n
+    assert tw.gpu.lengths(0, 0) == (130944, 128)
+    # the prefill chunk: one call, on a fresh sequence
+    kc, vc = W.generate_tokens(wl, 0, [chunk], seed_offset=9)
+    tw.append(0, kc, vc, [0, chunk])
+    assert tw.gpu.lengths(0, 1) == (3968, 128)
+    tw.check_codes(0, 1)
+    tw.check_dequant(0, 1)
+    tw.check_codes(0, 0)
+    q = W.generate_queries(wl, 0, 2)
+    _decode_and_check(tw, wl, 0, q, [0, 1])
+
+
+def test_qwen3_36_layers_ragged_sampled():
+    wl = W.qwen3_8b_layers()
+    ctx = wl.context
+    B = wl.batch
+    lo, hi = int(np.argmin(ctx)), int(np.argmax(ctx))
+    layers = [0, 4, 35]
+    tw = Twin(_cfg(wl, max(ctx) + 64), oracle_seqs=[lo, hi], oracle_layers=layers)
+    offs = np.concatenate([[0], np.cumsum(ctx)])
+    q = W.generate_queries(wl, 0, B)
+    for layer in range(wl.num_layers):
+        k, v = W.generate_tokens(wl, layer, ctx, device="cuda")
+        tw.gpu.append(layer, k, v, ctx)
+        if layer in layers:
+            for b in (lo, hi):
+                sl = slice(int(offs[b]), int(offs[b + 1]))
+                tw.ora[(layer, b)].append(k[sl].float().cpu().numpy(), v[sl].float().cpu().numpy())
+        del k, v
+        out = tw.gpu.decode_attention(layer, q.cuda(), softmax_scale=wl.softmax_scale)
+        assert torch.isfinite(out).all()
+    for b in range(B):
+        assert tw.gpu.lengths(35, b) == _expected_lengths(ctx[b], wl.residual, wl.group_k)
+    for layer in layers:
+        for b in (lo, hi):
+            tw.check_codes(layer, b)
+        _decode_and_check(tw, wl, layer, q, [lo, hi])

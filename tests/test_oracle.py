@@ -142,9 +142,9 @@ def test_block_word_arrangement():
     rng = np.random.default_rng(0)
     codes = rng.integers(0, 4, size=(G, H, D)).astype(np.uint8)
     kw = O.pack_key_block(codes, b)
-    assert kw.shape == (H, G * b // 32, D)
+    assert kw.shape == (H, D, G * b // 32)
     for h, w, d in [(0, 0, 0), (1, 1, 31), (0, 1, 7)]:
-        assert np.array_equal(O.unpack_codes(kw[h, w, d][None], b), codes[w * 16:(w + 1) * 16, h, d])
+        assert np.array_equal(O.unpack_codes(kw[h, d, w][None], b), codes[w * 16:(w + 1) * 16, h, d])
     vw = O.pack_value_block(codes, b)
     assert vw.shape == (H, G, D * b // 32)
     for h, t, w in [(0, 0, 0), (1, 31, 1), (1, 5, 0)]:
