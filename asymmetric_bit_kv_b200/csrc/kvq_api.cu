@@ -114,7 +114,11 @@ Plan make_plan(const kvq_config* c) {
   off = round_up(off + (int64_t)c->num_layers * c->max_batch * 2 * 4, 256);
   p.err_off = off;
   off = round_up(off + 4, 256);
-  p.slots = (int32_t)std::min<int64_t>(p.max_blocks, KVQ_MAX_SPLITS) + 1;
+  // partial slots per (sequence, query head): enough for the split kernel
+  // (one per split + the ring) and for the persistent kernel (4 for the ring,
+  // 4 per CTA range overlapping the sequence, at most 64 such ranges)
+  p.slots = (int32_t)std::max<int64_t>(std::min<int64_t>(p.max_blocks, KVQ_MAX_SPLITS) + 1,
+                                       4 + 4 * (std::min<int64_t>(p.max_blocks, 64) + 1));
   const int64_t partials = (int64_t)c->max_batch * c->num_q_heads * p.slots;
   p.ws_o_off = off;
   off = round_up(off + partials * D * 4, 256);
@@ -352,31 +356,19 @@ kvq_status kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, void
     mp = kvq::make_mma_plan(L);
     per_sm = kvq::mma_ctas_per_sm(L, mp);
   }
-  // Split plan: blocks per split chosen to minimise (waves of CTAs) x (blocks
-  // per CTA + a fixed per-CTA overhead), with at most slots-1 splits.
   std::vector<int> nblk(batch);
   int max_blk = 0;
+  int64_t total_blocks = 0;
   for (int b = 0; b < batch; ++b) {
     nblk[b] = c->q_len[(size_t)layer * cfg.max_batch + b] / G;
     max_blk = std::max(max_blk, nblk[b]);
+    total_blocks += (int64_t)nblk[b] * cfg.num_kv_heads;
   }
-  const int64_t slots_gpu = (int64_t)std::max(1, c->sm_count) * per_sm;
-  const int64_t min_bps = std::max<int64_t>(1, (max_blk + (c->slots - 1) - 1) / (c->slots - 1));
-  int64_t bps = std::max<int64_t>(min_bps, max_blk);
-  double best = 1e300;
-  for (int64_t cand = min_bps; cand <= std::max<int64_t>(min_bps, max_blk); ++cand) {
-    int64_t ctas = 0;
-    for (int b = 0; b < batch; ++b) ctas += (nblk[b] + cand - 1) / cand;
-    ctas *= cfg.num_kv_heads;
-    const double waves = (double)((ctas + slots_gpu - 1) / slots_gpu);
-    const double cost = waves * (double)(cand + 2);
-    if (cost < best) {
-      best = cost;
-      bps = cand;
-    }
-  }
-  const int max_splits = (int)((max_blk + bps - 1) / bps);
-  kvq::DecodeParams p;
+  if (total_blocks > INT32_MAX) return fail(KVQ_ERR_UNSUPPORTED, "more than 2^31 quantized blocks in one call");
+  kvq::DecodeParams* pp = new (std::nothrow) kvq::DecodeParams;
+  if (!pp) return fail(KVQ_ERR_INVALID_ARG, "out of host memory");
+  kvq::DecodeParams& p = *pp;
+  std::memset(pp, 0, sizeof *pp);
   p.L = L;
   p.q = q;
   p.out = out;
@@ -386,16 +378,57 @@ kvq_status kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, void
   p.out_dtype = out_dtype;
   p.batch = batch;
   p.num_q_heads = cfg.num_q_heads;
-  p.blocks_per_split = (int32_t)bps;
   p.slots = c->slots;
   p.err = reinterpret_cast<int32_t*>(c->arena + c->err_off);
+  cudaError_t e;
   if (use_mma) {
-    cudaError_t e = kvq::launch_decode_mma(p, mp, max_splits, static_cast<cudaStream_t>(stream));
+    // Persistent plan: one CTA per resident slot (fewer if there is little
+    // work), each taking a contiguous range of the concatenated blocks.
+    int64_t nctas = std::min<int64_t>((int64_t)std::max(1, c->sm_count) * per_sm,
+                                      std::max<int64_t>((int64_t)batch * cfg.num_kv_heads, (total_blocks + 3) / 4));
+    nctas = std::max<int64_t>(nctas, 1);
+    // every (sequence, head) must fit its partials in the workspace
+    int64_t acc = 0;
+    for (int b = 0; b < batch; ++b) {
+      p.nblk[b] = nblk[b];
+      p.seq_start[b] = (int32_t)acc;
+      acc += (int64_t)nblk[b] * cfg.num_kv_heads;
+    }
+    for (;;) {
+      int32_t need = kvq::kResidualSlots;
+      for (int b = 0; b < batch && total_blocks > 0; ++b)
+        for (int h = 0; h < cfg.num_kv_heads; ++h)
+          need = std::max(need, kvq::persistent_slots(total_blocks, (int32_t)nctas, p.seq_start[b] + h * nblk[b], nblk[b]));
+      if (need <= c->slots || nctas == 1) break;
+      nctas = std::max<int64_t>(1, nctas * 3 / 4);
+    }
+    p.persistent = 1;
+    p.total_blocks = (int32_t)total_blocks;
+    p.num_ctas = (int32_t)nctas;
+    e = kvq::launch_decode_mma(p, mp, 0, static_cast<cudaStream_t>(stream));
     if (e == cudaSuccess) e = kvq::launch_combine(p, static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-    return KVQ_OK;
+  } else {
+    // Split plan: blocks per split chosen to minimise (waves of CTAs) x
+    // (blocks per CTA + a fixed per-CTA overhead), with at most slots-1 splits.
+    const int64_t slots_gpu = (int64_t)std::max(1, c->sm_count) * per_sm;
+    const int64_t min_bps = std::max<int64_t>(1, (max_blk + (c->slots - 1) - 1) / (c->slots - 1));
+    int64_t bps = std::max<int64_t>(min_bps, max_blk);
+    double best = 1e300;
+    for (int64_t cand = min_bps; cand <= std::max<int64_t>(min_bps, max_blk); ++cand) {
+      int64_t ctas = 0;
+      for (int b = 0; b < batch; ++b) ctas += (nblk[b] + cand - 1) / cand;
+      ctas *= cfg.num_kv_heads;
+      const double waves = (double)((ctas + slots_gpu - 1) / slots_gpu);
+      const double cost = waves * (double)(cand + 2);
+      if (cost < best) {
+        best = cost;
+        bps = cand;
+      }
+    }
+    p.blocks_per_split = (int32_t)bps;
+    e = kvq::launch_decode(p, (int)((max_blk + bps - 1) / bps), static_cast<cudaStream_t>(stream));
   }
-  cudaError_t e = kvq::launch_decode(p, max_splits, static_cast<cudaStream_t>(stream));
+  delete pp;
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return KVQ_OK;
 }

@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_blocks_kernel(AppendPa
       uint32_t word = 0;
       for (int i = 0; i < per; ++i)
         word |= quant_code(bits_to_float(sk[(w * per + i) * D + d], dt), gp, kb) << (i * kb);
-      kc[d * nw + w] = word;
+      kc[kc_word_index(d, w, nw)] = word;
     }
   }
 
@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_blocks_kernel(AppendPa
     const GroupParams gp = group_params(mn, mx, vb);
     uint32_t word = 0;
     for (int i = 0; i < per; ++i) word |= quant_code(bits_to_float(xs[i], dt), gp, vb) << (i * vb);
-    vc[t * wpt + w] = word;
+    vc[vc_word_index(t, w, G, kb, wpt)] = word;
     if ((w % P) == 0) vsz[t * (D / Gv) + w / P] = __halves2half2(gp.d16, gp.m16);
   }
 }
@@ -157,11 +157,11 @@ __global__ void dequant_kernel(LayerView L, int seq, int t0, int n, float* k_out
       const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + L.kc_off);
       const __half2 ksz = reinterpret_cast<const __half2*>(rec + L.ksz_off)[d];
       const int kper = 32 / kb;
-      const uint32_t kq = (kc[d * (G / kper) + t / kper] >> ((t % kper) * kb)) & ((1u << kb) - 1);
+      const uint32_t kq = (kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb)) & ((1u << kb) - 1);
       k_out[o] = dequant_value(kq, __low2half(ksz), __high2half(ksz));
       const uint32_t* vc = reinterpret_cast<const uint32_t*>(rec + L.vc_off);
       const int vper = 32 / vb;
-      const uint32_t vq = (vc[t * (D / vper) + d / vper] >> ((d % vper) * vb)) & ((1u << vb) - 1);
+      const uint32_t vq = (vc[vc_word_index(t, d / vper, G, kb, D / vper)] >> ((d % vper) * vb)) & ((1u << vb) - 1);
       const __half2 vsz = reinterpret_cast<const __half2*>(rec + L.vsz_off)[t * (D / L.group_v) + d / L.group_v];
       v_out[o] = dequant_value(vq, __low2half(vsz), __high2half(vsz));
     } else {

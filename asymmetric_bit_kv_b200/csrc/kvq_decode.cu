@@ -122,8 +122,8 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int d = lane + 32 * c;
-          kcode[c] = (float)((kc[d * (G / kper) + t / kper] >> ((t % kper) * kb)) & kmask);
-          const uint32_t vq = (vc[t * (D / vper) + d / vper] >> ((d % vper) * vb)) & vmask;
+          kcode[c] = (float)((kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb)) & kmask);
+          const uint32_t vq = (vc[vc_word_index(t, d / vper, G, kb, D / vper)] >> ((d % vper) * vb)) & vmask;
           const __half2 sz = vsz[t * (D / Gv) + d / Gv];
           vv[c] = (float)vq * __low2float(sz) + __high2float(sz);
         }
@@ -174,8 +174,14 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeParams p) {
   const int hq = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const LayerView& L = p.L;
   constexpr int D = kHeadDim;
-  const int nblk = L.lens[2 * b] / L.group_k;
-  const int S = (nblk + p.blocks_per_split - 1) / p.blocks_per_split;
+  int S;  // slots 0..S hold this (sequence, head)'s partials
+  if (p.persistent) {
+    const int h = hq / (p.num_q_heads / L.num_kv_heads);
+    S = persistent_slots(p.total_blocks, p.num_ctas, p.seq_start[b] + h * p.nblk[b], p.nblk[b]) - 1;
+  } else {
+    const int nblk = L.lens[2 * b] / L.group_k;
+    S = (nblk + p.blocks_per_split - 1) / p.blocks_per_split;
+  }
   const int64_t base = ((int64_t)b * p.num_q_heads + hq) * p.slots;
   float M = -INFINITY;
   for (int s = 0; s <= S; ++s) {

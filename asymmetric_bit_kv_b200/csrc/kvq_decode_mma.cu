@@ -6,22 +6,29 @@
 //
 // Design (HBM-bound; tensor cores only take the dot products off the ALUs):
 //  * One CTA per (split, KV head, sequence); split 0 is the residual ring.
-//    Warp 4 is a producer: one lane streams whole block records from HBM into
-//    a ring of shared-memory stages with cp.async.bulk (1-D TMA) completing on
-//    mbarriers. Warps 0-3 each consume every fourth block.
+//    Warp roles: a producer warp (one lane) streams each block record from
+//    HBM into a ring of shared-memory stages with ONE cp.async.bulk (1-D TMA)
+//    completing on an mbarrier -- the record layout is already the
+//    bank-conflict-free shared-memory layout, so no per-row copies are
+//    needed; a prep warp turns each landed block's fp16 scales into the
+//    per-block operands (below) next to the record; NC consumer warps each
+//    own NS/NC stages. Stage hand-offs: full (TMA landed) -> ready (operands
+//    prepared) -> empty (consumed).
 //  * Keys: per block, q.k_hat = sum_d (q_d s_d) c_d + sum_d q_d z_d. The
-//    scaled query (q_d s_d) is split into an fp16 high part and an fp16
-//    low part (rows 0-7 and 8-15 of the m16n8k16 A operand), the codes c are
-//    the B operand. Codes reach registers with ldmatrix.trans from the
-//    channel-major key rows (two channels of the same tokens per register),
-//    and become exact fp16 integers with one lop3 (mask | 0x6400 exponent)
-//    and one hsub2 (minus 1024). A code taken from bit position p is c * 2^p;
-//    the score is rescaled by 2^-p afterwards (exact).
+//    scaled query (q_d s_d) is split into fp16 high and low parts, rows 0-7
+//    and 8-15 of the m16n8k16 A operand (the prep warp writes them in
+//    fragment order), the codes c are the B operand. Codes reach registers
+//    with ldmatrix.trans from the channel-major key rows (two channels of the
+//    same tokens per register) and become exact fp16 integers with one lop3
+//    (mask | 0x6400 exponent) and one hsub2 (minus 1024). A code taken from
+//    bit position p is c * 2^p; the score is rescaled by 2^-p (exact).
 //  * Values: o[ch][head] = sum_t (p_t s_t) c_t,ch + sum_t p_t z_t. The value
-//    codes of two tokens per register come from ldmatrix.trans over the
-//    token rows (the A operand, channels on M); the probabilities times the
-//    token's value scale are the fp16 B operand (tokens on K, heads on N).
-//    The zero-point term is accumulated in fp32 on the side.
+//    codes of two tokens per register come from ldmatrix.trans over token
+//    rows (the A operand, channels on M); p*s in fp16 (one hmul2 of the
+//    packed probabilities and the prep warp's packed scales) is the B operand
+//    (tokens on K, heads on N) built straight from the score accumulators'
+//    registers. The zero-point term sum_t p_t z_t is one more MMA per value
+//    group with an all-ones A operand.
 //  * Online softmax in log2 units per 64-token tile; fp32 partials per split
 //    are merged by the log-sum-exp combine kernel.
 #include "kvq_decode.cuh"
@@ -30,8 +37,9 @@ namespace kvq {
 
 namespace {
 
-constexpr int kConsumerWarps = 4;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kNC = 4;                    // consumer warps
+constexpr int kProdWarp = kNC;            // warp index of the producer warp
+constexpr int kThreads = (kNC + 1) * 32;
 constexpr long long kWaitCycles = 4000000000LL;  // a bounded wait gives up after ~2 s
 
 // ---------------------------------------------------------------- PTX helpers
@@ -90,13 +98,19 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// (a & b) | c in one instruction.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
 // Codes selected by `mask` in both 16-bit halves of x, as exact fp16 integers
 // (times the power of two of their bit position): (x & mask) | 1024.0h, then
 // minus 1024.0h.
-__device__ __forceinline__ uint32_t codes_to_f16(uint32_t x, uint32_t mask) {
-  uint32_t r = (x & mask) | 0x64006400u;
+__device__ __forceinline__ uint32_t codes_to_f16(uint32_t x, uint32_t mask, uint32_t magic) {
+  uint32_t r = and_or(x, mask, magic);
   __half2 h = *reinterpret_cast<__half2*>(&r);
-  h = __hsub2(h, __halves2half2(__ushort_as_half((unsigned short)0x6400), __ushort_as_half((unsigned short)0x6400)));
+  h = __hsub2(h, *reinterpret_cast<const __half2*>(&magic));
   return *reinterpret_cast<uint32_t*>(&h);
 }
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
@@ -106,99 +120,103 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
 __device__ __forceinline__ float2 unpack_f16(uint32_t x) {
   return __half22float2(*reinterpret_cast<__half2*>(&x));
 }
-__device__ __forceinline__ float warp_sum(float x) {
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
 }
 
 // ------------------------------------------------------- residual ring split
-// Exact attention over the ring tokens [Q, Q+n) of (b, h) with CUDA cores;
-// warps 0-3 each take every fourth token. Writes partial slot 0.
-__device__ void residual_partial(const DecodeParams& p, int b, int h, int NG, int Q, int n, uint8_t* smem) {
+// Consumer warp w takes every kNC-th ring token of unit (b, h) with CUDA
+// cores and writes its own partial (slot w). Lane l owns channels 4l..4l+3;
+// the K/V rows of kRB tokens are loaded (8-byte loads) before they are used.
+constexpr int kRB = 4;
+
+__device__ __forceinline__ void load4(const void* base, int64_t elem, int dtype, float (&x)[4]) {
+  const uint2 v = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(base) + elem);
+  const uint32_t w[2] = {v.x, v.y};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    if (dtype == KVQ_BF16) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    } else {
+      const float2 f = unpack_f16(w[i]);
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+  }
+}
+
+__device__ void residual_unit(const DecodeParams& p, int b, int h, int NG, const float* wq) {
   const LayerView& L = p.L;
   constexpr int D = kHeadDim;
-  float* sq = reinterpret_cast<float*>(smem);  // [8][D]
-  float* so = sq + 8 * D;                      // [4][8][D]
-  float* sm = so + 4 * 8 * D;                  // [4][8]
-  float* sl = sm + 32;                         // [4][8]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < NG * D; i += blockDim.x)
-    sq[i] = load_kv(p.q, ((int64_t)b * p.num_q_heads + h * NG) * D + i, L.kv_dtype) * p.scale_log2;
-  __syncthreads();
-  float m[8], l[8], o[8][4];
+  const int Q = L.lens[2 * b], n = L.lens[2 * b + 1];
+  float m[8], l[8], o[8][4], qv[8][4];
 #pragma unroll
   for (int hh = 0; hh < 8; ++hh) {
     m[hh] = -INFINITY;
     l[hh] = 0.f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) o[hh][c] = 0.f;
+    for (int c = 0; c < 4; ++c) {
+      o[hh][c] = 0.f;
+      qv[hh][c] = (hh < NG) ? wq[hh * D + 4 * lane + c] : 0.f;
+    }
   }
-  if (warp < kConsumerWarps) {
-    const int64_t base = ((int64_t)b * L.num_kv_heads + h) * L.residual;
-    for (int i = Q + warp; i < Q + n; i += kConsumerWarps) {
-      const int64_t row = (base + i % L.residual) * D;
-      float kv[4], vv[4];
+  const int64_t base = ((int64_t)b * L.num_kv_heads + h) * L.residual;
+  for (int i0 = Q + warp; i0 < Q + n; i0 += kNC * kRB) {
+    float kv[kRB][4], vv[kRB][4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        kv[c] = load_kv(L.ring_k, row + lane + 32 * c, L.kv_dtype);
-        vv[c] = load_kv(L.ring_v, row + lane + 32 * c, L.kv_dtype);
-      }
-#pragma unroll
-      for (int hh = 0; hh < 8; ++hh) {
-        if (hh < NG) {
-          float part = 0.f;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) part += sq[hh * D + lane + 32 * c] * kv[c];
-          const float sc = warp_sum(part);
-          const float mn = fmaxf(m[hh], sc);
-          const float alpha = ex2(m[hh] - mn);
-          const float pe = ex2(sc - mn);
-          l[hh] = l[hh] * alpha + pe;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) o[hh][c] = o[hh][c] * alpha + pe * vv[c];
-          m[hh] = mn;
-        }
+    for (int r = 0; r < kRB; ++r) {
+      const int i = i0 + r * kNC;
+      if (i < Q + n) {
+        const int64_t row = (base + i % L.residual) * D + 4 * lane;
+        load4(L.ring_k, row, L.kv_dtype, kv[r]);
+        load4(L.ring_v, row, L.kv_dtype, vv[r]);
       }
     }
 #pragma unroll
-    for (int hh = 0; hh < 8; ++hh) {
-      if (hh < NG) {
+    for (int r = 0; r < kRB; ++r) {
+      if (i0 + r * kNC < Q + n) {
+        float sc[8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) so[(warp * 8 + hh) * D + lane + 32 * c] = o[hh][c];
-        if (lane == 0) {
-          sm[warp * 8 + hh] = m[hh];
-          sl[warp * 8 + hh] = l[hh];
+        for (int hh = 0; hh < 8; ++hh)
+          sc[hh] = qv[hh][0] * kv[r][0] + qv[hh][1] * kv[r][1] + qv[hh][2] * kv[r][2] + qv[hh][3] * kv[r][3];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1)
+#pragma unroll
+          for (int hh = 0; hh < 8; ++hh)
+            if (hh < NG) sc[hh] += __shfl_xor_sync(0xffffffffu, sc[hh], off);
+#pragma unroll
+        for (int hh = 0; hh < 8; ++hh) {
+          if (hh < NG) {
+            const float mn = fmaxf(m[hh], sc[hh]);
+            const float alpha = ex2(m[hh] - mn);
+            const float pe = ex2(sc[hh] - mn);
+            l[hh] = l[hh] * alpha + pe;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) o[hh][c] = o[hh][c] * alpha + pe * vv[r][c];
+            m[hh] = mn;
+          }
         }
       }
     }
   }
-  __syncthreads();
-  const int d = threadIdx.x;
-  if (d < D) {
-    for (int hh = 0; hh < NG; ++hh) {
-      float M = -INFINITY;
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm[w * 8 + hh]);
-      float acc = 0.f, lsum = 0.f;
-      if (M != -INFINITY) {
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const float mw = sm[w * 8 + hh];
-          const float f = mw == -INFINITY ? 0.f : ex2(mw - M);
-          acc += so[(w * 8 + hh) * D + d] * f;
-          lsum += sl[w * 8 + hh] * f;
-        }
-      }
-      const int64_t slot = ((int64_t)b * p.num_q_heads + h * NG + hh) * p.slots;
-      p.ws_o[slot * D + d] = acc;
-      if (d == 0) p.ws_ml[slot] = make_float2(M, lsum);
+#pragma unroll
+  for (int hh = 0; hh < 8; ++hh) {
+    if (hh < NG) {
+      const int64_t slot = ((int64_t)b * p.num_q_heads + h * NG + hh) * p.slots + warp;
+      *reinterpret_cast<float4*>(p.ws_o + slot * D + 4 * lane) = make_float4(o[hh][0], o[hh][1], o[hh][2], o[hh][3]);
+      if (lane == 0) p.ws_ml[slot] = make_float2(m[hh], l[hh]);
     }
   }
 }
 
-// --------------------------------------------------------- quantized splits
-template <int KB, int VB, int TT, int NGRP>
+// --------------------------------------------------------- quantized blocks
+template <int KB, int VB, int NGRP>
 struct Shape {
   static constexpr int D = kHeadDim;
+  static constexpr int TT = 64;                 // tokens per tile
   static constexpr int CPT16 = 16 / KB;         // key tokens per 16-bit column
   static constexpr int SIGMA_TOK = 128 / KB;    // key tokens per 16-byte row chunk
   static constexpr int SIG = TT / SIGMA_TOK;    // 16-byte key chunks per tile
@@ -214,35 +232,121 @@ struct Shape {
   static_assert(CH_SPAN <= GV, "a value chunk must lie inside one value group");
 };
 
-template <int KB, int TT>
+// Token (within the tile) of column `col` of n-tile `idx`.
+template <int KB>
 __device__ __forceinline__ int tile_token(int idx, int col) {
   constexpr int CPT16 = 16 / KB, SIGMA_TOK = 128 / KB;
-  (void)TT;
   return (idx / CPT16) * SIGMA_TOK + col * CPT16 + (idx % CPT16);
 }
 
-template <int KB, int VB, int TT, int NGRP>
+// Walks the (sequence, head) units of consecutive global blocks.
+struct UnitCursor {
+  int b = 0, h = 0, start = 0, end = 0;  // current unit and its block range
+  __device__ void seek(const DecodeParams& p, int k) {
+    int lo = 0, hi = p.batch - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.seq_start[mid] <= k) lo = mid;
+      else hi = mid - 1;
+    }
+    b = lo;
+    const int nb = p.nblk[b];
+    h = (k - p.seq_start[b]) / nb;
+    start = p.seq_start[b] + h * nb;
+    end = start + nb;
+  }
+  __device__ void advance(const DecodeParams& p, int k) {
+    if (k >= end || k < start) seek(p, k);
+  }
+};
+
+// Per-warp scratch, rebuilt from each block's fp16 scales before its MMAs:
+//   afrag [8 kk][8 heads][4 t] uint4: rows g (fp16 high) and g+8 (fp16 low)
+//         of (q * s) for channels 16kk + 2t + {0,1,8,9} (A-fragment order);
+//   bias  [8] float: sum_d q_d z_d per head;
+//   vpair [k-step][4 t][groups] uint4: (s_X, s_Y, z_X, z_Y) fp16 pairs of the
+//         tokens thread t feeds into a PV k-step;
+//   wq    [8][D] float: the unit's queries times softmax_scale*log2(e).
+template <int KB, int VB, int NGRP>
+__device__ __forceinline__ void prep_block(const uint8_t* stage, const MmaPlan& mp, uint8_t* ws, int NG, int G,
+                                           int lane) {
+  using S = Shape<KB, VB, NGRP>;
+  constexpr int D = S::D;
+  const float* wq = reinterpret_cast<const float*>(ws + mp.wq_off);
+  uint4* af = reinterpret_cast<uint4*>(ws + mp.afrag_off);
+  const __half2* ksz = reinterpret_cast<const __half2*>(stage + mp.kc_bytes);
+  // (head, kk) pairs: lanes 8hh..8hh+7 take the 8 kk of head hh
+#pragma unroll
+  for (int rep = 0; rep < 2; ++rep) {
+    const int pr = lane + 32 * rep;
+    const int hh = pr >> 3, kk = pr & 7;
+    float bp = 0.f;
+    if (hh < NG) {
+      const float4* q4 = reinterpret_cast<const float4*>(wq + hh * D + 16 * kk);
+      const uint4* s4 = reinterpret_cast<const uint4*>(ksz + 16 * kk);
+      float x[16];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const float4 qq = q4[v];
+        const uint4 ss = s4[v];
+        const float qa[4] = {qq.x, qq.y, qq.z, qq.w};
+        const uint32_t sa[4] = {ss.x, ss.y, ss.z, ss.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 sz = unpack_f16(sa[e]);  // (scale, zero) of channel 16kk + 4v + e
+          x[4 * v + e] = qa[e] * sz.x;
+          bp += qa[e] * sz.y;
+        }
+      }
+#pragma unroll
+      for (int tt = 0; tt < 4; ++tt) {
+        const uint32_t h01 = pack_f16(x[2 * tt], x[2 * tt + 1]), h89 = pack_f16(x[2 * tt + 8], x[2 * tt + 9]);
+        const float2 f01 = unpack_f16(h01), f89 = unpack_f16(h89);
+        af[(kk * 8 + hh) * 4 + tt] = make_uint4(h01, pack_f16(x[2 * tt] - f01.x, x[2 * tt + 1] - f01.y), h89,
+                                                pack_f16(x[2 * tt + 8] - f89.x, x[2 * tt + 9] - f89.y));
+      }
+    }
+    if (rep == 1 && NG <= 4) break;
+    bp += __shfl_xor_sync(0xffffffffu, bp, 1);
+    bp += __shfl_xor_sync(0xffffffffu, bp, 2);
+    bp += __shfl_xor_sync(0xffffffffu, bp, 4);
+    if (kk == 0 && hh < NG) reinterpret_cast<float*>(ws + mp.bias_off)[hh] = bp;
+  }
+  const __half* vsz = reinterpret_cast<const __half*>(stage + mp.vsz_soff);
+  uint4* vp = reinterpret_cast<uint4*>(ws + mp.vpair_off);
+  const int nvp = (G / 16) * 4 * NGRP;
+  for (int e = lane; e < nvp; e += 32) {
+    const int gg = e % NGRP, tq = (e / NGRP) & 3, kst = e / (NGRP * 4);
+    const int tile = kst / S::KSTEPS, ks2 = kst % S::KSTEPS;
+    const int tb = tile * S::TT;
+    const int tx0 = tb + tile_token<KB>(2 * ks2, 2 * tq), tx1 = tb + tile_token<KB>(2 * ks2, 2 * tq + 1);
+    const int ty0 = tb + tile_token<KB>(2 * ks2 + 1, 2 * tq), ty1 = tb + tile_token<KB>(2 * ks2 + 1, 2 * tq + 1);
+    const uint32_t ax = *reinterpret_cast<const uint32_t*>(vsz + (tx0 * NGRP + gg) * 2);
+    const uint32_t bx = *reinterpret_cast<const uint32_t*>(vsz + (tx1 * NGRP + gg) * 2);
+    const uint32_t ay = *reinterpret_cast<const uint32_t*>(vsz + (ty0 * NGRP + gg) * 2);
+    const uint32_t by = *reinterpret_cast<const uint32_t*>(vsz + (ty1 * NGRP + gg) * 2);
+    // (s, z) halves of two tokens -> (s0, s1) and (z0, z1)
+    vp[e] = make_uint4(__byte_perm(ax, bx, 0x5410), __byte_perm(ay, by, 0x5410), __byte_perm(ax, bx, 0x7632),
+                       __byte_perm(ay, by, 0x7632));
+  }
+  __syncwarp();
+}
+
+template <int KB, int VB, int NGRP>
 __global__ void __launch_bounds__(kThreads) decode_mma_kernel(DecodeParams p, MmaPlan mp) {
-  using S = Shape<KB, VB, TT, NGRP>;
+  using S = Shape<KB, VB, NGRP>;
   constexpr int D = S::D;
   extern __shared__ __align__(128) uint8_t smem[];
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int c = blockIdx.x;
   const LayerView& L = p.L;
   const int NG = p.num_q_heads / L.num_kv_heads;
   const int G = L.group_k;
-  const int Q = L.lens[2 * b], n = L.lens[2 * b + 1];
-  const int nblk = Q / G;
-  const int bps = p.blocks_per_split;
-  const int nsplit = (nblk + bps - 1) / bps;
-  if (s > nsplit) return;
-  if (s == 0) {
-    residual_partial(p, b, h, NG, Q, n, smem);
-    return;
-  }
+  const int T = p.total_blocks;
+  const int rs = cta_first_block(T, p.num_ctas, c), re = cta_first_block(T, p.num_ctas, c + 1);
+  const int nb = re - rs;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j0 = (s - 1) * bps;
-  const int nb = min(s * bps, nblk) - j0;
   const int NS = mp.nstages;
+  const int stage_bytes = mp.stage_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + mp.bar_off);
   uint64_t* empty = full + NS;
   if (threadIdx.x == 0) {
@@ -253,21 +357,12 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(DecodeParams p, Mm
     fence_mbar_init();
   }
   __syncthreads();
-
-  const int g = lane >> 2, t = lane & 3;
-  float lsum = 0.f, m_run = (g < NG) ? -INFINITY : 0.f;
-  float zacc[NGRP];
-#pragma unroll
-  for (int gg = 0; gg < NGRP; ++gg) zacc[gg] = 0.f;
-  float O[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) O[i][0] = O[i][1] = O[i][2] = O[i][3] = 0.f;
   bool failed = false;
 
-  if (warp == kConsumerWarps) {
-    // ---------------- producer: one lane streams the split's block records
+  if (warp == kProdWarp) {
+    // ---------------- producer: one lane streams this CTA's block records
     if (lane == 0) {
-      const uint8_t* rec0 = record_ptr(L, b, h, j0);
+      UnitCursor u;
       int issued = 0;
       for (int i = 0; i < nb; ++i) {
         const int st = i % NS;
@@ -275,14 +370,10 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(DecodeParams p, Mm
           failed = true;
           break;
         }
-        const uint8_t* rec = rec0 + (int64_t)i * L.record_bytes;
-        uint8_t* dst = smem + (size_t)st * mp.stage_bytes;
+        const int k = rs + i;
+        u.advance(p, k);
         mbar_expect_tx(full + st, mp.tx_bytes);
-        bulk_g2s(dst, rec, mp.kc_bytes + D * 4, full + st);
-        for (int sg = 0; sg < mp.vseg_count; ++sg)
-          bulk_g2s(dst + mp.vc_soff + sg * (mp.vseg_bytes + 16), rec + L.vc_off + sg * mp.vseg_bytes, mp.vseg_bytes,
-                   full + st);
-        bulk_g2s(dst + mp.vsz_soff, rec + L.vsz_off, mp.vsz_bytes, full + st);
+        bulk_g2s(smem + (size_t)st * stage_bytes, record_ptr(L, u.b, u.h, k - u.start), mp.tx_bytes, full + st);
         issued = i + 1;
       }
       // Let every copy land before the CTA may leave.
@@ -291,244 +382,221 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(DecodeParams p, Mm
     }
   } else {
     // ---------------- consumers
-    // This thread's query values: head g, channels 16kk + 2t + {0, 1, 8, 9}.
-    float qreg[8][4];
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int d = 16 * kk + 2 * t + (e & 1) + 8 * (e >> 1);
-        qreg[kk][e] = (g < NG) ? load_kv(p.q, ((int64_t)b * p.num_q_heads + h * NG + g) * D + d, L.kv_dtype) *
-                                     p.scale_log2
-                               : 0.f;
-      }
-    const int kc_row = G * KB / 8;  // key code bytes per channel
-    for (int i = warp; i < nb; i += kConsumerWarps) {
-      const int st = i % NS;
-      if (!mbar_wait(full + st, (i / NS) & 1)) {
-        failed = true;
-        break;
-      }
-      const uint8_t* stage = smem + (size_t)st * mp.stage_bytes;
-      const __half2* ksz = reinterpret_cast<const __half2*>(stage + mp.kc_bytes);
-      const __half2* vsz = reinterpret_cast<const __half2*>(stage + mp.vsz_soff);
-      const uint32_t kc_s = smem_u32(stage);
-      const uint32_t vc_s = smem_u32(stage + mp.vc_soff);
-
-      // A operand: (q*s) split into fp16 high (rows g) and low (rows g+8)
-      // parts; bias = sum_d q_d z_d of head g.
-      uint32_t A[8][4];
-      float bias = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        if (g < NG) {
-          const int c0 = 16 * kk + 2 * t;
-          const uint2 pa = *reinterpret_cast<const uint2*>(ksz + c0);      // (s,z) of c0, c0+1
-          const uint2 pb = *reinterpret_cast<const uint2*>(ksz + c0 + 8);  // (s,z) of c0+8, c0+9
-          const float2 a0 = unpack_f16(pa.x), a1 = unpack_f16(pa.y);
-          const float2 b0 = unpack_f16(pb.x), b1 = unpack_f16(pb.y);
-          const float x0 = qreg[kk][0] * a0.x, x1 = qreg[kk][1] * a1.x;
-          const float x8 = qreg[kk][2] * b0.x, x9 = qreg[kk][3] * b1.x;
-          bias += qreg[kk][0] * a0.y + qreg[kk][1] * a1.y + qreg[kk][2] * b0.y + qreg[kk][3] * b1.y;
-          const uint32_t h01 = pack_f16(x0, x1), h89 = pack_f16(x8, x9);
-          const float2 f01 = unpack_f16(h01), f89 = unpack_f16(h89);
-          A[kk][0] = h01;
-          A[kk][1] = pack_f16(x0 - f01.x, x1 - f01.y);
-          A[kk][2] = h89;
-          A[kk][3] = pack_f16(x8 - f89.x, x9 - f89.y);
-        } else {
-          A[kk][0] = A[kk][1] = A[kk][2] = A[kk][3] = 0u;
-        }
-      }
-      bias += __shfl_xor_sync(0xffffffffu, bias, 1);
-      bias += __shfl_xor_sync(0xffffffffu, bias, 2);
-
-      for (int tile = 0; tile < G / TT; ++tile) {
-        // ---------------- scores: S[n-tile][.] = A x codes
-        float Sacc[S::NT][4];
-#pragma unroll
-        for (int i2 = 0; i2 < S::NT; ++i2) Sacc[i2][0] = Sacc[i2][1] = Sacc[i2][2] = Sacc[i2][3] = 0.f;
-        const int mi = lane >> 3, rr = lane & 7;
-#pragma unroll
-        for (int kk = 0; kk < 8; kk += 2) {
-          const int ch = 16 * (kk + (mi >> 1)) + 8 * (mi & 1) + rr;
-#pragma unroll
-          for (int sg = 0; sg < S::SIG; ++sg) {
-            uint32_t r[4];
-            ldsm_x4_t(kc_s + ch * kc_row + (tile * S::SIG + sg) * 16, r[0], r[1], r[2], r[3]);
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-              const uint32_t x0 = r[2 * jj], x1 = r[2 * jj + 1];
-              const uint32_t x0h = x0 >> 8, x1h = x1 >> 8;
-#pragma unroll
-              for (int j = 0; j < S::CPT16; ++j) {
-                constexpr uint32_t cm = (1u << KB) - 1;
-                const int sh = (j * KB) % 8;
-                const uint32_t mask = (cm << sh) | (cm << (sh + 16));
-                const bool hib = j * KB >= 8;
-                const uint32_t b0 = codes_to_f16(hib ? x0h : x0, mask);
-                const uint32_t b1 = codes_to_f16(hib ? x1h : x1, mask);
-                mma16816(Sacc[sg * S::CPT16 + j], A[kk + jj], b0, b1);
-              }
-            }
-          }
-        }
-        // ---------------- online softmax over the tile (log2 units)
-        float sc[S::NT][2];
-        float mt = -INFINITY;
-#pragma unroll
-        for (int i2 = 0; i2 < S::NT; ++i2) {
-          const float ks = 1.0f / (float)(1 << (((i2 % S::CPT16) * KB) % 8));
-          sc[i2][0] = (Sacc[i2][0] + Sacc[i2][2]) * ks + bias;
-          sc[i2][1] = (Sacc[i2][1] + Sacc[i2][3]) * ks + bias;
-          mt = fmaxf(mt, fmaxf(sc[i2][0], sc[i2][1]));
-        }
-        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
-        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
-        float alpha = 1.f;
-        if (g < NG) {
-          const float mnew = fmaxf(m_run, mt);
-          alpha = ex2(m_run - mnew);
-          m_run = mnew;
-        }
-        float pr[S::NT][2];
-        float psum = 0.f;
-#pragma unroll
-        for (int i2 = 0; i2 < S::NT; ++i2) {
-          pr[i2][0] = (g < NG) ? ex2(sc[i2][0] - m_run) : 0.f;
-          pr[i2][1] = (g < NG) ? ex2(sc[i2][1] - m_run) : 0.f;
-          psum += pr[i2][0] + pr[i2][1];
-        }
-        lsum = lsum * alpha + psum;
-#pragma unroll
-        for (int gg = 0; gg < NGRP; ++gg) zacc[gg] *= alpha;
-        if (!__all_sync(0xffffffffu, alpha == 1.f)) {
-          const float a_lo = __shfl_sync(0xffffffffu, alpha, (2 * t) * 4);
-          const float a_hi = __shfl_sync(0xffffffffu, alpha, (2 * t + 1) * 4);
-#pragma unroll
-          for (int i2 = 0; i2 < 8; ++i2) {
-            O[i2][0] *= a_lo;
-            O[i2][1] *= a_hi;
-            O[i2][2] *= a_lo;
-            O[i2][3] *= a_hi;
-          }
-        }
-        // ---------------- values: O += codes x (p * s), zacc += p * z
-#pragma unroll
-        for (int ks2 = 0; ks2 < S::KSTEPS; ++ks2) {
-          const int X = 2 * ks2, Y = 2 * ks2 + 1;
-          const int tb = tile * TT;
-          const int tX0 = tb + tile_token<KB, TT>(X, 2 * t), tX1 = tb + tile_token<KB, TT>(X, 2 * t + 1);
-          const int tY0 = tb + tile_token<KB, TT>(Y, 2 * t), tY1 = tb + tile_token<KB, TT>(Y, 2 * t + 1);
-          uint32_t B0[NGRP], B1[NGRP];
-#pragma unroll
-          for (int gg = 0; gg < NGRP; ++gg) {
-            {
-              const float2 sx0 = __half22float2(vsz[tX0 * NGRP + gg]), sx1 = __half22float2(vsz[tX1 * NGRP + gg]);
-              const float2 sy0 = __half22float2(vsz[tY0 * NGRP + gg]), sy1 = __half22float2(vsz[tY1 * NGRP + gg]);
-              B0[gg] = pack_f16(pr[X][0] * sx0.x, pr[X][1] * sx1.x);
-              B1[gg] = pack_f16(pr[Y][0] * sy0.x, pr[Y][1] * sy1.x);
-              zacc[gg] += pr[X][0] * sx0.y + pr[X][1] * sx1.y + pr[Y][0] * sy0.y + pr[Y][1] * sy1.y;
-            }
-          }
-          const int tokl = tb + tile_token<KB, TT>((mi & 1) ? Y : X, rr);
-          const uint32_t vrow = vc_s + (tokl / S::CPT16) * (mp.vseg_bytes + 16) + (tokl % S::CPT16) * S::VRB;
-#pragma unroll
-          for (int c = 0; c < S::NCH; c += 2) {
-            uint32_t r[4];
-            ldsm_x4_t(vrow + 16 * (c + (mi >> 1)), r[0], r[1], r[2], r[3]);
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-              const uint32_t xv = r[2 * cc], yv = r[2 * cc + 1];
-              const uint32_t xh = xv >> 8, yh = yv >> 8;
-              const int gg = ((c + cc) * S::CH_SPAN) / S::GV;
-#pragma unroll
-              for (int P = 0; P < S::MT_PER_CH; ++P) {
-                constexpr uint32_t cm = (1u << VB) - 1;
-                const int p0 = 2 * P, p1 = 2 * P + 1;
-                const int sh0 = (p0 * VB) % 8, sh1 = (p1 * VB) % 8;
-                const bool h0 = p0 * VB >= 8, h1 = p1 * VB >= 8;
-                const uint32_t m0 = (cm << sh0) | (cm << (sh0 + 16)), m1 = (cm << sh1) | (cm << (sh1 + 16));
-                uint32_t a[4];
-                a[0] = codes_to_f16(h0 ? xh : xv, m0);
-                a[1] = codes_to_f16(h1 ? xh : xv, m1);
-                a[2] = codes_to_f16(h0 ? yh : yv, m0);
-                a[3] = codes_to_f16(h1 ? yh : yv, m1);
-                mma16816(O[(c + cc) * S::MT_PER_CH + P], a, B0[gg], B1[gg]);
-              }
-            }
-          }
-        }
-      }
+    uint8_t* ws = smem + mp.ws_soff + warp * mp.ws_bytes;
+    float* wq = reinterpret_cast<float*>(ws + mp.wq_off);
+    {  // rows of heads >= NG stay zero
+      uint4* af = reinterpret_cast<uint4*>(ws + mp.afrag_off);
+      for (int e = lane; e < 8 * 8 * 4; e += 32)
+        if (((e >> 2) & 7) >= NG) af[e] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    auto stage_q = [&](int b, int h) {  // the unit's scaled queries into wq
       __syncwarp();
-      if (lane == 0) mbar_arrive(empty + st);
+      for (int e = lane; e < NG * D; e += 32)
+        wq[e] = load_kv(p.q, ((int64_t)b * p.num_q_heads + h * NG) * D + e, L.kv_dtype) * p.scale_log2;
+      __syncwarp();
+    };
+    // residual units of this CTA first (the producer already streams)
+    for (int r = c; r < p.batch * L.num_kv_heads; r += p.num_ctas) {
+      stage_q(r / L.num_kv_heads, r % L.num_kv_heads);
+      residual_unit(p, r / L.num_kv_heads, r % L.num_kv_heads, NG, wq);
+    }
+
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t magic = 0x64006400u;
+    const uint32_t ones[4] = {0x3c003c00u, 0x3c003c00u, 0x3c003c00u, 0x3c003c00u};  // fp16 1.0
+    const int kc_row = G * KB / 8;  // key code bytes per channel
+    const int ncol = G / S::CPT16;  // value rows per key-column position
+    const int mi = lane >> 3, rr = lane & 7;
+    // ldmatrix rows of this lane: 8 consecutive rows, so the chunk swizzle of
+    // the record layout depends on the lane's row index only
+    const int swk = chunk_swizzle(rr, kc_row / 16);
+    const int swv = chunk_swizzle(rr, S::VRB / 16);
+    const uint4* afr = reinterpret_cast<const uint4*>(ws + mp.afrag_off);
+    const uint4* vpr = reinterpret_cast<const uint4*>(ws + mp.vpair_off);
+    const float* biasr = reinterpret_cast<const float*>(ws + mp.bias_off);
+    UnitCursor u;
+    int k = rs;
+    while (k < re && !failed) {
+      u.advance(p, k);
+      const int hi = min(u.end, re);
+      stage_q(u.b, u.h);
+      float lsum = 0.f, m_run = (g < NG) ? -INFINITY : 0.f;
+      float O[8][4], Z[NGRP][4];
+#pragma unroll
+      for (int i2 = 0; i2 < 8; ++i2) O[i2][0] = O[i2][1] = O[i2][2] = O[i2][3] = 0.f;
+#pragma unroll
+      for (int gg = 0; gg < NGRP; ++gg) Z[gg][0] = Z[gg][1] = Z[gg][2] = Z[gg][3] = 0.f;
+      // this warp's blocks of the unit: i = kb - rs with i % kNC == warp
+      const int first = k + ((warp - (k - rs)) % kNC + kNC) % kNC;
+      for (int kb = first; kb < hi; kb += kNC) {
+        const int i = kb - rs;
+        const int st = i % NS;
+        if (!mbar_wait(full + st, (i / NS) & 1)) {
+          failed = true;
+          break;
+        }
+        const uint8_t* stage = smem + (size_t)st * stage_bytes;
+        prep_block<KB, VB, NGRP>(stage, mp, ws, NG, G, lane);
+        const float bias = (g < NG) ? biasr[g] : 0.f;
+        const uint32_t kc_s = smem_u32(stage);
+        const uint32_t vc_s = smem_u32(stage + mp.vc_soff);
+
+        for (int tile = 0; tile < G / S::TT; ++tile) {
+          // ---------------- scores: S[n-tile][.] = A x codes
+          float Sacc[S::NT][4];
+#pragma unroll
+          for (int i2 = 0; i2 < S::NT; ++i2) Sacc[i2][0] = Sacc[i2][1] = Sacc[i2][2] = Sacc[i2][3] = 0.f;
+#pragma unroll
+          for (int kk = 0; kk < 8; kk += 2) {
+            const int ch = 16 * (kk + (mi >> 1)) + 8 * (mi & 1) + rr;
+#pragma unroll
+            for (int sg = 0; sg < S::SIG; ++sg) {
+              uint32_t r[4];
+              ldsm_x4_t(kc_s + ch * kc_row + (((tile * S::SIG + sg) ^ swk) << 4), r[0], r[1], r[2], r[3]);
+#pragma unroll
+              for (int jj = 0; jj < 2; ++jj) {
+                const uint4 av = afr[((kk + jj) * 8 + g) * 4 + t];
+                const uint32_t A[4] = {av.x, av.y, av.z, av.w};
+                const uint32_t x0 = r[2 * jj], x1 = r[2 * jj + 1];
+                const uint32_t x0h = x0 >> 8, x1h = x1 >> 8;
+#pragma unroll
+                for (int j = 0; j < S::CPT16; ++j) {
+                  constexpr uint32_t cm = (1u << KB) - 1;
+                  const int sh = (j * KB) % 8;
+                  const uint32_t mask = (cm << sh) | (cm << (sh + 16));
+                  const bool hib = j * KB >= 8;
+                  const uint32_t b0 = codes_to_f16(hib ? x0h : x0, mask, magic);
+                  const uint32_t b1 = codes_to_f16(hib ? x1h : x1, mask, magic);
+                  mma16816(Sacc[sg * S::CPT16 + j], A, b0, b1);
+                }
+              }
+            }
+          }
+          // ---------------- online softmax over the tile (log2 units)
+          float pr[S::NT][2];
+          float mt = -INFINITY;
+#pragma unroll
+          for (int i2 = 0; i2 < S::NT; ++i2) {
+            const float ks = 1.0f / (float)(1 << (((i2 % S::CPT16) * KB) % 8));
+            pr[i2][0] = (Sacc[i2][0] + Sacc[i2][2]) * ks + bias;
+            pr[i2][1] = (Sacc[i2][1] + Sacc[i2][3]) * ks + bias;
+            mt = fmaxf(mt, fmaxf(pr[i2][0], pr[i2][1]));
+          }
+          mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+          mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+          float alpha = 1.f;
+          if (g < NG) {
+            const float mnew = fmaxf(m_run, mt);
+            alpha = ex2(m_run - mnew);
+            m_run = mnew;
+          }
+          float psum = 0.f;
+#pragma unroll
+          for (int i2 = 0; i2 < S::NT; ++i2) {
+            pr[i2][0] = (g < NG) ? ex2(pr[i2][0] - m_run) : 0.f;
+            pr[i2][1] = (g < NG) ? ex2(pr[i2][1] - m_run) : 0.f;
+            psum += pr[i2][0] + pr[i2][1];
+          }
+          lsum = lsum * alpha + psum;
+          if (!__all_sync(0xffffffffu, alpha == 1.f)) {
+            const float a_lo = __shfl_sync(0xffffffffu, alpha, (2 * t) * 4);
+            const float a_hi = __shfl_sync(0xffffffffu, alpha, (2 * t + 1) * 4);
+#pragma unroll
+            for (int gg = 0; gg < NGRP; ++gg) {
+              Z[gg][0] *= a_lo;
+              Z[gg][1] *= a_hi;
+              Z[gg][2] *= a_lo;
+              Z[gg][3] *= a_hi;
+            }
+#pragma unroll
+            for (int i2 = 0; i2 < 8; ++i2) {
+              O[i2][0] *= a_lo;
+              O[i2][1] *= a_hi;
+              O[i2][2] *= a_lo;
+              O[i2][3] *= a_hi;
+            }
+          }
+          // ---------------- values: O += codes x (p * s), Z += ones x (p * z)
+#pragma unroll
+          for (int ks2 = 0; ks2 < S::KSTEPS; ++ks2) {
+            const int X = 2 * ks2, Y = 2 * ks2 + 1;
+            const int tb = tile * S::TT;
+            const uint32_t pX = pack_f16(pr[X][0], pr[X][1]), pY = pack_f16(pr[Y][0], pr[Y][1]);
+            uint32_t B0[NGRP], B1[NGRP];
+#pragma unroll
+            for (int gg = 0; gg < NGRP; ++gg) {
+              const uint4 v4 = vpr[((tile * S::KSTEPS + ks2) * 4 + t) * NGRP + gg];
+              B0[gg] = hmul2(pX, v4.x);
+              B1[gg] = hmul2(pY, v4.y);
+              mma16816(Z[gg], ones, hmul2(pX, v4.z), hmul2(pY, v4.w));
+            }
+            const int tokl = tb + tile_token<KB>((mi & 1) ? Y : X, rr);
+            const uint32_t vrow = vc_s + ((tokl % S::CPT16) * ncol + tokl / S::CPT16) * S::VRB;
+#pragma unroll
+            for (int cc0 = 0; cc0 < S::NCH; cc0 += 2) {
+              uint32_t r[4];
+              ldsm_x4_t(vrow + (((cc0 + (mi >> 1)) ^ swv) << 4), r[0], r[1], r[2], r[3]);
+#pragma unroll
+              for (int cc = 0; cc < 2; ++cc) {
+                const uint32_t xv = r[2 * cc], yv = r[2 * cc + 1];
+                const uint32_t xh = xv >> 8, yh = yv >> 8;
+                const int gg = ((cc0 + cc) * S::CH_SPAN) / S::GV;
+#pragma unroll
+                for (int P = 0; P < S::MT_PER_CH; ++P) {
+                  constexpr uint32_t cm = (1u << VB) - 1;
+                  const int p0 = 2 * P, p1 = 2 * P + 1;
+                  const int sh0 = (p0 * VB) % 8, sh1 = (p1 * VB) % 8;
+                  const bool h0 = p0 * VB >= 8, h1 = p1 * VB >= 8;
+                  const uint32_t m0 = (cm << sh0) | (cm << (sh0 + 16)), m1 = (cm << sh1) | (cm << (sh1 + 16));
+                  uint32_t a[4];
+                  a[0] = codes_to_f16(h0 ? xh : xv, m0, magic);
+                  a[1] = codes_to_f16(h1 ? xh : xv, m1, magic);
+                  a[2] = codes_to_f16(h0 ? yh : yv, m0, magic);
+                  a[3] = codes_to_f16(h1 ? yh : yv, m1, magic);
+                  mma16816(O[(cc0 + cc) * S::MT_PER_CH + P], a, B0[gg], B1[gg]);
+                }
+              }
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty + st);
+      }
+      // ---------------- this warp's partial for the unit
+      lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+      lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+      const int slot = kResidualSlots + 4 * (c - cta_of_block(T, p.num_ctas, u.start)) + warp;
+      const int h_lo = 2 * t, h_hi = 2 * t + 1;
+      const int64_t base_lo = ((int64_t)u.b * p.num_q_heads + u.h * NG + h_lo) * p.slots + slot;
+      const int64_t base_hi = ((int64_t)u.b * p.num_q_heads + u.h * NG + h_hi) * p.slots + slot;
+#pragma unroll
+      for (int mt2 = 0; mt2 < 8; ++mt2) {
+        const int cch = mt2 / S::MT_PER_CH, P = mt2 % S::MT_PER_CH;
+        const int gg = (cch * S::CH_SPAN) / S::GV;
+        const int p0 = 2 * P, p1 = 2 * P + 1;
+        const float rs0 = 1.0f / (float)(1 << ((p0 * VB) % 8)), rs1 = 1.0f / (float)(1 << ((p1 * VB) % 8));
+        const int ch0 = cch * S::CH_SPAN + g * S::VCPC + p0;
+        if (h_lo < NG) {
+          p.ws_o[base_lo * D + ch0] = O[mt2][0] * rs0 + Z[gg][0];
+          p.ws_o[base_lo * D + ch0 + 1] = O[mt2][2] * rs1 + Z[gg][0];
+        }
+        if (h_hi < NG) {
+          p.ws_o[base_hi * D + ch0] = O[mt2][1] * rs0 + Z[gg][1];
+          p.ws_o[base_hi * D + ch0 + 1] = O[mt2][3] * rs1 + Z[gg][1];
+        }
+      }
+      if (t == 0 && g < NG)
+        p.ws_ml[((int64_t)u.b * p.num_q_heads + u.h * NG + g) * p.slots + slot] = make_float2(m_run, lsum);
+      k = hi;
     }
   }
   if (failed) atomicOr(p.err, 1);
   __syncthreads();  // every stage is consumed and every copy has landed
-
-  // ---------------- merge the consumer warps' states through shared memory
-  float* so = reinterpret_cast<float*>(smem);  // [4][8][D]
-  float* sm = so + 4 * 8 * D;                  // [4][8]
-  float* sl = sm + 32;                         // [4][8]
-  if (warp < kConsumerWarps) {
-    lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
-    lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-#pragma unroll
-    for (int gg = 0; gg < NGRP; ++gg) {
-      zacc[gg] += __shfl_xor_sync(0xffffffffu, zacc[gg], 1);
-      zacc[gg] += __shfl_xor_sync(0xffffffffu, zacc[gg], 2);
-    }
-    const int h_lo = 2 * t, h_hi = 2 * t + 1;
-#pragma unroll
-    for (int mt2 = 0; mt2 < 8; ++mt2) {
-      const int c = mt2 / S::MT_PER_CH, P = mt2 % S::MT_PER_CH;
-      const int gg = (c * S::CH_SPAN) / S::GV;
-      const float z_lo = __shfl_sync(0xffffffffu, zacc[gg], h_lo * 4);
-      const float z_hi = __shfl_sync(0xffffffffu, zacc[gg], h_hi * 4);
-      const int p0 = 2 * P, p1 = 2 * P + 1;
-      const float rs0 = 1.0f / (float)(1 << ((p0 * VB) % 8)), rs1 = 1.0f / (float)(1 << ((p1 * VB) % 8));
-      const int ch0 = c * S::CH_SPAN + g * S::VCPC + p0;
-      if (h_lo < NG) {
-        so[(warp * 8 + h_lo) * D + ch0] = O[mt2][0] * rs0 + z_lo;
-        so[(warp * 8 + h_lo) * D + ch0 + 1] = O[mt2][2] * rs1 + z_lo;
-      }
-      if (h_hi < NG) {
-        so[(warp * 8 + h_hi) * D + ch0] = O[mt2][1] * rs0 + z_hi;
-        so[(warp * 8 + h_hi) * D + ch0 + 1] = O[mt2][3] * rs1 + z_hi;
-      }
-    }
-    if (t == 0 && g < NG) {
-      sm[warp * 8 + g] = m_run;
-      sl[warp * 8 + g] = lsum;
-    }
-  }
-  __syncthreads();
-  const int d = threadIdx.x;
-  if (d < D) {
-    for (int hh = 0; hh < NG; ++hh) {
-      float M = -INFINITY;
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm[w * 8 + hh]);
-      float acc = 0.f, ls = 0.f;
-      if (M != -INFINITY) {
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const float mw = sm[w * 8 + hh];
-          if (mw == -INFINITY) continue;
-          const float f = ex2(mw - M);
-          acc += so[(w * 8 + hh) * D + d] * f;
-          ls += sl[w * 8 + hh] * f;
-        }
-      }
-      const int64_t slot = ((int64_t)b * p.num_q_heads + h * NG + hh) * p.slots + s;
-      p.ws_o[slot * D + d] = acc;
-      if (d == 0) p.ws_ml[slot] = make_float2(M, ls);
-    }
-  }
 }
 
 template <int KB, int VB, int NGRP>
 cudaError_t launch_mma_inst(const DecodeParams& p, const MmaPlan& mp, int max_splits, cudaStream_t stream) {
-  auto kern = decode_mma_kernel<KB, VB, 64, NGRP>;
+  auto kern = decode_mma_kernel<KB, VB, NGRP>;
   static uint64_t attr_mask = 0;  // shared-memory opt-in per device
   static int attr_bytes[64] = {0};
   int dev = 0;
@@ -542,8 +610,8 @@ cudaError_t launch_mma_inst(const DecodeParams& p, const MmaPlan& mp, int max_sp
       attr_bytes[dev] = mp.smem_bytes;
     }
   }
-  dim3 grid(max_splits + 1, p.L.num_kv_heads, p.batch);
-  kern<<<grid, kThreads, mp.smem_bytes, stream>>>(p, mp);
+  (void)max_splits;
+  kern<<<p.num_ctas, kThreads, mp.smem_bytes, stream>>>(p, mp);
   return cudaGetLastError();
 }
 
@@ -564,23 +632,30 @@ bool mma_supported(const LayerView& L) {
 
 MmaPlan make_mma_plan(const LayerView& L) {
   MmaPlan mp;
-  const int G = L.group_k, D = L.head_dim, kb = L.k_bits, vb = L.v_bits;
-  mp.kc_bytes = G * kb / 8 * D;
-  const int cpt16 = 16 / kb;
-  mp.vseg_bytes = cpt16 * (D * vb / 8);
-  mp.vseg_count = G / cpt16;
-  mp.vsz_bytes = G * (D / L.group_v) * 4;
-  mp.vc_soff = mp.kc_bytes + D * 4;
-  mp.vsz_soff = mp.vc_soff + mp.vseg_count * (mp.vseg_bytes + 16);
-  mp.stage_bytes = mp.vsz_soff + mp.vsz_bytes;
-  mp.tx_bytes = mp.kc_bytes + D * 4 + mp.vseg_count * mp.vseg_bytes + mp.vsz_bytes;
-  const int merge_bytes = (8 * D + 4 * 8 * D + 64) * 4;  // residual split / final merge
-  int ns = (72 * 1024) / mp.stage_bytes;
-  if (ns < 4) ns = 4;
+  const int G = L.group_k, D = L.head_dim;
+  const int ngrp = D / L.group_v;
+  mp.tx_bytes = L.vsz_off + G * ngrp * 4;          // kc | ksz | vc | vsz, one copy
+  mp.kc_bytes = L.ksz_off;
+  mp.vc_soff = L.vc_off;
+  mp.vsz_soff = L.vsz_off;
+  mp.stage_bytes = (int32_t)round_up(mp.tx_bytes, 128);
+  // per-consumer-warp scratch
+  mp.afrag_off = 0;
+  mp.bias_off = 8 * 8 * 4 * 16;
+  mp.vpair_off = mp.bias_off + 64;
+  mp.wq_off = (int32_t)round_up(mp.vpair_off + (G / 16) * 4 * ngrp * 16, 16);
+  mp.ws_bytes = (int32_t)round_up(mp.wq_off + 8 * D * 4, 128);
+  // The stage count is a multiple of the consumer-warp count, so stage st is
+  // always consumed by warp st % kNC: every waiter of a stage's barriers then
+  // waits for its phases in order and never one phase too early (a parity
+  // wait two phases ahead would alias a completed phase).
+  int ns = (80 * 1024) / mp.stage_bytes;
+  ns -= ns % kNC;
+  if (ns < kNC) ns = kNC;
   if (ns > 16) ns = 16;
-  while (ns * mp.stage_bytes < merge_bytes) ++ns;
   mp.nstages = ns;
-  mp.bar_off = ns * mp.stage_bytes;
+  mp.ws_soff = ns * mp.stage_bytes;
+  mp.bar_off = mp.ws_soff + kNC * mp.ws_bytes;
   mp.smem_bytes = mp.bar_off + 2 * ns * 8;
   return mp;
 }
@@ -599,7 +674,7 @@ int mma_ctas_per_sm(const LayerView& L, const MmaPlan& mp) {
   const void* fn = nullptr;
   const int kb = L.k_bits, vb = L.v_bits, ng = kHeadDim / L.group_v;
 #define KVQ_FN(K, V, N) \
-  if (kb == K && vb == V && ng == N) fn = (const void*)decode_mma_kernel<K, V, 64, N>;
+  if (kb == K && vb == V && ng == N) fn = (const void*)decode_mma_kernel<K, V, N>;
   KVQ_MMA_INSTANCES(KVQ_FN)
 #undef KVQ_FN
   if (!fn) return 1;

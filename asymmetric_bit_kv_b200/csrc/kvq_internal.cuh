@@ -34,6 +34,44 @@ __host__ __device__ inline int64_t ksz_bytes(int D) { return (int64_t)D * 4; }
 __host__ __device__ inline int64_t vc_bytes(int G, int D, int vb) { return (int64_t)G * (D * vb / 32) * 4; }
 __host__ __device__ inline int64_t vsz_bytes(int G, int D, int gv) { return (int64_t)G * (D / gv) * 4; }
 
+// ---------------------------------------------------------------------------
+// Word placement inside a block record. Both code arrays are stored so that a
+// straight copy of the record into shared memory can be read with ldmatrix
+// without bank conflicts:
+//  * a row of n 16-byte chunks stores chunk c at position c ^ swizzle(row, n),
+//    where swizzle spreads 8 consecutive rows over 8 distinct 16-byte bank
+//    slots;
+//  * value rows are stored in "column-major token order": token t of a block
+//    sits in row (t % c) * (G / c) + t / c with c = 16 / k_bits, the number of
+//    tokens one 16-bit half of a key word holds (the tokens the decode kernel
+//    reads together for one n-tile are then 8 consecutive rows).
+// ---------------------------------------------------------------------------
+__host__ __device__ inline int chunk_swizzle(int row, int nchunks) {
+  if (nchunks <= 1) return 0;
+  if (nchunks >= 8) return row & 7;
+  return (row / (8 / nchunks)) % nchunks;
+}
+// Index (in 32-bit words) of word w of channel d inside the key code array
+// of a record; W = G * k_bits / 32 words per channel.
+__host__ __device__ inline int kc_word_index(int d, int w, int W) {
+  if (W < 4) return d * W + w;
+  const int c = w >> 2;
+  return d * W + ((c ^ chunk_swizzle(d, W / 4)) << 2) + (w & 3);
+}
+// Row of token t (0 <= t < G) in the value code array of a record.
+__host__ __device__ inline int vc_row(int t, int G, int kb) {
+  const int c = 16 / kb;
+  return (t % c) * (G / c) + t / c;
+}
+// Index (in words) of word w of token t inside the value code array; VW =
+// D * v_bits / 32 words per token.
+__host__ __device__ inline int vc_word_index(int t, int w, int G, int kb, int VW) {
+  const int r = vc_row(t, G, kb);
+  if (VW < 4) return r * VW + w;
+  const int c = w >> 2;
+  return r * VW + ((c ^ chunk_swizzle(r, VW / 4)) << 2) + (w & 3);
+}
+
 __device__ __forceinline__ uint8_t* record_ptr(const LayerView& L, int b, int h, int64_t j) {
   return L.blocks + (((int64_t)b * L.num_kv_heads + h) * L.max_blocks + j) * L.record_bytes;
 }

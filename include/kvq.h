@@ -92,15 +92,21 @@ typedef struct kvq_cache kvq_cache;
  * [j*G, (j+1)*G) of that sequence) the record starts at
  *   blocks + ((b * num_kv_heads + h) * max_blocks + j) * record_bytes
  * and holds, at the given byte offsets:
- *   kc  uint32 [D][G*k_bits/32]: word w of channel d packs the codes of
- *       tokens w*(32/k_bits) + i, i = 0.., code i at bits [i*k_bits, ...)
- *       (per-channel keys, packed along the token axis; each channel's
- *       words are contiguous);
+ *   kc  uint32 [D][W], W = G*k_bits/32: channel d's row holds W words; word
+ *       w packs the codes of tokens w*(32/k_bits) + i, i = 0.., code i at
+ *       bits [i*k_bits, ...) (per-channel keys packed along the token axis);
  *   ksz half2 [D]: (scale d, zero point m) of each channel's key group;
- *   vc  uint32 [G][D*v_bits/32]: word w of token t packs the codes of
- *       channels w*(32/v_bits) + i, code i at bits [i*v_bits, ...)
- *       (per-token values, packed along head_dim);
+ *   vc  uint32 [G][V], V = D*v_bits/32: one row of V words per token; word w
+ *       packs the codes of channels w*(32/v_bits) + i, code i at bits
+ *       [i*v_bits, ...) (per-token values packed along head_dim);
  *   vsz half2 [G][D/group_v]: (scale, zero point) of each value group.
+ * Placement inside kc and vc (so that one copy of a record is readable with
+ * ldmatrix without shared-memory bank conflicts): in a row of n >= 2
+ * 16-byte chunks (4 words each), chunk c of row r is stored at chunk
+ * position c ^ s(r, n), with s(r, n) = r & 7 for n >= 8 and
+ * (r / (8/n)) % n otherwise; rows of fewer than 4 words are not permuted.
+ * Value rows are stored in token order t -> (t % c) * (G/c) + t / c, with
+ * c = 16/k_bits. (kvq_internal.cuh: kc_word_index, vc_word_index.)
  * Ring: [max_batch][num_kv_heads][R][D] in kv_dtype; token i of a sequence
  * (quantized <= i < quantized + residual) sits in slot i % R.              */
 typedef struct kvq_layout {

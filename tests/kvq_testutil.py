@@ -33,6 +33,29 @@ def ulp(x: np.ndarray, dtype) -> np.ndarray:
     return 2.0 ** (e - mant)
 
 
+def chunk_swizzle(row: int, n: int) -> int:
+    """Chunk-position permutation of the record layout documented in kvq.h."""
+    if n <= 1:
+        return 0
+    if n >= 8:
+        return row & 7
+    return (row // (8 // n)) % n
+
+
+def kc_word_index(d: int, w: int, W: int) -> int:
+    if W < 4:
+        return d * W + w
+    return d * W + (((w >> 2) ^ chunk_swizzle(d, W // 4)) << 2) + (w & 3)
+
+
+def vc_word_index(t: int, w: int, G: int, kb: int, VW: int) -> int:
+    c = 16 // kb
+    r = (t % c) * (G // c) + t // c
+    if VW < 4:
+        return r * VW + w
+    return r * VW + (((w >> 2) ^ chunk_swizzle(r, VW // 4)) << 2) + (w & 3)
+
+
 class Twin:
     """A device cache and one oracle SequenceCache per (layer, sequence)."""
 
@@ -73,7 +96,8 @@ class Twin:
                 assert self.gpu.lengths(layer, b) == (o.quantized_tokens, o.residual_tokens), (layer, b)
 
     def read_records(self, layer: int, b: int, h: int, nblk: int):
-        """Device block records [0, nblk) of (sequence b, KV head h), split into parts."""
+        """Device block records [0, nblk) of (sequence b, KV head h), split into
+        parts, with the documented word placement undone (natural order)."""
         lay = self.gpu.layout(layer)
         cfg = self.cfg
         G, D, Gv = cfg.group_k, cfg.head_dim, cfg.group_v
@@ -86,10 +110,14 @@ class Twin:
 
         kcw = G * kb // 32
         vcw = D * vb // 32
+        kc = part(lay.kc_offset, kcw * D * 4, np.uint32, (D * kcw,))
+        vc = part(lay.vc_offset, G * vcw * 4, np.uint32, (G * vcw,))
+        kidx = np.array([[kc_word_index(d, w, kcw) for w in range(kcw)] for d in range(D)])
+        vidx = np.array([[vc_word_index(t, w, G, kb, vcw) for w in range(vcw)] for t in range(G)])
         return {
-            "kc": part(lay.kc_offset, kcw * D * 4, np.uint32, (D, kcw)),
+            "kc": kc[:, kidx],
             "ksz": part(lay.ksz_offset, D * 4, np.float16, (D, 2)),
-            "vc": part(lay.vc_offset, G * vcw * 4, np.uint32, (G, vcw)),
+            "vc": vc[:, vidx],
             "vsz": part(lay.vsz_offset, G * (D // Gv) * 4, np.float16, (G, D // Gv, 2)),
         }
 
