@@ -13,9 +13,9 @@ namespace kvq {
 //  * persistent mode (tensor-core kernel): the quantized blocks of all
 //    (sequence, KV head) units, concatenated in (sequence, head, block) order,
 //    are cut into num_ctas contiguous ranges (CTA c takes
-//    [c*T/num_ctas, (c+1)*T/num_ctas)); slots 0-3 hold the residual ring (one
-//    per consumer warp), slot 4 + 4*(c - c0) + w the blocks that warp w of
-//    CTA c processed for the unit, c0 being the unit's first CTA.
+//    [c*T/num_ctas, (c+1)*T/num_ctas)); slot 0 holds the residual ring,
+//    slot 1 + 4*(c - c0) + w the blocks that warp w of CTA c processed for
+//    the unit, c0 being the unit's first CTA.
 struct DecodeParams {
   LayerView L;
   const void* q;        // [batch][Hq][D], kv dtype
@@ -36,7 +36,7 @@ struct DecodeParams {
   int32_t seq_start[KVQ_MAX_BATCH];  // first global block of sequence b: sum_{b'<b} nblk*Hkv
 };
 
-constexpr int kResidualSlots = 4;  // persistent mode: one residual partial per consumer warp
+constexpr int kResidualSlots = 1;  // persistent mode: the residual ring's partial
 
 // Persistent mode: first global block of CTA c, and the CTA holding block k.
 __host__ __device__ inline int32_t cta_first_block(int64_t T, int32_t nctas, int32_t c) {

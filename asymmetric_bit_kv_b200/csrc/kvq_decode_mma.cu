@@ -126,88 +126,150 @@ __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
 }
 
 // ------------------------------------------------------- residual ring split
-// Consumer warp w takes every kNC-th ring token of unit (b, h) with CUDA
-// cores and writes its own partial (slot w). Lane l owns channels 4l..4l+3;
-// the K/V rows of kRB tokens are loaded (8-byte loads) before they are used.
-constexpr int kRB = 4;
-
-__device__ __forceinline__ void load4(const void* base, int64_t elem, int dtype, float (&x)[4]) {
-  const uint2 v = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(base) + elem);
-  const uint32_t w[2] = {v.x, v.y};
+// Exact attention over the ring tokens [Q, Q+n) of unit (b, h) by the 128
+// consumer threads (named barrier 1), in chunks of up to 128 tokens staged
+// in shared memory with cp.async (16-byte rows chunks stored at position
+// j ^ (row & 15), so per-row reads are bank-conflict-free):
+//   q.k: thread tau owns token tau of the chunk; p.v: thread d owns channel d.
+// Writes one partial (slot 0). Scratch (bytes): tile [128][256], q [8][128]
+// fp32, p [8][128] fp32, red [4][8][2] fp32.
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kNC * 32) : "memory"); }
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void bf16x8_or_f16x8(const uint4& v, int dtype, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
+  for (int e = 0; e < 4; ++e) {
     if (dtype == KVQ_BF16) {
-      x[2 * i] = __uint_as_float(w[i] << 16);
-      x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+      f[2 * e] = __uint_as_float(w[e] << 16);
+      f[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
     } else {
-      const float2 f = unpack_f16(w[i]);
-      x[2 * i] = f.x;
-      x[2 * i + 1] = f.y;
+      const float2 x = unpack_f16(w[e]);
+      f[2 * e] = x.x;
+      f[2 * e + 1] = x.y;
     }
   }
 }
+constexpr int kResTile = 128;                       // ring tokens per chunk
+constexpr int kResScratch = kResTile * 256 + 2 * 8 * 128 * 4 + 4 * 8 * 2 * 4;
 
-__device__ void residual_unit(const DecodeParams& p, int b, int h, int NG, const float* wq) {
+__device__ void residual_unit(const DecodeParams& p, int b, int h, int NG, uint8_t* scratch) {
   const LayerView& L = p.L;
   constexpr int D = kHeadDim;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint4* tile = reinterpret_cast<uint4*>(scratch);                     // [128 rows][16 chunks]
+  float* sq = reinterpret_cast<float*>(scratch + kResTile * 256);      // [8][D]
+  float* sp = sq + 8 * D;                                              // [8][kResTile]
+  float* red = sp + 8 * kResTile;                                      // [4][8][2]
   const int Q = L.lens[2 * b], n = L.lens[2 * b + 1];
-  float m[8], l[8], o[8][4], qv[8][4];
+  const int dt = L.kv_dtype;
+  const int64_t ring = ((int64_t)b * L.num_kv_heads + h) * L.residual;
+  consumers_sync();  // scratch is free
+  for (int e = tid; e < NG * D; e += kNC * 32)
+    sq[e] = load_kv(p.q, ((int64_t)b * p.num_q_heads + h * NG) * D + e, dt) * p.scale_log2;
+  float m[8], l[8], o[8];  // per head; o for channel d = tid
 #pragma unroll
   for (int hh = 0; hh < 8; ++hh) {
     m[hh] = -INFINITY;
     l[hh] = 0.f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      o[hh][c] = 0.f;
-      qv[hh][c] = (hh < NG) ? wq[hh * D + 4 * lane + c] : 0.f;
-    }
+    o[hh] = 0.f;
   }
-  const int64_t base = ((int64_t)b * L.num_kv_heads + h) * L.residual;
-  for (int i0 = Q + warp; i0 < Q + n; i0 += kNC * kRB) {
-    float kv[kRB][4], vv[kRB][4];
+  for (int c0 = 0; c0 < n; c0 += kResTile) {
+    const int cnt = min(kResTile, n - c0);
+    // ---- keys of the chunk
+    if (tid < cnt) {
+      const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(L.ring_k) +
+                                                        (ring + (Q + c0 + tid) % L.residual) * D);
 #pragma unroll
-    for (int r = 0; r < kRB; ++r) {
-      const int i = i0 + r * kNC;
-      if (i < Q + n) {
-        const int64_t row = (base + i % L.residual) * D + 4 * lane;
-        load4(L.ring_k, row, L.kv_dtype, kv[r]);
-        load4(L.ring_v, row, L.kv_dtype, vv[r]);
-      }
+      for (int j = 0; j < 16; ++j) cp_async16(tile + tid * 16 + (j ^ (tid & 15)), src + j);
     }
+    cp_async_wait_all();
+    consumers_sync();
+    float sc[8];
 #pragma unroll
-    for (int r = 0; r < kRB; ++r) {
-      if (i0 + r * kNC < Q + n) {
-        float sc[8];
-#pragma unroll
-        for (int hh = 0; hh < 8; ++hh)
-          sc[hh] = qv[hh][0] * kv[r][0] + qv[hh][1] * kv[r][1] + qv[hh][2] * kv[r][2] + qv[hh][3] * kv[r][3];
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1)
-#pragma unroll
-          for (int hh = 0; hh < 8; ++hh)
-            if (hh < NG) sc[hh] += __shfl_xor_sync(0xffffffffu, sc[hh], off);
+    for (int hh = 0; hh < 8; ++hh) sc[hh] = 0.f;
+    if (tid < cnt) {
+#pragma unroll 4
+      for (int j = 0; j < 16; ++j) {
+        float kf[8];
+        bf16x8_or_f16x8(tile[tid * 16 + (j ^ (tid & 15))], dt, kf);
 #pragma unroll
         for (int hh = 0; hh < 8; ++hh) {
           if (hh < NG) {
-            const float mn = fmaxf(m[hh], sc[hh]);
-            const float alpha = ex2(m[hh] - mn);
-            const float pe = ex2(sc[hh] - mn);
-            l[hh] = l[hh] * alpha + pe;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) o[hh][c] = o[hh][c] * alpha + pe * vv[r][c];
-            m[hh] = mn;
+            const float4 qa = reinterpret_cast<const float4*>(sq + hh * D + 8 * j)[0];
+            const float4 qb = reinterpret_cast<const float4*>(sq + hh * D + 8 * j)[1];
+            sc[hh] += qa.x * kf[0] + qa.y * kf[1] + qa.z * kf[2] + qa.w * kf[3] + qb.x * kf[4] + qb.y * kf[5] +
+                      qb.z * kf[6] + qb.w * kf[7];
           }
         }
       }
     }
+    // ---- chunk max and new running max per head
+    float cm[8];
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh) {
+      cm[hh] = (tid < cnt) ? sc[hh] : -INFINITY;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) cm[hh] = fmaxf(cm[hh], __shfl_xor_sync(0xffffffffu, cm[hh], off));
+    }
+    if (lane == 0)
+#pragma unroll
+      for (int hh = 0; hh < 8; ++hh) red[(warp * 8 + hh) * 2] = cm[hh];
+    consumers_sync();  // keys done (the tile can take the values), maxima visible
+    if (tid < cnt) {
+      const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(L.ring_v) +
+                                                        (ring + (Q + c0 + tid) % L.residual) * D);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) cp_async16(tile + tid * 16 + (j ^ (tid & 15)), src + j);
+    }
+    float alpha[8], ps[8];
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh) {
+      const float M = fmaxf(fmaxf(red[hh * 2], red[(8 + hh) * 2]), fmaxf(red[(16 + hh) * 2], red[(24 + hh) * 2]));
+      const float mn = fmaxf(m[hh], M);
+      alpha[hh] = (hh < NG) ? ex2(m[hh] - mn) : 1.f;
+      m[hh] = (hh < NG) ? mn : m[hh];
+      const float pv = (tid < cnt && hh < NG) ? ex2(sc[hh] - mn) : 0.f;
+      if (tid < kResTile && hh < NG) sp[hh * kResTile + tid] = pv;
+      ps[hh] = pv;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) ps[hh] += __shfl_xor_sync(0xffffffffu, ps[hh], off);
+    }
+    cp_async_wait_all();
+    consumers_sync();  // sums of the previous reads done; reuse red for the sums
+    if (lane == 0)
+#pragma unroll
+      for (int hh = 0; hh < 8; ++hh) red[(warp * 8 + hh) * 2 + 1] = ps[hh];
+    consumers_sync();  // values, probabilities and sums visible
+    const int d = tid;  // channel owned for p.v
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh) {
+      if (hh < NG) {
+        l[hh] = l[hh] * alpha[hh] + red[hh * 2 + 1] + red[(8 + hh) * 2 + 1] + red[(16 + hh) * 2 + 1] +
+                red[(24 + hh) * 2 + 1];
+        o[hh] *= alpha[hh];
+      }
+    }
+    const uint16_t* vrow = reinterpret_cast<const uint16_t*>(tile);
+    for (int tau = 0; tau < cnt; ++tau) {
+      const uint16_t bits = vrow[(tau * 16 + ((d >> 3) ^ (tau & 15))) * 8 + (d & 7)];
+      const float vf = (dt == KVQ_BF16) ? __uint_as_float((uint32_t)bits << 16) : __half2float(__ushort_as_half(bits));
+#pragma unroll
+      for (int hh = 0; hh < 8; ++hh)
+        if (hh < NG) o[hh] += sp[hh * kResTile + tau] * vf;
+    }
+    consumers_sync();  // tile and sp free for the next chunk
   }
 #pragma unroll
   for (int hh = 0; hh < 8; ++hh) {
     if (hh < NG) {
-      const int64_t slot = ((int64_t)b * p.num_q_heads + h * NG + hh) * p.slots + warp;
-      *reinterpret_cast<float4*>(p.ws_o + slot * D + 4 * lane) = make_float4(o[hh][0], o[hh][1], o[hh][2], o[hh][3]);
-      if (lane == 0) p.ws_ml[slot] = make_float2(m[hh], l[hh]);
+      const int64_t slot = ((int64_t)b * p.num_q_heads + h * NG + hh) * p.slots;
+      p.ws_o[slot * D + tid] = o[hh];
+      if (tid == 0) p.ws_ml[slot] = make_float2(m[hh], l[hh]);
     }
   }
 }
@@ -384,21 +446,49 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(DecodeParams p, Mm
     // ---------------- consumers
     uint8_t* ws = smem + mp.ws_soff + warp * mp.ws_bytes;
     float* wq = reinterpret_cast<float*>(ws + mp.wq_off);
+    auto stage_q = [&](int b, int h) {  // the unit's scaled queries into wq
+      __syncwarp();
+      // NG*D 16-bit values = NG*16 16-byte vectors; at most 4 per lane, all
+      // loads issued before any is used
+      const uint4* src =
+          reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.q) + ((int64_t)b * p.num_q_heads + h * NG) * D);
+      uint4 v[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (lane + 32 * i < NG * 16) v[i] = src[lane + 32 * i];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (lane + 32 * i < NG * 16) {
+          const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (L.kv_dtype == KVQ_BF16) {
+              f[2 * e] = __uint_as_float(w[e] << 16);
+              f[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+            } else {
+              const float2 x = unpack_f16(w[e]);
+              f[2 * e] = x.x;
+              f[2 * e + 1] = x.y;
+            }
+          }
+          float4* dst = reinterpret_cast<float4*>(wq + (lane + 32 * i) * 8);
+          dst[0] = make_float4(f[0] * p.scale_log2, f[1] * p.scale_log2, f[2] * p.scale_log2, f[3] * p.scale_log2);
+          dst[1] = make_float4(f[4] * p.scale_log2, f[5] * p.scale_log2, f[6] * p.scale_log2, f[7] * p.scale_log2);
+        }
+      }
+      __syncwarp();
+    };
+    // residual units of this CTA first (the producer already streams); the
+    // consumer scratch areas, contiguous, serve as the ring tile buffer
+    for (int r = c; r < p.batch * L.num_kv_heads; r += p.num_ctas)
+      residual_unit(p, r / L.num_kv_heads, r % L.num_kv_heads, NG, smem + mp.ws_soff);
+    __syncwarp();
+    consumers_sync();  // the scratch areas are per warp again
     {  // rows of heads >= NG stay zero
       uint4* af = reinterpret_cast<uint4*>(ws + mp.afrag_off);
       for (int e = lane; e < 8 * 8 * 4; e += 32)
         if (((e >> 2) & 7) >= NG) af[e] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    auto stage_q = [&](int b, int h) {  // the unit's scaled queries into wq
-      __syncwarp();
-      for (int e = lane; e < NG * D; e += 32)
-        wq[e] = load_kv(p.q, ((int64_t)b * p.num_q_heads + h * NG) * D + e, L.kv_dtype) * p.scale_log2;
-      __syncwarp();
-    };
-    // residual units of this CTA first (the producer already streams)
-    for (int r = c; r < p.batch * L.num_kv_heads; r += p.num_ctas) {
-      stage_q(r / L.num_kv_heads, r % L.num_kv_heads);
-      residual_unit(p, r / L.num_kv_heads, r % L.num_kv_heads, NG, wq);
     }
 
     const int g = lane >> 2, t = lane & 3;
@@ -645,6 +735,8 @@ MmaPlan make_mma_plan(const LayerView& L) {
   mp.vpair_off = mp.bias_off + 64;
   mp.wq_off = (int32_t)round_up(mp.vpair_off + (G / 16) * 4 * ngrp * 16, 16);
   mp.ws_bytes = (int32_t)round_up(mp.wq_off + 8 * D * 4, 128);
+  // the four scratch areas together also hold the residual ring tile
+  if (kNC * mp.ws_bytes < kResScratch) mp.ws_bytes = (int32_t)round_up((kResScratch + kNC - 1) / kNC, 128);
   // The stage count is a multiple of the consumer-warp count, so stage st is
   // always consumed by warp st % kNC: every waiter of a stage's barriers then
   // waits for its phases in order and never one phase too early (a parity
