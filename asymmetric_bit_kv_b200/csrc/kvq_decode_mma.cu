@@ -81,14 +81,17 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// Not volatile: the compiler may schedule these freely. ldmatrix keeps a
+// memory clobber so that it stays behind the barrier waits that publish the
+// shared memory it reads.
 __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
+  asm("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+      : "r"(addr)
+      : "memory");
 }
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -323,12 +326,16 @@ struct UnitCursor {
 };
 
 // Per-warp scratch, rebuilt from each block's fp16 scales before its MMAs:
-//   afrag [8 kk][8 heads][4 t] uint4: rows g (fp16 high) and g+8 (fp16 low)
-//         of (q * s) for channels 16kk + 2t + {0,1,8,9} (A-fragment order);
+//   afrag [8 kk][32 slots] uint4: slot (g*4 + t) ^ kk holds rows g (fp16
+//         high) and g+8 (fp16 low) of (q * s) for channels 16kk + 2t +
+//         {0,1,8,9} (A-fragment order; the XOR keeps both the writes and the
+//         reads of a k-chunk spread over all shared-memory banks);
 //   bias  [8] float: sum_d q_d z_d per head;
 //   vpair [k-step][4 t][groups] uint4: (s_X, s_Y, z_X, z_Y) fp16 pairs of the
 //         tokens thread t feeds into a PV k-step;
-//   wq    [8][D] float: the unit's queries times softmax_scale*log2(e).
+//   wq    [8 kk][8 heads][4 x 16 B] float: the unit's queries times
+//         softmax_scale*log2(e), k-chunk-major; piece v of row (kk, head) is
+//         stored at v ^ (kk & 3) so the prep's reads spread over all banks.
 template <int KB, int VB, int NGRP>
 __device__ __forceinline__ void prep_block(const uint8_t* stage, const MmaPlan& mp, uint8_t* ws, int NG, int G,
                                            int lane) {
@@ -344,12 +351,12 @@ __device__ __forceinline__ void prep_block(const uint8_t* stage, const MmaPlan& 
     const int hh = pr >> 3, kk = pr & 7;
     float bp = 0.f;
     if (hh < NG) {
-      const float4* q4 = reinterpret_cast<const float4*>(wq + hh * D + 16 * kk);
+      const float4* q4 = reinterpret_cast<const float4*>(wq + (kk * 8 + hh) * 16);
       const uint4* s4 = reinterpret_cast<const uint4*>(ksz + 16 * kk);
       float x[16];
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
-        const float4 qq = q4[v];
+        const float4 qq = q4[v ^ (kk & 3)];  // wq rows are stored XOR-swizzled by kk
         const uint4 ss = s4[v];
         const float qa[4] = {qq.x, qq.y, qq.z, qq.w};
         const uint32_t sa[4] = {ss.x, ss.y, ss.z, ss.w};
@@ -364,8 +371,8 @@ __device__ __forceinline__ void prep_block(const uint8_t* stage, const MmaPlan& 
       for (int tt = 0; tt < 4; ++tt) {
         const uint32_t h01 = pack_f16(x[2 * tt], x[2 * tt + 1]), h89 = pack_f16(x[2 * tt + 8], x[2 * tt + 9]);
         const float2 f01 = unpack_f16(h01), f89 = unpack_f16(h89);
-        af[(kk * 8 + hh) * 4 + tt] = make_uint4(h01, pack_f16(x[2 * tt] - f01.x, x[2 * tt + 1] - f01.y), h89,
-                                                pack_f16(x[2 * tt + 8] - f89.x, x[2 * tt + 9] - f89.y));
+        af[kk * 32 + ((hh * 4 + tt) ^ kk)] = make_uint4(h01, pack_f16(x[2 * tt] - f01.x, x[2 * tt + 1] - f01.y), h89,
+                                                        pack_f16(x[2 * tt + 8] - f89.x, x[2 * tt + 9] - f89.y));
       }
     }
     if (rep == 1 && NG <= 4) break;
@@ -472,9 +479,13 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(DecodeParams p, Mm
               f[2 * e + 1] = x.y;
             }
           }
-          float4* dst = reinterpret_cast<float4*>(wq + (lane + 32 * i) * 8);
-          dst[0] = make_float4(f[0] * p.scale_log2, f[1] * p.scale_log2, f[2] * p.scale_log2, f[3] * p.scale_log2);
-          dst[1] = make_float4(f[4] * p.scale_log2, f[5] * p.scale_log2, f[6] * p.scale_log2, f[7] * p.scale_log2);
+          const int e16 = lane + 32 * i;  // 8 channels: head e16/16, channels (e16%16)*8..
+          const int hh = e16 >> 4, kk = (e16 & 15) >> 1, v0 = (e16 & 1) * 2;
+          float4* row = reinterpret_cast<float4*>(wq + (kk * 8 + hh) * 16);
+          row[v0 ^ (kk & 3)] =
+              make_float4(f[0] * p.scale_log2, f[1] * p.scale_log2, f[2] * p.scale_log2, f[3] * p.scale_log2);
+          row[(v0 + 1) ^ (kk & 3)] =
+              make_float4(f[4] * p.scale_log2, f[5] * p.scale_log2, f[6] * p.scale_log2, f[7] * p.scale_log2);
         }
       }
       __syncwarp();
@@ -487,8 +498,8 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(DecodeParams p, Mm
     consumers_sync();  // the scratch areas are per warp again
     {  // rows of heads >= NG stay zero
       uint4* af = reinterpret_cast<uint4*>(ws + mp.afrag_off);
-      for (int e = lane; e < 8 * 8 * 4; e += 32)
-        if (((e >> 2) & 7) >= NG) af[e] = make_uint4(0u, 0u, 0u, 0u);
+      for (int e = lane; e < 8 * 8 * 4; e += 32)  // e = kk*32 + physical slot
+        if (((((e & 31) ^ (e >> 5)) >> 2) & 7) >= NG) af[e] = make_uint4(0u, 0u, 0u, 0u);
     }
 
     const int g = lane >> 2, t = lane & 3;
@@ -536,16 +547,25 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(DecodeParams p, Mm
           float Sacc[S::NT][4];
 #pragma unroll
           for (int i2 = 0; i2 < S::NT; ++i2) Sacc[i2][0] = Sacc[i2][1] = Sacc[i2][2] = Sacc[i2][3] = 0.f;
+          // all key code loads of the tile first (one ldmatrix.x4 per k-chunk
+          // pair and 16-byte chunk), then the conversions and MMAs
+          uint32_t rk[4][S::SIG][4];
+#pragma unroll
+          for (int kp = 0; kp < 4; ++kp) {
+            const int ch = 16 * (2 * kp + (mi >> 1)) + 8 * (mi & 1) + rr;
+#pragma unroll
+            for (int sg = 0; sg < S::SIG; ++sg)
+              ldsm_x4_t(kc_s + ch * kc_row + (((tile * S::SIG + sg) ^ swk) << 4), rk[kp][sg][0], rk[kp][sg][1],
+                        rk[kp][sg][2], rk[kp][sg][3]);
+          }
 #pragma unroll
           for (int kk = 0; kk < 8; kk += 2) {
-            const int ch = 16 * (kk + (mi >> 1)) + 8 * (mi & 1) + rr;
 #pragma unroll
             for (int sg = 0; sg < S::SIG; ++sg) {
-              uint32_t r[4];
-              ldsm_x4_t(kc_s + ch * kc_row + (((tile * S::SIG + sg) ^ swk) << 4), r[0], r[1], r[2], r[3]);
+              const uint32_t* r = rk[kk / 2][sg];
 #pragma unroll
               for (int jj = 0; jj < 2; ++jj) {
-                const uint4 av = afr[((kk + jj) * 8 + g) * 4 + t];
+                const uint4 av = afr[(kk + jj) * 32 + ((g * 4 + t) ^ (kk + jj))];
                 const uint32_t A[4] = {av.x, av.y, av.z, av.w};
                 const uint32_t x0 = r[2 * jj], x1 = r[2 * jj + 1];
                 const uint32_t x0h = x0 >> 8, x1h = x1 >> 8;
