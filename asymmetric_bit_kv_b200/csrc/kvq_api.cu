@@ -207,7 +207,149 @@ kvq_status enqueue_append(kvq_cache* c, int layer, const void* k, const void* v,
   return KVQ_OK;
 }
 
+// Points the split partials of p at `scratch` with a slot stride of `slots`;
+// false (and *status) if they do not fit.
+bool use_scratch(kvq::DecodeParams& p, const kvq::StaticScratch& scratch, int batch, int32_t slots, kvq_status* status) {
+  const int64_t partials = (int64_t)batch * p.num_q_heads * slots;
+  const int64_t o_bytes = kvq::round_up(partials * kvq::kHeadDim * 4, 256);
+  const int64_t need = o_bytes + partials * 8;
+  if (need > scratch.bytes) {
+    *status = fail(KVQ_ERR_WORKSPACE,
+                   "this decode needs %lld bytes of split partials (batch %d x %d query heads x %d slots); the "
+                   "static scratch holds %lld",
+                   (long long)need, batch, p.num_q_heads, slots, (long long)scratch.bytes);
+    return false;
+  }
+  p.slots = slots;
+  p.ws_o = reinterpret_cast<float*>(scratch.base);
+  p.ws_ml = reinterpret_cast<float2*>(scratch.base + o_bytes);
+  return true;
+}
+
 }  // namespace
+
+namespace kvq {
+
+// Decode attention of kvq_decode_attention. With scratch == nullptr the
+// split partials live in the arena's workspace (slot stride = the arena's
+// slot count); otherwise in `scratch`, with the slot stride cut to what this
+// call uses, and a call whose partials would not fit is rejected before
+// anything is enqueued.
+kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out, int32_t out_dtype,
+                          float softmax_scale, int32_t batch, void* stream, const StaticScratch* scratch) {
+  kvq_status s = check_cache_layer(c, layer);
+  if (s != KVQ_OK) return s;
+  if (batch < 0 || batch > c->cfg.max_batch)
+    return fail(KVQ_ERR_INVALID_ARG, "batch %d outside 0..%d", batch, c->cfg.max_batch);
+  if (out_dtype != KVQ_F32 && out_dtype != KVQ_F16 && out_dtype != KVQ_BF16)
+    return fail(KVQ_ERR_INVALID_ARG, "out_dtype %d", out_dtype);
+  if (!std::isfinite(softmax_scale)) return fail(KVQ_ERR_INVALID_ARG, "softmax_scale is not finite");
+  if (batch == 0) return KVQ_OK;
+  if (!q || !out) return fail(KVQ_ERR_INVALID_ARG, "q or out is null");
+  if (!aligned16(q) || !aligned16(out)) return fail(KVQ_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+  const kvq_config& cfg = c->cfg;
+  const int G = cfg.group_k;
+  const kvq::LayerView L = layer_view(c, layer);
+  const bool use_mma = kvq::mma_supported(L);
+  kvq::MmaPlan mp{};
+  int per_sm = 4;
+  if (use_mma) {
+    mp = kvq::make_mma_plan(L);
+    per_sm = kvq::mma_ctas_per_sm(L, mp);
+  }
+  std::vector<int> nblk(batch);
+  int max_blk = 0;
+  int64_t total_blocks = 0;
+  for (int b = 0; b < batch; ++b) {
+    nblk[b] = c->q_len[(size_t)layer * cfg.max_batch + b] / G;
+    max_blk = std::max(max_blk, nblk[b]);
+    total_blocks += (int64_t)nblk[b] * cfg.num_kv_heads;
+  }
+  if (total_blocks > INT32_MAX) return fail(KVQ_ERR_UNSUPPORTED, "more than 2^31 quantized blocks in one call");
+  kvq::DecodeParams* pp = new (std::nothrow) kvq::DecodeParams;
+  if (!pp) return fail(KVQ_ERR_INVALID_ARG, "out of host memory");
+  kvq::DecodeParams& p = *pp;
+  std::memset(pp, 0, sizeof *pp);
+  p.L = L;
+  p.q = q;
+  p.out = out;
+  p.ws_o = reinterpret_cast<float*>(c->arena + c->ws_o_off);
+  p.ws_ml = reinterpret_cast<float2*>(c->arena + c->ws_ml_off);
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.out_dtype = out_dtype;
+  p.batch = batch;
+  p.num_q_heads = cfg.num_q_heads;
+  p.slots = c->slots;
+  p.err = reinterpret_cast<int32_t*>(c->arena + c->err_off);
+  cudaError_t e;
+  int32_t used_slots = c->slots;  // partial slots per (sequence, query head) this call writes
+  if (use_mma) {
+    // Persistent plan: one CTA per resident slot (fewer if there is little
+    // work), each taking a contiguous range of the concatenated blocks.
+    int64_t nctas = std::min<int64_t>((int64_t)std::max(1, c->sm_count) * per_sm,
+                                      std::max<int64_t>((int64_t)batch * cfg.num_kv_heads, (total_blocks + 3) / 4));
+    nctas = std::max<int64_t>(nctas, 1);
+    // every (sequence, head) must fit its partials in the workspace
+    int64_t acc = 0;
+    for (int b = 0; b < batch; ++b) {
+      p.nblk[b] = nblk[b];
+      p.seq_start[b] = (int32_t)acc;
+      acc += (int64_t)nblk[b] * cfg.num_kv_heads;
+    }
+    for (;;) {
+      int32_t need = kvq::kResidualSlots;
+      for (int b = 0; b < batch && total_blocks > 0; ++b)
+        for (int h = 0; h < cfg.num_kv_heads; ++h)
+          need = std::max(need, kvq::persistent_slots(total_blocks, (int32_t)nctas, p.seq_start[b] + h * nblk[b], nblk[b]));
+      used_slots = need;
+      if (need <= c->slots || nctas == 1) break;
+      nctas = std::max<int64_t>(1, nctas * 3 / 4);
+    }
+    p.persistent = 1;
+    p.total_blocks = (int32_t)total_blocks;
+    p.num_ctas = (int32_t)nctas;
+    if (scratch && !use_scratch(p, *scratch, batch, used_slots, &s)) {
+      delete pp;
+      return s;
+    }
+    e = kvq::launch_decode_mma(p, mp, 0, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = kvq::launch_combine(p, static_cast<cudaStream_t>(stream));
+  } else {
+    // Split plan: blocks per split chosen to minimise (waves of CTAs) x
+    // (blocks per CTA + a fixed per-CTA overhead), with at most slots-1 splits.
+    const int64_t slots_gpu = (int64_t)std::max(1, c->sm_count) * per_sm;
+    const int64_t min_bps = std::max<int64_t>(1, (max_blk + (c->slots - 1) - 1) / (c->slots - 1));
+    int64_t bps = std::max<int64_t>(min_bps, max_blk);
+    double best = 1e300;
+    for (int64_t cand = min_bps; cand <= std::max<int64_t>(min_bps, max_blk); ++cand) {
+      int64_t ctas = 0;
+      for (int b = 0; b < batch; ++b) ctas += (nblk[b] + cand - 1) / cand;
+      ctas *= cfg.num_kv_heads;
+      const double waves = (double)((ctas + slots_gpu - 1) / slots_gpu);
+      const double cost = waves * (double)(cand + 2);
+      if (cost < best) {
+        best = cost;
+        bps = cand;
+      }
+    }
+    p.blocks_per_split = (int32_t)bps;
+    const int nsplits = (int)((max_blk + bps - 1) / bps);
+    used_slots = nsplits + 1;
+    if (scratch && !use_scratch(p, *scratch, batch, used_slots, &s)) {
+      delete pp;
+      return s;
+    }
+    e = kvq::launch_decode(p, nsplits, static_cast<cudaStream_t>(stream));
+  }
+  delete pp;
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return KVQ_OK;
+}
+
+void clear_last_error() { g_last_error.clear(); }
+kvq_status report_cuda_error(cudaError_t e, const char* what) { return cuda_fail(e, what); }
+
+}  // namespace kvq
 
 extern "C" {
 
@@ -336,101 +478,7 @@ kvq_status kvq_flush_residual(kvq_cache* c, int32_t layer, int32_t batch, void* 
 kvq_status kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, void* out, int32_t out_dtype,
                                 float softmax_scale, int32_t batch, void* stream) {
   g_last_error.clear();
-  kvq_status s = check_cache_layer(c, layer);
-  if (s != KVQ_OK) return s;
-  if (batch < 0 || batch > c->cfg.max_batch)
-    return fail(KVQ_ERR_INVALID_ARG, "batch %d outside 0..%d", batch, c->cfg.max_batch);
-  if (out_dtype != KVQ_F32 && out_dtype != KVQ_F16 && out_dtype != KVQ_BF16)
-    return fail(KVQ_ERR_INVALID_ARG, "out_dtype %d", out_dtype);
-  if (!std::isfinite(softmax_scale)) return fail(KVQ_ERR_INVALID_ARG, "softmax_scale is not finite");
-  if (batch == 0) return KVQ_OK;
-  if (!q || !out) return fail(KVQ_ERR_INVALID_ARG, "q or out is null");
-  if (!aligned16(q) || !aligned16(out)) return fail(KVQ_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
-  const kvq_config& cfg = c->cfg;
-  const int G = cfg.group_k;
-  const kvq::LayerView L = layer_view(c, layer);
-  const bool use_mma = kvq::mma_supported(L);
-  kvq::MmaPlan mp{};
-  int per_sm = 4;
-  if (use_mma) {
-    mp = kvq::make_mma_plan(L);
-    per_sm = kvq::mma_ctas_per_sm(L, mp);
-  }
-  std::vector<int> nblk(batch);
-  int max_blk = 0;
-  int64_t total_blocks = 0;
-  for (int b = 0; b < batch; ++b) {
-    nblk[b] = c->q_len[(size_t)layer * cfg.max_batch + b] / G;
-    max_blk = std::max(max_blk, nblk[b]);
-    total_blocks += (int64_t)nblk[b] * cfg.num_kv_heads;
-  }
-  if (total_blocks > INT32_MAX) return fail(KVQ_ERR_UNSUPPORTED, "more than 2^31 quantized blocks in one call");
-  kvq::DecodeParams* pp = new (std::nothrow) kvq::DecodeParams;
-  if (!pp) return fail(KVQ_ERR_INVALID_ARG, "out of host memory");
-  kvq::DecodeParams& p = *pp;
-  std::memset(pp, 0, sizeof *pp);
-  p.L = L;
-  p.q = q;
-  p.out = out;
-  p.ws_o = reinterpret_cast<float*>(c->arena + c->ws_o_off);
-  p.ws_ml = reinterpret_cast<float2*>(c->arena + c->ws_ml_off);
-  p.scale_log2 = softmax_scale * 1.4426950408889634f;
-  p.out_dtype = out_dtype;
-  p.batch = batch;
-  p.num_q_heads = cfg.num_q_heads;
-  p.slots = c->slots;
-  p.err = reinterpret_cast<int32_t*>(c->arena + c->err_off);
-  cudaError_t e;
-  if (use_mma) {
-    // Persistent plan: one CTA per resident slot (fewer if there is little
-    // work), each taking a contiguous range of the concatenated blocks.
-    int64_t nctas = std::min<int64_t>((int64_t)std::max(1, c->sm_count) * per_sm,
-                                      std::max<int64_t>((int64_t)batch * cfg.num_kv_heads, (total_blocks + 3) / 4));
-    nctas = std::max<int64_t>(nctas, 1);
-    // every (sequence, head) must fit its partials in the workspace
-    int64_t acc = 0;
-    for (int b = 0; b < batch; ++b) {
-      p.nblk[b] = nblk[b];
-      p.seq_start[b] = (int32_t)acc;
-      acc += (int64_t)nblk[b] * cfg.num_kv_heads;
-    }
-    for (;;) {
-      int32_t need = kvq::kResidualSlots;
-      for (int b = 0; b < batch && total_blocks > 0; ++b)
-        for (int h = 0; h < cfg.num_kv_heads; ++h)
-          need = std::max(need, kvq::persistent_slots(total_blocks, (int32_t)nctas, p.seq_start[b] + h * nblk[b], nblk[b]));
-      if (need <= c->slots || nctas == 1) break;
-      nctas = std::max<int64_t>(1, nctas * 3 / 4);
-    }
-    p.persistent = 1;
-    p.total_blocks = (int32_t)total_blocks;
-    p.num_ctas = (int32_t)nctas;
-    e = kvq::launch_decode_mma(p, mp, 0, static_cast<cudaStream_t>(stream));
-    if (e == cudaSuccess) e = kvq::launch_combine(p, static_cast<cudaStream_t>(stream));
-  } else {
-    // Split plan: blocks per split chosen to minimise (waves of CTAs) x
-    // (blocks per CTA + a fixed per-CTA overhead), with at most slots-1 splits.
-    const int64_t slots_gpu = (int64_t)std::max(1, c->sm_count) * per_sm;
-    const int64_t min_bps = std::max<int64_t>(1, (max_blk + (c->slots - 1) - 1) / (c->slots - 1));
-    int64_t bps = std::max<int64_t>(min_bps, max_blk);
-    double best = 1e300;
-    for (int64_t cand = min_bps; cand <= std::max<int64_t>(min_bps, max_blk); ++cand) {
-      int64_t ctas = 0;
-      for (int b = 0; b < batch; ++b) ctas += (nblk[b] + cand - 1) / cand;
-      ctas *= cfg.num_kv_heads;
-      const double waves = (double)((ctas + slots_gpu - 1) / slots_gpu);
-      const double cost = waves * (double)(cand + 2);
-      if (cost < best) {
-        best = cost;
-        bps = cand;
-      }
-    }
-    p.blocks_per_split = (int32_t)bps;
-    e = kvq::launch_decode(p, (int)((max_blk + bps - 1) / bps), static_cast<cudaStream_t>(stream));
-  }
-  delete pp;
-  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  return KVQ_OK;
+  return kvq::enqueue_decode(c, layer, q, out, out_dtype, softmax_scale, batch, stream, nullptr);
 }
 
 kvq_status kvq_dequant(kvq_cache* c, int32_t layer, int32_t seq, int32_t t0, int32_t t1, float* k_out,

@@ -89,4 +89,17 @@ cudaError_t launch_decode(const DecodeParams& p, int max_splits, cudaStream_t st
 // The log-sum-exp combine alone (after launch_decode_mma).
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream);
 
+// Device memory for the split partials other than the arena's workspace.
+struct StaticScratch {
+  uint8_t* base;   // device address, 256-byte aligned
+  int64_t bytes;
+};
+
+// Host side of kvq_decode_attention (kvq_api.cu): validation, split plan and
+// launches; the partials go to `scratch` when it is not null.
+kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out, int32_t out_dtype,
+                          float softmax_scale, int32_t batch, void* stream, const StaticScratch* scratch);
+void clear_last_error();
+kvq_status report_cuda_error(cudaError_t e, const char* what);
+
 }  // namespace kvq

@@ -84,6 +84,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kvq_append": (I32, [P, I32, P, P, ctypes.POINTER(I32), I32, P]),
         "kvq_flush_residual": (I32, [P, I32, I32, P]),
         "kvq_decode_attention": (I32, [P, I32, P, P, I32, F32, I32, P]),
+        "kvq_decode_attention_noalloc": (I32, [P, I32, P, P, I32, F32, I32, P]),
         "kvq_dequant": (I32, [P, I32, I32, I32, I32, P, P, P]),
         "kvq_get_layout": (I32, [P, I32, ctypes.POINTER(kvq_layout)]),
         "kvq_device_errors": (I32, [P, ctypes.POINTER(I32)]),
@@ -202,6 +203,20 @@ class KVCache:
         _check(self.lib.kvq_decode_attention(self.handle, layer, q.data_ptr(), out.data_ptr(), _DTYPE_CODE[out.dtype],
                                              float(softmax_scale), q.shape[0], _stream_ptr(stream)),
                "kvq_decode_attention")
+        return out
+
+    def decode_attention_noalloc(self, layer: int, q: torch.Tensor, out: torch.Tensor,
+                                 softmax_scale: float | None = None, stream=None):
+        """decode_attention with the split partials in the library's static
+        device scratch instead of the arena (kvq_decode_attention_noalloc)."""
+        _need(q, self.cfg.kv_dtype, "q")
+        _need(out, out.dtype, "out")
+        if softmax_scale is None:
+            softmax_scale = self.cfg.head_dim ** -0.5
+        _check(self.lib.kvq_decode_attention_noalloc(self.handle, layer, q.data_ptr(), out.data_ptr(),
+                                                     _DTYPE_CODE[out.dtype], float(softmax_scale), q.shape[0],
+                                                     _stream_ptr(stream)),
+               "kvq_decode_attention_noalloc")
         return out
 
     def dequant(self, layer: int, seq: int, t0: int, t1: int, stream=None):

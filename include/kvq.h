@@ -164,6 +164,34 @@ KVQ_API kvq_status kvq_decode_attention(kvq_cache* cache, int32_t layer, const v
                                 int32_t out_dtype, float softmax_scale, int32_t batch,
                                 void* stream);
 
+/* Size of the library's own device scratch for kvq_decode_attention_noalloc:
+ * 16 MiB, held on every GPU that loads the library until the process exits. */
+#define KVQ_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* Same result as kvq_decode_attention, for callers that cannot allocate
+ * device memory at the point of the call, for example an engine whose device
+ * memory is all handed to its own pool at start-up, or code running under a
+ * fixed memory budget where a cudaMalloc could fail or stall the device.
+ * This call allocates nothing. Its split partials go to a static device array
+ * of KVQ_STATIC_SCRATCH_BYTES that the library holds, not to the arena's
+ * workspace, which it leaves untouched. The pages have no counterpart: this
+ * is an interface choice of this library.
+ * - Size limit: the partials take batch * Hq * S * (4*head_dim + 8) bytes,
+ *   where S is the number of partial slots this call's split plan uses per
+ *   (sequence, query head). A call that needs more than the scratch holds
+ *   returns KVQ_ERR_WORKSPACE, enqueues nothing, and kvq_last_error() gives
+ *   both sizes.
+ * - Set-up: the first call on each device looks up the array's device
+ *   address (cudaGetSymbolAddress, with that device current). Make that first
+ *   call before any stream capture.
+ * - Sharing: every call on a device uses the same array and leaves the last
+ *   call's partials in it. Each call writes every partial it reads, so nothing
+ *   has to start at zero. Calls that may overlap on the GPU race on the array
+ *   (different streams, or several caches): order them.                   */
+KVQ_API kvq_status kvq_decode_attention_noalloc(kvq_cache* cache, int32_t layer, const void* q, void* out,
+                                        int32_t out_dtype, float softmax_scale, int32_t batch,
+                                        void* stream);
+
 /* Reconstruct tokens [t0, t1) of sequence `seq` as fp32: x_hat = q*d + m
  * (an fp32 product, then an fp32 sum; KV1 card, BQ2_0) for quantized tokens
  * and the exact stored value for ring tokens. k_out, v_out: device
