@@ -31,6 +31,8 @@
 //    group with an all-ones A operand.
 //  * Online softmax in log2 units per 64-token tile; fp32 partials per split
 //    are merged by the log-sum-exp combine kernel.
+#include <mutex>
+
 #include "kvq_decode.cuh"
 
 namespace kvq {
@@ -790,8 +792,24 @@ int mma_ctas_per_sm(const LayerView& L, const MmaPlan& mp) {
   KVQ_MMA_INSTANCES(KVQ_FN)
 #undef KVQ_FN
   if (!fn) return 1;
+  // one occupancy query per (device, instance, shared-memory size)
+  struct Entry {
+    int dev;
+    const void* fn;
+    int smem;
+    int n;
+  };
+  static Entry memo[64];
+  static int nmemo = 0;
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < nmemo; ++i)
+    if (memo[i].dev == dev && memo[i].fn == fn && memo[i].smem == mp.smem_bytes) return memo[i].n;
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, mp.smem_bytes) != cudaSuccess) return 1;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kThreads, mp.smem_bytes) != cudaSuccess || n < 1) return 1;
+  if (nmemo < 64) memo[nmemo++] = Entry{dev, fn, mp.smem_bytes, n};
   return n;
 }
 

@@ -216,6 +216,23 @@ def cpu_oracle_baseline(steps: int = 100, warmup: int = 2):
 # the library arm
 # --------------------------------------------------------------------------
 
+def _workload_config(wl, replicas, world, mean_ctx=None):
+    """The `config` object of the JSON line (shared by both arms)."""
+    cfg = {
+        "workload": wl.name,
+        "batch": wl.batch, "num_q_heads": wl.num_q_heads, "num_kv_heads": wl.num_kv_heads,
+        "head_dim": wl.head_dim, "context": wl.context[0], "k_bits": wl.k_bits[0], "v_bits": wl.v_bits[0],
+        "group_k": wl.group_k, "group_v": wl.group_v, "residual": wl.residual,
+        "kv_dtype": "bf16", "out_dtype": "bf16",
+        "replicas": replicas,
+        "l2": "inputs larger than L2: each step reads a different replica's ~248 MB cache",
+        "parallelism": f"dp{world} (independent replicas per rank)",
+    }
+    if mean_ctx is not None:
+        cfg["mean_context_timed"] = mean_ctx
+    return cfg
+
+
 def run_kvq(a):
     import torch
     import torch.distributed as dist
@@ -244,7 +261,6 @@ def run_kvq(a):
         del k, v
         caches.append(c)
     torch.cuda.synchronize()
-    n_new = max(a.warmup + a.steps, 1)
     gen = torch.Generator(device=dev).manual_seed(12345 + rank)
     pool = 64  # distinct per-step inputs, reused round-robin
     new_k = torch.randn(pool, B, Hkv, D, generator=gen, device=dev).to(wl.kv_dtype)
@@ -255,18 +271,7 @@ def run_kvq(a):
     stream = torch.cuda.current_stream()
     bytes_tok = O.quantized_bytes_per_token(Hkv, D, wl.k_bits[0], wl.v_bits[0], wl.group_k, wl.group_v)
 
-    lengths = [[ctx] * B for _ in range(R)]
-
-    def alg_bytes_and_tokens(r):
-        """Algorithmic bytes read+written by decode attention of replica r (its
-        current lengths): packed cache + residual ring + q + out."""
-        tot, toks = 0.0, 0
-        for b in range(B):
-            qn, n = caches[r].lengths(0, b)
-            tot += qn * bytes_tok + n * Hkv * D * 2 * 2
-            toks += qn + n
-        tot += 2 * B * Hq * D * 2
-        return tot, toks
+    G, Rw = wl.group_k, wl.residual
 
     def step(i, r, ev=None):
         caches[r].append(0, new_k[i % pool], new_v[i % pool], ones)
@@ -276,48 +281,58 @@ def run_kvq(a):
         if ev is not None:
             ev[1].record(stream)
 
-    # launches of this library per step: ring write + decode split + combine,
-    # plus one quantize launch on steps where a ring is full (lazy flush)
-    def launches_for(r):
-        q0, n0 = caches[r].lengths(0, 0)
-        return 3 + (1 if n0 == wl.residual else 0)
-
     for i in range(a.warmup):
         step(i, i % R)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
 
-    # per-step accounting (host mirror, before the step)
-    launches = 0
-    alg_total, tok_total = 0.0, 0
-    dec_events = []
+    # Per-step accounting, computed before the timed loop so that the loop only
+    # enqueues work: the (quantized, ring) lengths of every replica follow the
+    # flush rule (a token that finds a full ring first moves G ring tokens into
+    # the quantized cache), checked against the library's host mirror after.
+    lens = [[list(caches[r].lengths(0, b)) for b in range(B)] for r in range(R)]
+    plan = []  # (replica, launches, algorithmic bytes of the decode, KV tokens attended)
+    for i in range(a.steps):
+        r = (a.warmup + i) % R
+        launches = 3 + (1 if lens[r][0][1] == Rw else 0)  # ring write + decode + combine (+ flush)
+        ab, tk = 2 * B * Hq * D * 2, 0  # q in, out
+        for b in range(B):
+            qn, n = lens[r][b]
+            if n == Rw:
+                qn, n = qn + G, n - G
+            n += 1
+            lens[r][b] = [qn, n]
+            ab += qn * bytes_tok + n * Hkv * D * 2 * 2
+            tk += qn + n
+        plan.append((r, launches, ab, tk))
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+    launches = sum(x[1] for x in plan)
+    alg_total = float(sum(x[2] for x in plan))
+    tok_total = sum(x[3] for x in plan)
+
     clocks = ClockSampler(local)
     clocks.start()
-    time.sleep(0.1)
+    time.sleep(0.2)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0 = time.perf_counter()
     e0.record(stream)
     for i in range(a.steps):
-        r = (a.warmup + i) % R
-        launches += launches_for(r)
-        ab, tk = alg_bytes_and_tokens(r)
-        alg_total += ab
-        tok_total += tk + B  # the decode sees the appended token too
-        ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-        step(a.warmup + i, r, ev)
-        dec_events.append(ev)
+        step(a.warmup + i, plan[i][0], events[i])
     e1.record(stream)
+    host_s = time.perf_counter() - h0
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
+    for r in range(R):
+        for b in range(B):
+            assert tuple(lens[r][b]) == caches[r].lengths(0, b), "step accounting out of sync with the cache"
     ms = e0.elapsed_time(e1)
-    dec_ms = sum(x[0].elapsed_time(x[1]) for x in dec_events)
-    # the appended token adds B * Hkv * D * 2 (K, V) * 2 bytes to the residual read
-    alg_total += a.steps * B * Hkv * D * 2 * 2
+    dec_ms = sum(x[0].elapsed_time(x[1]) for x in events)
     if world > 1:
         t = torch.tensor([ms, dec_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -340,7 +355,12 @@ def run_kvq(a):
     tok_e2e = 0
     for i in range(e2e_steps):
         r = (a.warmup + a.steps + i) % R
-        tok_e2e += alg_bytes_and_tokens(r)[1] + B
+        for b in range(B):
+            qn, n = lens[r][b]
+            if n == Rw:
+                qn, n = qn + G, n - G
+            lens[r][b] = [qn, n + 1]
+            tok_e2e += qn + n + 1
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -381,17 +401,7 @@ def run_kvq(a):
             "vs_baseline": None,
             "dtype": "f32",
             "data": "synthetic (seeded; Llama-3-8B-shaped layer, no model weights)",
-            "config": {
-                "workload": wl.name,
-                "batch": B, "num_q_heads": Hq, "num_kv_heads": Hkv, "head_dim": D,
-                "context": ctx, "k_bits": wl.k_bits[0], "v_bits": wl.v_bits[0],
-                "group_k": wl.group_k, "group_v": wl.group_v, "residual": wl.residual,
-                "kv_dtype": "bf16", "out_dtype": "bf16",
-                "replicas": R,
-                "mean_context_timed": tok_total / (a.steps * B),
-                "l2": "inputs larger than L2: each step reads a different replica's ~248 MB cache",
-                "parallelism": f"dp{world} (independent replicas per rank)",
-            },
+            "config": _workload_config(wl, R, world, tok_total / (a.steps * B)),
             "roofline": {
                 "kernel": "decode attention (split-KV kernel + log-sum-exp combine), per call",
                 "bound": "hbm",
@@ -403,6 +413,7 @@ def run_kvq(a):
                 "frac_of_8tbs_nominal": achieved_gbs / 8000.0,
                 "traffic": traffic,
                 "decode_us_per_call": dec_ms / a.steps * 1e3,
+                "host_enqueue_us_per_step": host_s / a.steps * 1e6,
                 "alg_bytes_per_call": alg_total / a.steps,
             },
             "e2e": {"value": e2e_value, "unit": UNIT,
@@ -418,14 +429,31 @@ def run_kvq(a):
     return result
 
 
+def _kernel_source_hash():
+    import glob
+    import hashlib
+
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "asymmetric_bit_kv_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
 def _committed_traffic():
-    """DRAM bytes per launch of the decode kernel from the committed ncu summary, if any."""
+    """DRAM bytes (read + write) per decode launch from the committed ncu
+    capture, or None if there is none or the kernel sources changed since."""
     p = os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
         with open(p) as f:
-            return json.load(f).get("dram_bytes_per_launch")
+            rec = json.load(f)
     except Exception:
         return None
+    if rec.get("source_sha256") != _kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
 
 
 def run_reference(a):
@@ -466,7 +494,8 @@ def run_reference(a):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded; Llama-3-8B-shaped layer, no model weights)",
-        "config": {"workload": wl.name, "units_per_step": workers, "context": wl.context[0]},
+        "config": dict(_workload_config(wl, 1, world), units_per_step=workers,
+                       l2="host run: one bounded sample of the workload per step"),
         "cpu_baseline": base,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s": time.perf_counter() - t_start,
