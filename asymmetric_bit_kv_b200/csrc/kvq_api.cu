@@ -27,6 +27,7 @@ struct kvq_cache {
   int64_t lens_off;               // int32 [num_layers][max_batch][2]
   int64_t ws_o_off, ws_ml_off;    // split partials
   int64_t err_off;                // int32 device error word
+  int64_t ctr_off;                // int32 [max_batch][num_kv_heads] decode arrival counters
   int32_t slots;                  // partial slots per (sequence, query head)
   int32_t sm_count;
   std::vector<int32_t> q_len, n_len;  // host mirror [num_layers][max_batch]
@@ -85,7 +86,7 @@ kvq_status validate_config(const kvq_config* c) {
 
 struct Plan {
   std::vector<int64_t> blocks_off, ring_k_off, ring_v_off, record_bytes;
-  int64_t max_blocks, lens_off, err_off, ws_o_off, ws_ml_off, total;
+  int64_t max_blocks, lens_off, err_off, ctr_off, ws_o_off, ws_ml_off, total;
   int32_t slots;
 };
 
@@ -114,11 +115,16 @@ Plan make_plan(const kvq_config* c) {
   off = round_up(off + (int64_t)c->num_layers * c->max_batch * 2 * 4, 256);
   p.err_off = off;
   off = round_up(off + 4, 256);
+  p.ctr_off = off;
+  off = round_up(off + seqheads * 4, 256);
   // partial slots per (sequence, query head): enough for the split kernel
-  // (one per split + the ring) and for the persistent kernel (4 for the ring,
-  // 4 per CTA range overlapping the sequence, at most 64 such ranges)
-  p.slots = (int32_t)std::max<int64_t>(std::min<int64_t>(p.max_blocks, KVQ_MAX_SPLITS) + 1,
-                                       4 + 4 * (std::min<int64_t>(p.max_blocks, 64) + 1));
+  // (one per split + the ring) and for the persistent kernel (one per
+  // consumer warp of each CTA range overlapping the unit's work items, at
+  // most 65 such ranges)
+  p.slots = (int32_t)std::max<int64_t>(
+      std::min<int64_t>(p.max_blocks, KVQ_MAX_SPLITS) + 1,
+      kvq::kMmaConsumers *
+          (std::min<int64_t>(p.max_blocks + (c->residual + kvq::kResChunk - 1) / kvq::kResChunk, 64) + 1));
   const int64_t partials = (int64_t)c->max_batch * c->num_q_heads * p.slots;
   p.ws_o_off = off;
   off = round_up(off + partials * D * 4, 256);
@@ -254,8 +260,8 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out,
   kvq::MmaPlan mp{};
   int per_sm = 4;
   if (use_mma) {
-    mp = kvq::make_mma_plan(L);
-    per_sm = kvq::mma_ctas_per_sm(L, mp);
+    mp = kvq::make_mma_plan(L, cfg.num_q_heads);
+    per_sm = kvq::mma_ctas_per_sm(L, mp, cfg.num_q_heads);
   }
   std::vector<int> nblk(batch);
   int max_blk = 0;
@@ -281,39 +287,49 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out,
   p.num_q_heads = cfg.num_q_heads;
   p.slots = c->slots;
   p.err = reinterpret_cast<int32_t*>(c->arena + c->err_off);
+  p.unit_ctr = reinterpret_cast<int32_t*>(c->arena + c->ctr_off);
   cudaError_t e;
   int32_t used_slots = c->slots;  // partial slots per (sequence, query head) this call writes
   if (use_mma) {
-    // Persistent plan: one CTA per resident slot (fewer if there is little
-    // work), each taking a contiguous range of the concatenated blocks.
+    // Persistent plan: the work items of every (sequence, KV head) unit
+    // (quantized blocks, then ring chunks), concatenated and cut into one
+    // contiguous range per CTA, one CTA per resident slot (fewer if there is
+    // little work).
+    int64_t total = 0;
+    for (int b = 0; b < batch; ++b) {
+      const int nres = c->n_len[(size_t)layer * cfg.max_batch + b];
+      p.nblk[b] = nblk[b];
+      p.nres[b] = nres;
+      p.nitem[b] = kvq::unit_items(nblk[b], nres);
+      p.seq_start[b] = (int32_t)total;
+      total += (int64_t)p.nitem[b] * cfg.num_kv_heads;
+    }
+    if (total > INT32_MAX) {
+      delete pp;
+      return fail(KVQ_ERR_UNSUPPORTED, "more than 2^31 work items in one call");
+    }
     int64_t nctas = std::min<int64_t>((int64_t)std::max(1, c->sm_count) * per_sm,
-                                      std::max<int64_t>((int64_t)batch * cfg.num_kv_heads, (total_blocks + 3) / 4));
+                                      std::max<int64_t>((int64_t)batch * cfg.num_kv_heads, (total + 3) / 4));
     nctas = std::max<int64_t>(nctas, 1);
     // every (sequence, head) must fit its partials in the workspace
-    int64_t acc = 0;
-    for (int b = 0; b < batch; ++b) {
-      p.nblk[b] = nblk[b];
-      p.seq_start[b] = (int32_t)acc;
-      acc += (int64_t)nblk[b] * cfg.num_kv_heads;
-    }
     for (;;) {
-      int32_t need = kvq::kResidualSlots;
-      for (int b = 0; b < batch && total_blocks > 0; ++b)
+      int32_t need = 1;
+      for (int b = 0; b < batch; ++b)
         for (int h = 0; h < cfg.num_kv_heads; ++h)
-          need = std::max(need, kvq::persistent_slots(total_blocks, (int32_t)nctas, p.seq_start[b] + h * nblk[b], nblk[b]));
+          need = std::max(need, kvq::persistent_slots(total, (int32_t)nctas, p.seq_start[b] + h * p.nitem[b],
+                                                      p.nitem[b]));
       used_slots = need;
       if (need <= c->slots || nctas == 1) break;
       nctas = std::max<int64_t>(1, nctas * 3 / 4);
     }
     p.persistent = 1;
-    p.total_blocks = (int32_t)total_blocks;
+    p.total_blocks = (int32_t)total;
     p.num_ctas = (int32_t)nctas;
     if (scratch && !use_scratch(p, *scratch, batch, used_slots, &s)) {
       delete pp;
       return s;
     }
-    e = kvq::launch_decode_mma(p, mp, 0, static_cast<cudaStream_t>(stream));
-    if (e == cudaSuccess) e = kvq::launch_combine(p, static_cast<cudaStream_t>(stream));
+    e = kvq::launch_decode_mma(p, mp, static_cast<cudaStream_t>(stream));
   } else {
     // Split plan: blocks per split chosen to minimise (waves of CTAs) x
     // (blocks per CTA + a fixed per-CTA overhead), with at most slots-1 splits.
@@ -404,6 +420,7 @@ kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena
   c->ws_o_off = plan.ws_o_off;
   c->ws_ml_off = plan.ws_ml_off;
   c->err_off = plan.err_off;
+  c->ctr_off = plan.ctr_off;
   c->slots = plan.slots;
   c->q_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
   c->n_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
@@ -411,6 +428,15 @@ kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device);
   if (e == cudaSuccess) e = cudaMemset(c->arena + c->lens_off, 0, (size_t)cfg->num_layers * cfg->max_batch * 8);
   if (e == cudaSuccess) e = cudaMemset(c->arena + c->err_off, 0, 4);
+  if (e == cudaSuccess) e = cudaMemset(c->arena + c->ctr_off, 0, (size_t)cfg->max_batch * cfg->num_kv_heads * 4);
+  // Ring slots that no token has reached yet hold zeros, never stale bit
+  // patterns: the decode kernel reads whole 16-slot groups of the ring and
+  // masks the scores of slots past the sequence, so their values must be finite.
+  const size_t ring_bytes = (size_t)cfg->max_batch * cfg->num_kv_heads * cfg->residual * cfg->head_dim * 2;
+  for (int l = 0; l < cfg->num_layers && e == cudaSuccess; ++l) {
+    e = cudaMemset(c->arena + c->ring_k_off[l], 0, ring_bytes);
+    if (e == cudaSuccess) e = cudaMemset(c->arena + c->ring_v_off[l], 0, ring_bytes);
+  }
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     delete c;
@@ -432,6 +458,9 @@ kvq_status kvq_cache_reset(kvq_cache* c, void* stream) {
   if (!c) return fail(KVQ_ERR_INVALID_ARG, "cache is null");
   cudaError_t e = cudaMemsetAsync(c->arena + c->lens_off, 0, (size_t)c->cfg.num_layers * c->cfg.max_batch * 8,
                                   static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(c->arena + c->ctr_off, 0, (size_t)c->cfg.max_batch * c->cfg.num_kv_heads * 4,
+                        static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "reset");
   std::fill(c->q_len.begin(), c->q_len.end(), 0);
   std::fill(c->n_len.begin(), c->n_len.end(), 0);
@@ -505,6 +534,9 @@ kvq_status kvq_device_errors(kvq_cache* c, int32_t* flags) {
   int32_t v = 0;
   cudaError_t e = cudaMemcpy(&v, c->arena + c->err_off, 4, cudaMemcpyDeviceToHost);
   if (e == cudaSuccess && v != 0) e = cudaMemset(c->arena + c->err_off, 0, 4);
+  // a decode that gave up may have left arrival counters behind: clear them
+  if (e == cudaSuccess && v != 0)
+    e = cudaMemset(c->arena + c->ctr_off, 0, (size_t)c->cfg.max_batch * c->cfg.num_kv_heads * 4);
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
   *flags = v;
   return KVQ_OK;

@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeParams p) {
   int S;  // slots 0..S hold this (sequence, head)'s partials
   if (p.persistent) {
     const int h = hq / (p.num_q_heads / L.num_kv_heads);
-    S = persistent_slots(p.total_blocks, p.num_ctas, p.seq_start[b] + h * p.nblk[b], p.nblk[b]) - 1;
+    S = persistent_slots(p.total_blocks, p.num_ctas, p.seq_start[b] + h * p.nitem[b], p.nitem[b]) - 1;
   } else {
     const int nblk = L.lens[2 * b] / L.group_k;
     S = (nblk + p.blocks_per_split - 1) / p.blocks_per_split;

@@ -10,12 +10,16 @@ namespace kvq {
 //  * split mode (CUDA-core kernel): slot 0 is the residual ring; slot s >= 1
 //    covers quantized blocks [(s-1)*blocks_per_split, min(s*blocks_per_split,
 //    nblk));
-//  * persistent mode (tensor-core kernel): the quantized blocks of all
-//    (sequence, KV head) units, concatenated in (sequence, head, block) order,
-//    are cut into num_ctas contiguous ranges (CTA c takes
-//    [c*T/num_ctas, (c+1)*T/num_ctas)); slot 0 holds the residual ring,
-//    slot 1 + 4*(c - c0) + w the blocks that warp w of CTA c processed for
-//    the unit, c0 being the unit's first CTA.
+//  * persistent mode (tensor-core kernel): the work of a (sequence, KV head)
+//    unit is its quantized blocks followed by its ring tokens in chunks of
+//    kResChunk (one chunk even for an empty sequence); the work items of all
+//    units, concatenated in (sequence, head, item) order, are cut into
+//    num_ctas contiguous ranges (CTA c takes [c*T/num_ctas, (c+1)*T/num_ctas)),
+//    and slot kMmaConsumers*(c - c0) + w holds what consumer warp w of CTA c
+//    processed for the unit, c0 being the unit's first CTA. Every writer of a
+//    slot then counts itself in unit_ctr; the warp that writes a unit's last
+//    slot merges all of them (log-sum-exp) into the output and resets the
+//    counter to 0, so no separate combine launch is needed.
 struct DecodeParams {
   LayerView L;
   const void* q;        // [batch][Hq][D], kv dtype
@@ -29,14 +33,24 @@ struct DecodeParams {
   int32_t blocks_per_split;
   int32_t slots;        // partial slots per (sequence, query head)
   int32_t* err;         // device word: a kernel sets bit 0 when a bounded wait gave up
+  int32_t* unit_ctr;    // persistent mode: [batch][Hkv] partials written so far this call (0 between calls)
   int32_t persistent;   // 1: persistent-mode slots (see above)
-  int32_t total_blocks; // T, persistent mode
+  int32_t total_blocks; // T, persistent mode: work items of all units
   int32_t num_ctas;     // persistent mode
   int32_t nblk[KVQ_MAX_BATCH];       // quantized blocks per sequence (host mirror)
-  int32_t seq_start[KVQ_MAX_BATCH];  // first global block of sequence b: sum_{b'<b} nblk*Hkv
+  int32_t nres[KVQ_MAX_BATCH];       // ring tokens per sequence (host mirror)
+  int32_t nitem[KVQ_MAX_BATCH];      // persistent mode: work items per unit of sequence b
+  int32_t seq_start[KVQ_MAX_BATCH];  // first global item (block in split mode) of sequence b
 };
 
-constexpr int kResidualSlots = 1;  // persistent mode: the residual ring's partial
+constexpr int kMmaConsumers = 6;   // warps per CTA of the tensor-core kernel
+constexpr int kResChunk = 8;       // ring tokens per work item, persistent mode
+
+// Work items of one unit: quantized blocks, then ring chunks (at least one).
+__host__ __device__ inline int32_t unit_items(int32_t nblk, int32_t nres) {
+  const int32_t items = nblk + (nres + kResChunk - 1) / kResChunk;
+  return items > 0 ? items : 1;
+}
 
 // Persistent mode: first global block of CTA c, and the CTA holding block k.
 __host__ __device__ inline int32_t cta_first_block(int64_t T, int32_t nctas, int32_t c) {
@@ -48,38 +62,38 @@ __host__ __device__ inline int32_t cta_of_block(int64_t T, int32_t nctas, int32_
   while (c > 0 && cta_first_block(T, nctas, c) > k) --c;
   return c;
 }
-// Number of partial slots a (sequence, head) unit uses in persistent mode.
-__host__ __device__ inline int32_t persistent_slots(int64_t T, int32_t nctas, int32_t unit_start, int32_t nblk) {
-  if (nblk <= 0) return kResidualSlots;
+// Number of partial slots a (sequence, head) unit of nitem >= 1 work items
+// uses in persistent mode.
+__host__ __device__ inline int32_t persistent_slots(int64_t T, int32_t nctas, int32_t unit_start, int32_t nitem) {
   const int32_t c0 = cta_of_block(T, nctas, unit_start);
-  const int32_t c1 = cta_of_block(T, nctas, unit_start + nblk - 1);
-  return kResidualSlots + 4 * (c1 - c0 + 1);
+  const int32_t c1 = cta_of_block(T, nctas, unit_start + nitem - 1);
+  return kMmaConsumers * (c1 - c0 + 1);
 }
 
-// Shared-memory plan of the tensor-core decode kernel: NS stages, each one
-// block record exactly as stored (its layout is bank-conflict-free for
-// ldmatrix), then one scratch area per consumer warp.
+// Shared-memory plan of the tensor-core decode kernel: per warp nstages
+// stages (a block record exactly as stored, or the key and value rows of a
+// ring chunk), then one scratch area per warp, then the stage barriers.
 struct MmaPlan {
   int32_t tx_bytes;     // bytes of one record copy (kc | ksz | vc | vsz)
   int32_t kc_bytes;     // key codes (then 4*D bytes of key scale/zero)
   int32_t vc_soff;      // value codes
   int32_t vsz_soff;     // value scale/zero
   int32_t stage_bytes;
-  int32_t nstages;
+  int32_t nstages;      // stages per warp
   int32_t ws_soff;      // first consumer-warp scratch
   int32_t ws_bytes;     // bytes per consumer-warp scratch
-  int32_t afrag_off;    // scratch: A fragments (scaled query, fp16 high/low)
+  int32_t bfrag_off;    // scratch: key B fragments (q*s, fp16 high/low)
   int32_t bias_off;     // scratch: per-head sum_d q_d z_d
   int32_t vpair_off;    // scratch: value scale/zero of token pairs (fp16)
-  int32_t wq_off;       // scratch: the unit's scaled queries (fp32)
+  int32_t qbuf_off;     // scratch: the queries of the warp's current units (kv dtype)
   int32_t bar_off;      // offset of the mbarriers
   int32_t smem_bytes;   // dynamic shared memory per CTA
 };
 
 bool mma_supported(const LayerView& L);
-MmaPlan make_mma_plan(const LayerView& L);
-int mma_ctas_per_sm(const LayerView& L, const MmaPlan& mp);
-cudaError_t launch_decode_mma(const DecodeParams& p, const MmaPlan& mp, int max_splits, cudaStream_t stream);
+MmaPlan make_mma_plan(const LayerView& L, int num_q_heads);
+int mma_ctas_per_sm(const LayerView& L, const MmaPlan& mp, int num_q_heads);
+cudaError_t launch_decode_mma(const DecodeParams& p, const MmaPlan& mp, cudaStream_t stream);
 
 // Enqueue the CUDA-core split kernel (any supported shape) and the
 // log-sum-exp combine. max_splits is the largest quantized split count of any

@@ -1,0 +1,848 @@
+// Tensor-core split-KV decode attention over the packed cache (sm_100a):
+// the kernel template, instantiated per (key bits, value bits, value groups
+// per head, key n-tiles) in kvq_decode_tc_k{2,4,8}.cu.
+//
+// Method: decoding over per-channel-quantized keys and per-token-quantized
+// values plus the full-precision residual window ("KIVI" README, Overview;
+// GQA update), with x_hat = q*d + m ("KV1-1.2B" card, BQ2_0).
+//
+// Design (HBM-bound; the tensor cores only take the dot products off the ALUs):
+//  * Persistent CTAs of kNC warps. The work items of all (sequence, KV head)
+//    units -- a unit's quantized block records, then its ring tokens in
+//    chunks of kResChunk -- are concatenated and cut into one contiguous range
+//    per CTA; warp w of a CTA takes items w, w + kNC, ... of its range. Each
+//    warp streams its own items through a private ring of SPW shared-memory
+//    stages: one lane issues one cp.async.bulk (1-D TMA, no multicast) per
+//    record, completing on the stage's mbarrier, and refills a stage as soon
+//    as the warp is done with it, so no warp ever waits on another.
+//  * Quantized keys, tokens on M: S[token][col] = codes x (q*s). ldmatrix
+//    .trans over the channel-major key rows gives each thread two channels
+//    of 16/kb tokens in one register; one lop3 (mask | fp16 exponent 2^(10-p))
+//    and one hsub2 turn the code at bit position p into an exact fp16
+//    integer, the A operand. The B operand is q*s per channel, fp16 high and
+//    low parts in two columns per head (or two n-tiles for 8 heads), rebuilt
+//    per block from the block's fp16 scales.
+//  * Probabilities: after the online softmax (log2 units) each thread holds
+//    P[token][two heads] in the m8n8 fragment layout; movmatrix.trans turns
+//    it into the B operand of P.V (tokens on K, heads on N).
+//  * Values: O[channel][head] = sum_t codes * (p*s) + sum_t p*z: value codes
+//    of two tokens per register from ldmatrix.trans over token rows (channels
+//    on M), the zero-point term one MMA per value group with an all-ones A.
+//  * Ring chunks use bf16 (or f16) m16n8k16 directly on the ring values, with
+//    the query and the probabilities split into high and low parts, into the
+//    same accumulators as the unit's blocks.
+//  * Every warp's partial (o, m, l) of a unit is counted in a per-unit
+//    arrival counter; the warp writing a unit's last partial merges them
+//    (log-sum-exp) into the output. mbarrier waits are bounded (~2 s) and set
+//    the device error word instead of hanging.
+#pragma once
+
+#include "kvq_decode.cuh"
+
+namespace kvq {
+namespace tc {
+
+constexpr int kNC = kMmaConsumers;        // warps per CTA
+constexpr int kThreads = kNC * 32;
+constexpr long long kWaitCycles = 4000000000LL;  // a bounded wait gives up after ~2 s
+constexpr int kRowBytes = kHeadDim * 2;  // one ring row (token, KV head)
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* ptr) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Waits for the phase with the given parity to complete; false after ~2 s.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitCycles) return false;
+  return true;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// ldmatrix keeps a memory clobber so that it stays behind the barrier waits
+// that publish the shared memory it reads; the arithmetic asm is free to move.
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+      : "r"(addr)
+      : "memory");
+}
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Transpose of an m8n8 b16 matrix held in the mma fragment layout.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// (a & b) | c in one instruction.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+  __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ float2 unpack_f16(uint32_t x) {
+  return __half22float2(*reinterpret_cast<__half2*>(&x));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ float2 unpack_bf16(uint32_t x) {
+  return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xffff0000u));
+}
+__device__ __forceinline__ float2 unpack_kv(uint32_t x, bool bf16) { return bf16 ? unpack_bf16(x) : unpack_f16(x); }
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// Code j (width B bits) of both 16-bit halves of a register, as exact fp16
+// integers. x8 = x >> 8 serves codes that sit in the upper byte of a half.
+// The code field at bit position p (0..7) of the low byte becomes the low
+// mantissa bits of 2^(10-p), whose mantissa bit p weighs exactly 1; or-ing
+// the exponent in and subtracting 2^(10-p) leaves the code.
+template <int B>
+__device__ __forceinline__ uint32_t code_at(uint32_t x, uint32_t x8, int j) {
+  const int bit = B * j;
+  const int pos = bit & 7;
+  const uint32_t m = ((1u << B) - 1u) << pos;
+  const uint32_t e = (uint32_t)(25 - pos) << 10;
+  const uint32_t magic = e | (e << 16);
+  return hsub2(and_or(bit >= 8 ? x8 : x, m | (m << 16), magic), magic);
+}
+
+// Compile-time shape of one instance. A tile is 64 tokens of a block.
+template <int KB, int VB, int NGRP, int NKT>
+struct Shape {
+  static constexpr int D = kHeadDim;
+  static constexpr int TT = 64;              // tokens per tile
+  static constexpr int CPT16 = 16 / KB;      // key tokens per 16-bit column
+  static constexpr int TOKC = 128 / KB;      // key tokens per 16-byte chunk of a channel row
+  static constexpr int SIG = TT / TOKC;      // chunks of a channel row per tile
+  static constexpr int JP = CPT16 / 2;       // M-tiles per chunk
+  static constexpr int MT = SIG * JP;        // M-tiles (16 tokens) per tile
+  static constexpr int VRB = D * VB / 8;     // value code bytes per token
+  static constexpr int NCH = VRB / 16;       // 16-byte chunks per value row
+  static constexpr int VCPC = 16 / VB;       // value channels per 16-bit column
+  static constexpr int MT_PER_CH = VCPC / 2; // channel m-tiles per value chunk
+  static constexpr int CH_SPAN = 128 / VB;   // channels per value chunk
+  static constexpr int GV = D / NGRP;        // value group (channels)
+  static_assert(MT == 4, "a 64-token tile is four 16-token M-tiles");
+  static_assert(SIG >= 1, "tile too short for the key code width");
+  static_assert(CH_SPAN <= GV, "a value chunk must lie inside one value group");
+};
+
+// Token (0..63 inside the tile) on row r (0..15) of key M-tile mt: rows 0-7
+// take code 2*jp, rows 8-15 code 2*jp+1 of 16-bit column r%8 of chunk sg.
+template <int KB>
+__device__ __forceinline__ int tile_token(int mt, int r) {
+  constexpr int CPT16 = 16 / KB, TOKC = 128 / KB, JP = CPT16 / 2;
+  return (mt / JP) * TOKC + (r & 7) * CPT16 + 2 * (mt % JP) + (r >> 3);
+}
+
+// The fields of DecodeParams that the out-of-line helpers below need,
+// passed by value: the kernel's parameter block itself (4 KB with the
+// per-sequence tables) must not have its address taken, or it is copied to
+// the stack.
+struct PartialOut {
+  float* ws_o;
+  float2* ws_ml;
+  void* out;
+  int32_t out_dtype;
+  int32_t num_q_heads;
+  int32_t slots;
+  float scale_log2;
+};
+__device__ __forceinline__ PartialOut partial_out(const DecodeParams& p) {
+  return PartialOut{p.ws_o, p.ws_ml, p.out, p.out_dtype, p.num_q_heads, p.slots, p.scale_log2};
+}
+
+// ------------------------------------------------------ fused LSE combine
+// Merges the nslots partials of unit (b, h) into out[b][h*NG + hh][:]:
+// M = max_s m_s, out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s, empty
+// slots (l = 0, o finite) weighted 0, rounded to the output dtype (nearest
+// even). One warp: lane l owns channels 4l..4l+3 of every head (at most
+// kMaxNG); the loads of SB slots of all heads are issued together. Partials
+// written by other SMs are read through L2 (ld.global.cg).
+template <int kMaxNG>
+static __device__ __noinline__ void combine_unit(const PartialOut p, int b, int h, int NG, int nslots, int lane) {
+  constexpr int D = kHeadDim;
+  constexpr int SB = 16 / kMaxNG;
+  const int64_t base = ((int64_t)b * p.num_q_heads + h * NG) * p.slots;  // head hh: + hh * slots
+  float M[kMaxNG], lsum[kMaxNG];
+  float4 acc[kMaxNG];
+#pragma unroll
+  for (int hh = 0; hh < kMaxNG; ++hh) {
+    M[hh] = -INFINITY;
+    lsum[hh] = 0.f;
+    acc[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int s0 = 0; s0 < nslots; s0 += 32) {  // running maxima
+#pragma unroll
+    for (int hh = 0; hh < kMaxNG; ++hh) {
+      if (hh < NG && s0 + lane < nslots) {
+        const float2 ml = __ldcg(p.ws_ml + base + (int64_t)hh * p.slots + s0 + lane);
+        if (ml.y > 0.f) M[hh] = fmaxf(M[hh], ml.x);
+      }
+    }
+  }
+#pragma unroll
+  for (int hh = 0; hh < kMaxNG; ++hh)
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) M[hh] = fmaxf(M[hh], __shfl_xor_sync(0xffffffffu, M[hh], off));
+  for (int s0 = 0; s0 < nslots; s0 += 32) {
+    float w[kMaxNG];  // weight of slot s0 + lane, per head
+#pragma unroll
+    for (int hh = 0; hh < kMaxNG; ++hh) {
+      w[hh] = 0.f;
+      if (hh < NG && s0 + lane < nslots && M[hh] != -INFINITY) {
+        const float2 ml = __ldcg(p.ws_ml + base + (int64_t)hh * p.slots + s0 + lane);
+        if (ml.y > 0.f) {
+          w[hh] = exp2f(ml.x - M[hh]);
+          lsum[hh] += ml.y * w[hh];
+        }
+      }
+    }
+    const int cnt = min(32, nslots - s0);
+    for (int i0 = 0; i0 < cnt; i0 += SB) {
+      float4 o[SB][kMaxNG];
+#pragma unroll
+      for (int e = 0; e < SB; ++e)
+#pragma unroll
+        for (int hh = 0; hh < kMaxNG; ++hh)
+          o[e][hh] = (hh < NG && i0 + e < cnt)
+                         ? __ldcg(reinterpret_cast<const float4*>(p.ws_o + (base + (int64_t)hh * p.slots + s0 + i0 + e) * D) + lane)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int e = 0; e < SB; ++e) {
+#pragma unroll
+        for (int hh = 0; hh < kMaxNG; ++hh) {
+          const float wi = __shfl_sync(0xffffffffu, w[hh], (i0 + e) & 31);
+          acc[hh].x += wi * o[e][hh].x;
+          acc[hh].y += wi * o[e][hh].y;
+          acc[hh].z += wi * o[e][hh].z;
+          acc[hh].w += wi * o[e][hh].w;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int hh = 0; hh < kMaxNG; ++hh) {
+    if (hh >= NG) break;
+    float l = lsum[hh];
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+    float r[4] = {acc[hh].x, acc[hh].y, acc[hh].z, acc[hh].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) r[e] = l > 0.f ? __fdiv_rn(r[e], l) : 0.f;
+    const int64_t o = ((int64_t)b * p.num_q_heads + h * NG + hh) * D + 4 * lane;
+    if (p.out_dtype == KVQ_F32) {
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + o) = make_float4(r[0], r[1], r[2], r[3]);
+    } else if (p.out_dtype == KVQ_BF16) {
+      *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) + o) =
+          make_uint2(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]));
+    } else {
+      *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(p.out) + o) =
+          make_uint2(pack_f16(r[0], r[1]), pack_f16(r[2], r[3]));
+    }
+  }
+}
+
+// After this warp wrote one partial slot of unit (b, h): count it, and if it
+// was the unit's last one, merge the unit and reset its counter.
+template <int kMaxNG>
+__device__ __forceinline__ void arrive_unit(const DecodeParams& p, int b, int h, int NG, int lane) {
+  const LayerView& L = p.L;
+  __threadfence();  // this lane's partial stores before the count
+  __syncwarp();
+  const int u = b * L.num_kv_heads + h;
+  int old = 0;
+  if (lane == 0) old = atomicAdd(p.unit_ctr + u, 1);
+  old = __shfl_sync(0xffffffffu, old, 0);
+  const int nslots = persistent_slots(p.total_blocks, p.num_ctas, p.seq_start[b] + h * p.nitem[b], p.nitem[b]);
+  if (old != nslots - 1) return;
+  __threadfence();  // every other writer's partial is visible from here on
+  combine_unit<kMaxNG>(partial_out(p), b, h, NG, nslots, lane);
+  if (lane == 0) atomicExch(p.unit_ctr + u, 0);
+}
+
+// ------------------------------------------------------- residual ring chunks
+// The ring tokens are exact (kv dtype), so their dot products run on the
+// tensor cores in that dtype (bf16 or f16 m16n8k16), with the scaled query
+// and the probabilities split into high and low parts, which keeps both at
+// about 16 significant bits; the accumulators are the ones the quantized
+// blocks of the unit use.
+template <bool BF16>
+__device__ __forceinline__ void mma_kv(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (BF16) mma_bf16(d, a, b0, b1);
+  else mma_f16(d, a, b0, b1);
+}
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack_kv(float lo, float hi) {
+  if constexpr (BF16) return pack_bf16(lo, hi);
+  else return pack_f16(lo, hi);
+}
+template <bool BF16>
+__device__ __forceinline__ float2 unpack_kv2(uint32_t x) {
+  if constexpr (BF16) return unpack_bf16(x);
+  else return unpack_f16(x);
+}
+
+// --------------------------------------------------------- quantized blocks
+// Walks the (sequence, head) units of consecutive global work items.
+struct UnitCursor {
+  int b = 0, h = 0, start = 0, end = 0;  // current unit and its item range
+  __device__ void seek(const DecodeParams& p, int k) {
+    int lo = 0, hi = p.batch - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.seq_start[mid] <= k) lo = mid;
+      else hi = mid - 1;
+    }
+    b = lo;
+    const int nb = p.nitem[b];
+    h = (k - p.seq_start[b]) / nb;
+    start = p.seq_start[b] + h * nb;
+    end = start + nb;
+  }
+  __device__ void advance(const DecodeParams& p, int k) {
+    if (k >= end || k < start) seek(p, k);
+  }
+};
+
+// Per-consumer-warp scratch (byte offsets in MmaPlan), rebuilt per block
+// from its fp16 scales (prep_block); the unit's queries arrive with the
+// warp's first item of the unit:
+//   bfrag [NKT][8 kk][32 lanes] uint2: key B fragments. Column n of the
+//         n-tile holds q*s of head n%4, fp16 high part (n < 4) or low part
+//         (n >= 4); with 8 heads n-tile 0 holds the high and n-tile 1 the low
+//         parts of heads 0-7. Columns of absent heads stay zero.
+//   bias  [8] float: sum_d q_d z_d per head (log2 units);
+//   vpair [k-step][4 t][groups] uint4: (s, s), (s, s), (z, z), (z, z) fp16
+//         pairs of the value tokens that thread t feeds into a P.V k-step;
+//   qbuf  [nstages][NG][D] kv dtype: the queries of the warp's last units
+//         (one buffer per unit change, round robin), as stored in q.
+template <int KB, int VB, int NGRP, int NKT>
+__device__ __forceinline__ void prep_block(const uint8_t* stage, const MmaPlan& mp, uint8_t* ws, const uint32_t* qw,
+                                           int NG, int G, int lane, float scale_log2, bool bf16) {
+  using S = Shape<KB, VB, NGRP, NKT>;
+  uint32_t* bk = reinterpret_cast<uint32_t*>(ws + mp.bfrag_off);
+  const uint2* ksz2 = reinterpret_cast<const uint2*>(stage + mp.kc_bytes);  // (s, z) of channels 2c, 2c+1
+  float* biasw = reinterpret_cast<float*>(ws + mp.bias_off);
+  const int q = lane & 7, half = q >> 2, tq = q & 3;
+#pragma unroll
+  for (int rep = 0; rep < NKT; ++rep) {  // two passes exactly when there are 8 heads
+    const int hh = (lane >> 3) + 4 * rep;
+    float bp = 0.f;
+    if (hh < NG) {
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const float2 qf = unpack_kv(qw[hh * 64 + 8 * kk + q], bf16);  // channels 16kk + 2q, +1
+        const uint2 sz = ksz2[8 * kk + q];
+        const float2 c0 = unpack_f16(sz.x), c1 = unpack_f16(sz.y);
+        const float q0 = qf.x * scale_log2, q1 = qf.y * scale_log2;
+        const float x0 = q0 * c0.x, x1 = q1 * c1.x;
+        bp += q0 * c0.y + q1 * c1.y;
+        const uint32_t hi = pack_f16(x0, x1);
+        const float2 fh = unpack_f16(hi);
+        const uint32_t lo = pack_f16(x0 - fh.x, x1 - fh.y);
+        if (NKT == 1) {
+          bk[(kk * 32 + hh * 4 + tq) * 2 + half] = hi;
+          bk[(kk * 32 + (hh + 4) * 4 + tq) * 2 + half] = lo;
+        } else {
+          bk[(kk * 32 + hh * 4 + tq) * 2 + half] = hi;
+          bk[((8 + kk) * 32 + hh * 4 + tq) * 2 + half] = lo;
+        }
+      }
+    }
+    bp += __shfl_xor_sync(0xffffffffu, bp, 1);
+    bp += __shfl_xor_sync(0xffffffffu, bp, 2);
+    bp += __shfl_xor_sync(0xffffffffu, bp, 4);
+    if (q == 0 && hh < NG) biasw[hh] = bp;
+  }
+  const uint32_t* vsz = reinterpret_cast<const uint32_t*>(stage + mp.vsz_soff);  // [G][NGRP] (s, z)
+  uint4* vp = reinterpret_cast<uint4*>(ws + mp.vpair_off);
+  const int nvp = (G / 16) * 4 * NGRP;
+  for (int e = lane; e < nvp; e += 32) {
+    const int gg = e % NGRP, tv = (e / NGRP) & 3, kst = e / (NGRP * 4);
+    const int tb = (kst / S::MT) * S::TT, mt = kst % S::MT;
+    const uint32_t a = vsz[(tb + tile_token<KB>(mt, 2 * tv)) * NGRP + gg];
+    const uint32_t b = vsz[(tb + tile_token<KB>(mt, 2 * tv + 1)) * NGRP + gg];
+    const uint32_t c = vsz[(tb + tile_token<KB>(mt, 8 + 2 * tv)) * NGRP + gg];
+    const uint32_t d = vsz[(tb + tile_token<KB>(mt, 9 + 2 * tv)) * NGRP + gg];
+    vp[e] = make_uint4(__byte_perm(a, b, 0x5410), __byte_perm(c, d, 0x5410), __byte_perm(a, b, 0x7632),
+                       __byte_perm(c, d, 0x7632));
+  }
+  __syncwarp();
+}
+
+
+// Online-softmax update (log2 units) of this lane's two heads (2t and 2t+1)
+// with the scores sc of MTN M-tiles (registers 0/2: head 2t, rows g and g+8;
+// 1/3: head 2t+1; -inf where a token is absent). sc becomes the
+// probabilities; O and Z are rescaled when a running maximum grows.
+struct SoftState {
+  float m0, m1, l0, l1;
+};
+template <int MTN, int NGRP>
+__device__ __forceinline__ void softmax_update(float (&sc)[MTN][4], SoftState& st, bool v0, bool v1,
+                                               float (&O)[8][4], float (&Z)[NGRP][4]) {
+  float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+  for (int mt = 0; mt < MTN; ++mt) {
+    mx0 = fmaxf(mx0, fmaxf(sc[mt][0], sc[mt][2]));
+    mx1 = fmaxf(mx1, fmaxf(sc[mt][1], sc[mt][3]));
+  }
+#pragma unroll
+  for (int off = 4; off <= 16; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+  }
+  // a head with no finite score so far keeps m = -inf, alpha = 1, p = 0
+  const float n0 = v0 ? fmaxf(st.m0, mx0) : -INFINITY, n1 = v1 ? fmaxf(st.m1, mx1) : -INFINITY;
+  const float a0 = n0 == -INFINITY ? 1.f : ex2(st.m0 - n0), a1 = n1 == -INFINITY ? 1.f : ex2(st.m1 - n1);
+  st.m0 = n0;
+  st.m1 = n1;
+  float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+  for (int mt = 0; mt < MTN; ++mt) {
+    sc[mt][0] = n0 == -INFINITY ? 0.f : ex2(sc[mt][0] - n0);
+    sc[mt][2] = n0 == -INFINITY ? 0.f : ex2(sc[mt][2] - n0);
+    sc[mt][1] = n1 == -INFINITY ? 0.f : ex2(sc[mt][1] - n1);
+    sc[mt][3] = n1 == -INFINITY ? 0.f : ex2(sc[mt][3] - n1);
+    ps0 += sc[mt][0] + sc[mt][2];
+    ps1 += sc[mt][1] + sc[mt][3];
+  }
+  st.l0 = st.l0 * a0 + ps0;
+  st.l1 = st.l1 * a1 + ps1;
+  if (!__all_sync(0xffffffffu, a0 == 1.f && a1 == 1.f)) {
+#pragma unroll
+    for (int gg = 0; gg < NGRP; ++gg) {
+      Z[gg][0] *= a0;
+      Z[gg][1] *= a1;
+      Z[gg][2] *= a0;
+      Z[gg][3] *= a1;
+    }
+#pragma unroll
+    for (int i2 = 0; i2 < 8; ++i2) {
+      O[i2][0] *= a0;
+      O[i2][1] *= a1;
+      O[i2][2] *= a0;
+      O[i2][3] *= a1;
+    }
+  }
+}
+
+// Key scores of M-tile accumulators: high + low columns (or n-tiles) summed.
+template <int NKT>
+__device__ __forceinline__ float head_score(const float (&d)[NKT][4], int e) {
+  float x = d[0][e];
+  if constexpr (NKT == 2) x += d[1][e];
+  else x += __shfl_xor_sync(0xffffffffu, x, 2);
+  return x;
+}
+
+// One chunk of ring tokens (cnt of its kResChunk rows present, cnt <= 0
+// for the placeholder chunk of an empty sequence): stage = key rows
+// [kResChunk][D] then value rows, in the kv dtype; accumulated into the
+// unit's state like a quantized block. Keys, tokens on M: lane (g, t) holds
+// token g's words 2(kk%2) and 2(kk%2)+1 of 16-byte chunk t + 4(kk/2) for
+// k-step kk (rows 8-15 absent); the B operand is the scaled query split
+// into kv-dtype high and low parts in the same channel order, written over
+// the warp's key B fragments (bk, same layout) on its first chunk of the unit
+// (a unit's ring chunks come after all of its quantized blocks). P.V: after movmatrix, lane (g, t) holds the
+// probabilities of tokens 2t, 2t+1 for head g; each output m-tile takes the
+// value word of its channels (ch0, ch0+1) from both tokens, paired by one
+// byte permute; two MMAs (probability high and low parts).
+template <bool BF16, int VB, int NGRP, int NKT>
+__device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t* qw, uint2* bk, int cnt, int NG,
+                                           int lane, float scale_log2, bool v0, bool v1, bool& rq_ready,
+                                           SoftState& sst, float (&O)[8][4], float (&Z)[NGRP][4]) {
+  using S = Shape<2, VB, NGRP, NKT>;  // value-side constants only
+  const int g = lane >> 2, t = lane & 3;
+  if (!rq_ready) {
+    // column g: head g%4, high (g < 4) or low part; with two n-tiles, head g
+    const int head = NKT == 2 ? g : (g & 3);
+    const bool present = head < NG;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      uint32_t hi[2], lo[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int w = 4 * t + 16 * (kk >> 1) + 2 * (kk & 1) + e;  // channels 2w, 2w+1
+        const uint32_t raw = present ? qw[head * 64 + w] : 0u;
+        const float2 f = unpack_kv2<BF16>(raw);
+        const float x0 = f.x * scale_log2, x1 = f.y * scale_log2;
+        hi[e] = pack_kv<BF16>(x0, x1);
+        const float2 fh = unpack_kv2<BF16>(hi[e]);
+        lo[e] = pack_kv<BF16>(x0 - fh.x, x1 - fh.y);
+      }
+      if constexpr (NKT == 1) {
+        bk[kk * 32 + lane] = (g < 4) ? make_uint2(hi[0], hi[1]) : make_uint2(lo[0], lo[1]);
+      } else {
+        bk[kk * 32 + lane] = make_uint2(hi[0], hi[1]);
+        bk[(8 + kk) * 32 + lane] = make_uint2(lo[0], lo[1]);
+      }
+    }
+    __syncwarp();
+    rq_ready = true;
+  }
+  const uint4* K4 = reinterpret_cast<const uint4*>(stage);
+  float Dr[NKT][4];
+#pragma unroll
+  for (int nt = 0; nt < NKT; ++nt) Dr[nt][0] = Dr[nt][1] = Dr[nt][2] = Dr[nt][3] = 0.f;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const uint4 kv = K4[g * 16 + t + 4 * m];
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const uint32_t a[4] = {word_of(kv, 2 * hf), 0u, word_of(kv, 2 * hf + 1), 0u};
+#pragma unroll
+      for (int nt = 0; nt < NKT; ++nt) {
+        const uint2 bq = bk[(nt * 8 + 2 * m + hf) * 32 + lane];
+        mma_kv<BF16>(Dr[nt], a, bq.x, bq.y);
+      }
+    }
+  }
+  float sc[1][4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float x = head_score<NKT>(Dr, e);
+    sc[0][e] = (e < 2 && g < cnt) ? x : -INFINITY;
+  }
+  softmax_update<1, NGRP>(sc, sst, v0, v1, O, Z);
+  const uint32_t ph = pack_kv<BF16>(sc[0][0], sc[0][1]);
+  const float2 fh = unpack_kv2<BF16>(ph);
+  const uint32_t bh = movmatrix_t(ph), bl = movmatrix_t(pack_kv<BF16>(sc[0][0] - fh.x, sc[0][1] - fh.y));
+  const uint32_t* V32 = reinterpret_cast<const uint32_t*>(stage + kResChunk * kRowBytes);  // [rows][64 words]
+#pragma unroll
+  for (int mt2 = 0; mt2 < 8; ++mt2) {
+    const int cch = mt2 / S::MT_PER_CH, P = mt2 % S::MT_PER_CH;
+    const int w = (cch * S::CH_SPAN + g * S::VCPC) / 2 + P;
+    const uint32_t x = V32[(2 * t) * 64 + w], y = V32[(2 * t + 1) * 64 + w];
+    const uint32_t a[4] = {__byte_perm(x, y, 0x5410), __byte_perm(x, y, 0x7632), 0u, 0u};
+    mma_kv<BF16>(O[mt2], a, bh, 0u);
+    mma_kv<BF16>(O[mt2], a, bl, 0u);
+  }
+}
+
+// Issue side of a warp's item stream (one lane): the unit of the last issued
+// item and the number of unit changes so far.
+struct IssueState {
+  UnitCursor u;
+  int unit = -1, seq = -1;
+};
+
+// Issues the copy of work item k (a block record, or the key and value rows
+// of a ring chunk) into stage `dst`, completing on `bar`; on the first item
+// of a unit also the unit's queries, into query buffer seq % nstages.
+__device__ __forceinline__ void issue_item(const DecodeParams& p, const MmaPlan& mp, IssueState& is, int k,
+                                           uint8_t* dst, uint64_t* bar, uint8_t* qbuf, int NG) {
+  const LayerView& L = p.L;
+  UnitCursor& u = is.u;
+  u.advance(p, k);
+  const int j = k - u.start, nb = p.nblk[u.b];
+  const int unit = u.b * L.num_kv_heads + u.h;
+  const bool newq = unit != is.unit;
+  const uint32_t qbytes = NG * kRowBytes;
+  if (newq) {
+    is.unit = unit;
+    ++is.seq;
+  }
+  if (j < nb) {
+    mbar_expect_tx(bar, mp.tx_bytes + (newq ? qbytes : 0u));
+    bulk_g2s(dst, record_ptr(L, u.b, u.h, j), mp.tx_bytes, bar);
+  } else {
+    // ring chunk: kResChunk consecutive slots of keys, then of values
+    const int slot = (nb * L.group_k + (j - nb) * kResChunk) % L.residual;
+    const int64_t row = ((int64_t)u.b * L.num_kv_heads + u.h) * L.residual + slot;
+    constexpr uint32_t bytes = kResChunk * kRowBytes;
+    mbar_expect_tx(bar, 2 * bytes + (newq ? qbytes : 0u));
+    bulk_g2s(dst, reinterpret_cast<const uint8_t*>(L.ring_k) + row * kRowBytes, bytes, bar);
+    bulk_g2s(dst + bytes, reinterpret_cast<const uint8_t*>(L.ring_v) + row * kRowBytes, bytes, bar);
+  }
+  if (newq)
+    bulk_g2s(qbuf + (size_t)(is.seq % mp.nstages) * qbytes,
+             reinterpret_cast<const uint8_t*>(p.q) + ((int64_t)u.b * p.num_q_heads + u.h * NG) * kRowBytes, qbytes,
+             bar);
+}
+
+template <int KB, int VB, int NGRP, int NKT>
+__global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, MmaPlan mp) {
+  using S = Shape<KB, VB, NGRP, NKT>;
+  constexpr int D = S::D;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int c = blockIdx.x;
+  const LayerView& L = p.L;
+  const int Hkv = L.num_kv_heads;
+  const int NG = p.num_q_heads / Hkv;
+  const int G = L.group_k;
+  const int T = p.total_blocks;
+  const int rs = cta_first_block(T, p.num_ctas, c), re = cta_first_block(T, p.num_ctas, c + 1);
+  const bool bf16 = L.kv_dtype == KVQ_BF16;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // this warp's items: rs + warp + n*kNC, n = 0, 1, ...; item n lands in the
+  // warp's own stage n % SPW, and the warp issues item n + SPW as soon as it
+  // is done with item n
+  const int SPW = mp.nstages;  // stages per warp
+  uint8_t* stages = smem + (size_t)warp * SPW * mp.stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + mp.bar_off) + warp * SPW;
+  uint8_t* ws = smem + mp.ws_soff + warp * mp.ws_bytes;
+  const int nmine = rs + warp < re ? (re - rs - warp + kNC - 1) / kNC : 0;
+  uint8_t* qbuf = ws + mp.qbuf_off;
+  IssueState is;  // issue side (lane 0)
+  if (lane == 0) {
+    for (int i = 0; i < SPW; ++i) mbar_init(full + i, 1);
+    fence_mbar_init();
+    for (int n = 0; n < SPW && n < nmine; ++n)
+      issue_item(p, mp, is, rs + warp + n * kNC, stages + (size_t)n * mp.stage_bytes, full + n, qbuf, NG);
+  }
+  __syncwarp();
+  bool failed = false;
+  int n = 0;  // items of this warp consumed so far
+  {
+    {  // key B-fragment columns of absent heads stay zero
+      uint4* z = reinterpret_cast<uint4*>(ws + mp.bfrag_off);
+      for (int e = lane; e < NKT * 8 * 32 * 8 / 16; e += 32) z[e] = make_uint4(0u, 0u, 0u, 0u);
+      __syncwarp();
+    }
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t ones[4] = {0x3c003c00u, 0x3c003c00u, 0x3c003c00u, 0x3c003c00u};  // fp16 1.0
+    const int kc_row = G * KB / 8;  // key code bytes per channel
+    const int mi = lane >> 3, rr = lane & 7;
+    // ldmatrix rows of this lane: 8 consecutive rows, so the chunk swizzle of
+    // the record layout depends on the lane's row index only
+    const int swk = chunk_swizzle(rr, kc_row / 16);
+    const int swv = chunk_swizzle(rr, S::VRB / 16);
+    const uint2* bkr = reinterpret_cast<const uint2*>(ws + mp.bfrag_off);
+    uint2* bkw = reinterpret_cast<uint2*>(ws + mp.bfrag_off);
+    const uint4* vpr = reinterpret_cast<const uint4*>(ws + mp.vpair_off);
+    const float* biasr = reinterpret_cast<const float*>(ws + mp.bias_off);
+    int qseq = -1;  // unit changes seen by the consumer side (matches IssueState::seq)
+    const bool v0 = 2 * t < NG, v1 = 2 * t + 1 < NG;  // heads 2t, 2t+1 of this lane exist
+    UnitCursor u;
+    int k = rs;
+    while (k < re && !failed) {
+      u.advance(p, k);
+      const int hi = min(u.end, re);
+      const int nb = p.nblk[u.b];
+      SoftState sst{-INFINITY, -INFINITY, 0.f, 0.f};
+      float O[8][4], Z[NGRP][4];
+#pragma unroll
+      for (int i2 = 0; i2 < 8; ++i2) O[i2][0] = O[i2][1] = O[i2][2] = O[i2][3] = 0.f;
+#pragma unroll
+      for (int gg = 0; gg < NGRP; ++gg) Z[gg][0] = Z[gg][1] = Z[gg][2] = Z[gg][3] = 0.f;
+      bool rq_ready = false;  // the key B fragments hold the ring-chunk query (not a block's q*s)
+      // this warp's items of the unit: k' - rs = warp (mod kNC)
+      const int first = k + ((warp - (k - rs)) % kNC + kNC) % kNC;
+      for (int kb = first; kb < hi; kb += kNC, ++n) {
+        const int st = n % SPW;
+        if (!mbar_wait(full + st, (n / SPW) & 1)) {
+          failed = true;
+          break;
+        }
+        const uint8_t* stage = stages + (size_t)st * mp.stage_bytes;
+        if (kb == first) ++qseq;  // the warp's first item of the unit brought its queries
+        const uint32_t* qw = reinterpret_cast<const uint32_t*>(qbuf + (size_t)(qseq % SPW) * NG * kRowBytes);
+        const int j = kb - u.start;
+        if (j < nb) {
+          // ============ quantized block
+          prep_block<KB, VB, NGRP, NKT>(stage, mp, ws, qw, NG, G, lane, p.scale_log2, bf16);
+          const float bias0 = biasr[2 * t], bias1 = biasr[2 * t + 1];
+          const uint32_t kc_s = smem_u32(stage);
+          const uint32_t vc_s = smem_u32(stage + mp.vc_soff);
+          for (int tile = 0; tile < G / S::TT; ++tile) {
+            // ---- scores: Dk[M-tile][n-tile] = codes x (q*s)
+            float Dk[S::MT][NKT][4];
+#pragma unroll
+            for (int mt = 0; mt < S::MT; ++mt)
+#pragma unroll
+              for (int nt = 0; nt < NKT; ++nt) Dk[mt][nt][0] = Dk[mt][nt][1] = Dk[mt][nt][2] = Dk[mt][nt][3] = 0.f;
+#pragma unroll
+            for (int kp = 0; kp < 4; ++kp) {
+              uint2 bfr[2][NKT];
+#pragma unroll
+              for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                for (int nt = 0; nt < NKT; ++nt) bfr[hf][nt] = bkr[(nt * 8 + 2 * kp + hf) * 32 + lane];
+              const int ch = 16 * (2 * kp + (mi >> 1)) + 8 * (mi & 1) + rr;
+#pragma unroll
+              for (int sg = 0; sg < S::SIG; ++sg) {
+                uint32_t rk[4];
+                ldsm_x4_t(kc_s + ch * kc_row + (((tile * S::SIG + sg) ^ swk) << 4), rk[0], rk[1], rk[2], rk[3]);
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                  const uint32_t xl = rk[2 * hf], xh = rk[2 * hf + 1], xl8 = xl >> 8, xh8 = xh >> 8;
+#pragma unroll
+                  for (int jp = 0; jp < S::JP; ++jp) {
+                    const uint32_t a[4] = {code_at<KB>(xl, xl8, 2 * jp), code_at<KB>(xl, xl8, 2 * jp + 1),
+                                           code_at<KB>(xh, xh8, 2 * jp), code_at<KB>(xh, xh8, 2 * jp + 1)};
+#pragma unroll
+                    for (int nt = 0; nt < NKT; ++nt)
+                      mma_f16(Dk[sg * S::JP + jp][nt], a, bfr[hf][nt].x, bfr[hf][nt].y);
+                  }
+                }
+              }
+            }
+            // ---- online softmax over the tile
+            float sc[S::MT][4];
+#pragma unroll
+            for (int mt = 0; mt < S::MT; ++mt)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) sc[mt][e] = head_score<NKT>(Dk[mt], e) + ((e & 1) ? bias1 : bias0);
+            softmax_update<S::MT, NGRP>(sc, sst, v0, v1, O, Z);
+            // ---- values: O += codes x (p * s), Z += ones x (p * z)
+#pragma unroll
+            for (int mt = 0; mt < S::MT; ++mt) {
+              // P^T of the M-tile: tokens rows 2t, 2t+1 (bt) and 8+2t, 9+2t (bb), head g
+              const uint32_t bt = movmatrix_t(pack_f16(sc[mt][0], sc[mt][1]));
+              const uint32_t bb = movmatrix_t(pack_f16(sc[mt][2], sc[mt][3]));
+              const int kst = tile * S::MT + mt;
+              uint32_t B0[NGRP], B1[NGRP];
+#pragma unroll
+              for (int gg = 0; gg < NGRP; ++gg) {
+                const uint4 v4 = vpr[(kst * 4 + t) * NGRP + gg];
+                B0[gg] = hmul2(bt, v4.x);
+                B1[gg] = hmul2(bb, v4.y);
+                mma_f16(Z[gg], ones, hmul2(bt, v4.z), hmul2(bb, v4.w));
+              }
+              const int sg = mt / S::JP, jp = mt % S::JP;
+              const int vrow_idx = (2 * jp + (mi & 1)) * (G / S::CPT16) + tile * (S::TT / S::CPT16) + sg * 8 + rr;
+              const uint32_t vrow = vc_s + vrow_idx * S::VRB;
+#pragma unroll
+              for (int cc0 = 0; cc0 < S::NCH; cc0 += 2) {
+                uint32_t r[4];
+                ldsm_x4_t(vrow + (((cc0 + (mi >> 1)) ^ swv) << 4), r[0], r[1], r[2], r[3]);
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                  const uint32_t xv = r[2 * cc], yv = r[2 * cc + 1], xv8 = xv >> 8, yv8 = yv >> 8;
+                  const int gg = ((cc0 + cc) * S::CH_SPAN) / S::GV;
+#pragma unroll
+                  for (int P = 0; P < S::MT_PER_CH; ++P) {
+                    const uint32_t a[4] = {code_at<VB>(xv, xv8, 2 * P), code_at<VB>(xv, xv8, 2 * P + 1),
+                                           code_at<VB>(yv, yv8, 2 * P), code_at<VB>(yv, yv8, 2 * P + 1)};
+                    mma_f16(O[(cc0 + cc) * S::MT_PER_CH + P], a, B0[gg], B1[gg]);
+                  }
+                }
+              }
+            }
+          }
+        } else if (bf16) {
+          ring_chunk<true, VB, NGRP, NKT>(stage, qw, bkw, p.nres[u.b] - (j - nb) * kResChunk, NG, lane,
+                                         p.scale_log2, v0, v1, rq_ready, sst, O, Z);
+        } else {
+          ring_chunk<false, VB, NGRP, NKT>(stage, qw, bkw, p.nres[u.b] - (j - nb) * kResChunk, NG, lane,
+                                          p.scale_log2, v0, v1, rq_ready, sst, O, Z);
+        }
+        // every lane is done with the stage: refill it with item n + SPW
+        __syncwarp();
+        if (lane == 0 && n + SPW < nmine) {
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          issue_item(p, mp, is, rs + warp + (n + SPW) * kNC, stages + (size_t)st * mp.stage_bytes, full + st, qbuf, NG);
+        }
+      }
+      if (failed) break;
+      // ---------------- this warp's partial for the unit
+#pragma unroll
+      for (int off = 4; off <= 16; off <<= 1) {
+        sst.l0 += __shfl_xor_sync(0xffffffffu, sst.l0, off);
+        sst.l1 += __shfl_xor_sync(0xffffffffu, sst.l1, off);
+      }
+      const int slot = kNC * (c - cta_of_block(T, p.num_ctas, u.start)) + warp;
+      const int64_t base0 = ((int64_t)u.b * p.num_q_heads + u.h * NG + 2 * t) * p.slots + slot;
+      const int64_t base1 = base0 + p.slots;
+#pragma unroll
+      for (int mt2 = 0; mt2 < 8; ++mt2) {
+        const int cch = mt2 / S::MT_PER_CH, P = mt2 % S::MT_PER_CH;
+        const int gg = (cch * S::CH_SPAN) / S::GV;
+        const int ch0 = cch * S::CH_SPAN + g * S::VCPC + 2 * P;
+        if (v0)
+          *reinterpret_cast<float2*>(p.ws_o + base0 * D + ch0) = make_float2(O[mt2][0] + Z[gg][0], O[mt2][2] + Z[gg][0]);
+        if (v1)
+          *reinterpret_cast<float2*>(p.ws_o + base1 * D + ch0) = make_float2(O[mt2][1] + Z[gg][1], O[mt2][3] + Z[gg][1]);
+      }
+      if (g == 0) {
+        if (v0) p.ws_ml[base0] = make_float2(sst.m0, sst.l0);
+        if (v1) p.ws_ml[base1] = make_float2(sst.m1, sst.l1);
+      }
+      arrive_unit<4 * NKT>(p, u.b, u.h, NG, lane);
+      k = hi;
+    }
+  }
+  if (failed) {
+    // let the copies still in flight land before the CTA may leave
+    if (lane == 0)
+      for (int i = n; i < n + SPW && i < nmine; ++i) (void)mbar_wait(full + i % SPW, (i / SPW) & 1);
+    if (lane == 0) atomicOr(p.err, 1);
+  }
+}
+
+// Enqueues one instance. Its dynamic shared-memory size was opted in on this
+// device by mma_ctas_per_sm, which the host calls before every launch.
+template <int KB, int VB, int NGRP, int NKT>
+cudaError_t launch_instance(const DecodeParams& p, const MmaPlan& mp, cudaStream_t stream) {
+  decode_tc_kernel<KB, VB, NGRP, NKT><<<p.num_ctas, kThreads, mp.smem_bytes, stream>>>(p, mp);
+  return cudaGetLastError();
+}
+
+template <int KB, int VB, int NGRP, int NKT>
+const void* instance_fn() {
+  return reinterpret_cast<const void*>(decode_tc_kernel<KB, VB, NGRP, NKT>);
+}
+
+}  // namespace tc
+}  // namespace kvq

@@ -1,0 +1,4 @@
+// decode_tc_kernel instances with 4-bit keys and 1 key n-tile(s).
+#define KVQ_TC_KB 4
+#define KVQ_TC_NKT 1
+#include "kvq_decode_tc_inst.cuh"

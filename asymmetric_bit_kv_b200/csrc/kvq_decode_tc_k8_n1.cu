@@ -1,0 +1,4 @@
+// decode_tc_kernel instances with 8-bit keys and 1 key n-tile(s).
+#define KVQ_TC_KB 8
+#define KVQ_TC_NKT 1
+#include "kvq_decode_tc_inst.cuh"

@@ -295,7 +295,7 @@ def run_kvq(a):
     plan = []  # (replica, launches, algorithmic bytes of the decode, KV tokens attended)
     for i in range(a.steps):
         r = (a.warmup + i) % R
-        launches = 3 + (1 if lens[r][0][1] == Rw else 0)  # ring write + decode + combine (+ flush)
+        launches = 2 + (1 if lens[r][0][1] == Rw else 0)  # ring write + decode (+ flush)
         ab, tk = 2 * B * Hq * D * 2, 0  # q in, out
         for b in range(B):
             qn, n = lens[r][b]
