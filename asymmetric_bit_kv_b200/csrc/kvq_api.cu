@@ -3,6 +3,7 @@
 // split planner. All device work is enqueued by the launchers of
 // kvq_append.cu and kvq_decode.cu.
 #include <algorithm>
+#include <cstddef>
 #include <cmath>
 #include <cstdint>
 #include <cstdarg>
@@ -263,7 +264,9 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out,
     mp = kvq::make_mma_plan(L, cfg.num_q_heads);
     per_sm = kvq::mma_ctas_per_sm(L, mp, cfg.num_q_heads);
   }
-  std::vector<int> nblk(batch);
+  // per-call scratch of this thread (no heap traffic per call)
+  thread_local std::vector<int> nblk;
+  nblk.resize(batch);
   int max_blk = 0;
   int64_t total_blocks = 0;
   for (int b = 0; b < batch; ++b) {
@@ -272,10 +275,10 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out,
     total_blocks += (int64_t)nblk[b] * cfg.num_kv_heads;
   }
   if (total_blocks > INT32_MAX) return fail(KVQ_ERR_UNSUPPORTED, "more than 2^31 quantized blocks in one call");
-  kvq::DecodeParams* pp = new (std::nothrow) kvq::DecodeParams;
-  if (!pp) return fail(KVQ_ERR_INVALID_ARG, "out of host memory");
+  thread_local kvq::DecodeParams params;
+  kvq::DecodeParams* pp = &params;
   kvq::DecodeParams& p = *pp;
-  std::memset(pp, 0, sizeof *pp);
+  std::memset(pp, 0, offsetof(kvq::DecodeParams, nblk));  // the per-sequence tables are written below
   p.L = L;
   p.q = q;
   p.out = out;
@@ -304,10 +307,7 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out,
       p.seq_start[b] = (int32_t)total;
       total += (int64_t)p.nitem[b] * cfg.num_kv_heads;
     }
-    if (total > INT32_MAX) {
-      delete pp;
-      return fail(KVQ_ERR_UNSUPPORTED, "more than 2^31 work items in one call");
-    }
+    if (total > INT32_MAX) return fail(KVQ_ERR_UNSUPPORTED, "more than 2^31 work items in one call");
     int64_t nctas = std::min<int64_t>((int64_t)std::max(1, c->sm_count) * per_sm,
                                       std::max<int64_t>((int64_t)batch * cfg.num_kv_heads, (total + 3) / 4));
     nctas = std::max<int64_t>(nctas, 1);
@@ -325,10 +325,7 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out,
     p.persistent = 1;
     p.total_blocks = (int32_t)total;
     p.num_ctas = (int32_t)nctas;
-    if (scratch && !use_scratch(p, *scratch, batch, used_slots, &s)) {
-      delete pp;
-      return s;
-    }
+    if (scratch && !use_scratch(p, *scratch, batch, used_slots, &s)) return s;
     e = kvq::launch_decode_mma(p, mp, static_cast<cudaStream_t>(stream));
   } else {
     // Split plan: blocks per split chosen to minimise (waves of CTAs) x
@@ -351,13 +348,9 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out,
     p.blocks_per_split = (int32_t)bps;
     const int nsplits = (int)((max_blk + bps - 1) / bps);
     used_slots = nsplits + 1;
-    if (scratch && !use_scratch(p, *scratch, batch, used_slots, &s)) {
-      delete pp;
-      return s;
-    }
+    if (scratch && !use_scratch(p, *scratch, batch, used_slots, &s)) return s;
     e = kvq::launch_decode(p, nsplits, static_cast<cudaStream_t>(stream));
   }
-  delete pp;
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return KVQ_OK;
 }

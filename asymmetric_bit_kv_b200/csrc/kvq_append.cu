@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_blocks_kernel(AppendPa
   uint32_t* kc = reinterpret_cast<uint32_t*>(rec + L.kc_off);
   __half2* ksz = reinterpret_cast<__half2*>(rec + L.ksz_off);
   uint32_t* vc = reinterpret_cast<uint32_t*>(rec + L.vc_off);
-  __half2* vsz = reinterpret_cast<__half2*>(rec + L.vsz_off);
+  __half* vsz = reinterpret_cast<__half*>(rec + L.vsz_off);
   const int dt = L.kv_dtype;
 
   // Keys: one group per channel over the G tokens (KIVI: per-channel keys).
@@ -107,7 +107,10 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_blocks_kernel(AppendPa
     uint32_t word = 0;
     for (int i = 0; i < per; ++i) word |= quant_code(bits_to_float(xs[i], dt), gp, vb) << (i * vb);
     vc[vc_word_index(t, w, G, kb, wpt)] = word;
-    if ((w % P) == 0) vsz[t * (D / Gv) + w / P] = __halves2half2(gp.d16, gp.m16);
+    if ((w % P) == 0) {
+      vsz[vsz_half_index(t, w / P, G, kb, D / Gv, false)] = gp.d16;
+      vsz[vsz_half_index(t, w / P, G, kb, D / Gv, true)] = gp.m16;
+    }
   }
 }
 
@@ -162,8 +165,9 @@ __global__ void dequant_kernel(LayerView L, int seq, int t0, int n, float* k_out
       const uint32_t* vc = reinterpret_cast<const uint32_t*>(rec + L.vc_off);
       const int vper = 32 / vb;
       const uint32_t vq = (vc[vc_word_index(t, d / vper, G, kb, D / vper)] >> ((d % vper) * vb)) & ((1u << vb) - 1);
-      const __half2 vsz = reinterpret_cast<const __half2*>(rec + L.vsz_off)[t * (D / L.group_v) + d / L.group_v];
-      v_out[o] = dequant_value(vq, __low2half(vsz), __high2half(vsz));
+      const __half* vsz = reinterpret_cast<const __half*>(rec + L.vsz_off);
+      const int ng = D / L.group_v, gg = d / L.group_v;
+      v_out[o] = dequant_value(vq, vsz[vsz_half_index(t, gg, G, kb, ng, false)], vsz[vsz_half_index(t, gg, G, kb, ng, true)]);
     } else {
       const int64_t src = (((int64_t)seq * L.num_kv_heads + h) * R + tok % R) * D + d;
       k_out[o] = load_kv(L.ring_k, src, L.kv_dtype);

@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
       for (int hh = 0; hh < NG; ++hh) bias[hh] = sbias[0][hh] + sbias[1][hh] + sbias[2][hh] + sbias[3][hh];
       const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + L.kc_off);
       const uint32_t* vc = reinterpret_cast<const uint32_t*>(rec + L.vc_off);
-      const __half2* vsz = reinterpret_cast<const __half2*>(rec + L.vsz_off);
+      const __half* vsz = reinterpret_cast<const __half*>(rec + L.vsz_off);
       for (int t = warp; t < G; t += 4) {
         float kcode[4], vv[4];
 #pragma unroll
@@ -124,8 +124,9 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
           const int d = lane + 32 * c;
           kcode[c] = (float)((kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb)) & kmask);
           const uint32_t vq = (vc[vc_word_index(t, d / vper, G, kb, D / vper)] >> ((d % vper) * vb)) & vmask;
-          const __half2 sz = vsz[t * (D / Gv) + d / Gv];
-          vv[c] = (float)vq * __low2float(sz) + __high2float(sz);
+          const float vs = __half2float(vsz[vsz_half_index(t, d / Gv, G, kb, D / Gv, false)]);
+          const float vz = __half2float(vsz[vsz_half_index(t, d / Gv, G, kb, D / Gv, true)]);
+          vv[c] = (float)vq * vs + vz;
         }
 #pragma unroll
         for (int hh = 0; hh < NG; ++hh) {

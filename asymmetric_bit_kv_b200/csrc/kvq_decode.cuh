@@ -57,7 +57,13 @@ __host__ __device__ inline int32_t cta_first_block(int64_t T, int32_t nctas, int
   return (int32_t)((int64_t)c * T / nctas);
 }
 __host__ __device__ inline int32_t cta_of_block(int64_t T, int32_t nctas, int32_t k) {
+#ifdef __CUDA_ARCH__
   int32_t c = (int32_t)((int64_t)k * nctas / T);
+#else
+  int32_t c = (int32_t)((double)k * nctas / (double)T);  // a guess, corrected below
+  if (c < 0) c = 0;
+  if (c >= nctas) c = nctas - 1;
+#endif
   while (c + 1 < nctas && cta_first_block(T, nctas, c + 1) <= k) ++c;
   while (c > 0 && cta_first_block(T, nctas, c) > k) --c;
   return c;
@@ -84,7 +90,6 @@ struct MmaPlan {
   int32_t ws_bytes;     // bytes per consumer-warp scratch
   int32_t bfrag_off;    // scratch: key B fragments (q*s, fp16 high/low)
   int32_t bias_off;     // scratch: per-head sum_d q_d z_d
-  int32_t vpair_off;    // scratch: value scale/zero of token pairs (fp16)
   int32_t qbuf_off;     // scratch: the queries of the warp's current units (kv dtype)
   int32_t bar_off;      // offset of the mbarriers
   int32_t smem_bytes;   // dynamic shared memory per CTA

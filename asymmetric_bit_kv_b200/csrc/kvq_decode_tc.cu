@@ -57,8 +57,7 @@ MmaPlan make_mma_plan(const LayerView& L, int num_q_heads) {
   // per-consumer-warp scratch
   mp.bfrag_off = 0;
   mp.bias_off = nkt * 8 * 32 * 8;
-  mp.vpair_off = mp.bias_off + 32;
-  mp.qbuf_off = (int32_t)round_up(mp.vpair_off + (G / 16) * 4 * ngrp * 16, 128);
+  mp.qbuf_off = (int32_t)round_up(mp.bias_off + 32, 128);
   // Stages (and query buffers) per warp: two (one being read, one landing)
   // when two CTAs then fit an SM, else up to four with one CTA per SM.
   auto smem_for = [&](int spw) {

@@ -164,6 +164,21 @@ __device__ __forceinline__ uint32_t code_at(uint32_t x, uint32_t x8, int j) {
   const uint32_t magic = e | (e << 16);
   return hsub2(and_or(bit >= 8 ? x8 : x, m | (m << 16), magic), magic);
 }
+// Code j as 2^(10-p) + code (the value code_at would return plus the magic
+// of its bit position p), one instruction; the offset is taken out later.
+template <int B>
+__device__ __forceinline__ uint32_t code_raw(uint32_t x, uint32_t x8, int j) {
+  const int bit = B * j;
+  const int pos = bit & 7;
+  const uint32_t m = ((1u << B) - 1u) << pos;
+  const uint32_t e = (uint32_t)(25 - pos) << 10;
+  return and_or(bit >= 8 ? x8 : x, m | (m << 16), e | (e << 16));
+}
+// fp16 pair (-2^(10-p), -2^(10-p)) for the bit position p of code j.
+template <int B>
+__host__ __device__ constexpr uint32_t neg_magic2(int j) {
+  return ((0x8000u | ((uint32_t)(25 - ((B * j) & 7)) << 10)) * 0x10001u);
+}
 
 // Compile-time shape of one instance. A tile is 64 tokens of a block.
 template <int KB, int VB, int NGRP, int NKT>
@@ -372,14 +387,11 @@ struct UnitCursor {
 //         (n >= 4); with 8 heads n-tile 0 holds the high and n-tile 1 the low
 //         parts of heads 0-7. Columns of absent heads stay zero.
 //   bias  [8] float: sum_d q_d z_d per head (log2 units);
-//   vpair [k-step][4 t][groups] uint4: (s, s), (s, s), (z, z), (z, z) fp16
-//         pairs of the value tokens that thread t feeds into a P.V k-step;
 //   qbuf  [nstages][NG][D] kv dtype: the queries of the warp's last units
 //         (one buffer per unit change, round robin), as stored in q.
-template <int KB, int VB, int NGRP, int NKT>
+template <int NKT, bool BF16>
 __device__ __forceinline__ void prep_block(const uint8_t* stage, const MmaPlan& mp, uint8_t* ws, const uint32_t* qw,
-                                           int NG, int G, int lane, float scale_log2, bool bf16) {
-  using S = Shape<KB, VB, NGRP, NKT>;
+                                           int NG, int lane, float scale_log2) {
   uint32_t* bk = reinterpret_cast<uint32_t*>(ws + mp.bfrag_off);
   const uint2* ksz2 = reinterpret_cast<const uint2*>(stage + mp.kc_bytes);  // (s, z) of channels 2c, 2c+1
   float* biasw = reinterpret_cast<float*>(ws + mp.bias_off);
@@ -390,9 +402,10 @@ __device__ __forceinline__ void prep_block(const uint8_t* stage, const MmaPlan& 
     float bp = 0.f;
     if (hh < NG) {
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const float2 qf = unpack_kv(qw[hh * 64 + 8 * kk + q], bf16);  // channels 16kk + 2q, +1
-        const uint2 sz = ksz2[8 * kk + q];
+      for (int i = 0; i < 8; ++i) {
+        const int kk = i;
+        const float2 qf = BF16 ? unpack_bf16(qw[hh * 64 + 8 * kk + q]) : unpack_f16(qw[hh * 64 + 8 * kk + q]);
+        const uint2 sz = ksz2[8 * kk + q];  // channels 16kk + 2q, +1
         const float2 c0 = unpack_f16(sz.x), c1 = unpack_f16(sz.y);
         const float q0 = qf.x * scale_log2, q1 = qf.y * scale_log2;
         const float x0 = q0 * c0.x, x1 = q1 * c1.x;
@@ -414,31 +427,21 @@ __device__ __forceinline__ void prep_block(const uint8_t* stage, const MmaPlan& 
     bp += __shfl_xor_sync(0xffffffffu, bp, 4);
     if (q == 0 && hh < NG) biasw[hh] = bp;
   }
-  const uint32_t* vsz = reinterpret_cast<const uint32_t*>(stage + mp.vsz_soff);  // [G][NGRP] (s, z)
-  uint4* vp = reinterpret_cast<uint4*>(ws + mp.vpair_off);
-  const int nvp = (G / 16) * 4 * NGRP;
-  for (int e = lane; e < nvp; e += 32) {
-    const int gg = e % NGRP, tv = (e / NGRP) & 3, kst = e / (NGRP * 4);
-    const int tb = (kst / S::MT) * S::TT, mt = kst % S::MT;
-    const uint32_t a = vsz[(tb + tile_token<KB>(mt, 2 * tv)) * NGRP + gg];
-    const uint32_t b = vsz[(tb + tile_token<KB>(mt, 2 * tv + 1)) * NGRP + gg];
-    const uint32_t c = vsz[(tb + tile_token<KB>(mt, 8 + 2 * tv)) * NGRP + gg];
-    const uint32_t d = vsz[(tb + tile_token<KB>(mt, 9 + 2 * tv)) * NGRP + gg];
-    vp[e] = make_uint4(__byte_perm(a, b, 0x5410), __byte_perm(c, d, 0x5410), __byte_perm(a, b, 0x7632),
-                       __byte_perm(c, d, 0x7632));
-  }
   __syncwarp();
 }
 
 
 // Online-softmax update (log2 units) of this lane's two heads (2t and 2t+1)
 // with the scores sc of MTN M-tiles (registers 0/2: head 2t, rows g and g+8;
-// 1/3: head 2t+1; -inf where a token is absent). sc becomes the
-// probabilities; O and Z are rescaled when a running maximum grows.
+// 1/3: head 2t+1). sc becomes the probabilities; O and Z are rescaled when a
+// running maximum grows. GUARD: scores may be -inf (absent tokens) and a
+// whole update may see none, and heads beyond NG are zeroed (ring chunks);
+// without it every score is finite, and heads beyond NG just compute finite
+// values in columns that are never written (quantized tiles).
 struct SoftState {
   float m0, m1, l0, l1;
 };
-template <int MTN, int NGRP>
+template <int MTN, int NGRP, bool GUARD>
 __device__ __forceinline__ void softmax_update(float (&sc)[MTN][4], SoftState& st, bool v0, bool v1,
                                                float (&O)[8][4], float (&Z)[NGRP][4]) {
   float mx0 = -INFINITY, mx1 = -INFINITY;
@@ -452,18 +455,35 @@ __device__ __forceinline__ void softmax_update(float (&sc)[MTN][4], SoftState& s
     mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
   }
-  // a head with no finite score so far keeps m = -inf, alpha = 1, p = 0
-  const float n0 = v0 ? fmaxf(st.m0, mx0) : -INFINITY, n1 = v1 ? fmaxf(st.m1, mx1) : -INFINITY;
-  const float a0 = n0 == -INFINITY ? 1.f : ex2(st.m0 - n0), a1 = n1 == -INFINITY ? 1.f : ex2(st.m1 - n1);
+  float n0, n1, a0, a1;
+  if constexpr (GUARD) {
+    // a head with no finite score so far keeps m = -inf, alpha = 1, p = 0
+    n0 = v0 ? fmaxf(st.m0, mx0) : -INFINITY;
+    n1 = v1 ? fmaxf(st.m1, mx1) : -INFINITY;
+    a0 = n0 == -INFINITY ? 1.f : ex2(st.m0 - n0);
+    a1 = n1 == -INFINITY ? 1.f : ex2(st.m1 - n1);
+  } else {
+    n0 = fmaxf(st.m0, mx0);
+    n1 = fmaxf(st.m1, mx1);
+    a0 = ex2(st.m0 - n0);  // 0 on the first tile (m = -inf)
+    a1 = ex2(st.m1 - n1);
+  }
   st.m0 = n0;
   st.m1 = n1;
   float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
   for (int mt = 0; mt < MTN; ++mt) {
-    sc[mt][0] = n0 == -INFINITY ? 0.f : ex2(sc[mt][0] - n0);
-    sc[mt][2] = n0 == -INFINITY ? 0.f : ex2(sc[mt][2] - n0);
-    sc[mt][1] = n1 == -INFINITY ? 0.f : ex2(sc[mt][1] - n1);
-    sc[mt][3] = n1 == -INFINITY ? 0.f : ex2(sc[mt][3] - n1);
+    if constexpr (GUARD) {
+      sc[mt][0] = n0 == -INFINITY ? 0.f : ex2(sc[mt][0] - n0);
+      sc[mt][2] = n0 == -INFINITY ? 0.f : ex2(sc[mt][2] - n0);
+      sc[mt][1] = n1 == -INFINITY ? 0.f : ex2(sc[mt][1] - n1);
+      sc[mt][3] = n1 == -INFINITY ? 0.f : ex2(sc[mt][3] - n1);
+    } else {
+      sc[mt][0] = ex2(sc[mt][0] - n0);
+      sc[mt][2] = ex2(sc[mt][2] - n0);
+      sc[mt][1] = ex2(sc[mt][1] - n1);
+      sc[mt][3] = ex2(sc[mt][3] - n1);
+    }
     ps0 += sc[mt][0] + sc[mt][2];
     ps1 += sc[mt][1] + sc[mt][3];
   }
@@ -564,7 +584,7 @@ __device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t*
     const float x = head_score<NKT>(Dr, e);
     sc[0][e] = (e < 2 && g < cnt) ? x : -INFINITY;
   }
-  softmax_update<1, NGRP>(sc, sst, v0, v1, O, Z);
+  softmax_update<1, NGRP, true>(sc, sst, v0, v1, O, Z);
   const uint32_t ph = pack_kv<BF16>(sc[0][0], sc[0][1]);
   const float2 fh = unpack_kv2<BF16>(ph);
   const uint32_t bh = movmatrix_t(ph), bl = movmatrix_t(pack_kv<BF16>(sc[0][0] - fh.x, sc[0][1] - fh.y));
@@ -662,6 +682,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
     }
     const int g = lane >> 2, t = lane & 3;
     const uint32_t ones[4] = {0x3c003c00u, 0x3c003c00u, 0x3c003c00u, 0x3c003c00u};  // fp16 1.0
+    // Value codes of 4 or 8 bits keep the magic offset 2^(10-p) of their bit
+    // position (one instruction per pair instead of two): rows g and g+8 of
+    // every channel m-tile then carry the same offsets, here codes 0 and 1 of
+    // a 16-bit column, and one more MMA per value group with the constant A
+    // operand -offset(row) against the same B (p*s) takes offset(row) * sum_t
+    // p*s back out, into the zero-point accumulator Z. (2-bit codes alternate
+    // between two offset pairs across m-tiles and subtract per pair instead.)
+    constexpr bool RAWV = VB != 2;
+    const uint32_t vneg[4] = {neg_magic2<VB>(0), neg_magic2<VB>(1), neg_magic2<VB>(0), neg_magic2<VB>(1)};
     const int kc_row = G * KB / 8;  // key code bytes per channel
     const int mi = lane >> 3, rr = lane & 7;
     // ldmatrix rows of this lane: 8 consecutive rows, so the chunk swizzle of
@@ -670,7 +699,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
     const int swv = chunk_swizzle(rr, S::VRB / 16);
     const uint2* bkr = reinterpret_cast<const uint2*>(ws + mp.bfrag_off);
     uint2* bkw = reinterpret_cast<uint2*>(ws + mp.bfrag_off);
-    const uint4* vpr = reinterpret_cast<const uint4*>(ws + mp.vpair_off);
     const float* biasr = reinterpret_cast<const float*>(ws + mp.bias_off);
     int qseq = -1;  // unit changes seen by the consumer side (matches IssueState::seq)
     const bool v0 = 2 * t < NG, v1 = 2 * t + 1 < NG;  // heads 2t, 2t+1 of this lane exist
@@ -701,10 +729,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
         const int j = kb - u.start;
         if (j < nb) {
           // ============ quantized block
-          prep_block<KB, VB, NGRP, NKT>(stage, mp, ws, qw, NG, G, lane, p.scale_log2, bf16);
+          if (bf16) prep_block<NKT, true>(stage, mp, ws, qw, NG, lane, p.scale_log2);
+          else prep_block<NKT, false>(stage, mp, ws, qw, NG, lane, p.scale_log2);
           const float bias0 = biasr[2 * t], bias1 = biasr[2 * t + 1];
           const uint32_t kc_s = smem_u32(stage);
           const uint32_t vc_s = smem_u32(stage + mp.vc_soff);
+          const uint4* vsz4 = reinterpret_cast<const uint4*>(stage + mp.vsz_soff);
           for (int tile = 0; tile < G / S::TT; ++tile) {
             // ---- scores: Dk[M-tile][n-tile] = codes x (q*s)
             float Dk[S::MT][NKT][4];
@@ -744,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
             for (int mt = 0; mt < S::MT; ++mt)
 #pragma unroll
               for (int e = 0; e < 4; ++e) sc[mt][e] = head_score<NKT>(Dk[mt], e) + ((e & 1) ? bias1 : bias0);
-            softmax_update<S::MT, NGRP>(sc, sst, v0, v1, O, Z);
+            softmax_update<S::MT, NGRP, false>(sc, sst, v0, v1, O, Z);
             // ---- values: O += codes x (p * s), Z += ones x (p * z)
 #pragma unroll
             for (int mt = 0; mt < S::MT; ++mt) {
@@ -755,10 +785,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
               uint32_t B0[NGRP], B1[NGRP];
 #pragma unroll
               for (int gg = 0; gg < NGRP; ++gg) {
-                const uint4 v4 = vpr[(kst * 4 + t) * NGRP + gg];
+                const uint4 v4 = vsz4[(kst * 4 + t) * NGRP + gg];  // (s, s), (s, s), (z, z), (z, z) of rows 2t.. 9+2t
                 B0[gg] = hmul2(bt, v4.x);
                 B1[gg] = hmul2(bb, v4.y);
                 mma_f16(Z[gg], ones, hmul2(bt, v4.z), hmul2(bb, v4.w));
+                if constexpr (RAWV) mma_f16(Z[gg], vneg, B0[gg], B1[gg]);  // - offset(row) * sum_t p*s
               }
               const int sg = mt / S::JP, jp = mt % S::JP;
               const int vrow_idx = (2 * jp + (mi & 1)) * (G / S::CPT16) + tile * (S::TT / S::CPT16) + sg * 8 + rr;
@@ -773,8 +804,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
                   const int gg = ((cc0 + cc) * S::CH_SPAN) / S::GV;
 #pragma unroll
                   for (int P = 0; P < S::MT_PER_CH; ++P) {
-                    const uint32_t a[4] = {code_at<VB>(xv, xv8, 2 * P), code_at<VB>(xv, xv8, 2 * P + 1),
-                                           code_at<VB>(yv, yv8, 2 * P), code_at<VB>(yv, yv8, 2 * P + 1)};
+                    uint32_t a[4];
+                    if constexpr (RAWV) {
+                      a[0] = code_raw<VB>(xv, xv8, 2 * P);
+                      a[1] = code_raw<VB>(xv, xv8, 2 * P + 1);
+                      a[2] = code_raw<VB>(yv, yv8, 2 * P);
+                      a[3] = code_raw<VB>(yv, yv8, 2 * P + 1);
+                    } else {
+                      a[0] = code_at<VB>(xv, xv8, 2 * P);
+                      a[1] = code_at<VB>(xv, xv8, 2 * P + 1);
+                      a[2] = code_at<VB>(yv, yv8, 2 * P);
+                      a[3] = code_at<VB>(yv, yv8, 2 * P + 1);
+                    }
                     mma_f16(O[(cc0 + cc) * S::MT_PER_CH + P], a, B0[gg], B1[gg]);
                   }
                 }
@@ -810,10 +851,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
         const int cch = mt2 / S::MT_PER_CH, P = mt2 % S::MT_PER_CH;
         const int gg = (cch * S::CH_SPAN) / S::GV;
         const int ch0 = cch * S::CH_SPAN + g * S::VCPC + 2 * P;
+        // rows g (channel ch0) and g+8 (ch0 + 1); Z holds the zero-point term
+        // (and the offset correction) per row
         if (v0)
-          *reinterpret_cast<float2*>(p.ws_o + base0 * D + ch0) = make_float2(O[mt2][0] + Z[gg][0], O[mt2][2] + Z[gg][0]);
+          *reinterpret_cast<float2*>(p.ws_o + base0 * D + ch0) = make_float2(O[mt2][0] + Z[gg][0], O[mt2][2] + Z[gg][2]);
         if (v1)
-          *reinterpret_cast<float2*>(p.ws_o + base1 * D + ch0) = make_float2(O[mt2][1] + Z[gg][1], O[mt2][3] + Z[gg][1]);
+          *reinterpret_cast<float2*>(p.ws_o + base1 * D + ch0) = make_float2(O[mt2][1] + Z[gg][1], O[mt2][3] + Z[gg][3]);
       }
       if (g == 0) {
         if (v0) p.ws_ml[base0] = make_float2(sst.m0, sst.l0);

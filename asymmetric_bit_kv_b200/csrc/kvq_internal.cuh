@@ -72,6 +72,28 @@ __host__ __device__ inline int vc_word_index(int t, int w, int G, int kb, int VW
   return r * VW + ((c ^ chunk_swizzle(r, VW / 4)) << 2) + (w & 3);
 }
 
+// Position (in 16-bit halves) of the value scale (zero = false) or zero
+// point of token t (0 <= t < G) and value group gg inside the vsz array of a
+// record. Blocks of G >= 64 tokens keep them in the order the tensor-core
+// decode kernel feeds them to its P.V operands, so that a warp reads one
+// 16-byte entry per (k-step, lane quad, group) straight from the staged
+// record: a 64-token tile has four k-steps of 16 tokens, k-step mt row r
+// (0..15) being the token the key path puts on that row (the inverse of its
+// tile_token); entry ((tile*4 + mt)*4 + (r%8)/2, group) holds the scales of
+// rows 2q, 2q+1, 8+2q, 9+2q, then their zero points. Smaller blocks keep the
+// plain [G][groups] order of (scale, zero) pairs.
+__host__ __device__ inline int vsz_half_index(int t, int gg, int G, int kb, int ngrp, bool zero) {
+  if (G < 64) return (t * ngrp + gg) * 2 + (zero ? 1 : 0);
+  const int CPT16 = 16 / kb, TOKC = 128 / kb, JP = CPT16 / 2;
+  const int tile = t / 64, tt = t % 64;
+  const int sg = tt / TOKC, rem = tt % TOKC;
+  const int col = rem / CPT16, j = rem % CPT16;
+  const int mt = sg * JP + j / 2;  // key M-tile of the token
+  const int r = col + 8 * (j & 1);  // its row in that M-tile
+  const int entry = ((tile * 4 + mt) * 4 + ((r & 7) >> 1)) * ngrp + gg;
+  return entry * 8 + (zero ? 4 : 0) + 2 * (r >> 3) + (r & 1);
+}
+
 __device__ __forceinline__ uint8_t* record_ptr(const LayerView& L, int b, int h, int64_t j) {
   return L.blocks + (((int64_t)b * L.num_kv_heads + h) * L.max_blocks + j) * L.record_bytes;
 }

@@ -107,8 +107,13 @@ def _check(status: int, func: str):
 
 
 def _stream_ptr(stream) -> int:
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return s.cuda_stream
+    """cudaStream_t of `stream`: a torch.cuda.Stream, a raw handle (int), or
+    None for torch's current stream."""
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
 
 
 def _need(t: torch.Tensor, dtype, name):
@@ -152,6 +157,12 @@ def required_bytes(cfg: CacheConfig) -> int:
     return n.value
 
 
+def lens_array(new_lens) -> ctypes.Array:
+    """new_lens as the int32 array kvq_append takes (reusable across calls)."""
+    n = [int(x) for x in new_lens]
+    return (ctypes.c_int32 * len(n))(*n)
+
+
 class KVCache:
     """A packed KV cache bound to a torch-allocated device arena."""
 
@@ -180,12 +191,13 @@ class KVCache:
         _check(self.lib.kvq_cache_reset(self.handle, _stream_ptr(stream)), "kvq_cache_reset")
 
     def append(self, layer: int, k: torch.Tensor, v: torch.Tensor, new_lens, stream=None):
-        """k, v: [sum(new_lens), Hkv, D] in the cache dtype; new_lens: ints per sequence."""
+        """k, v: [sum(new_lens), Hkv, D] in the cache dtype; new_lens: ints per
+        sequence (a list, or a ctypes int32 array from lens_array() to skip the
+        per-call conversion)."""
         _need(k, self.cfg.kv_dtype, "k")
         _need(v, self.cfg.kv_dtype, "v")
-        n = list(int(x) for x in new_lens)
-        arr = (ctypes.c_int32 * max(len(n), 1))(*n)
-        _check(self.lib.kvq_append(self.handle, layer, k.data_ptr(), v.data_ptr(), arr, len(n), _stream_ptr(stream)),
+        arr = new_lens if isinstance(new_lens, ctypes.Array) else lens_array(new_lens)
+        _check(self.lib.kvq_append(self.handle, layer, k.data_ptr(), v.data_ptr(), arr, len(arr), _stream_ptr(stream)),
                "kvq_append")
 
     def flush_residual(self, layer: int, batch: int, stream=None):

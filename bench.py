@@ -267,19 +267,37 @@ def run_kvq(a):
     new_v = torch.randn(pool, B, Hkv, D, generator=gen, device=dev).to(wl.kv_dtype)
     qs = torch.randn(pool, B, Hq, D, generator=gen, device=dev).to(wl.kv_dtype)
     out = torch.empty(B, Hq, D, dtype=wl.kv_dtype, device=dev)
-    ones = [1] * B
+    from asymmetric_bit_kv_b200.kvq import lens_array
+    ones = lens_array([1] * B)
     stream = torch.cuda.current_stream()
+    # per-step inputs as views made once, so that the timed loop only enqueues
+    views = [(new_k[j], new_v[j], qs[j]) for j in range(pool)]
     bytes_tok = O.quantized_bytes_per_token(Hkv, D, wl.k_bits[0], wl.v_bits[0], wl.group_k, wl.group_v)
 
     G, Rw = wl.group_k, wl.residual
 
+    # The device-timed loop calls the C entry points (kvq_append,
+    # kvq_decode_attention) with arguments prepared here, so that Python
+    # overhead per call stays far below the GPU time of a step; the e2e leg
+    # below goes through the Python binding.
+    lib = caches[0].lib
+    c_append, c_decode = lib.kvq_append, lib.kvq_decode_attention
+    sh = stream.cuda_stream
+    handles = [c.handle for c in caches]
+    ptrs = [(kk.data_ptr(), vv.data_ptr(), qq.data_ptr()) for kk, vv, qq in views]
+    optr, oty, scale = out.data_ptr(), 1, float(wl.softmax_scale)  # out dtype code 1 = bf16
+
     def step(i, r, ev=None):
-        caches[r].append(0, new_k[i % pool], new_v[i % pool], ones)
+        kp, vp, qp = ptrs[i % pool]
+        h = handles[r]
+        st = c_append(h, 0, kp, vp, ones, B, sh)
         if ev is not None:
             ev[0].record(stream)
-        caches[r].decode_attention(0, qs[i % pool], out, softmax_scale=wl.softmax_scale)
+        st |= c_decode(h, 0, qp, optr, oty, scale, B, sh)
         if ev is not None:
             ev[1].record(stream)
+        if st:
+            raise RuntimeError(f"kvq call failed: {lib.kvq_last_error().decode()}")
 
     for i in range(a.warmup):
         step(i, i % R)
@@ -372,8 +390,8 @@ def run_kvq(a):
         dk.copy_(hk[j], non_blocking=True)
         dv.copy_(hv[j], non_blocking=True)
         dq.copy_(hq[j], non_blocking=True)
-        caches[r].append(0, dk, dv, ones)
-        caches[r].decode_attention(0, dq, out, softmax_scale=wl.softmax_scale)
+        caches[r].append(0, dk, dv, ones, stream=stream)
+        caches[r].decode_attention(0, dq, out, softmax_scale=wl.softmax_scale, stream=stream)
         hout.copy_(out, non_blocking=True)
     f1.record(stream)
     torch.cuda.synchronize()

@@ -99,7 +99,10 @@ typedef struct kvq_cache kvq_cache;
  *   vc  uint32 [G][V], V = D*v_bits/32: one row of V words per token; word w
  *       packs the codes of channels w*(32/v_bits) + i, code i at bits
  *       [i*v_bits, ...) (per-token values packed along head_dim);
- *   vsz half2 [G][D/group_v]: (scale, zero point) of each value group.
+ *   vsz fp16 scale and zero point of each (token, value group): for
+ *       G < 64 the pairs [G][D/group_v] of (scale, zero point); for G >= 64
+ *       16-byte entries in the order the decode kernel reads them (see
+ *       kvq_internal.cuh: vsz_half_index).
  * Placement inside kc and vc (so that one copy of a record is readable with
  * ldmatrix without shared-memory bank conflicts): in a row of n >= 2
  * 16-byte chunks (4 words each), chunk c of row r is stored at chunk
@@ -125,8 +128,9 @@ KVQ_API kvq_status kvq_cache_required_bytes(const kvq_config* cfg, size_t* bytes
 
 /* Validate cfg and bind a cache to dev_arena (device pointer, 256-byte
  * aligned, arena_bytes >= required), with the arena's device current. Every
- * sequence starts empty: the call zeroes the arena's length table and waits
- * for that to finish before it returns.                                    */
+ * sequence starts empty: the call zeroes the arena's length table, decode
+ * arrival counters and residual rings, and waits for that to finish before
+ * it returns.                                                              */
 KVQ_API kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena_bytes,
                             kvq_cache** out);
 

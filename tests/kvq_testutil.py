@@ -56,6 +56,22 @@ def vc_word_index(t: int, w: int, G: int, kb: int, VW: int) -> int:
     return r * VW + (((w >> 2) ^ chunk_swizzle(r, VW // 4)) << 2) + (w & 3)
 
 
+def vsz_half_index(t: int, gg: int, G: int, kb: int, ngrp: int, zero: bool) -> int:
+    """Half position of the value scale (or zero point) of token t, group gg,
+    in a record's vsz array (layout documented in kvq.h)."""
+    if G < 64:
+        return (t * ngrp + gg) * 2 + (1 if zero else 0)
+    cpt16, tokc = 16 // kb, 128 // kb
+    jp_count = cpt16 // 2
+    tile, tt = divmod(t, 64)
+    sg, rem = divmod(tt, tokc)
+    col, j = divmod(rem, cpt16)
+    mt = sg * jp_count + j // 2
+    r = col + 8 * (j & 1)
+    entry = ((tile * 4 + mt) * 4 + ((r & 7) >> 1)) * ngrp + gg
+    return entry * 8 + (4 if zero else 0) + 2 * (r >> 3) + (r & 1)
+
+
 class Twin:
     """A device cache and one oracle SequenceCache per (layer, sequence)."""
 
@@ -114,11 +130,15 @@ class Twin:
         vc = part(lay.vc_offset, G * vcw * 4, np.uint32, (G * vcw,))
         kidx = np.array([[kc_word_index(d, w, kcw) for w in range(kcw)] for d in range(D)])
         vidx = np.array([[vc_word_index(t, w, G, kb, vcw) for w in range(vcw)] for t in range(G)])
+        ng = D // Gv
+        vsz = part(lay.vsz_offset, G * ng * 4, np.float16, (G * ng * 2,))
+        sidx = np.array([[[vsz_half_index(t, gg, G, kb, ng, z) for z in (False, True)] for gg in range(ng)]
+                         for t in range(G)])
         return {
             "kc": kc[:, kidx],
             "ksz": part(lay.ksz_offset, D * 4, np.float16, (D, 2)),
             "vc": vc[:, vidx],
-            "vsz": part(lay.vsz_offset, G * (D // Gv) * 4, np.float16, (G, D // Gv, 2)),
+            "vsz": vsz[:, sidx],
         }
 
     def read_ring(self, layer: int, b: int):
