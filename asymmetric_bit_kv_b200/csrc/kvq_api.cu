@@ -28,7 +28,6 @@ struct kvq_cache {
   int64_t lens_off;               // int32 [num_layers][max_batch][2]
   int64_t ws_o_off, ws_ml_off;    // split partials
   int64_t err_off;                // int32 device error word
-  int64_t ctr_off;                // int32 [max_batch][num_kv_heads] decode arrival counters
   int32_t slots;                  // partial slots per (sequence, query head)
   int32_t sm_count;
   std::vector<int32_t> q_len, n_len;  // host mirror [num_layers][max_batch]
@@ -87,7 +86,7 @@ kvq_status validate_config(const kvq_config* c) {
 
 struct Plan {
   std::vector<int64_t> blocks_off, ring_k_off, ring_v_off, record_bytes;
-  int64_t max_blocks, lens_off, err_off, ctr_off, ws_o_off, ws_ml_off, total;
+  int64_t max_blocks, lens_off, err_off, ws_o_off, ws_ml_off, total;
   int32_t slots;
 };
 
@@ -116,8 +115,6 @@ Plan make_plan(const kvq_config* c) {
   off = round_up(off + (int64_t)c->num_layers * c->max_batch * 2 * 4, 256);
   p.err_off = off;
   off = round_up(off + 4, 256);
-  p.ctr_off = off;
-  off = round_up(off + seqheads * 4, 256);
   // partial slots per (sequence, query head): enough for the split kernel
   // (one per split + the ring) and for the persistent kernel (one per
   // consumer warp of each CTA range overlapping the unit's work items, at
@@ -290,7 +287,6 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out,
   p.num_q_heads = cfg.num_q_heads;
   p.slots = c->slots;
   p.err = reinterpret_cast<int32_t*>(c->arena + c->err_off);
-  p.unit_ctr = reinterpret_cast<int32_t*>(c->arena + c->ctr_off);
   cudaError_t e;
   int32_t used_slots = c->slots;  // partial slots per (sequence, query head) this call writes
   if (use_mma) {
@@ -327,6 +323,7 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out,
     p.num_ctas = (int32_t)nctas;
     if (scratch && !use_scratch(p, *scratch, batch, used_slots, &s)) return s;
     e = kvq::launch_decode_mma(p, mp, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = kvq::launch_combine(p, static_cast<cudaStream_t>(stream));
   } else {
     // Split plan: blocks per split chosen to minimise (waves of CTAs) x
     // (blocks per CTA + a fixed per-CTA overhead), with at most slots-1 splits.
@@ -413,7 +410,6 @@ kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena
   c->ws_o_off = plan.ws_o_off;
   c->ws_ml_off = plan.ws_ml_off;
   c->err_off = plan.err_off;
-  c->ctr_off = plan.ctr_off;
   c->slots = plan.slots;
   c->q_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
   c->n_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
@@ -421,7 +417,6 @@ kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device);
   if (e == cudaSuccess) e = cudaMemset(c->arena + c->lens_off, 0, (size_t)cfg->num_layers * cfg->max_batch * 8);
   if (e == cudaSuccess) e = cudaMemset(c->arena + c->err_off, 0, 4);
-  if (e == cudaSuccess) e = cudaMemset(c->arena + c->ctr_off, 0, (size_t)cfg->max_batch * cfg->num_kv_heads * 4);
   // Ring slots that no token has reached yet hold zeros, never stale bit
   // patterns: the decode kernel reads whole 16-slot groups of the ring and
   // masks the scores of slots past the sequence, so their values must be finite.
@@ -451,9 +446,6 @@ kvq_status kvq_cache_reset(kvq_cache* c, void* stream) {
   if (!c) return fail(KVQ_ERR_INVALID_ARG, "cache is null");
   cudaError_t e = cudaMemsetAsync(c->arena + c->lens_off, 0, (size_t)c->cfg.num_layers * c->cfg.max_batch * 8,
                                   static_cast<cudaStream_t>(stream));
-  if (e == cudaSuccess)
-    e = cudaMemsetAsync(c->arena + c->ctr_off, 0, (size_t)c->cfg.max_batch * c->cfg.num_kv_heads * 4,
-                        static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "reset");
   std::fill(c->q_len.begin(), c->q_len.end(), 0);
   std::fill(c->n_len.begin(), c->n_len.end(), 0);
@@ -527,9 +519,6 @@ kvq_status kvq_device_errors(kvq_cache* c, int32_t* flags) {
   int32_t v = 0;
   cudaError_t e = cudaMemcpy(&v, c->arena + c->err_off, 4, cudaMemcpyDeviceToHost);
   if (e == cudaSuccess && v != 0) e = cudaMemset(c->arena + c->err_off, 0, 4);
-  // a decode that gave up may have left arrival counters behind: clear them
-  if (e == cudaSuccess && v != 0)
-    e = cudaMemset(c->arena + c->ctr_off, 0, (size_t)c->cfg.max_batch * c->cfg.num_kv_heads * 4);
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
   *flags = v;
   return KVQ_OK;

@@ -170,35 +170,60 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
   }
 }
 
-// grid (Hq, batch); block D threads.
+// Log-sum-exp merge of the partial slots of one (sequence, query head):
+// M = max_s m_s over slots with l_s > 0, out = sum_s 2^(m_s-M) o_s / sum_s
+// 2^(m_s-M) l_s, rounded to the output dtype (nearest even); a sequence with
+// no tokens gives zeros. grid (Hq, batch), block D threads (thread d owns
+// channel d). The slots' (m, l) pass through shared memory once; each thread
+// then issues its slot loads eight at a time.
+constexpr int kCombineMaxSlots = 512;
+
 __global__ void __launch_bounds__(128) combine_kernel(DecodeParams p) {
-  const int hq = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  __shared__ float sw[kCombineMaxSlots];  // slot weights 2^(m_s - M), 0 for empty slots
+  __shared__ float sred[2][4];
+  const int hq = blockIdx.x, b = blockIdx.y, d = threadIdx.x, lane = d & 31, warp = d >> 5;
   const LayerView& L = p.L;
   constexpr int D = kHeadDim;
-  int S;  // slots 0..S hold this (sequence, head)'s partials
+  int S;  // slots of this (sequence, head)
   if (p.persistent) {
     const int h = hq / (p.num_q_heads / L.num_kv_heads);
-    S = persistent_slots(p.total_blocks, p.num_ctas, p.seq_start[b] + h * p.nitem[b], p.nitem[b]) - 1;
+    S = persistent_slots(p.total_blocks, p.num_ctas, p.seq_start[b] + h * p.nitem[b], p.nitem[b]);
   } else {
     const int nblk = L.lens[2 * b] / L.group_k;
-    S = (nblk + p.blocks_per_split - 1) / p.blocks_per_split;
+    S = (nblk + p.blocks_per_split - 1) / p.blocks_per_split + 1;
   }
+  S = min(S, kCombineMaxSlots);
   const int64_t base = ((int64_t)b * p.num_q_heads + hq) * p.slots;
-  float M = -INFINITY;
-  for (int s = 0; s <= S; ++s) {
-    const float2 ml = p.ws_ml[base + s];
-    if (ml.y > 0.f) M = fmaxf(M, ml.x);
+  float m = -INFINITY;
+  for (int s = d; s < S; s += D) {
+    const float2 ml = __ldcg(p.ws_ml + base + s);
+    if (ml.y > 0.f) m = fmaxf(m, ml.x);
   }
-  float acc = 0.f, lsum = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s <= S; ++s) {
-      const float2 ml = p.ws_ml[base + s];
-      if (ml.y > 0.f) {
-        const float f = exp2f(ml.x - M);
-        acc += p.ws_o[(base + s) * D + d] * f;
-        lsum += ml.y * f;
-      }
-    }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if (lane == 0) sred[0][warp] = m;
+  __syncthreads();
+  const float M = fmaxf(fmaxf(sred[0][0], sred[0][1]), fmaxf(sred[0][2], sred[0][3]));
+  float lpart = 0.f;
+  for (int s = d; s < S; s += D) {
+    const float2 ml = __ldcg(p.ws_ml + base + s);
+    const float w = (ml.y > 0.f && M != -INFINITY) ? exp2f(ml.x - M) : 0.f;
+    sw[s] = w;
+    lpart += w * ml.y;
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) lpart += __shfl_xor_sync(0xffffffffu, lpart, off);
+  if (lane == 0) sred[1][warp] = lpart;
+  __syncthreads();
+  const float lsum = sred[1][0] + sred[1][1] + sred[1][2] + sred[1][3];
+  float acc = 0.f;
+  for (int s0 = 0; s0 < S; s0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = (s0 + e < S) ? __ldcg(p.ws_o + (base + s0 + e) * D + d) : 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (s0 + e < S) acc += sw[s0 + e] * v[e];
   }
   const float r = lsum > 0.f ? __fdiv_rn(acc, lsum) : 0.f;
   const int64_t o = ((int64_t)b * p.num_q_heads + hq) * D + d;

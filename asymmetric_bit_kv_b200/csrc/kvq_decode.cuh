@@ -15,11 +15,9 @@ namespace kvq {
 //    kResChunk (one chunk even for an empty sequence); the work items of all
 //    units, concatenated in (sequence, head, item) order, are cut into
 //    num_ctas contiguous ranges (CTA c takes [c*T/num_ctas, (c+1)*T/num_ctas)),
-//    and slot kMmaConsumers*(c - c0) + w holds what consumer warp w of CTA c
-//    processed for the unit, c0 being the unit's first CTA. Every writer of a
-//    slot then counts itself in unit_ctr; the warp that writes a unit's last
-//    slot merges all of them (log-sum-exp) into the output and resets the
-//    counter to 0, so no separate combine launch is needed.
+//    and slot kMmaConsumers*(c - c0) + w holds what warp w of CTA c processed
+//    for the unit, c0 being the unit's first CTA; every warp writes its slot
+//    of every unit its CTA's range touches (zero weight if it had no items).
 struct DecodeParams {
   LayerView L;
   const void* q;        // [batch][Hq][D], kv dtype
@@ -33,7 +31,6 @@ struct DecodeParams {
   int32_t blocks_per_split;
   int32_t slots;        // partial slots per (sequence, query head)
   int32_t* err;         // device word: a kernel sets bit 0 when a bounded wait gave up
-  int32_t* unit_ctr;    // persistent mode: [batch][Hkv] partials written so far this call (0 between calls)
   int32_t persistent;   // 1: persistent-mode slots (see above)
   int32_t total_blocks; // T, persistent mode: work items of all units
   int32_t num_ctas;     // persistent mode
@@ -105,7 +102,7 @@ cudaError_t launch_decode_mma(const DecodeParams& p, const MmaPlan& mp, cudaStre
 // sequence (from the host mirror).
 cudaError_t launch_decode(const DecodeParams& p, int max_splits, cudaStream_t stream);
 
-// The log-sum-exp combine alone (after launch_decode_mma).
+// The log-sum-exp combine of the partial slots (after launch_decode_mma).
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream);
 
 // Device memory for the split partials other than the arena's workspace.

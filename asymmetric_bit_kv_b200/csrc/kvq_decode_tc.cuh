@@ -31,10 +31,9 @@
 //  * Ring chunks use bf16 (or f16) m16n8k16 directly on the ring values, with
 //    the query and the probabilities split into high and low parts, into the
 //    same accumulators as the unit's blocks.
-//  * Every warp's partial (o, m, l) of a unit is counted in a per-unit
-//    arrival counter; the warp writing a unit's last partial merges them
-//    (log-sum-exp) into the output. mbarrier waits are bounded (~2 s) and set
-//    the device error word instead of hanging.
+//  * Every warp writes one partial (o, m, l) per unit it passes through; the
+//    log-sum-exp combine kernel merges them. mbarrier waits are bounded
+//    (~2 s) and set the device error word instead of hanging.
 #pragma once
 
 #include "kvq_decode.cuh"
@@ -207,132 +206,6 @@ template <int KB>
 __device__ __forceinline__ int tile_token(int mt, int r) {
   constexpr int CPT16 = 16 / KB, TOKC = 128 / KB, JP = CPT16 / 2;
   return (mt / JP) * TOKC + (r & 7) * CPT16 + 2 * (mt % JP) + (r >> 3);
-}
-
-// The fields of DecodeParams that the out-of-line helpers below need,
-// passed by value: the kernel's parameter block itself (4 KB with the
-// per-sequence tables) must not have its address taken, or it is copied to
-// the stack.
-struct PartialOut {
-  float* ws_o;
-  float2* ws_ml;
-  void* out;
-  int32_t out_dtype;
-  int32_t num_q_heads;
-  int32_t slots;
-  float scale_log2;
-};
-__device__ __forceinline__ PartialOut partial_out(const DecodeParams& p) {
-  return PartialOut{p.ws_o, p.ws_ml, p.out, p.out_dtype, p.num_q_heads, p.slots, p.scale_log2};
-}
-
-// ------------------------------------------------------ fused LSE combine
-// Merges the nslots partials of unit (b, h) into out[b][h*NG + hh][:]:
-// M = max_s m_s, out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s, empty
-// slots (l = 0, o finite) weighted 0, rounded to the output dtype (nearest
-// even). One warp: lane l owns channels 4l..4l+3 of every head (at most
-// kMaxNG); the loads of SB slots of all heads are issued together. Partials
-// written by other SMs are read through L2 (ld.global.cg).
-template <int kMaxNG>
-static __device__ __noinline__ void combine_unit(const PartialOut p, int b, int h, int NG, int nslots, int lane) {
-  constexpr int D = kHeadDim;
-  constexpr int SB = 16 / kMaxNG;
-  const int64_t base = ((int64_t)b * p.num_q_heads + h * NG) * p.slots;  // head hh: + hh * slots
-  float M[kMaxNG], lsum[kMaxNG];
-  float4 acc[kMaxNG];
-#pragma unroll
-  for (int hh = 0; hh < kMaxNG; ++hh) {
-    M[hh] = -INFINITY;
-    lsum[hh] = 0.f;
-    acc[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  for (int s0 = 0; s0 < nslots; s0 += 32) {  // running maxima
-#pragma unroll
-    for (int hh = 0; hh < kMaxNG; ++hh) {
-      if (hh < NG && s0 + lane < nslots) {
-        const float2 ml = __ldcg(p.ws_ml + base + (int64_t)hh * p.slots + s0 + lane);
-        if (ml.y > 0.f) M[hh] = fmaxf(M[hh], ml.x);
-      }
-    }
-  }
-#pragma unroll
-  for (int hh = 0; hh < kMaxNG; ++hh)
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) M[hh] = fmaxf(M[hh], __shfl_xor_sync(0xffffffffu, M[hh], off));
-  for (int s0 = 0; s0 < nslots; s0 += 32) {
-    float w[kMaxNG];  // weight of slot s0 + lane, per head
-#pragma unroll
-    for (int hh = 0; hh < kMaxNG; ++hh) {
-      w[hh] = 0.f;
-      if (hh < NG && s0 + lane < nslots && M[hh] != -INFINITY) {
-        const float2 ml = __ldcg(p.ws_ml + base + (int64_t)hh * p.slots + s0 + lane);
-        if (ml.y > 0.f) {
-          w[hh] = exp2f(ml.x - M[hh]);
-          lsum[hh] += ml.y * w[hh];
-        }
-      }
-    }
-    const int cnt = min(32, nslots - s0);
-    for (int i0 = 0; i0 < cnt; i0 += SB) {
-      float4 o[SB][kMaxNG];
-#pragma unroll
-      for (int e = 0; e < SB; ++e)
-#pragma unroll
-        for (int hh = 0; hh < kMaxNG; ++hh)
-          o[e][hh] = (hh < NG && i0 + e < cnt)
-                         ? __ldcg(reinterpret_cast<const float4*>(p.ws_o + (base + (int64_t)hh * p.slots + s0 + i0 + e) * D) + lane)
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int e = 0; e < SB; ++e) {
-#pragma unroll
-        for (int hh = 0; hh < kMaxNG; ++hh) {
-          const float wi = __shfl_sync(0xffffffffu, w[hh], (i0 + e) & 31);
-          acc[hh].x += wi * o[e][hh].x;
-          acc[hh].y += wi * o[e][hh].y;
-          acc[hh].z += wi * o[e][hh].z;
-          acc[hh].w += wi * o[e][hh].w;
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int hh = 0; hh < kMaxNG; ++hh) {
-    if (hh >= NG) break;
-    float l = lsum[hh];
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-    float r[4] = {acc[hh].x, acc[hh].y, acc[hh].z, acc[hh].w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) r[e] = l > 0.f ? __fdiv_rn(r[e], l) : 0.f;
-    const int64_t o = ((int64_t)b * p.num_q_heads + h * NG + hh) * D + 4 * lane;
-    if (p.out_dtype == KVQ_F32) {
-      *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + o) = make_float4(r[0], r[1], r[2], r[3]);
-    } else if (p.out_dtype == KVQ_BF16) {
-      *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) + o) =
-          make_uint2(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]));
-    } else {
-      *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(p.out) + o) =
-          make_uint2(pack_f16(r[0], r[1]), pack_f16(r[2], r[3]));
-    }
-  }
-}
-
-// After this warp wrote one partial slot of unit (b, h): count it, and if it
-// was the unit's last one, merge the unit and reset its counter.
-template <int kMaxNG>
-__device__ __forceinline__ void arrive_unit(const DecodeParams& p, int b, int h, int NG, int lane) {
-  const LayerView& L = p.L;
-  __threadfence();  // this lane's partial stores before the count
-  __syncwarp();
-  const int u = b * L.num_kv_heads + h;
-  int old = 0;
-  if (lane == 0) old = atomicAdd(p.unit_ctr + u, 1);
-  old = __shfl_sync(0xffffffffu, old, 0);
-  const int nslots = persistent_slots(p.total_blocks, p.num_ctas, p.seq_start[b] + h * p.nitem[b], p.nitem[b]);
-  if (old != nslots - 1) return;
-  __threadfence();  // every other writer's partial is visible from here on
-  combine_unit<kMaxNG>(partial_out(p), b, h, NG, nslots, lane);
-  if (lane == 0) atomicExch(p.unit_ctr + u, 0);
 }
 
 // ------------------------------------------------------- residual ring chunks
@@ -862,7 +735,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
         if (v0) p.ws_ml[base0] = make_float2(sst.m0, sst.l0);
         if (v1) p.ws_ml[base1] = make_float2(sst.m1, sst.l1);
       }
-      arrive_unit<4 * NKT>(p, u.b, u.h, NG, lane);
       k = hi;
     }
   }

@@ -128,9 +128,8 @@ KVQ_API kvq_status kvq_cache_required_bytes(const kvq_config* cfg, size_t* bytes
 
 /* Validate cfg and bind a cache to dev_arena (device pointer, 256-byte
  * aligned, arena_bytes >= required), with the arena's device current. Every
- * sequence starts empty: the call zeroes the arena's length table, decode
- * arrival counters and residual rings, and waits for that to finish before
- * it returns.                                                              */
+ * sequence starts empty: the call zeroes the arena's length table and
+ * residual rings, and waits for that to finish before it returns.          */
 KVQ_API kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena_bytes,
                             kvq_cache** out);
 
