@@ -174,16 +174,15 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
 // M = max_s m_s over slots with l_s > 0, out = sum_s 2^(m_s-M) o_s / sum_s
 // 2^(m_s-M) l_s, rounded to the output dtype (nearest even); a sequence with
 // no tokens gives zeros. grid (Hq, batch), block D threads (thread d owns
-// channel d). The slots' (m, l) pass through shared memory once; each thread
-// then issues its slot loads eight at a time.
-constexpr int kCombineMaxSlots = 512;
-
+// channel d). Every thread issues the (m, l) and o loads of 16 slots at once
+// and merges them online, so a typical merge takes one round trip to L2.
 __global__ void __launch_bounds__(128) combine_kernel(DecodeParams p) {
-  __shared__ float sw[kCombineMaxSlots];  // slot weights 2^(m_s - M), 0 for empty slots
-  __shared__ float sred[2][4];
-  const int hq = blockIdx.x, b = blockIdx.y, d = threadIdx.x, lane = d & 31, warp = d >> 5;
+  // wait for the decode grid this launch depends on (no-op without one)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int hq = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const LayerView& L = p.L;
   constexpr int D = kHeadDim;
+  constexpr int C = 16;  // slots per batch of loads
   int S;  // slots of this (sequence, head)
   if (p.persistent) {
     const int h = hq / (p.num_q_heads / L.num_kv_heads);
@@ -192,38 +191,34 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeParams p) {
     const int nblk = L.lens[2 * b] / L.group_k;
     S = (nblk + p.blocks_per_split - 1) / p.blocks_per_split + 1;
   }
-  S = min(S, kCombineMaxSlots);
   const int64_t base = ((int64_t)b * p.num_q_heads + hq) * p.slots;
-  float m = -INFINITY;
-  for (int s = d; s < S; s += D) {
-    const float2 ml = __ldcg(p.ws_ml + base + s);
-    if (ml.y > 0.f) m = fmaxf(m, ml.x);
-  }
+  float M = -INFINITY, acc = 0.f, lsum = 0.f;
+  for (int s0 = 0; s0 < S; s0 += C) {
+    float2 ml[C];
+    float v[C];
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  if (lane == 0) sred[0][warp] = m;
-  __syncthreads();
-  const float M = fmaxf(fmaxf(sred[0][0], sred[0][1]), fmaxf(sred[0][2], sred[0][3]));
-  float lpart = 0.f;
-  for (int s = d; s < S; s += D) {
-    const float2 ml = __ldcg(p.ws_ml + base + s);
-    const float w = (ml.y > 0.f && M != -INFINITY) ? exp2f(ml.x - M) : 0.f;
-    sw[s] = w;
-    lpart += w * ml.y;
-  }
+    for (int e = 0; e < C; ++e) {
+      const bool in = s0 + e < S;
+      ml[e] = in ? __ldcg(p.ws_ml + base + s0 + e) : make_float2(-INFINITY, 0.f);
+      v[e] = in ? __ldcg(p.ws_o + (base + s0 + e) * D + d) : 0.f;
+    }
+    float mc = M;
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) lpart += __shfl_xor_sync(0xffffffffu, lpart, off);
-  if (lane == 0) sred[1][warp] = lpart;
-  __syncthreads();
-  const float lsum = sred[1][0] + sred[1][1] + sred[1][2] + sred[1][3];
-  float acc = 0.f;
-  for (int s0 = 0; s0 < S; s0 += 8) {
-    float v[8];
+    for (int e = 0; e < C; ++e)
+      if (ml[e].y > 0.f) mc = fmaxf(mc, ml[e].x);
+    if (mc == -INFINITY) continue;  // nothing yet
+    const float r = M == -INFINITY ? 0.f : exp2f(M - mc);
+    acc *= r;
+    lsum *= r;
+    M = mc;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = (s0 + e < S) ? __ldcg(p.ws_o + (base + s0 + e) * D + d) : 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-      if (s0 + e < S) acc += sw[s0 + e] * v[e];
+    for (int e = 0; e < C; ++e) {
+      if (ml[e].y > 0.f) {
+        const float w = exp2f(ml[e].x - M);
+        acc += w * v[e];
+        lsum += w * ml[e].y;
+      }
+    }
   }
   const float r = lsum > 0.f ? __fdiv_rn(acc, lsum) : 0.f;
   const int64_t o = ((int64_t)b * p.num_q_heads + hq) * D + d;
@@ -258,8 +253,20 @@ cudaError_t launch_decode(const DecodeParams& p, int max_splits, cudaStream_t st
 
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream) {
   if (p.batch <= 0) return cudaSuccess;
-  combine_kernel<<<dim3(p.num_q_heads, p.batch), kHeadDim, 0, stream>>>(p);
-  return cudaGetLastError();
+  // Programmatic dependent launch: the combine grid may be scheduled while
+  // the decode grid (which allows it at its start) is still running; each
+  // combine CTA waits for the decode grid to complete before it reads.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.num_q_heads, p.batch);
+  cfg.blockDim = dim3(kHeadDim);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = p.persistent ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, p);
 }
 
 }  // namespace kvq

@@ -528,6 +528,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
   const int rs = cta_first_block(T, p.num_ctas, c), re = cta_first_block(T, p.num_ctas, c + 1);
   const bool bf16 = L.kv_dtype == KVQ_BF16;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the combine launch that follows may be scheduled from now on; it waits
+  // for this grid to complete before reading any partial
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // this warp's items: rs + warp + n*kNC, n = 0, 1, ...; item n lands in the
   // warp's own stage n % SPW, and the warp issues item n + SPW as soon as it
   // is done with item n
