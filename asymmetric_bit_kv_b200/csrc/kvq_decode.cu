@@ -176,19 +176,18 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
 // no tokens gives zeros. grid (Hq, batch), block D threads (thread d owns
 // channel d). Every thread issues the (m, l) and o loads of 16 slots at once
 // and merges them online, so a typical merge takes one round trip to L2.
-__global__ void __launch_bounds__(128) combine_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(128) combine_kernel(CombineParams p) {
   // wait for the decode grid this launch depends on (no-op without one)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int hq = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
-  const LayerView& L = p.L;
   constexpr int D = kHeadDim;
   constexpr int C = 16;  // slots per batch of loads
   int S;  // slots of this (sequence, head)
   if (p.persistent) {
-    const int h = hq / (p.num_q_heads / L.num_kv_heads);
-    S = persistent_slots(p.total_blocks, p.num_ctas, p.seq_start[b] + h * p.nitem[b], p.nitem[b]);
+    const int h = hq / (p.num_q_heads / p.num_kv_heads);
+    S = __ldcg(p.unit_slots + b * p.num_kv_heads + h);
   } else {
-    const int nblk = L.lens[2 * b] / L.group_k;
+    const int nblk = p.lens[2 * b] / p.group_k;
     S = (nblk + p.blocks_per_split - 1) / p.blocks_per_split + 1;
   }
   const int64_t base = ((int64_t)b * p.num_q_heads + hq) * p.slots;
@@ -266,7 +265,10 @@ cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = p.persistent ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, combine_kernel, p);
+  const CombineParams cp{p.ws_o,         p.ws_ml,          p.out,           p.unit_slots,
+                         p.L.lens,       p.out_dtype,      p.num_q_heads,   p.L.num_kv_heads,
+                         p.slots,        p.L.group_k,      p.blocks_per_split, p.persistent};
+  return cudaLaunchKernelEx(&cfg, combine_kernel, cp);
 }
 
 }  // namespace kvq

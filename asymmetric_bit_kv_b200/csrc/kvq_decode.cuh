@@ -14,10 +14,13 @@ namespace kvq {
 //    unit is its quantized blocks followed by its ring tokens in chunks of
 //    kResChunk (one chunk even for an empty sequence); the work items of all
 //    units, concatenated in (sequence, head, item) order, are cut into
-//    num_ctas contiguous ranges (CTA c takes [c*T/num_ctas, (c+1)*T/num_ctas)),
+//    num_ctas contiguous ranges of about equal estimated cost (CTA c takes
+//    [cta_start[c], cta_start[c+1]), every range non-empty),
 //    and slot kMmaConsumers*(c - c0) + w holds what warp w of CTA c processed
 //    for the unit, c0 being the unit's first CTA; every warp writes its slot
 //    of every unit its CTA's range touches (zero weight if it had no items).
+constexpr int kMaxCtas = 1024;  // persistent mode: CTAs of one decode launch
+
 struct DecodeParams {
   LayerView L;
   const void* q;        // [batch][Hq][D], kv dtype
@@ -31,6 +34,7 @@ struct DecodeParams {
   int32_t blocks_per_split;
   int32_t slots;        // partial slots per (sequence, query head)
   int32_t* err;         // device word: a kernel sets bit 0 when a bounded wait gave up
+  int32_t* unit_slots;  // persistent mode: [batch][Hkv] slot count of each unit, written by the decode kernel
   int32_t persistent;   // 1: persistent-mode slots (see above)
   int32_t total_blocks; // T, persistent mode: work items of all units
   int32_t num_ctas;     // persistent mode
@@ -38,6 +42,7 @@ struct DecodeParams {
   int32_t nres[KVQ_MAX_BATCH];       // ring tokens per sequence (host mirror)
   int32_t nitem[KVQ_MAX_BATCH];      // persistent mode: work items per unit of sequence b
   int32_t seq_start[KVQ_MAX_BATCH];  // first global item (block in split mode) of sequence b
+  int32_t cta_start[kMaxCtas + 1];   // persistent mode: first global item of CTA c (cut by estimated cost)
 };
 
 constexpr int kMmaConsumers = 6;   // warps per CTA of the tensor-core kernel
@@ -49,27 +54,23 @@ __host__ __device__ inline int32_t unit_items(int32_t nblk, int32_t nres) {
   return items > 0 ? items : 1;
 }
 
-// Persistent mode: first global block of CTA c, and the CTA holding block k.
-__host__ __device__ inline int32_t cta_first_block(int64_t T, int32_t nctas, int32_t c) {
-  return (int32_t)((int64_t)c * T / nctas);
-}
-__host__ __device__ inline int32_t cta_of_block(int64_t T, int32_t nctas, int32_t k) {
-#ifdef __CUDA_ARCH__
-  int32_t c = (int32_t)((int64_t)k * nctas / T);
-#else
-  int32_t c = (int32_t)((double)k * nctas / (double)T);  // a guess, corrected below
-  if (c < 0) c = 0;
-  if (c >= nctas) c = nctas - 1;
-#endif
-  while (c + 1 < nctas && cta_first_block(T, nctas, c + 1) <= k) ++c;
-  while (c > 0 && cta_first_block(T, nctas, c) > k) --c;
-  return c;
+// Persistent mode: the CTA whose item range [starts[c], starts[c+1]) holds
+// item k (starts strictly increasing, starts[0] = 0).
+__host__ __device__ inline int32_t cta_of_item(const int32_t* starts, int32_t nctas, int32_t k) {
+  int32_t lo = 0, hi = nctas - 1;
+  while (lo < hi) {
+    const int32_t mid = (lo + hi + 1) >> 1;
+    if (starts[mid] <= k) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
 }
 // Number of partial slots a (sequence, head) unit of nitem >= 1 work items
-// uses in persistent mode.
-__host__ __device__ inline int32_t persistent_slots(int64_t T, int32_t nctas, int32_t unit_start, int32_t nitem) {
-  const int32_t c0 = cta_of_block(T, nctas, unit_start);
-  const int32_t c1 = cta_of_block(T, nctas, unit_start + nitem - 1);
+// starting at global item unit_start uses in persistent mode.
+__host__ __device__ inline int32_t persistent_slots(const int32_t* starts, int32_t nctas, int32_t unit_start,
+                                                    int32_t nitem) {
+  const int32_t c0 = cta_of_item(starts, nctas, unit_start);
+  const int32_t c1 = cta_of_item(starts, nctas, unit_start + nitem - 1);
   return kMmaConsumers * (c1 - c0 + 1);
 }
 
@@ -102,7 +103,17 @@ cudaError_t launch_decode_mma(const DecodeParams& p, const MmaPlan& mp, cudaStre
 // sequence (from the host mirror).
 cudaError_t launch_decode(const DecodeParams& p, int max_splits, cudaStream_t stream);
 
-// The log-sum-exp combine of the partial slots (after launch_decode_mma).
+// Parameters of the log-sum-exp combine (small: no per-sequence tables).
+struct CombineParams {
+  const float* ws_o;
+  const float2* ws_ml;
+  void* out;
+  const int32_t* unit_slots;  // persistent mode: slots per unit
+  const int32_t* lens;        // split mode: the layer's length table
+  int32_t out_dtype, num_q_heads, num_kv_heads, slots, group_k, blocks_per_split, persistent;
+};
+
+// The log-sum-exp combine of the partial slots (after the decode kernel).
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream);
 
 // Device memory for the split partials other than the arena's workspace.

@@ -85,6 +85,10 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// L2 prefetch of a global range (16-byte multiple), no shared-memory target.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 // ldmatrix keeps a memory clobber so that it stays behind the barrier waits
 // that publish the shared memory it reads; the arithmetic asm is free to move.
 __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -499,6 +503,13 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, const MmaPlan&
   if (j < nb) {
     mbar_expect_tx(bar, mp.tx_bytes + (newq ? qbytes : 0u));
     bulk_g2s(dst, record_ptr(L, u.b, u.h, j), mp.tx_bytes, bar);
+    if (j == nb - 1 && p.nres[u.b] > 0) {
+      // the unit's ring chunks come next: bring its ring rows into L2 so that
+      // those short items do not each wait a full HBM round trip
+      const int64_t ring = ((int64_t)u.b * L.num_kv_heads + u.h) * L.residual * kRowBytes;
+      bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(L.ring_k) + ring, L.residual * kRowBytes);
+      bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(L.ring_v) + ring, L.residual * kRowBytes);
+    }
   } else {
     // ring chunk: kResChunk consecutive slots of keys, then of values
     const int slot = (nb * L.group_k + (j - nb) * kResChunk) % L.residual;
@@ -524,8 +535,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
   const int Hkv = L.num_kv_heads;
   const int NG = p.num_q_heads / Hkv;
   const int G = L.group_k;
-  const int T = p.total_blocks;
-  const int rs = cta_first_block(T, p.num_ctas, c), re = cta_first_block(T, p.num_ctas, c + 1);
+  const int rs = p.cta_start[c], re = p.cta_start[c + 1];
   const bool bf16 = L.kv_dtype == KVQ_BF16;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // the combine launch that follows may be scheduled from now on; it waits
@@ -719,7 +729,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
         sst.l0 += __shfl_xor_sync(0xffffffffu, sst.l0, off);
         sst.l1 += __shfl_xor_sync(0xffffffffu, sst.l1, off);
       }
-      const int slot = kNC * (c - cta_of_block(T, p.num_ctas, u.start)) + warp;
+      const int c0 = cta_of_item(p.cta_start, p.num_ctas, u.start);
+      const int slot = kNC * (c - c0) + warp;
+      if (slot == 0 && lane == 0)  // the unit's slot count, for the combine kernel
+        p.unit_slots[u.b * Hkv + u.h] = kNC * (cta_of_item(p.cta_start, p.num_ctas, u.end - 1) - c0 + 1);
       const int64_t base0 = ((int64_t)u.b * p.num_q_heads + u.h * NG + 2 * t) * p.slots + slot;
       const int64_t base1 = base0 + p.slots;
 #pragma unroll
