@@ -57,6 +57,25 @@ def _dist_env():
     return rank, world, local
 
 
+def cross_rank_max(values, world, device):
+    """Per-rank timings -> their maximum over all ranks (every rank gets it).
+    Multi-GPU numbers are the slowest rank's (weak scaling: each rank times
+    its own replicas)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def replica_seed(rank, r):
+    """Seed offset of cache replica r on `rank`: every rank draws its own data."""
+    return 1000 * rank + r
+
+
 def _peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -256,7 +275,7 @@ def run_kvq(a):
     caches = []
     for r in range(R):
         c = KVCache(cfg, dev)
-        k, v = W.generate_tokens(wl, 0, [ctx] * B, device=dev, seed_offset=1000 * rank + r)
+        k, v = W.generate_tokens(wl, 0, [ctx] * B, device=dev, seed_offset=replica_seed(rank, r))
         c.append(0, k, v, [ctx] * B)
         del k, v
         caches.append(c)
@@ -313,7 +332,7 @@ def run_kvq(a):
     plan = []  # (replica, launches, algorithmic bytes of the decode, KV tokens attended)
     for i in range(a.steps):
         r = (a.warmup + i) % R
-        launches = 2 + (1 if lens[r][0][1] == Rw else 0)  # ring write + decode (+ flush)
+        launches = 3 + (1 if lens[r][0][1] == Rw else 0)  # ring write + decode + combine (+ flush)
         ab, tk = 2 * B * Hq * D * 2, 0  # q in, out
         for b in range(B):
             qn, n = lens[r][b]
@@ -351,10 +370,7 @@ def run_kvq(a):
             assert tuple(lens[r][b]) == caches[r].lengths(0, b), "step accounting out of sync with the cache"
     ms = e0.elapsed_time(e1)
     dec_ms = sum(x[0].elapsed_time(x[1]) for x in events)
-    if world > 1:
-        t = torch.tensor([ms, dec_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, dec_ms = float(t[0]), float(t[1])
+    ms, dec_ms = cross_rank_max([ms, dec_ms], world, dev)
     value = tok_total * world / (ms / 1e3)
     achieved_gbs = alg_total / (dec_ms / 1e3) / 1e9
 
@@ -396,10 +412,7 @@ def run_kvq(a):
     f1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = f0.elapsed_time(f1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    e2e_ms, = cross_rank_max([e2e_ms], world, dev)
     e2e_value = tok_e2e * world / (e2e_ms / 1e3)
 
     result = None
