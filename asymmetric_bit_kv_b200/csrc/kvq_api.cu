@@ -324,6 +324,17 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out,
   p.ws_o = reinterpret_cast<float*>(c->arena + c->ws_o_off);
   p.ws_ml = reinterpret_cast<float2*>(c->arena + c->ws_ml_off);
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  // the tensor-core kernel multiplies fp16 queries by fp16 key scales: a power
+  // of two near scale_log2 keeps those products as far from the fp16 limit as
+  // the scaled query would, exactly; the rest of the scale is applied to the
+  // fp32 scores
+  int scale_exp = 0;  // |scale_log2| in [2^scale_exp, 2^(scale_exp+1))
+  if (p.scale_log2 != 0.f) {
+    (void)std::frexp(std::fabs(p.scale_log2), &scale_exp);
+    scale_exp -= 1;
+  }
+  p.q_prescale = std::ldexp(1.f, std::min(0, std::max(-8, scale_exp)));
+  p.score_scale = p.scale_log2 / p.q_prescale;
   p.out_dtype = out_dtype;
   p.batch = batch;
   p.num_q_heads = cfg.num_q_heads;

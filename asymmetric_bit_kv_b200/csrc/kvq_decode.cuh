@@ -28,6 +28,8 @@ struct DecodeParams {
   float* ws_o;          // [max_batch][Hq][slots][D] unnormalised partial outputs
   float2* ws_ml;        // [max_batch][Hq][slots]: (running max in log2 units, sum)
   float scale_log2;     // softmax scale * log2(e)
+  float q_prescale;     // tensor-core kernel: power of two the queries are scaled by in fp16
+  float score_scale;    // scale_log2 / q_prescale
   int32_t out_dtype;
   int32_t batch;
   int32_t num_q_heads;

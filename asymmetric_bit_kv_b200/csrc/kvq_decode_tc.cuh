@@ -17,17 +17,20 @@
 //    as the warp is done with it, so no warp ever waits on another.
 //  * Quantized keys, tokens on M: S[token][col] = codes x (q*s). ldmatrix
 //    .trans over the channel-major key rows gives each thread two channels
-//    of 16/kb tokens in one register; one lop3 (mask | fp16 exponent 2^(10-p))
-//    and one hsub2 turn the code at bit position p into an exact fp16
-//    integer, the A operand. The B operand is q*s per channel, fp16 high and
-//    low parts in two columns per head (or two n-tiles for 8 heads), rebuilt
-//    per block from the block's fp16 scales.
+//    of 16/kb tokens in one register; one AND leaves the code at bit
+//    position p as the fp16 subnormal code * 2^(p-24), exact, the A operand
+//    (p depends only on the A row, whose accumulator is scaled back by
+//    2^(24-p)). The B operand is q*s per channel, fp16 high and low parts in
+//    two columns per head (or two n-tiles for 8 heads), rebuilt per block
+//    from the block's fp16 scales.
 //  * Probabilities: after the online softmax (log2 units) each thread holds
 //    P[token][two heads] in the m8n8 fragment layout; movmatrix.trans turns
 //    it into the B operand of P.V (tokens on K, heads on N).
 //  * Values: O[channel][head] = sum_t codes * (p*s) + sum_t p*z: value codes
 //    of two tokens per register from ldmatrix.trans over token rows (channels
-//    on M), the zero-point term one MMA per value group with an all-ones A.
+//    on M), as fp16 subnormals like the keys (the channel rows of O are
+//    scaled back when the partial is written), the zero-point term one MMA
+//    per value group with an all-ones A.
 //  * Ring chunks use bf16 (or f16) m16n8k16 directly on the ring values, with
 //    the query and the probabilities split into high and low parts, into the
 //    same accumulators as the unit's blocks.
@@ -126,13 +129,16 @@ __device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
-__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
-  __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
-  return *reinterpret_cast<uint32_t*>(&r);
-}
 __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
-  __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
-  return *reinterpret_cast<uint32_t*>(&r);
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+// a * b - c with one rounding.
+__device__ __forceinline__ uint32_t hfms2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("{\n\t.reg .b32 nc;\n\tneg.f16x2 nc, %3;\n\tfma.rn.f16x2 %0, %1, %2, nc;\n\t}" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
@@ -153,35 +159,32 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-// Code j (width B bits) of both 16-bit halves of a register, as exact fp16
-// integers. x8 = x >> 8 serves codes that sit in the upper byte of a half.
-// The code field at bit position p (0..7) of the low byte becomes the low
-// mantissa bits of 2^(10-p), whose mantissa bit p weighs exactly 1; or-ing
-// the exponent in and subtracting 2^(10-p) leaves the code.
+// Code j (width B bits) of both 16-bit halves of a register, as fp16
+// subnormals: masked in place at bit position p (0..7) of its byte, with the
+// exponent field zero, the code reads as the exact fp16 value code * 2^(p-24).
+// The MMAs thus multiply exact integers scaled by a power of two that depends
+// only on the code's index j, i.e. on the row of the A operand; the row's
+// accumulator is scaled back by 2^(24-p), exactly, where it is read. x8 =
+// x >> 8 serves codes that sit in the upper byte of a half. One instruction
+// per two codes.
 template <int B>
-__device__ __forceinline__ uint32_t code_at(uint32_t x, uint32_t x8, int j) {
+__device__ __forceinline__ uint32_t code_sub(uint32_t x, uint32_t x8, int j) {
   const int bit = B * j;
-  const int pos = bit & 7;
-  const uint32_t m = ((1u << B) - 1u) << pos;
-  const uint32_t e = (uint32_t)(25 - pos) << 10;
-  const uint32_t magic = e | (e << 16);
-  return hsub2(and_or(bit >= 8 ? x8 : x, m | (m << 16), magic), magic);
+  const uint32_t m = ((1u << B) - 1u) << (bit & 7);
+  return (bit >= 8 ? x8 : x) & (m | (m << 16));
 }
-// Code j as 2^(10-p) + code (the value code_at would return plus the magic
-// of its bit position p), one instruction; the offset is taken out later.
+// Bit position p of code j inside its byte, and 2^e as a float constant.
 template <int B>
-__device__ __forceinline__ uint32_t code_raw(uint32_t x, uint32_t x8, int j) {
-  const int bit = B * j;
-  const int pos = bit & 7;
-  const uint32_t m = ((1u << B) - 1u) << pos;
-  const uint32_t e = (uint32_t)(25 - pos) << 10;
-  return and_or(bit >= 8 ? x8 : x, m | (m << 16), e | (e << 16));
+__host__ __device__ constexpr int code_pos(int j) { return (B * j) & 7; }
+__host__ __device__ constexpr float pow2f(int e) {
+  float r = 1.f;
+  for (int i = 0; i < e; ++i) r *= 2.f;
+  for (int i = 0; i > e; --i) r *= 0.5f;
+  return r;
 }
-// fp16 pair (-2^(10-p), -2^(10-p)) for the bit position p of code j.
+// Row scale 2^(24-p) of the accumulator rows fed by code j.
 template <int B>
-__host__ __device__ constexpr uint32_t neg_magic2(int j) {
-  return ((0x8000u | ((uint32_t)(25 - ((B * j) & 7)) << 10)) * 0x10001u);
-}
+__host__ __device__ constexpr float code_unscale(int j) { return pow2f(24 - code_pos<B>(j)); }
 
 // Compile-time shape of one instance. A tile is 64 tokens of a block.
 template <int KB, int VB, int NGRP, int NKT>
@@ -264,11 +267,16 @@ struct UnitCursor {
 //         (n >= 4); with 8 heads n-tile 0 holds the high and n-tile 1 the low
 //         parts of heads 0-7. Columns of absent heads stay zero.
 //   bias  [8] float: sum_d q_d z_d per head (log2 units);
-//   qbuf  [nstages][NG][D] kv dtype: the queries of the warp's last units
-//         (one buffer per unit change, round robin), as stored in q.
-template <int NKT, bool BF16>
+//   qbuf  [nstages][NG][D]: the queries of the warp's last units (one buffer
+//         per unit change, round robin), copied in as stored in q and then
+//         converted in place to fp16 times q_prescale.
+// q (fp16, a power-of-two multiple of the query) times s (fp16) has at most
+// 22 significant bits, so the fp16 high part and the fp16 rounding of the
+// remainder (one fused multiply-subtract) hold it exactly; the softmax scale
+// is applied to the fp32 scores.
+template <int NKT>
 __device__ __forceinline__ void prep_block(const uint8_t* stage, const MmaPlan& mp, uint8_t* ws, const uint32_t* qw,
-                                           int NG, int lane, float scale_log2) {
+                                           int NG, int lane, float score_scale) {
   uint32_t* bk = reinterpret_cast<uint32_t*>(ws + mp.bfrag_off);
   const uint2* ksz2 = reinterpret_cast<const uint2*>(stage + mp.kc_bytes);  // (s, z) of channels 2c, 2c+1
   float* biasw = reinterpret_cast<float*>(ws + mp.bias_off);
@@ -279,17 +287,15 @@ __device__ __forceinline__ void prep_block(const uint8_t* stage, const MmaPlan& 
     float bp = 0.f;
     if (hh < NG) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int kk = i;
-        const float2 qf = BF16 ? unpack_bf16(qw[hh * 64 + 8 * kk + q]) : unpack_f16(qw[hh * 64 + 8 * kk + q]);
-        const uint2 sz = ksz2[8 * kk + q];  // channels 16kk + 2q, +1
-        const float2 c0 = unpack_f16(sz.x), c1 = unpack_f16(sz.y);
-        const float q0 = qf.x * scale_log2, q1 = qf.y * scale_log2;
-        const float x0 = q0 * c0.x, x1 = q1 * c1.x;
-        bp += q0 * c0.y + q1 * c1.y;
-        const uint32_t hi = pack_f16(x0, x1);
-        const float2 fh = unpack_f16(hi);
-        const uint32_t lo = pack_f16(x0 - fh.x, x1 - fh.y);
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t q2 = qw[hh * 64 + 8 * kk + q];  // channels 16kk + 2q, +1
+        const uint2 sz = ksz2[8 * kk + q];
+        const uint32_t s2 = __byte_perm(sz.x, sz.y, 0x5410), z2 = __byte_perm(sz.x, sz.y, 0x7632);
+        const float2 qf = unpack_f16(q2), zf = unpack_f16(z2);
+        bp = fmaf(qf.x, zf.x, bp);
+        bp = fmaf(qf.y, zf.y, bp);
+        const uint32_t hi = hmul2(q2, s2);
+        const uint32_t lo = hfms2(q2, s2, hi);
         if (NKT == 1) {
           bk[(kk * 32 + hh * 4 + tq) * 2 + half] = hi;
           bk[(kk * 32 + (hh + 4) * 4 + tq) * 2 + half] = lo;
@@ -302,7 +308,7 @@ __device__ __forceinline__ void prep_block(const uint8_t* stage, const MmaPlan& 
     bp += __shfl_xor_sync(0xffffffffu, bp, 1);
     bp += __shfl_xor_sync(0xffffffffu, bp, 2);
     bp += __shfl_xor_sync(0xffffffffu, bp, 4);
-    if (q == 0 && hh < NG) biasw[hh] = bp;
+    if (q == 0 && hh < NG) biasw[hh] = bp * score_scale;
   }
   __syncwarp();
 }
@@ -401,13 +407,16 @@ __device__ __forceinline__ float head_score(const float (&d)[NKT][4], int e) {
 // k-step kk (rows 8-15 absent); the B operand is the scaled query split
 // into kv-dtype high and low parts in the same channel order, written over
 // the warp's key B fragments (bk, same layout) on its first chunk of the unit
-// (a unit's ring chunks come after all of its quantized blocks). P.V: after movmatrix, lane (g, t) holds the
-// probabilities of tokens 2t, 2t+1 for head g; each output m-tile takes the
-// value word of its channels (ch0, ch0+1) from both tokens, paired by one
-// byte permute; two MMAs (probability high and low parts).
+// (a unit's ring chunks come after all of its quantized blocks; qw holds the
+// fp16 queries times q_prescale, and score_scale = scale_log2 / q_prescale).
+// P.V: after movmatrix, lane (g, t) holds the probabilities of tokens 2t,
+// 2t+1 for head g; each output m-tile takes the value word of its channels
+// (ch0, ch0+1) from both tokens, paired by one byte permute; two MMAs
+// (probability high and low parts) into a scratch accumulator, added to O at
+// the row scale of the quantized blocks' value codes (2^(p-24)).
 template <bool BF16, int VB, int NGRP, int NKT>
 __device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t* qw, uint2* bk, int cnt, int NG,
-                                           int lane, float scale_log2, bool v0, bool v1, bool& rq_ready,
+                                           int lane, float score_scale, bool v0, bool v1, bool& rq_ready,
                                            SoftState& sst, float (&O)[8][4], float (&Z)[NGRP][4]) {
   using S = Shape<2, VB, NGRP, NKT>;  // value-side constants only
   const int g = lane >> 2, t = lane & 3;
@@ -422,8 +431,8 @@ __device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t*
       for (int e = 0; e < 2; ++e) {
         const int w = 4 * t + 16 * (kk >> 1) + 2 * (kk & 1) + e;  // channels 2w, 2w+1
         const uint32_t raw = present ? qw[head * 64 + w] : 0u;
-        const float2 f = unpack_kv2<BF16>(raw);
-        const float x0 = f.x * scale_log2, x1 = f.y * scale_log2;
+        const float2 f = unpack_f16(raw);
+        const float x0 = f.x * score_scale, x1 = f.y * score_scale;
         hi[e] = pack_kv<BF16>(x0, x1);
         const float2 fh = unpack_kv2<BF16>(hi[e]);
         lo[e] = pack_kv<BF16>(x0 - fh.x, x1 - fh.y);
@@ -472,8 +481,14 @@ __device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t*
     const int w = (cch * S::CH_SPAN + g * S::VCPC) / 2 + P;
     const uint32_t x = V32[(2 * t) * 64 + w], y = V32[(2 * t + 1) * 64 + w];
     const uint32_t a[4] = {__byte_perm(x, y, 0x5410), __byte_perm(x, y, 0x7632), 0u, 0u};
-    mma_kv<BF16>(O[mt2], a, bh, 0u);
-    mma_kv<BF16>(O[mt2], a, bl, 0u);
+    float r[4] = {0.f, 0.f, 0.f, 0.f};
+    mma_kv<BF16>(r, a, bh, 0u);
+    mma_kv<BF16>(r, a, bl, 0u);
+    const float s0 = pow2f(code_pos<VB>(2 * P) - 24), s1 = pow2f(code_pos<VB>(2 * P + 1) - 24);
+    O[mt2][0] = fmaf(r[0], s0, O[mt2][0]);
+    O[mt2][1] = fmaf(r[1], s0, O[mt2][1]);
+    O[mt2][2] = fmaf(r[2], s1, O[mt2][2]);
+    O[mt2][3] = fmaf(r[3], s1, O[mt2][3]);
   }
 }
 
@@ -561,22 +576,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
   bool failed = false;
   int n = 0;  // items of this warp consumed so far
   {
-    {  // key B-fragment columns of absent heads stay zero
+    {  // key B-fragment columns and biases of absent heads stay zero
       uint4* z = reinterpret_cast<uint4*>(ws + mp.bfrag_off);
-      for (int e = lane; e < NKT * 8 * 32 * 8 / 16; e += 32) z[e] = make_uint4(0u, 0u, 0u, 0u);
+      for (int e = lane; e < (mp.bias_off + 32) / 16; e += 32) z[e] = make_uint4(0u, 0u, 0u, 0u);
       __syncwarp();
     }
     const int g = lane >> 2, t = lane & 3;
     const uint32_t ones[4] = {0x3c003c00u, 0x3c003c00u, 0x3c003c00u, 0x3c003c00u};  // fp16 1.0
-    // Value codes of 4 or 8 bits keep the magic offset 2^(10-p) of their bit
-    // position (one instruction per pair instead of two): rows g and g+8 of
-    // every channel m-tile then carry the same offsets, here codes 0 and 1 of
-    // a 16-bit column, and one more MMA per value group with the constant A
-    // operand -offset(row) against the same B (p*s) takes offset(row) * sum_t
-    // p*s back out, into the zero-point accumulator Z. (2-bit codes alternate
-    // between two offset pairs across m-tiles and subtract per pair instead.)
-    constexpr bool RAWV = VB != 2;
-    const uint32_t vneg[4] = {neg_magic2<VB>(0), neg_magic2<VB>(1), neg_magic2<VB>(0), neg_magic2<VB>(1)};
     const int kc_row = G * KB / 8;  // key code bytes per channel
     const int mi = lane >> 3, rr = lane & 7;
     // ldmatrix rows of this lane: 8 consecutive rows, so the chunk swizzle of
@@ -610,13 +616,21 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
           break;
         }
         const uint8_t* stage = stages + (size_t)st * mp.stage_bytes;
-        if (kb == first) ++qseq;  // the warp's first item of the unit brought its queries
-        const uint32_t* qw = reinterpret_cast<const uint32_t*>(qbuf + (size_t)(qseq % SPW) * NG * kRowBytes);
+        uint32_t* qw = reinterpret_cast<uint32_t*>(qbuf + (size_t)((qseq + (kb == first)) % SPW) * NG * kRowBytes);
+        if (kb == first) {
+          // the warp's first item of the unit brought its queries: to fp16
+          // times q_prescale, in place
+          ++qseq;
+          for (int w = lane; w < NG * (D / 2); w += 32) {
+            const float2 f = bf16 ? unpack_bf16(qw[w]) : unpack_f16(qw[w]);
+            qw[w] = pack_f16(f.x * p.q_prescale, f.y * p.q_prescale);
+          }
+          __syncwarp();
+        }
         const int j = kb - u.start;
         if (j < nb) {
           // ============ quantized block
-          if (bf16) prep_block<NKT, true>(stage, mp, ws, qw, NG, lane, p.scale_log2);
-          else prep_block<NKT, false>(stage, mp, ws, qw, NG, lane, p.scale_log2);
+          prep_block<NKT>(stage, mp, ws, qw, NG, lane, p.score_scale);
           const float bias0 = biasr[2 * t], bias1 = biasr[2 * t + 1];
           const uint32_t kc_s = smem_u32(stage);
           const uint32_t vc_s = smem_u32(stage + mp.vc_soff);
@@ -645,8 +659,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
                   const uint32_t xl = rk[2 * hf], xh = rk[2 * hf + 1], xl8 = xl >> 8, xh8 = xh >> 8;
 #pragma unroll
                   for (int jp = 0; jp < S::JP; ++jp) {
-                    const uint32_t a[4] = {code_at<KB>(xl, xl8, 2 * jp), code_at<KB>(xl, xl8, 2 * jp + 1),
-                                           code_at<KB>(xh, xh8, 2 * jp), code_at<KB>(xh, xh8, 2 * jp + 1)};
+                    const uint32_t a[4] = {code_sub<KB>(xl, xl8, 2 * jp), code_sub<KB>(xl, xl8, 2 * jp + 1),
+                                           code_sub<KB>(xh, xh8, 2 * jp), code_sub<KB>(xh, xh8, 2 * jp + 1)};
 #pragma unroll
                     for (int nt = 0; nt < NKT; ++nt)
                       mma_f16(Dk[sg * S::JP + jp][nt], a, bfr[hf][nt].x, bfr[hf][nt].y);
@@ -654,12 +668,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
                 }
               }
             }
-            // ---- online softmax over the tile
+            // ---- online softmax over the tile; row r of M-tile mt read code
+            // 2*(mt % JP) + r/8 of its column
             float sc[S::MT][4];
 #pragma unroll
             for (int mt = 0; mt < S::MT; ++mt)
 #pragma unroll
-              for (int e = 0; e < 4; ++e) sc[mt][e] = head_score<NKT>(Dk[mt], e) + ((e & 1) ? bias1 : bias0);
+              for (int e = 0; e < 4; ++e) {
+                const float rs = p.score_scale * code_unscale<KB>(2 * (mt % S::JP) + (e >> 1));
+                sc[mt][e] = fmaf(head_score<NKT>(Dk[mt], e), rs, (e & 1) ? bias1 : bias0);
+              }
             softmax_update<S::MT, NGRP, false>(sc, sst, v0, v1, O, Z);
             // ---- values: O += codes x (p * s), Z += ones x (p * z)
 #pragma unroll
@@ -675,7 +693,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
                 B0[gg] = hmul2(bt, v4.x);
                 B1[gg] = hmul2(bb, v4.y);
                 mma_f16(Z[gg], ones, hmul2(bt, v4.z), hmul2(bb, v4.w));
-                if constexpr (RAWV) mma_f16(Z[gg], vneg, B0[gg], B1[gg]);  // - offset(row) * sum_t p*s
               }
               const int sg = mt / S::JP, jp = mt % S::JP;
               const int vrow_idx = (2 * jp + (mi & 1)) * (G / S::CPT16) + tile * (S::TT / S::CPT16) + sg * 8 + rr;
@@ -690,18 +707,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
                   const int gg = ((cc0 + cc) * S::CH_SPAN) / S::GV;
 #pragma unroll
                   for (int P = 0; P < S::MT_PER_CH; ++P) {
-                    uint32_t a[4];
-                    if constexpr (RAWV) {
-                      a[0] = code_raw<VB>(xv, xv8, 2 * P);
-                      a[1] = code_raw<VB>(xv, xv8, 2 * P + 1);
-                      a[2] = code_raw<VB>(yv, yv8, 2 * P);
-                      a[3] = code_raw<VB>(yv, yv8, 2 * P + 1);
-                    } else {
-                      a[0] = code_at<VB>(xv, xv8, 2 * P);
-                      a[1] = code_at<VB>(xv, xv8, 2 * P + 1);
-                      a[2] = code_at<VB>(yv, yv8, 2 * P);
-                      a[3] = code_at<VB>(yv, yv8, 2 * P + 1);
-                    }
+                    const uint32_t a[4] = {code_sub<VB>(xv, xv8, 2 * P), code_sub<VB>(xv, xv8, 2 * P + 1),
+                                           code_sub<VB>(yv, yv8, 2 * P), code_sub<VB>(yv, yv8, 2 * P + 1)};
                     mma_f16(O[(cc0 + cc) * S::MT_PER_CH + P], a, B0[gg], B1[gg]);
                   }
                 }
@@ -710,10 +717,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
           }
         } else if (bf16) {
           ring_chunk<true, VB, NGRP, NKT>(stage, qw, bkw, p.nres[u.b] - (j - nb) * kResChunk, NG, lane,
-                                         p.scale_log2, v0, v1, rq_ready, sst, O, Z);
+                                         p.score_scale, v0, v1, rq_ready, sst, O, Z);
         } else {
           ring_chunk<false, VB, NGRP, NKT>(stage, qw, bkw, p.nres[u.b] - (j - nb) * kResChunk, NG, lane,
-                                          p.scale_log2, v0, v1, rq_ready, sst, O, Z);
+                                          p.score_scale, v0, v1, rq_ready, sst, O, Z);
         }
         // every lane is done with the stage: refill it with item n + SPW
         __syncwarp();
@@ -740,12 +747,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
         const int cch = mt2 / S::MT_PER_CH, P = mt2 % S::MT_PER_CH;
         const int gg = (cch * S::CH_SPAN) / S::GV;
         const int ch0 = cch * S::CH_SPAN + g * S::VCPC + 2 * P;
-        // rows g (channel ch0) and g+8 (ch0 + 1); Z holds the zero-point term
-        // (and the offset correction) per row
+        // rows g (channel ch0, code 2P of its column, held at 2^(p-24)) and
+        // g+8 (ch0 + 1, code 2P+1); Z holds the zero-point term per row
+        const float u0 = code_unscale<VB>(2 * P), u1 = code_unscale<VB>(2 * P + 1);
         if (v0)
-          *reinterpret_cast<float2*>(p.ws_o + base0 * D + ch0) = make_float2(O[mt2][0] + Z[gg][0], O[mt2][2] + Z[gg][2]);
+          *reinterpret_cast<float2*>(p.ws_o + base0 * D + ch0) =
+              make_float2(fmaf(O[mt2][0], u0, Z[gg][0]), fmaf(O[mt2][2], u1, Z[gg][2]));
         if (v1)
-          *reinterpret_cast<float2*>(p.ws_o + base1 * D + ch0) = make_float2(O[mt2][1] + Z[gg][1], O[mt2][3] + Z[gg][3]);
+          *reinterpret_cast<float2*>(p.ws_o + base1 * D + ch0) =
+              make_float2(fmaf(O[mt2][1], u0, Z[gg][1]), fmaf(O[mt2][3], u1, Z[gg][3]));
       }
       if (g == 0) {
         if (v0) p.ws_ml[base0] = make_float2(sst.m0, sst.l0);
