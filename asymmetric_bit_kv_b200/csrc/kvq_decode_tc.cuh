@@ -134,6 +134,16 @@ __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
+// acc + q.lo * z0 + q.hi * z1 (z0, z1: the high halves of sz0, sz1), each
+// product of two fp16 exact and added to the fp32 accumulator with one
+// rounding (mixed-precision fma).
+__device__ __forceinline__ float fma_q_z(uint32_t q, uint32_t sz0, uint32_t sz1, float acc) {
+  asm("{\n\t.reg .b16 ql, qh, s0, z0, s1, z1;\n\tmov.b32 {ql, qh}, %1;\n\tmov.b32 {s0, z0}, %2;\n\t"
+      "mov.b32 {s1, z1}, %3;\n\tfma.rn.f32.f16 %0, ql, z0, %0;\n\tfma.rn.f32.f16 %0, qh, z1, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(q), "r"(sz0), "r"(sz1));
+  return acc;
+}
 // a * b - c with one rounding.
 __device__ __forceinline__ uint32_t hfms2(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
@@ -263,17 +273,21 @@ struct UnitCursor {
 // from its fp16 scales (prep_block); the unit's queries arrive with the
 // warp's first item of the unit:
 //   bfrag [NKT][8 kk][32 lanes] uint2: key B fragments. Column n of the
-//         n-tile holds q*s of head n%4, fp16 high part (n < 4) or low part
-//         (n >= 4); with 8 heads n-tile 0 holds the high and n-tile 1 the low
+//         n-tile holds q*s of head n/2, fp16 high part (n even) or low part
+//         (n odd); with 8 heads n-tile 0 holds the high and n-tile 1 the low
 //         parts of heads 0-7. Columns of absent heads stay zero.
 //   bias  [8] float: sum_d q_d z_d per head (log2 units);
 //   qbuf  [nstages][NG][D]: the queries of the warp's last units (one buffer
 //         per unit change, round robin), copied in as stored in q and then
-//         converted in place to fp16 times q_prescale.
+//         converted in place to fp16 times q_prescale, the channel pair
+//         (2w, 2w+1) of head h at word h*64 + (w%8)*8 + w/8 (q_word), so that
+//         the eight pairs prep_block takes per lane are contiguous.
 // q (fp16, a power-of-two multiple of the query) times s (fp16) has at most
 // 22 significant bits, so the fp16 high part and the fp16 rounding of the
 // remainder (one fused multiply-subtract) hold it exactly; the softmax scale
 // is applied to the fp32 scores.
+__host__ __device__ constexpr int q_word(int h, int w) { return h * 64 + (w & 7) * 8 + (w >> 3); }
+
 template <int NKT>
 __device__ __forceinline__ void prep_block(const uint8_t* stage, const MmaPlan& mp, uint8_t* ws, const uint32_t* qw,
                                            int NG, int lane, float score_scale) {
@@ -286,19 +300,19 @@ __device__ __forceinline__ void prep_block(const uint8_t* stage, const MmaPlan& 
     const int hh = (lane >> 3) + 4 * rep;
     float bp = 0.f;
     if (hh < NG) {
+      const uint4* q4 = reinterpret_cast<const uint4*>(qw + q_word(hh, q));  // words of kk = 0..7
+      const uint4 qa = q4[0], qb = q4[1];
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t q2 = qw[hh * 64 + 8 * kk + q];  // channels 16kk + 2q, +1
+        const uint32_t q2 = word_of(kk < 4 ? qa : qb, kk & 3);  // channels 16kk + 2q, +1
         const uint2 sz = ksz2[8 * kk + q];
-        const uint32_t s2 = __byte_perm(sz.x, sz.y, 0x5410), z2 = __byte_perm(sz.x, sz.y, 0x7632);
-        const float2 qf = unpack_f16(q2), zf = unpack_f16(z2);
-        bp = fmaf(qf.x, zf.x, bp);
-        bp = fmaf(qf.y, zf.y, bp);
+        const uint32_t s2 = __byte_perm(sz.x, sz.y, 0x5410);
+        bp = fma_q_z(q2, sz.x, sz.y, bp);
         const uint32_t hi = hmul2(q2, s2);
         const uint32_t lo = hfms2(q2, s2, hi);
         if (NKT == 1) {
-          bk[(kk * 32 + hh * 4 + tq) * 2 + half] = hi;
-          bk[(kk * 32 + (hh + 4) * 4 + tq) * 2 + half] = lo;
+          bk[(kk * 32 + (2 * hh) * 4 + tq) * 2 + half] = hi;
+          bk[(kk * 32 + (2 * hh + 1) * 4 + tq) * 2 + half] = lo;
         } else {
           bk[(kk * 32 + hh * 4 + tq) * 2 + half] = hi;
           bk[((8 + kk) * 32 + hh * 4 + tq) * 2 + half] = lo;
@@ -314,65 +328,81 @@ __device__ __forceinline__ void prep_block(const uint8_t* stage, const MmaPlan& 
 }
 
 
-// Online-softmax update (log2 units) of this lane's two heads (2t and 2t+1)
-// with the scores sc of MTN M-tiles (registers 0/2: head 2t, rows g and g+8;
-// 1/3: head 2t+1). sc becomes the probabilities; O and Z are rescaled when a
-// running maximum grows. GUARD: scores may be -inf (absent tokens) and a
-// whole update may see none, and heads beyond NG are zeroed (ring chunks);
-// without it every score is finite, and heads beyond NG just compute finite
-// values in columns that are never written (quantized tiles).
+// Heads per lane of the score layout. With 8 query heads per KV head (two
+// key n-tiles: high parts, low parts) lane (g, t) holds heads 2t and 2t+1;
+// with at most 4 (one n-tile, columns 2h / 2h+1 = high / low part of head
+// h) it holds head t, both parts in its own two columns.
+template <int NKT>
+constexpr int heads_per_lane() { return NKT == 2 ? 2 : 1; }
+
+// Online-softmax state of this lane's heads (log2 units).
+template <int HPL>
 struct SoftState {
-  float m0, m1, l0, l1;
+  float m[HPL], l[HPL];
 };
-template <int MTN, int NGRP, bool GUARD>
-__device__ __forceinline__ void softmax_update(float (&sc)[MTN][4], SoftState& st, bool v0, bool v1,
-                                               float (&O)[8][4], float (&Z)[NGRP][4]) {
-  float mx0 = -INFINITY, mx1 = -INFINITY;
+
+// Key score of row r (0: g, 1: g+8) and lane head h of an M-tile's
+// accumulators: high part + low part.
+template <int NKT>
+__device__ __forceinline__ float head_score(const float (&d)[NKT][4], int r, int h) {
+  if constexpr (NKT == 2) return d[0][2 * r + h] + d[1][2 * r + h];
+  else return d[0][2 * r] + d[0][2 * r + 1];
+}
+
+// Online-softmax update of this lane's HPL heads with the scores of MTN
+// M-tiles, sc[mt][r * HPL + h] for row r (g, g+8) and lane head h; sc becomes
+// the probabilities; O and Z (columns = heads 2t, 2t+1) are rescaled when a
+// running maximum grows. GUARD: scores may be -inf (absent tokens), a whole
+// update may see none, and absent heads (valid false) are zeroed (ring
+// chunks); without it every score is finite, and absent heads just compute
+// finite values in columns that are never written (quantized tiles).
+template <int MTN, int HPL, int NGRP, bool GUARD>
+__device__ __forceinline__ void softmax_update(float (&sc)[MTN][2 * HPL], SoftState<HPL>& st,
+                                               const bool (&valid)[HPL], float (&O)[8][4], float (&Z)[NGRP][4],
+                                               int lane) {
+  float n[HPL], a[HPL];
 #pragma unroll
-  for (int mt = 0; mt < MTN; ++mt) {
-    mx0 = fmaxf(mx0, fmaxf(sc[mt][0], sc[mt][2]));
-    mx1 = fmaxf(mx1, fmaxf(sc[mt][1], sc[mt][3]));
-  }
+  for (int h = 0; h < HPL; ++h) {
+    float mx = -INFINITY;
 #pragma unroll
-  for (int off = 4; off <= 16; off <<= 1) {
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-  }
-  float n0, n1, a0, a1;
-  if constexpr (GUARD) {
-    // a head with no finite score so far keeps m = -inf, alpha = 1, p = 0
-    n0 = v0 ? fmaxf(st.m0, mx0) : -INFINITY;
-    n1 = v1 ? fmaxf(st.m1, mx1) : -INFINITY;
-    a0 = n0 == -INFINITY ? 1.f : ex2(st.m0 - n0);
-    a1 = n1 == -INFINITY ? 1.f : ex2(st.m1 - n1);
-  } else {
-    n0 = fmaxf(st.m0, mx0);
-    n1 = fmaxf(st.m1, mx1);
-    a0 = ex2(st.m0 - n0);  // 0 on the first tile (m = -inf)
-    a1 = ex2(st.m1 - n1);
-  }
-  st.m0 = n0;
-  st.m1 = n1;
-  float ps0 = 0.f, ps1 = 0.f;
+    for (int mt = 0; mt < MTN; ++mt) mx = fmaxf(mx, fmaxf(sc[mt][h], sc[mt][HPL + h]));
 #pragma unroll
-  for (int mt = 0; mt < MTN; ++mt) {
+    for (int off = 4; off <= 16; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     if constexpr (GUARD) {
-      sc[mt][0] = n0 == -INFINITY ? 0.f : ex2(sc[mt][0] - n0);
-      sc[mt][2] = n0 == -INFINITY ? 0.f : ex2(sc[mt][2] - n0);
-      sc[mt][1] = n1 == -INFINITY ? 0.f : ex2(sc[mt][1] - n1);
-      sc[mt][3] = n1 == -INFINITY ? 0.f : ex2(sc[mt][3] - n1);
+      // a head with no finite score so far keeps m = -inf, alpha = 1, p = 0
+      n[h] = valid[h] ? fmaxf(st.m[h], mx) : -INFINITY;
+      a[h] = n[h] == -INFINITY ? 1.f : ex2(st.m[h] - n[h]);
     } else {
-      sc[mt][0] = ex2(sc[mt][0] - n0);
-      sc[mt][2] = ex2(sc[mt][2] - n0);
-      sc[mt][1] = ex2(sc[mt][1] - n1);
-      sc[mt][3] = ex2(sc[mt][3] - n1);
+      n[h] = fmaxf(st.m[h], mx);
+      a[h] = ex2(st.m[h] - n[h]);  // 0 on the first tile (m = -inf)
     }
-    ps0 += sc[mt][0] + sc[mt][2];
-    ps1 += sc[mt][1] + sc[mt][3];
+    st.m[h] = n[h];
+    float ps = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < MTN; ++mt)
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        float& x = sc[mt][r * HPL + h];
+        if constexpr (GUARD) x = n[h] == -INFINITY ? 0.f : ex2(x - n[h]);
+        else x = ex2(x - n[h]);
+        ps += x;
+      }
+    st.l[h] = st.l[h] * a[h] + ps;
   }
-  st.l0 = st.l0 * a0 + ps0;
-  st.l1 = st.l1 * a1 + ps1;
-  if (!__all_sync(0xffffffffu, a0 == 1.f && a1 == 1.f)) {
+  bool same = true;
+#pragma unroll
+  for (int h = 0; h < HPL; ++h) same = same && a[h] == 1.f;
+  if (!__all_sync(0xffffffffu, same)) {
+    // alpha of the output columns (heads 2t, 2t+1) of this lane
+    float a0, a1;
+    if constexpr (HPL == 2) {
+      a0 = a[0];
+      a1 = a[1];
+    } else {
+      const int t = lane & 3, base = lane & ~3;
+      a0 = __shfl_sync(0xffffffffu, a[0], base + ((2 * t) & 3));
+      a1 = __shfl_sync(0xffffffffu, a[0], base + ((2 * t + 1) & 3));
+    }
 #pragma unroll
     for (int gg = 0; gg < NGRP; ++gg) {
       Z[gg][0] *= a0;
@@ -390,13 +420,25 @@ __device__ __forceinline__ void softmax_update(float (&sc)[MTN][4], SoftState& s
   }
 }
 
-// Key scores of M-tile accumulators: high + low columns (or n-tiles) summed.
-template <int NKT>
-__device__ __forceinline__ float head_score(const float (&d)[NKT][4], int e) {
-  float x = d[0][e];
-  if constexpr (NKT == 2) x += d[1][e];
-  else x += __shfl_xor_sync(0xffffffffu, x, 2);
-  return x;
+// The P.V B operand of one M-tile from its probabilities (rows g and g+8 of
+// this lane's heads): bt holds tokens 2t, 2t+1 (rows 0-7) and bb tokens
+// 8+2t, 9+2t of head g, as two kv-dtype or fp16 values. With two heads per
+// lane the rows are transposed by movmatrix; with one, lane (g, t) fetches
+// its two tokens from lanes (2t, g) and (2t+1, g) (rows g and g+8 packed in
+// one register there).
+template <int HPL>
+__device__ __forceinline__ void prob_operand(uint32_t row_g, uint32_t row_g8, uint32_t packed, int lane,
+                                             uint32_t& bt, uint32_t& bb) {
+  if constexpr (HPL == 2) {
+    bt = movmatrix_t(row_g);
+    bb = movmatrix_t(row_g8);
+  } else {
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t u = __shfl_sync(0xffffffffu, packed, 8 * t + g);
+    const uint32_t v = __shfl_sync(0xffffffffu, packed, 8 * t + 4 + g);
+    bt = __byte_perm(u, v, 0x5410);
+    bb = __byte_perm(u, v, 0x7632);
+  }
 }
 
 // One chunk of ring tokens (cnt of its kResChunk rows present, cnt <= 0
@@ -416,13 +458,15 @@ __device__ __forceinline__ float head_score(const float (&d)[NKT][4], int e) {
 // the row scale of the quantized blocks' value codes (2^(p-24)).
 template <bool BF16, int VB, int NGRP, int NKT>
 __device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t* qw, uint2* bk, int cnt, int NG,
-                                           int lane, float score_scale, bool v0, bool v1, bool& rq_ready,
-                                           SoftState& sst, float (&O)[8][4], float (&Z)[NGRP][4]) {
+                                           int lane, float score_scale, const bool (&valid)[heads_per_lane<NKT>()],
+                                           bool& rq_ready, SoftState<heads_per_lane<NKT>()>& sst, float (&O)[8][4],
+                                           float (&Z)[NGRP][4]) {
   using S = Shape<2, VB, NGRP, NKT>;  // value-side constants only
+  constexpr int HPL = heads_per_lane<NKT>();
   const int g = lane >> 2, t = lane & 3;
   if (!rq_ready) {
-    // column g: head g%4, high (g < 4) or low part; with two n-tiles, head g
-    const int head = NKT == 2 ? g : (g & 3);
+    // column g: head g (two n-tiles) or head g/2, high (g even) or low part
+    const int head = NKT == 2 ? g : (g >> 1);
     const bool present = head < NG;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
@@ -430,7 +474,7 @@ __device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t*
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int w = 4 * t + 16 * (kk >> 1) + 2 * (kk & 1) + e;  // channels 2w, 2w+1
-        const uint32_t raw = present ? qw[head * 64 + w] : 0u;
+        const uint32_t raw = present ? qw[q_word(head, w)] : 0u;
         const float2 f = unpack_f16(raw);
         const float x0 = f.x * score_scale, x1 = f.y * score_scale;
         hi[e] = pack_kv<BF16>(x0, x1);
@@ -438,7 +482,7 @@ __device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t*
         lo[e] = pack_kv<BF16>(x0 - fh.x, x1 - fh.y);
       }
       if constexpr (NKT == 1) {
-        bk[kk * 32 + lane] = (g < 4) ? make_uint2(hi[0], hi[1]) : make_uint2(lo[0], lo[1]);
+        bk[kk * 32 + lane] = (g & 1) ? make_uint2(lo[0], lo[1]) : make_uint2(hi[0], hi[1]);
       } else {
         bk[kk * 32 + lane] = make_uint2(hi[0], hi[1]);
         bk[(8 + kk) * 32 + lane] = make_uint2(lo[0], lo[1]);
@@ -464,16 +508,27 @@ __device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t*
       }
     }
   }
-  float sc[1][4];
+  // rows 8-15 are absent; row g holds ring token g of the chunk
+  float sc[1][2 * HPL];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float x = head_score<NKT>(Dr, e);
-    sc[0][e] = (e < 2 && g < cnt) ? x : -INFINITY;
+  for (int h = 0; h < HPL; ++h) {
+    sc[0][h] = g < cnt ? head_score<NKT>(Dr, 0, h) : -INFINITY;
+    sc[0][HPL + h] = -INFINITY;
   }
-  softmax_update<1, NGRP, true>(sc, sst, v0, v1, O, Z);
-  const uint32_t ph = pack_kv<BF16>(sc[0][0], sc[0][1]);
-  const float2 fh = unpack_kv2<BF16>(ph);
-  const uint32_t bh = movmatrix_t(ph), bl = movmatrix_t(pack_kv<BF16>(sc[0][0] - fh.x, sc[0][1] - fh.y));
+  softmax_update<1, HPL, NGRP, true>(sc, sst, valid, O, Z, lane);
+  // probabilities in kv-dtype high and low parts (only tokens 0-7 exist)
+  uint32_t bh, bl, dummy;
+  if constexpr (HPL == 2) {
+    const uint32_t ph = pack_kv<BF16>(sc[0][0], sc[0][1]);
+    const float2 fh = unpack_kv2<BF16>(ph);
+    prob_operand<HPL>(ph, pack_kv<BF16>(sc[0][0] - fh.x, sc[0][1] - fh.y), 0u, lane, bh, bl);
+  } else {
+    const uint32_t ph = pack_kv<BF16>(sc[0][0], 0.f);
+    const float hf = unpack_kv2<BF16>(ph).x;
+    const uint32_t hl = pack_kv<BF16>(sc[0][0], sc[0][0] - hf);  // (high, low) of row g
+    prob_operand<HPL>(0u, 0u, hl, lane, bh, dummy);              // bh = high parts of tokens 2t, 2t+1
+    bl = dummy;                                                  // bb = low parts
+  }
   const uint32_t* V32 = reinterpret_cast<const uint32_t*>(stage + kResChunk * kRowBytes);  // [rows][64 words]
 #pragma unroll
   for (int mt2 = 0; mt2 < 8; ++mt2) {
@@ -593,14 +648,27 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
     uint2* bkw = reinterpret_cast<uint2*>(ws + mp.bfrag_off);
     const float* biasr = reinterpret_cast<const float*>(ws + mp.bias_off);
     int qseq = -1;  // unit changes seen by the consumer side (matches IssueState::seq)
-    const bool v0 = 2 * t < NG, v1 = 2 * t + 1 < NG;  // heads 2t, 2t+1 of this lane exist
+    const bool v0 = 2 * t < NG, v1 = 2 * t + 1 < NG;  // output columns (heads 2t, 2t+1) of this lane exist
+    constexpr int HPL = heads_per_lane<NKT>();
+    bool valid[HPL];  // score heads of this lane exist
+    if constexpr (HPL == 2) {
+      valid[0] = v0;
+      valid[1] = v1;
+    } else {
+      valid[0] = t < NG;
+    }
     UnitCursor u;
     int k = rs;
     while (k < re && !failed) {
       u.advance(p, k);
       const int hi = min(u.end, re);
       const int nb = p.nblk[u.b];
-      SoftState sst{-INFINITY, -INFINITY, 0.f, 0.f};
+      SoftState<HPL> sst;
+#pragma unroll
+      for (int h = 0; h < HPL; ++h) {
+        sst.m[h] = -INFINITY;
+        sst.l[h] = 0.f;
+      }
       float O[8][4], Z[NGRP][4];
 #pragma unroll
       for (int i2 = 0; i2 < 8; ++i2) O[i2][0] = O[i2][1] = O[i2][2] = O[i2][3] = 0.f;
@@ -621,17 +689,33 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
           // the warp's first item of the unit brought its queries: to fp16
           // times q_prescale, in place
           ++qseq;
-          for (int w = lane; w < NG * (D / 2); w += 32) {
-            const float2 f = bf16 ? unpack_bf16(qw[w]) : unpack_f16(qw[w]);
-            qw[w] = pack_f16(f.x * p.q_prescale, f.y * p.q_prescale);
+          // (the permutation stays inside each head: four heads at a time)
+          for (int h0 = 0; h0 < NG; h0 += 4) {
+            uint32_t cv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int w = h0 * (D / 2) + lane + 32 * i;
+              if (w < NG * (D / 2)) {
+                const float2 f = bf16 ? unpack_bf16(qw[w]) : unpack_f16(qw[w]);
+                cv[i] = pack_f16(f.x * p.q_prescale, f.y * p.q_prescale);
+              }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int w = h0 * (D / 2) + lane + 32 * i;
+              if (w < NG * (D / 2)) qw[q_word(w / (D / 2), w % (D / 2))] = cv[i];
+            }
+            __syncwarp();
           }
-          __syncwarp();
         }
         const int j = kb - u.start;
         if (j < nb) {
           // ============ quantized block
           prep_block<NKT>(stage, mp, ws, qw, NG, lane, p.score_scale);
-          const float bias0 = biasr[2 * t], bias1 = biasr[2 * t + 1];
+          float bias[HPL];
+#pragma unroll
+          for (int h = 0; h < HPL; ++h) bias[h] = biasr[HPL == 2 ? 2 * t + h : t];
           const uint32_t kc_s = smem_u32(stage);
           const uint32_t vc_s = smem_u32(stage + mp.vc_soff);
           const uint4* vsz4 = reinterpret_cast<const uint4*>(stage + mp.vsz_soff);
@@ -670,21 +754,25 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
             }
             // ---- online softmax over the tile; row r of M-tile mt read code
             // 2*(mt % JP) + r/8 of its column
-            float sc[S::MT][4];
+            float sc[S::MT][2 * HPL];
 #pragma unroll
             for (int mt = 0; mt < S::MT; ++mt)
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float rs = p.score_scale * code_unscale<KB>(2 * (mt % S::JP) + (e >> 1));
-                sc[mt][e] = fmaf(head_score<NKT>(Dk[mt], e), rs, (e & 1) ? bias1 : bias0);
+              for (int r = 0; r < 2; ++r) {
+                const float rs = p.score_scale * code_unscale<KB>(2 * (mt % S::JP) + r);
+#pragma unroll
+                for (int h = 0; h < HPL; ++h) sc[mt][r * HPL + h] = fmaf(head_score<NKT>(Dk[mt], r, h), rs, bias[h]);
               }
-            softmax_update<S::MT, NGRP, false>(sc, sst, v0, v1, O, Z);
+            softmax_update<S::MT, HPL, NGRP, false>(sc, sst, valid, O, Z, lane);
             // ---- values: O += codes x (p * s), Z += ones x (p * z)
 #pragma unroll
             for (int mt = 0; mt < S::MT; ++mt) {
               // P^T of the M-tile: tokens rows 2t, 2t+1 (bt) and 8+2t, 9+2t (bb), head g
-              const uint32_t bt = movmatrix_t(pack_f16(sc[mt][0], sc[mt][1]));
-              const uint32_t bb = movmatrix_t(pack_f16(sc[mt][2], sc[mt][3]));
+              uint32_t bt, bb;
+              if constexpr (HPL == 2)
+                prob_operand<HPL>(pack_f16(sc[mt][0], sc[mt][1]), pack_f16(sc[mt][2], sc[mt][3]), 0u, lane, bt, bb);
+              else
+                prob_operand<HPL>(0u, 0u, pack_f16(sc[mt][0], sc[mt][1]), lane, bt, bb);
               const int kst = tile * S::MT + mt;
               uint32_t B0[NGRP], B1[NGRP];
 #pragma unroll
@@ -717,10 +805,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
           }
         } else if (bf16) {
           ring_chunk<true, VB, NGRP, NKT>(stage, qw, bkw, p.nres[u.b] - (j - nb) * kResChunk, NG, lane,
-                                         p.score_scale, v0, v1, rq_ready, sst, O, Z);
+                                         p.score_scale, valid, rq_ready, sst, O, Z);
         } else {
           ring_chunk<false, VB, NGRP, NKT>(stage, qw, bkw, p.nres[u.b] - (j - nb) * kResChunk, NG, lane,
-                                          p.score_scale, v0, v1, rq_ready, sst, O, Z);
+                                          p.score_scale, valid, rq_ready, sst, O, Z);
         }
         // every lane is done with the stage: refill it with item n + SPW
         __syncwarp();
@@ -732,10 +820,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
       if (failed) break;
       // ---------------- this warp's partial for the unit
 #pragma unroll
-      for (int off = 4; off <= 16; off <<= 1) {
-        sst.l0 += __shfl_xor_sync(0xffffffffu, sst.l0, off);
-        sst.l1 += __shfl_xor_sync(0xffffffffu, sst.l1, off);
-      }
+      for (int off = 4; off <= 16; off <<= 1)
+#pragma unroll
+        for (int h = 0; h < HPL; ++h) sst.l[h] += __shfl_xor_sync(0xffffffffu, sst.l[h], off);
       const int c0 = cta_of_item(p.cta_start, p.num_ctas, u.start);
       const int slot = kNC * (c - c0) + warp;
       if (slot == 0 && lane == 0)  // the unit's slot count, for the combine kernel
@@ -758,8 +845,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
               make_float2(fmaf(O[mt2][1], u0, Z[gg][1]), fmaf(O[mt2][3], u1, Z[gg][3]));
       }
       if (g == 0) {
-        if (v0) p.ws_ml[base0] = make_float2(sst.m0, sst.l0);
-        if (v1) p.ws_ml[base1] = make_float2(sst.m1, sst.l1);
+        if constexpr (HPL == 2) {
+          if (v0) p.ws_ml[base0] = make_float2(sst.m[0], sst.l[0]);
+          if (v1) p.ws_ml[base1] = make_float2(sst.m[1], sst.l[1]);
+        } else if (valid[0]) {  // head t
+          p.ws_ml[((int64_t)u.b * p.num_q_heads + u.h * NG + t) * p.slots + slot] = make_float2(sst.m[0], sst.l[0]);
+        }
       }
       k = hi;
     }
