@@ -43,6 +43,12 @@ the design notes of the repository):
    dequantized values for quantized tokens and the exact stored values for the
    residual window. Query head h reads KV head ``h // (Hq / Hkv)`` (GQA).
    A sequence with no cached tokens yields a zero output.
+6. Attention sinks ("KV1-1.2B" card: the first 4 tokens of every sequence
+   keep fp16 K/V; BQ2_0 section: positions 0-3 keep full-precision K/V): with
+   ``sinks = S`` the first S tokens appended to a sequence are stored exactly
+   and never quantized; everything above (ring, flushes, key groups) applies
+   to the tokens after them, so key group j covers tokens S + jG .. S + jG +
+   G - 1. Decode attention reads the sinks exactly, like the ring.
 
 Floating point: the quantizer runs in IEEE fp32 (the precision the KV1 card
 fixes); numpy evaluates each fp32 operation with one rounding and never
@@ -204,11 +210,14 @@ class SequenceCache:
     cache's storage type (fp16 or bf16); the ring keeps them unchanged.
     """
 
-    def __init__(self, num_kv_heads, head_dim, k_bits, v_bits, group_k, group_v, residual):
-        assert residual % group_k == 0 and residual >= group_k
+    def __init__(self, num_kv_heads, head_dim, k_bits, v_bits, group_k, group_v, residual, sinks=0):
+        assert residual % group_k == 0 and residual >= group_k and sinks >= 0
         self.H, self.D = num_kv_heads, head_dim
         self.k_bits, self.v_bits = k_bits, v_bits
         self.group_k, self.group_v, self.residual = group_k, group_v, residual
+        self.sinks = sinks
+        self.sink_k: list[np.ndarray] = []  # the first `sinks` tokens, exact, each [H, D]
+        self.sink_v: list[np.ndarray] = []
         self.blocks: list[QuantizedBlock] = []
         self.ring_k: list[np.ndarray] = []   # oldest first, each [H, D]
         self.ring_v: list[np.ndarray] = []
@@ -222,8 +231,12 @@ class SequenceCache:
         return len(self.ring_k)
 
     @property
+    def sink_tokens(self) -> int:
+        return len(self.sink_k)
+
+    @property
     def length(self) -> int:
-        return self.quantized_tokens + self.residual_tokens
+        return self.sink_tokens + self.quantized_tokens + self.residual_tokens
 
     def _flush_oldest_block(self):
         G = self.group_k
@@ -236,7 +249,12 @@ class SequenceCache:
         self.blocks.append(QuantizedBlock(kc, kd, km, vc, vd, vm))
 
     def append_token(self, k: np.ndarray, v: np.ndarray):
-        """Append one token ([H, D] each); a full ring first flushes G tokens."""
+        """Append one token ([H, D] each): one of the first `sinks` tokens is
+        kept as it is; otherwise a full ring first flushes G tokens."""
+        if len(self.sink_k) < self.sinks:
+            self.sink_k.append(np.asarray(k, dtype=F32).copy())
+            self.sink_v.append(np.asarray(v, dtype=F32).copy())
+            return
         if len(self.ring_k) == self.residual:
             self._flush_oldest_block()
         self.ring_k.append(np.asarray(k, dtype=F32).copy())
@@ -253,8 +271,12 @@ class SequenceCache:
             self._flush_oldest_block()
 
     def dequantized(self):
-        """(K~, V~) as fp32 [L, H, D]: dequantized blocks, then the ring."""
+        """(K~, V~) as fp32 [L, H, D] in token order: the exact sinks, the
+        dequantized blocks, then the ring."""
         ks, vs = [], []
+        if self.sink_k:
+            ks.append(np.stack(self.sink_k))
+            vs.append(np.stack(self.sink_v))
         for b in self.blocks:
             ks.append(dequantize_key_block(b.kc, b.kd, b.km))
             vs.append(dequantize_value_block(b.vc, b.vd, b.vm))
@@ -297,7 +319,8 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.n
 
 
 def decode_attention(cache: SequenceCache, q: np.ndarray, scale: float) -> np.ndarray:
-    """Decode attention of one sequence over its quantized blocks and ring."""
+    """Decode attention of one sequence over its sinks, quantized blocks and
+    ring."""
     k, v = cache.dequantized()
     return attention(q, k, v, scale)
 

@@ -340,6 +340,74 @@ def test_quantized_cache_attention_matches_sdpa_on_dequantized():
 
 
 # --------------------------------------------------------------------------
+# Attention sinks (KV1-1.2B card: the first 4 tokens keep full precision)
+# --------------------------------------------------------------------------
+
+
+def _blocks_equal(a, b):
+    return len(a) == len(b) and all(
+        np.array_equal(getattr(x, f), getattr(y, f)) for x, y in zip(a, b) for f in ("kc", "kd", "km", "vc", "vd", "vm"))
+
+
+@pytest.mark.parametrize("S", [1, 4, 8])
+def test_sinks_shift_the_quantized_stream(S):
+    # the tokens after the sinks are cached exactly as a sink-free cache
+    # caches the same tokens: same blocks (codes, scales) and the same ring
+    H, D, G, R = 2, 32, 32, 64
+    rng = np.random.default_rng(40 + S)
+    L = S + 5 * G + 17
+    k = (rng.standard_normal((L, H, D)) * 3).astype(np.float32)
+    v = rng.standard_normal((L, H, D)).astype(np.float32)
+    k[:S] *= 100.0  # outlier sink keys must not reach any key group
+    a = O.SequenceCache(H, D, 2, 4, G, 32, R, sinks=S)
+    b = O.SequenceCache(H, D, 2, 4, G, 32, R)
+    for t in range(L):
+        a.append_token(k[t], v[t])
+    b.append(k[S:], v[S:])
+    assert a.sink_tokens == S and a.length == L
+    assert _blocks_equal(a.blocks, b.blocks)
+    assert all(np.array_equal(x, y) for x, y in zip(a.ring_k, b.ring_k)) and len(a.ring_k) == len(b.ring_k)
+    assert all(np.array_equal(x, k[t]) for t, x in enumerate(a.sink_k))
+    a.flush_residual()
+    b.flush_residual()
+    assert _blocks_equal(a.blocks, b.blocks) and a.sink_tokens == S  # sinks are never flushed
+
+
+def test_sinks_are_read_exactly_in_token_order():
+    H, D, G, R, S = 2, 32, 32, 64, 4
+    rng = np.random.default_rng(44)
+    L = 200
+    k = rng.standard_normal((L, H, D)).astype(np.float32)
+    v = rng.standard_normal((L, H, D)).astype(np.float32)
+    a = O.SequenceCache(H, D, 4, 2, G, 32, R, sinks=S)
+    a.append(k, v)
+    K, V = a.dequantized()
+    assert K.shape[0] == L
+    assert np.array_equal(K[:S], k[:S]) and np.array_equal(V[:S], v[:S])
+    b = O.SequenceCache(H, D, 4, 2, G, 32, R)
+    b.append(k[S:], v[S:])
+    Kb, Vb = b.dequantized()
+    assert np.array_equal(K[S:], Kb) and np.array_equal(V[S:], Vb)
+    q = rng.standard_normal((8, D))
+    o = O.decode_attention(a, q, 0.2)
+    assert np.abs(o - _sdpa(q, K, V, 0.2)).max() < 1e-12
+
+
+def test_short_sequence_is_all_sinks_and_exact():
+    # a sequence no longer than S holds only sinks: plain softmax attention
+    H, D, S = 1, 4, 4
+    k = np.array([[[1.0, 0, 0, 0]], [[0, 2.0, 0, 0]], [[0, 0, 0, 0]]], np.float32)
+    v = np.array([[[1.0, 2, 3, 4]], [[5.0, 6, 7, 8]], [[9.0, 10, 11, 12]]], np.float32)
+    c = O.SequenceCache(H, D, 2, 2, 32, 32, 64, sinks=S)
+    c.append(k, v)
+    assert (c.sink_tokens, c.quantized_tokens, c.residual_tokens) == (3, 0, 0)
+    q = np.array([[math.log(2.0), math.log(3.0) / 2, 0, 0]])
+    # scores ln2, ln3, 0 -> weights 2/6, 3/6, 1/6
+    want = (2 * v[0, 0] + 3 * v[1, 0] + 1 * v[2, 0]) / 6
+    assert np.allclose(O.decode_attention(c, q, 1.0)[0], want, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
 # Sizes (KV1-1.2B card, Memory)
 # --------------------------------------------------------------------------
 
