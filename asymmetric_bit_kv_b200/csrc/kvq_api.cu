@@ -23,15 +23,15 @@ struct kvq_cache {
   size_t arena_bytes;
   int device;
   // per layer
-  std::vector<int64_t> blocks_off, ring_k_off, ring_v_off, record_bytes;
+  std::vector<int64_t> blocks_off, ring_k_off, ring_v_off, sink_k_off, sink_v_off, record_bytes;
   int64_t max_blocks;
-  int64_t lens_off;               // int32 [num_layers][max_batch][2]
+  int64_t lens_off;               // int32 [num_layers][max_batch][3]
   int64_t ws_o_off, ws_ml_off;    // split partials
   int64_t err_off;                // int32 device error word
   int64_t uslots_off;             // int32 [max_batch][num_kv_heads] slots per unit (decode -> combine)
   int32_t slots;                  // partial slots per (sequence, query head)
   int32_t sm_count;
-  std::vector<int32_t> q_len, n_len;  // host mirror [num_layers][max_batch]
+  std::vector<int32_t> q_len, n_len, s_len;  // host mirror [num_layers][max_batch]
 };
 
 namespace {
@@ -76,6 +76,8 @@ kvq_status validate_config(const kvq_config* c) {
     return fail(KVQ_ERR_INVALID_ARG, "residual %d must be a positive multiple of group_k %d", c->residual,
                 c->group_k);
   if (c->max_tokens < 1) return fail(KVQ_ERR_INVALID_ARG, "max_tokens %d < 1", c->max_tokens);
+  if (c->sink_tokens < 0 || c->sink_tokens > KVQ_MAX_SINKS)
+    return fail(KVQ_ERR_INVALID_ARG, "sink_tokens %d outside 0..%d", c->sink_tokens, KVQ_MAX_SINKS);
   if (c->kv_dtype != KVQ_F16 && c->kv_dtype != KVQ_BF16)
     return fail(KVQ_ERR_UNSUPPORTED, "kv_dtype %d: only F16 and BF16", c->kv_dtype);
   if (!c->k_bits || !c->v_bits) return fail(KVQ_ERR_INVALID_ARG, "k_bits / v_bits is null");
@@ -86,7 +88,7 @@ kvq_status validate_config(const kvq_config* c) {
 }
 
 struct Plan {
-  std::vector<int64_t> blocks_off, ring_k_off, ring_v_off, record_bytes;
+  std::vector<int64_t> blocks_off, ring_k_off, ring_v_off, sink_k_off, sink_v_off, record_bytes;
   int64_t max_blocks, lens_off, err_off, uslots_off, ws_o_off, ws_ml_off, total;
   int32_t slots;
 };
@@ -111,9 +113,14 @@ Plan make_plan(const kvq_config* c) {
     off = round_up(off + ring, 256);
     p.ring_v_off.push_back(off);
     off = round_up(off + ring, 256);
+    const int64_t sink = c->sink_tokens > 0 ? seqheads * KVQ_MAX_SINKS * D * 2 : 0;
+    p.sink_k_off.push_back(off);
+    off = round_up(off + sink, 256);
+    p.sink_v_off.push_back(off);
+    off = round_up(off + sink, 256);
   }
   p.lens_off = off;
-  off = round_up(off + (int64_t)c->num_layers * c->max_batch * 2 * 4, 256);
+  off = round_up(off + (int64_t)c->num_layers * c->max_batch * 3 * 4, 256);
   p.err_off = off;
   off = round_up(off + 4, 256);
   p.uslots_off = off;
@@ -125,7 +132,7 @@ Plan make_plan(const kvq_config* c) {
   p.slots = (int32_t)std::max<int64_t>(
       std::min<int64_t>(p.max_blocks, KVQ_MAX_SPLITS) + 1,
       kvq::kMmaConsumers *
-          (std::min<int64_t>(p.max_blocks + (c->residual + kvq::kResChunk - 1) / kvq::kResChunk, 64) + 1));
+          (std::min<int64_t>(p.max_blocks + (c->residual + kvq::kResChunk - 1) / kvq::kResChunk + 1, 64) + 1));
   const int64_t partials = (int64_t)c->max_batch * c->num_q_heads * p.slots;
   p.ws_o_off = off;
   off = round_up(off + partials * D * 4, 256);
@@ -143,7 +150,10 @@ kvq::LayerView layer_view(const kvq_cache* c, int layer) {
   v.blocks = c->arena + c->blocks_off[layer];
   v.ring_k = c->arena + c->ring_k_off[layer];
   v.ring_v = c->arena + c->ring_v_off[layer];
-  v.lens = reinterpret_cast<int32_t*>(c->arena + c->lens_off) + (int64_t)layer * cfg.max_batch * 2;
+  v.sink_k = c->arena + c->sink_k_off[layer];
+  v.sink_v = c->arena + c->sink_v_off[layer];
+  v.sinks = cfg.sink_tokens;
+  v.lens = reinterpret_cast<int32_t*>(c->arena + c->lens_off) + (int64_t)layer * cfg.max_batch * 3;
   v.record_bytes = c->record_bytes[layer];
   v.max_blocks = c->max_blocks;
   v.kc_off = 0;
@@ -185,10 +195,17 @@ kvq_status enqueue_append(kvq_cache* c, int layer, const void* k, const void* v,
   p->batch = batch;
   int32_t* ql = &c->q_len[(size_t)layer * cfg.max_batch];
   int32_t* nl = &c->n_len[(size_t)layer * cfg.max_batch];
+  int32_t* sl = &c->s_len[(size_t)layer * cfg.max_batch];
   int max_flush = 0;
   int64_t off = 0;
   for (int b = 0; b < batch; ++b) {
-    const int T = flush_all ? 0 : new_lens[b];
+    // the sequence's first sink_tokens tokens go to its sinks
+    const int all = flush_all ? 0 : new_lens[b];
+    const int take = std::min(all, cfg.sink_tokens - sl[b]);
+    p->s_old[b] = sl[b];
+    p->s_take[b] = take;
+    off += take;
+    const int T = all - take;
     int f;
     if (flush_all) f = nl[b] / G;
     else f = (nl[b] + T <= R) ? 0 : (nl[b] + T - R + G - 1) / G;
@@ -207,6 +224,7 @@ kvq_status enqueue_append(kvq_cache* c, int layer, const void* k, const void* v,
       const int end = p->q_old[b] + p->n_old[b] + p->t_new[b];
       ql[b] = qn;
       nl[b] = end - qn;
+      sl[b] += p->s_take[b];
     }
   }
   delete p;
@@ -345,7 +363,7 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out,
   int32_t used_slots = c->slots;  // partial slots per (sequence, query head) this call writes
   if (use_mma) {
     // Persistent plan: the work items of every (sequence, KV head) unit
-    // (quantized blocks, then ring chunks), concatenated and cut into one
+    // (quantized blocks, ring chunks, sinks), concatenated and cut into one
     // contiguous range per CTA, one CTA per resident slot (fewer if there is
     // little work).
     int64_t total = 0;
@@ -353,7 +371,7 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out,
       const int nres = c->n_len[(size_t)layer * cfg.max_batch + b];
       p.nblk[b] = nblk[b];
       p.nres[b] = nres;
-      p.nitem[b] = kvq::unit_items(nblk[b], nres);
+      p.nitem[b] = kvq::unit_items(nblk[b], nres, c->s_len[(size_t)layer * cfg.max_batch + b]);
       p.seq_start[b] = (int32_t)total;
       total += (int64_t)p.nitem[b] * cfg.num_kv_heads;
     }
@@ -459,6 +477,8 @@ kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena
   c->blocks_off = plan.blocks_off;
   c->ring_k_off = plan.ring_k_off;
   c->ring_v_off = plan.ring_v_off;
+  c->sink_k_off = plan.sink_k_off;
+  c->sink_v_off = plan.sink_v_off;
   c->record_bytes = plan.record_bytes;
   c->max_blocks = plan.max_blocks;
   c->lens_off = plan.lens_off;
@@ -469,17 +489,23 @@ kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena
   c->slots = plan.slots;
   c->q_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
   c->n_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
+  c->s_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
   cudaError_t e = cudaGetDevice(&c->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device);
-  if (e == cudaSuccess) e = cudaMemset(c->arena + c->lens_off, 0, (size_t)cfg->num_layers * cfg->max_batch * 8);
+  if (e == cudaSuccess) e = cudaMemset(c->arena + c->lens_off, 0, (size_t)cfg->num_layers * cfg->max_batch * 12);
   if (e == cudaSuccess) e = cudaMemset(c->arena + c->err_off, 0, 4);
-  // Ring slots that no token has reached yet hold zeros, never stale bit
-  // patterns: the decode kernel reads whole 16-slot groups of the ring and
-  // masks the scores of slots past the sequence, so their values must be finite.
+  // Ring slots and sink rows that no token has reached yet hold zeros, never
+  // stale bit patterns: the decode kernel reads whole chunks of ring slots
+  // and sink rows and masks the scores of those past the sequence, so their
+  // values must be finite.
   const size_t ring_bytes = (size_t)cfg->max_batch * cfg->num_kv_heads * cfg->residual * cfg->head_dim * 2;
+  const size_t sink_bytes =
+      cfg->sink_tokens > 0 ? (size_t)cfg->max_batch * cfg->num_kv_heads * KVQ_MAX_SINKS * cfg->head_dim * 2 : 0;
   for (int l = 0; l < cfg->num_layers && e == cudaSuccess; ++l) {
     e = cudaMemset(c->arena + c->ring_k_off[l], 0, ring_bytes);
     if (e == cudaSuccess) e = cudaMemset(c->arena + c->ring_v_off[l], 0, ring_bytes);
+    if (e == cudaSuccess && sink_bytes) e = cudaMemset(c->arena + c->sink_k_off[l], 0, sink_bytes);
+    if (e == cudaSuccess && sink_bytes) e = cudaMemset(c->arena + c->sink_v_off[l], 0, sink_bytes);
   }
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
@@ -500,11 +526,12 @@ kvq_status kvq_cache_destroy(kvq_cache* c) {
 kvq_status kvq_cache_reset(kvq_cache* c, void* stream) {
   g_last_error.clear();
   if (!c) return fail(KVQ_ERR_INVALID_ARG, "cache is null");
-  cudaError_t e = cudaMemsetAsync(c->arena + c->lens_off, 0, (size_t)c->cfg.num_layers * c->cfg.max_batch * 8,
+  cudaError_t e = cudaMemsetAsync(c->arena + c->lens_off, 0, (size_t)c->cfg.num_layers * c->cfg.max_batch * 12,
                                   static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "reset");
   std::fill(c->q_len.begin(), c->q_len.end(), 0);
   std::fill(c->n_len.begin(), c->n_len.end(), 0);
+  std::fill(c->s_len.begin(), c->s_len.end(), 0);
   return KVQ_OK;
 }
 
@@ -519,8 +546,8 @@ kvq_status kvq_append(kvq_cache* c, int32_t layer, const void* k, const void* v,
   int64_t total = 0;
   for (int b = 0; b < batch; ++b) {
     if (new_lens[b] < 0) return fail(KVQ_ERR_INVALID_ARG, "new_lens[%d] = %d < 0", b, new_lens[b]);
-    const int64_t L = (int64_t)c->q_len[(size_t)layer * c->cfg.max_batch + b] +
-                      c->n_len[(size_t)layer * c->cfg.max_batch + b] + new_lens[b];
+    const size_t i = (size_t)layer * c->cfg.max_batch + b;
+    const int64_t L = (int64_t)c->s_len[i] + c->q_len[i] + c->n_len[i] + new_lens[b];
     if (L > c->cfg.max_tokens)
       return fail(KVQ_ERR_CAPACITY, "sequence %d would hold %lld tokens > max_tokens %d", b, (long long)L,
                   c->cfg.max_tokens);
@@ -558,12 +585,12 @@ kvq_status kvq_dequant(kvq_cache* c, int32_t layer, int32_t seq, int32_t t0, int
   if (s != KVQ_OK) return s;
   if (seq < 0 || seq >= c->cfg.max_batch) return fail(KVQ_ERR_INVALID_ARG, "seq %d out of range", seq);
   const size_t i = (size_t)layer * c->cfg.max_batch + seq;
-  const int L = c->q_len[i] + c->n_len[i];
+  const int L = c->s_len[i] + c->q_len[i] + c->n_len[i];
   if (t0 < 0 || t0 > t1 || t1 > L)
     return fail(KVQ_ERR_INVALID_ARG, "token range [%d,%d) outside [0,%d]", t0, t1, L);
   if (t1 == t0) return KVQ_OK;
   if (!k_out || !v_out) return fail(KVQ_ERR_INVALID_ARG, "k_out or v_out is null");
-  cudaError_t e = kvq::launch_dequant(layer_view(c, layer), seq, t0, t1, k_out, v_out,
+  cudaError_t e = kvq::launch_dequant(layer_view(c, layer), seq, c->s_len[i], t0, t1, k_out, v_out,
                                       static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "dequant launch");
   return KVQ_OK;
@@ -597,6 +624,8 @@ kvq_status kvq_get_layout(const kvq_cache* c, int32_t layer, kvq_layout* out) {
   out->ring_v = v.ring_v;
   out->k_bits = v.k_bits;
   out->v_bits = v.v_bits;
+  out->sink_k = v.sink_k;
+  out->sink_v = v.sink_v;
   return KVQ_OK;
 }
 
@@ -610,6 +639,16 @@ kvq_status kvq_seq_lengths(const kvq_cache* c, int32_t layer, int32_t seq, int32
   const size_t i = (size_t)layer * c->cfg.max_batch + seq;
   *quantized = c->q_len[i];
   *residual = c->n_len[i];
+  return KVQ_OK;
+}
+
+kvq_status kvq_seq_sinks(const kvq_cache* c, int32_t layer, int32_t seq, int32_t* sinks) {
+  g_last_error.clear();
+  kvq_status s = check_cache_layer(c, layer);
+  if (s != KVQ_OK) return s;
+  if (seq < 0 || seq >= c->cfg.max_batch) return fail(KVQ_ERR_INVALID_ARG, "seq %d out of range", seq);
+  if (!sinks) return fail(KVQ_ERR_INVALID_ARG, "output pointer is null");
+  *sinks = c->s_len[(size_t)layer * c->cfg.max_batch + seq];
   return KVQ_OK;
 }
 

@@ -114,8 +114,8 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_blocks_kernel(AppendPa
   }
 }
 
-// grid (batch, Hkv); copies this call's unflushed new tokens into the ring and
-// records the new lengths.
+// grid (batch, Hkv); copies this call's sink tokens to the sinks and its
+// unflushed new tokens into the ring, and records the new lengths.
 __global__ void ring_write_kernel(AppendParams p) {
   const int b = blockIdx.x, h = blockIdx.y;
   const LayerView& L = p.L;
@@ -125,6 +125,18 @@ __global__ void ring_write_kernel(AppendParams p) {
   const int end = boundary + p.t_new[b];
   const int first = max(boundary, q_new);
   const int vec_per_tok = D / 8;
+  const int ns = p.s_take[b];
+  const int64_t sink_base = ((int64_t)b * L.num_kv_heads + h) * KVQ_MAX_SINKS + p.s_old[b];
+  for (int idx = threadIdx.x; idx < ns * vec_per_tok; idx += blockDim.x) {
+    const int i = idx / vec_per_tok, c = (idx % vec_per_tok) * 8;
+    const int64_t row = (int64_t)p.in_off[b] - ns + i;
+    const int64_t src = (row * L.num_kv_heads + h) * D + c;
+    const int64_t dst = (sink_base + i) * D + c;
+    *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(L.sink_k) + dst) =
+        *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.k_in) + src);
+    *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(L.sink_v) + dst) =
+        *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.v_in) + src);
+  }
   const int64_t ring_base = ((int64_t)b * L.num_kv_heads + h) * R;
   for (int idx = threadIdx.x; idx < (end - first) * vec_per_tok; idx += blockDim.x) {
     const int i = first + idx / vec_per_tok, c = (idx % vec_per_tok) * 8;
@@ -137,23 +149,31 @@ __global__ void ring_write_kernel(AppendParams p) {
         *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.v_in) + src);
   }
   if (h == 0 && threadIdx.x == 0) {
-    L.lens[2 * b] = q_new;
-    L.lens[2 * b + 1] = end - q_new;
+    L.lens[3 * b] = q_new;
+    L.lens[3 * b + 1] = end - q_new;
+    L.lens[3 * b + 2] = p.s_old[b] + ns;
   }
 }
 
-// grid (ceil(n / 8), Hkv); block D threads. Token t0 + i of sequence `seq`.
-__global__ void dequant_kernel(LayerView L, int seq, int t0, int n, float* k_out, float* v_out) {
+// grid (ceil(n / 8), Hkv); block D threads. Token t0 + i of sequence `seq`,
+// whose first `sinks` tokens are its sinks.
+__global__ void dequant_kernel(LayerView L, int seq, int sinks, int t0, int n, float* k_out, float* v_out) {
   const int h = blockIdx.y;
   const int d = threadIdx.x;
   const int G = L.group_k, D = L.head_dim, R = L.residual;
-  const int Q = L.lens[2 * seq];
+  const int Q = L.lens[3 * seq];
   const int kb = L.k_bits, vb = L.v_bits;
   for (int r = 0; r < 8; ++r) {
     const int i = blockIdx.x * 8 + r;
     if (i >= n || d >= D) continue;
-    const int tok = t0 + i;
     const int64_t o = ((int64_t)i * L.num_kv_heads + h) * D + d;
+    if (t0 + i < sinks) {
+      const int64_t src = (((int64_t)seq * L.num_kv_heads + h) * KVQ_MAX_SINKS + t0 + i) * D + d;
+      k_out[o] = load_kv(L.sink_k, src, L.kv_dtype);
+      v_out[o] = load_kv(L.sink_v, src, L.kv_dtype);
+      continue;
+    }
+    const int tok = t0 + i - sinks;  // position after the sinks
     if (tok < Q) {
       const uint8_t* rec = record_ptr(L, seq, h, tok / G);
       const int t = tok % G;
@@ -201,12 +221,12 @@ cudaError_t launch_append(const AppendParams& p, int max_flush, cudaStream_t str
   return cudaGetLastError();
 }
 
-cudaError_t launch_dequant(const LayerView& L, int seq, int t0, int t1, float* k_out, float* v_out,
+cudaError_t launch_dequant(const LayerView& L, int seq, int sinks, int t0, int t1, float* k_out, float* v_out,
                            cudaStream_t stream) {
   const int n = t1 - t0;
   if (n <= 0) return cudaSuccess;
   dim3 grid((n + 7) / 8, L.num_kv_heads);
-  dequant_kernel<<<grid, L.head_dim, 0, stream>>>(L, seq, t0, n, k_out, v_out);
+  dequant_kernel<<<grid, L.head_dim, 0, stream>>>(L, seq, sinks, t0, n, k_out, v_out);
   return cudaGetLastError();
 }
 

@@ -16,13 +16,15 @@ struct AppendParams {
   int32_t batch;
   int32_t q_old[KVQ_MAX_BATCH];   // quantized tokens before the call
   int32_t n_old[KVQ_MAX_BATCH];   // ring tokens before the call
-  int32_t t_new[KVQ_MAX_BATCH];   // tokens appended by the call
-  int32_t in_off[KVQ_MAX_BATCH];  // first input row of each sequence
+  int32_t t_new[KVQ_MAX_BATCH];   // tokens appended by the call after the sinks
+  int32_t in_off[KVQ_MAX_BATCH];  // first input row of each sequence after its sinks
   int32_t flush[KVQ_MAX_BATCH];   // G-token blocks quantized by the call
+  int32_t s_old[KVQ_MAX_BATCH];   // sink tokens before the call
+  int32_t s_take[KVQ_MAX_BATCH];  // sink tokens taken by the call (input rows in_off - s_take ..)
 };
 
 cudaError_t launch_append(const AppendParams& p, int max_flush, cudaStream_t stream);
-cudaError_t launch_dequant(const LayerView& L, int seq, int t0, int t1, float* k_out, float* v_out,
+cudaError_t launch_dequant(const LayerView& L, int seq, int sinks, int t0, int t1, float* k_out, float* v_out,
                            cudaStream_t stream);
 
 }  // namespace kvq

@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const LayerView& L = p.L;
   const int G = L.group_k, R = L.residual;
-  const int Q = L.lens[2 * b], n = L.lens[2 * b + 1];
+  const int Q = L.lens[3 * b], n = L.lens[3 * b + 1], nsink = L.lens[3 * b + 2];
   const int nblk = Q / G;
   const int bps = p.blocks_per_split;
   const int S = (nblk + bps - 1) / bps;
@@ -74,15 +74,20 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
   st.init();
 
   if (s == 0) {
-    // Residual ring: exact stored values.
+    // Sinks and the residual ring: exact stored values.
+    const int64_t sbase = ((int64_t)b * L.num_kv_heads + h) * KVQ_MAX_SINKS;
     const int64_t base = ((int64_t)b * L.num_kv_heads + h) * R;
-    for (int i = Q + warp; i < Q + n; i += 4) {
-      const int64_t row = (base + i % R) * D;
+    for (int e = warp; e < nsink + n; e += 4) {
+      // e < nsink: sink e; otherwise the ring token at position Q + e - nsink
+      const bool sink = e < nsink;
+      const int64_t row = (sink ? sbase + e : base + (Q + e - nsink) % R) * D;
+      const void* ksrc = sink ? L.sink_k : L.ring_k;
+      const void* vsrc = sink ? L.sink_v : L.ring_v;
       float kv[4], vv[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        kv[c] = load_kv(L.ring_k, row + lane + 32 * c, L.kv_dtype);
-        vv[c] = load_kv(L.ring_v, row + lane + 32 * c, L.kv_dtype);
+        kv[c] = load_kv(ksrc, row + lane + 32 * c, L.kv_dtype);
+        vv[c] = load_kv(vsrc, row + lane + 32 * c, L.kv_dtype);
       }
 #pragma unroll
       for (int hh = 0; hh < NG; ++hh) {
@@ -187,7 +192,7 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineParams p) {
     const int h = hq / (p.num_q_heads / p.num_kv_heads);
     S = __ldcg(p.unit_slots + b * p.num_kv_heads + h);
   } else {
-    const int nblk = p.lens[2 * b] / p.group_k;
+    const int nblk = p.lens[3 * b] / p.group_k;
     S = (nblk + p.blocks_per_split - 1) / p.blocks_per_split + 1;
   }
   const int64_t base = ((int64_t)b * p.num_q_heads + hq) * p.slots;

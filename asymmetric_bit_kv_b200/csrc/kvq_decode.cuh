@@ -49,10 +49,13 @@ struct DecodeParams {
 
 constexpr int kMmaConsumers = 6;   // warps per CTA of the tensor-core kernel
 constexpr int kResChunk = 8;       // ring tokens per work item, persistent mode
+static_assert(KVQ_MAX_SINKS == kResChunk, "the sink rows of a unit are one exact-token chunk");
 
-// Work items of one unit: quantized blocks, then ring chunks (at least one).
-__host__ __device__ inline int32_t unit_items(int32_t nblk, int32_t nres) {
-  const int32_t items = nblk + (nres + kResChunk - 1) / kResChunk;
+// Work items of one unit: quantized blocks, then ring chunks, then one chunk
+// of sink tokens if the sequence has any (at least one item: an empty
+// sequence gets one ring chunk with no tokens).
+__host__ __device__ inline int32_t unit_items(int32_t nblk, int32_t nres, int32_t nsink) {
+  const int32_t items = nblk + (nres + kResChunk - 1) / kResChunk + (nsink > 0 ? 1 : 0);
   return items > 0 ? items : 1;
 }
 

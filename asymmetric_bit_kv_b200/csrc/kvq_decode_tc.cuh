@@ -547,6 +547,20 @@ __device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t*
   }
 }
 
+// Exact-token chunk r of a unit (the items after its quantized blocks): ring
+// chunk r while r < ceil(nres / kResChunk), then the sink chunk if the
+// sequence has sinks; an empty sequence's one item is a ring chunk with no
+// tokens. Returns the tokens present (<= 0 for none) and whether it is the
+// sink chunk.
+__device__ __forceinline__ int exact_chunk(const DecodeParams& p, int b, int r, bool& sink) {
+  const int nres = p.nres[b];
+  sink = false;
+  if (r < (nres + kResChunk - 1) / kResChunk) return nres - r * kResChunk;
+  const int nsink = p.L.sinks > 0 ? p.L.lens[3 * b + 2] : 0;
+  sink = nsink > 0;
+  return sink ? nsink : nres - r * kResChunk;
+}
+
 // Issue side of a warp's item stream (one lane): the unit of the last issued
 // item and the number of unit changes so far.
 struct IssueState {
@@ -581,13 +595,23 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, const MmaPlan&
       bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(L.ring_v) + ring, L.residual * kRowBytes);
     }
   } else {
-    // ring chunk: kResChunk consecutive slots of keys, then of values
-    const int slot = (nb * L.group_k + (j - nb) * kResChunk) % L.residual;
-    const int64_t row = ((int64_t)u.b * L.num_kv_heads + u.h) * L.residual + slot;
+    // ring chunk: kResChunk consecutive slots of keys, then of values (or
+    // the kResChunk sink rows of the unit)
+    bool sink;
+    (void)exact_chunk(p, u.b, j - nb, sink);
+    const void* ksrc = sink ? L.sink_k : L.ring_k;
+    const void* vsrc = sink ? L.sink_v : L.ring_v;
+    int64_t row;
+    if (sink) {
+      row = ((int64_t)u.b * L.num_kv_heads + u.h) * KVQ_MAX_SINKS;
+    } else {
+      const int slot = (nb * L.group_k + (j - nb) * kResChunk) % L.residual;
+      row = ((int64_t)u.b * L.num_kv_heads + u.h) * L.residual + slot;
+    }
     constexpr uint32_t bytes = kResChunk * kRowBytes;
     mbar_expect_tx(bar, 2 * bytes + (newq ? qbytes : 0u));
-    bulk_g2s(dst, reinterpret_cast<const uint8_t*>(L.ring_k) + row * kRowBytes, bytes, bar);
-    bulk_g2s(dst + bytes, reinterpret_cast<const uint8_t*>(L.ring_v) + row * kRowBytes, bytes, bar);
+    bulk_g2s(dst, reinterpret_cast<const uint8_t*>(ksrc) + row * kRowBytes, bytes, bar);
+    bulk_g2s(dst + bytes, reinterpret_cast<const uint8_t*>(vsrc) + row * kRowBytes, bytes, bar);
   }
   if (newq)
     bulk_g2s(qbuf + (size_t)(is.seq % mp.nstages) * qbytes,
@@ -803,12 +827,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
               }
             }
           }
-        } else if (bf16) {
-          ring_chunk<true, VB, NGRP, NKT>(stage, qw, bkw, p.nres[u.b] - (j - nb) * kResChunk, NG, lane,
-                                         p.score_scale, valid, rq_ready, sst, O, Z);
         } else {
-          ring_chunk<false, VB, NGRP, NKT>(stage, qw, bkw, p.nres[u.b] - (j - nb) * kResChunk, NG, lane,
-                                          p.score_scale, valid, rq_ready, sst, O, Z);
+          bool sink;
+          const int cnt = exact_chunk(p, u.b, j - nb, sink);
+          if (bf16)
+            ring_chunk<true, VB, NGRP, NKT>(stage, qw, bkw, cnt, NG, lane, p.score_scale, valid, rq_ready, sst, O, Z);
+          else
+            ring_chunk<false, VB, NGRP, NKT>(stage, qw, bkw, cnt, NG, lane, p.score_scale, valid, rq_ready, sst, O, Z);
         }
         // every lane is done with the stage: refill it with item n + SPW
         __syncwarp();

@@ -17,13 +17,16 @@ struct LayerView {
   uint8_t* blocks;        // block records [max_batch][Hkv][max_blocks]
   void* ring_k;           // [max_batch][Hkv][R][D] kv dtype
   void* ring_v;
-  int32_t* lens;          // [max_batch][2]: quantized tokens, ring tokens
+  void* sink_k;           // [max_batch][Hkv][KVQ_MAX_SINKS][D] kv dtype (sink_tokens > 0)
+  void* sink_v;
+  int32_t* lens;          // [max_batch][3]: quantized tokens, ring tokens, sink tokens
   int64_t record_bytes;
   int64_t max_blocks;
   int32_t kc_off, ksz_off, vc_off, vsz_off;  // byte offsets inside a record
   int32_t k_bits, v_bits;
   int32_t num_kv_heads, head_dim, group_k, group_v, residual;
   int32_t kv_dtype;       // KVQ_F16 / KVQ_BF16
+  int32_t sinks;          // S: sink tokens kept exact at the start of each sequence
 };
 
 __host__ __device__ inline int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }

@@ -44,6 +44,7 @@ class kvq_config(ctypes.Structure):
         ("kv_dtype", ctypes.c_int32),
         ("k_bits", ctypes.POINTER(ctypes.c_int8)),
         ("v_bits", ctypes.POINTER(ctypes.c_int8)),
+        ("sink_tokens", ctypes.c_int32),
     ]
 
 
@@ -60,6 +61,8 @@ class kvq_layout(ctypes.Structure):
         ("ring_v", ctypes.c_void_p),
         ("k_bits", ctypes.c_int32),
         ("v_bits", ctypes.c_int32),
+        ("sink_k", ctypes.c_void_p),
+        ("sink_v", ctypes.c_void_p),
     ]
 
 
@@ -89,6 +92,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kvq_get_layout": (I32, [P, I32, ctypes.POINTER(kvq_layout)]),
         "kvq_device_errors": (I32, [P, ctypes.POINTER(I32)]),
         "kvq_seq_lengths": (I32, [P, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32)]),
+        "kvq_seq_sinks": (I32, [P, I32, I32, ctypes.POINTER(I32)]),
         "kvq_status_string": (ctypes.c_char_p, [I32]),
         "kvq_last_error": (ctypes.c_char_p, []),
     }
@@ -139,13 +143,15 @@ class CacheConfig:
     kv_dtype: torch.dtype
     k_bits: list
     v_bits: list
+    sink_tokens: int = 0
 
     def to_c(self):
         kb = (ctypes.c_int8 * self.num_layers)(*self.k_bits)
         vb = (ctypes.c_int8 * self.num_layers)(*self.v_bits)
         c = kvq_config(self.num_layers, self.max_batch, self.num_q_heads, self.num_kv_heads, self.head_dim,
                        self.max_tokens, self.group_k, self.group_v, self.residual, _DTYPE_CODE[self.kv_dtype],
-                       ctypes.cast(kb, ctypes.POINTER(ctypes.c_int8)), ctypes.cast(vb, ctypes.POINTER(ctypes.c_int8)))
+                       ctypes.cast(kb, ctypes.POINTER(ctypes.c_int8)), ctypes.cast(vb, ctypes.POINTER(ctypes.c_int8)),
+                       self.sink_tokens)
         return c, (kb, vb)
 
 
@@ -256,3 +262,8 @@ class KVCache:
         n = ctypes.c_int32()
         _check(self.lib.kvq_seq_lengths(self.handle, layer, seq, ctypes.byref(q), ctypes.byref(n)), "kvq_seq_lengths")
         return q.value, n.value
+
+    def sinks(self, layer: int, seq: int) -> int:
+        s = ctypes.c_int32()
+        _check(self.lib.kvq_seq_sinks(self.handle, layer, seq, ctypes.byref(s)), "kvq_seq_sinks")
+        return s.value

@@ -64,6 +64,7 @@ typedef enum kvq_dtype { KVQ_F16 = 0, KVQ_BF16 = 1, KVQ_F32 = 2 } kvq_dtype;
 #define KVQ_MAX_BATCH 512  /* sequences per cache                        */
 #define KVQ_MAX_LAYERS 512 /* layers per cache                           */
 #define KVQ_MAX_SPLITS 256 /* quantized splits per (sequence, KV head)   */
+#define KVQ_MAX_SINKS 8    /* sink tokens per sequence                   */
 
 /* Cache shape. Names follow the KIVI README "Example" (k_bits, v_bits,
  * group_size, residual_length) with the group size given per tensor as in
@@ -74,7 +75,7 @@ typedef struct kvq_config {
   int32_t num_q_heads;  /* Hq, a multiple of num_kv_heads                   */
   int32_t num_kv_heads; /* Hkv; Hq/Hkv in {1, 2, 4, 8}                      */
   int32_t head_dim;     /* D = 128                                          */
-  int32_t max_tokens;   /* per-sequence capacity, quantized + residual      */
+  int32_t max_tokens;   /* per-sequence capacity: sinks + quantized + residual */
   int32_t group_k;      /* G: tokens per key group (one group per channel);
                            32, 64 or 128. Flushes move G tokens at a time.  */
   int32_t group_v;      /* channels per value group (one group per token);
@@ -83,12 +84,18 @@ typedef struct kvq_config {
   int32_t kv_dtype;     /* KVQ_F16 or KVQ_BF16: keys, values, ring, queries */
   const int8_t* k_bits; /* host [num_layers], each 2, 4 or 8 (copied)       */
   const int8_t* v_bits; /* host [num_layers], each 2, 4 or 8 (copied)       */
+  int32_t sink_tokens;  /* S, 0..KVQ_MAX_SINKS: the first S tokens of every
+                           sequence are kept exact and never quantized
+                           (KV1-1.2B card: attention sinks, 4 in KV1);
+                           quantization and the ring start at token S      */
 } kvq_config;
 
 typedef struct kvq_cache kvq_cache;
 
 /* Where one layer's packed cache lives, for tests and tools that read it.
- * Block records: for sequence b, KV head h and key block j (tokens
+ * Token positions below are counted after the sequence's s sink tokens
+ * (s = min(S, tokens appended so far)): position i is token s + i.
+ * Block records: for sequence b, KV head h and key block j (positions
  * [j*G, (j+1)*G) of that sequence) the record starts at
  *   blocks + ((b * num_kv_heads + h) * max_blocks + j) * record_bytes
  * and holds, at the given byte offsets:
@@ -110,8 +117,10 @@ typedef struct kvq_cache kvq_cache;
  * (r / (8/n)) % n otherwise; rows of fewer than 4 words are not permuted.
  * Value rows are stored in token order t -> (t % c) * (G/c) + t / c, with
  * c = 16/k_bits. (kvq_internal.cuh: kc_word_index, vc_word_index.)
- * Ring: [max_batch][num_kv_heads][R][D] in kv_dtype; token i of a sequence
- * (quantized <= i < quantized + residual) sits in slot i % R.              */
+ * Ring: [max_batch][num_kv_heads][R][D] in kv_dtype; position i of a
+ * sequence (quantized <= i < quantized + residual) sits in slot i % R.
+ * Sinks: [max_batch][num_kv_heads][KVQ_MAX_SINKS][D] in kv_dtype; sink
+ * token i (< s) in row i, the other rows zero.                             */
 typedef struct kvq_layout {
   void* blocks;
   int64_t record_bytes;
@@ -120,6 +129,8 @@ typedef struct kvq_layout {
   void* ring_k;
   void* ring_v;
   int32_t k_bits, v_bits;
+  void* sink_k;
+  void* sink_v;
 } kvq_layout;
 
 /* Device bytes the arena must hold for cfg: all layers' block records and
@@ -143,13 +154,15 @@ KVQ_API kvq_status kvq_cache_reset(kvq_cache* cache, void* stream);
  * k, v: device, token-major [sum(new_lens)][num_kv_heads][head_dim] in
  * kv_dtype, sequences in order. new_lens: host [batch], each >= 0.
  * Semantics (KIVI README: residual window of recent full-precision tokens;
- * KV1 card: each token quantized once when it enters the cache): tokens are
- * appended one by one; a token that finds the ring full (R tokens) first
+ * KV1 card: each token quantized once when it enters the cache, the first
+ * S kept exact): tokens are appended one by one; each of a sequence's first
+ * S tokens goes to its sinks as it is; a later token that finds the ring
+ * full (R tokens) first
  * causes the oldest G ring tokens to be quantized -- keys per channel over
  * the G tokens, values per token over group_v channels -- into one block
  * record. Blocks that a long append would quantize straight away are read
  * from k, v directly. Fails with KVQ_ERR_CAPACITY if a sequence would exceed
- * max_tokens.                                                              */
+ * max_tokens (sinks included).                                             */
 KVQ_API kvq_status kvq_append(kvq_cache* cache, int32_t layer, const void* k, const void* v,
                       const int32_t* new_lens, int32_t batch, void* stream);
 
@@ -158,8 +171,8 @@ KVQ_API kvq_status kvq_append(kvq_cache* cache, int32_t layer, const void* k, co
 KVQ_API kvq_status kvq_flush_residual(kvq_cache* cache, int32_t layer, int32_t batch, void* stream);
 
 /* One decode query per sequence: out[b][h] = softmax(scale * q[b][h] K~^T) V~
- * over all cached tokens of sequence b (no mask), K~/V~ the dequantized
- * blocks and the exact ring tokens; query head h reads KV head
+ * over all cached tokens of sequence b (no mask), K~/V~ the exact sinks, the
+ * dequantized blocks and the exact ring tokens; query head h reads KV head
  * h / (Hq/Hkv) (GQA). q: device [batch][Hq][D] in kv_dtype. out: device
  * [batch][Hq][D] in out_dtype (F32, F16 or BF16; round to nearest even).
  * A sequence with no tokens gives zeros. Uses the arena's workspace.       */
@@ -197,7 +210,8 @@ KVQ_API kvq_status kvq_decode_attention_noalloc(kvq_cache* cache, int32_t layer,
 
 /* Reconstruct tokens [t0, t1) of sequence `seq` as fp32: x_hat = q*d + m
  * (an fp32 product, then an fp32 sum; KV1 card, BQ2_0) for quantized tokens
- * and the exact stored value for ring tokens. k_out, v_out: device
+ * and the exact stored value for sink and ring tokens (t counts every token
+ * of the sequence, sinks first). k_out, v_out: device
  * [t1-t0][num_kv_heads][head_dim] fp32. 0 <= t0 <= t1 <= sequence length.  */
 KVQ_API kvq_status kvq_dequant(kvq_cache* cache, int32_t layer, int32_t seq, int32_t t0, int32_t t1,
                        float* k_out, float* v_out, void* stream);
@@ -212,9 +226,13 @@ KVQ_API kvq_status kvq_device_errors(kvq_cache* cache, int32_t* flags);
 KVQ_API kvq_status kvq_get_layout(const kvq_cache* cache, int32_t layer, kvq_layout* out);
 
 /* Host mirror of a sequence's lengths: quantized tokens (a multiple of G)
- * and ring tokens.                                                         */
+ * and ring tokens (the sink tokens come on top: kvq_seq_sinks).             */
 KVQ_API kvq_status kvq_seq_lengths(const kvq_cache* cache, int32_t layer, int32_t seq,
                            int32_t* quantized, int32_t* residual);
+
+/* Host mirror of a sequence's sink tokens, min(S, tokens appended). No
+ * counterpart on the pages beyond the sinks themselves (KV1 card).         */
+KVQ_API kvq_status kvq_seq_sinks(const kvq_cache* cache, int32_t layer, int32_t seq, int32_t* sinks);
 
 /* Static description of a status code.                                     */
 KVQ_API const char* kvq_status_string(kvq_status status);

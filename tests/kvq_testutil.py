@@ -85,7 +85,8 @@ class Twin:
         for layer in self.oracle_layers:
             for b in self.oracle_seqs:
                 self.ora[(layer, b)] = O.SequenceCache(cfg.num_kv_heads, cfg.head_dim, cfg.k_bits[layer],
-                                                       cfg.v_bits[layer], cfg.group_k, cfg.group_v, cfg.residual)
+                                                       cfg.v_bits[layer], cfg.group_k, cfg.group_v, cfg.residual,
+                                                       sinks=cfg.sink_tokens)
 
     def append(self, layer: int, k: torch.Tensor, v: torch.Tensor, new_lens):
         """k, v: [sum(new_lens), Hkv, D] in the cache dtype (any device)."""
@@ -110,6 +111,7 @@ class Twin:
             if (layer, b) in self.ora:
                 o = self.ora[(layer, b)]
                 assert self.gpu.lengths(layer, b) == (o.quantized_tokens, o.residual_tokens), (layer, b)
+                assert self.gpu.sinks(layer, b) == o.sink_tokens, (layer, b, "sinks")
 
     def read_records(self, layer: int, b: int, h: int, nblk: int):
         """Device block records [0, nblk) of (sequence b, KV head h), split into
@@ -152,6 +154,17 @@ class Twin:
             out.append(raw.view(cfg.kv_dtype).float().numpy().reshape(cfg.num_kv_heads, cfg.residual, cfg.head_dim))
         return out
 
+    def read_sinks(self, layer: int, b: int):
+        lay = self.gpu.layout(layer)
+        cfg = self.cfg
+        n = cfg.num_kv_heads * 8 * cfg.head_dim * 2  # KVQ_MAX_SINKS rows per (sequence, KV head)
+        out = []
+        for ptr in (lay.sink_k, lay.sink_v):
+            start = ptr - self.gpu.arena.data_ptr() + b * n
+            raw = self.gpu.arena[start:start + n].cpu()
+            out.append(raw.view(cfg.kv_dtype).float().numpy().reshape(cfg.num_kv_heads, 8, cfg.head_dim))
+        return out
+
     def check_codes(self, layer: int, b: int):
         """Every packed block and ring token of sequence b equals the oracle's, bit for bit."""
         o = self.ora[(layer, b)]
@@ -170,6 +183,11 @@ class Twin:
                     assert np.array_equal(rec["vc"][j], vw), (layer, b, h, j, "value codes")
                     assert np.array_equal(rec["vsz"][j][..., 0].view(np.uint16), blk.vd[:, h].view(np.uint16)), (b, h, j, "value scale")
                     assert np.array_equal(rec["vsz"][j][..., 1].view(np.uint16), blk.vm[:, h].view(np.uint16)), (b, h, j, "value zero")
+        if o.sink_tokens:
+            sk, sv = self.read_sinks(layer, b)
+            for t in range(o.sink_tokens):
+                assert np.array_equal(sk[:, t], o.sink_k[t]), (layer, b, t, "sink key")
+                assert np.array_equal(sv[:, t], o.sink_v[t]), (layer, b, t, "sink value")
         if o.residual_tokens:
             rk, rv = self.read_ring(layer, b)
             Q = o.quantized_tokens
