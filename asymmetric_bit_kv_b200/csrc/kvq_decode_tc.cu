@@ -102,8 +102,11 @@ int mma_ctas_per_sm(const LayerView& L, const MmaPlan& mp, int num_q_heads) {
   if (nmemo + 2 > 256) return 1;
   if (!opted) {
     int optin = 0;
+    cudaFuncAttributes fa;
     if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
-        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess) {
+        cudaFuncGetAttributes(&fa, fn) != cudaSuccess ||
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes) !=
+            cudaSuccess) {
       (void)cudaGetLastError();  // the launch reports its own error, not this one
       return 1;
     }
