@@ -178,13 +178,16 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
 // Log-sum-exp merge of the partial slots of one (sequence, query head):
 // M = max_s m_s over slots with l_s > 0, out = sum_s 2^(m_s-M) o_s / sum_s
 // 2^(m_s-M) l_s, rounded to the output dtype (nearest even); a sequence with
-// no tokens gives zeros. grid (Hq, batch), block D threads (thread d owns
-// channel d). Every thread issues the (m, l) and o loads of 16 slots at once
-// and merges them online, so a typical merge takes one round trip to L2.
+// no tokens gives zeros. One warp per (sequence, query head), lane L owning
+// channels 4L..4L+3 (one 16-byte load per slot); 4 warps per block, grid
+// (ceil(Hq / 4), batch). Every lane issues the loads of 16 slots at once and
+// merges them online, so a typical merge takes one round trip to L2.
 __global__ void __launch_bounds__(128) combine_kernel(CombineParams p) {
   // wait for the decode grid this launch depends on (no-op without one)
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int hq = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hq = blockIdx.x * 4 + warp, b = blockIdx.y;
+  if (hq >= p.num_q_heads) return;
   constexpr int D = kHeadDim;
   constexpr int C = 16;  // slots per batch of loads
   int S;  // slots of this (sequence, head)
@@ -196,15 +199,18 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineParams p) {
     S = (nblk + p.blocks_per_split - 1) / p.blocks_per_split + 1;
   }
   const int64_t base = ((int64_t)b * p.num_q_heads + hq) * p.slots;
-  float M = -INFINITY, acc = 0.f, lsum = 0.f;
+  const float2* ml_p = p.ws_ml + base;
+  const float4* o_p = reinterpret_cast<const float4*>(p.ws_o + base * D) + lane;  // slot s at o_p[s * D / 4]
+  float M = -INFINITY, lsum = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s0 = 0; s0 < S; s0 += C) {
     float2 ml[C];
-    float v[C];
+    float4 v[C];
 #pragma unroll
     for (int e = 0; e < C; ++e) {
       const bool in = s0 + e < S;
-      ml[e] = in ? __ldcg(p.ws_ml + base + s0 + e) : make_float2(-INFINITY, 0.f);
-      v[e] = in ? __ldcg(p.ws_o + (base + s0 + e) * D + d) : 0.f;
+      ml[e] = in ? __ldcg(ml_p + s0 + e) : make_float2(-INFINITY, 0.f);
+      v[e] = in ? __ldcg(o_p + (s0 + e) * (D / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     float mc = M;
 #pragma unroll
@@ -212,23 +218,43 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineParams p) {
       if (ml[e].y > 0.f) mc = fmaxf(mc, ml[e].x);
     if (mc == -INFINITY) continue;  // nothing yet
     const float r = M == -INFINITY ? 0.f : exp2f(M - mc);
-    acc *= r;
+    acc.x *= r;
+    acc.y *= r;
+    acc.z *= r;
+    acc.w *= r;
     lsum *= r;
     M = mc;
 #pragma unroll
     for (int e = 0; e < C; ++e) {
       if (ml[e].y > 0.f) {
         const float w = exp2f(ml[e].x - M);
-        acc += w * v[e];
+        acc.x += w * v[e].x;
+        acc.y += w * v[e].y;
+        acc.z += w * v[e].z;
+        acc.w += w * v[e].w;
         lsum += w * ml[e].y;
       }
     }
   }
-  const float r = lsum > 0.f ? __fdiv_rn(acc, lsum) : 0.f;
-  const int64_t o = ((int64_t)b * p.num_q_heads + hq) * D + d;
-  if (p.out_dtype == KVQ_F32) reinterpret_cast<float*>(p.out)[o] = r;
-  else if (p.out_dtype == KVQ_BF16) reinterpret_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(r);
-  else reinterpret_cast<__half*>(p.out)[o] = __float2half_rn(r);
+  float r[4] = {0.f, 0.f, 0.f, 0.f};
+  if (lsum > 0.f) {
+    r[0] = __fdiv_rn(acc.x, lsum);
+    r[1] = __fdiv_rn(acc.y, lsum);
+    r[2] = __fdiv_rn(acc.z, lsum);
+    r[3] = __fdiv_rn(acc.w, lsum);
+  }
+  const int64_t o = ((int64_t)b * p.num_q_heads + hq) * D + 4 * lane;
+  if (p.out_dtype == KVQ_F32) {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + o) = make_float4(r[0], r[1], r[2], r[3]);
+  } else if (p.out_dtype == KVQ_BF16) {
+    __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>(p.out) + o;
+    *reinterpret_cast<__nv_bfloat162*>(d) = __floats2bfloat162_rn(r[0], r[1]);
+    *reinterpret_cast<__nv_bfloat162*>(d + 2) = __floats2bfloat162_rn(r[2], r[3]);
+  } else {
+    __half* d = reinterpret_cast<__half*>(p.out) + o;
+    *reinterpret_cast<__half2*>(d) = __floats2half2_rn(r[0], r[1]);
+    *reinterpret_cast<__half2*>(d + 2) = __floats2half2_rn(r[2], r[3]);
+  }
 }
 
 template <int NG>
@@ -261,8 +287,8 @@ cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream) {
   // the decode grid (which allows it at its start) is still running; each
   // combine CTA waits for the decode grid to complete before it reads.
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.num_q_heads, p.batch);
-  cfg.blockDim = dim3(kHeadDim);
+  cfg.gridDim = dim3((p.num_q_heads + 3) / 4, p.batch);
+  cfg.blockDim = dim3(128);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
