@@ -299,7 +299,7 @@ namespace kvq {
 // slot count); otherwise in `scratch`, with the slot stride cut to what this
 // call uses, and a call whose partials would not fit is rejected before
 // anything is enqueued.
-kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out, int32_t out_dtype,
+kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const void* new_v, const void* q, void* out, int32_t out_dtype,
                           float softmax_scale, int32_t batch, void* stream, const StaticScratch* scratch) {
   kvq_status s = check_cache_layer(c, layer);
   if (s != KVQ_OK) return s;
@@ -337,6 +337,8 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out,
   kvq::DecodeParams& p = *pp;
   std::memset(pp, 0, offsetof(kvq::DecodeParams, nblk));  // the per-sequence tables are written below
   p.L = L;
+  p.new_k = new_k;
+  p.new_v = new_v;
   p.q = q;
   p.out = out;
   p.ws_o = reinterpret_cast<float*>(c->arena + c->ws_o_off);
@@ -575,7 +577,49 @@ kvq_status kvq_flush_residual(kvq_cache* c, int32_t layer, int32_t batch, void* 
 kvq_status kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, void* out, int32_t out_dtype,
                                 float softmax_scale, int32_t batch, void* stream) {
   g_last_error.clear();
-  return kvq::enqueue_decode(c, layer, q, out, out_dtype, softmax_scale, batch, stream, nullptr);
+  return kvq::enqueue_decode(c, layer, nullptr, nullptr, q, out, out_dtype, softmax_scale, batch, stream, nullptr);
+}
+
+kvq_status kvq_decode_step(kvq_cache* c, int32_t layer, const void* k, const void* v, const void* q, void* out,
+                           int32_t out_dtype, float softmax_scale, int32_t batch, void* stream) {
+  g_last_error.clear();
+  kvq_status s = check_cache_layer(c, layer);
+  if (s != KVQ_OK) return s;
+  if (batch < 0 || batch > c->cfg.max_batch)
+    return fail(KVQ_ERR_INVALID_ARG, "batch %d outside 0..%d", batch, c->cfg.max_batch);
+  if (out_dtype != KVQ_F32 && out_dtype != KVQ_F16 && out_dtype != KVQ_BF16)
+    return fail(KVQ_ERR_INVALID_ARG, "out_dtype %d", out_dtype);
+  if (!std::isfinite(softmax_scale)) return fail(KVQ_ERR_INVALID_ARG, "softmax_scale is not finite");
+  if (batch == 0) return KVQ_OK;
+  if (!k || !v || !q || !out) return fail(KVQ_ERR_INVALID_ARG, "k, v, q or out is null");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(q) || !aligned16(out))
+    return fail(KVQ_ERR_INVALID_ARG, "k, v, q and out must be 16-byte aligned");
+  const kvq_config& cfg = c->cfg;
+  const size_t base = (size_t)layer * cfg.max_batch;
+  // The new tokens ride along with the decode when every one of them lands in
+  // a ring slot without a flush (ring not full, sinks complete) and the layer
+  // runs on the tensor-core kernel; otherwise append, then decode.
+  bool fused = kvq::mma_supported(layer_view(c, layer));
+  for (int b = 0; b < batch; ++b) {
+    const int64_t L = (int64_t)c->s_len[base + b] + c->q_len[base + b] + c->n_len[base + b] + 1;
+    if (L > cfg.max_tokens)
+      return fail(KVQ_ERR_CAPACITY, "sequence %d would hold %lld tokens > max_tokens %d", b, (long long)L,
+                  cfg.max_tokens);
+    if (c->n_len[base + b] >= cfg.residual || c->s_len[base + b] < cfg.sink_tokens) fused = false;
+  }
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!fused) {
+    thread_local std::vector<int32_t> ones;
+    ones.assign(batch, 1);
+    s = enqueue_append(c, layer, k, v, ones.data(), batch, false, st);
+    if (s != KVQ_OK) return s;
+    return kvq::enqueue_decode(c, layer, nullptr, nullptr, q, out, out_dtype, softmax_scale, batch, stream, nullptr);
+  }
+  for (int b = 0; b < batch; ++b) ++c->n_len[base + b];
+  s = kvq::enqueue_decode(c, layer, k, v, q, out, out_dtype, softmax_scale, batch, stream, nullptr);
+  if (s != KVQ_OK)
+    for (int b = 0; b < batch; ++b) --c->n_len[base + b];
+  return s;
 }
 
 kvq_status kvq_dequant(kvq_cache* c, int32_t layer, int32_t seq, int32_t t0, int32_t t1, float* k_out,

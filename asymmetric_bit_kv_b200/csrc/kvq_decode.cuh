@@ -27,6 +27,8 @@ struct DecodeParams {
   void* out;            // [batch][Hq][D], out dtype
   float* ws_o;          // [max_batch][Hq][slots][D] unnormalised partial outputs
   float2* ws_ml;        // [max_batch][Hq][slots]: (running max in log2 units, sum)
+  const void* new_k;    // fused decode step: this call's new token per sequence, [batch][Hkv][D]
+  const void* new_v;    //   (ring index nres[b] - 1; null: no new token)
   float scale_log2;     // softmax scale * log2(e)
   float q_prescale;     // tensor-core kernel: power of two the queries are scaled by in fp16
   float score_scale;    // scale_log2 / q_prescale
@@ -129,7 +131,7 @@ struct StaticScratch {
 
 // Host side of kvq_decode_attention (kvq_api.cu): validation, split plan and
 // launches; the partials go to `scratch` when it is not null.
-kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* q, void* out, int32_t out_dtype,
+kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const void* new_v, const void* q, void* out, int32_t out_dtype,
                           float softmax_scale, int32_t batch, void* stream, const StaticScratch* scratch);
 void clear_last_error();
 kvq_status report_cuda_error(cudaError_t e, const char* what);

@@ -561,6 +561,25 @@ __device__ __forceinline__ int exact_chunk(const DecodeParams& p, int b, int r, 
   return sink ? nsink : nres - r * kResChunk;
 }
 
+// Fused decode step: the copy of the chunk holding this call's new token
+// (ring index nres - 1) took that row from the input (issue_item); the warp
+// also stores it into its ring slot for later calls (no other item of this
+// call reads that slot), and the unit of KV head 0 records the sequence's new
+// ring count.
+__device__ __forceinline__ void store_new_token(const DecodeParams& p, int b, int h, int nb, const uint8_t* stage,
+                                                int lane) {
+  const LayerView& L = p.L;
+  const int i = p.nres[b] - 1;
+  const int row = i % kResChunk;
+  const int slot = (nb * L.group_k + i) % L.residual;
+  const int64_t dst = (((int64_t)b * L.num_kv_heads + h) * L.residual + slot) * kRowBytes;
+  reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(L.ring_k) + dst)[lane] =
+      reinterpret_cast<const uint2*>(stage + row * kRowBytes)[lane];
+  reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(L.ring_v) + dst)[lane] =
+      reinterpret_cast<const uint2*>(stage + (kResChunk + row) * kRowBytes)[lane];
+  if (h == 0 && lane == 0) L.lens[3 * b + 1] = p.nres[b];
+}
+
 // Issue side of a warp's item stream (one lane): the unit of the last issued
 // item and the number of unit changes so far.
 struct IssueState {
@@ -610,8 +629,28 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, const MmaPlan&
     }
     constexpr uint32_t bytes = kResChunk * kRowBytes;
     mbar_expect_tx(bar, 2 * bytes + (newq ? qbytes : 0u));
-    bulk_g2s(dst, reinterpret_cast<const uint8_t*>(ksrc) + row * kRowBytes, bytes, bar);
-    bulk_g2s(dst + bytes, reinterpret_cast<const uint8_t*>(vsrc) + row * kRowBytes, bytes, bar);
+    const uint8_t* kr = reinterpret_cast<const uint8_t*>(ksrc) + row * kRowBytes;
+    const uint8_t* vr = reinterpret_cast<const uint8_t*>(vsrc) + row * kRowBytes;
+    if (p.new_k && !sink && j - nb == (p.nres[u.b] - 1) / kResChunk) {
+      // fused decode step: row i of this chunk is the new token, from the
+      // input; the ring rows around it as they are
+      const int i = (p.nres[u.b] - 1) % kResChunk;
+      const uint32_t lo = i * kRowBytes, hi = (kResChunk - 1 - i) * kRowBytes;
+      const int64_t in = ((int64_t)u.b * L.num_kv_heads + u.h) * kRowBytes;
+      if (lo) {
+        bulk_g2s(dst, kr, lo, bar);
+        bulk_g2s(dst + bytes, vr, lo, bar);
+      }
+      if (hi) {
+        bulk_g2s(dst + lo + kRowBytes, kr + lo + kRowBytes, hi, bar);
+        bulk_g2s(dst + bytes + lo + kRowBytes, vr + lo + kRowBytes, hi, bar);
+      }
+      bulk_g2s(dst + lo, reinterpret_cast<const uint8_t*>(p.new_k) + in, kRowBytes, bar);
+      bulk_g2s(dst + bytes + lo, reinterpret_cast<const uint8_t*>(p.new_v) + in, kRowBytes, bar);
+    } else {
+      bulk_g2s(dst, kr, bytes, bar);
+      bulk_g2s(dst + bytes, vr, bytes, bar);
+    }
   }
   if (newq)
     bulk_g2s(qbuf + (size_t)(is.seq % mp.nstages) * qbytes,
@@ -830,6 +869,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
         } else {
           bool sink;
           const int cnt = exact_chunk(p, u.b, j - nb, sink);
+          if (p.new_k && !sink && j - nb == (p.nres[u.b] - 1) / kResChunk) store_new_token(p, u.b, u.h, nb, stage, lane);
           if (bf16)
             ring_chunk<true, VB, NGRP, NKT>(stage, qw, bkw, cnt, NG, lane, p.score_scale, valid, rq_ready, sst, O, Z);
           else

@@ -51,7 +51,7 @@ kvq_status kvq_decode_attention_noalloc(kvq_cache* c, int32_t layer, const void*
   uint8_t* base = scratch_address(&e);
   if (!base) return kvq::report_cuda_error(e, "looking up the static decode scratch");
   const kvq::StaticScratch scratch{base, (int64_t)KVQ_STATIC_SCRATCH_BYTES};
-  return kvq::enqueue_decode(c, layer, q, out, out_dtype, softmax_scale, batch, stream, &scratch);
+  return kvq::enqueue_decode(c, layer, nullptr, nullptr, q, out, out_dtype, softmax_scale, batch, stream, &scratch);
 }
 
 }  // extern "C"

@@ -88,6 +88,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kvq_flush_residual": (I32, [P, I32, I32, P]),
         "kvq_decode_attention": (I32, [P, I32, P, P, I32, F32, I32, P]),
         "kvq_decode_attention_noalloc": (I32, [P, I32, P, P, I32, F32, I32, P]),
+        "kvq_decode_step": (I32, [P, I32, P, P, P, P, I32, F32, I32, P]),
         "kvq_dequant": (I32, [P, I32, I32, I32, I32, P, P, P]),
         "kvq_get_layout": (I32, [P, I32, ctypes.POINTER(kvq_layout)]),
         "kvq_device_errors": (I32, [P, ctypes.POINTER(I32)]),
@@ -221,6 +222,24 @@ class KVCache:
         _check(self.lib.kvq_decode_attention(self.handle, layer, q.data_ptr(), out.data_ptr(), _DTYPE_CODE[out.dtype],
                                              float(softmax_scale), q.shape[0], _stream_ptr(stream)),
                "kvq_decode_attention")
+        return out
+
+    def decode_step(self, layer: int, k: torch.Tensor, v: torch.Tensor, q: torch.Tensor,
+                    out: torch.Tensor | None = None, out_dtype=torch.float32, softmax_scale: float | None = None,
+                    stream=None):
+        """Append one token per sequence (k, v: [batch, Hkv, D]) and decode
+        (q: [batch, Hq, D]); kvq_decode_step. Returns out [batch, Hq, D]."""
+        _need(k, self.cfg.kv_dtype, "k")
+        _need(v, self.cfg.kv_dtype, "v")
+        _need(q, self.cfg.kv_dtype, "q")
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        _need(out, out.dtype, "out")
+        if softmax_scale is None:
+            softmax_scale = self.cfg.head_dim ** -0.5
+        _check(self.lib.kvq_decode_step(self.handle, layer, k.data_ptr(), v.data_ptr(), q.data_ptr(), out.data_ptr(),
+                                        _DTYPE_CODE[out.dtype], float(softmax_scale), q.shape[0], _stream_ptr(stream)),
+               "kvq_decode_step")
         return out
 
     def decode_attention_noalloc(self, layer: int, q: torch.Tensor, out: torch.Tensor,

@@ -286,8 +286,6 @@ def run_kvq(a):
     new_v = torch.randn(pool, B, Hkv, D, generator=gen, device=dev).to(wl.kv_dtype)
     qs = torch.randn(pool, B, Hq, D, generator=gen, device=dev).to(wl.kv_dtype)
     out = torch.empty(B, Hq, D, dtype=wl.kv_dtype, device=dev)
-    from asymmetric_bit_kv_b200.kvq import lens_array
-    ones = lens_array([1] * B)
     stream = torch.cuda.current_stream()
     # per-step inputs as views made once, so that the timed loop only enqueues
     views = [(new_k[j], new_v[j], qs[j]) for j in range(pool)]
@@ -295,12 +293,13 @@ def run_kvq(a):
 
     G, Rw = wl.group_k, wl.residual
 
-    # The device-timed loop calls the C entry points (kvq_append,
-    # kvq_decode_attention) with arguments prepared here, so that Python
-    # overhead per call stays far below the GPU time of a step; the e2e leg
-    # below goes through the Python binding.
+    # The device-timed loop calls the C entry point kvq_decode_step (append
+    # one token per sequence + decode attention; the append rides inside the
+    # decode launch unless a ring must be flushed) with arguments prepared
+    # here, so that Python overhead per call stays far below the GPU time of a
+    # step; the e2e leg below goes through the Python binding.
     lib = caches[0].lib
-    c_append, c_decode = lib.kvq_append, lib.kvq_decode_attention
+    c_step = lib.kvq_decode_step
     sh = stream.cuda_stream
     handles = [c.handle for c in caches]
     ptrs = [(kk.data_ptr(), vv.data_ptr(), qq.data_ptr()) for kk, vv, qq in views]
@@ -309,10 +308,9 @@ def run_kvq(a):
     def step(i, r, ev=None):
         kp, vp, qp = ptrs[i % pool]
         h = handles[r]
-        st = c_append(h, 0, kp, vp, ones, B, sh)
         if ev is not None:
             ev[0].record(stream)
-        st |= c_decode(h, 0, qp, optr, oty, scale, B, sh)
+        st = c_step(h, 0, kp, vp, qp, optr, oty, scale, B, sh)
         if ev is not None:
             ev[1].record(stream)
         if st:
@@ -329,11 +327,13 @@ def run_kvq(a):
     # flush rule (a token that finds a full ring first moves G ring tokens into
     # the quantized cache), checked against the library's host mirror after.
     lens = [[list(caches[r].lengths(0, b)) for b in range(B)] for r in range(R)]
-    plan = []  # (replica, launches, algorithmic bytes of the decode, KV tokens attended)
+    plan = []  # (replica, launches, algorithmic bytes of the step, KV tokens attended)
     for i in range(a.steps):
         r = (a.warmup + i) % R
-        launches = 3 + (1 if lens[r][0][1] == Rw else 0)  # ring write + decode + combine (+ flush)
-        ab, tk = 2 * B * Hq * D * 2, 0  # q in, out
+        # fused: decode + combine; a step that flushes a ring first runs the
+        # quantize and ring-write kernels
+        launches = 2 + (2 if lens[r][0][1] == Rw else 0)
+        ab, tk = 2 * B * Hq * D * 2 + 2 * (2 * B * Hkv * D * 2), 0  # q in, out; new k, v in and into the ring
         for b in range(B):
             qn, n = lens[r][b]
             if n == Rw:
@@ -406,8 +406,7 @@ def run_kvq(a):
         dk.copy_(hk[j], non_blocking=True)
         dv.copy_(hv[j], non_blocking=True)
         dq.copy_(hq[j], non_blocking=True)
-        caches[r].append(0, dk, dv, ones, stream=stream)
-        caches[r].decode_attention(0, dq, out, softmax_scale=wl.softmax_scale, stream=stream)
+        caches[r].decode_step(0, dk, dv, dq, out, softmax_scale=wl.softmax_scale, stream=stream)
         hout.copy_(out, non_blocking=True)
     f1.record(stream)
     torch.cuda.synchronize()
@@ -434,7 +433,7 @@ def run_kvq(a):
             "data": "synthetic (seeded; Llama-3-8B-shaped layer, no model weights)",
             "config": _workload_config(wl, R, world, tok_total / (a.steps * B)),
             "roofline": {
-                "kernel": "decode attention (split-KV kernel + log-sum-exp combine), per call",
+                "kernel": "decode step: one token appended per sequence inside the split-KV decode kernel, + log-sum-exp combine, per call (a ring flush adds the quantize and ring kernels)",
                 "bound": "hbm",
                 "achieved": achieved_gbs,
                 "peak": peak,

@@ -208,6 +208,18 @@ KVQ_API kvq_status kvq_decode_attention_noalloc(kvq_cache* cache, int32_t layer,
                                         int32_t out_dtype, float softmax_scale, int32_t batch,
                                         void* stream);
 
+/* One decode step: append one token to each sequence b < batch (k, v:
+ * device [batch][num_kv_heads][head_dim] in kv_dtype, as kvq_append with
+ * new_lens all 1), then decode attention for q over every token including
+ * the new one (as kvq_decode_attention). Same results as those two calls;
+ * when no sequence needs a flush or a sink (its ring not full, its sinks
+ * complete) and the layer runs on the tensor-core kernel, the new tokens are
+ * written and attended to inside the decode launch (one launch fewer; the
+ * fused append+decode step the KV1 card's quantize-on-entry decode loop
+ * suggests). All checks run before anything is enqueued.                  */
+KVQ_API kvq_status kvq_decode_step(kvq_cache* cache, int32_t layer, const void* k, const void* v, const void* q,
+                                   void* out, int32_t out_dtype, float softmax_scale, int32_t batch, void* stream);
+
 /* Reconstruct tokens [t0, t1) of sequence `seq` as fp32: x_hat = q*d + m
  * (an fp32 product, then an fp32 sum; KV1 card, BQ2_0) for quantized tokens
  * and the exact stored value for sink and ring tokens (t counts every token
