@@ -49,6 +49,17 @@ the design notes of the repository):
    and never quantized; everything above (ring, flushes, key groups) applies
    to the tokens after them, so key group j covers tokens S + jG .. S + jG +
    G - 1. Decode attention reads the sinks exactly, like the ring.
+7. BQ2_0 ("KV1-1.2B" card, Quantization Format): keys quantized per token
+   (``k_axis = 1``) are grouped like values, over ``group_v`` channels of one
+   (token, KV head). The Hadamard rotation (``hadamard``) multiplies every
+   stored K and V head vector by the normalized Sylvester matrix H (H.H = I)
+   before it is quantized; here it is applied when a block is quantized, so
+   the ring and the sinks keep the exact tokens. Scores of quantized tokens
+   use Hq and their values' contribution is multiplied by H again, i.e.
+   attention sees the effective keys and values (dequantized) . H. In fp32 the
+   product x.H is the radix-2 butterfly (stages of half-width 1, 2, 4, ...;
+   a pair (a, b) becomes (a + b, a - b), each one fp32 rounding) followed by
+   one fp32 multiplication by fp32(1/sqrt(D)).
 
 Floating point: the quantizer runs in IEEE fp32 (the precision the KV1 card
 fixes); numpy evaluates each fp32 operation with one rounding and never
@@ -194,6 +205,37 @@ def pack_value_block(codes: np.ndarray, bits: int) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # Cache state machine (KIVI README: residual window of recent fp16 tokens)
 # ---------------------------------------------------------------------------
+# Hadamard rotation ("KV1-1.2B", BQ2_0: normalized Sylvester Hadamard matrix)
+# ---------------------------------------------------------------------------
+
+
+def sylvester(D: int) -> np.ndarray:
+    """The normalized D x D Sylvester Hadamard matrix in fp64 (H . H = I)."""
+    H = np.array([[1.0]])
+    while H.shape[0] < D:
+        H = np.block([[H, H], [H, -H]])
+    assert H.shape[0] == D, "D must be a power of two"
+    return H / np.sqrt(D)
+
+
+def rotate_fp32(x: np.ndarray) -> np.ndarray:
+    """x . H over the last axis in fp32: the butterfly stages of half-width
+    1, 2, 4, ... D/2 (pair (a, b) at positions i, i + w with bit w of i clear
+    becomes (a + b, a - b)), then one multiplication by fp32(1/sqrt(D))."""
+    y = np.array(x, dtype=F32, copy=True)
+    D = y.shape[-1]
+    w = 1
+    while w < D:
+        v = y.reshape(y.shape[:-1] + (D // (2 * w), 2, w))
+        a = v[..., 0, :].copy()
+        b = v[..., 1, :].copy()
+        v[..., 0, :] = a + b
+        v[..., 1, :] = a - b
+        w *= 2
+    return (y * F32(1.0 / np.sqrt(D))).astype(F32)
+
+
+# ---------------------------------------------------------------------------
 
 
 class QuantizedBlock:
@@ -210,12 +252,14 @@ class SequenceCache:
     cache's storage type (fp16 or bf16); the ring keeps them unchanged.
     """
 
-    def __init__(self, num_kv_heads, head_dim, k_bits, v_bits, group_k, group_v, residual, sinks=0):
-        assert residual % group_k == 0 and residual >= group_k and sinks >= 0
+    def __init__(self, num_kv_heads, head_dim, k_bits, v_bits, group_k, group_v, residual, sinks=0, k_axis=0,
+                 hadamard=False):
+        assert residual % group_k == 0 and residual >= group_k and sinks >= 0 and k_axis in (0, 1)
         self.H, self.D = num_kv_heads, head_dim
         self.k_bits, self.v_bits = k_bits, v_bits
         self.group_k, self.group_v, self.residual = group_k, group_v, residual
         self.sinks = sinks
+        self.k_axis, self.hadamard = k_axis, bool(hadamard)
         self.sink_k: list[np.ndarray] = []  # the first `sinks` tokens, exact, each [H, D]
         self.sink_v: list[np.ndarray] = []
         self.blocks: list[QuantizedBlock] = []
@@ -244,7 +288,12 @@ class SequenceCache:
         v = np.stack(self.ring_v[:G]).astype(F32)
         del self.ring_k[:G]
         del self.ring_v[:G]
-        kc, kd, km = quantize_key_block(k, self.k_bits)
+        if self.hadamard:
+            k, v = rotate_fp32(k), rotate_fp32(v)
+        if self.k_axis == 1:  # per-token keys, grouped like values
+            kc, kd, km = quantize_value_block(k, self.k_bits, self.group_v)
+        else:
+            kc, kd, km = quantize_key_block(k, self.k_bits)
         vc, vd, vm = quantize_value_block(v, self.v_bits, self.group_v)
         self.blocks.append(QuantizedBlock(kc, kd, km, vc, vd, vm))
 
@@ -270,23 +319,34 @@ class SequenceCache:
         while len(self.ring_k) >= self.group_k:
             self._flush_oldest_block()
 
-    def dequantized(self):
+    def dequantized(self, effective=False):
         """(K~, V~) as fp32 [L, H, D] in token order: the exact sinks, the
-        dequantized blocks, then the ring."""
+        dequantized blocks (as stored: in the rotated basis for a Hadamard
+        cache), then the ring. effective=True: fp64, with the blocks rotated
+        back (. H), the keys and values attention sees."""
         ks, vs = [], []
         if self.sink_k:
             ks.append(np.stack(self.sink_k))
             vs.append(np.stack(self.sink_v))
+        Hm = sylvester(self.D) if (effective and self.hadamard) else None
         for b in self.blocks:
-            ks.append(dequantize_key_block(b.kc, b.kd, b.km))
-            vs.append(dequantize_value_block(b.vc, b.vd, b.vm))
+            if self.k_axis == 1:
+                kq = dequantize_value_block(b.kc, b.kd, b.km)
+            else:
+                kq = dequantize_key_block(b.kc, b.kd, b.km)
+            vq = dequantize_value_block(b.vc, b.vd, b.vm)
+            if Hm is not None:
+                kq, vq = kq.astype(np.float64) @ Hm, vq.astype(np.float64) @ Hm
+            ks.append(kq)
+            vs.append(vq)
         if self.ring_k:
             ks.append(np.stack(self.ring_k))
             vs.append(np.stack(self.ring_v))
+        dt = np.float64 if effective else F32
         if not ks:
-            z = np.zeros((0, self.H, self.D), F32)
+            z = np.zeros((0, self.H, self.D), dt)
             return z, z.copy()
-        return np.concatenate(ks).astype(F32), np.concatenate(vs).astype(F32)
+        return np.concatenate(ks).astype(dt), np.concatenate(vs).astype(dt)
 
 
 # ---------------------------------------------------------------------------
@@ -320,8 +380,8 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.n
 
 def decode_attention(cache: SequenceCache, q: np.ndarray, scale: float) -> np.ndarray:
     """Decode attention of one sequence over its sinks, quantized blocks and
-    ring."""
-    k, v = cache.dequantized()
+    ring (for a Hadamard cache, the effective keys and values)."""
+    k, v = cache.dequantized(effective=True)
     return attention(q, k, v, scale)
 
 
@@ -330,12 +390,14 @@ def decode_attention(cache: SequenceCache, q: np.ndarray, scale: float) -> np.nd
 # ---------------------------------------------------------------------------
 
 
-def quantized_bytes_per_token(num_kv_heads, head_dim, k_bits, v_bits, group_k, group_v) -> float:
+def quantized_bytes_per_token(num_kv_heads, head_dim, k_bits, v_bits, group_k, group_v, k_axis=0) -> float:
     """Bytes per cached token over all KV heads of one layer.
 
     Codes take ``D*(bk+bv)/8`` bytes; each key group (one channel over group_k
-    tokens) and each value group (group_v channels of one token) adds an fp16
-    scale and an fp16 zero point, i.e. 4 bytes.
+    tokens, or group_v channels of one token with per-token keys) and each
+    value group (group_v channels of one token) adds an fp16 scale and an
+    fp16 zero point, i.e. 4 bytes.
     """
     D = head_dim
-    return num_kv_heads * (D * (k_bits + v_bits) / 8 + 4 * D / group_k + 4 * D / group_v)
+    kgroups = D / group_v if k_axis == 1 else D / group_k
+    return num_kv_heads * (D * (k_bits + v_bits) / 8 + 4 * kgroups + 4 * D / group_v)

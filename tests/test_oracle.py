@@ -408,6 +408,88 @@ def test_short_sequence_is_all_sinks_and_exact():
 
 
 # --------------------------------------------------------------------------
+# BQ2_0: Hadamard rotation and per-token keys (KV1-1.2B card, BQ2_0)
+# --------------------------------------------------------------------------
+
+
+def test_rotation_hand_example_and_basis_columns():
+    # [1, 2, 3, 4] . H4 = [10, -2, -4, 0] / 2 (H4 symmetric)
+    assert np.array_equal(O.rotate_fp32(np.array([1, 2, 3, 4], np.float32)), np.array([5, -1, -2, 0], np.float32))
+    D = 128
+    H = O.sylvester(D)
+    assert np.allclose(H @ H, np.eye(D), atol=1e-12) and np.array_equal(H, H.T)
+    s = np.float32(1.0 / np.sqrt(D))
+    for i in (0, 1, 37, 127):
+        e = np.zeros(D, np.float32)
+        e[i] = 1.0
+        # butterflies of a basis vector give exactly +-1: one rounding, by s
+        assert np.array_equal(O.rotate_fp32(e), (np.sign(H[i]) * s).astype(np.float32))
+
+
+def test_rotation_is_the_matrix_product_and_an_involution():
+    D = 128
+    rng = np.random.default_rng(50)
+    x = rng.standard_normal((7, 3, D)).astype(np.float32)
+    H = O.sylvester(D)
+    y = O.rotate_fp32(x)
+    ref = x.astype(np.float64) @ H
+    assert np.abs(y - ref).max() <= 1e-5 * np.abs(x).max()   # 7 fp32 roundings of partial sums
+    assert np.abs(O.rotate_fp32(y) - x).max() <= 2e-5 * np.abs(x).max()
+
+
+def test_per_token_key_blocks_use_the_value_quantizer():
+    H, D, G, Gv, R = 2, 64, 32, 64, 64
+    rng = np.random.default_rng(51)
+    k = (rng.standard_normal((G + 3, H, D)) * 2).astype(np.float32)
+    v = rng.standard_normal((G + 3, H, D)).astype(np.float32)
+    c = O.SequenceCache(H, D, 2, 2, G, Gv, R, k_axis=1)
+    c.append(k, v)
+    c.flush_residual()
+    blk = c.blocks[0]
+    kc, kd, km = O.quantize_groups(k[:G].reshape(G, H, 1, D), 2)  # one group per (token, head) over 64 channels
+    assert np.array_equal(blk.kc, kc.reshape(G, H, D)) and np.array_equal(blk.kd, kd) and np.array_equal(blk.km, km)
+    # BQ2_0 size: 2-bit codes of 64 values + fp16 scale and zero = 20 bytes
+    assert O.quantized_bytes_per_token(1, 64, 2, 2, 32, 64, k_axis=1) == 40.0
+
+
+def test_hadamard_cache_quantizes_rotated_vectors_and_attends_in_the_original_basis():
+    H, D, G, Gv, R = 2, 128, 32, 64, 64
+    rng = np.random.default_rng(52)
+    L = 3 * G + 40
+    k = (rng.standard_normal((L, H, D)) * np.exp(rng.standard_normal((1, H, D)))).astype(np.float32)
+    v = rng.standard_normal((L, H, D)).astype(np.float32)
+    c = O.SequenceCache(H, D, 2, 4, G, Gv, R, k_axis=1, hadamard=True)
+    c.append(k, v)
+    # the stored blocks are the quantizer applied to the rotated tokens
+    kc, kd, km = O.quantize_value_block(O.rotate_fp32(k[:G]), 2, Gv)
+    assert np.array_equal(c.blocks[0].kc, kc) and np.array_equal(c.blocks[0].kd, kd)
+    vc, vd, vm = O.quantize_value_block(O.rotate_fp32(v[:G]), 4, Gv)
+    assert np.array_equal(c.blocks[0].vc, vc) and np.array_equal(c.blocks[0].vm, vm)
+    # attention computed independently in the rotated basis: scores of
+    # quantized tokens from Hq, their values' contribution multiplied by H
+    Hm = O.sylvester(D)
+    q = rng.standard_normal((8, D))
+    Ks, Vs = c.dequantized()            # stored basis
+    Q = c.quantized_tokens
+    scale = D ** -0.5
+    out = np.zeros((8, D))
+    for h in range(8):
+        kv = h // 4
+        s_q = scale * (Ks[:Q, kv].astype(np.float64) @ (Hm @ q[h]))
+        s_r = scale * (Ks[Q:, kv].astype(np.float64) @ q[h])
+        s_all = np.concatenate([s_q, s_r])
+        p = np.exp(s_all - s_all.max())
+        o_rot = p[:Q] @ Vs[:Q, kv].astype(np.float64)
+        out[h] = (Hm @ o_rot + p[Q:] @ Vs[Q:, kv].astype(np.float64)) / p.sum()
+    assert np.abs(O.decode_attention(c, q, scale) - out).max() < 1e-12
+    # with 8-bit codes the rotated cache stays close to exact attention on the
+    # raw tokens (a missing or transposed rotation would not)
+    c8 = O.SequenceCache(H, D, 8, 8, G, Gv, R, k_axis=1, hadamard=True)
+    c8.append(k, v)
+    assert np.abs(O.decode_attention(c8, q, scale) - _sdpa(q, k, v, scale)).max() < 0.05
+
+
+# --------------------------------------------------------------------------
 # Sizes (KV1-1.2B card, Memory)
 # --------------------------------------------------------------------------
 
