@@ -17,8 +17,8 @@
 #include "kvq_decode.cuh"
 
 struct kvq_cache {
-  kvq_config cfg;                 // k_bits / v_bits point at the vectors below
-  std::vector<int8_t> k_bits, v_bits;
+  kvq_config cfg;                 // k_bits / v_bits / k_axis point at the vectors below
+  std::vector<int8_t> k_bits, v_bits, k_axis;
   uint8_t* arena;
   size_t arena_bytes;
   int device;
@@ -84,6 +84,11 @@ kvq_status validate_config(const kvq_config* c) {
   for (int l = 0; l < c->num_layers; ++l)
     if (!is_bits(c->k_bits[l]) || !is_bits(c->v_bits[l]))
       return fail(KVQ_ERR_UNSUPPORTED, "layer %d bits k=%d v=%d not in {2,4,8}", l, c->k_bits[l], c->v_bits[l]);
+  if (c->k_axis)
+    for (int l = 0; l < c->num_layers; ++l)
+      if (c->k_axis[l] != 0 && c->k_axis[l] != 1)
+        return fail(KVQ_ERR_INVALID_ARG, "layer %d k_axis %d not 0 or 1", l, c->k_axis[l]);
+  if (c->hadamard != 0 && c->hadamard != 1) return fail(KVQ_ERR_INVALID_ARG, "hadamard %d not 0 or 1", c->hadamard);
   return KVQ_OK;
 }
 
@@ -102,7 +107,9 @@ Plan make_plan(const kvq_config* c) {
   int64_t off = 0;
   for (int l = 0; l < c->num_layers; ++l) {
     const int kb = c->k_bits[l], vb = c->v_bits[l];
-    const int64_t rec = round_up(kvq::kc_bytes(G, D, kb) + kvq::ksz_bytes(D) + kvq::vc_bytes(G, D, vb) +
+    const bool per_token = c->k_axis && c->k_axis[l] == 1;
+    const int64_t ksz = per_token ? kvq::ksz_token_bytes(G, D, c->group_v) : kvq::ksz_bytes(D);
+    const int64_t rec = round_up(kvq::kc_bytes(G, D, kb) + ksz + kvq::vc_bytes(G, D, vb) +
                                      kvq::vsz_bytes(G, D, c->group_v),
                                  16);
     p.record_bytes.push_back(rec);
@@ -158,7 +165,9 @@ kvq::LayerView layer_view(const kvq_cache* c, int layer) {
   v.max_blocks = c->max_blocks;
   v.kc_off = 0;
   v.ksz_off = (int32_t)kvq::kc_bytes(G, D, kb);
-  v.vc_off = v.ksz_off + (int32_t)kvq::ksz_bytes(D);
+  v.k_axis = c->k_axis[layer];
+  v.hadamard = cfg.hadamard;
+  v.vc_off = v.ksz_off + (int32_t)(v.k_axis == 1 ? kvq::ksz_token_bytes(G, D, cfg.group_v) : kvq::ksz_bytes(D));
   v.vsz_off = v.vc_off + (int32_t)kvq::vc_bytes(G, D, vb);
   v.k_bits = kb;
   v.v_bits = vb;
@@ -472,8 +481,11 @@ kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena
   c->cfg = *cfg;
   c->k_bits.assign(cfg->k_bits, cfg->k_bits + cfg->num_layers);
   c->v_bits.assign(cfg->v_bits, cfg->v_bits + cfg->num_layers);
+  if (cfg->k_axis) c->k_axis.assign(cfg->k_axis, cfg->k_axis + cfg->num_layers);
+  else c->k_axis.assign(cfg->num_layers, 0);
   c->cfg.k_bits = c->k_bits.data();
   c->cfg.v_bits = c->v_bits.data();
+  c->cfg.k_axis = c->k_axis.data();
   c->arena = static_cast<uint8_t*>(dev_arena);
   c->arena_bytes = arena_bytes;
   c->blocks_off = plan.blocks_off;
@@ -670,6 +682,8 @@ kvq_status kvq_get_layout(const kvq_cache* c, int32_t layer, kvq_layout* out) {
   out->v_bits = v.v_bits;
   out->sink_k = v.sink_k;
   out->sink_v = v.sink_v;
+  out->k_axis = v.k_axis;
+  out->hadamard = v.hadamard;
   return KVQ_OK;
 }
 

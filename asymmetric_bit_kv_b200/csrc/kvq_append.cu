@@ -21,18 +21,58 @@ __device__ __forceinline__ float bits_to_float(uint16_t v, int dtype) {
 
 }  // namespace
 
-// grid (max flush blocks, batch, Hkv); block kQuantThreads; dynamic smem 2*G*D*2 bytes.
+// One group quantizer pass over rows of D values: every (row, run of gv
+// channels) is one group; each thread owns one output word (32/bits
+// channels) and the gv/(32/bits) threads of a group combine their min/max
+// with xor shuffles. val(t, d) reads value d of row t; put_word(t, w, word)
+// and put_sz(t, g, d16, m16) store the codes and the group's scale and zero.
+template <class Val, class PutWord, class PutSz>
+__device__ __forceinline__ void quantize_rows(int rows, int D, int bits, int gv, Val val, PutWord put_word,
+                                              PutSz put_sz) {
+  const int per = 32 / bits;
+  const int wpt = D / per;  // words per row
+  const int P = gv / per;   // threads per group, a power of two <= 32
+  for (int widx = threadIdx.x; widx < rows * wpt; widx += blockDim.x) {
+    const int t = widx / wpt, w = widx % wpt;
+    float mn = val(t, w * per), mx = mn;
+    for (int i = 1; i < per; ++i) {
+      const float x = val(t, w * per + i);
+      mn = fminf(mn, x);
+      mx = fmaxf(mx, x);
+    }
+    for (int o = P / 2; o >= 1; o >>= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    const GroupParams gp = group_params(mn, mx, bits);
+    uint32_t word = 0;
+    for (int i = 0; i < per; ++i) word |= quant_code(val(t, w * per + i), gp, bits) << (i * bits);
+    put_word(t, w, word);
+    if ((w % P) == 0) put_sz(t, w / P, gp.d16, gp.m16);
+  }
+}
+
+// grid (max flush blocks, batch, Hkv); block kQuantThreads; dynamic smem
+// 2*G*D*2 bytes (ROT: 2*G*D*4). ROT: the G x D block of keys and of values is
+// staged as fp32 and every token's head vector is multiplied by the
+// normalized Sylvester Hadamard matrix (radix-2 butterflies of half-width 1,
+// 2, 4, ..., then one fp32 multiplication by fp32(1/sqrt(D))) before it is
+// quantized ("KV1-1.2B" card, BQ2_0).
+template <bool ROT>
 __global__ void __launch_bounds__(kQuantThreads) quantize_blocks_kernel(AppendParams p) {
   const int j = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
   if (j >= p.flush[b]) return;
   const LayerView& L = p.L;
   const int G = L.group_k, D = L.head_dim, R = L.residual;
   const int kb = L.k_bits, vb = L.v_bits, Gv = L.group_v;
-  extern __shared__ uint16_t smem[];
-  uint16_t* sk = smem;              // [G][D]
-  uint16_t* sv = smem + G * D;      // [G][D]
+  const int dt = L.kv_dtype;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint16_t* sk = reinterpret_cast<uint16_t*>(smem_raw);  // [G][D] raw (not ROT)
+  uint16_t* sv = sk + G * D;
+  float* fk = reinterpret_cast<float*>(smem_raw);  // [G][D] fp32 (ROT)
+  float* fv = fk + G * D;
 
-  const int first = p.q_old[b] + j * G;  // absolute index of the block's first token
+  const int first = p.q_old[b] + j * G;  // position of the block's first token (after the sinks)
   const int boundary = p.q_old[b] + p.n_old[b];
   const int64_t ring_base = ((int64_t)b * L.num_kv_heads + h) * R;
   // Stage the G x D block, 8 values (16 bytes) per load.
@@ -52,66 +92,90 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_blocks_kernel(AppendPa
       ksrc = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.k_in) + off);
       vsrc = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.v_in) + off);
     }
-    *reinterpret_cast<uint4*>(sk + t * D + c) = *ksrc;
-    *reinterpret_cast<uint4*>(sv + t * D + c) = *vsrc;
+    const uint4 kx = *ksrc, vx = *vsrc;
+    if constexpr (ROT) {
+      const uint16_t* k16 = reinterpret_cast<const uint16_t*>(&kx);
+      const uint16_t* v16 = reinterpret_cast<const uint16_t*>(&vx);
+      for (int e = 0; e < 8; ++e) {
+        fk[t * D + c + e] = bits_to_float(k16[e], dt);
+        fv[t * D + c + e] = bits_to_float(v16[e], dt);
+      }
+    } else {
+      *reinterpret_cast<uint4*>(sk + t * D + c) = kx;
+      *reinterpret_cast<uint4*>(sv + t * D + c) = vx;
+    }
   }
   __syncthreads();
+  if constexpr (ROT) {
+    for (int w = 1; w < D; w *= 2) {
+      for (int idx = threadIdx.x; idx < 2 * G * (D / 2); idx += blockDim.x) {
+        float* x = (idx < G * (D / 2) ? fk : fv);
+        const int r = idx % (G * (D / 2));
+        const int t = r / (D / 2), pi = r % (D / 2);
+        const int i = t * D + (pi / w) * 2 * w + pi % w;  // bit w of the channel clear
+        const float a = x[i], c = x[i + w];
+        x[i] = __fadd_rn(a, c);
+        x[i + w] = __fsub_rn(a, c);
+      }
+      __syncthreads();
+    }
+    const float s = (float)(1.0 / sqrt((double)D));
+    for (int idx = threadIdx.x; idx < 2 * G * D; idx += blockDim.x) {
+      float* x = idx < G * D ? fk : fv;
+      x[idx % (G * D)] = __fmul_rn(x[idx % (G * D)], s);
+    }
+    __syncthreads();
+  }
+  auto kval = [&](int t, int d) -> float {
+    if constexpr (ROT) return fk[t * D + d];
+    else return bits_to_float(sk[t * D + d], dt);
+  };
+  auto vval = [&](int t, int d) -> float {
+    if constexpr (ROT) return fv[t * D + d];
+    else return bits_to_float(sv[t * D + d], dt);
+  };
 
   uint8_t* rec = record_ptr(L, b, h, p.q_old[b] / G + j);
   uint32_t* kc = reinterpret_cast<uint32_t*>(rec + L.kc_off);
   __half2* ksz = reinterpret_cast<__half2*>(rec + L.ksz_off);
   uint32_t* vc = reinterpret_cast<uint32_t*>(rec + L.vc_off);
   __half* vsz = reinterpret_cast<__half*>(rec + L.vsz_off);
-  const int dt = L.kv_dtype;
 
-  // Keys: one group per channel over the G tokens (KIVI: per-channel keys).
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float mn = bits_to_float(sk[d], dt), mx = mn;
-    for (int t = 1; t < G; ++t) {
-      const float x = bits_to_float(sk[t * D + d], dt);
-      mn = fminf(mn, x);
-      mx = fmaxf(mx, x);
+  if (L.k_axis == 0) {
+    // Keys: one group per channel over the G tokens (KIVI: per-channel keys).
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+      float mn = kval(0, d), mx = mn;
+      for (int t = 1; t < G; ++t) {
+        const float x = kval(t, d);
+        mn = fminf(mn, x);
+        mx = fmaxf(mx, x);
+      }
+      const GroupParams gp = group_params(mn, mx, kb);
+      ksz[d] = __halves2half2(gp.d16, gp.m16);
+      const int per = 32 / kb;
+      const int nw = G / per;  // words per channel, stored contiguously
+      for (int w = 0; w < nw; ++w) {
+        uint32_t word = 0;
+        for (int i = 0; i < per; ++i) word |= quant_code(kval(w * per + i, d), gp, kb) << (i * kb);
+        kc[kc_word_index(d, w, nw)] = word;
+      }
     }
-    const GroupParams gp = group_params(mn, mx, kb);
-    ksz[d] = __halves2half2(gp.d16, gp.m16);
-    const int per = 32 / kb;
-    const int nw = G / per;  // words per channel, stored contiguously
-    for (int w = 0; w < nw; ++w) {
-      uint32_t word = 0;
-      for (int i = 0; i < per; ++i)
-        word |= quant_code(bits_to_float(sk[(w * per + i) * D + d], dt), gp, kb) << (i * kb);
-      kc[kc_word_index(d, w, nw)] = word;
-    }
+  } else {
+    // Keys per token (BQ2_0), grouped like values: words [G][D*kb/32] and
+    // (scale, zero) pairs [G][D/group_v], row-major.
+    const int kw = D * kb / 32, ng = D / Gv;
+    quantize_rows(G, D, kb, Gv, kval, [&](int t, int w, uint32_t word) { kc[t * kw + w] = word; },
+                  [&](int t, int g, __half d16, __half m16) { ksz[t * ng + g] = __halves2half2(d16, m16); });
   }
 
-  // Values: one group per group_v channels of a token (KIVI: per-token
-  // values). Each thread owns one output word (32/vb channels); the P threads
-  // of a group combine their min/max with xor shuffles.
-  const int per = 32 / vb;
-  const int wpt = D / per;      // words per token
-  const int P = Gv / per;       // threads per group, a power of two <= 32
-  for (int widx = threadIdx.x; widx < G * wpt; widx += blockDim.x) {
-    const int t = widx / wpt, w = widx % wpt;
-    const uint16_t* xs = sv + t * D + w * per;
-    float mn = bits_to_float(xs[0], dt), mx = mn;
-    for (int i = 1; i < per; ++i) {
-      const float x = bits_to_float(xs[i], dt);
-      mn = fminf(mn, x);
-      mx = fmaxf(mx, x);
-    }
-    for (int o = P / 2; o >= 1; o >>= 1) {
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    }
-    const GroupParams gp = group_params(mn, mx, vb);
-    uint32_t word = 0;
-    for (int i = 0; i < per; ++i) word |= quant_code(bits_to_float(xs[i], dt), gp, vb) << (i * vb);
-    vc[vc_word_index(t, w, G, kb, wpt)] = word;
-    if ((w % P) == 0) {
-      vsz[vsz_half_index(t, w / P, G, kb, D / Gv, false)] = gp.d16;
-      vsz[vsz_half_index(t, w / P, G, kb, D / Gv, true)] = gp.m16;
-    }
-  }
+  // Values: one group per group_v channels of a token (KIVI: per-token values).
+  const int vwpt = D * vb / 32;
+  quantize_rows(G, D, vb, Gv, vval,
+                [&](int t, int w, uint32_t word) { vc[vc_word_index(t, w, G, kb, vwpt)] = word; },
+                [&](int t, int g, __half d16, __half m16) {
+                  vsz[vsz_half_index(t, g, G, kb, D / Gv, false)] = d16;
+                  vsz[vsz_half_index(t, g, G, kb, D / Gv, true)] = m16;
+                });
 }
 
 // grid (batch, Hkv); copies this call's sink tokens to the sinks and its
@@ -178,10 +242,17 @@ __global__ void dequant_kernel(LayerView L, int seq, int sinks, int t0, int n, f
       const uint8_t* rec = record_ptr(L, seq, h, tok / G);
       const int t = tok % G;
       const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + L.kc_off);
-      const __half2 ksz = reinterpret_cast<const __half2*>(rec + L.ksz_off)[d];
       const int kper = 32 / kb;
-      const uint32_t kq = (kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb)) & ((1u << kb) - 1);
-      k_out[o] = dequant_value(kq, __low2half(ksz), __high2half(ksz));
+      __half2 ksz;
+      uint32_t kw;
+      if (L.k_axis == 0) {
+        ksz = reinterpret_cast<const __half2*>(rec + L.ksz_off)[d];
+        kw = kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb);
+      } else {  // per-token keys: row-major words and (scale, zero) pairs
+        ksz = reinterpret_cast<const __half2*>(rec + L.ksz_off)[t * (D / L.group_v) + d / L.group_v];
+        kw = kc[t * (D / kper) + d / kper] >> ((d % kper) * kb);
+      }
+      k_out[o] = dequant_value(kw & ((1u << kb) - 1), __low2half(ksz), __high2half(ksz));
       const uint32_t* vc = reinterpret_cast<const uint32_t*>(rec + L.vc_off);
       const int vper = 32 / vb;
       const uint32_t vq = (vc[vc_word_index(t, d / vper, G, kb, D / vper)] >> ((d % vper) * vb)) & ((1u << vb) - 1);
@@ -199,20 +270,24 @@ __global__ void dequant_kernel(LayerView L, int seq, int sinks, int t0, int n, f
 cudaError_t launch_append(const AppendParams& p, int max_flush, cudaStream_t stream) {
   const LayerView& L = p.L;
   if (max_flush > 0) {
-    const size_t smem = (size_t)2 * L.group_k * L.head_dim * sizeof(uint16_t);
+    const bool rot = L.hadamard != 0;
+    const size_t smem = (size_t)2 * L.group_k * L.head_dim * (rot ? sizeof(float) : sizeof(uint16_t));
     // The shared-memory opt-in is per function and per device.
-    static uint64_t attr_set_mask = 0;
+    static uint64_t attr_set_mask[2] = {0, 0};
     int dev = 0;
     cudaError_t e0 = cudaGetDevice(&dev);
     if (e0 != cudaSuccess) return e0;
-    if (dev >= 64 || !(attr_set_mask & (1ull << dev))) {
-      e0 = cudaFuncSetAttribute(quantize_blocks_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                2 * 128 * kHeadDim * (int)sizeof(uint16_t));
+    if (dev >= 64 || !(attr_set_mask[rot] & (1ull << dev))) {
+      e0 = rot ? cudaFuncSetAttribute(quantize_blocks_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      2 * 128 * kHeadDim * (int)sizeof(float))
+               : cudaFuncSetAttribute(quantize_blocks_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      2 * 128 * kHeadDim * (int)sizeof(uint16_t));
       if (e0 != cudaSuccess) return e0;
-      if (dev < 64) attr_set_mask |= 1ull << dev;
+      if (dev < 64) attr_set_mask[rot] |= 1ull << dev;
     }
     dim3 grid(max_flush, p.batch, L.num_kv_heads);
-    quantize_blocks_kernel<<<grid, kQuantThreads, smem, stream>>>(p);
+    if (rot) quantize_blocks_kernel<true><<<grid, kQuantThreads, smem, stream>>>(p);
+    else quantize_blocks_kernel<false><<<grid, kQuantThreads, smem, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -69,6 +69,24 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
     sq[hh][d] = load_kv(p.q, ((int64_t)b * p.num_q_heads + h * NG + hh) * D + d, L.kv_dtype) * p.scale_log2;
   }
   __syncthreads();
+  if (L.hadamard && s > 0) {
+    // quantized tokens live in the rotated basis: score them against Hq
+    // (radix-2 butterflies, then 1/sqrt(D)); their partial is rotated back by
+    // the combine
+    for (int w = 1; w < D; w *= 2) {
+      for (int i = threadIdx.x; i < NG * (D / 2); i += blockDim.x) {
+        const int hh = i / (D / 2), pi = i % (D / 2);
+        const int c = (pi / w) * 2 * w + pi % w;
+        const float a = sq[hh][c], e = sq[hh][c + w];
+        sq[hh][c] = a + e;
+        sq[hh][c + w] = a - e;
+      }
+      __syncthreads();
+    }
+    const float rs = (float)(1.0 / sqrt((double)D));
+    for (int i = threadIdx.x; i < NG * D; i += blockDim.x) sq[i / D][i % D] *= rs;
+    __syncthreads();
+  }
 
   SoftmaxState<NG> st;
   st.init();
@@ -104,6 +122,35 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
     const int j0 = (s - 1) * bps, j1 = min(s * bps, nblk);
     for (int j = j0; j < j1; ++j) {
       const uint8_t* rec = record_ptr(L, b, h, j);
+      if (L.k_axis == 1) {
+        // per-token keys (BQ2_0): dequantize each key and dot it with q
+        const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + L.kc_off);
+        const __half2* ksz = reinterpret_cast<const __half2*>(rec + L.ksz_off);
+        const uint32_t* vc = reinterpret_cast<const uint32_t*>(rec + L.vc_off);
+        const __half* vsz = reinterpret_cast<const __half*>(rec + L.vsz_off);
+        const int ng = D / Gv;
+        for (int t = warp; t < G; t += 4) {
+          float kv[4], vv[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int d = lane + 32 * c;
+            const __half2 sz = ksz[t * ng + d / Gv];
+            const uint32_t kq = (kc[t * (D / kper) + d / kper] >> ((d % kper) * kb)) & kmask;
+            kv[c] = dequant_value(kq, __low2half(sz), __high2half(sz));
+            const uint32_t vq = (vc[vc_word_index(t, d / vper, G, kb, D / vper)] >> ((d % vper) * vb)) & vmask;
+            vv[c] = dequant_value(vq, vsz[vsz_half_index(t, d / Gv, G, kb, D / Gv, false)],
+                                  vsz[vsz_half_index(t, d / Gv, G, kb, D / Gv, true)]);
+          }
+#pragma unroll
+          for (int hh = 0; hh < NG; ++hh) {
+            float part = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) part += sq[hh][lane + 32 * c] * kv[c];
+            st.update(hh, warp_sum(part), vv);
+          }
+        }
+        continue;
+      }
       {
         const int d = threadIdx.x;
         const __half2 sz = reinterpret_cast<const __half2*>(rec + L.ksz_off)[d];
@@ -203,6 +250,8 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineParams p) {
   const float4* o_p = reinterpret_cast<const float4*>(p.ws_o + base * D) + lane;  // slot s at o_p[s * D / 4]
   float M = -INFINITY, lsum = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f);  // hadamard: the exact-token slot 0, kept apart
+  const bool rot = p.hadamard && !p.persistent;
   for (int s0 = 0; s0 < S; s0 += C) {
     float2 ml[C];
     float4 v[C];
@@ -222,19 +271,54 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineParams p) {
     acc.y *= r;
     acc.z *= r;
     acc.w *= r;
+    acc0.x *= r;
+    acc0.y *= r;
+    acc0.z *= r;
+    acc0.w *= r;
     lsum *= r;
     M = mc;
 #pragma unroll
     for (int e = 0; e < C; ++e) {
       if (ml[e].y > 0.f) {
         const float w = exp2f(ml[e].x - M);
-        acc.x += w * v[e].x;
-        acc.y += w * v[e].y;
-        acc.z += w * v[e].z;
-        acc.w += w * v[e].w;
+        float4& a = (rot && s0 + e == 0) ? acc0 : acc;
+        a.x += w * v[e].x;
+        a.y += w * v[e].y;
+        a.z += w * v[e].z;
+        a.w += w * v[e].w;
         lsum += w * ml[e].y;
       }
     }
+  }
+  if (rot) {
+    // the quantized part back to the original basis: acc . H over the warp's
+    // 128 channels (lane L holds 4L..4L+3): butterflies of half-width 1 and 2
+    // inside the lane, 4..64 across lanes, then 1/sqrt(D)
+    float x[4] = {acc.x, acc.y, acc.z, acc.w};
+    float a0 = x[0], a1 = x[1];
+    x[0] = a0 + a1;
+    x[1] = a0 - a1;
+    a0 = x[2];
+    a1 = x[3];
+    x[2] = a0 + a1;
+    x[3] = a0 - a1;
+    a0 = x[0];
+    a1 = x[1];
+    x[0] = a0 + x[2];
+    x[1] = a1 + x[3];
+    x[2] = a0 - x[2];
+    x[3] = a1 - x[3];
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const bool upper = (lane & m) != 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float y = __shfl_xor_sync(0xffffffffu, x[e], m);
+        x[e] = upper ? y - x[e] : x[e] + y;
+      }
+    }
+    const float rs = (float)(1.0 / sqrt((double)D));
+    acc = make_float4(x[0] * rs + acc0.x, x[1] * rs + acc0.y, x[2] * rs + acc0.z, x[3] * rs + acc0.w);
   }
   float r[4] = {0.f, 0.f, 0.f, 0.f};
   if (lsum > 0.f) {
@@ -298,7 +382,7 @@ cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream) {
   cfg.numAttrs = 1;
   const CombineParams cp{p.ws_o,         p.ws_ml,          p.out,           p.unit_slots,
                          p.L.lens,       p.out_dtype,      p.num_q_heads,   p.L.num_kv_heads,
-                         p.slots,        p.L.group_k,      p.blocks_per_split, p.persistent};
+                         p.slots,        p.L.group_k,      p.blocks_per_split, p.persistent, p.L.hadamard};
   return cudaLaunchKernelEx(&cfg, combine_kernel, cp);
 }
 

@@ -118,6 +118,7 @@ struct CombineParams {
   const int32_t* unit_slots;  // persistent mode: slots per unit
   const int32_t* lens;        // split mode: the layer's length table
   int32_t out_dtype, num_q_heads, num_kv_heads, slots, group_k, blocks_per_split, persistent;
+  int32_t hadamard;  // split mode: slots >= 1 (quantized tokens) hold rotated partials
 };
 
 // The log-sum-exp combine of the partial slots (after the decode kernel).

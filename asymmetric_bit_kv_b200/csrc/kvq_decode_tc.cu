@@ -37,6 +37,7 @@ const void* instance_for(const LayerView& L, int num_q_heads) {
 
 bool mma_supported(const LayerView& L) {
   if (L.head_dim != kHeadDim) return false;
+  if (L.k_axis != 0 || L.hadamard) return false;  // BQ2_0 layers run on the CUDA-core kernel
   if (L.group_k < 64) return false;                   // tiles of 64 tokens
   if (L.v_bits == 2 && L.group_v < 64) return false;  // a 2-bit value chunk spans 64 channels
   return true;

@@ -27,6 +27,8 @@ struct LayerView {
   int32_t num_kv_heads, head_dim, group_k, group_v, residual;
   int32_t kv_dtype;       // KVQ_F16 / KVQ_BF16
   int32_t sinks;          // S: sink tokens kept exact at the start of each sequence
+  int32_t k_axis;         // 0: keys per channel over G tokens (KIVI); 1: per token over group_v channels (BQ2_0)
+  int32_t hadamard;       // 1: K and V rotated by the normalized Sylvester matrix before quantization
 };
 
 __host__ __device__ inline int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
@@ -34,6 +36,8 @@ __host__ __device__ inline int64_t round_up(int64_t x, int64_t a) { return (x + 
 // Byte sizes of the four parts of a block record.
 __host__ __device__ inline int64_t kc_bytes(int G, int D, int kb) { return (int64_t)G * kb / 32 * D * 4; }
 __host__ __device__ inline int64_t ksz_bytes(int D) { return (int64_t)D * 4; }
+// Per-token keys: (scale, zero) pairs [G][D/group_v].
+__host__ __device__ inline int64_t ksz_token_bytes(int G, int D, int gv) { return (int64_t)G * (D / gv) * 4; }
 __host__ __device__ inline int64_t vc_bytes(int G, int D, int vb) { return (int64_t)G * (D * vb / 32) * 4; }
 __host__ __device__ inline int64_t vsz_bytes(int G, int D, int gv) { return (int64_t)G * (D / gv) * 4; }
 

@@ -45,6 +45,8 @@ class kvq_config(ctypes.Structure):
         ("k_bits", ctypes.POINTER(ctypes.c_int8)),
         ("v_bits", ctypes.POINTER(ctypes.c_int8)),
         ("sink_tokens", ctypes.c_int32),
+        ("k_axis", ctypes.POINTER(ctypes.c_int8)),
+        ("hadamard", ctypes.c_int32),
     ]
 
 
@@ -63,6 +65,8 @@ class kvq_layout(ctypes.Structure):
         ("v_bits", ctypes.c_int32),
         ("sink_k", ctypes.c_void_p),
         ("sink_v", ctypes.c_void_p),
+        ("k_axis", ctypes.c_int32),
+        ("hadamard", ctypes.c_int32),
     ]
 
 
@@ -145,15 +149,18 @@ class CacheConfig:
     k_bits: list
     v_bits: list
     sink_tokens: int = 0
+    k_axis: list | None = None  # per layer: 0 keys per channel (KIVI), 1 per token (BQ2_0)
+    hadamard: int = 0
 
     def to_c(self):
         kb = (ctypes.c_int8 * self.num_layers)(*self.k_bits)
         vb = (ctypes.c_int8 * self.num_layers)(*self.v_bits)
+        ka = (ctypes.c_int8 * self.num_layers)(*(self.k_axis or [0] * self.num_layers))
         c = kvq_config(self.num_layers, self.max_batch, self.num_q_heads, self.num_kv_heads, self.head_dim,
                        self.max_tokens, self.group_k, self.group_v, self.residual, _DTYPE_CODE[self.kv_dtype],
                        ctypes.cast(kb, ctypes.POINTER(ctypes.c_int8)), ctypes.cast(vb, ctypes.POINTER(ctypes.c_int8)),
-                       self.sink_tokens)
-        return c, (kb, vb)
+                       self.sink_tokens, ctypes.cast(ka, ctypes.POINTER(ctypes.c_int8)), self.hadamard)
+        return c, (kb, vb, ka)
 
 
 def required_bytes(cfg: CacheConfig) -> int:

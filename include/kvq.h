@@ -88,6 +88,14 @@ typedef struct kvq_config {
                            sequence are kept exact and never quantized
                            (KV1-1.2B card: attention sinks, 4 in KV1);
                            quantization and the ring start at token S      */
+  const int8_t* k_axis; /* host [num_layers] or null (all 0), copied: 0 keys
+                           per channel over G tokens (KIVI), 1 keys per token
+                           over group_v channels like values (KV1 BQ2_0)    */
+  int32_t hadamard;     /* 1: every K and V head vector is multiplied by the
+                           normalized Sylvester Hadamard matrix H before it
+                           is quantized, queries by H for quantized tokens
+                           and their output contribution by H again (KV1
+                           BQ2_0); sinks and ring stay exact. 0: none       */
 } kvq_config;
 
 typedef struct kvq_cache kvq_cache;
@@ -103,6 +111,9 @@ typedef struct kvq_cache kvq_cache;
  *       w packs the codes of tokens w*(32/k_bits) + i, i = 0.., code i at
  *       bits [i*k_bits, ...) (per-channel keys packed along the token axis);
  *   ksz half2 [D]: (scale d, zero point m) of each channel's key group;
+ *   (k_axis 1: kc uint32 [G][D*k_bits/32], token t's row of words, word w
+ *   packing channels w*(32/k_bits) + i; ksz half2 [G][D/group_v] per
+ *   (token, channel group); both row-major, unpermuted);
  *   vc  uint32 [G][V], V = D*v_bits/32: one row of V words per token; word w
  *       packs the codes of channels w*(32/v_bits) + i, code i at bits
  *       [i*v_bits, ...) (per-token values packed along head_dim);
@@ -131,6 +142,7 @@ typedef struct kvq_layout {
   int32_t k_bits, v_bits;
   void* sink_k;
   void* sink_v;
+  int32_t k_axis, hadamard;
 } kvq_layout;
 
 /* Device bytes the arena must hold for cfg: all layers' block records and
@@ -222,8 +234,9 @@ KVQ_API kvq_status kvq_decode_step(kvq_cache* cache, int32_t layer, const void* 
 
 /* Reconstruct tokens [t0, t1) of sequence `seq` as fp32: x_hat = q*d + m
  * (an fp32 product, then an fp32 sum; KV1 card, BQ2_0) for quantized tokens
- * and the exact stored value for sink and ring tokens (t counts every token
- * of the sequence, sinks first). k_out, v_out: device
+ * (in the rotated basis for a hadamard cache: as stored) and the exact
+ * stored value for sink and ring tokens (t counts every token of the
+ * sequence, sinks first). k_out, v_out: device
  * [t1-t0][num_kv_heads][head_dim] fp32. 0 <= t0 <= t1 <= sequence length.  */
 KVQ_API kvq_status kvq_dequant(kvq_cache* cache, int32_t layer, int32_t seq, int32_t t0, int32_t t1,
                        float* k_out, float* v_out, void* stream);

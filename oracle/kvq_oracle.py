@@ -203,8 +203,6 @@ def pack_value_block(codes: np.ndarray, bits: int) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
-# Cache state machine (KIVI README: residual window of recent fp16 tokens)
-# ---------------------------------------------------------------------------
 # Hadamard rotation ("KV1-1.2B", BQ2_0: normalized Sylvester Hadamard matrix)
 # ---------------------------------------------------------------------------
 
@@ -235,6 +233,8 @@ def rotate_fp32(x: np.ndarray) -> np.ndarray:
     return (y * F32(1.0 / np.sqrt(D))).astype(F32)
 
 
+# ---------------------------------------------------------------------------
+# Cache state machine (KIVI README: residual window of recent fp16 tokens)
 # ---------------------------------------------------------------------------
 
 

@@ -86,7 +86,9 @@ class Twin:
             for b in self.oracle_seqs:
                 self.ora[(layer, b)] = O.SequenceCache(cfg.num_kv_heads, cfg.head_dim, cfg.k_bits[layer],
                                                        cfg.v_bits[layer], cfg.group_k, cfg.group_v, cfg.residual,
-                                                       sinks=cfg.sink_tokens)
+                                                       sinks=cfg.sink_tokens,
+                                                       k_axis=(cfg.k_axis or [0] * cfg.num_layers)[layer],
+                                                       hadamard=bool(cfg.hadamard))
 
     def append(self, layer: int, k: torch.Tensor, v: torch.Tensor, new_lens):
         """k, v: [sum(new_lens), Hkv, D] in the cache dtype (any device)."""
@@ -128,11 +130,22 @@ class Twin:
 
         kcw = G * kb // 32
         vcw = D * vb // 32
-        kc = part(lay.kc_offset, kcw * D * 4, np.uint32, (D * kcw,))
-        vc = part(lay.vc_offset, G * vcw * 4, np.uint32, (G * vcw,))
-        kidx = np.array([[kc_word_index(d, w, kcw) for w in range(kcw)] for d in range(D)])
-        vidx = np.array([[vc_word_index(t, w, G, kb, vcw) for w in range(vcw)] for t in range(G)])
         ng = D // Gv
+        vc = part(lay.vc_offset, G * vcw * 4, np.uint32, (G * vcw,))
+        vidx = np.array([[vc_word_index(t, w, G, kb, vcw) for w in range(vcw)] for t in range(G)])
+        if lay.k_axis == 1:  # per-token keys: row-major words and (scale, zero) pairs
+            kw = D * kb // 32
+            vsz = part(lay.vsz_offset, G * ng * 4, np.float16, (G * ng * 2,))
+            sidx = np.array([[[vsz_half_index(t, gg, G, kb, ng, z) for z in (False, True)] for gg in range(ng)]
+                             for t in range(G)])
+            return {
+                "kc": part(lay.kc_offset, G * kw * 4, np.uint32, (G, kw)),
+                "ksz": part(lay.ksz_offset, G * ng * 4, np.float16, (G, ng, 2)),
+                "vc": vc[:, vidx],
+                "vsz": vsz[:, sidx],
+            }
+        kc = part(lay.kc_offset, kcw * D * 4, np.uint32, (D * kcw,))
+        kidx = np.array([[kc_word_index(d, w, kcw) for w in range(kcw)] for d in range(D)])
         vsz = part(lay.vsz_offset, G * ng * 4, np.float16, (G * ng * 2,))
         sidx = np.array([[[vsz_half_index(t, gg, G, kb, ng, z) for z in (False, True)] for gg in range(ng)]
                          for t in range(G)])
@@ -175,10 +188,16 @@ class Twin:
             if nblk:
                 rec = self.read_records(layer, b, h, nblk)
                 for j, blk in enumerate(o.blocks):
-                    kw = O.pack_key_block(blk.kc, kb)[h]
-                    assert np.array_equal(rec["kc"][j], kw), (layer, b, h, j, "key codes")
-                    assert np.array_equal(rec["ksz"][j][:, 0].view(np.uint16), blk.kd[h].view(np.uint16)), (b, h, j, "key scale")
-                    assert np.array_equal(rec["ksz"][j][:, 1].view(np.uint16), blk.km[h].view(np.uint16)), (b, h, j, "key zero")
+                    if o.k_axis == 1:
+                        kw = O.pack_value_block(blk.kc, kb)[h]
+                        assert np.array_equal(rec["kc"][j], kw), (layer, b, h, j, "per-token key codes")
+                        assert np.array_equal(rec["ksz"][j][..., 0].view(np.uint16), blk.kd[:, h].view(np.uint16)), (b, h, j, "key scale")
+                        assert np.array_equal(rec["ksz"][j][..., 1].view(np.uint16), blk.km[:, h].view(np.uint16)), (b, h, j, "key zero")
+                    else:
+                        kw = O.pack_key_block(blk.kc, kb)[h]
+                        assert np.array_equal(rec["kc"][j], kw), (layer, b, h, j, "key codes")
+                        assert np.array_equal(rec["ksz"][j][:, 0].view(np.uint16), blk.kd[h].view(np.uint16)), (b, h, j, "key scale")
+                        assert np.array_equal(rec["ksz"][j][:, 1].view(np.uint16), blk.km[h].view(np.uint16)), (b, h, j, "key zero")
                     vw = O.pack_value_block(blk.vc, vb)[h]
                     assert np.array_equal(rec["vc"][j], vw), (layer, b, h, j, "value codes")
                     assert np.array_equal(rec["vsz"][j][..., 0].view(np.uint16), blk.vd[:, h].view(np.uint16)), (b, h, j, "value scale")
