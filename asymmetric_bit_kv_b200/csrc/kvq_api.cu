@@ -326,6 +326,7 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const 
   const bool use_mma = kvq::mma_supported(L);
   kvq::MmaPlan mp{};
   int per_sm = 4;
+  if (!use_mma) per_sm = kvq::split_ctas_per_sm(cfg.num_q_heads, cfg.num_kv_heads);
   if (use_mma) {
     mp = kvq::make_mma_plan(L, cfg.num_q_heads);
     per_sm = kvq::mma_ctas_per_sm(L, mp, cfg.num_q_heads);

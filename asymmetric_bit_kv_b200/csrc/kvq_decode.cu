@@ -42,6 +42,40 @@ struct SoftmaxState {
   }
 };
 
+// Value of token t of a block record at this lane's channels lane + 32c,
+// dequantized (x_hat = q*d + m, two roundings): the record's word placement
+// and its (scale, zero) order are resolved once per token, not per channel.
+__device__ __forceinline__ void token_values(const LayerView& L, const uint8_t* rec, int t, int lane,
+                                             float (&vv)[4]) {
+  constexpr int D = kHeadDim;
+  const int G = L.group_k, kb = L.k_bits, vb = L.v_bits, Gv = L.group_v;
+  const int vper = 32 / vb, VW = D / vper, ng = D / Gv;
+  const uint32_t* vc = reinterpret_cast<const uint32_t*>(rec + L.vc_off);
+  const __half* vsz = reinterpret_cast<const __half*>(rec + L.vsz_off);
+  const int row = vc_row(t, G, kb);
+  const int sw = VW >= 4 ? chunk_swizzle(row, VW / 4) : 0;
+  // (scale, zero) of group gg at vsz[zi(gg)] / vsz[zi(gg) + zoff]
+  int zbase, zstride, zoff;
+  if (G < 64) {
+    zbase = t * ng * 2;
+    zstride = 2;
+    zoff = 1;
+  } else {
+    const int i0 = vsz_half_index(t, 0, G, kb, ng, false);
+    zstride = ng > 1 ? vsz_half_index(t, 1, G, kb, ng, false) - i0 : 0;
+    zbase = i0;
+    zoff = 4;
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int d = lane + 32 * c, w = d / vper, gg = d / Gv;
+    const int wi = VW < 4 ? row * VW + w : row * VW + (((w >> 2) ^ sw) << 2) + (w & 3);
+    const uint32_t vq = (vc[wi] >> ((d % vper) * vb)) & ((1u << vb) - 1);
+    const int zi = zbase + gg * zstride;
+    vv[c] = dequant_value(vq, vsz[zi], vsz[zi + zoff]);
+  }
+}
+
 // One CTA = one split of one (sequence, KV head); 4 warps, each warp walks a
 // quarter of the split's tokens with its own online-softmax state; lane owns
 // channels lane + 32c, c = 0..3.
@@ -116,9 +150,9 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
       }
     }
   } else {
-    const int kb = L.k_bits, vb = L.v_bits, Gv = L.group_v;
-    const int kper = 32 / kb, vper = 32 / vb;
-    const uint32_t kmask = (1u << kb) - 1, vmask = (1u << vb) - 1;
+    const int kb = L.k_bits, Gv = L.group_v;
+    const int kper = 32 / kb;
+    const uint32_t kmask = (1u << kb) - 1;
     const int j0 = (s - 1) * bps, j1 = min(s * bps, nblk);
     for (int j = j0; j < j1; ++j) {
       const uint8_t* rec = record_ptr(L, b, h, j);
@@ -126,9 +160,8 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
         // per-token keys (BQ2_0): dequantize each key and dot it with q
         const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + L.kc_off);
         const __half2* ksz = reinterpret_cast<const __half2*>(rec + L.ksz_off);
-        const uint32_t* vc = reinterpret_cast<const uint32_t*>(rec + L.vc_off);
-        const __half* vsz = reinterpret_cast<const __half*>(rec + L.vsz_off);
         const int ng = D / Gv;
+#pragma unroll 2
         for (int t = warp; t < G; t += 4) {
           float kv[4], vv[4];
 #pragma unroll
@@ -137,10 +170,8 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
             const __half2 sz = ksz[t * ng + d / Gv];
             const uint32_t kq = (kc[t * (D / kper) + d / kper] >> ((d % kper) * kb)) & kmask;
             kv[c] = dequant_value(kq, __low2half(sz), __high2half(sz));
-            const uint32_t vq = (vc[vc_word_index(t, d / vper, G, kb, D / vper)] >> ((d % vper) * vb)) & vmask;
-            vv[c] = dequant_value(vq, vsz[vsz_half_index(t, d / Gv, G, kb, D / Gv, false)],
-                                  vsz[vsz_half_index(t, d / Gv, G, kb, D / Gv, true)]);
           }
+          token_values(L, rec, t, lane, vv);
 #pragma unroll
           for (int hh = 0; hh < NG; ++hh) {
             float part = 0.f;
@@ -167,19 +198,15 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
 #pragma unroll
       for (int hh = 0; hh < NG; ++hh) bias[hh] = sbias[0][hh] + sbias[1][hh] + sbias[2][hh] + sbias[3][hh];
       const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + L.kc_off);
-      const uint32_t* vc = reinterpret_cast<const uint32_t*>(rec + L.vc_off);
-      const __half* vsz = reinterpret_cast<const __half*>(rec + L.vsz_off);
       for (int t = warp; t < G; t += 4) {
         float kcode[4], vv[4];
+        const int kw = t / kper, ksh = (t % kper) * kb;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int d = lane + 32 * c;
-          kcode[c] = (float)((kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb)) & kmask);
-          const uint32_t vq = (vc[vc_word_index(t, d / vper, G, kb, D / vper)] >> ((d % vper) * vb)) & vmask;
-          const float vs = __half2float(vsz[vsz_half_index(t, d / Gv, G, kb, D / Gv, false)]);
-          const float vz = __half2float(vsz[vsz_half_index(t, d / Gv, G, kb, D / Gv, true)]);
-          vv[c] = (float)vq * vs + vz;
+          kcode[c] = (float)((kc[kc_word_index(d, kw, G / kper)] >> ksh) & kmask);
         }
+        token_values(L, rec, t, lane, vv);
 #pragma unroll
         for (int hh = 0; hh < NG; ++hh) {
           float part = 0.f;
@@ -349,6 +376,23 @@ cudaError_t launch_simple(const DecodeParams& p, int max_splits, cudaStream_t st
 }
 
 }  // namespace
+
+int split_ctas_per_sm(int num_q_heads, int num_kv_heads) {
+  const int g = num_q_heads / num_kv_heads;
+  const void* fn = g == 1   ? reinterpret_cast<const void*>(decode_split_simple_kernel<1>)
+                   : g == 2 ? reinterpret_cast<const void*>(decode_split_simple_kernel<2>)
+                   : g == 4 ? reinterpret_cast<const void*>(decode_split_simple_kernel<4>)
+                            : reinterpret_cast<const void*>(decode_split_simple_kernel<8>);
+  static int memo[9] = {0};  // per head ratio (one device type per process)
+  if (memo[g] > 0) return memo[g];
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, 128, 0) != cudaSuccess || n < 1) {
+    (void)cudaGetLastError();
+    return 4;
+  }
+  memo[g] = n;
+  return n;
+}
 
 cudaError_t launch_decode(const DecodeParams& p, int max_splits, cudaStream_t stream) {
   if (p.batch <= 0) return cudaSuccess;

@@ -109,6 +109,8 @@ cudaError_t launch_decode_mma(const DecodeParams& p, const MmaPlan& mp, cudaStre
 // log-sum-exp combine. max_splits is the largest quantized split count of any
 // sequence (from the host mirror).
 cudaError_t launch_decode(const DecodeParams& p, int max_splits, cudaStream_t stream);
+// Resident CTAs per SM of the CUDA-core split kernel for this head ratio.
+int split_ctas_per_sm(int num_q_heads, int num_kv_heads);
 
 // Parameters of the log-sum-exp combine (small: no per-sequence tables).
 struct CombineParams {

@@ -70,6 +70,15 @@ def llama3_8b_gqa() -> Workload:
                     torch.bfloat16, "lognormal", 1.0, seed=2)
 
 
+def kv1_bq2_gqa() -> Workload:
+    """The Llama-3-8B-shaped GQA layer with the KV1 card's BQ2_0 cache: keys
+    and values 2-bit per token over one whole head vector (group 128), the
+    Hadamard rotation, 4 sink tokens; G64 blocks, R128."""
+    return Workload("kv1_bq2_gqa_k2v2_tok_gv128_rot_s4_r128_b32_ctx8192", 32, 32, 8, 128, [8192] * 32, [2], [2], 64,
+                    128, 128, torch.bfloat16, "lognormal", 1.0, seed=2,
+                    extra={"k_axis": [1], "hadamard": 1, "sinks": 4})
+
+
 def long_context_gqa() -> Workload:
     """Long-context GQA decode: 1 x (32 q / 8 kv) x 128, context 131072, bf16
     distributed as the Llama-2 layer; K2 V2, G128, R128; plus a 4096-token
@@ -93,7 +102,7 @@ def qwen3_8b_layers(seed: int = 4) -> Workload:
 
 
 ALL = {"tiny": tiny_mha, "llama2": llama2_7b_mha, "llama3": llama3_8b_gqa, "long": long_context_gqa,
-       "qwen3": qwen3_8b_layers}
+       "qwen3": qwen3_8b_layers, "kv1": kv1_bq2_gqa}
 
 
 def key_channel_scale(wl: Workload, layer: int, gen: torch.Generator) -> torch.Tensor:

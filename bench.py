@@ -47,7 +47,20 @@ def _args():
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--replicas", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="llama3", choices=["llama3", "kv1"],
+                    help="llama3: the headline KIVI layer (default); kv1: the same shapes with the KV1 card's BQ2_0 cache")
     return ap.parse_args()
+
+
+def _bench_workload(name):
+    from asymmetric_bit_kv_b200 import workloads as W
+
+    return W.llama3_8b_gqa() if name == "llama3" else W.kv1_bq2_gqa()
+
+
+def _layout(wl):
+    """(sinks, k_axis, hadamard) of a workload's cache."""
+    return wl.extra.get("sinks", 0), wl.extra.get("k_axis", [0])[0], wl.extra.get("hadamard", 0)
 
 
 def _dist_env():
@@ -137,7 +150,7 @@ class ClockSampler:
 # CPU oracle baseline (host cores, spawned worker processes)
 # --------------------------------------------------------------------------
 
-def _oracle_worker(conn, unit, ctx):
+def _oracle_worker(conn, unit, ctx, wname="llama3"):
     """One unit of the workload -- one (sequence, KV head) with its 4 query
     heads -- held in the oracle. Prefill is untimed; each 'step' command appends
     one token and runs decode attention, and replies with the tokens attended."""
@@ -147,7 +160,8 @@ def _oracle_worker(conn, unit, ctx):
     from oracle import kvq_oracle as O
 
     with threadpool_limits(1):
-        wl = W.llama3_8b_gqa()
+        wl = _bench_workload(wname)
+        sinks, k_axis, rot = _layout(wl)
         g = wl.num_q_heads // wl.num_kv_heads
         unit_wl = W.Workload(wl.name, 1, g, 1, wl.head_dim, [ctx], wl.k_bits, wl.v_bits, wl.group_k, wl.group_v,
                              wl.residual, wl.kv_dtype, wl.key_dist, wl.value_std, wl.seed)
@@ -155,7 +169,8 @@ def _oracle_worker(conn, unit, ctx):
         k, v = W.generate_tokens(unit_wl, 0, [ctx + extra], seed_offset=7000 + unit)
         k = k.float().numpy()
         v = v.float().numpy()
-        c = O.SequenceCache(1, wl.head_dim, wl.k_bits[0], wl.v_bits[0], wl.group_k, wl.group_v, wl.residual)
+        c = O.SequenceCache(1, wl.head_dim, wl.k_bits[0], wl.v_bits[0], wl.group_k, wl.group_v, wl.residual,
+                            sinks=sinks, k_axis=k_axis, hadamard=bool(rot))
         c.append(k[:ctx], v[:ctx])
         conn.send("ready")
         i = 0
@@ -175,14 +190,14 @@ def _oracle_worker(conn, unit, ctx):
 class OracleRunner:
     """`workers` spawned processes, one workload unit each, stepped together."""
 
-    def __init__(self, workers: int, ctx: int = 8192):
+    def __init__(self, workers: int, ctx: int = 8192, wname: str = "llama3"):
         import multiprocessing as mp
 
         ctxm = mp.get_context("spawn")
         self.conns, self.procs = [], []
         for u in range(workers):
             a, b = ctxm.Pipe()
-            p = ctxm.Process(target=_oracle_worker, args=(b, u, ctx), daemon=True)
+            p = ctxm.Process(target=_oracle_worker, args=(b, u, ctx, wname), daemon=True)
             p.start()
             self.conns.append(a)
             self.procs.append(p)
@@ -215,9 +230,9 @@ class OracleRunner:
                 f"{steps} timed steps; KV tokens counted as unit tokens / 8 KV heads")
 
 
-def cpu_oracle_baseline(steps: int = 100, warmup: int = 2):
+def cpu_oracle_baseline(steps: int = 100, warmup: int = 2, wname: str = "llama3"):
     workers = max(1, min(os.cpu_count() or 1, 16))
-    run = OracleRunner(workers)
+    run = OracleRunner(workers, wname=wname)
     try:
         for _ in range(warmup):
             run.step()
@@ -242,6 +257,7 @@ def _workload_config(wl, replicas, world, mean_ctx=None):
         "batch": wl.batch, "num_q_heads": wl.num_q_heads, "num_kv_heads": wl.num_kv_heads,
         "head_dim": wl.head_dim, "context": wl.context[0], "k_bits": wl.k_bits[0], "v_bits": wl.v_bits[0],
         "group_k": wl.group_k, "group_v": wl.group_v, "residual": wl.residual,
+        "sinks": _layout(wl)[0], "key_axis": "token" if _layout(wl)[1] else "channel", "hadamard": _layout(wl)[2],
         "kv_dtype": "bf16", "out_dtype": "bf16",
         "replicas": replicas,
         "l2": "inputs larger than L2: each step reads a different replica's ~248 MB cache",
@@ -265,13 +281,16 @@ def run_kvq(a):
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    wl = W.llama3_8b_gqa()
+    wl = _bench_workload(a.workload)
+    sinks, k_axis, rot = _layout(wl)
+    fused = k_axis == 0 and not rot  # tensor-core layers take the new token inside the decode launch
     B, Hq, Hkv, D = wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim
     ctx = wl.context[0]
     R = a.replicas
     steps_per_rep = math.ceil((a.warmup + 2 * a.steps) / R) + 2
     cap = ctx + steps_per_rep + wl.group_k
-    cfg = CacheConfig(1, B, Hq, Hkv, D, cap, wl.group_k, wl.group_v, wl.residual, wl.kv_dtype, wl.k_bits, wl.v_bits)
+    cfg = CacheConfig(1, B, Hq, Hkv, D, cap, wl.group_k, wl.group_v, wl.residual, wl.kv_dtype, wl.k_bits, wl.v_bits,
+                      sink_tokens=sinks, k_axis=[k_axis], hadamard=rot)
     caches = []
     for r in range(R):
         c = KVCache(cfg, dev)
@@ -289,7 +308,7 @@ def run_kvq(a):
     stream = torch.cuda.current_stream()
     # per-step inputs as views made once, so that the timed loop only enqueues
     views = [(new_k[j], new_v[j], qs[j]) for j in range(pool)]
-    bytes_tok = O.quantized_bytes_per_token(Hkv, D, wl.k_bits[0], wl.v_bits[0], wl.group_k, wl.group_v)
+    bytes_tok = O.quantized_bytes_per_token(Hkv, D, wl.k_bits[0], wl.v_bits[0], wl.group_k, wl.group_v, k_axis)
 
     G, Rw = wl.group_k, wl.residual
 
@@ -331,9 +350,13 @@ def run_kvq(a):
     for i in range(a.steps):
         r = (a.warmup + i) % R
         # fused: decode + combine; a step that flushes a ring first runs the
-        # quantize and ring-write kernels
-        launches = 2 + (2 if lens[r][0][1] == Rw else 0)
+        # quantize and ring-write kernels (unfused: ring write, split kernel,
+        # combine, and the quantize kernel on a flush)
+        flush = lens[r][0][1] == Rw
+        launches = (2 + (2 if flush else 0)) if fused else (3 + (1 if flush else 0))
         ab, tk = 2 * B * Hq * D * 2 + 2 * (2 * B * Hkv * D * 2), 0  # q in, out; new k, v in and into the ring
+        ab += B * sinks * Hkv * D * 2 * 2  # the exact sink tokens
+        tk += B * sinks
         for b in range(B):
             qn, n = lens[r][b]
             if n == Rw:
@@ -394,7 +417,7 @@ def run_kvq(a):
             if n == Rw:
                 qn, n = qn + G, n - G
             lens[r][b] = [qn, n + 1]
-            tok_e2e += qn + n + 1
+            tok_e2e += sinks + qn + n + 1
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -417,7 +440,7 @@ def run_kvq(a):
     result = None
     if rank == 0:
         peak, peak_kind = _peaks()
-        traffic = _committed_traffic()
+        traffic = _committed_traffic() if a.workload == "llama3" else None
         result = {
             "metric": METRIC,
             "value": value,
@@ -433,7 +456,10 @@ def run_kvq(a):
             "data": "synthetic (seeded; Llama-3-8B-shaped layer, no model weights)",
             "config": _workload_config(wl, R, world, tok_total / (a.steps * B)),
             "roofline": {
-                "kernel": "decode step: one token appended per sequence inside the split-KV decode kernel, + log-sum-exp combine, per call (a ring flush adds the quantize and ring kernels)",
+                "kernel": ("decode step: one token appended per sequence inside the split-KV decode kernel, + log-sum-exp "
+                           "combine, per call (a ring flush adds the quantize and ring kernels)") if fused else
+                          ("decode step: ring write, CUDA-core split-KV decode kernel and log-sum-exp combine, per call "
+                           "(a ring flush adds the quantize kernel)"),
                 "bound": "hbm",
                 "achieved": achieved_gbs,
                 "peak": peak,
@@ -492,12 +518,11 @@ def run_reference(a):
     rank, world, _ = _dist_env()
     if rank != 0:
         return None
-    from asymmetric_bit_kv_b200 import workloads as W
-
-    wl = W.llama3_8b_gqa()
+    wname = getattr(a, "workload", "llama3")
+    wl = _bench_workload(wname)
     workers = max(1, min(os.cpu_count() or 1, 16))
     t_start = time.perf_counter()
-    run = OracleRunner(workers, wl.context[0])
+    run = OracleRunner(workers, wl.context[0], wname)
     try:
         for _ in range(a.warmup):
             run.step()
@@ -542,7 +567,7 @@ def main():
     rank, world, _ = _dist_env()
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        cpu = cpu_oracle_baseline()   # spawned before any CUDA work in this process
+        cpu = cpu_oracle_baseline(wname=a.workload)   # spawned before any CUDA work in this process
     res = run_kvq(a)
     if res is not None:
         res["cpu_baseline"] = cpu
