@@ -323,7 +323,7 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const 
   const kvq_config& cfg = c->cfg;
   const int G = cfg.group_k;
   const kvq::LayerView L = layer_view(c, layer);
-  const bool use_mma = kvq::mma_supported(L);
+  const bool use_mma = kvq::mma_supported(L, cfg.num_q_heads);
   kvq::MmaPlan mp{};
   int per_sm = 4;
   if (!use_mma) per_sm = kvq::split_ctas_per_sm(cfg.num_q_heads, cfg.num_kv_heads);
@@ -612,7 +612,7 @@ kvq_status kvq_decode_step(kvq_cache* c, int32_t layer, const void* k, const voi
   // The new tokens ride along with the decode when every one of them lands in
   // a ring slot without a flush (ring not full, sinks complete) and the layer
   // runs on the tensor-core kernel; otherwise append, then decode.
-  bool fused = kvq::mma_supported(layer_view(c, layer));
+  bool fused = kvq::mma_supported(layer_view(c, layer), c->cfg.num_q_heads);
   for (int b = 0; b < batch; ++b) {
     const int64_t L = (int64_t)c->s_len[base + b] + c->q_len[base + b] + c->n_len[base + b] + 1;
     if (L > cfg.max_tokens)

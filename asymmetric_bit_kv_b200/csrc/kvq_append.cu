@@ -161,11 +161,30 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_blocks_kernel(AppendPa
       }
     }
   } else {
-    // Keys per token (BQ2_0), grouped like values: words [G][D*kb/32] and
-    // (scale, zero) pairs [G][D/group_v], row-major.
-    const int kw = D * kb / 32, ng = D / Gv;
-    quantize_rows(G, D, kb, Gv, kval, [&](int t, int w, uint32_t word) { kc[t * kw + w] = word; },
+    // Keys per token (BQ2_0), grouped like values over group_v channels:
+    // (scale, zero) pairs [G][D/group_v] row-major, then the codes packed
+    // along the token axis in the per-channel key layout, so that the decode
+    // kernels read both key axes' codes the same way.
+    const int ng = D / Gv;
+    quantize_rows(G, D, kb, Gv, kval, [](int, int, uint32_t) {},
                   [&](int t, int g, __half d16, __half m16) { ksz[t * ng + g] = __halves2half2(d16, m16); });
+    __syncthreads();  // the pairs just stored are read back below
+    const int per = 32 / kb, nw = G / per;
+    for (int idx = threadIdx.x; idx < D * nw; idx += blockDim.x) {
+      const int d = idx / nw, w = idx % nw;
+      uint32_t word = 0;
+      for (int i = 0; i < per; ++i) {
+        const int t = w * per + i;
+        const __half2 sz = ksz[t * ng + d / Gv];
+        GroupParams gp;
+        gp.d16 = __low2half(sz);
+        gp.m16 = __high2half(sz);
+        gp.d = __half2float(gp.d16);
+        gp.m = __half2float(gp.m16);
+        word |= quant_code(kval(t, d), gp, kb) << (i * kb);
+      }
+      kc[kc_word_index(d, w, nw)] = word;
+    }
   }
 
   // Values: one group per group_v channels of a token (KIVI: per-token values).
@@ -248,9 +267,9 @@ __global__ void dequant_kernel(LayerView L, int seq, int sinks, int t0, int n, f
       if (L.k_axis == 0) {
         ksz = reinterpret_cast<const __half2*>(rec + L.ksz_off)[d];
         kw = kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb);
-      } else {  // per-token keys: row-major words and (scale, zero) pairs
+      } else {  // per-token keys: (scale, zero) per (token, channel group), codes as above
         ksz = reinterpret_cast<const __half2*>(rec + L.ksz_off)[t * (D / L.group_v) + d / L.group_v];
-        kw = kc[t * (D / kper) + d / kper] >> ((d % kper) * kb);
+        kw = kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb);
       }
       k_out[o] = dequant_value(kw & ((1u << kb) - 1), __low2half(ksz), __high2half(ksz));
       const uint32_t* vc = reinterpret_cast<const uint32_t*>(rec + L.vc_off);

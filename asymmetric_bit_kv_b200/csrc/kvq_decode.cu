@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
           for (int c = 0; c < 4; ++c) {
             const int d = lane + 32 * c;
             const __half2 sz = ksz[t * ng + d / Gv];
-            const uint32_t kq = (kc[t * (D / kper) + d / kper] >> ((d % kper) * kb)) & kmask;
+            const uint32_t kq = (kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb)) & kmask;
             kv[c] = dequant_value(kq, __low2half(sz), __high2half(sz));
           }
           token_values(L, rec, t, lane, vv);

@@ -100,7 +100,7 @@ struct MmaPlan {
   int32_t smem_bytes;   // dynamic shared memory per CTA
 };
 
-bool mma_supported(const LayerView& L);
+bool mma_supported(const LayerView& L, int num_q_heads);
 MmaPlan make_mma_plan(const LayerView& L, int num_q_heads);
 int mma_ctas_per_sm(const LayerView& L, const MmaPlan& mp, int num_q_heads);
 cudaError_t launch_decode_mma(const DecodeParams& p, const MmaPlan& mp, cudaStream_t stream);

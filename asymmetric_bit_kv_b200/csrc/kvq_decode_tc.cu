@@ -9,8 +9,9 @@
 namespace kvq {
 namespace tc {
 #define KVQ_TC_DECL(K, N)                                                                                   \
-  cudaError_t launch_tc_k##K##_##N(int vb, int ngrp, const DecodeParams& p, const MmaPlan& mp, cudaStream_t s); \
-  const void* fn_tc_k##K##_##N(int vb, int ngrp);
+  cudaError_t launch_tc_k##K##_##N(int vb, int ngrp, bool pt, const DecodeParams& p, const MmaPlan& mp,           \
+                                   cudaStream_t s);                                                              \
+  const void* fn_tc_k##K##_##N(int vb, int ngrp, bool pt);
 KVQ_TC_DECL(2, 1)
 KVQ_TC_DECL(2, 2)
 KVQ_TC_DECL(4, 1)
@@ -27,7 +28,7 @@ int key_ntiles(const LayerView& L, int num_q_heads) { return num_q_heads / L.num
 const void* instance_for(const LayerView& L, int num_q_heads) {
   const int vb = L.v_bits, ng = kHeadDim / L.group_v, nkt = key_ntiles(L, num_q_heads);
 #define KVQ_TC_PICK(K, N) \
-  if (L.k_bits == K && nkt == N) return tc::fn_tc_k##K##_##N(vb, ng);
+  if (L.k_bits == K && nkt == N) return tc::fn_tc_k##K##_##N(vb, ng, L.k_axis == 1);
   KVQ_TC_PICK(2, 1) KVQ_TC_PICK(2, 2) KVQ_TC_PICK(4, 1) KVQ_TC_PICK(4, 2) KVQ_TC_PICK(8, 1) KVQ_TC_PICK(8, 2)
 #undef KVQ_TC_PICK
   return nullptr;
@@ -35,12 +36,37 @@ const void* instance_for(const LayerView& L, int num_q_heads) {
 
 }  // namespace
 
-bool mma_supported(const LayerView& L) {
+// Largest dynamic shared memory a CTA of the current device may opt in to,
+// less 1 KB for the kernel's static shared memory; 0 if unknown.
+int smem_limit() {
+  static int memo[64];  // per device, +1 (0: not queried yet)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  if (dev < 64 && memo[dev] > 0) return memo[dev] - 1;
+  int optin = 0;
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  const int lim = std::max(0, optin - 1024);
+  if (dev < 64) memo[dev] = lim + 1;
+  return lim;
+}
+
+bool mma_supported(const LayerView& L, int num_q_heads) {
   if (L.head_dim != kHeadDim) return false;
-  if (L.k_axis != 0 || L.hadamard) return false;  // BQ2_0 layers run on the CUDA-core kernel
+  // per-token keys with one group per head vector (BQ2_0), with or without
+  // the rotation; the rotation with per-channel keys runs on the CUDA-core
+  // kernel
+  if (L.k_axis == 1 && L.group_v != kHeadDim) return false;
+  if (L.hadamard && L.k_axis != 1) return false;
   if (L.group_k < 64) return false;                   // tiles of 64 tokens
   if (L.v_bits == 2 && L.group_v < 64) return false;  // a 2-bit value chunk spans 64 channels
-  return true;
+  // two stages per warp must fit (8-bit keys in blocks of 128 tokens do not)
+  return make_mma_plan(L, num_q_heads).smem_bytes <= smem_limit();
 }
 
 MmaPlan make_mma_plan(const LayerView& L, int num_q_heads) {
@@ -125,7 +151,7 @@ cudaError_t launch_decode_mma(const DecodeParams& p, const MmaPlan& mp, cudaStre
   const LayerView& L = p.L;
   const int vb = L.v_bits, ng = kHeadDim / L.group_v, nkt = key_ntiles(L, p.num_q_heads);
 #define KVQ_TC_GO(K, N) \
-  if (L.k_bits == K && nkt == N) return tc::launch_tc_k##K##_##N(vb, ng, p, mp, stream);
+  if (L.k_bits == K && nkt == N) return tc::launch_tc_k##K##_##N(vb, ng, L.k_axis == 1, p, mp, stream);
   KVQ_TC_GO(2, 1) KVQ_TC_GO(2, 2) KVQ_TC_GO(4, 1) KVQ_TC_GO(4, 2) KVQ_TC_GO(8, 1) KVQ_TC_GO(8, 2)
 #undef KVQ_TC_GO
   return cudaErrorInvalidValue;

@@ -547,6 +547,139 @@ __device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t*
   }
 }
 
+// ------------------------------------------- per-token keys and the rotation
+// Keys quantized per token over whole head vectors ("KV1-1.2B" card, BQ2_0)
+// keep the per-channel code layout, so the A operand is built the same way;
+// only the scales move: S[t][h] = d_t * (codes . q')[t][h] + m_t * sum(q'_h).
+// The B operand is then the unit's query itself (fp16 high and low parts,
+// the same columns as q*s), built once per unit instead of once per block,
+// and d_t, m_t scale the rows of the fp32 scores. With the rotation, q' = H q
+// for the quantized tokens; their part of O is in the rotated basis and is
+// multiplied by H again (H . H = I) before any exact-token chunk adds to O,
+// and before the partial is written.
+
+// x . H for the 128 channels of one head spread over a warp, channels 4l..4l+3
+// in lane l: radix-2 butterflies of half-width 1, 2, 4, ..., 64 (the first two
+// inside the lane, the others with the lane at xor distance w/4), then one
+// fp32 multiplication by fp32(1/sqrt(128)) -- the order in which the quantizer
+// rotates the keys and values.
+__device__ __forceinline__ void rotate_lane(float (&x)[4], int lane) {
+  float a = x[0], c = x[1];
+  x[0] = __fadd_rn(a, c);
+  x[1] = __fsub_rn(a, c);
+  a = x[2], c = x[3];
+  x[2] = __fadd_rn(a, c);
+  x[3] = __fsub_rn(a, c);
+  a = x[0], c = x[2];
+  x[0] = __fadd_rn(a, c);
+  x[2] = __fsub_rn(a, c);
+  a = x[1], c = x[3];
+  x[1] = __fadd_rn(a, c);
+  x[3] = __fsub_rn(a, c);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const bool upper = lane & o;  // this lane holds the x[i + w] side of its pairs
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float other = __shfl_xor_sync(0xffffffffu, x[e], o);
+      x[e] = upper ? __fsub_rn(other, x[e]) : __fadd_rn(x[e], other);
+    }
+  }
+  const float s = (float)(1.0 / sqrt((double)kHeadDim));
+#pragma unroll
+  for (int e = 0; e < 4; ++e) x[e] = __fmul_rn(x[e], s);
+}
+
+// Per-token keys: the key B fragments (same columns as prep_block's, every
+// column written, absent heads zero) and bias[h] = sum_d q'_hd * score_scale
+// of the unit's query q' (rotated when rot), from qw (fp16 x q_prescale).
+template <int NKT>
+__device__ __forceinline__ void unit_query(const uint32_t* qw, uint8_t* ws, const MmaPlan& mp, int NG, int lane,
+                                           float score_scale, bool rot) {
+  uint32_t* bk = reinterpret_cast<uint32_t*>(ws + mp.bfrag_off);
+  float* biasw = reinterpret_cast<float*>(ws + mp.bias_off);
+#pragma unroll 1
+  for (int hh = 0; hh < 4 * NKT; ++hh) {
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    if (hh < NG) {
+      const float2 a = unpack_f16(qw[q_word(hh, 2 * lane)]), c = unpack_f16(qw[q_word(hh, 2 * lane + 1)]);
+      x[0] = a.x, x[1] = a.y, x[2] = c.x, x[3] = c.y;
+      if (rot) rotate_lane(x, lane);
+    }
+    float sum = (x[0] + x[1]) + (x[2] + x[3]);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int w = 2 * lane + e;  // channels 2w, 2w+1
+      const uint32_t hi = pack_f16(x[2 * e], x[2 * e + 1]);
+      const float2 fh = unpack_f16(hi);
+      const uint32_t lo = pack_f16(x[2 * e] - fh.x, x[2 * e + 1] - fh.y);
+      const int kk = w >> 3, q = w & 7, half = q >> 2, tq = q & 3;
+      if (NKT == 1) {
+        bk[(kk * 32 + (2 * hh) * 4 + tq) * 2 + half] = hi;
+        bk[(kk * 32 + (2 * hh + 1) * 4 + tq) * 2 + half] = lo;
+      } else {
+        bk[(kk * 32 + hh * 4 + tq) * 2 + half] = hi;
+        bk[((8 + kk) * 32 + hh * 4 + tq) * 2 + half] = lo;
+      }
+    }
+    if (lane == 0) biasw[hh] = sum * score_scale;
+  }
+  __syncwarp();
+}
+
+// O (with its zero-point terms Z folded in) times H over the channels, in
+// place: each lane's outputs of heads 2t, 2t+1 go to scr [NG][128] fp32 (the
+// warp's key B-fragment area, which the caller rebuilds afterwards), every
+// head is rotated by the warp, and O is read back at its rows' code scale
+// (2^(p-24), exact), Z cleared.
+template <int VB, int NGRP>
+__device__ __forceinline__ void unrotate_output(float (&O)[8][4], float (&Z)[NGRP][4], float* scr, int NG, int lane,
+                                                bool v0, bool v1) {
+  using S = Shape<2, VB, NGRP, 1>;  // value-side constants only
+  const int g = lane >> 2, t = lane & 3;
+  __syncwarp();  // every lane is done with the B fragments
+#pragma unroll
+  for (int mt2 = 0; mt2 < 8; ++mt2) {
+    const int cch = mt2 / S::MT_PER_CH, P = mt2 % S::MT_PER_CH;
+    const int gg = (cch * S::CH_SPAN) / S::GV;
+    const int ch0 = cch * S::CH_SPAN + g * S::VCPC + 2 * P;
+    const float u0 = code_unscale<VB>(2 * P), u1 = code_unscale<VB>(2 * P + 1);
+    if (v0) {
+      scr[(2 * t) * kHeadDim + ch0] = fmaf(O[mt2][0], u0, Z[gg][0]);
+      scr[(2 * t) * kHeadDim + ch0 + 1] = fmaf(O[mt2][2], u1, Z[gg][2]);
+    }
+    if (v1) {
+      scr[(2 * t + 1) * kHeadDim + ch0] = fmaf(O[mt2][1], u0, Z[gg][1]);
+      scr[(2 * t + 1) * kHeadDim + ch0 + 1] = fmaf(O[mt2][3], u1, Z[gg][3]);
+    }
+  }
+  __syncwarp();
+#pragma unroll 1
+  for (int h = 0; h < NG; ++h) {
+    float4* row = reinterpret_cast<float4*>(scr + h * kHeadDim);
+    const float4 v = row[lane];
+    float x[4] = {v.x, v.y, v.z, v.w};
+    rotate_lane(x, lane);
+    row[lane] = make_float4(x[0], x[1], x[2], x[3]);
+  }
+  __syncwarp();
+#pragma unroll
+  for (int mt2 = 0; mt2 < 8; ++mt2) {
+    const int cch = mt2 / S::MT_PER_CH, P = mt2 % S::MT_PER_CH;
+    const int ch0 = cch * S::CH_SPAN + g * S::VCPC + 2 * P;
+    const float r0 = pow2f(code_pos<VB>(2 * P) - 24), r1 = pow2f(code_pos<VB>(2 * P + 1) - 24);
+    O[mt2][0] = v0 ? scr[(2 * t) * kHeadDim + ch0] * r0 : 0.f;
+    O[mt2][2] = v0 ? scr[(2 * t) * kHeadDim + ch0 + 1] * r1 : 0.f;
+    O[mt2][1] = v1 ? scr[(2 * t + 1) * kHeadDim + ch0] * r0 : 0.f;
+    O[mt2][3] = v1 ? scr[(2 * t + 1) * kHeadDim + ch0 + 1] * r1 : 0.f;
+  }
+#pragma unroll
+  for (int gg = 0; gg < NGRP; ++gg) Z[gg][0] = Z[gg][1] = Z[gg][2] = Z[gg][3] = 0.f;
+  __syncwarp();
+}
+
 // Exact-token chunk r of a unit (the items after its quantized blocks): ring
 // chunk r while r < ceil(nres / kResChunk), then the sink chunk if the
 // sequence has sinks; an empty sequence's one item is a ring chunk with no
@@ -658,7 +791,9 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, const MmaPlan&
              bar);
 }
 
-template <int KB, int VB, int NGRP, int NKT>
+// PT: keys per token over whole head vectors, with the rotation when the
+// layer has it (see unit_query); otherwise per-channel keys.
+template <int KB, int VB, int NGRP, int NKT, bool PT>
 __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, MmaPlan mp) {
   using S = Shape<KB, VB, NGRP, NKT>;
   constexpr int D = S::D;
@@ -738,6 +873,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
 #pragma unroll
       for (int gg = 0; gg < NGRP; ++gg) Z[gg][0] = Z[gg][1] = Z[gg][2] = Z[gg][3] = 0.f;
       bool rq_ready = false;  // the key B fragments hold the ring-chunk query (not a block's q*s)
+      bool uq_ready = false;  // PT: they hold the unit's query for its quantized blocks
+      bool rotated = false;   // PT with the rotation: O holds rotated-basis terms
       // this warp's items of the unit: k' - rs = warp (mod kNC)
       const int first = k + ((warp - (k - rs)) % kNC + kNC) % kNC;
       for (int kb = first; kb < hi; kb += kNC, ++n) {
@@ -775,7 +912,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
         const int j = kb - u.start;
         if (j < nb) {
           // ============ quantized block
-          prep_block<NKT>(stage, mp, ws, qw, NG, lane, p.score_scale);
+          if constexpr (PT) {
+            if (!uq_ready) {
+              unit_query<NKT>(qw, ws, mp, NG, lane, p.score_scale, L.hadamard != 0);
+              uq_ready = true;
+              rq_ready = false;
+            }
+            rotated = L.hadamard != 0;
+          } else {
+            prep_block<NKT>(stage, mp, ws, qw, NG, lane, p.score_scale);
+          }
           float bias[HPL];
 #pragma unroll
           for (int h = 0; h < HPL; ++h) bias[h] = biasr[HPL == 2 ? 2 * t + h : t];
@@ -823,8 +969,20 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
 #pragma unroll
               for (int r = 0; r < 2; ++r) {
                 const float rs = p.score_scale * code_unscale<KB>(2 * (mt % S::JP) + r);
+                if constexpr (PT) {
+                  // (scale, zero point) of the row's token
+                  const __half2 sz = reinterpret_cast<const __half2*>(stage + mp.kc_bytes)[tile * S::TT +
+                                                                                         tile_token<KB>(mt, g + 8 * r)];
+                  const float2 dz = __half22float2(sz);
+                  const float rst = rs * dz.x;
 #pragma unroll
-                for (int h = 0; h < HPL; ++h) sc[mt][r * HPL + h] = fmaf(head_score<NKT>(Dk[mt], r, h), rs, bias[h]);
+                  for (int h = 0; h < HPL; ++h)
+                    sc[mt][r * HPL + h] = fmaf(head_score<NKT>(Dk[mt], r, h), rst, dz.y * bias[h]);
+                } else {
+#pragma unroll
+                  for (int h = 0; h < HPL; ++h)
+                    sc[mt][r * HPL + h] = fmaf(head_score<NKT>(Dk[mt], r, h), rs, bias[h]);
+                }
               }
             softmax_update<S::MT, HPL, NGRP, false>(sc, sst, valid, O, Z, lane);
             // ---- values: O += codes x (p * s), Z += ones x (p * z)
@@ -838,12 +996,25 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
                 prob_operand<HPL>(0u, 0u, pack_f16(sc[mt][0], sc[mt][1]), lane, bt, bb);
               const int kst = tile * S::MT + mt;
               uint32_t B0[NGRP], B1[NGRP];
+              uint32_t R0[PT ? NGRP : 1], R1[PT ? NGRP : 1];
 #pragma unroll
               for (int gg = 0; gg < NGRP; ++gg) {
                 const uint4 v4 = vsz4[(kst * 4 + t) * NGRP + gg];  // (s, s), (s, s), (z, z), (z, z) of rows 2t.. 9+2t
                 B0[gg] = hmul2(bt, v4.x);
                 B1[gg] = hmul2(bb, v4.y);
-                mma_f16(Z[gg], ones, hmul2(bt, v4.z), hmul2(bb, v4.w));
+                if constexpr (PT) {
+                  // whole-vector value groups have scales and zero points
+                  // that are large next to the values they encode: p*s and
+                  // p*z also keep their fp16 remainders (exact), one more
+                  // MMA each
+                  R0[gg] = hfms2(bt, v4.x, B0[gg]);
+                  R1[gg] = hfms2(bb, v4.y, B1[gg]);
+                  const uint32_t z0 = hmul2(bt, v4.z), z1 = hmul2(bb, v4.w);
+                  mma_f16(Z[gg], ones, z0, z1);
+                  mma_f16(Z[gg], ones, hfms2(bt, v4.z, z0), hfms2(bb, v4.w, z1));
+                } else {
+                  mma_f16(Z[gg], ones, hmul2(bt, v4.z), hmul2(bb, v4.w));
+                }
               }
               const int sg = mt / S::JP, jp = mt % S::JP;
               const int vrow_idx = (2 * jp + (mi & 1)) * (G / S::CPT16) + tile * (S::TT / S::CPT16) + sg * 8 + rr;
@@ -861,12 +1032,21 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
                     const uint32_t a[4] = {code_sub<VB>(xv, xv8, 2 * P), code_sub<VB>(xv, xv8, 2 * P + 1),
                                            code_sub<VB>(yv, yv8, 2 * P), code_sub<VB>(yv, yv8, 2 * P + 1)};
                     mma_f16(O[(cc0 + cc) * S::MT_PER_CH + P], a, B0[gg], B1[gg]);
+                    if constexpr (PT) mma_f16(O[(cc0 + cc) * S::MT_PER_CH + P], a, R0[gg], R1[gg]);
                   }
                 }
               }
             }
           }
         } else {
+          if constexpr (PT) {
+            if (rotated) {  // exact tokens add in the original basis
+              unrotate_output<VB, NGRP>(O, Z, reinterpret_cast<float*>(ws + mp.bfrag_off), NG, lane, v0, v1);
+              rotated = false;
+              rq_ready = false;
+            }
+            uq_ready = false;  // ring_chunk writes its own query over the B fragments
+          }
           bool sink;
           const int cnt = exact_chunk(p, u.b, j - nb, sink);
           if (p.new_k && !sink && j - nb == (p.nres[u.b] - 1) / kResChunk) store_new_token(p, u.b, u.h, nb, stage, lane);
@@ -883,6 +1063,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
         }
       }
       if (failed) break;
+      if constexpr (PT)
+        if (rotated) unrotate_output<VB, NGRP>(O, Z, reinterpret_cast<float*>(ws + mp.bfrag_off), NG, lane, v0, v1);
       // ---------------- this warp's partial for the unit
 #pragma unroll
       for (int off = 4; off <= 16; off <<= 1)
@@ -930,15 +1112,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
 
 // Enqueues one instance. Its dynamic shared-memory size was opted in on this
 // device by mma_ctas_per_sm, which the host calls before every launch.
-template <int KB, int VB, int NGRP, int NKT>
+template <int KB, int VB, int NGRP, int NKT, bool PT>
 cudaError_t launch_instance(const DecodeParams& p, const MmaPlan& mp, cudaStream_t stream) {
-  decode_tc_kernel<KB, VB, NGRP, NKT><<<p.num_ctas, kThreads, mp.smem_bytes, stream>>>(p, mp);
+  decode_tc_kernel<KB, VB, NGRP, NKT, PT><<<p.num_ctas, kThreads, mp.smem_bytes, stream>>>(p, mp);
   return cudaGetLastError();
 }
 
-template <int KB, int VB, int NGRP, int NKT>
+template <int KB, int VB, int NGRP, int NKT, bool PT>
 const void* instance_fn() {
-  return reinterpret_cast<const void*>(decode_tc_kernel<KB, VB, NGRP, NKT>);
+  return reinterpret_cast<const void*>(decode_tc_kernel<KB, VB, NGRP, NKT, PT>);
 }
 
 }  // namespace tc

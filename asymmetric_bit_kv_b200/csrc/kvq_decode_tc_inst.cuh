@@ -12,21 +12,31 @@
 namespace kvq {
 namespace tc {
 
-// (value bits, value groups per head) pairs with a value chunk inside one group
+// (value bits, value groups per head) pairs with a value chunk inside one
+// group; per-token keys (pt) take one group per head vector
 #define KVQ_TC_VB_NG(X) X(2, 1) X(2, 2) X(4, 1) X(4, 2) X(4, 4) X(8, 1) X(8, 2) X(8, 4)
+#define KVQ_TC_VB_PT(X) X(2, 1) X(4, 1) X(8, 1)
 
-cudaError_t KVQ_TC_LAUNCH(int vb, int ngrp, const DecodeParams& p, const MmaPlan& mp, cudaStream_t stream) {
+cudaError_t KVQ_TC_LAUNCH(int vb, int ngrp, bool pt, const DecodeParams& p, const MmaPlan& mp, cudaStream_t stream) {
 #define KVQ_TC_CASE(V, N) \
-  if (vb == V && ngrp == N) return launch_instance<KVQ_TC_KB, V, N, KVQ_TC_NKT>(p, mp, stream);
+  if (!pt && vb == V && ngrp == N) return launch_instance<KVQ_TC_KB, V, N, KVQ_TC_NKT, false>(p, mp, stream);
   KVQ_TC_VB_NG(KVQ_TC_CASE)
+#undef KVQ_TC_CASE
+#define KVQ_TC_CASE(V, N) \
+  if (pt && vb == V && ngrp == N) return launch_instance<KVQ_TC_KB, V, N, KVQ_TC_NKT, true>(p, mp, stream);
+  KVQ_TC_VB_PT(KVQ_TC_CASE)
 #undef KVQ_TC_CASE
   return cudaErrorInvalidValue;
 }
 
-const void* KVQ_TC_FN(int vb, int ngrp) {
+const void* KVQ_TC_FN(int vb, int ngrp, bool pt) {
 #define KVQ_TC_CASE(V, N) \
-  if (vb == V && ngrp == N) return instance_fn<KVQ_TC_KB, V, N, KVQ_TC_NKT>();
+  if (!pt && vb == V && ngrp == N) return instance_fn<KVQ_TC_KB, V, N, KVQ_TC_NKT, false>();
   KVQ_TC_VB_NG(KVQ_TC_CASE)
+#undef KVQ_TC_CASE
+#define KVQ_TC_CASE(V, N) \
+  if (pt && vb == V && ngrp == N) return instance_fn<KVQ_TC_KB, V, N, KVQ_TC_NKT, true>();
+  KVQ_TC_VB_PT(KVQ_TC_CASE)
 #undef KVQ_TC_CASE
   return nullptr;
 }

@@ -111,9 +111,9 @@ typedef struct kvq_cache kvq_cache;
  *       w packs the codes of tokens w*(32/k_bits) + i, i = 0.., code i at
  *       bits [i*k_bits, ...) (per-channel keys packed along the token axis);
  *   ksz half2 [D]: (scale d, zero point m) of each channel's key group;
- *   (k_axis 1: kc uint32 [G][D*k_bits/32], token t's row of words, word w
- *   packing channels w*(32/k_bits) + i; ksz half2 [G][D/group_v] per
- *   (token, channel group); both row-major, unpermuted);
+ *   (k_axis 1: kc exactly as above, codes of each channel packed along the
+ *   token axis; ksz half2 [G][D/group_v], (scale, zero point) per (token,
+ *   channel group), row-major);
  *   vc  uint32 [G][V], V = D*v_bits/32: one row of V words per token; word w
  *       packs the codes of channels w*(32/v_bits) + i, code i at bits
  *       [i*v_bits, ...) (per-token values packed along head_dim);

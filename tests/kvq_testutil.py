@@ -133,25 +133,19 @@ class Twin:
         ng = D // Gv
         vc = part(lay.vc_offset, G * vcw * 4, np.uint32, (G * vcw,))
         vidx = np.array([[vc_word_index(t, w, G, kb, vcw) for w in range(vcw)] for t in range(G)])
-        if lay.k_axis == 1:  # per-token keys: row-major words and (scale, zero) pairs
-            kw = D * kb // 32
-            vsz = part(lay.vsz_offset, G * ng * 4, np.float16, (G * ng * 2,))
-            sidx = np.array([[[vsz_half_index(t, gg, G, kb, ng, z) for z in (False, True)] for gg in range(ng)]
-                             for t in range(G)])
-            return {
-                "kc": part(lay.kc_offset, G * kw * 4, np.uint32, (G, kw)),
-                "ksz": part(lay.ksz_offset, G * ng * 4, np.float16, (G, ng, 2)),
-                "vc": vc[:, vidx],
-                "vsz": vsz[:, sidx],
-            }
+        # key codes: channel rows of words along the token axis, for both key axes
         kc = part(lay.kc_offset, kcw * D * 4, np.uint32, (D * kcw,))
         kidx = np.array([[kc_word_index(d, w, kcw) for w in range(kcw)] for d in range(D)])
         vsz = part(lay.vsz_offset, G * ng * 4, np.float16, (G * ng * 2,))
         sidx = np.array([[[vsz_half_index(t, gg, G, kb, ng, z) for z in (False, True)] for gg in range(ng)]
                          for t in range(G)])
+        if lay.k_axis == 1:  # per-token keys: (scale, zero) pairs [G][groups], row-major
+            ksz = part(lay.ksz_offset, G * ng * 4, np.float16, (G, ng, 2))
+        else:
+            ksz = part(lay.ksz_offset, D * 4, np.float16, (D, 2))
         return {
             "kc": kc[:, kidx],
-            "ksz": part(lay.ksz_offset, D * 4, np.float16, (D, 2)),
+            "ksz": ksz,
             "vc": vc[:, vidx],
             "vsz": vsz[:, sidx],
         }
@@ -189,7 +183,7 @@ class Twin:
                 rec = self.read_records(layer, b, h, nblk)
                 for j, blk in enumerate(o.blocks):
                     if o.k_axis == 1:
-                        kw = O.pack_value_block(blk.kc, kb)[h]
+                        kw = O.pack_key_block(blk.kc, kb)[h]
                         assert np.array_equal(rec["kc"][j], kw), (layer, b, h, j, "per-token key codes")
                         assert np.array_equal(rec["ksz"][j][..., 0].view(np.uint16), blk.kd[:, h].view(np.uint16)), (b, h, j, "key scale")
                         assert np.array_equal(rec["ksz"][j][..., 1].view(np.uint16), blk.km[:, h].view(np.uint16)), (b, h, j, "key zero")

@@ -6,8 +6,10 @@ BQ2_0), with and without sinks.
 Codes, scales, zero points and dequantized values (in the rotated basis, as
 stored) must match the oracle bit for bit -- the rotation is the same fp32
 butterfly on both sides; attention within the usual tolerance (max-abs 2e-3,
-max-rel 1e-2 against max(|ref|, 0.2)). These layers decode on the CUDA-core
-split kernel; the combine rotates the quantized part back.
+max-rel 1e-2 against max(|ref|, 0.2)). Layers with one key group per head
+vector (group_v = head_dim, group_k >= 64) decode on the tensor-core kernel,
+which multiplies the quantized tokens' part of the output by H itself; the
+others on the CUDA-core split kernel, whose combine rotates that part back.
 """
 
 import numpy as np
@@ -21,12 +23,17 @@ pytestmark = pytest.mark.gpu
 
 # (k bits, v bits, group_k, group_v, residual, dtype, hadamard, sinks)
 CASES = [
-    (2, 2, 64, 128, 128, torch.bfloat16, 1, 4),   # KV1-like: 2-bit, one group per head vector, rotation, 4 sinks
-    (2, 4, 32, 64, 64, torch.float16, 0, 0),      # per-token keys, no rotation
-    (4, 2, 64, 32, 64, torch.bfloat16, 1, 0),     # rotation, 4 value groups
-    (8, 8, 128, 64, 128, torch.bfloat16, 1, 2),
+    (2, 2, 64, 128, 128, torch.bfloat16, 1, 4),   # KV1-like: 2-bit, one group per head vector, rotation, 4 sinks (TC)
+    (2, 4, 32, 64, 64, torch.float16, 0, 0),      # per-token keys, no rotation (split)
+    (4, 2, 64, 32, 64, torch.bfloat16, 1, 0),     # rotation, 4 value groups (split)
+    (8, 8, 128, 64, 128, torch.bfloat16, 1, 2),   # (split)
+    (4, 4, 64, 128, 64, torch.float16, 1, 0),     # rotation, f16 (TC)
+    (8, 2, 64, 128, 128, torch.bfloat16, 0, 2),   # per-token keys without rotation, 2 sinks (TC)
+    (8, 4, 128, 128, 128, torch.bfloat16, 1, 0),  # two stages of 8-bit 128-token blocks do not fit: split
+    (4, 2, 128, 128, 128, torch.float16, 1, 3),   # 128-token blocks (TC)
 ]
-IDS = ["kv1_k2v2_gv128_rot_s4", "k2v4_g32_norot", "k4v2_gv32_rot", "k8v8_g128_rot_s2"]
+IDS = ["kv1_k2v2_gv128_rot_s4", "k2v4_g32_norot", "k4v2_gv32_rot", "k8v8_g128_rot_s2", "tc_k4v4_rot_f16",
+       "tc_k8v2_norot_s2", "k8v4_g128_rot", "tc_k4v2_g128_rot_s3"]
 
 
 def _cfg(case, batch=4, hq=8, hkv=2, layers=1):
@@ -63,7 +70,7 @@ def test_bq2_codes_and_dequant_bit_exact(case):
         tw.check_dequant(0, b)
 
 
-@pytest.mark.parametrize("g", [1, 4])
+@pytest.mark.parametrize("g", [1, 4, 8])
 @pytest.mark.parametrize("case", CASES, ids=IDS)
 def test_bq2_decode_matches_oracle(case, g):
     G, R = case[2], case[4]
@@ -86,8 +93,8 @@ def test_bq2_decode_matches_oracle(case, g):
 
 
 def test_bq2_next_to_kivi_layers_and_decode_steps():
-    # layer 0 KIVI (per-channel keys, tensor-core kernel, fused steps),
-    # layer 1 BQ2_0 with rotation (split kernel, append-then-decode steps)
+    # a rotated cache with group_v 64: layer 0 per-channel keys, layer 1
+    # per-token keys, both on the split kernel (append-then-decode steps)
     cfg = CacheConfig(2, 3, 8, 2, 128, 2048, 64, 64, 128, torch.bfloat16, [2, 2], [4, 2], k_axis=[0, 1], hadamard=1)
     tw = Twin(cfg)
     gen = torch.Generator().manual_seed(7)
@@ -112,3 +119,37 @@ def test_bq2_next_to_kivi_layers_and_decode_steps():
         tw.check_lengths(layer, 3)
         for b in range(3):
             tw.check_codes(layer, b)
+
+
+def test_bq2_whole_vector_layers_take_the_fused_step():
+    # the KV1 layout (2-bit per-token keys and values over whole head vectors,
+    # rotation, 4 sinks) on the tensor-core kernel: fused decode steps between
+    # flushes, append-then-decode steps at them; 8 and 4 query heads per KV head
+    for hq in (16, 8):
+        cfg = CacheConfig(2, 3, hq, 2, 128, 2048, 64, 128, 128, torch.bfloat16, [2, 2], [2, 4], sink_tokens=4,
+                          k_axis=[1, 1], hadamard=1)
+        tw = Twin(cfg)
+        gen = torch.Generator().manual_seed(17 + hq)
+        lens = [300, 2, 191]
+        scale = 128 ** -0.5
+        for layer in (0, 1):
+            k, v = _tokens(sum(lens), 2, cfg.kv_dtype, gen)
+            tw.append(layer, k, v, lens)
+        for step in range(80):
+            for layer in (0, 1):
+                k, v = _tokens(3, 2, cfg.kv_dtype, gen)
+                q = torch.randn(3, hq, 128, generator=gen).to(cfg.kv_dtype)
+                out = tw.gpu.decode_step(layer, k.cuda(), v.cuda(), q.cuda(), out_dtype=torch.float32,
+                                         softmax_scale=scale)
+                for b in range(3):
+                    tw.ora[(layer, b)].append(k[b:b + 1].float().numpy(), v[b:b + 1].float().numpy())
+                if step % 13 == 0 or step == 79:
+                    o = out.cpu().numpy()
+                    for b in range(3):
+                        assert_attention_close(o[b], tw.oracle_decode(layer, b, q[b].float().numpy(), scale),
+                                               f"hq {hq} layer {layer} step {step} seq {b}")
+        assert tw.gpu.device_errors() == 0
+        for layer in (0, 1):
+            tw.check_lengths(layer, 3)
+            for b in range(3):
+                tw.check_codes(layer, b)
