@@ -53,10 +53,10 @@ __device__ __forceinline__ void quantize_rows(int rows, int D, int bits, int gv,
 }
 
 // grid (max flush blocks, batch, Hkv); block kQuantThreads; dynamic smem
-// 2*G*D*2 bytes (ROT: 2*G*D*4). ROT: the G x D block of keys and of values is
-// staged as fp32 and every token's head vector is multiplied by the
-// normalized Sylvester Hadamard matrix (radix-2 butterflies of half-width 1,
-// 2, 4, ..., then one fp32 multiplication by fp32(1/sqrt(D))) before it is
+// 2*G*D*2 bytes (ROT: 2*G*D*4). ROT: every token's key and value head vector
+// is multiplied by the normalized Sylvester Hadamard matrix (rotate_lane:
+// radix-2 butterflies of half-width 1, 2, 4, ..., then one fp32
+// multiplication by fp32(1/sqrt(D))) and staged as fp32 before the block is
 // quantized ("KV1-1.2B" card, BQ2_0).
 template <bool ROT>
 __global__ void __launch_bounds__(kQuantThreads) quantize_blocks_kernel(AppendParams p) {
@@ -75,57 +75,38 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_blocks_kernel(AppendPa
   const int first = p.q_old[b] + j * G;  // position of the block's first token (after the sinks)
   const int boundary = p.q_old[b] + p.n_old[b];
   const int64_t ring_base = ((int64_t)b * L.num_kv_heads + h) * R;
-  // Stage the G x D block, 8 values (16 bytes) per load.
-  const int vec_per_tok = D / 8;
-  for (int idx = threadIdx.x; idx < G * vec_per_tok; idx += blockDim.x) {
-    const int t = idx / vec_per_tok, c = (idx % vec_per_tok) * 8;
+  // Row t of the block (token first + t) of the keys or the values: in the
+  // ring, or in this call's input.
+  auto row_ptr = [&](int t, bool value) -> const uint16_t* {
     const int i = first + t;
-    const uint4* ksrc;
-    const uint4* vsrc;
-    if (i < boundary) {
-      const int64_t off = (ring_base + i % R) * D + c;
-      ksrc = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(L.ring_k) + off);
-      vsrc = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(L.ring_v) + off);
-    } else {
-      const int64_t row = (int64_t)p.in_off[b] + (i - boundary);
-      const int64_t off = (row * L.num_kv_heads + h) * D + c;
-      ksrc = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.k_in) + off);
-      vsrc = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.v_in) + off);
+    if (i < boundary)
+      return reinterpret_cast<const uint16_t*>(value ? L.ring_v : L.ring_k) + (ring_base + i % R) * D;
+    const int64_t row = (int64_t)p.in_off[b] + (i - boundary);
+    return reinterpret_cast<const uint16_t*>(value ? p.v_in : p.k_in) + (row * L.num_kv_heads + h) * D;
+  };
+  if constexpr (ROT) {
+    // one warp per row of G keys then G values, 4 channels per lane, rotated
+    // in registers (D = 128)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int row = warp; row < 2 * G; row += kQuantThreads / 32) {
+      const bool value = row >= G;
+      const int t = value ? row - G : row;
+      const uint2 raw = *reinterpret_cast<const uint2*>(row_ptr(t, value) + 4 * lane);
+      float x[4] = {bits_to_float(raw.x & 0xffffu, dt), bits_to_float(raw.x >> 16, dt),
+                    bits_to_float(raw.y & 0xffffu, dt), bits_to_float(raw.y >> 16, dt)};
+      rotate_lane(x, lane);
+      *reinterpret_cast<float4*>((value ? fv : fk) + t * D + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
     }
-    const uint4 kx = *ksrc, vx = *vsrc;
-    if constexpr (ROT) {
-      const uint16_t* k16 = reinterpret_cast<const uint16_t*>(&kx);
-      const uint16_t* v16 = reinterpret_cast<const uint16_t*>(&vx);
-      for (int e = 0; e < 8; ++e) {
-        fk[t * D + c + e] = bits_to_float(k16[e], dt);
-        fv[t * D + c + e] = bits_to_float(v16[e], dt);
-      }
-    } else {
-      *reinterpret_cast<uint4*>(sk + t * D + c) = kx;
-      *reinterpret_cast<uint4*>(sv + t * D + c) = vx;
+  } else {
+    // Stage the G x D block, 8 values (16 bytes) per load.
+    const int vec_per_tok = D / 8;
+    for (int idx = threadIdx.x; idx < G * vec_per_tok; idx += blockDim.x) {
+      const int t = idx / vec_per_tok, c = (idx % vec_per_tok) * 8;
+      *reinterpret_cast<uint4*>(sk + t * D + c) = *reinterpret_cast<const uint4*>(row_ptr(t, false) + c);
+      *reinterpret_cast<uint4*>(sv + t * D + c) = *reinterpret_cast<const uint4*>(row_ptr(t, true) + c);
     }
   }
   __syncthreads();
-  if constexpr (ROT) {
-    for (int w = 1; w < D; w *= 2) {
-      for (int idx = threadIdx.x; idx < 2 * G * (D / 2); idx += blockDim.x) {
-        float* x = (idx < G * (D / 2) ? fk : fv);
-        const int r = idx % (G * (D / 2));
-        const int t = r / (D / 2), pi = r % (D / 2);
-        const int i = t * D + (pi / w) * 2 * w + pi % w;  // bit w of the channel clear
-        const float a = x[i], c = x[i + w];
-        x[i] = __fadd_rn(a, c);
-        x[i + w] = __fsub_rn(a, c);
-      }
-      __syncthreads();
-    }
-    const float s = (float)(1.0 / sqrt((double)D));
-    for (int idx = threadIdx.x; idx < 2 * G * D; idx += blockDim.x) {
-      float* x = idx < G * D ? fk : fv;
-      x[idx % (G * D)] = __fmul_rn(x[idx % (G * D)], s);
-    }
-    __syncthreads();
-  }
   auto kval = [&](int t, int d) -> float {
     if constexpr (ROT) return fk[t * D + d];
     else return bits_to_float(sk[t * D + d], dt);
@@ -165,9 +146,11 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_blocks_kernel(AppendPa
     // (scale, zero) pairs [G][D/group_v] row-major, then the codes packed
     // along the token axis in the per-channel key layout, so that the decode
     // kernels read both key axes' codes the same way.
+    __shared__ __half2 s_ksz[128 * 4];  // G <= 128 tokens x D/group_v <= 4 groups
     const int ng = D / Gv;
-    quantize_rows(G, D, kb, Gv, kval, [](int, int, uint32_t) {},
-                  [&](int t, int g, __half d16, __half m16) { ksz[t * ng + g] = __halves2half2(d16, m16); });
+    quantize_rows(G, D, kb, Gv, kval, [](int, int, uint32_t) {}, [&](int t, int g, __half d16, __half m16) {
+      ksz[t * ng + g] = s_ksz[t * ng + g] = __halves2half2(d16, m16);
+    });
     __syncthreads();  // the pairs just stored are read back below
     const int per = 32 / kb, nw = G / per;
     for (int idx = threadIdx.x; idx < D * nw; idx += blockDim.x) {
@@ -175,7 +158,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_blocks_kernel(AppendPa
       uint32_t word = 0;
       for (int i = 0; i < per; ++i) {
         const int t = w * per + i;
-        const __half2 sz = ksz[t * ng + d / Gv];
+        const __half2 sz = s_ksz[t * ng + d / Gv];
         GroupParams gp;
         gp.d16 = __low2half(sz);
         gp.m16 = __high2half(sz);

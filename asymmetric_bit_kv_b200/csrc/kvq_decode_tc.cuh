@@ -441,6 +441,32 @@ __device__ __forceinline__ void prob_operand(uint32_t row_g, uint32_t row_g8, ui
   }
 }
 
+// prob_operand with one head per lane where the B columns 4-7 repeat columns
+// 0-3 (at most 4 heads per KV head leave them free): lane (g, t) takes the
+// tokens of head g & 3, so that columns 4-7 can carry the remainders of
+// columns 0-3.
+__device__ __forceinline__ void prob_operand_dup(uint32_t packed, int lane, uint32_t& bt, uint32_t& bb) {
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t u = __shfl_sync(0xffffffffu, packed, 8 * t + (g & 3));
+  const uint32_t v = __shfl_sync(0xffffffffu, packed, 8 * t + 4 + (g & 3));
+  bt = __byte_perm(u, v, 0x5410);
+  bb = __byte_perm(u, v, 0x7632);
+}
+
+// Adds O and Z columns 4-7 into columns 0-3 (lane t += lane t ^ 2): the
+// remainder columns of prob_operand_dup, folded into their heads.
+template <int NGRP>
+__device__ __forceinline__ void fold_remainders(float (&O)[8][4], float (&Z)[NGRP][4]) {
+#pragma unroll
+  for (int i2 = 0; i2 < 8; ++i2)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) O[i2][e] += __shfl_xor_sync(0xffffffffu, O[i2][e], 2);
+#pragma unroll
+  for (int gg = 0; gg < NGRP; ++gg)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) Z[gg][e] += __shfl_xor_sync(0xffffffffu, Z[gg][e], 2);
+}
+
 // One chunk of ring tokens (cnt of its kResChunk rows present, cnt <= 0
 // for the placeholder chunk of an empty sequence): stage = key rows
 // [kResChunk][D] then value rows, in the kv dtype; accumulated into the
@@ -528,6 +554,7 @@ __device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t*
     const uint32_t hl = pack_kv<BF16>(sc[0][0], sc[0][0] - hf);  // (high, low) of row g
     prob_operand<HPL>(0u, 0u, hl, lane, bh, dummy);              // bh = high parts of tokens 2t, 2t+1
     bl = dummy;                                                  // bb = low parts
+    if (g >= 4) bh = bl = 0u;  // columns 4-7 hold no head here (see prob_operand_dup)
   }
   const uint32_t* V32 = reinterpret_cast<const uint32_t*>(stage + kResChunk * kRowBytes);  // [rows][64 words]
 #pragma unroll
@@ -557,38 +584,6 @@ __device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t*
 // for the quantized tokens; their part of O is in the rotated basis and is
 // multiplied by H again (H . H = I) before any exact-token chunk adds to O,
 // and before the partial is written.
-
-// x . H for the 128 channels of one head spread over a warp, channels 4l..4l+3
-// in lane l: radix-2 butterflies of half-width 1, 2, 4, ..., 64 (the first two
-// inside the lane, the others with the lane at xor distance w/4), then one
-// fp32 multiplication by fp32(1/sqrt(128)) -- the order in which the quantizer
-// rotates the keys and values.
-__device__ __forceinline__ void rotate_lane(float (&x)[4], int lane) {
-  float a = x[0], c = x[1];
-  x[0] = __fadd_rn(a, c);
-  x[1] = __fsub_rn(a, c);
-  a = x[2], c = x[3];
-  x[2] = __fadd_rn(a, c);
-  x[3] = __fsub_rn(a, c);
-  a = x[0], c = x[2];
-  x[0] = __fadd_rn(a, c);
-  x[2] = __fsub_rn(a, c);
-  a = x[1], c = x[3];
-  x[1] = __fadd_rn(a, c);
-  x[3] = __fsub_rn(a, c);
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const bool upper = lane & o;  // this lane holds the x[i + w] side of its pairs
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float other = __shfl_xor_sync(0xffffffffu, x[e], o);
-      x[e] = upper ? __fsub_rn(other, x[e]) : __fadd_rn(x[e], other);
-    }
-  }
-  const float s = (float)(1.0 / sqrt((double)kHeadDim));
-#pragma unroll
-  for (int e = 0; e < 4; ++e) x[e] = __fmul_rn(x[e], s);
-}
 
 // Per-token keys: the key B fragments (same columns as prep_block's, every
 // column written, absent heads zero) and bias[h] = sum_d q'_hd * score_scale
@@ -629,16 +624,18 @@ __device__ __forceinline__ void unit_query(const uint32_t* qw, uint8_t* ws, cons
   __syncwarp();
 }
 
-// O (with its zero-point terms Z folded in) times H over the channels, in
-// place: each lane's outputs of heads 2t, 2t+1 go to scr [NG][128] fp32 (the
+// O (with its zero-point terms Z folded in; FOLD: and its remainder columns)
+// times H over the channels, in place: each lane's outputs of heads 2t, 2t+1
+// go to scr [NG][128] fp32 (the
 // warp's key B-fragment area, which the caller rebuilds afterwards), every
 // head is rotated by the warp, and O is read back at its rows' code scale
 // (2^(p-24), exact), Z cleared.
-template <int VB, int NGRP>
+template <int VB, int NGRP, bool FOLD>
 __device__ __forceinline__ void unrotate_output(float (&O)[8][4], float (&Z)[NGRP][4], float* scr, int NG, int lane,
                                                 bool v0, bool v1) {
   using S = Shape<2, VB, NGRP, 1>;  // value-side constants only
   const int g = lane >> 2, t = lane & 3;
+  if constexpr (FOLD) fold_remainders<NGRP>(O, Z);
   __syncwarp();  // every lane is done with the B fragments
 #pragma unroll
   for (int mt2 = 0; mt2 < 8; ++mt2) {
@@ -992,6 +989,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
               uint32_t bt, bb;
               if constexpr (HPL == 2)
                 prob_operand<HPL>(pack_f16(sc[mt][0], sc[mt][1]), pack_f16(sc[mt][2], sc[mt][3]), 0u, lane, bt, bb);
+              else if constexpr (PT)
+                prob_operand_dup(pack_f16(sc[mt][0], sc[mt][1]), lane, bt, bb);
               else
                 prob_operand<HPL>(0u, 0u, pack_f16(sc[mt][0], sc[mt][1]), lane, bt, bb);
               const int kst = tile * S::MT + mt;
@@ -1002,11 +1001,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
                 const uint4 v4 = vsz4[(kst * 4 + t) * NGRP + gg];  // (s, s), (s, s), (z, z), (z, z) of rows 2t.. 9+2t
                 B0[gg] = hmul2(bt, v4.x);
                 B1[gg] = hmul2(bb, v4.y);
-                if constexpr (PT) {
-                  // whole-vector value groups have scales and zero points
-                  // that are large next to the values they encode: p*s and
-                  // p*z also keep their fp16 remainders (exact), one more
-                  // MMA each
+                // PT: whole-vector value groups have scales and zero points
+                // that are large next to the values they encode, so p*s and
+                // p*z also keep their fp16 remainders (exact): in the free
+                // columns 4-7 with at most 4 heads, else in one more MMA each
+                if constexpr (PT && HPL == 1) {
+                  const bool rem = g >= 4;
+                  B0[gg] = rem ? hfms2(bt, v4.x, B0[gg]) : B0[gg];
+                  B1[gg] = rem ? hfms2(bb, v4.y, B1[gg]) : B1[gg];
+                  const uint32_t z0 = hmul2(bt, v4.z), z1 = hmul2(bb, v4.w);
+                  mma_f16(Z[gg], ones, rem ? hfms2(bt, v4.z, z0) : z0, rem ? hfms2(bb, v4.w, z1) : z1);
+                } else if constexpr (PT) {
                   R0[gg] = hfms2(bt, v4.x, B0[gg]);
                   R1[gg] = hfms2(bb, v4.y, B1[gg]);
                   const uint32_t z0 = hmul2(bt, v4.z), z1 = hmul2(bb, v4.w);
@@ -1032,7 +1037,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
                     const uint32_t a[4] = {code_sub<VB>(xv, xv8, 2 * P), code_sub<VB>(xv, xv8, 2 * P + 1),
                                            code_sub<VB>(yv, yv8, 2 * P), code_sub<VB>(yv, yv8, 2 * P + 1)};
                     mma_f16(O[(cc0 + cc) * S::MT_PER_CH + P], a, B0[gg], B1[gg]);
-                    if constexpr (PT) mma_f16(O[(cc0 + cc) * S::MT_PER_CH + P], a, R0[gg], R1[gg]);
+                    if constexpr (PT && HPL == 2) mma_f16(O[(cc0 + cc) * S::MT_PER_CH + P], a, R0[gg], R1[gg]);
                   }
                 }
               }
@@ -1041,7 +1046,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
         } else {
           if constexpr (PT) {
             if (rotated) {  // exact tokens add in the original basis
-              unrotate_output<VB, NGRP>(O, Z, reinterpret_cast<float*>(ws + mp.bfrag_off), NG, lane, v0, v1);
+              unrotate_output<VB, NGRP, HPL == 1>(O, Z, reinterpret_cast<float*>(ws + mp.bfrag_off), NG, lane, v0,
+                                                  v1);
               rotated = false;
               rq_ready = false;
             }
@@ -1063,8 +1069,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
         }
       }
       if (failed) break;
-      if constexpr (PT)
-        if (rotated) unrotate_output<VB, NGRP>(O, Z, reinterpret_cast<float*>(ws + mp.bfrag_off), NG, lane, v0, v1);
+      if constexpr (PT) {
+        if (rotated)
+          unrotate_output<VB, NGRP, HPL == 1>(O, Z, reinterpret_cast<float*>(ws + mp.bfrag_off), NG, lane, v0, v1);
+        else if constexpr (HPL == 1)
+          fold_remainders<NGRP>(O, Z);
+      }
       // ---------------- this warp's partial for the unit
 #pragma unroll
       for (int off = 4; off <= 16; off <<= 1)

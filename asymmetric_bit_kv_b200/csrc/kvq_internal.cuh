@@ -110,6 +110,38 @@ __device__ __forceinline__ float load_kv(const void* p, int64_t i, int dtype) {
   return __half2float(reinterpret_cast<const __half*>(p)[i]);
 }
 
+// x . H for the 128 channels of one head spread over a warp, channels 4l..4l+3
+// in lane l: radix-2 butterflies of half-width 1, 2, 4, ..., 64 (the first two
+// inside the lane, the others with the lane at xor distance w/4), then one
+// fp32 multiplication by fp32(1/sqrt(128)). The quantizer rotates the keys
+// and values and the decode kernel the queries and outputs in this order.
+__device__ __forceinline__ void rotate_lane(float (&x)[4], int lane) {
+  float a = x[0], c = x[1];
+  x[0] = __fadd_rn(a, c);
+  x[1] = __fsub_rn(a, c);
+  a = x[2], c = x[3];
+  x[2] = __fadd_rn(a, c);
+  x[3] = __fsub_rn(a, c);
+  a = x[0], c = x[2];
+  x[0] = __fadd_rn(a, c);
+  x[2] = __fsub_rn(a, c);
+  a = x[1], c = x[3];
+  x[1] = __fadd_rn(a, c);
+  x[3] = __fsub_rn(a, c);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const bool upper = lane & o;  // this lane holds the x[i + w] side of its pairs
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float other = __shfl_xor_sync(0xffffffffu, x[e], o);
+      x[e] = upper ? __fsub_rn(other, x[e]) : __fadd_rn(x[e], other);
+    }
+  }
+  const float s = (float)(1.0 / sqrt((double)kHeadDim));
+#pragma unroll
+  for (int e = 0; e < 4; ++e) x[e] = __fmul_rn(x[e], s);
+}
+
 // ---------------------------------------------------------------------------
 // The quantizer of the "KV1-1.2B" card (section "Quantization Format: KV1.cpp
 // BQ2_0"), widened from 3 to 2^b - 1 levels. Every operation is an explicitly
