@@ -6,13 +6,15 @@ sequence over the whole cache. The workload is the Llama-3-8B-shaped GQA
 layer: batch 32, 32 query / 8 KV heads, head_dim 128, context 8192, bf16
 keys N(0,1) x log-normal channel magnitudes and values N(0,1), keys 2-bit per
 channel in groups of 64 tokens, values 4-bit per token in groups of 64
-channels, residual window 128.
+channels, residual window 128. `--workload kv1` runs the KV1 card's BQ2_0
+layout on the same shapes (2-bit keys and values per token over whole head
+vectors, Hadamard rotation, 4 exact sink tokens).
 
 Timing: W warm-up steps, then exactly K steps between barriers and device
 synchronisations, timed with CUDA events on the launching stream; the job
 value is the max over ranks. Each step works on the next of several
-independent cache replicas, so every step streams a different 248 MB cache
-(more than the 126 MB L2) and every replica's context grows only by K/replicas
+independent cache replicas, so every step streams a different cache (235 MB;
+151 MB for kv1: more than the 126 MB L2) and every replica's context grows only by K/replicas
 tokens. Multi-GPU runs (torchrun) give every rank its own replicas: weak
 scaling, no collective on the data path.
 
@@ -250,6 +252,16 @@ def cpu_oracle_baseline(steps: int = 100, warmup: int = 2, wname: str = "llama3"
 # the library arm
 # --------------------------------------------------------------------------
 
+def _cache_mb(wl):
+    """Quantized cache bytes of one replica (MB), from the record layout of
+    the method (codes + fp16 scale and zero point per group)."""
+    D, G, Gv = wl.head_dim, wl.group_k, wl.group_v
+    per_token_keys = _layout(wl)[1]
+    kgroups = D / Gv if per_token_keys else D / G
+    per_tok = wl.num_kv_heads * (D * (wl.k_bits[0] + wl.v_bits[0]) / 8 + 4 * kgroups + 4 * D / Gv)
+    return wl.batch * wl.context[0] * per_tok / 1e6
+
+
 def _workload_config(wl, replicas, world, mean_ctx=None):
     """The `config` object of the JSON line (shared by both arms)."""
     cfg = {
@@ -260,7 +272,7 @@ def _workload_config(wl, replicas, world, mean_ctx=None):
         "sinks": _layout(wl)[0], "key_axis": "token" if _layout(wl)[1] else "channel", "hadamard": _layout(wl)[2],
         "kv_dtype": "bf16", "out_dtype": "bf16",
         "replicas": replicas,
-        "l2": "inputs larger than L2: each step reads a different replica's ~248 MB cache",
+        "l2": f"inputs larger than L2: each step reads a different replica's ~{_cache_mb(wl):.0f} MB cache",
         "parallelism": f"dp{world} (independent replicas per rank)",
     }
     if mean_ctx is not None:
@@ -274,7 +286,6 @@ def run_kvq(a):
 
     from asymmetric_bit_kv_b200 import CacheConfig, KVCache
     from asymmetric_bit_kv_b200 import workloads as W
-    from oracle import kvq_oracle as O  # sizes only (closed-form bytes/token), never on the timed path
 
     rank, world, local = _dist_env()
     if world > 1:
@@ -283,7 +294,9 @@ def run_kvq(a):
     dev = torch.device("cuda", local)
     wl = _bench_workload(a.workload)
     sinks, k_axis, rot = _layout(wl)
-    fused = k_axis == 0 and not rot  # tensor-core layers take the new token inside the decode launch
+    # tensor-core layers take the new token inside the decode launch: per-channel
+    # keys without the rotation, or per-token keys over whole head vectors
+    fused = (k_axis == 0 and not rot) or (k_axis == 1 and wl.group_v == wl.head_dim)
     B, Hq, Hkv, D = wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim
     ctx = wl.context[0]
     R = a.replicas
@@ -308,7 +321,9 @@ def run_kvq(a):
     stream = torch.cuda.current_stream()
     # per-step inputs as views made once, so that the timed loop only enqueues
     views = [(new_k[j], new_v[j], qs[j]) for j in range(pool)]
-    bytes_tok = O.quantized_bytes_per_token(Hkv, D, wl.k_bits[0], wl.v_bits[0], wl.group_k, wl.group_v, k_axis)
+    # quantized bytes per token (all KV heads): the library's block record
+    # (codes, scales and zero points of G tokens of one KV head) / G
+    bytes_tok = Hkv * caches[0].layout(0).record_bytes / wl.group_k
 
     G, Rw = wl.group_k, wl.residual
 
@@ -398,17 +413,19 @@ def run_kvq(a):
     achieved_gbs = alg_total / (dec_ms / 1e3) / 1e9
 
     # ---- end to end through the public API with host buffers ----
+    # each step's k, v and q sit back to back in one pinned host buffer and
+    # travel in one host-to-device copy
     e2e_steps = min(a.steps, 512)
-    hk = torch.empty(pool, B, Hkv, D, dtype=wl.kv_dtype).pin_memory()
-    hv = torch.empty_like(hk).pin_memory()
-    hq = torch.empty(pool, B, Hq, D, dtype=wl.kv_dtype).pin_memory()
-    hk.copy_(new_k.cpu())
-    hv.copy_(new_v.cpu())
-    hq.copy_(qs.cpu())
+    nk, nq = B * Hkv * D, B * Hq * D
+    hkvq = torch.empty(pool, 2 * nk + nq, dtype=wl.kv_dtype).pin_memory()
+    hkvq[:, :nk].copy_(new_k.reshape(pool, nk).cpu())
+    hkvq[:, nk:2 * nk].copy_(new_v.reshape(pool, nk).cpu())
+    hkvq[:, 2 * nk:].copy_(qs.reshape(pool, nq).cpu())
     hout = torch.empty(B, Hq, D, dtype=wl.kv_dtype).pin_memory()
-    dk = torch.empty(B, Hkv, D, dtype=wl.kv_dtype, device=dev)
-    dv = torch.empty_like(dk)
-    dq = torch.empty(B, Hq, D, dtype=wl.kv_dtype, device=dev)
+    dkvq = torch.empty(2 * nk + nq, dtype=wl.kv_dtype, device=dev)
+    dk = dkvq[:nk].view(B, Hkv, D)
+    dv = dkvq[nk:2 * nk].view(B, Hkv, D)
+    dq = dkvq[2 * nk:].view(B, Hq, D)
     tok_e2e = 0
     for i in range(e2e_steps):
         r = (a.warmup + a.steps + i) % R
@@ -426,9 +443,7 @@ def run_kvq(a):
     for i in range(e2e_steps):
         r = (a.warmup + a.steps + i) % R
         j = i % pool
-        dk.copy_(hk[j], non_blocking=True)
-        dv.copy_(hv[j], non_blocking=True)
-        dq.copy_(hq[j], non_blocking=True)
+        dkvq.copy_(hkvq[j], non_blocking=True)
         caches[r].decode_step(0, dk, dv, dq, out, softmax_scale=wl.softmax_scale, stream=stream)
         hout.copy_(out, non_blocking=True)
     f1.record(stream)
