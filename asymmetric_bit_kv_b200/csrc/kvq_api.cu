@@ -32,6 +32,12 @@ struct kvq_cache {
   int32_t slots;                  // partial slots per (sequence, query head)
   int32_t sm_count;
   std::vector<int32_t> q_len, n_len, s_len;  // host mirror [num_layers][max_batch]
+  // paged block pools (cfg.page_blocks >= 1)
+  std::vector<int64_t> pt_off;                   // per layer: int32 page table [max_batch][max_pages]
+  int32_t max_pages = 0;                         // page-table entries per sequence
+  std::vector<std::vector<int32_t>> free_pages;  // per layer: free page ids (a stack)
+  std::vector<int32_t> pt_host;                  // [num_layers][max_batch][max_pages] mirror
+  std::vector<int32_t> pages_held;               // [num_layers][max_batch]
 };
 
 namespace {
@@ -89,13 +95,20 @@ kvq_status validate_config(const kvq_config* c) {
       if (c->k_axis[l] != 0 && c->k_axis[l] != 1)
         return fail(KVQ_ERR_INVALID_ARG, "layer %d k_axis %d not 0 or 1", l, c->k_axis[l]);
   if (c->hadamard != 0 && c->hadamard != 1) return fail(KVQ_ERR_INVALID_ARG, "hadamard %d not 0 or 1", c->hadamard);
+  if (c->page_blocks < 0) return fail(KVQ_ERR_INVALID_ARG, "page_blocks %d < 0", c->page_blocks);
+  if (c->page_blocks > 0) {
+    if (c->pool_pages < 1) return fail(KVQ_ERR_INVALID_ARG, "pool_pages %d < 1 with page_blocks %d", c->pool_pages,
+                                       c->page_blocks);
+    if ((int64_t)c->pool_pages * c->num_kv_heads * c->page_blocks > INT32_MAX)
+      return fail(KVQ_ERR_UNSUPPORTED, "more than 2^31 block records in one layer's pool");
+  }
   return KVQ_OK;
 }
 
 struct Plan {
-  std::vector<int64_t> blocks_off, ring_k_off, ring_v_off, sink_k_off, sink_v_off, record_bytes;
+  std::vector<int64_t> blocks_off, ring_k_off, ring_v_off, sink_k_off, sink_v_off, record_bytes, pt_off;
   int64_t max_blocks, lens_off, err_off, uslots_off, ws_o_off, ws_ml_off, total;
-  int32_t slots;
+  int32_t slots, max_pages;
 };
 
 Plan make_plan(const kvq_config* c) {
@@ -104,6 +117,10 @@ Plan make_plan(const kvq_config* c) {
   const int G = c->group_k, D = c->head_dim;
   const int64_t seqheads = (int64_t)c->max_batch * c->num_kv_heads;
   p.max_blocks = c->max_tokens / G;
+  const bool paged = c->page_blocks > 0;
+  p.max_pages = paged ? (int32_t)((p.max_blocks + c->page_blocks - 1) / c->page_blocks) : 0;
+  // block records per layer: every sequence's capacity, or the page pool
+  const int64_t records = paged ? (int64_t)c->pool_pages * c->num_kv_heads * c->page_blocks : seqheads * p.max_blocks;
   int64_t off = 0;
   for (int l = 0; l < c->num_layers; ++l) {
     const int kb = c->k_bits[l], vb = c->v_bits[l];
@@ -114,7 +131,7 @@ Plan make_plan(const kvq_config* c) {
                                  16);
     p.record_bytes.push_back(rec);
     p.blocks_off.push_back(off);
-    off = round_up(off + seqheads * p.max_blocks * rec, 256);
+    off = round_up(off + records * rec, 256);
     const int64_t ring = seqheads * c->residual * D * 2;
     p.ring_k_off.push_back(off);
     off = round_up(off + ring, 256);
@@ -125,6 +142,8 @@ Plan make_plan(const kvq_config* c) {
     off = round_up(off + sink, 256);
     p.sink_v_off.push_back(off);
     off = round_up(off + sink, 256);
+    p.pt_off.push_back(off);
+    off = round_up(off + (paged ? (int64_t)c->max_batch * p.max_pages * 4 : 0), 256);
   }
   p.lens_off = off;
   off = round_up(off + (int64_t)c->num_layers * c->max_batch * 3 * 4, 256);
@@ -177,6 +196,10 @@ kvq::LayerView layer_view(const kvq_cache* c, int layer) {
   v.group_v = cfg.group_v;
   v.residual = cfg.residual;
   v.kv_dtype = cfg.kv_dtype;
+  const bool paged = cfg.page_blocks > 0;
+  v.page_table = paged ? reinterpret_cast<const int32_t*>(c->arena + c->pt_off[layer]) : nullptr;
+  v.page_blocks = paged ? cfg.page_blocks : 0;
+  v.max_pages = c->max_pages;
   return v;
 }
 
@@ -188,6 +211,51 @@ kvq_status check_cache_layer(const kvq_cache* c, int layer) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Paged caches: gives each sequence of the call the pages that its blocks
+// after the call need (taken from the layer's pool) and enqueues the
+// page-table update; fails before changing anything if the pool is short.
+kvq_status take_pages(kvq_cache* c, int layer, const kvq::AppendParams& p, int batch, cudaStream_t stream) {
+  const kvq_config& cfg = c->cfg;
+  const int G = cfg.group_k, P = cfg.page_blocks;
+  int32_t* held = &c->pages_held[(size_t)layer * cfg.max_batch];
+  std::vector<int32_t>& pool = c->free_pages[layer];
+  auto pages_after = [&](int b) {
+    const int64_t blocks = (p.q_old[b] + (int64_t)p.flush[b] * G) / G;
+    return (int32_t)((blocks + P - 1) / P);
+  };
+  int64_t need = 0;
+  for (int b = 0; b < batch; ++b) need += std::max<int64_t>(0, pages_after(b) - held[b]);
+  if (need == 0) return KVQ_OK;
+  if (need > (int64_t)pool.size())
+    return fail(KVQ_ERR_CAPACITY, "layer %d: the call needs %lld new pages; the pool has %zu free of %d", layer,
+                (long long)need, pool.size(), cfg.pool_pages);
+  kvq::PageTableUpdate* u = new (std::nothrow) kvq::PageTableUpdate;
+  if (!u) return fail(KVQ_ERR_INVALID_ARG, "out of host memory");
+  u->table = reinterpret_cast<int32_t*>(c->arena + c->pt_off[layer]);
+  u->n = 0;
+  cudaError_t e = cudaSuccess;
+  for (int b = 0; b < batch && e == cudaSuccess; ++b) {
+    const int32_t want = pages_after(b);
+    int32_t* row = &c->pt_host[((size_t)layer * cfg.max_batch + b) * c->max_pages];
+    while (held[b] < want && e == cudaSuccess) {
+      const int32_t page = pool.back();
+      pool.pop_back();
+      row[held[b]] = page;
+      u->idx[u->n] = b * c->max_pages + held[b];
+      u->page[u->n] = page;
+      ++held[b];
+      if (++u->n == kvq::kMaxPageUpdates) {
+        e = kvq::launch_page_table_update(*u, stream);
+        u->n = 0;
+      }
+    }
+  }
+  if (e == cudaSuccess) e = kvq::launch_page_table_update(*u, stream);
+  delete u;
+  if (e != cudaSuccess) return cuda_fail(e, "page-table update");
+  return KVQ_OK;
+}
 
 // Shared by kvq_append (t_new from the caller) and kvq_flush_residual
 // (t_new = 0, every complete group of the ring flushed).
@@ -225,6 +293,13 @@ kvq_status enqueue_append(kvq_cache* c, int layer, const void* k, const void* v,
     p->flush[b] = f;
     off += T;
     if (f > max_flush) max_flush = f;
+  }
+  if (cfg.page_blocks > 0) {
+    const kvq_status ps = take_pages(c, layer, *p, batch, stream);
+    if (ps != KVQ_OK) {
+      delete p;
+      return ps;
+    }
   }
   cudaError_t e = kvq::launch_append(*p, max_flush, stream);
   if (e == cudaSuccess) {
@@ -502,6 +577,15 @@ kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena
   c->err_off = plan.err_off;
   c->uslots_off = plan.uslots_off;
   c->slots = plan.slots;
+  c->pt_off = plan.pt_off;
+  c->max_pages = plan.max_pages;
+  if (cfg->page_blocks > 0) {
+    c->free_pages.assign(cfg->num_layers, {});
+    for (auto& f : c->free_pages)
+      for (int32_t i = cfg->pool_pages - 1; i >= 0; --i) f.push_back(i);
+    c->pt_host.assign((size_t)cfg->num_layers * cfg->max_batch * c->max_pages, 0);
+    c->pages_held.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
+  }
   c->q_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
   c->n_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
   c->s_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
@@ -521,6 +605,8 @@ kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena
     if (e == cudaSuccess) e = cudaMemset(c->arena + c->ring_v_off[l], 0, ring_bytes);
     if (e == cudaSuccess && sink_bytes) e = cudaMemset(c->arena + c->sink_k_off[l], 0, sink_bytes);
     if (e == cudaSuccess && sink_bytes) e = cudaMemset(c->arena + c->sink_v_off[l], 0, sink_bytes);
+    if (e == cudaSuccess && cfg->page_blocks > 0)  // entries not yet given out name page 0 (valid memory)
+      e = cudaMemset(c->arena + c->pt_off[l], 0, (size_t)cfg->max_batch * c->max_pages * 4);
   }
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
@@ -547,6 +633,35 @@ kvq_status kvq_cache_reset(kvq_cache* c, void* stream) {
   std::fill(c->q_len.begin(), c->q_len.end(), 0);
   std::fill(c->n_len.begin(), c->n_len.end(), 0);
   std::fill(c->s_len.begin(), c->s_len.end(), 0);
+  if (c->cfg.page_blocks > 0) {
+    for (auto& f : c->free_pages) {
+      f.clear();
+      for (int32_t i = c->cfg.pool_pages - 1; i >= 0; --i) f.push_back(i);
+    }
+    std::fill(c->pages_held.begin(), c->pages_held.end(), 0);
+  }
+  return KVQ_OK;
+}
+
+kvq_status kvq_release_sequence(kvq_cache* c, int32_t seq, void* stream) {
+  g_last_error.clear();
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "cache is null");
+  const kvq_config& cfg = c->cfg;
+  if (seq < 0 || seq >= cfg.max_batch) return fail(KVQ_ERR_INVALID_ARG, "seq %d outside 0..%d", seq, cfg.max_batch - 1);
+  for (int l = 0; l < cfg.num_layers; ++l) {
+    cudaError_t e = cudaMemsetAsync(c->arena + c->lens_off + ((size_t)l * cfg.max_batch + seq) * 12, 0, 12,
+                                    static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "release");
+  }
+  for (int l = 0; l < cfg.num_layers; ++l) {
+    const size_t i = (size_t)l * cfg.max_batch + seq;
+    c->q_len[i] = c->n_len[i] = c->s_len[i] = 0;
+    if (cfg.page_blocks > 0) {
+      const int32_t* row = &c->pt_host[i * c->max_pages];
+      for (int32_t k = c->pages_held[i] - 1; k >= 0; --k) c->free_pages[l].push_back(row[k]);
+      c->pages_held[i] = 0;
+    }
+  }
   return KVQ_OK;
 }
 
@@ -685,6 +800,9 @@ kvq_status kvq_get_layout(const kvq_cache* c, int32_t layer, kvq_layout* out) {
   out->sink_v = v.sink_v;
   out->k_axis = v.k_axis;
   out->hadamard = v.hadamard;
+  out->page_table = const_cast<int32_t*>(v.page_table);
+  out->page_blocks = v.page_blocks;
+  out->max_pages = v.max_pages;
   return KVQ_OK;
 }
 

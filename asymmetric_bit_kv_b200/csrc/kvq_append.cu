@@ -298,6 +298,16 @@ cudaError_t launch_append(const AppendParams& p, int max_flush, cudaStream_t str
   return cudaGetLastError();
 }
 
+__global__ void page_table_kernel(PageTableUpdate u) {
+  for (int i = threadIdx.x; i < u.n; i += blockDim.x) u.table[u.idx[i]] = u.page[i];
+}
+
+cudaError_t launch_page_table_update(const PageTableUpdate& u, cudaStream_t stream) {
+  if (u.n <= 0) return cudaSuccess;
+  page_table_kernel<<<1, 256, 0, stream>>>(u);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dequant(const LayerView& L, int seq, int sinks, int t0, int t1, float* k_out, float* v_out,
                            cudaStream_t stream) {
   const int n = t1 - t0;

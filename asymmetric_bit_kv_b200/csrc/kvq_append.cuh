@@ -24,6 +24,17 @@ struct AppendParams {
 };
 
 cudaError_t launch_append(const AppendParams& p, int max_flush, cudaStream_t stream);
+
+// Paged caches: page-table entries set by one launch (table[idx[i]] =
+// page[i]), enqueued before the append kernels that write the new pages.
+constexpr int kMaxPageUpdates = 1536;
+struct PageTableUpdate {
+  int32_t* table;
+  int32_t n;
+  int32_t idx[kMaxPageUpdates];
+  int32_t page[kMaxPageUpdates];
+};
+cudaError_t launch_page_table_update(const PageTableUpdate& u, cudaStream_t stream);
 cudaError_t launch_dequant(const LayerView& L, int seq, int sinks, int t0, int t1, float* k_out, float* v_out,
                            cudaStream_t stream);
 

@@ -715,6 +715,8 @@ __device__ __forceinline__ void store_new_token(const DecodeParams& p, int b, in
 struct IssueState {
   UnitCursor u;
   int unit = -1, seq = -1;
+  int run = -1;           // paged cache: page-table entry (j / page_blocks) of the unit held in `page`
+  int64_t page = 0;
 };
 
 // Issues the copy of work item k (a block record, or the key and value rows
@@ -735,7 +737,18 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, const MmaPlan&
   }
   if (j < nb) {
     mbar_expect_tx(bar, mp.tx_bytes + (newq ? qbytes : 0u));
-    bulk_g2s(dst, record_ptr(L, u.b, u.h, j), mp.tx_bytes, bar);
+    const uint8_t* rec;
+    if (L.page_table) {  // one page-table read per run of page_blocks blocks of the unit
+      const int run = j / L.page_blocks;
+      if (newq || run != is.run) {
+        is.run = run;
+        is.page = __ldg(L.page_table + (int64_t)u.b * L.max_pages + run);
+      }
+      rec = L.blocks + ((is.page * L.num_kv_heads + u.h) * L.page_blocks + j % L.page_blocks) * L.record_bytes;
+    } else {
+      rec = record_ptr(L, u.b, u.h, j);
+    }
+    bulk_g2s(dst, rec, mp.tx_bytes, bar);
     if (j == nb - 1 && p.nres[u.b] > 0) {
       // the unit's ring chunks come next: bring its ring rows into L2 so that
       // those short items do not each wait a full HBM round trip

@@ -14,7 +14,7 @@ constexpr int kHeadDim = 128;  // the decode kernels are specialised for D = 128
 
 // Per-layer view of the packed cache, passed by value to kernels.
 struct LayerView {
-  uint8_t* blocks;        // block records [max_batch][Hkv][max_blocks]
+  uint8_t* blocks;        // block records [max_batch][Hkv][max_blocks], or the page pool (paged)
   void* ring_k;           // [max_batch][Hkv][R][D] kv dtype
   void* ring_v;
   void* sink_k;           // [max_batch][Hkv][KVQ_MAX_SINKS][D] kv dtype (sink_tokens > 0)
@@ -29,6 +29,9 @@ struct LayerView {
   int32_t sinks;          // S: sink tokens kept exact at the start of each sequence
   int32_t k_axis;         // 0: keys per channel over G tokens (KIVI); 1: per token over group_v channels (BQ2_0)
   int32_t hadamard;       // 1: K and V rotated by the normalized Sylvester matrix before quantization
+  const int32_t* page_table;  // paged: [max_batch][max_pages] page of block run j / page_blocks; else null
+  int32_t page_blocks;        // paged: blocks per page (a page holds them for every KV head)
+  int32_t max_pages;          // paged: page-table entries per sequence
 };
 
 __host__ __device__ inline int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
@@ -101,7 +104,13 @@ __host__ __device__ inline int vsz_half_index(int t, int gg, int G, int kb, int 
   return entry * 8 + (zero ? 4 : 0) + 2 * (r >> 3) + (r & 1);
 }
 
+// Block record j of (sequence b, KV head h): contiguous per (b, h), or in a
+// paged cache record (page * Hkv + h) * page_blocks + j % page_blocks.
 __device__ __forceinline__ uint8_t* record_ptr(const LayerView& L, int b, int h, int64_t j) {
+  if (L.page_table) {
+    const int64_t page = __ldg(L.page_table + (int64_t)b * L.max_pages + j / L.page_blocks);
+    return L.blocks + ((page * L.num_kv_heads + h) * L.page_blocks + j % L.page_blocks) * L.record_bytes;
+  }
   return L.blocks + (((int64_t)b * L.num_kv_heads + h) * L.max_blocks + j) * L.record_bytes;
 }
 

@@ -47,6 +47,8 @@ class kvq_config(ctypes.Structure):
         ("sink_tokens", ctypes.c_int32),
         ("k_axis", ctypes.POINTER(ctypes.c_int8)),
         ("hadamard", ctypes.c_int32),
+        ("page_blocks", ctypes.c_int32),
+        ("pool_pages", ctypes.c_int32),
     ]
 
 
@@ -67,6 +69,9 @@ class kvq_layout(ctypes.Structure):
         ("sink_v", ctypes.c_void_p),
         ("k_axis", ctypes.c_int32),
         ("hadamard", ctypes.c_int32),
+        ("page_table", ctypes.c_void_p),
+        ("page_blocks", ctypes.c_int32),
+        ("max_pages", ctypes.c_int32),
     ]
 
 
@@ -88,6 +93,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kvq_cache_create": (I32, [cfgp, P, SZ, ctypes.POINTER(P)]),
         "kvq_cache_destroy": (I32, [P]),
         "kvq_cache_reset": (I32, [P, P]),
+        "kvq_release_sequence": (I32, [P, I32, P]),
         "kvq_append": (I32, [P, I32, P, P, ctypes.POINTER(I32), I32, P]),
         "kvq_flush_residual": (I32, [P, I32, I32, P]),
         "kvq_decode_attention": (I32, [P, I32, P, P, I32, F32, I32, P]),
@@ -151,6 +157,8 @@ class CacheConfig:
     sink_tokens: int = 0
     k_axis: list | None = None  # per layer: 0 keys per channel (KIVI), 1 per token (BQ2_0)
     hadamard: int = 0
+    page_blocks: int = 0  # >= 1: block records in pages of this many blocks from a pool
+    pool_pages: int = 0   # pages per layer (paged)
 
     def to_c(self):
         kb = (ctypes.c_int8 * self.num_layers)(*self.k_bits)
@@ -159,7 +167,8 @@ class CacheConfig:
         c = kvq_config(self.num_layers, self.max_batch, self.num_q_heads, self.num_kv_heads, self.head_dim,
                        self.max_tokens, self.group_k, self.group_v, self.residual, _DTYPE_CODE[self.kv_dtype],
                        ctypes.cast(kb, ctypes.POINTER(ctypes.c_int8)), ctypes.cast(vb, ctypes.POINTER(ctypes.c_int8)),
-                       self.sink_tokens, ctypes.cast(ka, ctypes.POINTER(ctypes.c_int8)), self.hadamard)
+                       self.sink_tokens, ctypes.cast(ka, ctypes.POINTER(ctypes.c_int8)), self.hadamard,
+                       self.page_blocks, self.pool_pages)
         return c, (kb, vb, ka)
 
 
@@ -203,6 +212,11 @@ class KVCache:
 
     def reset(self, stream=None):
         _check(self.lib.kvq_cache_reset(self.handle, _stream_ptr(stream)), "kvq_cache_reset")
+
+    def release_sequence(self, seq: int, stream=None):
+        """Empty sequence seq in every layer; a paged cache returns its pages
+        (kvq_release_sequence)."""
+        _check(self.lib.kvq_release_sequence(self.handle, seq, _stream_ptr(stream)), "kvq_release_sequence")
 
     def append(self, layer: int, k: torch.Tensor, v: torch.Tensor, new_lens, stream=None):
         """k, v: [sum(new_lens), Hkv, D] in the cache dtype; new_lens: ints per

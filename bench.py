@@ -51,6 +51,8 @@ def _args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="llama3", choices=["llama3", "kv1"],
                     help="llama3: the headline KIVI layer (default); kv1: the same shapes with the KV1 card's BQ2_0 cache")
+    ap.add_argument("--page-blocks", type=int, default=0,
+                    help="block records in pages of this many blocks drawn from a pool (0: contiguous)")
     return ap.parse_args()
 
 
@@ -303,7 +305,8 @@ def run_kvq(a):
     steps_per_rep = math.ceil((a.warmup + 2 * a.steps) / R) + 2
     cap = ctx + steps_per_rep + wl.group_k
     cfg = CacheConfig(1, B, Hq, Hkv, D, cap, wl.group_k, wl.group_v, wl.residual, wl.kv_dtype, wl.k_bits, wl.v_bits,
-                      sink_tokens=sinks, k_axis=[k_axis], hadamard=rot)
+                      sink_tokens=sinks, k_axis=[k_axis], hadamard=rot, page_blocks=a.page_blocks,
+                      pool_pages=B * -(-(cap // wl.group_k) // a.page_blocks) if a.page_blocks else 0)
     caches = []
     for r in range(R):
         c = KVCache(cfg, dev)
@@ -469,7 +472,8 @@ def run_kvq(a):
             "vs_baseline": None,
             "dtype": "f32",
             "data": "synthetic (seeded; Llama-3-8B-shaped layer, no model weights)",
-            "config": _workload_config(wl, R, world, tok_total / (a.steps * B)),
+            "config": dict(_workload_config(wl, R, world, tok_total / (a.steps * B)),
+                           **({"page_blocks": a.page_blocks} if a.page_blocks else {})),
             "roofline": {
                 "kernel": ("decode step: one token appended per sequence inside the split-KV decode kernel, + log-sum-exp "
                            "combine, per call (a ring flush adds the quantize and ring kernels)") if fused else

@@ -54,7 +54,8 @@ typedef enum kvq_status {
   KVQ_OK = 0,
   KVQ_ERR_INVALID_ARG = -1, /* null pointer, bad index, bad shape or size  */
   KVQ_ERR_UNSUPPORTED = -2, /* valid but not built: bits, dims, dtype      */
-  KVQ_ERR_CAPACITY = -3,    /* a sequence would exceed max_tokens          */
+  KVQ_ERR_CAPACITY = -3,    /* a sequence would exceed max_tokens, or a
+                               paged layer's pool has too few free pages   */
   KVQ_ERR_WORKSPACE = -4,   /* arena smaller than kvq_cache_required_bytes */
   KVQ_ERR_CUDA = -5         /* a CUDA launch or call failed                */
 } kvq_status;
@@ -96,6 +97,15 @@ typedef struct kvq_config {
                            is quantized, queries by H for quantized tokens
                            and their output contribution by H again (KV1
                            BQ2_0); sinks and ring stay exact. 0: none       */
+  int32_t page_blocks;  /* 0: every (sequence, KV head) owns max_tokens/G
+                           block records up front (contiguous). >= 1: block
+                           records live in pages of page_blocks blocks of
+                           one sequence (all its KV heads), drawn per layer
+                           from a pool of pool_pages pages as the sequence's
+                           quantized part grows and returned by
+                           kvq_release_sequence / kvq_cache_reset, so a
+                           ragged batch holds only the pages it uses        */
+  int32_t pool_pages;   /* pages per layer when page_blocks >= 1            */
 } kvq_config;
 
 typedef struct kvq_cache kvq_cache;
@@ -106,7 +116,8 @@ typedef struct kvq_cache kvq_cache;
  * Block records: for sequence b, KV head h and key block j (positions
  * [j*G, (j+1)*G) of that sequence) the record starts at
  *   blocks + ((b * num_kv_heads + h) * max_blocks + j) * record_bytes
- * and holds, at the given byte offsets:
+ * (a paged cache: see page_table below) and holds, at the given byte
+ * offsets:
  *   kc  uint32 [D][W], W = G*k_bits/32: channel d's row holds W words; word
  *       w packs the codes of tokens w*(32/k_bits) + i, i = 0.., code i at
  *       bits [i*k_bits, ...) (per-channel keys packed along the token axis);
@@ -143,6 +154,12 @@ typedef struct kvq_layout {
   void* sink_k;
   void* sink_v;
   int32_t k_axis, hadamard;
+  /* paged caches (page_blocks >= 1): block j of (b, h) is record
+   * (page * num_kv_heads + h) * page_blocks + j % page_blocks of `blocks`,
+   * page = page_table[b * max_pages + j / page_blocks] (int32, device);
+   * max_blocks is then the per-sequence capacity in blocks.               */
+  void* page_table;
+  int32_t page_blocks, max_pages;
 } kvq_layout;
 
 /* Device bytes the arena must hold for cfg: all layers' block records and
@@ -162,6 +179,11 @@ KVQ_API kvq_status kvq_cache_destroy(kvq_cache* cache);
 /* Empty every sequence of every layer (stream-ordered).                    */
 KVQ_API kvq_status kvq_cache_reset(kvq_cache* cache, void* stream);
 
+/* Empty sequence `seq` in every layer (stream-ordered) and, in a paged
+ * cache, return its pages to the pools. Calls that use the pages again are
+ * ordered after this one on the same stream.                              */
+KVQ_API kvq_status kvq_release_sequence(kvq_cache* cache, int32_t seq, void* stream);
+
 /* Append new_lens[b] tokens to sequence b of `layer`, b < batch.
  * k, v: device, token-major [sum(new_lens)][num_kv_heads][head_dim] in
  * kv_dtype, sequences in order. new_lens: host [batch], each >= 0.
@@ -174,7 +196,10 @@ KVQ_API kvq_status kvq_cache_reset(kvq_cache* cache, void* stream);
  * the G tokens, values per token over group_v channels -- into one block
  * record. Blocks that a long append would quantize straight away are read
  * from k, v directly. Fails with KVQ_ERR_CAPACITY if a sequence would exceed
- * max_tokens (sinks included).                                             */
+ * max_tokens (sinks included) or, in a paged cache, if the layer's pool has
+ * fewer free pages than the call's new blocks need; nothing is enqueued
+ * then. A paged cache takes the pages in this call (and in
+ * kvq_flush_residual and kvq_decode_step).                                 */
 KVQ_API kvq_status kvq_append(kvq_cache* cache, int32_t layer, const void* k, const void* v,
                       const int32_t* new_lens, int32_t batch, void* stream);
 

@@ -102,6 +102,18 @@ class Twin:
                     self.ora[(layer, b)].append(kk, vv)
                 off += n
 
+    def release_sequence(self, b: int):
+        """Empty sequence b in every layer on both sides."""
+        self.gpu.release_sequence(b)
+        cfg = self.cfg
+        for layer in self.oracle_layers:
+            if (layer, b) in self.ora:
+                self.ora[(layer, b)] = O.SequenceCache(cfg.num_kv_heads, cfg.head_dim, cfg.k_bits[layer],
+                                                       cfg.v_bits[layer], cfg.group_k, cfg.group_v, cfg.residual,
+                                                       sinks=cfg.sink_tokens,
+                                                       k_axis=(cfg.k_axis or [0] * cfg.num_layers)[layer],
+                                                       hadamard=bool(cfg.hadamard))
+
     def flush_residual(self, layer: int, batch: int):
         self.gpu.flush_residual(layer, batch)
         for b in range(batch):
@@ -122,8 +134,19 @@ class Twin:
         cfg = self.cfg
         G, D, Gv = cfg.group_k, cfg.head_dim, cfg.group_v
         kb, vb = lay.k_bits, lay.v_bits
-        start = lay.blocks - self.gpu.arena.data_ptr() + ((b * cfg.num_kv_heads + h) * lay.max_blocks) * lay.record_bytes
-        raw = self.gpu.arena[start:start + nblk * lay.record_bytes].cpu().numpy().reshape(nblk, lay.record_bytes)
+        base = lay.blocks - self.gpu.arena.data_ptr()
+        if lay.page_blocks:  # paged: record (page * Hkv + h) * P + j % P, page from the device page table
+            P = lay.page_blocks
+            pt_off = lay.page_table - self.gpu.arena.data_ptr()
+            row = self.gpu.arena[pt_off + b * lay.max_pages * 4:pt_off + (b + 1) * lay.max_pages * 4]
+            pages = row.cpu().view(torch.int32).numpy()
+            recs = [((int(pages[j // P]) * cfg.num_kv_heads + h) * P + j % P) for j in range(nblk)]
+            arena = self.gpu.arena
+            raw = np.stack([arena[base + r * lay.record_bytes:base + (r + 1) * lay.record_bytes].cpu().numpy()
+                            for r in recs]) if nblk else np.zeros((0, lay.record_bytes), np.uint8)
+        else:
+            start = base + ((b * cfg.num_kv_heads + h) * lay.max_blocks) * lay.record_bytes
+            raw = self.gpu.arena[start:start + nblk * lay.record_bytes].cpu().numpy().reshape(nblk, lay.record_bytes)
 
         def part(off, nbytes, dtype, shape):
             return np.ascontiguousarray(raw[:, off:off + nbytes]).view(dtype).reshape((nblk,) + shape)
