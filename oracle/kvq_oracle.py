@@ -61,6 +61,12 @@ the design notes of the repository):
    a pair (a, b) becomes (a + b, a - b), each one fp32 rounding) followed by
    one fp32 multiplication by fp32(1/sqrt(D)).
 
+8. Several query tokens per sequence (verifying T drafted tokens in one
+   pass, a serving pattern none of the pages describes; the plainest reading
+   of their decoding rule): the T tokens' keys and values are appended first,
+   and query t, at position L - T + t, attends causally to the tokens up to
+   its own position. T = 1 is reading 5.
+
 Floating point: the quantizer runs in IEEE fp32 (the precision the KV1 card
 fixes); numpy evaluates each fp32 operation with one rounding and never
 contracts a multiply-add. Attention runs in fp64.
@@ -383,6 +389,19 @@ def decode_attention(cache: SequenceCache, q: np.ndarray, scale: float) -> np.nd
     ring (for a Hadamard cache, the effective keys and values)."""
     k, v = cache.dequantized(effective=True)
     return attention(q, k, v, scale)
+
+
+def decode_attention_multi(cache: SequenceCache, q: np.ndarray, scale: float) -> np.ndarray:
+    """Decode attention of T query tokens of one sequence ([T, Hq, D]) whose
+    own keys and values are the sequence's T newest cached tokens (reading 8):
+    query t sits at position L - T + t and attends to tokens 0 .. L - T + t.
+    Returns fp64 [T, Hq, D]."""
+    q = np.asarray(q, dtype=np.float64)
+    T = q.shape[0]
+    k, v = cache.dequantized(effective=True)
+    L = k.shape[0]
+    assert 1 <= T <= L
+    return np.stack([attention(q[t], k[:L - T + t + 1], v[:L - T + t + 1], scale) for t in range(T)])
 
 
 # ---------------------------------------------------------------------------

@@ -508,3 +508,59 @@ def test_kv1_memory_table():
         assert round(per_tok / 1024, 1) == row["per_token_kib"], row
         assert round(per_tok * 8192 / 2 ** 20) == row["ctx_8k_mib"], row
         assert round(per_tok * 32768 / 2 ** 20) == row["ctx_32k_mib"], row
+
+
+# ---------------------------------------------------------------------------
+# Several query tokens per sequence (oracle reading 8)
+# ---------------------------------------------------------------------------
+
+
+def _cache(seed, L, R=64, G=32, kb=2, vb=4, H=2, S=0):
+    rng = np.random.default_rng(seed)
+    k = (rng.standard_normal((L, H, 16)) * np.exp(rng.standard_normal((1, H, 16)))).astype(np.float16).astype(np.float32)
+    v = rng.standard_normal((L, H, 16)).astype(np.float16).astype(np.float32)
+    c = O.SequenceCache(H, 16, kb, vb, G, 16, R, sinks=S)
+    c.append(k, v)
+    return c, k, v
+
+
+def test_multi_query_is_causal_sdpa_over_the_effective_cache():
+    c, _, _ = _cache(3, 150)
+    K, V = c.dequantized(effective=True)
+    L, T = K.shape[0], 5
+    q = np.random.default_rng(4).standard_normal((T, 4, 16))
+    o = O.decode_attention_multi(c, q, 0.25)
+    # torch SDPA with an explicit mask: query t sees keys j <= L - T + t
+    mask = torch.from_numpy(np.arange(L)[None, :] <= (L - T + np.arange(T))[:, None])
+    kk = torch.from_numpy(K).permute(1, 0, 2).repeat_interleave(2, 0)   # [Hq, L, D]
+    vv = torch.from_numpy(V).permute(1, 0, 2).repeat_interleave(2, 0)
+    qq = torch.from_numpy(q).permute(1, 0, 2)                          # [Hq, T, D]
+    ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, attn_mask=mask, scale=0.25)
+    assert np.abs(o - ref.permute(1, 0, 2).numpy()).max() < 1e-12
+
+
+def test_multi_query_rows_equal_single_decodes_of_the_prefixes():
+    # no flush among the last T appends (the ring had room): the cache of the
+    # first L - T + t + 1 tokens holds the same blocks, so query t equals a
+    # single-token decode of that shorter cache
+    L, T = 150, 4            # R 64, G 32: 96 quantized + 54 in the ring, also for 147..149 tokens
+    full, k, v = _cache(8, L)
+    assert full.residual_tokens >= T + 32
+    q = np.random.default_rng(9).standard_normal((T, 4, 16))
+    o = O.decode_attention_multi(full, q, 0.3)
+    for t in range(T):
+        part = O.SequenceCache(2, 16, 2, 4, 32, 16, 64)
+        part.append(k[:L - T + t + 1], v[:L - T + t + 1])
+        assert part.quantized_tokens == full.quantized_tokens
+        assert np.array_equal(o[t], O.decode_attention(part, q[t], 0.3))
+
+
+def test_multi_query_single_token_is_decode_and_sinks_stay_visible():
+    c, _, _ = _cache(5, 90, S=3)
+    q = np.random.default_rng(6).standard_normal((1, 4, 16))
+    assert np.array_equal(O.decode_attention_multi(c, q, 0.2)[0], O.decode_attention(c, q[0], 0.2))
+    # uniform scores (q = 0): query t averages the values of tokens 0 .. L - T + t
+    _, V = c.dequantized(effective=True)
+    o = O.decode_attention_multi(c, np.zeros((3, 4, 16)), 0.2)
+    for t in range(3):
+        assert np.allclose(o[t, 0], V[:90 - 3 + t + 1, 0].mean(0), atol=1e-12)
