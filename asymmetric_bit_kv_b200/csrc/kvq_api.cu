@@ -384,7 +384,8 @@ namespace kvq {
 // call uses, and a call whose partials would not fit is rejected before
 // anything is enqueued.
 kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const void* new_v, const void* q, void* out, int32_t out_dtype,
-                          float softmax_scale, int32_t batch, void* stream, const StaticScratch* scratch) {
+                          float softmax_scale, int32_t batch, void* stream, const StaticScratch* scratch,
+                          const QueryGroup* qg) {
   kvq_status s = check_cache_layer(c, layer);
   if (s != KVQ_OK) return s;
   if (batch < 0 || batch > c->cfg.max_batch)
@@ -398,14 +399,25 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const 
   const kvq_config& cfg = c->cfg;
   const int G = cfg.group_k;
   const kvq::LayerView L = layer_view(c, layer);
-  const bool use_mma = kvq::mma_supported(L, cfg.num_q_heads);
+  // query rows per launch: the query heads of each of the group's tokens
+  const int qtok = qg ? qg->qtok : 1;
+  const int Hv = cfg.num_q_heads * qtok;
+  const bool use_mma = kvq::mma_supported(L, Hv);
   kvq::MmaPlan mp{};
   int per_sm = 4;
-  if (!use_mma) per_sm = kvq::split_ctas_per_sm(cfg.num_q_heads, cfg.num_kv_heads);
+  if (!use_mma) per_sm = kvq::split_ctas_per_sm(Hv, cfg.num_kv_heads);
   if (use_mma) {
-    mp = kvq::make_mma_plan(L, cfg.num_q_heads);
-    per_sm = kvq::mma_ctas_per_sm(L, mp, cfg.num_q_heads);
+    mp = kvq::make_mma_plan(L, Hv);
+    per_sm = kvq::mma_ctas_per_sm(L, mp, Hv);
   }
+  // partial slots per (sequence, query row) that fit the arena's workspace
+  // (sized for num_q_heads rows): all of them for one query token, fewer for
+  // a group, whose slot stride is then cut to what the launch uses
+  const int32_t slot_cap =
+      qg ? (int32_t)std::min<int64_t>(c->slots, (int64_t)cfg.max_batch * cfg.num_q_heads * c->slots /
+                                                    ((int64_t)batch * Hv))
+         : c->slots;
+  if (slot_cap < 2) return fail(KVQ_ERR_WORKSPACE, "the workspace holds too few partial slots for %d query rows", Hv);
   // per-call scratch of this thread (no heap traffic per call)
   thread_local std::vector<int> nblk;
   nblk.resize(batch);
@@ -442,7 +454,11 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const 
   p.score_scale = p.scale_log2 / p.q_prescale;
   p.out_dtype = out_dtype;
   p.batch = batch;
-  p.num_q_heads = cfg.num_q_heads;
+  p.num_q_heads = Hv;
+  p.q_heads = cfg.num_q_heads;
+  p.q_rows = qg ? qg->q_rows : cfg.num_q_heads;
+  p.qtok = qtok;
+  p.lag_base = qg ? qg->lag_base : 0;
   p.slots = c->slots;
   p.err = reinterpret_cast<int32_t*>(c->arena + c->err_off);
   p.unit_slots = reinterpret_cast<int32_t*>(c->arena + c->uslots_off);
@@ -475,12 +491,16 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const 
           need = std::max(need, kvq::persistent_slots(p.cta_start, (int32_t)nctas, p.seq_start[b] + h * p.nitem[b],
                                                       p.nitem[b]));
       used_slots = need;
-      if (need <= c->slots || nctas == 1) break;
+      if (need <= slot_cap || nctas == 1) break;
       nctas = std::max<int64_t>(1, nctas * 3 / 4);
     }
     p.persistent = 1;
     p.total_blocks = (int32_t)total;
     p.num_ctas = (int32_t)nctas;
+    if (used_slots > slot_cap)
+      return fail(KVQ_ERR_WORKSPACE, "the workspace holds %d partial slots per query row; this call needs %d",
+                  slot_cap, used_slots);
+    if (qg) p.slots = used_slots;
     if (scratch && !use_scratch(p, *scratch, batch, used_slots, &s)) return s;
     e = kvq::launch_decode_mma(p, mp, static_cast<cudaStream_t>(stream));
     if (e == cudaSuccess) e = kvq::launch_combine(p, static_cast<cudaStream_t>(stream));
@@ -488,7 +508,7 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const 
     // Split plan: blocks per split chosen to minimise (waves of CTAs) x
     // (blocks per CTA + a fixed per-CTA overhead), with at most slots-1 splits.
     const int64_t slots_gpu = (int64_t)std::max(1, c->sm_count) * per_sm;
-    const int64_t min_bps = std::max<int64_t>(1, (max_blk + (c->slots - 1) - 1) / (c->slots - 1));
+    const int64_t min_bps = std::max<int64_t>(1, (max_blk + (slot_cap - 1) - 1) / (slot_cap - 1));
     int64_t bps = std::max<int64_t>(min_bps, max_blk);
     double best = 1e300;
     for (int64_t cand = min_bps; cand <= std::max<int64_t>(min_bps, max_blk); ++cand) {
@@ -505,6 +525,7 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const 
     p.blocks_per_split = (int32_t)bps;
     const int nsplits = (int)((max_blk + bps - 1) / bps);
     used_slots = nsplits + 1;
+    if (qg) p.slots = used_slots;
     if (scratch && !use_scratch(p, *scratch, batch, used_slots, &s)) return s;
     e = kvq::launch_decode(p, nsplits, static_cast<cudaStream_t>(stream));
   }
@@ -706,6 +727,47 @@ kvq_status kvq_decode_attention(kvq_cache* c, int32_t layer, const void* q, void
                                 float softmax_scale, int32_t batch, void* stream) {
   g_last_error.clear();
   return kvq::enqueue_decode(c, layer, nullptr, nullptr, q, out, out_dtype, softmax_scale, batch, stream, nullptr);
+}
+
+kvq_status kvq_decode_attention_multi(kvq_cache* c, int32_t layer, const void* q, void* out, int32_t out_dtype,
+                                      float softmax_scale, int32_t batch, int32_t num_tokens, void* stream) {
+  g_last_error.clear();
+  kvq_status s = check_cache_layer(c, layer);
+  if (s != KVQ_OK) return s;
+  if (batch < 0 || batch > c->cfg.max_batch)
+    return fail(KVQ_ERR_INVALID_ARG, "batch %d outside 0..%d", batch, c->cfg.max_batch);
+  if (num_tokens < 1 || num_tokens > c->cfg.residual)
+    return fail(KVQ_ERR_INVALID_ARG, "num_tokens %d outside 1..%d (the residual window)", num_tokens,
+                c->cfg.residual);
+  if (out_dtype != KVQ_F32 && out_dtype != KVQ_F16 && out_dtype != KVQ_BF16)
+    return fail(KVQ_ERR_INVALID_ARG, "out_dtype %d", out_dtype);
+  if (batch == 0) return KVQ_OK;
+  if (!q || !out) return fail(KVQ_ERR_INVALID_ARG, "q or out is null");
+  const kvq_config& cfg = c->cfg;
+  // the query tokens' own keys and values are the newest cached tokens,
+  // still in the ring, where the causal mask applies
+  for (int b = 0; b < batch; ++b) {
+    const int n = c->n_len[(size_t)layer * cfg.max_batch + b];
+    if (n < num_tokens)
+      return fail(KVQ_ERR_UNSUPPORTED,
+                  "sequence %d has %d ring tokens: its %d query tokens must be its newest tokens, in the ring", b,
+                  n, num_tokens);
+  }
+  // groups of query tokens, at most 8 query rows per KV head per launch
+  const int ngr = cfg.num_q_heads / cfg.num_kv_heads;
+  const int64_t qrow = (int64_t)cfg.num_q_heads * cfg.head_dim;  // elements per query token of a sequence
+  const int out_size = out_dtype == KVQ_F32 ? 4 : 2;
+  for (int t0 = 0; t0 < num_tokens;) {
+    int tp = 1;
+    while (2 * tp * ngr <= 8 && t0 + 2 * tp <= num_tokens) tp *= 2;
+    const kvq::QueryGroup g{num_tokens * cfg.num_q_heads, tp, num_tokens - 1 - t0};
+    s = kvq::enqueue_decode(c, layer, nullptr, nullptr, static_cast<const uint8_t*>(q) + t0 * qrow * 2,
+                            static_cast<uint8_t*>(out) + t0 * qrow * out_size, out_dtype, softmax_scale, batch,
+                            stream, nullptr, &g);
+    if (s != KVQ_OK) return s;
+    t0 += tp;
+  }
+  return KVQ_OK;
 }
 
 kvq_status kvq_decode_step(kvq_cache* c, int32_t layer, const void* k, const void* v, const void* q, void* out,

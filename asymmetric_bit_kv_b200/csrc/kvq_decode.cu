@@ -98,9 +98,11 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
   __shared__ float sm[4][NG], sl[4][NG];
   __shared__ float so[4][NG][D];
 
+  const int ngr = p.q_heads / L.num_kv_heads;  // query rows hh: token hh / ngr, head h * ngr + hh % ngr
   for (int i = threadIdx.x; i < NG * D; i += blockDim.x) {
     const int hh = i / D, d = i % D;
-    sq[hh][d] = load_kv(p.q, ((int64_t)b * p.num_q_heads + h * NG + hh) * D + d, L.kv_dtype) * p.scale_log2;
+    const int64_t row = (int64_t)b * p.q_rows + (hh / ngr) * p.q_heads + h * ngr + hh % ngr;
+    sq[hh][d] = load_kv(p.q, row * D + d, L.kv_dtype) * p.scale_log2;
   }
   __syncthreads();
   if (L.hadamard && s > 0) {
@@ -143,6 +145,8 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
       }
 #pragma unroll
       for (int hh = 0; hh < NG; ++hh) {
+        // query token hh / ngr does not see the ring's last lag_base - hh / ngr tokens
+        if (!sink && e - nsink >= n - (p.lag_base - hh / ngr)) continue;
         float part = 0.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) part += sq[hh][lane + 32 * c] * kv[c];
@@ -354,7 +358,10 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineParams p) {
     r[2] = __fdiv_rn(acc.z, lsum);
     r[3] = __fdiv_rn(acc.w, lsum);
   }
-  const int64_t o = ((int64_t)b * p.num_q_heads + hq) * D + 4 * lane;
+  // output row of query row hq: query token jv / ngr, head h * ngr + jv % ngr
+  const int ngv = p.num_q_heads / p.num_kv_heads, ngr = p.q_heads / p.num_kv_heads;
+  const int jv = hq % ngv;
+  const int64_t o = ((int64_t)b * p.q_rows + (jv / ngr) * p.q_heads + (hq / ngv) * ngr + jv % ngr) * D + 4 * lane;
   if (p.out_dtype == KVQ_F32) {
     *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + o) = make_float4(r[0], r[1], r[2], r[3]);
   } else if (p.out_dtype == KVQ_BF16) {
@@ -426,7 +433,8 @@ cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream) {
   cfg.numAttrs = 1;
   const CombineParams cp{p.ws_o,         p.ws_ml,          p.out,           p.unit_slots,
                          p.L.lens,       p.out_dtype,      p.num_q_heads,   p.L.num_kv_heads,
-                         p.slots,        p.L.group_k,      p.blocks_per_split, p.persistent, p.L.hadamard};
+                         p.slots,        p.L.group_k,      p.blocks_per_split, p.persistent, p.L.hadamard,
+                         p.q_heads,      p.q_rows};
   return cudaLaunchKernelEx(&cfg, combine_kernel, cp);
 }
 

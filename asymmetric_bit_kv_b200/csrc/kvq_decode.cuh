@@ -42,6 +42,17 @@ struct DecodeParams {
   int32_t persistent;   // 1: persistent-mode slots (see above)
   int32_t total_blocks; // T, persistent mode: work items of all units
   int32_t num_ctas;     // persistent mode
+  // Query rows. A unit (sequence b, KV head h) has num_q_heads / Hkv rows:
+  // row j is query token t = j / (q_heads / Hkv) of this launch and head
+  // h * (q_heads / Hkv) + j % (q_heads / Hkv), read from row
+  // b * q_rows + t * q_heads + that head of q (written to the same row of
+  // out). Query token t attends to the ring except its last lag_base - t
+  // tokens (several query tokens per sequence; one token: q_rows = q_heads,
+  // lag_base = 0).
+  int32_t q_heads;      // Hq of the q and out arrays
+  int32_t q_rows;       // rows of q and out per sequence
+  int32_t qtok;         // query tokens of this launch
+  int32_t lag_base;
   int32_t nblk[KVQ_MAX_BATCH];       // quantized blocks per sequence (host mirror)
   int32_t nres[KVQ_MAX_BATCH];       // ring tokens per sequence (host mirror)
   int32_t nitem[KVQ_MAX_BATCH];      // persistent mode: work items per unit of sequence b
@@ -121,6 +132,7 @@ struct CombineParams {
   const int32_t* lens;        // split mode: the layer's length table
   int32_t out_dtype, num_q_heads, num_kv_heads, slots, group_k, blocks_per_split, persistent;
   int32_t hadamard;  // split mode: slots >= 1 (quantized tokens) hold rotated partials
+  int32_t q_heads, q_rows;  // output row of query row j of a unit: see DecodeParams
 };
 
 // The log-sum-exp combine of the partial slots (after the decode kernel).
@@ -132,10 +144,18 @@ struct StaticScratch {
   int64_t bytes;
 };
 
+// Several query tokens per sequence, one launch's share (see DecodeParams):
+// q and out point at the group's first query token.
+struct QueryGroup {
+  int32_t q_rows, qtok, lag_base;
+};
+
 // Host side of kvq_decode_attention (kvq_api.cu): validation, split plan and
-// launches; the partials go to `scratch` when it is not null.
+// launches; the partials go to `scratch` when it is not null; qg: a group of
+// query tokens (null: one query token per sequence).
 kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const void* new_v, const void* q, void* out, int32_t out_dtype,
-                          float softmax_scale, int32_t batch, void* stream, const StaticScratch* scratch);
+                          float softmax_scale, int32_t batch, void* stream, const StaticScratch* scratch,
+                          const QueryGroup* qg = nullptr);
 void clear_last_error();
 kvq_status report_cuda_error(cudaError_t e, const char* what);
 

@@ -483,7 +483,8 @@ __device__ __forceinline__ void fold_remainders(float (&O)[8][4], float (&Z)[NGR
 // (probability high and low parts) into a scratch accumulator, added to O at
 // the row scale of the quantized blocks' value codes (2^(p-24)).
 template <bool BF16, int VB, int NGRP, int NKT>
-__device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t* qw, uint2* bk, int cnt, int NG,
+__device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t* qw, uint2* bk,
+                                           const int (&cnt)[heads_per_lane<NKT>()], int NG,
                                            int lane, float score_scale, const bool (&valid)[heads_per_lane<NKT>()],
                                            bool& rq_ready, SoftState<heads_per_lane<NKT>()>& sst, float (&O)[8][4],
                                            float (&Z)[NGRP][4]) {
@@ -538,7 +539,7 @@ __device__ __forceinline__ void ring_chunk(const uint8_t* stage, const uint32_t*
   float sc[1][2 * HPL];
 #pragma unroll
   for (int h = 0; h < HPL; ++h) {
-    sc[0][h] = g < cnt ? head_score<NKT>(Dr, 0, h) : -INFINITY;
+    sc[0][h] = g < cnt[h] ? head_score<NKT>(Dr, 0, h) : -INFINITY;
     sc[0][HPL + h] = -INFINITY;
   }
   softmax_update<1, HPL, NGRP, true>(sc, sst, valid, O, Z, lane);
@@ -795,10 +796,16 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, const MmaPlan&
       bulk_g2s(dst + bytes, vr, bytes, bar);
     }
   }
-  if (newq)
-    bulk_g2s(qbuf + (size_t)(is.seq % mp.nstages) * qbytes,
-             reinterpret_cast<const uint8_t*>(p.q) + ((int64_t)u.b * p.num_q_heads + u.h * NG) * kRowBytes, qbytes,
-             bar);
+  if (newq) {
+    // the unit's query rows: ngr heads of each of the launch's query tokens
+    const int ngr = p.q_heads / L.num_kv_heads;
+    uint8_t* qdst = qbuf + (size_t)(is.seq % mp.nstages) * qbytes;
+    for (int t = 0; t < p.qtok; ++t)
+      bulk_g2s(qdst + (size_t)t * ngr * kRowBytes,
+               reinterpret_cast<const uint8_t*>(p.q) +
+                   ((int64_t)u.b * p.q_rows + (int64_t)t * p.q_heads + u.h * ngr) * kRowBytes,
+               ngr * kRowBytes, bar);
+  }
 }
 
 // PT: keys per token over whole head vectors, with the rotation when the
@@ -811,7 +818,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
   const int c = blockIdx.x;
   const LayerView& L = p.L;
   const int Hkv = L.num_kv_heads;
-  const int NG = p.num_q_heads / Hkv;
+  const int NG = p.num_q_heads / Hkv;  // query rows per unit
+  const int ngr = p.q_heads / Hkv;      // query heads per KV head (rows per query token)
   const int G = L.group_k;
   const int rs = p.cta_start[c], re = p.cta_start[c + 1];
   const bool bf16 = L.kv_dtype == KVQ_BF16;
@@ -1067,7 +1075,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
             uq_ready = false;  // ring_chunk writes its own query over the B fragments
           }
           bool sink;
-          const int cnt = exact_chunk(p, u.b, j - nb, sink);
+          const int cnt0 = exact_chunk(p, u.b, j - nb, sink);
+          // tokens of the chunk each lane head sees: a ring chunk hides its
+          // last lag_base - t tokens from query token t (several per sequence)
+          int cnt[HPL];
+#pragma unroll
+          for (int h = 0; h < HPL; ++h)
+            cnt[h] = sink ? cnt0 : cnt0 - (p.lag_base - (HPL == 2 ? 2 * t + h : t) / ngr);
           if (p.new_k && !sink && j - nb == (p.nres[u.b] - 1) / kResChunk) store_new_token(p, u.b, u.h, nb, stage, lane);
           if (bf16)
             ring_chunk<true, VB, NGRP, NKT>(stage, qw, bkw, cnt, NG, lane, p.score_scale, valid, rq_ready, sst, O, Z);

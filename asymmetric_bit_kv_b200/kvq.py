@@ -94,6 +94,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kvq_cache_destroy": (I32, [P]),
         "kvq_cache_reset": (I32, [P, P]),
         "kvq_release_sequence": (I32, [P, I32, P]),
+        "kvq_decode_attention_multi": (I32, [P, I32, P, P, I32, F32, I32, I32, P]),
         "kvq_append": (I32, [P, I32, P, P, ctypes.POINTER(I32), I32, P]),
         "kvq_flush_residual": (I32, [P, I32, I32, P]),
         "kvq_decode_attention": (I32, [P, I32, P, P, I32, F32, I32, P]),
@@ -261,6 +262,21 @@ class KVCache:
         _check(self.lib.kvq_decode_step(self.handle, layer, k.data_ptr(), v.data_ptr(), q.data_ptr(), out.data_ptr(),
                                         _DTYPE_CODE[out.dtype], float(softmax_scale), q.shape[0], _stream_ptr(stream)),
                "kvq_decode_step")
+        return out
+
+    def decode_attention_multi(self, layer: int, q: torch.Tensor, out_dtype=torch.float32,
+                               softmax_scale: float | None = None, stream=None):
+        """Several query tokens per sequence (q: [batch, T, Hq, D]), causal over
+        the sequences' T newest tokens (kvq_decode_attention_multi). Returns
+        out [batch, T, Hq, D]."""
+        _need(q, self.cfg.kv_dtype, "q")
+        out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        if softmax_scale is None:
+            softmax_scale = self.cfg.head_dim ** -0.5
+        _check(self.lib.kvq_decode_attention_multi(self.handle, layer, q.data_ptr(), out.data_ptr(),
+                                                   _DTYPE_CODE[out.dtype], float(softmax_scale), q.shape[0],
+                                                   q.shape[1], _stream_ptr(stream)),
+               "kvq_decode_attention_multi")
         return out
 
     def decode_attention_noalloc(self, layer: int, q: torch.Tensor, out: torch.Tensor,

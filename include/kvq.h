@@ -221,6 +221,21 @@ KVQ_API kvq_status kvq_decode_attention(kvq_cache* cache, int32_t layer, const v
  * 16 MiB, held on every GPU that loads the library until the process exits. */
 #define KVQ_STATIC_SCRATCH_BYTES (16u << 20)
 
+/* Decode attention of num_tokens query tokens per sequence (verifying
+ * drafted tokens in one pass). q: device [batch][num_tokens][Hq][D] in
+ * kv_dtype; out: device [batch][num_tokens][Hq][D] in out_dtype. The query
+ * tokens' keys and values must already be the sequence's num_tokens newest
+ * cached tokens (kvq_append first): query token t, at position L - T + t,
+ * attends to tokens 0 .. L - T + t (causal among the T). Those tokens must
+ * still be in the ring: a sequence with fewer than num_tokens ring tokens is
+ * refused with KVQ_ERR_UNSUPPORTED before anything is enqueued;
+ * 1 <= num_tokens <= residual. num_tokens = 1 is kvq_decode_attention.
+ * Runs as ceil(num_tokens * Hq / Hkv / 8) or a few more decode passes over
+ * the cache (at most 8 query rows per KV head per pass).                   */
+KVQ_API kvq_status kvq_decode_attention_multi(kvq_cache* cache, int32_t layer, const void* q, void* out,
+                                              int32_t out_dtype, float softmax_scale, int32_t batch,
+                                              int32_t num_tokens, void* stream);
+
 /* Same result as kvq_decode_attention, for callers that cannot allocate
  * device memory at the point of the call, for example an engine whose device
  * memory is all handed to its own pool at start-up, or code running under a
