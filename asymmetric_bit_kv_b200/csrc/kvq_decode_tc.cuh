@@ -1,6 +1,6 @@
 // Tensor-core split-KV decode attention over the packed cache (sm_100a):
 // the kernel template, instantiated per (key bits, value bits, value groups
-// per head, key n-tiles) in kvq_decode_tc_k{2,4,8}.cu.
+// per head, key n-tiles, key axis) in kvq_decode_tc_k{2,4,8}_n{1,2}.cu.
 //
 // Method: decoding over per-channel-quantized keys and per-token-quantized
 // values plus the full-precision residual window ("KIVI" README, Overview;
@@ -37,6 +37,13 @@
 //  * Every warp writes one partial (o, m, l) per unit it passes through; the
 //    log-sum-exp combine kernel merges them. mbarrier waits are bounded
 //    (~2 s) and set the device error word instead of hanging.
+//  * Keys quantized per token (KV1 BQ2_0, the PT instances): the same code
+//    layout and A operand, the unit's (rotated) query as B, the token scales
+//    on the score rows; see unit_query / unrotate_output.
+//  * A unit's query rows may span several query tokens (verifying drafted
+//    tokens): ring chunks hide from each its later tokens (DecodeParams).
+//  * Paged caches: the issuing lane reads a unit's page once per run of
+//    page_blocks blocks.
 #pragma once
 
 #include "kvq_decode.cuh"

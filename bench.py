@@ -51,6 +51,8 @@ def _args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="llama3", choices=["llama3", "kv1"],
                     help="llama3: the headline KIVI layer (default); kv1: the same shapes with the KV1 card's BQ2_0 cache")
+    ap.add_argument("--query-tokens", type=int, default=1,
+                    help="query tokens per sequence and step (> 1: append them, then kvq_decode_attention_multi)")
     ap.add_argument("--page-blocks", type=int, default=0,
                     help="block records in pages of this many blocks drawn from a pool (0: contiguous)")
     return ap.parse_args()
@@ -287,6 +289,7 @@ def run_kvq(a):
     import torch.distributed as dist
 
     from asymmetric_bit_kv_b200 import CacheConfig, KVCache
+    from asymmetric_bit_kv_b200 import kvq as K
     from asymmetric_bit_kv_b200 import workloads as W
 
     rank, world, local = _dist_env()
@@ -317,10 +320,11 @@ def run_kvq(a):
     torch.cuda.synchronize()
     gen = torch.Generator(device=dev).manual_seed(12345 + rank)
     pool = 64  # distinct per-step inputs, reused round-robin
-    new_k = torch.randn(pool, B, Hkv, D, generator=gen, device=dev).to(wl.kv_dtype)
-    new_v = torch.randn(pool, B, Hkv, D, generator=gen, device=dev).to(wl.kv_dtype)
-    qs = torch.randn(pool, B, Hq, D, generator=gen, device=dev).to(wl.kv_dtype)
-    out = torch.empty(B, Hq, D, dtype=wl.kv_dtype, device=dev)
+    T = a.query_tokens  # query tokens per sequence and step (their keys and values are appended first)
+    new_k = torch.randn(pool, B * T, Hkv, D, generator=gen, device=dev).to(wl.kv_dtype)
+    new_v = torch.randn(pool, B * T, Hkv, D, generator=gen, device=dev).to(wl.kv_dtype)
+    qs = torch.randn(pool, B * T, Hq, D, generator=gen, device=dev).to(wl.kv_dtype)
+    out = torch.empty(B * T, Hq, D, dtype=wl.kv_dtype, device=dev)
     stream = torch.cuda.current_stream()
     # per-step inputs as views made once, so that the timed loop only enqueues
     views = [(new_k[j], new_v[j], qs[j]) for j in range(pool)]
@@ -337,6 +341,8 @@ def run_kvq(a):
     # step; the e2e leg below goes through the Python binding.
     lib = caches[0].lib
     c_step = lib.kvq_decode_step
+    c_append, c_multi = lib.kvq_append, lib.kvq_decode_attention_multi
+    t_lens = K.lens_array([T] * B)
     sh = stream.cuda_stream
     handles = [c.handle for c in caches]
     ptrs = [(kk.data_ptr(), vv.data_ptr(), qq.data_ptr()) for kk, vv, qq in views]
@@ -347,7 +353,10 @@ def run_kvq(a):
         h = handles[r]
         if ev is not None:
             ev[0].record(stream)
-        st = c_step(h, 0, kp, vp, qp, optr, oty, scale, B, sh)
+        if T == 1:
+            st = c_step(h, 0, kp, vp, qp, optr, oty, scale, B, sh)
+        else:  # the T tokens' keys and values, then the T queries of every sequence
+            st = c_append(h, 0, kp, vp, t_lens, B, sh) or c_multi(h, 0, qp, optr, oty, scale, B, T, sh)
         if ev is not None:
             ev[1].record(stream)
         if st:
@@ -370,19 +379,33 @@ def run_kvq(a):
         # fused: decode + combine; a step that flushes a ring first runs the
         # quantize and ring-write kernels (unfused: ring write, split kernel,
         # combine, and the quantize kernel on a flush)
-        flush = lens[r][0][1] == Rw
-        launches = (2 + (2 if flush else 0)) if fused else (3 + (1 if flush else 0))
-        ab, tk = 2 * B * Hq * D * 2 + 2 * (2 * B * Hkv * D * 2), 0  # q in, out; new k, v in and into the ring
+        ab, tk = T * (2 * B * Hq * D * 2 + 2 * (2 * B * Hkv * D * 2)), 0  # q in, out; new k, v in and into the ring
         ab += B * sinks * Hkv * D * 2 * 2  # the exact sink tokens
-        tk += B * sinks
+        tk += B * T * sinks
+        flush = False
         for b in range(B):
             qn, n = lens[r][b]
-            if n == Rw:
-                qn, n = qn + G, n - G
-            n += 1
+            f = 0 if n + T <= Rw else -(-(n + T - Rw) // G)  # blocks the T appends flush
+            flush = flush or f > 0
+            qn, n = qn + f * G, n + T - f * G
             lens[r][b] = [qn, n]
             ab += qn * bytes_tok + n * Hkv * D * 2 * 2
-            tk += qn + n
+            tk += T * (qn + n) - T * (T - 1) // 2  # query t sees the tokens up to its own position
+        if T == 1:
+            # fused: decode + combine; a step that flushes a ring first runs the
+            # quantize and ring-write kernels (unfused: ring write, split
+            # kernel, combine, and the quantize kernel on a flush)
+            launches = (2 + (2 if flush else 0)) if fused else (3 + (1 if flush else 0))
+        else:
+            # append (ring write, + quantize on a flush), then decode + combine
+            # per group of query tokens (at most 8 query rows per KV head)
+            groups, t0, ngr = 0, 0, Hq // Hkv
+            while t0 < T:
+                tp = 1
+                while 2 * tp * ngr <= 8 and t0 + 2 * tp <= T:
+                    tp *= 2
+                groups, t0 = groups + 1, t0 + tp
+            launches = 1 + (1 if flush else 0) + 2 * groups
         plan.append((r, launches, ab, tk))
     events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
     launches = sum(x[1] for x in plan)
@@ -419,25 +442,25 @@ def run_kvq(a):
     # each step's k, v and q sit back to back in one pinned host buffer and
     # travel in one host-to-device copy
     e2e_steps = min(a.steps, 512)
-    nk, nq = B * Hkv * D, B * Hq * D
+    nk, nq = B * T * Hkv * D, B * T * Hq * D
     hkvq = torch.empty(pool, 2 * nk + nq, dtype=wl.kv_dtype).pin_memory()
     hkvq[:, :nk].copy_(new_k.reshape(pool, nk).cpu())
     hkvq[:, nk:2 * nk].copy_(new_v.reshape(pool, nk).cpu())
     hkvq[:, 2 * nk:].copy_(qs.reshape(pool, nq).cpu())
-    hout = torch.empty(B, Hq, D, dtype=wl.kv_dtype).pin_memory()
+    hout = torch.empty(B * T, Hq, D, dtype=wl.kv_dtype).pin_memory()
     dkvq = torch.empty(2 * nk + nq, dtype=wl.kv_dtype, device=dev)
-    dk = dkvq[:nk].view(B, Hkv, D)
-    dv = dkvq[nk:2 * nk].view(B, Hkv, D)
-    dq = dkvq[2 * nk:].view(B, Hq, D)
+    dk = dkvq[:nk].view(B * T, Hkv, D)
+    dv = dkvq[nk:2 * nk].view(B * T, Hkv, D)
+    dq = dkvq[2 * nk:].view(B * T, Hq, D)
     tok_e2e = 0
     for i in range(e2e_steps):
         r = (a.warmup + a.steps + i) % R
         for b in range(B):
             qn, n = lens[r][b]
-            if n == Rw:
-                qn, n = qn + G, n - G
-            lens[r][b] = [qn, n + 1]
-            tok_e2e += sinks + qn + n + 1
+            f = 0 if n + T <= Rw else -(-(n + T - Rw) // G)
+            qn, n = qn + f * G, n + T - f * G
+            lens[r][b] = [qn, n]
+            tok_e2e += T * (sinks + qn + n) - T * (T - 1) // 2
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -447,8 +470,14 @@ def run_kvq(a):
         r = (a.warmup + a.steps + i) % R
         j = i % pool
         dkvq.copy_(hkvq[j], non_blocking=True)
-        caches[r].decode_step(0, dk, dv, dq, out, softmax_scale=wl.softmax_scale, stream=stream)
-        hout.copy_(out, non_blocking=True)
+        if T == 1:
+            caches[r].decode_step(0, dk, dv, dq, out, softmax_scale=wl.softmax_scale, stream=stream)
+            hout.copy_(out, non_blocking=True)
+        else:
+            caches[r].append(0, dk, dv, [T] * B, stream=stream)
+            o = caches[r].decode_attention_multi(0, dq.view(B, T, Hq, D), out_dtype=wl.kv_dtype,
+                                                 softmax_scale=wl.softmax_scale, stream=stream)
+            hout.copy_(o.view(B * T, Hq, D), non_blocking=True)
     f1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = f0.elapsed_time(f1)
@@ -472,10 +501,14 @@ def run_kvq(a):
             "vs_baseline": None,
             "dtype": "f32",
             "data": "synthetic (seeded; Llama-3-8B-shaped layer, no model weights)",
-            "config": dict(_workload_config(wl, R, world, tok_total / (a.steps * B)),
-                           **({"page_blocks": a.page_blocks} if a.page_blocks else {})),
+            "config": dict(_workload_config(wl, R, world, tok_total / (a.steps * B * T)),
+                           **({"page_blocks": a.page_blocks} if a.page_blocks else {}),
+                           **({"query_tokens": T} if T > 1 else {})),
             "roofline": {
-                "kernel": ("decode step: one token appended per sequence inside the split-KV decode kernel, + log-sum-exp "
+                "kernel": (f"verify step: {T} tokens appended per sequence (ring write, quantize on a flush), then "
+                           "decode of their queries, causal among them (split-KV decode + combine per group of query "
+                           "tokens)") if T > 1 else
+                          ("decode step: one token appended per sequence inside the split-KV decode kernel, + log-sum-exp "
                            "combine, per call (a ring flush adds the quantize and ring kernels)") if fused else
                           ("decode step: ring write, CUDA-core split-KV decode kernel and log-sum-exp combine, per call "
                            "(a ring flush adds the quantize kernel)"),
@@ -585,7 +618,7 @@ def main():
         return
     rank, world, _ = _dist_env()
     cpu = None
-    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+    if rank == 0 and world == 1 and not a.no_cpu_baseline and a.query_tokens == 1:
         cpu = cpu_oracle_baseline(wname=a.workload)   # spawned before any CUDA work in this process
     res = run_kvq(a)
     if res is not None:
