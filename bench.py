@@ -306,7 +306,7 @@ def run_kvq(a):
     ctx = wl.context[0]
     R = a.replicas
     steps_per_rep = math.ceil((a.warmup + 2 * a.steps) / R) + 2
-    cap = ctx + steps_per_rep + wl.group_k
+    cap = ctx + steps_per_rep * a.query_tokens + wl.group_k
     cfg = CacheConfig(1, B, Hq, Hkv, D, cap, wl.group_k, wl.group_v, wl.residual, wl.kv_dtype, wl.k_bits, wl.v_bits,
                       sink_tokens=sinks, k_axis=[k_axis], hadamard=rot, page_blocks=a.page_blocks,
                       pool_pages=B * -(-(cap // wl.group_k) // a.page_blocks) if a.page_blocks else 0)
