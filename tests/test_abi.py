@@ -91,3 +91,24 @@ def test_create_rejects_bad_arena_on_host():
     assert b"required" in lib.kvq_last_error()
     assert lib.kvq_append(None, 0, None, None, None, 0, None) == K.KVQ_ERR_INVALID_ARG
     assert lib.kvq_decode_attention(None, 0, None, None, 0, 1.0, 1, None) == K.KVQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kb,vb,G,Gv,k_axis", [
+    (2, 4, 64, 64, 0), (2, 2, 32, 32, 0), (4, 2, 128, 64, 0), (8, 8, 64, 128, 0),
+    (2, 2, 64, 128, 1), (4, 4, 32, 64, 1), (8, 2, 128, 32, 1),
+])
+def test_block_record_bytes_match_the_closed_form(kb, vb, G, Gv, k_axis):
+    # one more run of 16 blocks per sequence grows the arena by exactly that
+    # many block records per (sequence, KV head, layer); a record holds G
+    # tokens at the closed-form bytes per token (KV1 card, Memory: codes plus
+    # an fp16 scale and zero point per group)
+    def cfg(max_tokens, **kw):
+        return CacheConfig(2, 3, 8, 2, 128, max_tokens, G, Gv, 128, torch.bfloat16, [kb] * 2, [vb] * 2,
+                           k_axis=[k_axis] * 2, **kw)
+    m = 200 * G  # large enough that the split workspace no longer grows
+    grow = required_bytes(cfg(m + 16 * G)) - required_bytes(cfg(m))
+    per_head_token = O.quantized_bytes_per_token(1, 128, kb, vb, G, Gv, k_axis=k_axis)
+    assert grow == 2 * 3 * 2 * 16 * G * per_head_token
+    # a paged layer: one more page of 4 blocks per layer, for every KV head
+    paged = [required_bytes(cfg(m, page_blocks=4, pool_pages=p)) for p in (10, 11)]
+    assert paged[1] - paged[0] == 2 * 2 * 4 * G * per_head_token
