@@ -231,7 +231,10 @@ KVQ_API kvq_status kvq_decode_attention(kvq_cache* cache, int32_t layer, const v
  * refused with KVQ_ERR_UNSUPPORTED before anything is enqueued;
  * 1 <= num_tokens <= residual. num_tokens = 1 is kvq_decode_attention.
  * Runs as ceil(num_tokens * Hq / Hkv / 8) or a few more decode passes over
- * the cache (at most 8 query rows per KV head per pass).                   */
+ * the cache (at most 8 query rows per KV head per pass); a launch failure in
+ * a later pass leaves the earlier passes' rows of out written. The pages do
+ * not describe several query tokens per sequence: this is the plainest
+ * extension of their decoding rule (causal, like prefill).                 */
 KVQ_API kvq_status kvq_decode_attention_multi(kvq_cache* cache, int32_t layer, const void* q, void* out,
                                               int32_t out_dtype, float softmax_scale, int32_t batch,
                                               int32_t num_tokens, void* stream);
