@@ -249,7 +249,20 @@ def cpu_oracle_baseline(steps: int = 100, warmup: int = 2, wname: str = "llama3"
             secs += s
     finally:
         run.close()
-    return {"value": toks / secs, "unit": UNIT, "cores": workers, "kind": "oracle", "sample": run.describe(steps)}
+    res = {"value": toks / secs, "unit": UNIT, "cores": workers, "kind": "oracle", "sample": run.describe(steps)}
+    # the same unit work on one core alone (a few steps)
+    one = OracleRunner(1, wname=wname)
+    try:
+        one.step()
+        toks1, secs1 = 0, 0.0
+        for _ in range(max(3, steps // 10)):
+            t, s = one.step()
+            toks1 += t
+            secs1 += s
+    finally:
+        one.close()
+    res["value_1_core"] = toks1 / secs1
+    return res
 
 
 # --------------------------------------------------------------------------
