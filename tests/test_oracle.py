@@ -564,3 +564,25 @@ def test_multi_query_single_token_is_decode_and_sinks_stay_visible():
     o = O.decode_attention_multi(c, np.zeros((3, 4, 16)), 0.2)
     for t in range(3):
         assert np.allclose(o[t, 0], V[:90 - 3 + t + 1, 0].mean(0), atol=1e-12)
+
+
+def test_multi_query_prefixes_with_sinks_and_rotation():
+    # the prefix property on the KV1 layout: per-token keys, rotation, sinks
+    rng = np.random.default_rng(21)
+    L, T, H = 4 + 96 + 40, 3, 2   # 4 sinks, 3 blocks of 32, ring of 40 (R 64, G 32)
+    k = rng.standard_normal((L, H, 16)).astype(np.float16).astype(np.float32)
+    v = rng.standard_normal((L, H, 16)).astype(np.float16).astype(np.float32)
+
+    def cache(n):
+        c = O.SequenceCache(H, 16, 2, 2, 32, 16, 64, sinks=4, k_axis=1, hadamard=True)
+        c.append(k[:n], v[:n])
+        return c
+
+    full = cache(L)
+    assert full.sink_tokens == 4 and full.quantized_tokens == 96 and full.residual_tokens == 40
+    q = rng.standard_normal((T, 4, 16))
+    o = O.decode_attention_multi(full, q, 0.25)
+    for t in range(T):
+        part = cache(L - T + t + 1)
+        assert part.quantized_tokens == full.quantized_tokens
+        assert np.array_equal(o[t], O.decode_attention(part, q[t], 0.25))
