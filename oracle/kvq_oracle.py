@@ -67,6 +67,16 @@ the design notes of the repository):
    and query t, at position L - T + t, attends causally to the tokens up to
    its own position. T = 1 is reading 5.
 
+9. Separate residual lengths for keys and values ("Quantize What Counts",
+   KV Cache Quantization: ``residual_length`` and ``group_size`` are given
+   per tensor): each tensor keeps its own ring -- ``residual`` keys and
+   ``residual_v`` values -- and applies reading 4 on its own, flushing its
+   oldest ``group_k`` tokens when its ring is full. A token's key and value
+   may then be one quantized and one exact. Values are flushed in blocks of
+   ``group_k`` tokens too (their groups run along channels, so any block
+   length would do; this one keeps the blocks of both tensors aligned). Equal
+   lengths give exactly the single-window cache.
+
 Floating point: the quantizer runs in IEEE fp32 (the precision the KV1 card
 fixes); numpy evaluates each fp32 operation with one rounding and never
 contracts a multiply-add. Attention runs in fp64.
@@ -255,30 +265,61 @@ class SequenceCache:
     """KV cache of one sequence in one layer.
 
     Token values are fp32 arrays holding values exactly representable in the
-    cache's storage type (fp16 or bf16); the ring keeps them unchanged.
+    cache's storage type (fp16 or bf16); the rings keep them unchanged.
+
+    Keys and values each keep their own residual window ("Quantize What
+    Counts", KV Cache Quantization: ``residual_length`` given per tensor as
+    ``{"k": ..., "v": ...}``): ``residual`` recent keys and ``residual_v``
+    recent values (default: the same length) stay exact, and each tensor
+    flushes its own oldest ``group_k`` tokens when its ring is full (reading
+    4 applied to each tensor on its own). With equal lengths both flush
+    together, on the same tokens.
     """
 
     def __init__(self, num_kv_heads, head_dim, k_bits, v_bits, group_k, group_v, residual, sinks=0, k_axis=0,
-                 hadamard=False):
-        assert residual % group_k == 0 and residual >= group_k and sinks >= 0 and k_axis in (0, 1)
+                 hadamard=False, residual_v=None):
+        residual_v = residual if residual_v is None else residual_v
+        for r in (residual, residual_v):
+            assert r % group_k == 0 and r >= group_k
+        assert sinks >= 0 and k_axis in (0, 1)
         self.H, self.D = num_kv_heads, head_dim
         self.k_bits, self.v_bits = k_bits, v_bits
         self.group_k, self.group_v, self.residual = group_k, group_v, residual
+        self.residual_v = residual_v
         self.sinks = sinks
         self.k_axis, self.hadamard = k_axis, bool(hadamard)
         self.sink_k: list[np.ndarray] = []  # the first `sinks` tokens, exact, each [H, D]
         self.sink_v: list[np.ndarray] = []
-        self.blocks: list[QuantizedBlock] = []
+        self.key_blocks: list[tuple] = []    # (codes [G, H, D], scale, zero) per flushed key block
+        self.value_blocks: list[tuple] = []  # (codes [G, H, D], scale [G, H, groups], zero) per value block
         self.ring_k: list[np.ndarray] = []   # oldest first, each [H, D]
         self.ring_v: list[np.ndarray] = []
 
     @property
+    def blocks(self) -> list:
+        """Blocks whose keys and values are both quantized, as QuantizedBlock
+        (every block when the two residual lengths are equal)."""
+        return [QuantizedBlock(*kb, *vb) for kb, vb in zip(self.key_blocks, self.value_blocks)]
+
+    @property
     def quantized_tokens(self) -> int:
-        return len(self.blocks) * self.group_k
+        """Quantized keys (after the sinks)."""
+        return len(self.key_blocks) * self.group_k
+
+    @property
+    def quantized_tokens_v(self) -> int:
+        """Quantized values (after the sinks)."""
+        return len(self.value_blocks) * self.group_k
 
     @property
     def residual_tokens(self) -> int:
+        """Exact keys in the key ring."""
         return len(self.ring_k)
+
+    @property
+    def residual_tokens_v(self) -> int:
+        """Exact values in the value ring."""
+        return len(self.ring_v)
 
     @property
     def sink_tokens(self) -> int:
@@ -288,30 +329,37 @@ class SequenceCache:
     def length(self) -> int:
         return self.sink_tokens + self.quantized_tokens + self.residual_tokens
 
-    def _flush_oldest_block(self):
+    def _flush_keys(self):
         G = self.group_k
         k = np.stack(self.ring_k[:G]).astype(F32)
-        v = np.stack(self.ring_v[:G]).astype(F32)
         del self.ring_k[:G]
+        if self.hadamard:
+            k = rotate_fp32(k)
+        if self.k_axis == 1:  # per-token keys, grouped like values
+            self.key_blocks.append(quantize_value_block(k, self.k_bits, self.group_v))
+        else:
+            self.key_blocks.append(quantize_key_block(k, self.k_bits))
+
+    def _flush_values(self):
+        G = self.group_k
+        v = np.stack(self.ring_v[:G]).astype(F32)
         del self.ring_v[:G]
         if self.hadamard:
-            k, v = rotate_fp32(k), rotate_fp32(v)
-        if self.k_axis == 1:  # per-token keys, grouped like values
-            kc, kd, km = quantize_value_block(k, self.k_bits, self.group_v)
-        else:
-            kc, kd, km = quantize_key_block(k, self.k_bits)
-        vc, vd, vm = quantize_value_block(v, self.v_bits, self.group_v)
-        self.blocks.append(QuantizedBlock(kc, kd, km, vc, vd, vm))
+            v = rotate_fp32(v)
+        self.value_blocks.append(quantize_value_block(v, self.v_bits, self.group_v))
 
     def append_token(self, k: np.ndarray, v: np.ndarray):
         """Append one token ([H, D] each): one of the first `sinks` tokens is
-        kept as it is; otherwise a full ring first flushes G tokens."""
+        kept as it is; otherwise a full key ring first flushes its oldest G
+        keys, and a full value ring its oldest G values."""
         if len(self.sink_k) < self.sinks:
             self.sink_k.append(np.asarray(k, dtype=F32).copy())
             self.sink_v.append(np.asarray(v, dtype=F32).copy())
             return
         if len(self.ring_k) == self.residual:
-            self._flush_oldest_block()
+            self._flush_keys()
+        if len(self.ring_v) == self.residual_v:
+            self._flush_values()
         self.ring_k.append(np.asarray(k, dtype=F32).copy())
         self.ring_v.append(np.asarray(v, dtype=F32).copy())
 
@@ -321,32 +369,35 @@ class SequenceCache:
             self.append_token(k[t], v[t])
 
     def flush_residual(self):
-        """Quantize every complete block of group_k tokens left in the ring."""
+        """Quantize every complete block of group_k tokens left in either ring."""
         while len(self.ring_k) >= self.group_k:
-            self._flush_oldest_block()
+            self._flush_keys()
+        while len(self.ring_v) >= self.group_k:
+            self._flush_values()
 
     def dequantized(self, effective=False):
         """(K~, V~) as fp32 [L, H, D] in token order: the exact sinks, the
         dequantized blocks (as stored: in the rotated basis for a Hadamard
-        cache), then the ring. effective=True: fp64, with the blocks rotated
-        back (. H), the keys and values attention sees."""
+        cache), then the ring; keys and values each with their own quantized
+        and exact parts. effective=True: fp64, with the blocks rotated back
+        (. H), the keys and values attention sees."""
         ks, vs = [], []
         if self.sink_k:
             ks.append(np.stack(self.sink_k))
             vs.append(np.stack(self.sink_v))
         Hm = sylvester(self.D) if (effective and self.hadamard) else None
-        for b in self.blocks:
+        for kc, kd, km in self.key_blocks:
             if self.k_axis == 1:
-                kq = dequantize_value_block(b.kc, b.kd, b.km)
+                kq = dequantize_value_block(kc, kd, km)
             else:
-                kq = dequantize_key_block(b.kc, b.kd, b.km)
-            vq = dequantize_value_block(b.vc, b.vd, b.vm)
-            if Hm is not None:
-                kq, vq = kq.astype(np.float64) @ Hm, vq.astype(np.float64) @ Hm
-            ks.append(kq)
-            vs.append(vq)
+                kq = dequantize_key_block(kc, kd, km)
+            ks.append(kq.astype(np.float64) @ Hm if Hm is not None else kq)
+        for vc, vd, vm in self.value_blocks:
+            vq = dequantize_value_block(vc, vd, vm)
+            vs.append(vq.astype(np.float64) @ Hm if Hm is not None else vq)
         if self.ring_k:
             ks.append(np.stack(self.ring_k))
+        if self.ring_v:
             vs.append(np.stack(self.ring_v))
         dt = np.float64 if effective else F32
         if not ks:

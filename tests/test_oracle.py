@@ -266,6 +266,124 @@ def test_flush_residual():
 
 
 # --------------------------------------------------------------------------
+# Separate residual lengths for keys and values ("Quantize What Counts", KV
+# Cache Quantization: residual_length {"k", "v"}); reading 9 of the oracle
+# --------------------------------------------------------------------------
+
+
+def _single_window_counts(L, R, G):
+    """(quantized, exact) tokens of one tensor after L single-token appends
+    to a ring of R slots that flushes G tokens when full, in closed form."""
+    if L <= R:
+        return 0, L
+    n = R - G + 1 + (L - R - 1) % G
+    return L - n, n
+
+
+@pytest.mark.parametrize("Rk,Rv,G,S", [(64, 128, 32, 0), (128, 64, 32, 0), (32, 96, 32, 2), (128, 256, 64, 0),
+                                       (256, 128, 128, 1), (64, 64, 32, 0)])
+def test_split_residual_counts_closed_form(Rk, Rv, G, S):
+    H, D = 1, 16
+    c = O.SequenceCache(H, D, 2, 2, G, 16, Rk, sinks=S, residual_v=Rv)
+    rng = np.random.default_rng(Rk + 3 * Rv + G)
+    for L in range(1, 3 * max(Rk, Rv) + G + 3):
+        c.append_token(rng.standard_normal((H, D)), rng.standard_normal((H, D)))
+        s = min(L, S)
+        assert c.sink_tokens == s
+        assert (c.quantized_tokens, c.residual_tokens) == _single_window_counts(L - s, Rk, G), L
+        assert (c.quantized_tokens_v, c.residual_tokens_v) == _single_window_counts(L - s, Rv, G), L
+        assert c.length == L
+
+
+def test_single_window_closed_form_agrees_with_the_table():
+    # the closed form above and the ceil form of the single-window test are one rule
+    for R, G in [(32, 32), (128, 32), (128, 64), (96, 32)]:
+        for L in range(1, 4 * R):
+            assert _single_window_counts(L, R, G) == _expected_split(L, R, G), (L, R, G)
+
+
+def _tensor_state(c, key):
+    if key:
+        return c.key_blocks, c.ring_k
+    return c.value_blocks, c.ring_v
+
+
+def _same_tensor(a, b, key):
+    ba, ra = _tensor_state(a, key)
+    bb, rb = _tensor_state(b, key)
+    if len(ba) != len(bb) or len(ra) != len(rb):
+        return False
+    for x, y in zip(ba, bb):
+        if not all(np.array_equal(np.asarray(u).view(np.uint8), np.asarray(w).view(np.uint8)) for u, w in zip(x, y)):
+            return False
+    return all(np.array_equal(u, w) for u, w in zip(ra, rb))
+
+
+@pytest.mark.parametrize("k_axis,rot", [(0, False), (1, True)])
+def test_split_residual_tensors_equal_single_window_caches(k_axis, rot):
+    # keys depend only on the key window and values only on the value window:
+    # a (Rk, Rv) cache holds the keys of an (Rk, Rk) cache and the values of
+    # an (Rv, Rv) cache, bit for bit, after appends and after flush_residual
+    H, D, G, Rk, Rv, gv = 2, 32, 32, 64, 160, 32 if k_axis == 0 else 32
+    rng = np.random.default_rng(31 + k_axis)
+    L = 7 * G + 13
+    k = rng.standard_normal((L, H, D)).astype(np.float32) * np.exp(rng.standard_normal(D)).astype(np.float32)
+    v = rng.standard_normal((L, H, D)).astype(np.float32)
+    mk = lambda r, rv: O.SequenceCache(H, D, 2, 4, G, gv, r, sinks=1, k_axis=k_axis, hadamard=rot, residual_v=rv)
+    split, kref, vref = mk(Rk, Rv), mk(Rk, Rk), mk(Rv, Rv)
+    pos = 0
+    for n in [1, 40, 3, 97, 1, 1, 80, L - 223]:
+        for c in (split, kref, vref):
+            c.append(k[pos:pos + n], v[pos:pos + n])
+        pos += n
+        assert _same_tensor(split, kref, True) and _same_tensor(split, vref, False), pos
+    assert pos == L
+    assert split.quantized_tokens != split.quantized_tokens_v  # the windows really differ here
+    for c in (split, kref, vref):
+        c.flush_residual()
+    assert _same_tensor(split, kref, True) and _same_tensor(split, vref, False)
+    assert split.residual_tokens == split.residual_tokens_v == (L - 1) % G
+
+
+def test_split_residual_exact_tokens_are_the_appended_ones():
+    # token i's key is exact iff i >= sinks + quantized keys, its value iff
+    # i >= sinks + quantized values; the exact ones are the appended values
+    H, D, G, Rk, Rv, S = 2, 32, 32, 128, 64, 2
+    rng = np.random.default_rng(41)
+    L = S + 6 * G + 5
+    k = rng.standard_normal((L, H, D)).astype(np.float32)
+    v = rng.standard_normal((L, H, D)).astype(np.float32)
+    c = O.SequenceCache(H, D, 2, 2, G, 32, Rk, sinks=S, residual_v=Rv)
+    c.append(k, v)
+    K, V = c.dequantized()
+    qk, qv = S + c.quantized_tokens, S + c.quantized_tokens_v
+    assert qk < qv
+    assert np.array_equal(K[:S], k[:S]) and np.array_equal(V[:S], v[:S])
+    assert np.array_equal(K[qk:], k[qk:]) and np.array_equal(V[qv:], v[qv:])
+    # a quantized 2-bit token is never exact for N(0,1) data
+    assert np.all(np.any(K[S:qk] != k[S:qk], axis=(1, 2))) and np.all(np.any(V[S:qv] != v[S:qv], axis=(1, 2)))
+
+
+def test_split_residual_attention_matches_sdpa_on_mixed_cache():
+    # the attention of a split cache is textbook attention over the keys of
+    # the (Rk, Rk) cache and the values of the (Rv, Rv) cache
+    H, Hq, D, G, Rk, Rv = 2, 8, 32, 32, 96, 32
+    rng = np.random.default_rng(43)
+    L = 9 * G + 21
+    k = rng.standard_normal((L, H, D)).astype(np.float32)
+    v = rng.standard_normal((L, H, D)).astype(np.float32)
+    split = O.SequenceCache(H, D, 2, 4, G, 32, Rk, residual_v=Rv)
+    kref = O.SequenceCache(H, D, 2, 4, G, 32, Rk)
+    vref = O.SequenceCache(H, D, 2, 4, G, 32, Rv)
+    for c in (split, kref, vref):
+        c.append(k, v)
+    Kk, _ = kref.dequantized()
+    _, Vv = vref.dequantized()
+    q = rng.standard_normal((Hq, D))
+    assert np.abs(O.decode_attention(split, q, D ** -0.5) - _sdpa(q, Kk, Vv, D ** -0.5)).max() < 1e-12
+
+
+# --------------------------------------------------------------------------
 # Attention: hand example, closed forms, and an independent library routine
 # --------------------------------------------------------------------------
 
