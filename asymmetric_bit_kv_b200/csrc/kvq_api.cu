@@ -25,13 +25,15 @@ struct kvq_cache {
   // per layer
   std::vector<int64_t> blocks_off, ring_k_off, ring_v_off, sink_k_off, sink_v_off, record_bytes;
   int64_t max_blocks;
-  int64_t lens_off;               // int32 [num_layers][max_batch][3]
+  int64_t lens_off;               // int32 [num_layers][max_batch][kLensStride]
   int64_t ws_o_off, ws_ml_off;    // split partials
   int64_t err_off;                // int32 device error word
   int64_t uslots_off;             // int32 [max_batch][num_kv_heads] slots per unit (decode -> combine)
   int32_t slots;                  // partial slots per (sequence, query head)
   int32_t sm_count;
-  std::vector<int32_t> q_len, n_len, s_len;  // host mirror [num_layers][max_batch]
+  // host mirror [num_layers][max_batch]: quantized keys, key ring tokens,
+  // sinks, quantized values (the value ring holds q_len + n_len - qv_len)
+  std::vector<int32_t> q_len, n_len, s_len, qv_len;
   // paged block pools (cfg.page_blocks >= 1)
   std::vector<int64_t> pt_off;                   // per layer: int32 page table [max_batch][max_pages]
   int32_t max_pages = 0;                         // page-table entries per sequence
@@ -81,6 +83,11 @@ kvq_status validate_config(const kvq_config* c) {
   if (c->residual < c->group_k || c->residual % c->group_k != 0)
     return fail(KVQ_ERR_INVALID_ARG, "residual %d must be a positive multiple of group_k %d", c->residual,
                 c->group_k);
+  if (c->residual_v != 0 && (c->residual_v < c->group_k || c->residual_v % c->group_k != 0))
+    return fail(KVQ_ERR_INVALID_ARG, "residual_v %d must be 0 or a positive multiple of group_k %d", c->residual_v,
+                c->group_k);
+  if (c->residual_v != 0 && c->residual_v != c->residual && c->hadamard)
+    return fail(KVQ_ERR_UNSUPPORTED, "separate key and value residual lengths with the Hadamard rotation");
   if (c->max_tokens < 1) return fail(KVQ_ERR_INVALID_ARG, "max_tokens %d < 1", c->max_tokens);
   if (c->sink_tokens < 0 || c->sink_tokens > KVQ_MAX_SINKS)
     return fail(KVQ_ERR_INVALID_ARG, "sink_tokens %d outside 0..%d", c->sink_tokens, KVQ_MAX_SINKS);
@@ -102,8 +109,14 @@ kvq_status validate_config(const kvq_config* c) {
     if ((int64_t)c->pool_pages * c->num_kv_heads * c->page_blocks > INT32_MAX)
       return fail(KVQ_ERR_UNSUPPORTED, "more than 2^31 block records in one layer's pool");
   }
+  // the work items of one decode launch are counted in int32
+  const int64_t items = (int64_t)c->max_batch * c->num_kv_heads *
+                        ((int64_t)c->max_tokens / c->group_k + std::max(c->residual, c->residual_v) / 8 + 2);
+  if (items > INT32_MAX / 2) return fail(KVQ_ERR_UNSUPPORTED, "max_batch x num_kv_heads x max_tokens too large");
   return KVQ_OK;
 }
+
+int residual_v_of(const kvq_config& c) { return c.residual_v > 0 ? c.residual_v : c.residual; }
 
 struct Plan {
   std::vector<int64_t> blocks_off, ring_k_off, ring_v_off, sink_k_off, sink_v_off, record_bytes, pt_off;
@@ -132,11 +145,10 @@ Plan make_plan(const kvq_config* c) {
     p.record_bytes.push_back(rec);
     p.blocks_off.push_back(off);
     off = round_up(off + records * rec, 256);
-    const int64_t ring = seqheads * c->residual * D * 2;
     p.ring_k_off.push_back(off);
-    off = round_up(off + ring, 256);
+    off = round_up(off + seqheads * c->residual * D * 2, 256);
     p.ring_v_off.push_back(off);
-    off = round_up(off + ring, 256);
+    off = round_up(off + seqheads * residual_v_of(*c) * D * 2, 256);
     const int64_t sink = c->sink_tokens > 0 ? seqheads * KVQ_MAX_SINKS * D * 2 : 0;
     p.sink_k_off.push_back(off);
     off = round_up(off + sink, 256);
@@ -146,7 +158,7 @@ Plan make_plan(const kvq_config* c) {
     off = round_up(off + (paged ? (int64_t)c->max_batch * p.max_pages * 4 : 0), 256);
   }
   p.lens_off = off;
-  off = round_up(off + (int64_t)c->num_layers * c->max_batch * 3 * 4, 256);
+  off = round_up(off + (int64_t)c->num_layers * c->max_batch * kvq::kLensStride * 4, 256);
   p.err_off = off;
   off = round_up(off + 4, 256);
   p.uslots_off = off;
@@ -158,7 +170,7 @@ Plan make_plan(const kvq_config* c) {
   p.slots = (int32_t)std::max<int64_t>(
       std::min<int64_t>(p.max_blocks, KVQ_MAX_SPLITS) + 1,
       kvq::kMmaConsumers *
-          (std::min<int64_t>(p.max_blocks + (c->residual + kvq::kResChunk - 1) / kvq::kResChunk + 1, 64) + 1));
+          (std::min<int64_t>(p.max_blocks + (c->residual + kvq::kResChunk - 1) / kvq::kResChunk + 1, 64) + 2));
   const int64_t partials = (int64_t)c->max_batch * c->num_q_heads * p.slots;
   p.ws_o_off = off;
   off = round_up(off + partials * D * 4, 256);
@@ -179,7 +191,7 @@ kvq::LayerView layer_view(const kvq_cache* c, int layer) {
   v.sink_k = c->arena + c->sink_k_off[layer];
   v.sink_v = c->arena + c->sink_v_off[layer];
   v.sinks = cfg.sink_tokens;
-  v.lens = reinterpret_cast<int32_t*>(c->arena + c->lens_off) + (int64_t)layer * cfg.max_batch * 3;
+  v.lens = reinterpret_cast<int32_t*>(c->arena + c->lens_off) + (int64_t)layer * cfg.max_batch * kvq::kLensStride;
   v.record_bytes = c->record_bytes[layer];
   v.max_blocks = c->max_blocks;
   v.kc_off = 0;
@@ -195,6 +207,7 @@ kvq::LayerView layer_view(const kvq_cache* c, int layer) {
   v.group_k = G;
   v.group_v = cfg.group_v;
   v.residual = cfg.residual;
+  v.residual_v = residual_v_of(cfg);
   v.kv_dtype = cfg.kv_dtype;
   const bool paged = cfg.page_blocks > 0;
   v.page_table = paged ? reinterpret_cast<const int32_t*>(c->arena + c->pt_off[layer]) : nullptr;
@@ -212,18 +225,16 @@ kvq_status check_cache_layer(const kvq_cache* c, int layer) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Paged caches: gives each sequence of the call the pages that its blocks
-// after the call need (taken from the layer's pool) and enqueues the
-// page-table update; fails before changing anything if the pool is short.
-kvq_status take_pages(kvq_cache* c, int layer, const kvq::AppendParams& p, int batch, cudaStream_t stream) {
+// Paged caches: gives each sequence b < batch the pages that its
+// blocks_after[b] block records need (taken from the layer's pool) and
+// enqueues the page-table update; fails before changing anything if the
+// pool is short.
+kvq_status take_pages(kvq_cache* c, int layer, const int32_t* blocks_after, int batch, cudaStream_t stream) {
   const kvq_config& cfg = c->cfg;
-  const int G = cfg.group_k, P = cfg.page_blocks;
+  const int P = cfg.page_blocks;
   int32_t* held = &c->pages_held[(size_t)layer * cfg.max_batch];
   std::vector<int32_t>& pool = c->free_pages[layer];
-  auto pages_after = [&](int b) {
-    const int64_t blocks = (p.q_old[b] + (int64_t)p.flush[b] * G) / G;
-    return (int32_t)((blocks + P - 1) / P);
-  };
+  auto pages_after = [&](int b) { return (int32_t)(((int64_t)blocks_after[b] + P - 1) / P); };
   int64_t need = 0;
   for (int b = 0; b < batch; ++b) need += std::max<int64_t>(0, pages_after(b) - held[b]);
   if (need == 0) return KVQ_OK;
@@ -257,12 +268,21 @@ kvq_status take_pages(kvq_cache* c, int layer, const kvq::AppendParams& p, int b
   return KVQ_OK;
 }
 
+// Key or value blocks that a ring holding n of its R slots flushes when T
+// tokens arrive one by one (a token that finds the ring full first moves
+// its oldest G tokens to a block), or every complete group (flush_all).
+int ring_flushes(int n, int T, int R, int G, bool flush_all) {
+  if (flush_all) return n / G;
+  return n + T <= R ? 0 : (n + T - R + G - 1) / G;
+}
+
 // Shared by kvq_append (t_new from the caller) and kvq_flush_residual
-// (t_new = 0, every complete group of the ring flushed).
+// (t_new = 0, every complete group of each ring flushed). Keys and values
+// each follow their own ring.
 kvq_status enqueue_append(kvq_cache* c, int layer, const void* k, const void* v, const int32_t* new_lens,
                           int batch, bool flush_all, cudaStream_t stream) {
   const kvq_config& cfg = c->cfg;
-  const int G = cfg.group_k, R = cfg.residual;
+  const int G = cfg.group_k, R = cfg.residual, RV = residual_v_of(cfg);
   kvq::AppendParams* p = new (std::nothrow) kvq::AppendParams;
   if (!p) return fail(KVQ_ERR_INVALID_ARG, "out of host memory");
   std::memset(p, 0, sizeof *p);
@@ -270,11 +290,15 @@ kvq_status enqueue_append(kvq_cache* c, int layer, const void* k, const void* v,
   p->k_in = k;
   p->v_in = v;
   p->batch = batch;
-  int32_t* ql = &c->q_len[(size_t)layer * cfg.max_batch];
-  int32_t* nl = &c->n_len[(size_t)layer * cfg.max_batch];
-  int32_t* sl = &c->s_len[(size_t)layer * cfg.max_batch];
+  const size_t base = (size_t)layer * cfg.max_batch;
+  int32_t* ql = &c->q_len[base];
+  int32_t* nl = &c->n_len[base];
+  int32_t* sl = &c->s_len[base];
+  int32_t* qvl = &c->qv_len[base];
   int max_flush = 0;
   int64_t off = 0;
+  thread_local std::vector<int32_t> blocks_after;
+  blocks_after.resize(batch);
   for (int b = 0; b < batch; ++b) {
     // the sequence's first sink_tokens tokens go to its sinks
     const int all = flush_all ? 0 : new_lens[b];
@@ -283,19 +307,22 @@ kvq_status enqueue_append(kvq_cache* c, int layer, const void* k, const void* v,
     p->s_take[b] = take;
     off += take;
     const int T = all - take;
-    int f;
-    if (flush_all) f = nl[b] / G;
-    else f = (nl[b] + T <= R) ? 0 : (nl[b] + T - R + G - 1) / G;
+    const int len = ql[b] + nl[b];
+    const int fk = ring_flushes(nl[b], T, R, G, flush_all);
+    const int fv = ring_flushes(len - qvl[b], T, RV, G, flush_all);
     p->q_old[b] = ql[b];
-    p->n_old[b] = nl[b];
+    p->qv_old[b] = qvl[b];
+    p->len_old[b] = len;
     p->t_new[b] = T;
     p->in_off[b] = (int32_t)off;
-    p->flush[b] = f;
+    p->flush[b] = fk;
+    p->flush_v[b] = fv;
     off += T;
-    if (f > max_flush) max_flush = f;
+    max_flush = std::max(max_flush, std::max(fk, fv));
+    blocks_after[b] = std::max(ql[b] + fk * G, qvl[b] + fv * G) / G;
   }
   if (cfg.page_blocks > 0) {
-    const kvq_status ps = take_pages(c, layer, *p, batch, stream);
+    const kvq_status ps = take_pages(c, layer, blocks_after.data(), batch, stream);
     if (ps != KVQ_OK) {
       delete p;
       return ps;
@@ -305,9 +332,10 @@ kvq_status enqueue_append(kvq_cache* c, int layer, const void* k, const void* v,
   if (e == cudaSuccess) {
     for (int b = 0; b < batch; ++b) {
       const int qn = p->q_old[b] + p->flush[b] * G;
-      const int end = p->q_old[b] + p->n_old[b] + p->t_new[b];
+      const int end = p->len_old[b] + p->t_new[b];
       ql[b] = qn;
       nl[b] = end - qn;
+      qvl[b] = p->qv_old[b] + p->flush_v[b] * G;
       sl[b] += p->s_take[b];
     }
   }
@@ -316,76 +344,71 @@ kvq_status enqueue_append(kvq_cache* c, int layer, const void* k, const void* v,
   return KVQ_OK;
 }
 
-// Cuts the concatenated work items of all units (p.nblk, p.nitem, p.seq_start
-// set) into nctas contiguous, non-empty CTA ranges of about equal estimated
-// cost: a quantized block counts 1, a ring chunk kRingChunkCost. A ring chunk
-// has far less arithmetic than a block, but as a short item in a warp's
-// two-stage copy pipeline it leaves the next copy little time to land; on the
-// Llama-3-8B-shaped workload weights 0.3 to 0.6 gave the shortest decode on
-// B200 (83.5 us; 1.2 gave 85.6 us).
-constexpr double kRingChunkCost = 0.5;
-
-void plan_cta_ranges(kvq::DecodeParams& p, int batch, int hkv, int32_t nctas, int32_t total) {
-  double total_cost = 0.0;
-  for (int b = 0; b < batch; ++b)
-    total_cost += (double)hkv * (p.nblk[b] + kRingChunkCost * (p.nitem[b] - p.nblk[b]));
-  const double per = total_cost / nctas;
-  int32_t* st = p.cta_start;
-  st[0] = 0;
-  int32_t c = 1;
-  double cum = 0.0;
-  int64_t item0 = 0;
-  for (int b = 0; b < batch && c < nctas; ++b) {
-    const double cb = p.nblk[b], cr = kRingChunkCost * (p.nitem[b] - p.nblk[b]);
-    for (int h = 0; h < hkv && c < nctas; ++h) {
-      while (c < nctas && c * per <= cum + cb + cr) {
-        const double x = c * per - cum;  // cost into this unit
-        int64_t idx = x <= cb ? (int64_t)std::ceil(x) : p.nblk[b] + (int64_t)std::ceil((x - cb) / kRingChunkCost);
-        idx = std::min<int64_t>(idx, p.nitem[b]);
-        st[c++] = (int32_t)(item0 + idx);
-      }
-      cum += cb + cr;
-      item0 += p.nitem[b];
+// Persistent-mode plan of a decode launch from p.nblk, p.nres, p.nitem
+// (batch sequences, Hkv units each): p.seq_start, the number of CTAs and
+// their item ranges p.cta_start, cut at equal cost (a quantized block costs 2,
+// an exact-token chunk 1, in half units): CTA c starts at the item whose cost
+// interval [P(k), P(k+1)) holds c*C/N, compared in exact integer arithmetic
+// as P*N against c*C. N is at most max_ctas and max(units, items / 4); at
+// most C / (largest item cost), so that no range is empty; and small enough
+// that no unit overlaps more than slot_cap / kMmaConsumers ranges (a unit of
+// cost u overlaps at most floor(u*N/C) + 2 of them). One pass over the
+// sequences and the CTAs.
+void plan_cta_starts(kvq::DecodeParams& p, int batch, int hkv, int64_t max_ctas, int32_t slot_cap) {
+  int64_t T = 0, C = 0, cu_max = 0;
+  bool blocks = false;
+  for (int b = 0; b < batch; ++b) {
+    p.seq_start[b] = (int32_t)T;
+    T += (int64_t)hkv * p.nitem[b];
+    const int64_t cu = kvq::unit_cost(p.nblk[b], p.nitem[b]);
+    C += (int64_t)hkv * cu;
+    cu_max = std::max(cu_max, cu);
+    blocks = blocks || p.nblk[b] > 0;
+  }
+  int64_t N = std::min<int64_t>(max_ctas, std::max<int64_t>((int64_t)batch * hkv, (T + 3) / 4));
+  N = std::min<int64_t>(N, C / (blocks ? 2 : 1));
+  const int64_t kmax = slot_cap / kvq::kMmaConsumers - 2;
+  N = kmax < 0 ? 1 : std::min<int64_t>(N, ((kmax + 1) * C + cu_max - 1) / cu_max - 1);
+  N = std::max<int64_t>(1, std::min<int64_t>(N, kvq::kMaxCtas));
+  p.total_blocks = (int32_t)T;
+  p.num_ctas = (int32_t)N;
+  p.cta_start[0] = 0;
+  int b = 0;
+  int64_t cost0 = 0;  // cost before sequence b
+  for (int64_t c = 1; c < N; ++c) {
+    const int64_t x = c * C;  // threshold, scaled by N
+    int64_t cs = (int64_t)hkv * kvq::unit_cost(p.nblk[b], p.nitem[b]);
+    while ((cost0 + cs) * N <= x) {
+      cost0 += cs;
+      ++b;
+      cs = (int64_t)hkv * kvq::unit_cost(p.nblk[b], p.nitem[b]);
     }
+    const int64_t cu = kvq::unit_cost(p.nblk[b], p.nitem[b]);
+    const int64_t r = x - cost0 * N;
+    const int64_t h = r / (cu * N);
+    const int64_t r2 = r - h * cu * N;
+    const int64_t nb = p.nblk[b];
+    const int64_t j = r2 < 2 * nb * N ? r2 / (2 * N) : nb + (r2 - 2 * nb * N) / N;
+    p.cta_start[c] = (int32_t)(p.seq_start[b] + h * p.nitem[b] + j);
   }
-  while (c < nctas) st[c++] = total;
-  st[nctas] = total;
-  // strictly increasing, every range non-empty (total >= nctas)
-  for (int32_t i = 1; i < nctas; ++i) st[i] = std::max(st[i], st[i - 1] + 1);
-  for (int32_t i = nctas - 1; i >= 1; --i) st[i] = std::min(st[i], st[i + 1] - 1);
-}
-
-// Points the split partials of p at `scratch` with a slot stride of `slots`;
-// false (and *status) if they do not fit.
-bool use_scratch(kvq::DecodeParams& p, const kvq::StaticScratch& scratch, int batch, int32_t slots, kvq_status* status) {
-  const int64_t partials = (int64_t)batch * p.num_q_heads * slots;
-  const int64_t o_bytes = kvq::round_up(partials * kvq::kHeadDim * 4, 256);
-  const int64_t need = o_bytes + partials * 8;
-  if (need > scratch.bytes) {
-    *status = fail(KVQ_ERR_WORKSPACE,
-                   "this decode needs %lld bytes of split partials (batch %d x %d query heads x %d slots); the "
-                   "static scratch holds %lld",
-                   (long long)need, batch, p.num_q_heads, slots, (long long)scratch.bytes);
-    return false;
-  }
-  p.slots = slots;
-  p.ws_o = reinterpret_cast<float*>(scratch.base);
-  p.ws_ml = reinterpret_cast<float2*>(scratch.base + o_bytes);
-  return true;
+  p.cta_start[N] = (int32_t)T;
 }
 
 }  // namespace
 
 namespace kvq {
 
-// Decode attention of kvq_decode_attention. With scratch == nullptr the
-// split partials live in the arena's workspace (slot stride = the arena's
-// slot count); otherwise in `scratch`, with the slot stride cut to what this
-// call uses, and a call whose partials would not fit is rejected before
-// anything is enqueued.
-kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const void* new_v, const void* q, void* out, int32_t out_dtype,
-                          float softmax_scale, int32_t batch, void* stream, const StaticScratch* scratch,
-                          const QueryGroup* qg) {
+// Decode attention of kvq_decode_attention and its variants. The split
+// partials live in the arena's workspace (slot stride: the arena's slot
+// count, or what the workspace holds for a group of query tokens), or, with
+// `scratch`, in that memory together with the unit slot counts (the slot
+// stride then cut to what fits; a call for which no split fits is rejected
+// before anything is enqueued). new_k/new_v: a fused decode step's new
+// tokens, already counted in the host mirror; after_flush: that step's flush
+// kernel was enqueued just before.
+kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const void* new_v, const void* q, void* out,
+                          int32_t out_dtype, float softmax_scale, int32_t batch, void* stream,
+                          const StaticScratch* scratch, const QueryGroup* qg, bool after_flush) {
   kvq_status s = check_cache_layer(c, layer);
   if (s != KVQ_OK) return s;
   if (batch < 0 || batch > c->cfg.max_batch)
@@ -399,40 +422,21 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const 
   const kvq_config& cfg = c->cfg;
   const int G = cfg.group_k;
   const kvq::LayerView L = layer_view(c, layer);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
   // query rows per launch: the query heads of each of the group's tokens
   const int qtok = qg ? qg->qtok : 1;
   const int Hv = cfg.num_q_heads * qtok;
   const bool use_mma = kvq::mma_supported(L, Hv);
-  kvq::MmaPlan mp{};
-  int per_sm = 4;
-  if (!use_mma) per_sm = kvq::split_ctas_per_sm(Hv, cfg.num_kv_heads);
-  if (use_mma) {
-    mp = kvq::make_mma_plan(L, Hv);
-    per_sm = kvq::mma_ctas_per_sm(L, mp, Hv);
-  }
   // partial slots per (sequence, query row) that fit the arena's workspace
   // (sized for num_q_heads rows): all of them for one query token, fewer for
   // a group, whose slot stride is then cut to what the launch uses
-  const int32_t slot_cap =
+  int32_t slot_cap =
       qg ? (int32_t)std::min<int64_t>(c->slots, (int64_t)cfg.max_batch * cfg.num_q_heads * c->slots /
                                                     ((int64_t)batch * Hv))
          : c->slots;
-  if (slot_cap < 2) return fail(KVQ_ERR_WORKSPACE, "the workspace holds too few partial slots for %d query rows", Hv);
-  // per-call scratch of this thread (no heap traffic per call)
-  thread_local std::vector<int> nblk;
-  nblk.resize(batch);
-  int max_blk = 0;
-  int64_t total_blocks = 0;
-  for (int b = 0; b < batch; ++b) {
-    nblk[b] = c->q_len[(size_t)layer * cfg.max_batch + b] / G;
-    max_blk = std::max(max_blk, nblk[b]);
-    total_blocks += (int64_t)nblk[b] * cfg.num_kv_heads;
-  }
-  if (total_blocks > INT32_MAX) return fail(KVQ_ERR_UNSUPPORTED, "more than 2^31 quantized blocks in one call");
-  thread_local kvq::DecodeParams params;
-  kvq::DecodeParams* pp = &params;
-  kvq::DecodeParams& p = *pp;
-  std::memset(pp, 0, offsetof(kvq::DecodeParams, nblk));  // the per-sequence tables are written below
+  thread_local DecodeParams params;  // large (per-sequence tables): one per thread, not on the stack
+  DecodeParams& p = params;
+  std::memset(&p, 0, offsetof(DecodeParams, nblk));  // the per-sequence tables are written below
   p.L = L;
   p.new_k = new_k;
   p.new_v = new_v;
@@ -440,6 +444,29 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const 
   p.out = out;
   p.ws_o = reinterpret_cast<float*>(c->arena + c->ws_o_off);
   p.ws_ml = reinterpret_cast<float2*>(c->arena + c->ws_ml_off);
+  p.unit_slots = reinterpret_cast<int32_t*>(c->arena + c->uslots_off);
+  if (scratch) {
+    // unit slot counts, then the partials (o, then (m, l)), 256-byte aligned
+    const int64_t plan_b = 0;
+    const int64_t us_b = kvq::round_up((int64_t)batch * cfg.num_kv_heads * 4, 256);
+    const int64_t per_slot = (int64_t)batch * Hv * (kHeadDim * 4 + 8);
+    const int64_t room = scratch->bytes - plan_b - us_b - 256;
+    const int64_t fit = room > 0 ? room / per_slot : 0;
+    slot_cap = (int32_t)std::min<int64_t>(fit, c->slots);
+    if (slot_cap < (use_mma ? kMmaConsumers : 2))
+      return fail(KVQ_ERR_WORKSPACE,
+                  "the static scratch (%lld bytes) holds %d partial slots per query row for batch %d x %d query rows; "
+                  "this decode needs at least %d",
+                  (long long)scratch->bytes, slot_cap, batch, Hv, use_mma ? kMmaConsumers : 2);
+    uint8_t* base = scratch->base;
+    p.unit_slots = reinterpret_cast<int32_t*>(base + plan_b);
+    p.ws_o = reinterpret_cast<float*>(base + plan_b + us_b);
+    p.ws_ml = reinterpret_cast<float2*>(base + plan_b + us_b +
+                                        kvq::round_up((int64_t)batch * Hv * slot_cap * kHeadDim * 4, 256));
+  }
+  if (use_mma && slot_cap < kMmaConsumers)
+    return fail(KVQ_ERR_WORKSPACE, "the workspace holds %d partial slots per query row for %d query rows; need %d",
+                slot_cap, Hv, kMmaConsumers);
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   // the tensor-core kernel multiplies fp16 queries by fp16 key scales: a power
   // of two near scale_log2 keeps those products as far from the fp16 limit as
@@ -459,54 +486,40 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const 
   p.q_rows = qg ? qg->q_rows : cfg.num_q_heads;
   p.qtok = qtok;
   p.lag_base = qg ? qg->lag_base : 0;
-  p.slots = c->slots;
   p.err = reinterpret_cast<int32_t*>(c->arena + c->err_off);
-  p.unit_slots = reinterpret_cast<int32_t*>(c->arena + c->uslots_off);
   cudaError_t e;
-  int32_t used_slots = c->slots;  // partial slots per (sequence, query head) this call writes
   if (use_mma) {
-    // Persistent plan: the work items of every (sequence, KV head) unit
-    // (quantized blocks, ring chunks, sinks), concatenated and cut into one
-    // contiguous range per CTA, one CTA per resident slot (fewer if there is
-    // little work).
-    int64_t total = 0;
+    // Persistent plan from the host mirror: the work items of every
+    // (sequence, KV head) unit (quantized blocks, ring chunks, sinks),
+    // concatenated and cut into one contiguous range of equal cost per CTA,
+    // one CTA per resident slot (fewer if there is little work).
+    const kvq::MmaPlan mp = kvq::make_mma_plan(L, Hv);
+    const int per_sm = kvq::mma_ctas_per_sm(L, mp, Hv);
     for (int b = 0; b < batch; ++b) {
-      const int nres = c->n_len[(size_t)layer * cfg.max_batch + b];
-      p.nblk[b] = nblk[b];
-      p.nres[b] = nres;
-      p.nitem[b] = kvq::unit_items(nblk[b], nres, c->s_len[(size_t)layer * cfg.max_batch + b]);
-      p.seq_start[b] = (int32_t)total;
-      total += (int64_t)p.nitem[b] * cfg.num_kv_heads;
-    }
-    if (total > INT32_MAX) return fail(KVQ_ERR_UNSUPPORTED, "more than 2^31 work items in one call");
-    int64_t nctas = std::min<int64_t>((int64_t)std::max(1, c->sm_count) * per_sm,
-                                      std::max<int64_t>((int64_t)batch * cfg.num_kv_heads, (total + 3) / 4));
-    nctas = std::max<int64_t>(1, std::min<int64_t>(nctas, std::min<int64_t>(kvq::kMaxCtas, total)));
-    // every (sequence, head) must fit its partials in the workspace
-    for (;;) {
-      plan_cta_ranges(p, batch, cfg.num_kv_heads, (int32_t)nctas, (int32_t)total);
-      int32_t need = 1;
-      for (int b = 0; b < batch; ++b)
-        for (int h = 0; h < cfg.num_kv_heads; ++h)
-          need = std::max(need, kvq::persistent_slots(p.cta_start, (int32_t)nctas, p.seq_start[b] + h * p.nitem[b],
-                                                      p.nitem[b]));
-      used_slots = need;
-      if (need <= slot_cap || nctas == 1) break;
-      nctas = std::max<int64_t>(1, nctas * 3 / 4);
+      const size_t i = (size_t)layer * cfg.max_batch + b;
+      p.nblk[b] = c->q_len[i] / G;
+      p.nres[b] = c->n_len[i];
+      p.nitem[b] = kvq::unit_items(p.nblk[b], p.nres[b], c->s_len[i]);
     }
     p.persistent = 1;
-    p.total_blocks = (int32_t)total;
-    p.num_ctas = (int32_t)nctas;
-    if (used_slots > slot_cap)
-      return fail(KVQ_ERR_WORKSPACE, "the workspace holds %d partial slots per query row; this call needs %d",
-                  slot_cap, used_slots);
-    if (qg) p.slots = used_slots;
-    if (scratch && !use_scratch(p, *scratch, batch, used_slots, &s)) return s;
-    e = kvq::launch_decode_mma(p, mp, static_cast<cudaStream_t>(stream));
-    if (e == cudaSuccess) e = kvq::launch_combine(p, static_cast<cudaStream_t>(stream));
+    p.slots = slot_cap;
+    p.after_flush = after_flush ? 1 : 0;
+    plan_cta_starts(p, batch, cfg.num_kv_heads, (int64_t)std::max(1, c->sm_count) * per_sm, slot_cap);
+    e = kvq::launch_decode_mma(p, mp, st);
+    if (e == cudaSuccess) e = kvq::launch_combine(p, st);
   } else {
-    // Split plan: blocks per split chosen to minimise (waves of CTAs) x
-    // (blocks per CTA + a fixed per-CTA overhead), with at most slots-1 splits.
+    // Split plan (host mirror): blocks per split chosen to minimise (waves
+    // of CTAs) x (blocks per CTA + a fixed per-CTA overhead), with at most
+    // slot_cap - 1 splits.
+    const int per_sm = kvq::split_ctas_per_sm(Hv, cfg.num_kv_heads);
+    thread_local std::vector<int> nblk;
+    nblk.resize(batch);
+    int max_blk = 0;
+    for (int b = 0; b < batch; ++b) {
+      const size_t i = (size_t)layer * cfg.max_batch + b;
+      nblk[b] = std::max(c->q_len[i], c->qv_len[i]) / G;
+      max_blk = std::max(max_blk, nblk[b]);
+    }
     const int64_t slots_gpu = (int64_t)std::max(1, c->sm_count) * per_sm;
     const int64_t min_bps = std::max<int64_t>(1, (max_blk + (slot_cap - 1) - 1) / (slot_cap - 1));
     int64_t bps = std::max<int64_t>(min_bps, max_blk);
@@ -524,10 +537,8 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const 
     }
     p.blocks_per_split = (int32_t)bps;
     const int nsplits = (int)((max_blk + bps - 1) / bps);
-    used_slots = nsplits + 1;
-    if (qg) p.slots = used_slots;
-    if (scratch && !use_scratch(p, *scratch, batch, used_slots, &s)) return s;
-    e = kvq::launch_decode(p, nsplits, static_cast<cudaStream_t>(stream));
+    p.slots = slot_cap;
+    e = kvq::launch_decode(p, nsplits, st);
   }
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return KVQ_OK;
@@ -535,6 +546,8 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const 
 
 void clear_last_error() { g_last_error.clear(); }
 kvq_status report_cuda_error(cudaError_t e, const char* what) { return cuda_fail(e, what); }
+kvq_status report_status(kvq_status s, const char* what) { return fail(s, "%s", what); }
+int cache_device(const kvq_cache* c) { return c->device; }
 
 }  // namespace kvq
 
@@ -546,7 +559,7 @@ const char* kvq_status_string(kvq_status s) {
     case KVQ_ERR_INVALID_ARG: return "invalid argument";
     case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
     case KVQ_ERR_CAPACITY: return "sequence capacity exceeded";
-    case KVQ_ERR_WORKSPACE: return "arena too small";
+    case KVQ_ERR_WORKSPACE: return "arena or static scratch too small";
     case KVQ_ERR_CUDA: return "CUDA error";
   }
   return "unknown status";
@@ -610,20 +623,23 @@ kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena
   c->q_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
   c->n_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
   c->s_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
+  c->qv_len.assign((size_t)cfg->num_layers * cfg->max_batch, 0);
+  const size_t lens_bytes = (size_t)cfg->num_layers * cfg->max_batch * kvq::kLensStride * 4;
   cudaError_t e = cudaGetDevice(&c->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device);
-  if (e == cudaSuccess) e = cudaMemset(c->arena + c->lens_off, 0, (size_t)cfg->num_layers * cfg->max_batch * 12);
+  if (e == cudaSuccess) e = cudaMemset(c->arena + c->lens_off, 0, lens_bytes);
   if (e == cudaSuccess) e = cudaMemset(c->arena + c->err_off, 0, 4);
   // Ring slots and sink rows that no token has reached yet hold zeros, never
   // stale bit patterns: the decode kernel reads whole chunks of ring slots
   // and sink rows and masks the scores of those past the sequence, so their
   // values must be finite.
   const size_t ring_bytes = (size_t)cfg->max_batch * cfg->num_kv_heads * cfg->residual * cfg->head_dim * 2;
+  const size_t ring_v_bytes = (size_t)cfg->max_batch * cfg->num_kv_heads * residual_v_of(*cfg) * cfg->head_dim * 2;
   const size_t sink_bytes =
       cfg->sink_tokens > 0 ? (size_t)cfg->max_batch * cfg->num_kv_heads * KVQ_MAX_SINKS * cfg->head_dim * 2 : 0;
   for (int l = 0; l < cfg->num_layers && e == cudaSuccess; ++l) {
     e = cudaMemset(c->arena + c->ring_k_off[l], 0, ring_bytes);
-    if (e == cudaSuccess) e = cudaMemset(c->arena + c->ring_v_off[l], 0, ring_bytes);
+    if (e == cudaSuccess) e = cudaMemset(c->arena + c->ring_v_off[l], 0, ring_v_bytes);
     if (e == cudaSuccess && sink_bytes) e = cudaMemset(c->arena + c->sink_k_off[l], 0, sink_bytes);
     if (e == cudaSuccess && sink_bytes) e = cudaMemset(c->arena + c->sink_v_off[l], 0, sink_bytes);
     if (e == cudaSuccess && cfg->page_blocks > 0)  // entries not yet given out name page 0 (valid memory)
@@ -648,12 +664,14 @@ kvq_status kvq_cache_destroy(kvq_cache* c) {
 kvq_status kvq_cache_reset(kvq_cache* c, void* stream) {
   g_last_error.clear();
   if (!c) return fail(KVQ_ERR_INVALID_ARG, "cache is null");
-  cudaError_t e = cudaMemsetAsync(c->arena + c->lens_off, 0, (size_t)c->cfg.num_layers * c->cfg.max_batch * 12,
+  cudaError_t e = cudaMemsetAsync(c->arena + c->lens_off, 0,
+                                  (size_t)c->cfg.num_layers * c->cfg.max_batch * kvq::kLensStride * 4,
                                   static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "reset");
   std::fill(c->q_len.begin(), c->q_len.end(), 0);
   std::fill(c->n_len.begin(), c->n_len.end(), 0);
   std::fill(c->s_len.begin(), c->s_len.end(), 0);
+  std::fill(c->qv_len.begin(), c->qv_len.end(), 0);
   if (c->cfg.page_blocks > 0) {
     for (auto& f : c->free_pages) {
       f.clear();
@@ -670,13 +688,13 @@ kvq_status kvq_release_sequence(kvq_cache* c, int32_t seq, void* stream) {
   const kvq_config& cfg = c->cfg;
   if (seq < 0 || seq >= cfg.max_batch) return fail(KVQ_ERR_INVALID_ARG, "seq %d outside 0..%d", seq, cfg.max_batch - 1);
   for (int l = 0; l < cfg.num_layers; ++l) {
-    cudaError_t e = cudaMemsetAsync(c->arena + c->lens_off + ((size_t)l * cfg.max_batch + seq) * 12, 0, 12,
-                                    static_cast<cudaStream_t>(stream));
+    cudaError_t e = cudaMemsetAsync(c->arena + c->lens_off + ((size_t)l * cfg.max_batch + seq) * kvq::kLensStride * 4,
+                                    0, kvq::kLensStride * 4, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "release");
   }
   for (int l = 0; l < cfg.num_layers; ++l) {
     const size_t i = (size_t)l * cfg.max_batch + seq;
-    c->q_len[i] = c->n_len[i] = c->s_len[i] = 0;
+    c->q_len[i] = c->n_len[i] = c->s_len[i] = c->qv_len[i] = 0;
     if (cfg.page_blocks > 0) {
       const int32_t* row = &c->pt_host[i * c->max_pages];
       for (int32_t k = c->pages_held[i] - 1; k >= 0; --k) c->free_pages[l].push_back(row[k]);
@@ -747,7 +765,8 @@ kvq_status kvq_decode_attention_multi(kvq_cache* c, int32_t layer, const void* q
   // the query tokens' own keys and values are the newest cached tokens,
   // still in the ring, where the causal mask applies
   for (int b = 0; b < batch; ++b) {
-    const int n = c->n_len[(size_t)layer * cfg.max_batch + b];
+    const size_t i = (size_t)layer * cfg.max_batch + b;
+    const int n = std::min(c->n_len[i], c->q_len[i] + c->n_len[i] - c->qv_len[i]);
     if (n < num_tokens)
       return fail(KVQ_ERR_UNSUPPORTED,
                   "sequence %d has %d ring tokens: its %d query tokens must be its newest tokens, in the ring", b,
@@ -786,16 +805,21 @@ kvq_status kvq_decode_step(kvq_cache* c, int32_t layer, const void* k, const voi
     return fail(KVQ_ERR_INVALID_ARG, "k, v, q and out must be 16-byte aligned");
   const kvq_config& cfg = c->cfg;
   const size_t base = (size_t)layer * cfg.max_batch;
-  // The new tokens ride along with the decode when every one of them lands in
-  // a ring slot without a flush (ring not full, sinks complete) and the layer
-  // runs on the tensor-core kernel; otherwise append, then decode.
-  bool fused = kvq::mma_supported(layer_view(c, layer), c->cfg.num_q_heads);
+  // The new tokens ride along with the decode when the layer runs on the
+  // tensor-core kernel, every sequence's sinks are complete and keys and
+  // values share one ring: the prep kernel then quantizes the oldest G
+  // tokens of every full ring (one block per such sequence and KV head),
+  // its plan counts the new tokens, and the decode kernel writes them into
+  // their ring slots. Otherwise: append, then decode.
+  bool fused = kvq::mma_supported(layer_view(c, layer), c->cfg.num_q_heads) && residual_v_of(cfg) == cfg.residual;
+  bool flush = false;
   for (int b = 0; b < batch; ++b) {
     const int64_t L = (int64_t)c->s_len[base + b] + c->q_len[base + b] + c->n_len[base + b] + 1;
     if (L > cfg.max_tokens)
       return fail(KVQ_ERR_CAPACITY, "sequence %d would hold %lld tokens > max_tokens %d", b, (long long)L,
                   cfg.max_tokens);
-    if (c->n_len[base + b] >= cfg.residual || c->s_len[base + b] < cfg.sink_tokens) fused = false;
+    if (c->s_len[base + b] < cfg.sink_tokens) fused = false;
+    flush = flush || c->n_len[base + b] == cfg.residual;
   }
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (!fused) {
@@ -805,10 +829,44 @@ kvq_status kvq_decode_step(kvq_cache* c, int32_t layer, const void* k, const voi
     if (s != KVQ_OK) return s;
     return kvq::enqueue_decode(c, layer, nullptr, nullptr, q, out, out_dtype, softmax_scale, batch, stream, nullptr);
   }
-  for (int b = 0; b < batch; ++b) ++c->n_len[base + b];
-  s = kvq::enqueue_decode(c, layer, k, v, q, out, out_dtype, softmax_scale, batch, stream, nullptr);
+  const int G = cfg.group_k;
+  if (flush && cfg.page_blocks > 0) {
+    thread_local std::vector<int32_t> blocks_after;
+    blocks_after.resize(batch);
+    for (int b = 0; b < batch; ++b)
+      blocks_after[b] = (c->q_len[base + b] + (c->n_len[base + b] == cfg.residual ? G : 0)) / G;
+    s = take_pages(c, layer, blocks_after.data(), batch, st);
+    if (s != KVQ_OK) return s;
+  }
+  thread_local std::vector<int32_t> flushed;
+  flushed.assign(batch, 0);
+  for (int b = 0; b < batch; ++b) {
+    if (c->n_len[base + b] == cfg.residual) {
+      flushed[b] = 1;
+      c->q_len[base + b] += G;
+      c->qv_len[base + b] += G;
+      c->n_len[base + b] -= G;
+    }
+    ++c->n_len[base + b];
+  }
+  if (flush) {
+    kvq::FlushParams fp;
+    fp.L = layer_view(c, layer);
+    fp.ctas = batch * cfg.num_kv_heads;
+    const cudaError_t e = kvq::launch_step_flush(fp, st);
+    if (e != cudaSuccess) s = cuda_fail(e, "flush launch");
+  }
+  if (s == KVQ_OK)
+    s = kvq::enqueue_decode(c, layer, k, v, q, out, out_dtype, softmax_scale, batch, stream, nullptr, nullptr, flush);
   if (s != KVQ_OK)
-    for (int b = 0; b < batch; ++b) --c->n_len[base + b];
+    for (int b = 0; b < batch; ++b) {
+      --c->n_len[base + b];
+      if (flushed[b]) {
+        c->q_len[base + b] -= G;
+        c->qv_len[base + b] -= G;
+        c->n_len[base + b] += G;
+      }
+    }
   return s;
 }
 
@@ -878,6 +936,19 @@ kvq_status kvq_seq_lengths(const kvq_cache* c, int32_t layer, int32_t seq, int32
   const size_t i = (size_t)layer * c->cfg.max_batch + seq;
   *quantized = c->q_len[i];
   *residual = c->n_len[i];
+  return KVQ_OK;
+}
+
+kvq_status kvq_seq_value_lengths(const kvq_cache* c, int32_t layer, int32_t seq, int32_t* quantized,
+                                 int32_t* residual) {
+  g_last_error.clear();
+  kvq_status s = check_cache_layer(c, layer);
+  if (s != KVQ_OK) return s;
+  if (seq < 0 || seq >= c->cfg.max_batch) return fail(KVQ_ERR_INVALID_ARG, "seq %d out of range", seq);
+  if (!quantized || !residual) return fail(KVQ_ERR_INVALID_ARG, "output pointer is null");
+  const size_t i = (size_t)layer * c->cfg.max_batch + seq;
+  *quantized = c->qv_len[i];
+  *residual = c->q_len[i] + c->n_len[i] - c->qv_len[i];
   return KVQ_OK;
 }
 

@@ -1,198 +1,441 @@
 // Append / flush / dequantize kernels.
 //
 // Method: "KIVI" README, sections "Overview" and "Example" (keys per channel,
-// values per token, residual window of recent full-precision tokens) and the
+// values per token, residual window of recent full-precision tokens), the
 // quantizer of the "KV1-1.2B" card, section "Quantization Format: KV1.cpp
-// BQ2_0". One CTA quantizes one G-token block of one (sequence, KV head):
-// the block is staged in shared memory as raw 16-bit values, keys are reduced
-// per channel (one thread per channel), values per group_v channels of a token
-// with warp __shfl_xor min/max reductions, and codes are packed into 32-bit
-// words lowest bits first.
+// BQ2_0", and per-tensor residual windows ("Quantize What Counts", KV Cache
+// Quantization: residual_length {k, v}).
+//
+// One CTA of kQuantThreads threads quantizes one G-token key block and/or one
+// G-token value block of one (sequence, KV head). The G x D rows are staged in
+// shared memory with 16-byte loads (all of a thread's loads issued before any
+// store). Per-channel keys: every thread takes one channel pair and a slice of
+// 32/k_bits tokens (one output word per channel), reduces min/max over its
+// slice, the slices of a channel are combined through shared memory, and the
+// same thread then packs the slice's codes -- so G*D values are spread over
+// D/2 * G*k_bits/32 threads instead of one thread per channel. Values (and the
+// scales of per-token keys): one thread per output word of 32/v_bits channels
+// of a token, the min/max of a group combined with __shfl_xor. Codes use
+// IEEE-rounded fp32 arithmetic (__fsub_rn, __fdiv_rn, rintf), bit-exact with
+// the oracle.
 #include "kvq_append.cuh"
+#include "kvq_decode.cuh"
 
 namespace kvq {
 
 namespace {
 
-__device__ __forceinline__ float bits_to_float(uint16_t v, int dtype) {
-  if (dtype == KVQ_BF16) return __uint_as_float((uint32_t)v << 16);
-  return __half2float(__ushort_as_half(v));
+__device__ __forceinline__ float bits_to_float(uint32_t v, int dtype) {
+  if (dtype == KVQ_BF16) return __uint_as_float(v << 16);
+  return __half2float(__ushort_as_half((unsigned short)v));
 }
 
-}  // namespace
+// Where row t (0 <= t < G) of a block comes from: the ring (positions before
+// `boundary`) or this call's input (row in_row0 + position - boundary).
+struct BlockRows {
+  const uint16_t* ring;  // ring of (b, h): [R][D]
+  const uint16_t* in;    // input [rows][Hkv][D] (null: ring only)
+  int64_t in_row0;
+  int32_t first;         // position of the block's first token
+  int32_t boundary;
+  int32_t R, Hkv, h;
+  __device__ __forceinline__ const uint16_t* row(int t) const {
+    const int i = first + t;
+    if (i < boundary) return ring + (int64_t)(i % R) * kHeadDim;
+    return in + ((in_row0 + (i - boundary)) * Hkv + h) * kHeadDim;
+  }
+};
 
-// One group quantizer pass over rows of D values: every (row, run of gv
-// channels) is one group; each thread owns one output word (32/bits
-// channels) and the gv/(32/bits) threads of a group combine their min/max
-// with xor shuffles. val(t, d) reads value d of row t; put_word(t, w, word)
-// and put_sz(t, g, d16, m16) store the codes and the group's scale and zero.
-template <class Val, class PutWord, class PutSz>
-__device__ __forceinline__ void quantize_rows(int rows, int D, int bits, int gv, Val val, PutWord put_word,
-                                              PutSz put_sz) {
-  const int per = 32 / bits;
-  const int wpt = D / per;  // words per row
-  const int P = gv / per;   // threads per group, a power of two <= 32
-  for (int widx = threadIdx.x; widx < rows * wpt; widx += blockDim.x) {
-    const int t = widx / wpt, w = widx % wpt;
-    float mn = val(t, w * per), mx = mn;
-    for (int i = 1; i < per; ++i) {
-      const float x = val(t, w * per + i);
-      mn = fminf(mn, x);
-      mx = fmaxf(mx, x);
+// One CTA quantizes one part of one tensor of a G-token block: per-channel
+// keys split by channels (the min/max of a channel runs over all G tokens),
+// values and per-token keys split by tokens. The fused step's flush uses
+// kStepParts parts per tensor (its grid is only batch x Hkv blocks); appends
+// use one.
+constexpr int kStepParts = 2;
+
+struct PartShape {
+  bool key;
+  int t0, nt;  // staged tokens [t0, t0 + nt) of the block
+  int c0, nc;  // quantized channels [c0, c0 + nc) (per-channel keys; else all)
+  int sc0, snc;  // staged channels (the rotation needs whole rows)
+};
+__host__ __device__ inline PartShape part_shape(bool key, int part, int parts, int G, int k_axis, bool rot) {
+  PartShape s;
+  s.key = key;
+  if (key && k_axis == 0) {
+    s.t0 = 0, s.nt = G;
+    s.nc = kHeadDim / parts, s.c0 = part * s.nc;
+  } else {
+    s.nt = G / parts, s.t0 = part * s.nt;
+    s.c0 = 0, s.nc = kHeadDim;
+  }
+  s.sc0 = rot ? 0 : s.c0;
+  s.snc = rot ? kHeadDim : s.nc;
+  return s;
+}
+
+// Shared memory of one part CTA (bytes): staged rows [nt][snc] (raw 16-bit,
+// or fp32 when rotated), then per-channel keys' slice min/max float2
+// [W][nc], then the key groups' fp32 (scale, zero, 1/scale) float4.
+struct QuantSmem {
+  int rows, red, kpar, total;
+};
+__host__ __device__ inline QuantSmem part_smem(const PartShape& s, int G, int kb, int gv, int k_axis, bool rot) {
+  QuantSmem q;
+  q.rows = s.nt * s.snc * (rot ? 4 : 2);
+  q.red = (s.key && k_axis == 0) ? (G * kb / 32) * s.nc * 8 : 0;
+  q.kpar = !s.key ? 0 : (k_axis == 0 ? s.nc : s.nt * (kHeadDim / gv)) * 16;
+  q.total = q.rows + q.red + q.kpar;
+  return q;
+}
+// The largest over the part CTAs of a launch with `parts` parts per tensor.
+__host__ __device__ inline int quant_smem_bytes(int G, int kb, int gv, int k_axis, bool rot, int parts) {
+  const int a = part_smem(part_shape(true, 0, parts, G, k_axis, rot), G, kb, gv, k_axis, rot).total;
+  const int b = part_smem(part_shape(false, 0, parts, G, k_axis, rot), G, kb, gv, k_axis, rot).total;
+  return a > b ? a : b;
+}
+
+// Stages rows t0 .. t0+nt-1, channels c0 .. c0+nc-1 of a block as raw
+// 16-bit values ([nt][nc]) with 16-byte loads, two per thread in flight at
+// a time.
+__device__ __forceinline__ void stage_raw(const BlockRows& src, int t0, int nt, int c0, int nc, uint16_t* dst) {
+  const int cpr = nc / 8;  // 16-byte chunks per staged row
+  const int n = nt * cpr;
+  for (int idx = threadIdx.x; idx < n; idx += 2 * kQuantThreads) {
+    const int i2 = idx + kQuantThreads;
+    const uint4 a = *reinterpret_cast<const uint4*>(src.row(t0 + idx / cpr) + c0 + (idx % cpr) * 8);
+    uint4 b2;
+    if (i2 < n) b2 = *reinterpret_cast<const uint4*>(src.row(t0 + i2 / cpr) + c0 + (i2 % cpr) * 8);
+    *reinterpret_cast<uint4*>(dst + (idx / cpr) * nc + (idx % cpr) * 8) = a;
+    if (i2 < n) *reinterpret_cast<uint4*>(dst + (i2 / cpr) * nc + (i2 % cpr) * 8) = b2;
+  }
+}
+
+// Stages rows t0 .. t0+nt-1 rotated (x . H, rotate_lane) as fp32 [nt][D]:
+// one warp per row.
+__device__ __forceinline__ void stage_rotated(const BlockRows& src, int t0, int nt, int dt, float* dst) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int t = warp; t < nt; t += kQuantThreads / 32) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(src.row(t0 + t) + 4 * lane);
+    float x[4] = {bits_to_float(raw.x & 0xffffu, dt), bits_to_float(raw.x >> 16, dt),
+                  bits_to_float(raw.y & 0xffffu, dt), bits_to_float(raw.y >> 16, dt)};
+    rotate_lane(x, lane);
+    *reinterpret_cast<float4*>(dst + t * kHeadDim + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
+  }
+}
+
+// Values x[0..N) of channels c .. c+N-1 of staged row t (rows of `pitch`
+// channels).
+template <bool ROT, int N>
+__device__ __forceinline__ void row_values(const uint8_t* rows, int pitch, int t, int c, int dt, float (&x)[N]) {
+  if constexpr (ROT) {
+    const float4* f = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(rows) + t * pitch + c);
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const float4 q = f[i];
+      x[4 * i] = q.x, x[4 * i + 1] = q.y, x[4 * i + 2] = q.z, x[4 * i + 3] = q.w;
+    }
+  } else {
+    const uint16_t* r = reinterpret_cast<const uint16_t*>(rows) + t * pitch + c;
+    if constexpr (N >= 8) {
+#pragma unroll
+      for (int i = 0; i < N / 8; ++i) {
+        const uint4 q = reinterpret_cast<const uint4*>(r)[i];
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          x[8 * i + 2 * e] = bits_to_float(w[e] & 0xffffu, dt);
+          x[8 * i + 2 * e + 1] = bits_to_float(w[e] >> 16, dt);
+        }
+      }
+    } else {
+      const uint2 q = *reinterpret_cast<const uint2*>(r);
+      x[0] = bits_to_float(q.x & 0xffffu, dt), x[1] = bits_to_float(q.x >> 16, dt);
+      x[2] = bits_to_float(q.y & 0xffffu, dt), x[3] = bits_to_float(q.y >> 16, dt);
+    }
+  }
+}
+
+// One staged value: row t, column c (rows of `pitch` channels).
+template <bool ROT>
+__device__ __forceinline__ float staged(const uint8_t* rows, int pitch, int t, int c, int dt) {
+  if constexpr (ROT) return reinterpret_cast<const float*>(rows)[t * pitch + c];
+  return bits_to_float(reinterpret_cast<const uint16_t*>(rows)[t * pitch + c], dt);
+}
+
+// Word index of word w of channel d in a record's key code array (the
+// kc_word_index placement) with W = 2^lgW words per channel.
+__device__ __forceinline__ int kc_index_p2(int d, int w, int lgW) {
+  const int W = 1 << lgW;
+  if (lgW < 2) return (d << lgW) + w;
+  const int lgn = lgW - 2;  // 16-byte chunks per row: 2^lgn
+  const int sw = lgn >= 3 ? (d & 7) : ((d >> (3 - lgn)) & ((1 << lgn) - 1));
+  return d * W + ((((w >> 2) ^ sw)) << 2) + (w & 3);
+}
+
+// Groups of gv channels of staged rows [0, nt) (tokens t0 + row), BITS-wide
+// codes: one thread per output word (PER = 32/BITS channels); the gv/PER
+// threads of a group combine their min/max with xor shuffles. put_word(t, w,
+// word) and put_sz(t, g, params) receive the results (t: token of the block).
+template <bool ROT, int BITS, bool CODES, class PutWord, class PutSz>
+__device__ __forceinline__ void quantize_token_groups(const uint8_t* rows, int t0, int nt, int gv, int dt,
+                                                      PutWord put_word, PutSz put_sz) {
+  constexpr int PER = 32 / BITS;
+  constexpr int WPT = kHeadDim / PER;  // words per row
+  const int P = gv / PER;              // threads per group: a power of two, <= 32, dividing WPT
+  for (int item = threadIdx.x; item < nt * WPT; item += kQuantThreads) {
+    const int t = item / WPT, w = item % WPT;
+    float x[PER];
+    row_values<ROT, PER>(rows, kHeadDim, t, w * PER, dt, x);
+    float mn = x[0], mx = x[0];
+#pragma unroll
+    for (int i = 1; i < PER; ++i) {
+      mn = fminf(mn, x[i]);
+      mx = fmaxf(mx, x[i]);
     }
     for (int o = P / 2; o >= 1; o >>= 1) {
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
-    const GroupParams gp = group_params(mn, mx, bits);
-    uint32_t word = 0;
-    for (int i = 0; i < per; ++i) word |= quant_code(val(t, w * per + i), gp, bits) << (i * bits);
-    put_word(t, w, word);
-    if ((w % P) == 0) put_sz(t, w / P, gp.d16, gp.m16);
+    const GroupParams gp = group_params(mn, mx, BITS);
+    if constexpr (CODES) put_word(t0 + t, w, quant_word_rcp<BITS, PER>(x, gp.m, gp.d, __frcp_rn(gp.d)));
+    if ((w % P) == 0) put_sz(t0 + t, w / P, gp);
   }
 }
 
-// grid (max flush blocks, batch, Hkv); block kQuantThreads; dynamic smem
-// 2*G*D*2 bytes (ROT: 2*G*D*4). ROT: every token's key and value head vector
-// is multiplied by the normalized Sylvester Hadamard matrix (rotate_lane:
-// radix-2 butterflies of half-width 1, 2, 4, ..., then one fp32
-// multiplication by fp32(1/sqrt(D))) and staged as fp32 before the block is
-// quantized ("KV1-1.2B" card, BQ2_0).
-template <bool ROT>
-__global__ void __launch_bounds__(kQuantThreads) quantize_blocks_kernel(AppendParams p) {
-  const int j = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
-  if (j >= p.flush[b]) return;
-  const LayerView& L = p.L;
-  const int G = L.group_k, D = L.head_dim, R = L.residual;
-  const int kb = L.k_bits, vb = L.v_bits, Gv = L.group_v;
-  const int dt = L.kv_dtype;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  uint16_t* sk = reinterpret_cast<uint16_t*>(smem_raw);  // [G][D] raw (not ROT)
-  uint16_t* sv = sk + G * D;
-  float* fk = reinterpret_cast<float*>(smem_raw);  // [G][D] fp32 (ROT)
-  float* fv = fk + G * D;
+// Key codes packed along the token axis (kc layout) for channels [c0, c0+nc)
+// and token words [w0, w0 + nw): thread item (channel d, word w) packs
+// tokens w*PER .. w*PER+PER-1 of channel d (staged row of token t at t - t0,
+// column d - sc0) with the fp32 (scale, zero, 1/scale) par(t, d).
+template <bool ROT, int KB, bool PT, class Par>
+__device__ __forceinline__ void pack_key_codes(const uint8_t* rows, int pitch, int t0, int sc0, int c0, int nc, int w0,
+                                               int nw, int lgW, int dt, uint32_t* kc, Par par) {
+  constexpr int PER = 32 / KB;
+  for (int item = threadIdx.x; item < nc * nw; item += kQuantThreads) {
+    const int d = c0 + item % nc, w = w0 + item / nc;
+    float x[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) x[i] = staged<ROT>(rows, pitch, w * PER + i - t0, d - sc0, dt);
+    uint32_t word;
+    if constexpr (PT) {  // per-token keys: each token has its own (scale, zero)
+      word = 0;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const float4 pr = par(w * PER + i, d);
+        float xi[1] = {x[i]};
+        word |= quant_word_rcp<KB, 1>(xi, pr.y, pr.x, pr.z) << (i * KB);
+      }
+    } else {  // per-channel keys: one (scale, zero) for the channel
+      const float4 pr = par(0, d);
+      word = quant_word_rcp<KB, PER>(x, pr.y, pr.x, pr.z);
+    }
+    kc[kc_index_p2(d, w, lgW)] = word;
+  }
+}
 
-  const int first = p.q_old[b] + j * G;  // position of the block's first token (after the sinks)
-  const int boundary = p.q_old[b] + p.n_old[b];
-  const int64_t ring_base = ((int64_t)b * L.num_kv_heads + h) * R;
-  // Row t of the block (token first + t) of the keys or the values: in the
-  // ring, or in this call's input.
-  auto row_ptr = [&](int t, bool value) -> const uint16_t* {
-    const int i = first + t;
-    if (i < boundary)
-      return reinterpret_cast<const uint16_t*>(value ? L.ring_v : L.ring_k) + (ring_base + i % R) * D;
-    const int64_t row = (int64_t)p.in_off[b] + (i - boundary);
-    return reinterpret_cast<const uint16_t*>(value ? p.v_in : p.k_in) + (row * L.num_kv_heads + h) * D;
-  };
-  if constexpr (ROT) {
-    // one warp per row of G keys then G values, 4 channels per lane, rotated
-    // in registers (D = 128)
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int row = warp; row < 2 * G; row += kQuantThreads / 32) {
-      const bool value = row >= G;
-      const int t = value ? row - G : row;
-      const uint2 raw = *reinterpret_cast<const uint2*>(row_ptr(t, value) + 4 * lane);
-      float x[4] = {bits_to_float(raw.x & 0xffffu, dt), bits_to_float(raw.x >> 16, dt),
-                    bits_to_float(raw.y & 0xffffu, dt), bits_to_float(raw.y >> 16, dt)};
-      rotate_lane(x, lane);
-      *reinterpret_cast<float4*>((value ? fv : fk) + t * D + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
+// Keys per channel (KIVI): channels [c0, c0 + nc) over all G tokens; the
+// min/max of every (channel, word-slice) item, combined through shared
+// memory, then the codes.
+template <bool ROT, int KB>
+__device__ __forceinline__ void quantize_key_channels(const uint8_t* rows, const PartShape& s, int G, int dt,
+                                                      uint8_t* rec, const LayerView& L, float2* red, float4* kpar) {
+  constexpr int PER = 32 / KB;
+  const int W = G / PER, lgW = __ffs(W) - 1;
+  for (int item = threadIdx.x; item < s.nc * W; item += kQuantThreads) {
+    const int dl = item % s.nc, w = item / s.nc;
+    const int col = s.c0 + dl - s.sc0;
+    float mn = staged<ROT>(rows, s.snc, w * PER, col, dt), mx = mn;
+#pragma unroll 4
+    for (int i = 1; i < PER; ++i) {
+      const float x = staged<ROT>(rows, s.snc, w * PER + i, col, dt);
+      mn = fminf(mn, x);
+      mx = fmaxf(mx, x);
     }
-  } else {
-    // Stage the G x D block, 8 values (16 bytes) per load.
-    const int vec_per_tok = D / 8;
-    for (int idx = threadIdx.x; idx < G * vec_per_tok; idx += blockDim.x) {
-      const int t = idx / vec_per_tok, c = (idx % vec_per_tok) * 8;
-      *reinterpret_cast<uint4*>(sk + t * D + c) = *reinterpret_cast<const uint4*>(row_ptr(t, false) + c);
-      *reinterpret_cast<uint4*>(sv + t * D + c) = *reinterpret_cast<const uint4*>(row_ptr(t, true) + c);
-    }
+    red[w * s.nc + dl] = make_float2(mn, mx);
   }
   __syncthreads();
-  auto kval = [&](int t, int d) -> float {
-    if constexpr (ROT) return fk[t * D + d];
-    else return bits_to_float(sk[t * D + d], dt);
-  };
-  auto vval = [&](int t, int d) -> float {
-    if constexpr (ROT) return fv[t * D + d];
-    else return bits_to_float(sv[t * D + d], dt);
-  };
-
-  uint8_t* rec = record_ptr(L, b, h, p.q_old[b] / G + j);
-  uint32_t* kc = reinterpret_cast<uint32_t*>(rec + L.kc_off);
   __half2* ksz = reinterpret_cast<__half2*>(rec + L.ksz_off);
+  for (int dl = threadIdx.x; dl < s.nc; dl += kQuantThreads) {
+    float mn = INFINITY, mx = -INFINITY;
+    for (int w = 0; w < W; ++w) {
+      const float2 r = red[w * s.nc + dl];
+      mn = fminf(mn, r.x);
+      mx = fmaxf(mx, r.y);
+    }
+    const GroupParams gp = group_params(mn, mx, KB);
+    ksz[s.c0 + dl] = __halves2half2(gp.d16, gp.m16);
+    kpar[dl] = make_float4(gp.d, gp.m, __frcp_rn(gp.d), 0.f);
+  }
+  __syncthreads();
+  pack_key_codes<ROT, KB, false>(rows, s.snc, 0, s.sc0, s.c0, s.nc, 0, W, lgW, dt, reinterpret_cast<uint32_t*>(rec + L.kc_off),
+                          [&](int, int d) { return kpar[d - s.c0]; });
+}
+
+// Keys per token over group_v channels (BQ2_0), tokens [t0, t0 + nt): the
+// token groups' scales and zero points, then the codes of those tokens
+// packed along the token axis.
+template <bool ROT, int KB>
+__device__ __forceinline__ void quantize_key_tokens(const uint8_t* rows, const PartShape& s, int G, int dt,
+                                                    uint8_t* rec, const LayerView& L, float4* kpar) {
+  constexpr int PER = 32 / KB;
+  const int ng = kHeadDim / L.group_v, gv = L.group_v;
+  __half2* ksz = reinterpret_cast<__half2*>(rec + L.ksz_off);
+  quantize_token_groups<ROT, KB, false>(rows, s.t0, s.nt, gv, dt, [](int, int, uint32_t) {},
+                                        [&](int t, int g, const GroupParams& gp) {
+                                          ksz[t * ng + g] = __halves2half2(gp.d16, gp.m16);
+                                          kpar[(t - s.t0) * ng + g] = make_float4(gp.d, gp.m, __frcp_rn(gp.d), 0.f);
+                                        });
+  __syncthreads();
+  const int W = G / PER, lgW = __ffs(W) - 1;
+  pack_key_codes<ROT, KB, true>(rows, kHeadDim, s.t0, 0, 0, kHeadDim, s.t0 / PER, s.nt / PER, lgW, dt,
+                          reinterpret_cast<uint32_t*>(rec + L.kc_off),
+                          [&](int t, int d) { return kpar[(t - s.t0) * ng + d / gv]; });
+}
+
+// Values per token over group_v channels (KIVI), tokens [t0, t0 + nt),
+// codes packed along head_dim.
+template <bool ROT, int KB, int VB>
+__device__ __forceinline__ void quantize_value_tokens(const uint8_t* rows, const PartShape& s, int G, int dt,
+                                                      uint8_t* rec, const LayerView& L) {
   uint32_t* vc = reinterpret_cast<uint32_t*>(rec + L.vc_off);
   __half* vsz = reinterpret_cast<__half*>(rec + L.vsz_off);
+  const int ng = kHeadDim / L.group_v;
+  constexpr int VW = kHeadDim * VB / 32;
+  quantize_token_groups<ROT, VB, true>(rows, s.t0, s.nt, L.group_v, dt,
+                                       [&](int t, int w, uint32_t word) { vc[vc_word_index(t, w, G, KB, VW)] = word; },
+                                       [&](int t, int g, const GroupParams& gp) {
+                                         vsz[vsz_half_index(t, g, G, KB, ng, false)] = gp.d16;
+                                         vsz[vsz_half_index(t, g, G, KB, ng, true)] = gp.m16;
+                                       });
+}
 
-  if (L.k_axis == 0) {
-    // Keys: one group per channel over the G tokens (KIVI: per-channel keys).
-    for (int d = threadIdx.x; d < D; d += blockDim.x) {
-      float mn = kval(0, d), mx = mn;
-      for (int t = 1; t < G; ++t) {
-        const float x = kval(t, d);
-        mn = fminf(mn, x);
-        mx = fmaxf(mx, x);
-      }
-      const GroupParams gp = group_params(mn, mx, kb);
-      ksz[d] = __halves2half2(gp.d16, gp.m16);
-      const int per = 32 / kb;
-      const int nw = G / per;  // words per channel, stored contiguously
-      for (int w = 0; w < nw; ++w) {
-        uint32_t word = 0;
-        for (int i = 0; i < per; ++i) word |= quant_code(kval(w * per + i, d), gp, kb) << (i * kb);
-        kc[kc_word_index(d, w, nw)] = word;
-      }
-    }
-  } else {
-    // Keys per token (BQ2_0), grouped like values over group_v channels:
-    // (scale, zero) pairs [G][D/group_v] row-major, then the codes packed
-    // along the token axis in the per-channel key layout, so that the decode
-    // kernels read both key axes' codes the same way.
-    __shared__ __half2 s_ksz[128 * 4];  // G <= 128 tokens x D/group_v <= 4 groups
-    const int ng = D / Gv;
-    quantize_rows(G, D, kb, Gv, kval, [](int, int, uint32_t) {}, [&](int t, int g, __half d16, __half m16) {
-      ksz[t * ng + g] = s_ksz[t * ng + g] = __halves2half2(d16, m16);
-    });
-    __syncthreads();  // the pairs just stored are read back below
-    const int per = 32 / kb, nw = G / per;
-    for (int idx = threadIdx.x; idx < D * nw; idx += blockDim.x) {
-      const int d = idx / nw, w = idx % nw;
-      uint32_t word = 0;
-      for (int i = 0; i < per; ++i) {
-        const int t = w * per + i;
-        const __half2 sz = s_ksz[t * ng + d / Gv];
-        GroupParams gp;
-        gp.d16 = __low2half(sz);
-        gp.m16 = __high2half(sz);
-        gp.d = __half2float(gp.d16);
-        gp.m = __half2float(gp.m16);
-        word |= quant_code(kval(t, d), gp, kb) << (i * kb);
-      }
-      kc[kc_word_index(d, w, nw)] = word;
-    }
+// One part CTA: stages its rows, then quantizes keys (record jk) or values
+// (record jv). ROT: the rows are multiplied by the normalized Sylvester
+// Hadamard matrix first (rotate_lane: radix-2 butterflies of half-width 1,
+// 2, 4, ..., then one fp32 multiply by fp32(1/sqrt(D)); "KV1-1.2B" card,
+// BQ2_0).
+template <bool ROT, int KB>
+__device__ __forceinline__ void quantize_key_part(const LayerView& L, int b, int h, int64_t jk, const BlockRows& src,
+                                                  const PartShape& s, uint8_t* smem) {
+  const int G = L.group_k, dt = L.kv_dtype;
+  const QuantSmem sm = part_smem(s, G, KB, L.group_v, L.k_axis, ROT);
+  if constexpr (ROT) stage_rotated(src, s.t0, s.nt, dt, reinterpret_cast<float*>(smem));
+  else stage_raw(src, s.t0, s.nt, s.sc0, s.snc, reinterpret_cast<uint16_t*>(smem));
+  __syncthreads();
+  uint8_t* rec = record_ptr(L, b, h, jk);
+  float4* kpar = reinterpret_cast<float4*>(smem + sm.rows + sm.red);
+  if (L.k_axis == 0) quantize_key_channels<ROT, KB>(smem, s, G, dt, rec, L, reinterpret_cast<float2*>(smem + sm.rows), kpar);
+  else quantize_key_tokens<ROT, KB>(smem, s, G, dt, rec, L, kpar);
+}
+
+template <bool ROT, int KB, int VB>
+__device__ __forceinline__ void quantize_value_part(const LayerView& L, int b, int h, int64_t jv, const BlockRows& src,
+                                                    const PartShape& s, uint8_t* smem) {
+  const int G = L.group_k, dt = L.kv_dtype;
+  if constexpr (ROT) stage_rotated(src, s.t0, s.nt, dt, reinterpret_cast<float*>(smem));
+  else stage_raw(src, s.t0, s.nt, 0, kHeadDim, reinterpret_cast<uint16_t*>(smem));
+  __syncthreads();
+  quantize_value_tokens<ROT, KB, VB>(smem, s, G, dt, record_ptr(L, b, h, jv), L);
+}
+
+// Part `part` of `parts` of the key block jk (key) or the value block jv of
+// (sequence b, KV head h), rows from src.
+template <bool ROT>
+__device__ __forceinline__ void quantize_part(const LayerView& L, int b, int h, bool key, int part, int parts,
+                                              int64_t j, const BlockRows& src, uint8_t* smem) {
+  const PartShape s = part_shape(key, part, parts, L.group_k, L.k_axis, ROT);
+  if (key) {
+    if (L.k_bits == 2) quantize_key_part<ROT, 2>(L, b, h, j, src, s, smem);
+    else if (L.k_bits == 4) quantize_key_part<ROT, 4>(L, b, h, j, src, s, smem);
+    else quantize_key_part<ROT, 8>(L, b, h, j, src, s, smem);
+    return;
   }
+#define KVQ_VPART(K, V) \
+  if (L.k_bits == K && L.v_bits == V) return quantize_value_part<ROT, K, V>(L, b, h, j, src, s, smem);
+  KVQ_VPART(2, 2) KVQ_VPART(2, 4) KVQ_VPART(2, 8) KVQ_VPART(4, 2) KVQ_VPART(4, 4) KVQ_VPART(4, 8)
+  KVQ_VPART(8, 2) KVQ_VPART(8, 4) KVQ_VPART(8, 8)
+#undef KVQ_VPART
+}
 
-  // Values: one group per group_v channels of a token (KIVI: per-token values).
-  const int vwpt = D * vb / 32;
-  quantize_rows(G, D, vb, Gv, vval,
-                [&](int t, int w, uint32_t word) { vc[vc_word_index(t, w, G, kb, vwpt)] = word; },
-                [&](int t, int g, __half d16, __half m16) {
-                  vsz[vsz_half_index(t, g, G, kb, D / Gv, false)] = d16;
-                  vsz[vsz_half_index(t, g, G, kb, D / Gv, true)] = m16;
-                });
+}  // namespace
+
+cudaError_t opt_in_max_smem(const void* kernel, uint64_t& done_mask);
+
+// grid (max flush blocks * 2, batch, Hkv); block kQuantThreads; dynamic smem
+// quant_smem_bytes(..., 1). x = 2j + tensor: key block j of sequence b
+// covers positions q_old[b] + j*G .., value block j positions qv_old[b] +
+// j*G ..: ring tokens before the call's first new token, this call's input
+// after.
+template <bool ROT>
+__global__ void __launch_bounds__(kQuantThreads, 6) quantize_blocks_kernel(AppendParams p) {
+  const int j = blockIdx.x >> 1, b = blockIdx.y, h = blockIdx.z;
+  const bool key = (blockIdx.x & 1) == 0;
+  if (j >= (key ? p.flush[b] : p.flush_v[b])) return;
+  extern __shared__ __align__(16) uint8_t smem_q[];
+  const LayerView& L = p.L;
+  const int G = L.group_k;
+  const int64_t unit = (int64_t)b * L.num_kv_heads + h;
+  const int R = key ? L.residual : L.residual_v;
+  const BlockRows src{reinterpret_cast<const uint16_t*>(key ? L.ring_k : L.ring_v) + unit * R * kHeadDim,
+                      reinterpret_cast<const uint16_t*>(key ? p.k_in : p.v_in), p.in_off[b],
+                      (key ? p.q_old[b] : p.qv_old[b]) + j * G, p.len_old[b], R, L.num_kv_heads, h};
+  quantize_part<ROT>(L, b, h, key, 0, 1, (key ? p.q_old[b] : p.qv_old[b]) / G + j, src, smem_q);
+}
+
+// grid (batch * Hkv * 2 * kStepParts); block kQuantThreads. The flush of a
+// fused decode step: for (sequence, KV head) whose ring holds R tokens, the
+// oldest G ring tokens become the next block record (one ring shared by keys
+// and values); CTA x = ((b * Hkv + h) * 2 + tensor) * kStepParts + part. The
+// decode launch that follows is its programmatic dependent and waits for it
+// (griddepcontrol.wait) before reading records; the decode kernel records
+// the new lengths.
+template <bool ROT>
+__global__ void __launch_bounds__(kQuantThreads, 6) step_flush_kernel(FlushParams p) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  extern __shared__ __align__(16) uint8_t smem_q[];
+  const LayerView& L = p.L;
+  const int part = blockIdx.x % kStepParts;
+  const bool key = ((blockIdx.x / kStepParts) & 1) == 0;
+  const int unit_i = blockIdx.x / (2 * kStepParts);
+  const int b = unit_i / L.num_kv_heads, h = unit_i % L.num_kv_heads;
+  const int32_t* len = L.lens + (int64_t)b * kLensStride;
+  const int q = len[kLenQ], n = len[kLenN];
+  if (n != L.residual) return;
+  const int64_t unit = (int64_t)b * L.num_kv_heads + h;
+  const BlockRows src{reinterpret_cast<const uint16_t*>(key ? L.ring_k : L.ring_v) + unit * L.residual * kHeadDim,
+                      nullptr, 0, q, q + n, L.residual, L.num_kv_heads, h};
+  quantize_part<ROT>(L, b, h, key, part, kStepParts, q / L.group_k, src, smem_q);
+}
+
+cudaError_t launch_step_flush(const FlushParams& p, cudaStream_t stream) {
+  const LayerView& L = p.L;
+  const bool rot = L.hadamard != 0;
+  const int smem = quant_smem_bytes(L.group_k, L.k_bits, L.group_v, L.k_axis, rot, kStepParts);
+  static uint64_t done_rot = 0, done_raw = 0;
+  cudaError_t e = rot ? opt_in_max_smem(reinterpret_cast<const void*>(step_flush_kernel<true>), done_rot)
+                      : opt_in_max_smem(reinterpret_cast<const void*>(step_flush_kernel<false>), done_raw);
+  if (e != cudaSuccess) return e;
+  const int grid = p.ctas * 2 * kStepParts;
+  if (rot) step_flush_kernel<true><<<grid, kQuantThreads, smem, stream>>>(p);
+  else step_flush_kernel<false><<<grid, kQuantThreads, smem, stream>>>(p);
+  return cudaGetLastError();
 }
 
 // grid (batch, Hkv); copies this call's sink tokens to the sinks and its
-// unflushed new tokens into the ring, and records the new lengths.
+// tokens that stay exact into the key and value rings, and records the new
+// lengths.
 __global__ void ring_write_kernel(AppendParams p) {
   const int b = blockIdx.x, h = blockIdx.y;
   const LayerView& L = p.L;
-  const int G = L.group_k, D = L.head_dim, R = L.residual;
-  const int boundary = p.q_old[b] + p.n_old[b];
+  const int G = L.group_k, D = L.head_dim;
+  const int boundary = p.len_old[b];
   const int q_new = p.q_old[b] + p.flush[b] * G;
+  const int qv_new = p.qv_old[b] + p.flush_v[b] * G;
   const int end = boundary + p.t_new[b];
-  const int first = max(boundary, q_new);
   const int vec_per_tok = D / 8;
   const int ns = p.s_take[b];
-  const int64_t sink_base = ((int64_t)b * L.num_kv_heads + h) * KVQ_MAX_SINKS + p.s_old[b];
+  const int64_t unit = (int64_t)b * L.num_kv_heads + h;
+  const int64_t sink_base = unit * KVQ_MAX_SINKS + p.s_old[b];
   for (int idx = threadIdx.x; idx < ns * vec_per_tok; idx += blockDim.x) {
     const int i = idx / vec_per_tok, c = (idx % vec_per_tok) * 8;
     const int64_t row = (int64_t)p.in_off[b] - ns + i;
@@ -203,21 +446,41 @@ __global__ void ring_write_kernel(AppendParams p) {
     *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(L.sink_v) + dst) =
         *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.v_in) + src);
   }
-  const int64_t ring_base = ((int64_t)b * L.num_kv_heads + h) * R;
-  for (int idx = threadIdx.x; idx < (end - first) * vec_per_tok; idx += blockDim.x) {
-    const int i = first + idx / vec_per_tok, c = (idx % vec_per_tok) * 8;
-    const int64_t row = (int64_t)p.in_off[b] + (i - boundary);
-    const int64_t src = (row * L.num_kv_heads + h) * D + c;
-    const int64_t dst = (ring_base + i % R) * D + c;
-    *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(L.ring_k) + dst) =
-        *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.k_in) + src);
-    *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(L.ring_v) + dst) =
-        *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.v_in) + src);
+  // keys from max(boundary, q_new), values from max(boundary, qv_new); each
+  // thread issues the loads of up to 4 chunks before their stores
+  const int first_k = max(boundary, q_new), first_v = max(boundary, qv_new);
+  const int first = min(first_k, first_v);
+  const int total = (end - first) * vec_per_tok;
+  const uint16_t* kin = reinterpret_cast<const uint16_t*>(p.k_in);
+  const uint16_t* vin = reinterpret_cast<const uint16_t*>(p.v_in);
+  uint16_t* rk = reinterpret_cast<uint16_t*>(L.ring_k);
+  uint16_t* rv = reinterpret_cast<uint16_t*>(L.ring_v);
+  for (int base = threadIdx.x; base < total; base += 4 * blockDim.x) {
+    uint4 tk[4], tv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * blockDim.x;
+      if (idx >= total) break;
+      const int i = first + idx / vec_per_tok, c = (idx % vec_per_tok) * 8;
+      const int64_t src = (((int64_t)p.in_off[b] + (i - boundary)) * L.num_kv_heads + h) * D + c;
+      if (i >= first_k) tk[u] = *reinterpret_cast<const uint4*>(kin + src);
+      if (i >= first_v) tv[u] = *reinterpret_cast<const uint4*>(vin + src);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * blockDim.x;
+      if (idx >= total) break;
+      const int i = first + idx / vec_per_tok, c = (idx % vec_per_tok) * 8;
+      if (i >= first_k) *reinterpret_cast<uint4*>(rk + (unit * L.residual + i % L.residual) * D + c) = tk[u];
+      if (i >= first_v) *reinterpret_cast<uint4*>(rv + (unit * L.residual_v + i % L.residual_v) * D + c) = tv[u];
+    }
   }
   if (h == 0 && threadIdx.x == 0) {
-    L.lens[3 * b] = q_new;
-    L.lens[3 * b + 1] = end - q_new;
-    L.lens[3 * b + 2] = p.s_old[b] + ns;
+    int32_t* len = L.lens + (int64_t)b * kLensStride;
+    len[kLenQ] = q_new;
+    len[kLenN] = end - q_new;
+    len[kLenS] = p.s_old[b] + ns;
+    len[kLenQV] = qv_new;
   }
 }
 
@@ -226,35 +489,38 @@ __global__ void ring_write_kernel(AppendParams p) {
 __global__ void dequant_kernel(LayerView L, int seq, int sinks, int t0, int n, float* k_out, float* v_out) {
   const int h = blockIdx.y;
   const int d = threadIdx.x;
-  const int G = L.group_k, D = L.head_dim, R = L.residual;
-  const int Q = L.lens[3 * seq];
+  const int G = L.group_k, D = L.head_dim;
+  const int Q = L.lens[(int64_t)seq * kLensStride + kLenQ];
+  const int QV = L.lens[(int64_t)seq * kLensStride + kLenQV];
   const int kb = L.k_bits, vb = L.v_bits;
+  const int64_t unit = (int64_t)seq * L.num_kv_heads + h;
   for (int r = 0; r < 8; ++r) {
     const int i = blockIdx.x * 8 + r;
     if (i >= n || d >= D) continue;
     const int64_t o = ((int64_t)i * L.num_kv_heads + h) * D + d;
     if (t0 + i < sinks) {
-      const int64_t src = (((int64_t)seq * L.num_kv_heads + h) * KVQ_MAX_SINKS + t0 + i) * D + d;
+      const int64_t src = (unit * KVQ_MAX_SINKS + t0 + i) * D + d;
       k_out[o] = load_kv(L.sink_k, src, L.kv_dtype);
       v_out[o] = load_kv(L.sink_v, src, L.kv_dtype);
       continue;
     }
     const int tok = t0 + i - sinks;  // position after the sinks
+    const int t = tok % G;
     if (tok < Q) {
       const uint8_t* rec = record_ptr(L, seq, h, tok / G);
-      const int t = tok % G;
       const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + L.kc_off);
       const int kper = 32 / kb;
-      __half2 ksz;
-      uint32_t kw;
-      if (L.k_axis == 0) {
-        ksz = reinterpret_cast<const __half2*>(rec + L.ksz_off)[d];
-        kw = kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb);
-      } else {  // per-token keys: (scale, zero) per (token, channel group), codes as above
-        ksz = reinterpret_cast<const __half2*>(rec + L.ksz_off)[t * (D / L.group_v) + d / L.group_v];
-        kw = kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb);
-      }
+      const __half2 ksz = L.k_axis == 0
+                              ? reinterpret_cast<const __half2*>(rec + L.ksz_off)[d]
+                              // per-token keys: (scale, zero) per (token, channel group)
+                              : reinterpret_cast<const __half2*>(rec + L.ksz_off)[t * (D / L.group_v) + d / L.group_v];
+      const uint32_t kw = kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb);
       k_out[o] = dequant_value(kw & ((1u << kb) - 1), __low2half(ksz), __high2half(ksz));
+    } else {
+      k_out[o] = load_kv(L.ring_k, (unit * L.residual + tok % L.residual) * D + d, L.kv_dtype);
+    }
+    if (tok < QV) {
+      const uint8_t* rec = record_ptr(L, seq, h, tok / G);
       const uint32_t* vc = reinterpret_cast<const uint32_t*>(rec + L.vc_off);
       const int vper = 32 / vb;
       const uint32_t vq = (vc[vc_word_index(t, d / vper, G, kb, D / vper)] >> ((d % vper) * vb)) & ((1u << vb) - 1);
@@ -262,39 +528,50 @@ __global__ void dequant_kernel(LayerView L, int seq, int sinks, int t0, int n, f
       const int ng = D / L.group_v, gg = d / L.group_v;
       v_out[o] = dequant_value(vq, vsz[vsz_half_index(t, gg, G, kb, ng, false)], vsz[vsz_half_index(t, gg, G, kb, ng, true)]);
     } else {
-      const int64_t src = (((int64_t)seq * L.num_kv_heads + h) * R + tok % R) * D + d;
-      k_out[o] = load_kv(L.ring_k, src, L.kv_dtype);
-      v_out[o] = load_kv(L.ring_v, src, L.kv_dtype);
+      v_out[o] = load_kv(L.ring_v, (unit * L.residual_v + tok % L.residual_v) * D + d, L.kv_dtype);
     }
   }
+}
+
+// Opts a kernel in to the device's largest dynamic shared memory, once per
+// (kernel, device): launches then pass what they use.
+cudaError_t opt_in_max_smem(const void* kernel, uint64_t& done_mask) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && (done_mask & (1ull << dev))) return cudaSuccess;
+  int optin = 0;
+  cudaFuncAttributes fa;
+  e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, kernel);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes);
+  if (e == cudaSuccess && dev < 64) done_mask |= 1ull << dev;
+  return e;
+}
+
+cudaError_t launch_quantize(const AppendParams& p, int max_flush, cudaStream_t stream) {
+  const LayerView& L = p.L;
+  const bool rot = L.hadamard != 0;
+  const int smem = quant_smem_bytes(L.group_k, L.k_bits, L.group_v, L.k_axis, rot, 1);
+  static uint64_t done_rot = 0, done_raw = 0;
+  cudaError_t e = rot ? opt_in_max_smem(reinterpret_cast<const void*>(quantize_blocks_kernel<true>), done_rot)
+                      : opt_in_max_smem(reinterpret_cast<const void*>(quantize_blocks_kernel<false>), done_raw);
+  if (e != cudaSuccess) return e;
+  dim3 grid(2 * max_flush, p.batch, L.num_kv_heads);
+  if (rot) quantize_blocks_kernel<true><<<grid, kQuantThreads, smem, stream>>>(p);
+  else quantize_blocks_kernel<false><<<grid, kQuantThreads, smem, stream>>>(p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_append(const AppendParams& p, int max_flush, cudaStream_t stream) {
   const LayerView& L = p.L;
   if (max_flush > 0) {
-    const bool rot = L.hadamard != 0;
-    const size_t smem = (size_t)2 * L.group_k * L.head_dim * (rot ? sizeof(float) : sizeof(uint16_t));
-    // The shared-memory opt-in is per function and per device.
-    static uint64_t attr_set_mask[2] = {0, 0};
-    int dev = 0;
-    cudaError_t e0 = cudaGetDevice(&dev);
-    if (e0 != cudaSuccess) return e0;
-    if (dev >= 64 || !(attr_set_mask[rot] & (1ull << dev))) {
-      e0 = rot ? cudaFuncSetAttribute(quantize_blocks_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      2 * 128 * kHeadDim * (int)sizeof(float))
-               : cudaFuncSetAttribute(quantize_blocks_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      2 * 128 * kHeadDim * (int)sizeof(uint16_t));
-      if (e0 != cudaSuccess) return e0;
-      if (dev < 64) attr_set_mask[rot] |= 1ull << dev;
-    }
-    dim3 grid(max_flush, p.batch, L.num_kv_heads);
-    if (rot) quantize_blocks_kernel<true><<<grid, kQuantThreads, smem, stream>>>(p);
-    else quantize_blocks_kernel<false><<<grid, kQuantThreads, smem, stream>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_quantize(p, max_flush, stream);
     if (e != cudaSuccess) return e;
   }
   dim3 grid2(p.batch, L.num_kv_heads);
-  ring_write_kernel<<<grid2, 128, 0, stream>>>(p);
+  ring_write_kernel<<<grid2, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

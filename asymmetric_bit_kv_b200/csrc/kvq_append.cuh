@@ -5,24 +5,30 @@
 
 namespace kvq {
 
-constexpr int kQuantThreads = 128;
+constexpr int kQuantThreads = 256;
 
 // Per-call append plan, passed by value (kernel parameter space up to 32 KB).
-// Lengths are the host mirror's values before the call.
+// Lengths are the host mirror's values before the call, as token positions
+// after the sinks. Keys and values flush on their own (each tensor has its
+// own ring); with one residual length their plans coincide.
 struct AppendParams {
   LayerView L;
   const void* k_in;  // [sum t_new][Hkv][D], kv dtype
   const void* v_in;
   int32_t batch;
-  int32_t q_old[KVQ_MAX_BATCH];   // quantized tokens before the call
-  int32_t n_old[KVQ_MAX_BATCH];   // ring tokens before the call
-  int32_t t_new[KVQ_MAX_BATCH];   // tokens appended by the call after the sinks
-  int32_t in_off[KVQ_MAX_BATCH];  // first input row of each sequence after its sinks
-  int32_t flush[KVQ_MAX_BATCH];   // G-token blocks quantized by the call
-  int32_t s_old[KVQ_MAX_BATCH];   // sink tokens before the call
-  int32_t s_take[KVQ_MAX_BATCH];  // sink tokens taken by the call (input rows in_off - s_take ..)
+  int32_t q_old[KVQ_MAX_BATCH];    // quantized keys before the call
+  int32_t qv_old[KVQ_MAX_BATCH];   // quantized values before the call
+  int32_t len_old[KVQ_MAX_BATCH];  // tokens before the call (quantized keys + key ring)
+  int32_t t_new[KVQ_MAX_BATCH];    // tokens appended by the call after the sinks
+  int32_t in_off[KVQ_MAX_BATCH];   // first input row of each sequence after its sinks
+  int32_t flush[KVQ_MAX_BATCH];    // G-token key blocks quantized by the call
+  int32_t flush_v[KVQ_MAX_BATCH];  // G-token value blocks quantized by the call
+  int32_t s_old[KVQ_MAX_BATCH];    // sink tokens before the call
+  int32_t s_take[KVQ_MAX_BATCH];   // sink tokens taken by the call (input rows in_off - s_take ..)
 };
 
+// Enqueues the quantize kernel (max_flush = the largest key or value block
+// count of any sequence; none if 0) and the ring / sink / length-table write.
 cudaError_t launch_append(const AppendParams& p, int max_flush, cudaStream_t stream);
 
 // Paged caches: page-table entries set by one launch (table[idx[i]] =

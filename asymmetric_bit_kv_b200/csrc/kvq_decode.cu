@@ -83,9 +83,13 @@ template <int NG>
 __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p) {
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const LayerView& L = p.L;
-  const int G = L.group_k, R = L.residual;
-  const int Q = L.lens[3 * b], n = L.lens[3 * b + 1], nsink = L.lens[3 * b + 2];
-  const int nblk = Q / G;
+  const int G = L.group_k, R = L.residual, RV = L.residual_v;
+  const int32_t* len = L.lens + (int64_t)b * kLensStride;
+  const int Q = len[kLenQ], n = len[kLenN], nsink = len[kLenS], QV = len[kLenQV];
+  // blocks with a quantized key or value part; a block below one boundary
+  // and above the other reads that tensor's tokens from its ring (separate
+  // residual lengths for keys and values)
+  const int QM = max(Q, QV), nblk = QM / G;
   const int bps = p.blocks_per_split;
   const int S = (nblk + bps - 1) / bps;
   if (s > S) return;
@@ -129,24 +133,26 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
 
   if (s == 0) {
     // Sinks and the residual ring: exact stored values.
-    const int64_t sbase = ((int64_t)b * L.num_kv_heads + h) * KVQ_MAX_SINKS;
-    const int64_t base = ((int64_t)b * L.num_kv_heads + h) * R;
-    for (int e = warp; e < nsink + n; e += 4) {
-      // e < nsink: sink e; otherwise the ring token at position Q + e - nsink
+    const int64_t unit = (int64_t)b * L.num_kv_heads + h;
+    const int nx = Q + n - QM;  // tokens exact in both tensors
+    for (int e = warp; e < nsink + nx; e += 4) {
+      // e < nsink: sink e; otherwise the token at position QM + e - nsink
       const bool sink = e < nsink;
-      const int64_t row = (sink ? sbase + e : base + (Q + e - nsink) % R) * D;
+      const int i = QM + e - nsink;
+      const int64_t krow = sink ? (unit * KVQ_MAX_SINKS + e) * D : (unit * R + i % R) * D;
+      const int64_t vrow = sink ? (unit * KVQ_MAX_SINKS + e) * D : (unit * RV + i % RV) * D;
       const void* ksrc = sink ? L.sink_k : L.ring_k;
       const void* vsrc = sink ? L.sink_v : L.ring_v;
       float kv[4], vv[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        kv[c] = load_kv(ksrc, row + lane + 32 * c, L.kv_dtype);
-        vv[c] = load_kv(vsrc, row + lane + 32 * c, L.kv_dtype);
+        kv[c] = load_kv(ksrc, krow + lane + 32 * c, L.kv_dtype);
+        vv[c] = load_kv(vsrc, vrow + lane + 32 * c, L.kv_dtype);
       }
 #pragma unroll
       for (int hh = 0; hh < NG; ++hh) {
-        // query token hh / ngr does not see the ring's last lag_base - hh / ngr tokens
-        if (!sink && e - nsink >= n - (p.lag_base - hh / ngr)) continue;
+        // query token hh / ngr does not see the sequence's last lag_base - hh / ngr tokens
+        if (!sink && i - Q >= n - (p.lag_base - hh / ngr)) continue;
         float part = 0.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) part += sq[hh][lane + 32 * c] * kv[c];
@@ -158,8 +164,49 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
     const int kper = 32 / kb;
     const uint32_t kmask = (1u << kb) - 1;
     const int j0 = (s - 1) * bps, j1 = min(s * bps, nblk);
+    const int64_t unit = (int64_t)b * L.num_kv_heads + h;
     for (int j = j0; j < j1; ++j) {
       const uint8_t* rec = record_ptr(L, b, h, j);
+      if (j * G >= Q || j * G >= QV) {
+        // keys or values of this block still exact, in their ring (never
+        // with the rotation: a rotated cache has one residual length)
+        const bool kq = j * G < Q, vq = j * G < QV;
+        const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + L.kc_off);
+        const int ng = D / Gv;
+#pragma unroll 1
+        for (int t = warp; t < G; t += 4) {
+          const int i = j * G + t;
+          float kv[4], vv[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int d = lane + 32 * c;
+            if (kq) {
+              const __half2 sz = L.k_axis == 1 ? reinterpret_cast<const __half2*>(rec + L.ksz_off)[t * ng + d / Gv]
+                                               : reinterpret_cast<const __half2*>(rec + L.ksz_off)[d];
+              const uint32_t kq2 = (kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb)) & kmask;
+              kv[c] = dequant_value(kq2, __low2half(sz), __high2half(sz));
+            } else {
+              kv[c] = load_kv(L.ring_k, (unit * R + i % R) * D + d, L.kv_dtype);
+            }
+          }
+          if (vq) {
+            token_values(L, rec, t, lane, vv);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) vv[c] = load_kv(L.ring_v, (unit * RV + i % RV) * D + lane + 32 * c, L.kv_dtype);
+          }
+#pragma unroll
+          for (int hh = 0; hh < NG; ++hh) {
+            // a multi-token launch hides the newest tokens from earlier query tokens
+            if (i - Q >= n - (p.lag_base - hh / ngr)) continue;
+            float part = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) part += sq[hh][lane + 32 * c] * kv[c];
+            st.update(hh, warp_sum(part), vv);
+          }
+        }
+        continue;
+      }
       if (L.k_axis == 1) {
         // per-token keys (BQ2_0): dequantize each key and dot it with q
         const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + L.kc_off);
@@ -273,7 +320,8 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineParams p) {
     const int h = hq / (p.num_q_heads / p.num_kv_heads);
     S = __ldcg(p.unit_slots + b * p.num_kv_heads + h);
   } else {
-    const int nblk = p.lens[3 * b] / p.group_k;
+    const int32_t* len = p.lens + (int64_t)b * kLensStride;
+    const int nblk = max(len[kLenQ], len[kLenQV]) / p.group_k;
     S = (nblk + p.blocks_per_split - 1) / p.blocks_per_split + 1;
   }
   const int64_t base = ((int64_t)b * p.num_q_heads + hq) * p.slots;

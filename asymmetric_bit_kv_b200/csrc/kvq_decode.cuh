@@ -14,19 +14,19 @@ namespace kvq {
 //    unit is its quantized blocks followed by its ring tokens in chunks of
 //    kResChunk (one chunk even for an empty sequence); the work items of all
 //    units, concatenated in (sequence, head, item) order, are cut into
-//    num_ctas contiguous ranges of about equal estimated cost (CTA c takes
-//    [cta_start[c], cta_start[c+1]), every range non-empty),
-//    and slot kMmaConsumers*(c - c0) + w holds what warp w of CTA c processed
-//    for the unit, c0 being the unit's first CTA; every warp writes its slot
-//    of every unit its CTA's range touches (zero weight if it had no items).
+//    num_ctas contiguous ranges of equal cost (CTA c takes [cta_start[c],
+//    cta_start[c+1]), every range non-empty; see plan_cta_starts), and slot
+//    kMmaConsumers*(c - c0) + w holds what warp w of CTA c processed for the
+//    unit, c0 being the unit's first CTA; every warp writes its slot of every
+//    unit its CTA's range touches (zero weight if it had no items).
 constexpr int kMaxCtas = 1024;  // persistent mode: CTAs of one decode launch
 
 struct DecodeParams {
   LayerView L;
   const void* q;        // [batch][Hq][D], kv dtype
   void* out;            // [batch][Hq][D], out dtype
-  float* ws_o;          // [max_batch][Hq][slots][D] unnormalised partial outputs
-  float2* ws_ml;        // [max_batch][Hq][slots]: (running max in log2 units, sum)
+  float* ws_o;          // [batch][Hq][slots][D] unnormalised partial outputs
+  float2* ws_ml;        // [batch][Hq][slots]: (running max in log2 units, sum)
   const void* new_k;    // fused decode step: this call's new token per sequence, [batch][Hkv][D]
   const void* new_v;    //   (ring index nres[b] - 1; null: no new token)
   float scale_log2;     // softmax scale * log2(e)
@@ -36,12 +36,13 @@ struct DecodeParams {
   int32_t batch;
   int32_t num_q_heads;
   int32_t blocks_per_split;
-  int32_t slots;        // partial slots per (sequence, query head)
+  int32_t slots;        // partial slots per (sequence, query head): the slot stride
   int32_t* err;         // device word: a kernel sets bit 0 when a bounded wait gave up
   int32_t* unit_slots;  // persistent mode: [batch][Hkv] slot count of each unit, written by the decode kernel
   int32_t persistent;   // 1: persistent-mode slots (see above)
   int32_t total_blocks; // T, persistent mode: work items of all units
   int32_t num_ctas;     // persistent mode
+  int32_t after_flush;  // persistent mode: launched after the flush kernel of a fused decode step
   // Query rows. A unit (sequence b, KV head h) has num_q_heads / Hkv rows:
   // row j is query token t = j / (q_heads / Hkv) of this launch and head
   // h * (q_heads / Hkv) + j % (q_heads / Hkv), read from row
@@ -57,7 +58,7 @@ struct DecodeParams {
   int32_t nres[KVQ_MAX_BATCH];       // ring tokens per sequence (host mirror)
   int32_t nitem[KVQ_MAX_BATCH];      // persistent mode: work items per unit of sequence b
   int32_t seq_start[KVQ_MAX_BATCH];  // first global item (block in split mode) of sequence b
-  int32_t cta_start[kMaxCtas + 1];   // persistent mode: first global item of CTA c (cut by estimated cost)
+  int32_t cta_start[kMaxCtas + 1];   // persistent mode: first global item of CTA c
 };
 
 constexpr int kMmaConsumers = 6;   // warps per CTA of the tensor-core kernel
@@ -83,14 +84,21 @@ __host__ __device__ inline int32_t cta_of_item(const int32_t* starts, int32_t nc
   }
   return lo;
 }
-// Number of partial slots a (sequence, head) unit of nitem >= 1 work items
-// starting at global item unit_start uses in persistent mode.
-__host__ __device__ inline int32_t persistent_slots(const int32_t* starts, int32_t nctas, int32_t unit_start,
-                                                    int32_t nitem) {
-  const int32_t c0 = cta_of_item(starts, nctas, unit_start);
-  const int32_t c1 = cta_of_item(starts, nctas, unit_start + nitem - 1);
-  return kMmaConsumers * (c1 - c0 + 1);
-}
+
+// Cost of a unit's items in half units: a quantized block 2, an exact-token
+// chunk 1. CTA c of N starts at the item whose cost interval holds c*C/N (C:
+// the total cost), so N <= C / (largest item cost) keeps every range
+// non-empty, and a unit of cost u overlaps at most floor(u*N/C) + 2 ranges.
+__host__ __device__ inline int64_t unit_cost(int32_t nblk, int32_t nitem) { return 2 * (int64_t)nblk + (nitem - nblk); }
+
+// Parameters of the flush kernel of a fused decode step: CTA i quantizes,
+// for (sequence i / Hkv, KV head i % Hkv) whose ring holds R tokens, the
+// oldest G ring tokens into the next block record.
+struct FlushParams {
+  LayerView L;
+  int32_t ctas;  // batch * Hkv
+};
+cudaError_t launch_step_flush(const FlushParams& p, cudaStream_t stream);
 
 // Shared-memory plan of the tensor-core decode kernel: per warp nstages
 // stages (a block record exactly as stored, or the key and value rows of a
@@ -129,7 +137,7 @@ struct CombineParams {
   const float2* ws_ml;
   void* out;
   const int32_t* unit_slots;  // persistent mode: slots per unit
-  const int32_t* lens;        // split mode: the layer's length table
+  const int32_t* lens;        // split mode: the layer's length table (kLensStride per sequence)
   int32_t out_dtype, num_q_heads, num_kv_heads, slots, group_k, blocks_per_split, persistent;
   int32_t hadamard;  // split mode: slots >= 1 (quantized tokens) hold rotated partials
   int32_t q_heads, q_rows;  // output row of query row j of a unit: see DecodeParams
@@ -151,12 +159,16 @@ struct QueryGroup {
 };
 
 // Host side of kvq_decode_attention (kvq_api.cu): validation, split plan and
-// launches; the partials go to `scratch` when it is not null; qg: a group of
-// query tokens (null: one query token per sequence).
-kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const void* new_v, const void* q, void* out, int32_t out_dtype,
-                          float softmax_scale, int32_t batch, void* stream, const StaticScratch* scratch,
-                          const QueryGroup* qg = nullptr);
+// launches; the partials (and the slot table) go to `scratch` when it is not
+// null; qg: a group of query tokens (null: one query token per sequence);
+// new_k/new_v: a fused decode step's new tokens; after_flush: the step's
+// flush kernel was enqueued just before.
+kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const void* new_v, const void* q, void* out,
+                          int32_t out_dtype, float softmax_scale, int32_t batch, void* stream,
+                          const StaticScratch* scratch, const QueryGroup* qg = nullptr, bool after_flush = false);
 void clear_last_error();
 kvq_status report_cuda_error(cudaError_t e, const char* what);
+kvq_status report_status(kvq_status s, const char* what);
+int cache_device(const kvq_cache* c);  // the device current when the cache was created
 
 }  // namespace kvq

@@ -64,6 +64,7 @@ bool mma_supported(const LayerView& L, int num_q_heads) {
   if (L.k_axis == 1 && L.group_v != kHeadDim) return false;
   if (L.hadamard && L.k_axis != 1) return false;
   if (L.group_k < 64) return false;                   // tiles of 64 tokens
+  if (L.residual_v != L.residual) return false;       // one ring for keys and values
   if (L.v_bits == 2 && L.group_v < 64) return false;  // a 2-bit value chunk spans 64 channels
   // two stages per warp must fit (8-bit keys in blocks of 128 tokens do not)
   return make_mma_plan(L, num_q_heads).smem_bytes <= smem_limit();

@@ -694,7 +694,7 @@ __device__ __forceinline__ int exact_chunk(const DecodeParams& p, int b, int r, 
   const int nres = p.nres[b];
   sink = false;
   if (r < (nres + kResChunk - 1) / kResChunk) return nres - r * kResChunk;
-  const int nsink = p.L.sinks > 0 ? p.L.lens[3 * b + 2] : 0;
+  const int nsink = p.L.sinks > 0 ? p.L.lens[(int64_t)b * kLensStride + kLenS] : 0;
   sink = nsink > 0;
   return sink ? nsink : nres - r * kResChunk;
 }
@@ -703,7 +703,7 @@ __device__ __forceinline__ int exact_chunk(const DecodeParams& p, int b, int r, 
 // (ring index nres - 1) took that row from the input (issue_item); the warp
 // also stores it into its ring slot for later calls (no other item of this
 // call reads that slot), and the unit of KV head 0 records the sequence's new
-// ring count.
+// lengths.
 __device__ __forceinline__ void store_new_token(const DecodeParams& p, int b, int h, int nb, const uint8_t* stage,
                                                 int lane) {
   const LayerView& L = p.L;
@@ -715,7 +715,12 @@ __device__ __forceinline__ void store_new_token(const DecodeParams& p, int b, in
       reinterpret_cast<const uint2*>(stage + row * kRowBytes)[lane];
   reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(L.ring_v) + dst)[lane] =
       reinterpret_cast<const uint2*>(stage + (kResChunk + row) * kRowBytes)[lane];
-  if (h == 0 && lane == 0) L.lens[3 * b + 1] = p.nres[b];
+  if (h == 0 && lane == 0) {  // the step's lengths (a flush of this step moved G tokens to block nb - 1)
+    int32_t* len = L.lens + (int64_t)b * kLensStride;
+    len[kLenQ] = nb * L.group_k;
+    len[kLenN] = p.nres[b];
+    len[kLenQV] = nb * L.group_k;
+  }
 }
 
 // Issue side of a warp's item stream (one lane): the unit of the last issued
@@ -834,6 +839,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
   // the combine launch that follows may be scheduled from now on; it waits
   // for this grid to complete before reading any partial
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // a fused decode step that flushes launches this kernel as a dependent of
+  // the kernel quantizing the flushed blocks: wait for those records (no-op
+  // otherwise)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // this warp's items: rs + warp + n*kNC, n = 0, 1, ...; item n lands in the
   // warp's own stage n % SPW, and the warp issues item n + SPW as soon as it
   // is done with item n
@@ -1155,11 +1164,23 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
 }
 
 // Enqueues one instance. Its dynamic shared-memory size was opted in on this
-// device by mma_ctas_per_sm, which the host calls before every launch.
+// device by mma_ctas_per_sm, which the host calls before every launch. After
+// the flush kernel of a fused decode step (p.after_flush) it is a
+// programmatic dependent of that kernel: its CTAs may start while the flush
+// runs and wait for it (griddepcontrol.wait) before reading any record.
 template <int KB, int VB, int NGRP, int NKT, bool PT>
 cudaError_t launch_instance(const DecodeParams& p, const MmaPlan& mp, cudaStream_t stream) {
-  decode_tc_kernel<KB, VB, NGRP, NKT, PT><<<p.num_ctas, kThreads, mp.smem_bytes, stream>>>(p, mp);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.num_ctas);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = mp.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = p.after_flush ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<KB, VB, NGRP, NKT, PT>, p, mp);
 }
 
 template <int KB, int VB, int NGRP, int NKT, bool PT>

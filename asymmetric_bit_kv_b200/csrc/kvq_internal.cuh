@@ -12,6 +12,13 @@ namespace kvq {
 
 constexpr int kHeadDim = 128;  // the decode kernels are specialised for D = 128
 
+// Length table of a layer: int32 [max_batch][kLensStride] per sequence --
+// quantized keys, key ring tokens, sink tokens, quantized values (token
+// positions after the sinks). The value ring holds the tokens from the
+// quantized values up to the end: keys + key ring - quantized values.
+constexpr int kLensStride = 4;
+constexpr int kLenQ = 0, kLenN = 1, kLenS = 2, kLenQV = 3;
+
 // Per-layer view of the packed cache, passed by value to kernels.
 struct LayerView {
   uint8_t* blocks;        // block records [max_batch][Hkv][max_blocks], or the page pool (paged)
@@ -19,12 +26,13 @@ struct LayerView {
   void* ring_v;
   void* sink_k;           // [max_batch][Hkv][KVQ_MAX_SINKS][D] kv dtype (sink_tokens > 0)
   void* sink_v;
-  int32_t* lens;          // [max_batch][3]: quantized tokens, ring tokens, sink tokens
+  int32_t* lens;          // [max_batch][kLensStride] length table (see kLensStride)
   int64_t record_bytes;
   int64_t max_blocks;
   int32_t kc_off, ksz_off, vc_off, vsz_off;  // byte offsets inside a record
   int32_t k_bits, v_bits;
   int32_t num_kv_heads, head_dim, group_k, group_v, residual;
+  int32_t residual_v;     // value ring slots (= residual unless the cache sets its own)
   int32_t kv_dtype;       // KVQ_F16 / KVQ_BF16
   int32_t sinks;          // S: sink tokens kept exact at the start of each sequence
   int32_t k_axis;         // 0: keys per channel over G tokens (KIVI); 1: per token over group_v channels (BQ2_0)
@@ -177,6 +185,71 @@ __device__ __forceinline__ uint32_t quant_code(float x, const GroupParams& g, in
   const float t = __fdiv_rn(__fsub_rn(x, g.m), g.d);
   const float r = fminf(fmaxf(rintf(t), 0.0f), (float)((1 << bits) - 1));  // rint: ties to even
   return (uint32_t)r;
+}
+
+// The same code with one multiplication instead of a division: r is 1/d
+// rounded to nearest (__frcp_rn, once per group). With a = fl(x - m), the
+// product t = fl(a * r) and the quotient fl(a / d) both lie within a
+// relative 2^-24 per rounding of a/d (two roundings for t, one for the
+// quotient), so they differ by less than |t| * 2^-22. Hence whenever t is
+// farther than |t| * 2^-21 from its nearest half-integer (which keeps every
+// other half-integer at least 0.5 away) both lie strictly inside the same
+// rounding interval and rint(t) = rint(quotient); inside that window (and
+// always for |t| >= 2^21) the quotient itself is computed. rint(t) comes
+// from one fp32 addition: for |t| < 2^22, t + 1.5 * 2^23 lies in [2^23,
+// 2^24), where the spacing is 1, so the sum is rounded to an integer with
+// ties to even and its bits minus those of 1.5 * 2^23 are rint(t); e = t -
+// rint(t) is exact (Sterbenz), and 0.5 - |e| is the distance to the nearest
+// half-integer (exact when it matters, |e| >= 1/4). Only FMA- and ALU-pipe
+// instructions on the common path. Bit-exact with quant_code.
+__device__ __forceinline__ uint32_t quant_code_rcp(float x, float m, float d, float r, int bits) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const float a = __fsub_rn(x, m);
+  const float t = __fmul_rn(a, r);
+  const float tm = __fadd_rn(t, kRound);
+  const float e = __fsub_rn(t, __fsub_rn(tm, kRound));
+  int k;
+  if (__fsub_rn(0.5f, fabsf(e)) <= fabsf(t) * 0x1p-21f) {
+    k = (int)fminf(fmaxf(rintf(__fdiv_rn(a, d)), 0.0f), (float)((1 << bits) - 1));  // rint: ties to even
+  } else {
+    k = __float_as_int(tm) - __float_as_int(kRound);
+  }
+  return (uint32_t)min(max(k, 0), (1 << bits) - 1);
+}
+
+// A word of N = 32/BITS codes of one group with the reasoning of
+// quant_code_rcp, but one branch per word: t is first clamped to
+// [-0.49, qmax + 0.49] (every t outside lies beyond a boundary half-integer
+// whose both sides clamp to the same code, 0 or qmax, so the code is
+// unchanged), which bounds |t| <= qmax + 0.49 and lets one constant
+// threshold, (qmax + 0.5) * 2^-21 >= |t| * 2^-21, serve every value: if any
+// value of the word falls within it of a half-integer, the whole word is
+// recomputed from the exact quotients.
+template <int BITS, int N>
+__device__ __forceinline__ uint32_t quant_word_rcp(const float (&x)[N], float m, float d, float r) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr int qmax = (1 << BITS) - 1;
+  constexpr float lo = -0.49f, hi = (float)qmax + 0.49f;
+  constexpr float near = 0.5f - ((float)qmax + 0.5f) * 0x1p-21f;  // |e| above this: within the window
+  uint32_t word = 0;
+  bool close = false;
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    const float t = fminf(fmaxf(__fmul_rn(__fsub_rn(x[i], m), r), lo), hi);
+    const float tm = __fadd_rn(t, kRound);
+    const float e = __fsub_rn(t, __fsub_rn(tm, kRound));
+    close = close || fabsf(e) > near;
+    word |= (uint32_t)(__float_as_int(tm) - __float_as_int(kRound)) << (i * BITS);
+  }
+  if (close) {
+    word = 0;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      const float q = fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(x[i], m), d)), 0.0f), (float)qmax);  // ties to even
+      word |= (uint32_t)q << (i * BITS);
+    }
+  }
+  return word;
 }
 
 // x_hat = q * d + m with two roundings (no fused multiply-add).

@@ -47,7 +47,14 @@ extern "C" {
 kvq_status kvq_decode_attention_noalloc(kvq_cache* c, int32_t layer, const void* q, void* out, int32_t out_dtype,
                                         float softmax_scale, int32_t batch, void* stream) {
   kvq::clear_last_error();
-  cudaError_t e = cudaSuccess;
+  if (!c) return kvq::report_status(KVQ_ERR_INVALID_ARG, "cache is null");
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return kvq::report_cuda_error(e, "cudaGetDevice");
+  // the array looked up below belongs to the current device: it must be the
+  // device that holds the cache's arena
+  if (dev != kvq::cache_device(c))
+    return kvq::report_status(KVQ_ERR_INVALID_ARG, "the current device is not the cache's device");
   uint8_t* base = scratch_address(&e);
   if (!base) return kvq::report_cuda_error(e, "looking up the static decode scratch");
   const kvq::StaticScratch scratch{base, (int64_t)KVQ_STATIC_SCRATCH_BYTES};

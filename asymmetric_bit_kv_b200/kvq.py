@@ -49,6 +49,7 @@ class kvq_config(ctypes.Structure):
         ("hadamard", ctypes.c_int32),
         ("page_blocks", ctypes.c_int32),
         ("pool_pages", ctypes.c_int32),
+        ("residual_v", ctypes.c_int32),
     ]
 
 
@@ -105,6 +106,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kvq_device_errors": (I32, [P, ctypes.POINTER(I32)]),
         "kvq_seq_lengths": (I32, [P, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32)]),
         "kvq_seq_sinks": (I32, [P, I32, I32, ctypes.POINTER(I32)]),
+        "kvq_seq_value_lengths": (I32, [P, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32)]),
         "kvq_status_string": (ctypes.c_char_p, [I32]),
         "kvq_last_error": (ctypes.c_char_p, []),
     }
@@ -160,6 +162,7 @@ class CacheConfig:
     hadamard: int = 0
     page_blocks: int = 0  # >= 1: block records in pages of this many blocks from a pool
     pool_pages: int = 0   # pages per layer (paged)
+    residual_v: int = 0   # value ring slots when values keep their own window (0: residual)
 
     def to_c(self):
         kb = (ctypes.c_int8 * self.num_layers)(*self.k_bits)
@@ -169,7 +172,7 @@ class CacheConfig:
                        self.max_tokens, self.group_k, self.group_v, self.residual, _DTYPE_CODE[self.kv_dtype],
                        ctypes.cast(kb, ctypes.POINTER(ctypes.c_int8)), ctypes.cast(vb, ctypes.POINTER(ctypes.c_int8)),
                        self.sink_tokens, ctypes.cast(ka, ctypes.POINTER(ctypes.c_int8)), self.hadamard,
-                       self.page_blocks, self.pool_pages)
+                       self.page_blocks, self.pool_pages, self.residual_v)
         return c, (kb, vb, ka)
 
 
@@ -317,6 +320,14 @@ class KVCache:
         q = ctypes.c_int32()
         n = ctypes.c_int32()
         _check(self.lib.kvq_seq_lengths(self.handle, layer, seq, ctypes.byref(q), ctypes.byref(n)), "kvq_seq_lengths")
+        return q.value, n.value
+
+    def value_lengths(self, layer: int, seq: int):
+        """(quantized values, value ring tokens) of one sequence (kvq_seq_value_lengths)."""
+        q = ctypes.c_int32()
+        n = ctypes.c_int32()
+        _check(self.lib.kvq_seq_value_lengths(self.handle, layer, seq, ctypes.byref(q), ctypes.byref(n)),
+               "kvq_seq_value_lengths")
         return q.value, n.value
 
     def sinks(self, layer: int, seq: int) -> int:

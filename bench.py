@@ -405,10 +405,10 @@ def run_kvq(a):
             ab += qn * bytes_tok + n * Hkv * D * 2 * 2
             tk += T * (qn + n) - T * (T - 1) // 2  # query t sees the tokens up to its own position
         if T == 1:
-            # fused: decode + combine; a step that flushes a ring first runs the
-            # quantize and ring-write kernels (unfused: ring write, split
-            # kernel, combine, and the quantize kernel on a flush)
-            launches = (2 + (2 if flush else 0)) if fused else (3 + (1 if flush else 0))
+            # fused: prep (plan; on a flush step also the quantize CTAs),
+            # decode, combine; unfused: ring write (+ quantize on a flush),
+            # split kernel, combine
+            launches = 3 if fused else (3 + (1 if flush else 0))
         else:
             # append (ring write, + quantize on a flush), then decode + combine
             # per group of query tokens (at most 8 query rows per KV head)
@@ -419,7 +419,7 @@ def run_kvq(a):
                     tp *= 2
                 groups, t0 = groups + 1, t0 + tp
             launches = 1 + (1 if flush else 0) + 2 * groups
-        plan.append((r, launches, ab, tk))
+        plan.append((r, launches, ab, tk, flush))
     events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
     launches = sum(x[1] for x in plan)
     alg_total = float(sum(x[2] for x in plan))
@@ -446,8 +446,13 @@ def run_kvq(a):
         for b in range(B):
             assert tuple(lens[r][b]) == caches[r].lengths(0, b), "step accounting out of sync with the cache"
     ms = e0.elapsed_time(e1)
-    dec_ms = sum(x[0].elapsed_time(x[1]) for x in events)
-    ms, dec_ms = cross_rank_max([ms, dec_ms], world, dev)
+    call_ms = [x[0].elapsed_time(x[1]) for x in events]
+    dec_ms = sum(call_ms)
+    fl = [m for m, x in zip(call_ms, plan) if x[4]]
+    nf = [m for m, x in zip(call_ms, plan) if not x[4]]
+    fl_us = 1e3 * sum(fl) / len(fl) if fl else 0.0
+    nf_us = 1e3 * sum(nf) / len(nf) if nf else 0.0
+    ms, dec_ms, fl_us, nf_us = cross_rank_max([ms, dec_ms, fl_us, nf_us], world, dev)
     value = tok_total * world / (ms / 1e3)
     achieved_gbs = alg_total / (dec_ms / 1e3) / 1e9
 
@@ -512,7 +517,10 @@ def run_kvq(a):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "f32",
+            "dtype": "bf16",
+            "dtype_detail": ("bf16 keys, values, queries and outputs; quantizer in fp32; attention on fp16 "
+                             "tensor-core operands (codes exact, q*s and p*s as fp16 high and low parts) and "
+                             "bf16 ones for exact tokens, fp32 accumulation and softmax"),
             "data": "synthetic (seeded; Llama-3-8B-shaped layer, no model weights)",
             "config": dict(_workload_config(wl, R, world, tok_total / (a.steps * B * T)),
                            **({"page_blocks": a.page_blocks} if a.page_blocks else {}),
@@ -522,7 +530,8 @@ def run_kvq(a):
                            "decode of their queries, causal among them (split-KV decode + combine per group of query "
                            "tokens)") if T > 1 else
                           ("decode step: one token appended per sequence inside the split-KV decode kernel, + log-sum-exp "
-                           "combine, per call (a ring flush adds the quantize and ring kernels)") if fused else
+                           "combine, per call (a step in which rings are full first runs the flush kernel that quantizes "
+                           "their oldest G tokens)") if fused else
                           ("decode step: ring write, CUDA-core split-KV decode kernel and log-sum-exp combine, per call "
                            "(a ring flush adds the quantize kernel)"),
                 "bound": "hbm",
@@ -534,6 +543,10 @@ def run_kvq(a):
                 "frac_of_8tbs_nominal": achieved_gbs / 8000.0,
                 "traffic": traffic,
                 "decode_us_per_call": dec_ms / a.steps * 1e3,
+                "flush_step_us": fl_us if fl else None,
+                "flush_steps": len(fl),
+                "nonflush_step_us": nf_us if nf else None,
+                "nonflush_steps": len(nf),
                 "host_enqueue_us_per_step": host_s / a.steps * 1e6,
                 "alg_bytes_per_call": alg_total / a.steps,
             },
@@ -622,8 +635,27 @@ def run_reference(a):
     }
 
 
+def _launch_ranks(n):
+    """Re-run this command as n ranks, one process per GPU, under
+    torch.distributed.run on this node (the way a multi-GPU run is launched);
+    returns its exit status."""
+    import socket
+
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     a = _args()
+    if "WORLD_SIZE" not in os.environ and a.gpus > 1:
+        sys.exit(_launch_ranks(a.gpus))
+    if int(os.environ.get("WORLD_SIZE", "1")) != a.gpus:
+        sys.exit(f"bench.py: --gpus {a.gpus} but WORLD_SIZE is {os.environ.get('WORLD_SIZE')}: "
+                 "launch one rank per GPU (torchrun --nproc-per-node N) or let bench.py launch them")
     if a.impl == "reference":
         res = run_reference(a)
         if res is not None:

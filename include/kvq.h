@@ -15,7 +15,8 @@
  *    lowest bits first.
  *  - "Quantize What Counts: More For Keys, Less For Values", section "KV Cache
  *    Quantization": key and value bit widths chosen independently and per
- *    layer (bit range up to 8).
+ *    layer (bit range up to 8); residual length, group size and axis given
+ *    per tensor ({"k": ..., "v": ...}).
  *
  * Ownership. The caller allocates one device arena per cache (size from
  * kvq_cache_required_bytes) and owns it, every input and output buffer and
@@ -30,7 +31,7 @@
  * given stream (a cudaStream_t; NULL = legacy default stream); faults during
  * execution surface at the caller's next synchronisation, as for any CUDA
  * kernel. Calls on one cache must be ordered on one stream: they share the
- * arena's length table and split-partial workspace.
+ * arena's length table, decode plan and split-partial workspace.
  *
  * Threading. A handle is not thread-safe; distinct handles are independent.
  */
@@ -56,7 +57,10 @@ typedef enum kvq_status {
   KVQ_ERR_UNSUPPORTED = -2, /* valid but not built: bits, dims, dtype      */
   KVQ_ERR_CAPACITY = -3,    /* a sequence would exceed max_tokens, or a
                                paged layer's pool has too few free pages   */
-  KVQ_ERR_WORKSPACE = -4,   /* arena smaller than kvq_cache_required_bytes */
+  KVQ_ERR_WORKSPACE = -4,   /* arena smaller than kvq_cache_required_bytes,
+                               or a call's split partials do not fit the
+                               memory they go to (arena workspace or the
+                               static scratch of the no-alloc decode)      */
   KVQ_ERR_CUDA = -5         /* a CUDA launch or call failed                */
 } kvq_status;
 
@@ -68,8 +72,9 @@ typedef enum kvq_dtype { KVQ_F16 = 0, KVQ_BF16 = 1, KVQ_F32 = 2 } kvq_dtype;
 #define KVQ_MAX_SINKS 8    /* sink tokens per sequence                   */
 
 /* Cache shape. Names follow the KIVI README "Example" (k_bits, v_bits,
- * group_size, residual_length) with the group size given per tensor as in
- * "Quantize What Counts" (group_size {"k", "v"}).                          */
+ * group_size, residual_length) with the group size and residual length
+ * given per tensor as in "Quantize What Counts", KV Cache Quantization
+ * (group_size {"k", "v"}, residual_length {"k", "v"}).                     */
 typedef struct kvq_config {
   int32_t num_layers;   /* 1 .. KVQ_MAX_LAYERS                              */
   int32_t max_batch;    /* sequences, 1 .. KVQ_MAX_BATCH                    */
@@ -81,7 +86,8 @@ typedef struct kvq_config {
                            32, 64 or 128. Flushes move G tokens at a time.  */
   int32_t group_v;      /* channels per value group (one group per token);
                            32, 64 or 128, dividing head_dim                 */
-  int32_t residual;     /* R: full-precision ring slots; a multiple of G    */
+  int32_t residual;     /* R: full-precision key ring slots (and value ring
+                           slots unless residual_v is set); a multiple of G */
   int32_t kv_dtype;     /* KVQ_F16 or KVQ_BF16: keys, values, ring, queries */
   const int8_t* k_bits; /* host [num_layers], each 2, 4 or 8 (copied)       */
   const int8_t* v_bits; /* host [num_layers], each 2, 4 or 8 (copied)       */
@@ -106,6 +112,13 @@ typedef struct kvq_config {
                            kvq_release_sequence / kvq_cache_reset, so a
                            ragged batch holds only the pages it uses        */
   int32_t pool_pages;   /* pages per layer when page_blocks >= 1            */
+  int32_t residual_v;   /* 0: values share R. Else the value ring's slots, a
+                           multiple of G: keys and values then keep their own
+                           full-precision windows and each flushes its own
+                           oldest G tokens when its ring is full ("Quantize
+                           What Counts": residual_length {"k", "v"}). Not
+                           with hadamard. Layers run on the CUDA-core
+                           decode kernel when it differs from residual.     */
 } kvq_config;
 
 typedef struct kvq_cache kvq_cache;
@@ -139,8 +152,12 @@ typedef struct kvq_cache kvq_cache;
  * (r / (8/n)) % n otherwise; rows of fewer than 4 words are not permuted.
  * Value rows are stored in token order t -> (t % c) * (G/c) + t / c, with
  * c = 16/k_bits. (kvq_internal.cuh: kc_word_index, vc_word_index.)
- * Ring: [max_batch][num_kv_heads][R][D] in kv_dtype; position i of a
- * sequence (quantized <= i < quantized + residual) sits in slot i % R.
+ * Rings: keys [max_batch][num_kv_heads][R][D] and values
+ * [max_batch][num_kv_heads][RV][D] in kv_dtype (RV = residual_v, or R);
+ * position i of a sequence whose key (value) is exact sits in slot i % R
+ * (i % RV). With separate residual lengths a block record may hold only its
+ * key part or only its value part (the other tensor's tokens are still in
+ * their ring); kvq_seq_lengths / kvq_seq_value_lengths tell which.
  * Sinks: [max_batch][num_kv_heads][KVQ_MAX_SINKS][D] in kv_dtype; sink
  * token i (< s) in row i, the other rows zero.                             */
 typedef struct kvq_layout {
@@ -163,13 +180,19 @@ typedef struct kvq_layout {
 } kvq_layout;
 
 /* Device bytes the arena must hold for cfg: all layers' block records and
- * rings, the length table and the split-partial workspace.                 */
+ * rings, the length table, the decode plan and the split-partial workspace.
+ * Sizes follow from the method's layout (KV1-1.2B card, Quantization Format:
+ * b-bit codes plus an fp16 scale and zero point per group; KIVI README,
+ * Overview: keys grouped per channel, values per token, R exact tokens).   */
 KVQ_API kvq_status kvq_cache_required_bytes(const kvq_config* cfg, size_t* bytes);
 
 /* Validate cfg and bind a cache to dev_arena (device pointer, 256-byte
  * aligned, arena_bytes >= required), with the arena's device current. Every
  * sequence starts empty: the call zeroes the arena's length table and
- * residual rings, and waits for that to finish before it returns.          */
+ * residual rings, and waits for that to finish before it returns. The cache
+ * is the KIVI README's quantized KV cache ("Overview": per-channel keys,
+ * per-token values, a full-precision residual window; "Example": k_bits,
+ * v_bits, group_size, residual_length), one per model, all layers.         */
 KVQ_API kvq_status kvq_cache_create(const kvq_config* cfg, void* dev_arena, size_t arena_bytes,
                             kvq_cache** out);
 
@@ -203,8 +226,11 @@ KVQ_API kvq_status kvq_release_sequence(kvq_cache* cache, int32_t seq, void* str
 KVQ_API kvq_status kvq_append(kvq_cache* cache, int32_t layer, const void* k, const void* v,
                       const int32_t* new_lens, int32_t batch, void* stream);
 
-/* Quantize every complete group of G tokens left in the ring of sequences
- * 0..batch-1 of `layer`: residual n becomes n % G.                         */
+/* Quantize every complete group of G tokens left in the rings of sequences
+ * 0..batch-1 of `layer`: a ring of n tokens keeps n % G (KIVI README,
+ * Overview: tokens leave the full-precision window in groups; the
+ * end-of-prefill flush of its "Example"). Keys and values each flush their
+ * own ring.                                                                */
 KVQ_API kvq_status kvq_flush_residual(kvq_cache* cache, int32_t layer, int32_t batch, void* stream);
 
 /* One decode query per sequence: out[b][h] = softmax(scale * q[b][h] K~^T) V~
@@ -212,7 +238,11 @@ KVQ_API kvq_status kvq_flush_residual(kvq_cache* cache, int32_t layer, int32_t b
  * dequantized blocks and the exact ring tokens; query head h reads KV head
  * h / (Hq/Hkv) (GQA). q: device [batch][Hq][D] in kv_dtype. out: device
  * [batch][Hq][D] in out_dtype (F32, F16 or BF16; round to nearest even).
- * A sequence with no tokens gives zeros. Uses the arena's workspace.       */
+ * A sequence with no tokens gives zeros. Uses the arena's decode plan and
+ * workspace. This is the KIVI README's decoding over the quantized cache
+ * ("Overview": attention over quantized keys and values plus the
+ * full-precision recent tokens; GQA per its 2025.01.18 update), with
+ * x_hat = q*d + m of the KV1-1.2B card (Quantization Format).              */
 KVQ_API kvq_status kvq_decode_attention(kvq_cache* cache, int32_t layer, const void* q, void* out,
                                 int32_t out_dtype, float softmax_scale, int32_t batch,
                                 void* stream);
@@ -243,22 +273,31 @@ KVQ_API kvq_status kvq_decode_attention_multi(kvq_cache* cache, int32_t layer, c
  * device memory at the point of the call, for example an engine whose device
  * memory is all handed to its own pool at start-up, or code running under a
  * fixed memory budget where a cudaMalloc could fail or stall the device.
- * This call allocates nothing. Its split partials go to a static device array
- * of KVQ_STATIC_SCRATCH_BYTES that the library holds, not to the arena's
- * workspace, which it leaves untouched. The pages have no counterpart: this
- * is an interface choice of this library.
- * - Size limit: the partials take batch * Hq * S * (4*head_dim + 8) bytes,
- *   where S is the number of partial slots this call's split plan uses per
- *   (sequence, query head). A call that needs more than the scratch holds
- *   returns KVQ_ERR_WORKSPACE, enqueues nothing, and kvq_last_error() gives
- *   both sizes.
+ * This call allocates nothing. Its decode plan, per-unit slot counts and
+ * split partials go to a static device array of KVQ_STATIC_SCRATCH_BYTES
+ * that the library holds, not to the arena, whose workspace, plan and slot
+ * table it leaves untouched; it still writes the cache's device error word
+ * if a bounded wait gives up (kvq_device_errors). The pages have no
+ * counterpart: this is an interface choice of this library.
+ * - Size limit: after the plan (about 32 * batch bytes) and the slot table
+ *   (4 * batch * Hkv bytes), each partial slot takes batch * Hq *
+ *   (4*head_dim + 8) bytes; the call plans its split so that the slots a
+ *   (sequence, query head) uses fit what remains, down to one CTA per unit.
+ *   A call for which even that does not fit (fewer than 6 slots on the
+ *   tensor-core kernel, 2 on the CUDA-core one) returns KVQ_ERR_WORKSPACE,
+ *   enqueues nothing, and kvq_last_error() gives the sizes.
+ * - Device: the current device must be the one the cache was created on
+ *   (else KVQ_ERR_INVALID_ARG): the array is per device.
  * - Set-up: the first call on each device looks up the array's device
- *   address (cudaGetSymbolAddress, with that device current). Make that first
- *   call before any stream capture.
+ *   address (cudaGetSymbolAddress, with that device current) and keeps it
+ *   for the process. Make that first call before any stream capture. A
+ *   cudaDeviceReset invalidates the kept address: do not call this entry
+ *   point after one.
  * - Sharing: every call on a device uses the same array and leaves the last
- *   call's partials in it. Each call writes every partial it reads, so nothing
- *   has to start at zero. Calls that may overlap on the GPU race on the array
- *   (different streams, or several caches): order them.                   */
+ *   call's contents in it. Each call writes every plan entry, slot count and
+ *   partial it reads before reading it, so nothing has to start at zero.
+ *   Calls that may overlap on the GPU race on the array (different streams,
+ *   or several caches): order them.                                        */
 KVQ_API kvq_status kvq_decode_attention_noalloc(kvq_cache* cache, int32_t layer, const void* q, void* out,
                                         int32_t out_dtype, float softmax_scale, int32_t batch,
                                         void* stream);
@@ -266,12 +305,16 @@ KVQ_API kvq_status kvq_decode_attention_noalloc(kvq_cache* cache, int32_t layer,
 /* One decode step: append one token to each sequence b < batch (k, v:
  * device [batch][num_kv_heads][head_dim] in kv_dtype, as kvq_append with
  * new_lens all 1), then decode attention for q over every token including
- * the new one (as kvq_decode_attention). Same results as those two calls;
- * when no sequence needs a flush or a sink (its ring not full, its sinks
- * complete) and the layer runs on the tensor-core kernel, the new tokens are
- * written and attended to inside the decode launch (one launch fewer; the
- * fused append+decode step the KV1 card's quantize-on-entry decode loop
- * suggests). All checks run before anything is enqueued.                  */
+ * the new one (as kvq_decode_attention). Same results as those two calls.
+ * When the layer runs on the tensor-core kernel, keys and values share one
+ * residual length and every sequence's sinks are complete, the step is
+ * fused: a small prep launch quantizes the oldest G tokens of every full
+ * ring (only in steps where some ring is full) and plans the decode, and
+ * the decode launch attends to the new tokens and writes them into their
+ * ring slots -- no separate append kernels (the decode loop of the KV1-1.2B
+ * card, Quickstart, where each token is quantized once as it enters the
+ * cache; KIVI README, Overview, for the window). All checks run before
+ * anything is enqueued.                                                   */
 KVQ_API kvq_status kvq_decode_step(kvq_cache* cache, int32_t layer, const void* k, const void* v, const void* q,
                                    void* out, int32_t out_dtype, float softmax_scale, int32_t batch, void* stream);
 
@@ -286,17 +329,30 @@ KVQ_API kvq_status kvq_dequant(kvq_cache* cache, int32_t layer, int32_t seq, int
 
 /* Device-side failures recorded since the last call, then cleared: bit 0 =
  * a decode kernel gave up a bounded wait on its copy pipeline (its partial
- * results are invalid). Synchronous: waits for the device to finish its
- * work.                                                                   */
+ * results are invalid); bit 1 = a decode CTA found an empty work range in
+ * its plan (results invalid; not expected). Synchronous: waits for the
+ * device to finish its work. No counterpart on the pages: a diagnostic of
+ * this library.                                                           */
 KVQ_API kvq_status kvq_device_errors(kvq_cache* cache, int32_t* flags);
 
-/* Layer layout (see kvq_layout).                                           */
+/* Layer layout (see kvq_layout): where the packed codes, scales and zero
+ * points of the KV1-1.2B card's format (Quantization Format) and the
+ * KIVI README's full-precision window live. For tests and tools that read
+ * the cache; no counterpart on the pages beyond the format itself.         */
 KVQ_API kvq_status kvq_get_layout(const kvq_cache* cache, int32_t layer, kvq_layout* out);
 
-/* Host mirror of a sequence's lengths: quantized tokens (a multiple of G)
- * and ring tokens (the sink tokens come on top: kvq_seq_sinks).             */
+/* Host mirror of a sequence's key lengths: quantized keys (a multiple of G)
+ * and key ring tokens (the sink tokens come on top: kvq_seq_sinks). The
+ * split of the KIVI README's Overview (quantized tokens, full-precision
+ * window); a test accessor, no counterpart on the pages otherwise.          */
 KVQ_API kvq_status kvq_seq_lengths(const kvq_cache* cache, int32_t layer, int32_t seq,
                            int32_t* quantized, int32_t* residual);
+
+/* The same for the values: quantized values and value ring tokens (equal to
+ * the key lengths unless residual_v differs from residual; "Quantize What
+ * Counts", residual_length {"k", "v"}). A test accessor.                   */
+KVQ_API kvq_status kvq_seq_value_lengths(const kvq_cache* cache, int32_t layer, int32_t seq,
+                                 int32_t* quantized, int32_t* residual);
 
 /* Host mirror of a sequence's sink tokens, min(S, tokens appended). No
  * counterpart on the pages beyond the sinks themselves (KV1 card).         */

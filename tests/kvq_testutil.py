@@ -84,11 +84,14 @@ class Twin:
         self.ora = {}
         for layer in self.oracle_layers:
             for b in self.oracle_seqs:
-                self.ora[(layer, b)] = O.SequenceCache(cfg.num_kv_heads, cfg.head_dim, cfg.k_bits[layer],
-                                                       cfg.v_bits[layer], cfg.group_k, cfg.group_v, cfg.residual,
-                                                       sinks=cfg.sink_tokens,
-                                                       k_axis=(cfg.k_axis or [0] * cfg.num_layers)[layer],
-                                                       hadamard=bool(cfg.hadamard))
+                self.ora[(layer, b)] = self._new_oracle(layer)
+
+    def _new_oracle(self, layer):
+        cfg = self.cfg
+        return O.SequenceCache(cfg.num_kv_heads, cfg.head_dim, cfg.k_bits[layer], cfg.v_bits[layer], cfg.group_k,
+                               cfg.group_v, cfg.residual, sinks=cfg.sink_tokens,
+                               k_axis=(cfg.k_axis or [0] * cfg.num_layers)[layer], hadamard=bool(cfg.hadamard),
+                               residual_v=cfg.residual_v or None)
 
     def append(self, layer: int, k: torch.Tensor, v: torch.Tensor, new_lens):
         """k, v: [sum(new_lens), Hkv, D] in the cache dtype (any device)."""
@@ -105,14 +108,9 @@ class Twin:
     def release_sequence(self, b: int):
         """Empty sequence b in every layer on both sides."""
         self.gpu.release_sequence(b)
-        cfg = self.cfg
         for layer in self.oracle_layers:
             if (layer, b) in self.ora:
-                self.ora[(layer, b)] = O.SequenceCache(cfg.num_kv_heads, cfg.head_dim, cfg.k_bits[layer],
-                                                       cfg.v_bits[layer], cfg.group_k, cfg.group_v, cfg.residual,
-                                                       sinks=cfg.sink_tokens,
-                                                       k_axis=(cfg.k_axis or [0] * cfg.num_layers)[layer],
-                                                       hadamard=bool(cfg.hadamard))
+                self.ora[(layer, b)] = self._new_oracle(layer)
 
     def flush_residual(self, layer: int, batch: int):
         self.gpu.flush_residual(layer, batch)
@@ -125,6 +123,7 @@ class Twin:
             if (layer, b) in self.ora:
                 o = self.ora[(layer, b)]
                 assert self.gpu.lengths(layer, b) == (o.quantized_tokens, o.residual_tokens), (layer, b)
+                assert self.gpu.value_lengths(layer, b) == (o.quantized_tokens_v, o.residual_tokens_v), (layer, b)
                 assert self.gpu.sinks(layer, b) == o.sink_tokens, (layer, b, "sinks")
 
     def read_records(self, layer: int, b: int, h: int, nblk: int):
@@ -174,14 +173,15 @@ class Twin:
         }
 
     def read_ring(self, layer: int, b: int):
+        """(key ring [H, R, D], value ring [H, RV, D]) of sequence b."""
         lay = self.gpu.layout(layer)
         cfg = self.cfg
-        n = cfg.num_kv_heads * cfg.residual * cfg.head_dim * 2
         out = []
-        for ptr in (lay.ring_k, lay.ring_v):
+        for ptr, R in ((lay.ring_k, cfg.residual), (lay.ring_v, cfg.residual_v or cfg.residual)):
+            n = cfg.num_kv_heads * R * cfg.head_dim * 2
             start = ptr - self.gpu.arena.data_ptr() + b * n
             raw = self.gpu.arena[start:start + n].cpu()
-            out.append(raw.view(cfg.kv_dtype).float().numpy().reshape(cfg.num_kv_heads, cfg.residual, cfg.head_dim))
+            out.append(raw.view(cfg.kv_dtype).float().numpy().reshape(cfg.num_kv_heads, R, cfg.head_dim))
         return out
 
     def read_sinks(self, layer: int, b: int):
@@ -196,41 +196,45 @@ class Twin:
         return out
 
     def check_codes(self, layer: int, b: int):
-        """Every packed block and ring token of sequence b equals the oracle's, bit for bit."""
+        """Every packed block part and ring token of sequence b equals the
+        oracle's, bit for bit (keys and values each up to their own
+        quantized length)."""
         o = self.ora[(layer, b)]
         cfg = self.cfg
         kb, vb = cfg.k_bits[layer], cfg.v_bits[layer]
-        nblk = len(o.blocks)
+        nk, nv = len(o.key_blocks), len(o.value_blocks)
+        nblk = max(nk, nv)
         for h in range(cfg.num_kv_heads):
             if nblk:
                 rec = self.read_records(layer, b, h, nblk)
-                for j, blk in enumerate(o.blocks):
+                for j in range(nk):
+                    kc, kd, km = o.key_blocks[j]
+                    kw = O.pack_key_block(kc, kb)[h]
+                    assert np.array_equal(rec["kc"][j], kw), (layer, b, h, j, "key codes")
                     if o.k_axis == 1:
-                        kw = O.pack_key_block(blk.kc, kb)[h]
-                        assert np.array_equal(rec["kc"][j], kw), (layer, b, h, j, "per-token key codes")
-                        assert np.array_equal(rec["ksz"][j][..., 0].view(np.uint16), blk.kd[:, h].view(np.uint16)), (b, h, j, "key scale")
-                        assert np.array_equal(rec["ksz"][j][..., 1].view(np.uint16), blk.km[:, h].view(np.uint16)), (b, h, j, "key zero")
+                        assert np.array_equal(rec["ksz"][j][..., 0].view(np.uint16), kd[:, h].view(np.uint16)), (b, h, j, "key scale")
+                        assert np.array_equal(rec["ksz"][j][..., 1].view(np.uint16), km[:, h].view(np.uint16)), (b, h, j, "key zero")
                     else:
-                        kw = O.pack_key_block(blk.kc, kb)[h]
-                        assert np.array_equal(rec["kc"][j], kw), (layer, b, h, j, "key codes")
-                        assert np.array_equal(rec["ksz"][j][:, 0].view(np.uint16), blk.kd[h].view(np.uint16)), (b, h, j, "key scale")
-                        assert np.array_equal(rec["ksz"][j][:, 1].view(np.uint16), blk.km[h].view(np.uint16)), (b, h, j, "key zero")
-                    vw = O.pack_value_block(blk.vc, vb)[h]
+                        assert np.array_equal(rec["ksz"][j][:, 0].view(np.uint16), kd[h].view(np.uint16)), (b, h, j, "key scale")
+                        assert np.array_equal(rec["ksz"][j][:, 1].view(np.uint16), km[h].view(np.uint16)), (b, h, j, "key zero")
+                for j in range(nv):
+                    vc, vd, vm = o.value_blocks[j]
+                    vw = O.pack_value_block(vc, vb)[h]
                     assert np.array_equal(rec["vc"][j], vw), (layer, b, h, j, "value codes")
-                    assert np.array_equal(rec["vsz"][j][..., 0].view(np.uint16), blk.vd[:, h].view(np.uint16)), (b, h, j, "value scale")
-                    assert np.array_equal(rec["vsz"][j][..., 1].view(np.uint16), blk.vm[:, h].view(np.uint16)), (b, h, j, "value zero")
+                    assert np.array_equal(rec["vsz"][j][..., 0].view(np.uint16), vd[:, h].view(np.uint16)), (b, h, j, "value scale")
+                    assert np.array_equal(rec["vsz"][j][..., 1].view(np.uint16), vm[:, h].view(np.uint16)), (b, h, j, "value zero")
         if o.sink_tokens:
             sk, sv = self.read_sinks(layer, b)
             for t in range(o.sink_tokens):
                 assert np.array_equal(sk[:, t], o.sink_k[t]), (layer, b, t, "sink key")
                 assert np.array_equal(sv[:, t], o.sink_v[t]), (layer, b, t, "sink value")
-        if o.residual_tokens:
+        if o.residual_tokens or o.residual_tokens_v:
             rk, rv = self.read_ring(layer, b)
-            Q = o.quantized_tokens
+            R, RV = cfg.residual, cfg.residual_v or cfg.residual
             for t in range(o.residual_tokens):
-                slot = (Q + t) % cfg.residual
-                assert np.array_equal(rk[:, slot], o.ring_k[t]), (layer, b, t, "ring key")
-                assert np.array_equal(rv[:, slot], o.ring_v[t]), (layer, b, t, "ring value")
+                assert np.array_equal(rk[:, (o.quantized_tokens + t) % R], o.ring_k[t]), (layer, b, t, "ring key")
+            for t in range(o.residual_tokens_v):
+                assert np.array_equal(rv[:, (o.quantized_tokens_v + t) % RV], o.ring_v[t]), (layer, b, t, "ring value")
 
     def check_dequant(self, layer: int, b: int):
         o = self.ora[(layer, b)]

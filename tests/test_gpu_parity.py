@@ -19,9 +19,21 @@ def _cfg(*, batch=3, hq=4, hkv=2, G=32, Gv=32, R=64, kb=2, vb=2, dtype=torch.bfl
     return CacheConfig(layers, batch, hq, hkv, 128, max_tokens, G, Gv, R, dtype, [kb] * layers, [vb] * layers)
 
 
-def _adversarial_tokens(T, H, D, dtype, gen):
+def _tie_pattern(bits, n, dtype):
+    """n values repeating 0, (2^bits - 1) * 0.75 and every half-step
+    (k + 1/2) * 0.75: a group holding whole periods has the scale 0.75
+    exactly -- whose reciprocal is not exact in fp32 -- and its codes round
+    exact ties half to even; None if the pattern is not exact in dtype."""
+    qmax = (1 << bits) - 1
+    period = [0.0, qmax * 0.75] + [(k + 0.5) * 0.75 for k in range(qmax)]  # every block holds whole periods
+    t = torch.tensor([period[i % len(period)] for i in range(n)], dtype=torch.float64)
+    return t if torch.equal(t.to(dtype).double(), t) else None
+
+
+def _adversarial_tokens(T, H, D, dtype, gen, kb=None, vb=None, gv=None):
     """Random tokens with planted edge cases: constant channels, constant
-    value groups, signed zeros, exact half-step ties and large magnitudes."""
+    value groups, signed zeros, exact half-step ties (with a scale of 1 and
+    of 0.75) and large magnitudes."""
     k = torch.randn(T, H, D, generator=gen) * torch.exp(torch.randn(1, H, D, generator=gen))
     v = torch.randn(T, H, D, generator=gen)
     k[:, 0, 5] = 0.75                         # constant key channel
@@ -32,6 +44,15 @@ def _adversarial_tokens(T, H, D, dtype, gen):
         v[0, 0, :4] = torch.tensor([0.0, 1.0, 1.5, 3.0])
     k[:, 0, 100] = 6.0e4 * torch.sign(torch.randn(T, generator=gen))  # near the fp16 limit
     k[:, 0, 101] = k[:, 0, 101] * 1e-4        # tiny range -> scale floor
+    if kb is not None:  # a key channel on exact ties of a scale whose reciprocal is inexact
+        t = _tie_pattern(kb, T, dtype)
+        if t is not None:
+            k[:, 0, 11] = t.float()
+    if vb is not None and gv is not None and T >= 2:  # a value group of two tokens on such ties
+        t = _tie_pattern(vb, gv, dtype)
+        if t is not None:
+            v[1, 0, D - gv:D] = t.float()
+            v[0, H - 1, 0:gv] = t.flip(0).float()
     return k.to(dtype), v.to(dtype)
 
 
@@ -57,7 +78,7 @@ def test_append_codes_ring_and_dequant_bit_exact(case):
     plans = [[3 * G + 5, 1, 1, R - 3, 7, 2 * G + 1], [0, 7, 0, 1, 0, 0], [R + 2 * G + 1, G - 1, 1, 1, 3, 0]]
     for step in range(len(plans[0])):
         lens = [p[step] for p in plans]
-        k, v = _adversarial_tokens(sum(lens), H, D, cfg.kv_dtype, gen)
+        k, v = _adversarial_tokens(sum(lens), H, D, cfg.kv_dtype, gen, case["kb"], case["vb"], case["Gv"])
         tw.append(0, k, v, lens)
         tw.check_lengths(0, cfg.max_batch)
     torch.cuda.synchronize()

@@ -5,8 +5,11 @@ decode (for example an engine that gives all of its device memory to its own
 pool at start-up): its split partials go to a fixed-size array that the library
 itself holds on the device. Its output must agree with kvq_decode_attention on
 the same cache, within the attention tolerance, on consecutive calls (the array
-keeps the previous call's contents). A call that needs more scratch than the
-array holds must be refused before anything runs.
+keeps the previous call's contents): between the two checked calls a call on
+another cache, with another layout and values a hundred times larger, fills the
+array with very different contents, so a partial left over from an earlier call
+would show. A call that needs more scratch than the array holds must be refused
+before anything runs.
 
 The file name makes pytest collect it last.
 """
@@ -39,15 +42,23 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("case", CASES, ids=["tensor_core_G64", "cuda_core_G32"])
-def test_noalloc_matches_decode_attention_on_consecutive_calls(case):
+def _filled(case, gen, magnitude=1.0):
     kb, vb, G, Gv, R, B, Hq, Hkv, lens = case
     cfg = CacheConfig(1, B, Hq, Hkv, 128, 8192, G, Gv, R, torch.bfloat16, [kb], [vb])
     cache = KVCache(cfg, "cuda")
-    gen = torch.Generator().manual_seed(11)
     k = (torch.randn(sum(lens), Hkv, 128, generator=gen) * torch.exp(torch.randn(1, Hkv, 128, generator=gen)))
-    v = torch.randn(sum(lens), Hkv, 128, generator=gen)
-    cache.append(0, k.to(torch.bfloat16).cuda(), v.to(torch.bfloat16).cuda(), lens)
+    v = torch.randn(sum(lens), Hkv, 128, generator=gen) * magnitude
+    cache.append(0, (k * magnitude).to(torch.bfloat16).cuda(), v.to(torch.bfloat16).cuda(), lens)
+    return cache
+
+
+@pytest.mark.parametrize("case", CASES, ids=["tensor_core_G64", "cuda_core_G32"])
+def test_noalloc_matches_decode_attention_on_consecutive_calls(case):
+    kb, vb, G, Gv, R, B, Hq, Hkv, lens = case
+    gen = torch.Generator().manual_seed(11)
+    cache = _filled(case, gen)
+    other_case = CASES[1] if case is CASES[0] else CASES[0]
+    other = _filled(other_case, gen, magnitude=100.0)
     scale = 128 ** -0.5
     for call in range(2):
         q = torch.randn(B, Hq, 128, generator=gen).to(torch.bfloat16).cuda()
@@ -62,7 +73,15 @@ def test_noalloc_matches_decode_attention_on_consecutive_calls(case):
             k1 = torch.randn(B, Hkv, 128, generator=gen).to(torch.bfloat16).cuda()
             v1 = torch.randn(B, Hkv, 128, generator=gen).to(torch.bfloat16).cuda()
             cache.append(0, k1, v1, [1] * B)
+            # the other cache's decode overwrites the shared array
+            Bo, Hqo = other_case[5], other_case[6]
+            qo = torch.randn(Bo, Hqo, 128, generator=gen).to(torch.bfloat16).cuda()
+            oo = torch.empty(Bo, Hqo, 128, device="cuda")
+            assert _call(other, "kvq_decode_attention_noalloc", qo, oo, scale) == K.KVQ_OK
+            torch.cuda.synchronize()
+            assert float(oo.abs().max()) > 10.0  # values of the other cache are large
     cache.close()
+    other.close()
 
 
 def test_noalloc_rejects_a_call_beyond_the_static_scratch():
@@ -79,7 +98,7 @@ def test_noalloc_rejects_a_call_beyond_the_static_scratch():
     st = _call(cache, "kvq_decode_attention_noalloc", q, out, 0.1)
     assert st == K.KVQ_ERR_WORKSPACE
     msg = K.load_library().kvq_last_error().decode()
-    assert "static scratch holds 16777216" in msg, msg
+    assert "static scratch (16777216 bytes)" in msg, msg
     torch.cuda.synchronize()
     assert float(out.abs().max()) == 0.0  # nothing was enqueued
     # a smaller batch of the same cache fits and agrees with the arena path
