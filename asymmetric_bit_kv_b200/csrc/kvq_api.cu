@@ -372,6 +372,7 @@ void plan_cta_starts(kvq::DecodeParams& p, int batch, int hkv, int64_t max_ctas,
   N = std::max<int64_t>(1, std::min<int64_t>(N, kvq::kMaxCtas));
   p.total_blocks = (int32_t)T;
   p.num_ctas = (int32_t)N;
+  p.max_unit_slots = (int32_t)std::min<int64_t>(slot_cap, kvq::kMmaConsumers * (cu_max * N / C + 2));
   p.cta_start[0] = 0;
   int b = 0;
   int64_t cost0 = 0;  // cost before sequence b

@@ -303,72 +303,100 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
 // Log-sum-exp merge of the partial slots of one (sequence, query head):
 // M = max_s m_s over slots with l_s > 0, out = sum_s 2^(m_s-M) o_s / sum_s
 // 2^(m_s-M) l_s, rounded to the output dtype (nearest even); a sequence with
-// no tokens gives zeros. One warp per (sequence, query head), lane L owning
-// channels 4L..4L+3 (one 16-byte load per slot); 4 warps per block, grid
-// (ceil(Hq / 4), batch). Every lane issues the loads of 16 slots at once and
-// merges them online, so a typical merge takes one round trip to L2.
-__global__ void __launch_bounds__(128) combine_kernel(CombineParams p) {
+// no tokens gives zeros. WPH warps per (sequence, query head), lane L owning
+// channels 4L..4L+3 (one 16-byte load per slot): warp w of a head merges
+// slots w, w + WPH, ... online, issuing the loads of 16 of its slots at once
+// (one round trip to L2 per 16 slots), and the head's warps then merge their
+// states through shared memory. CTAs of max(4, WPH) warps, grid
+// (ceil(Hq * WPH / warps), batch).
+struct MergeState {
+  float M, l;
+  float4 acc, acc0;  // acc0: hadamard split mode, the exact-token slot 0 (kept apart)
+};
+
+__device__ __forceinline__ void merge_into(MergeState& a, const MergeState& b) {
+  const float M = fmaxf(a.M, b.M);
+  if (M == -INFINITY) return;
+  const float ra = a.M == -INFINITY ? 0.f : exp2f(a.M - M), rb = b.M == -INFINITY ? 0.f : exp2f(b.M - M);
+  a.acc = make_float4(a.acc.x * ra + b.acc.x * rb, a.acc.y * ra + b.acc.y * rb, a.acc.z * ra + b.acc.z * rb,
+                      a.acc.w * ra + b.acc.w * rb);
+  a.acc0 = make_float4(a.acc0.x * ra + b.acc0.x * rb, a.acc0.y * ra + b.acc0.y * rb, a.acc0.z * ra + b.acc0.z * rb,
+                       a.acc0.w * ra + b.acc0.w * rb);
+  a.l = a.l * ra + b.l * rb;
+  a.M = M;
+}
+
+template <int WPH>
+__global__ void __launch_bounds__(32 * (WPH > 4 ? WPH : 4)) combine_kernel(CombineParams p) {
+  constexpr int kWarps = WPH > 4 ? WPH : 4, kHeads = kWarps / WPH;
+  __shared__ MergeState s_st[kWarps][32];
   // wait for the decode grid this launch depends on (no-op without one)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hq = blockIdx.x * 4 + warp, b = blockIdx.y;
-  if (hq >= p.num_q_heads) return;
+  const int hw = warp / WPH, wi = warp % WPH;  // head of the CTA, warp within the head
+  const int hq = blockIdx.x * kHeads + hw, b = blockIdx.y;
+  const bool active = hq < p.num_q_heads;
   constexpr int D = kHeadDim;
   constexpr int C = 16;  // slots per batch of loads
-  int S;  // slots of this (sequence, head)
-  if (p.persistent) {
-    const int h = hq / (p.num_q_heads / p.num_kv_heads);
-    S = __ldcg(p.unit_slots + b * p.num_kv_heads + h);
-  } else {
-    const int32_t* len = p.lens + (int64_t)b * kLensStride;
-    const int nblk = max(len[kLenQ], len[kLenQV]) / p.group_k;
-    S = (nblk + p.blocks_per_split - 1) / p.blocks_per_split + 1;
+  int S = 0;  // slots of this (sequence, head)
+  if (active) {
+    if (p.persistent) {
+      const int h = hq / (p.num_q_heads / p.num_kv_heads);
+      S = __ldcg(p.unit_slots + b * p.num_kv_heads + h);
+    } else {
+      const int32_t* len = p.lens + (int64_t)b * kLensStride;
+      const int nblk = max(len[kLenQ], len[kLenQV]) / p.group_k;
+      S = (nblk + p.blocks_per_split - 1) / p.blocks_per_split + 1;
+    }
   }
   const int64_t base = ((int64_t)b * p.num_q_heads + hq) * p.slots;
   const float2* ml_p = p.ws_ml + base;
   const float4* o_p = reinterpret_cast<const float4*>(p.ws_o + base * D) + lane;  // slot s at o_p[s * D / 4]
-  float M = -INFINITY, lsum = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f);  // hadamard: the exact-token slot 0, kept apart
+  MergeState st{-INFINITY, 0.f, make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
   const bool rot = p.hadamard && !p.persistent;
-  for (int s0 = 0; s0 < S; s0 += C) {
+  for (int s0 = wi; s0 < S; s0 += C * WPH) {
     float2 ml[C];
     float4 v[C];
 #pragma unroll
     for (int e = 0; e < C; ++e) {
-      const bool in = s0 + e < S;
-      ml[e] = in ? __ldcg(ml_p + s0 + e) : make_float2(-INFINITY, 0.f);
-      v[e] = in ? __ldcg(o_p + (s0 + e) * (D / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const int s = s0 + e * WPH;
+      const bool in = s < S;
+      ml[e] = in ? __ldcg(ml_p + s) : make_float2(-INFINITY, 0.f);
+      v[e] = in ? __ldcg(o_p + (int64_t)s * (D / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    float mc = M;
+    float mc = st.M;
 #pragma unroll
     for (int e = 0; e < C; ++e)
       if (ml[e].y > 0.f) mc = fmaxf(mc, ml[e].x);
     if (mc == -INFINITY) continue;  // nothing yet
-    const float r = M == -INFINITY ? 0.f : exp2f(M - mc);
-    acc.x *= r;
-    acc.y *= r;
-    acc.z *= r;
-    acc.w *= r;
-    acc0.x *= r;
-    acc0.y *= r;
-    acc0.z *= r;
-    acc0.w *= r;
-    lsum *= r;
-    M = mc;
+    const float r = st.M == -INFINITY ? 0.f : exp2f(st.M - mc);
+    st.acc = make_float4(st.acc.x * r, st.acc.y * r, st.acc.z * r, st.acc.w * r);
+    st.acc0 = make_float4(st.acc0.x * r, st.acc0.y * r, st.acc0.z * r, st.acc0.w * r);
+    st.l *= r;
+    st.M = mc;
 #pragma unroll
     for (int e = 0; e < C; ++e) {
       if (ml[e].y > 0.f) {
-        const float w = exp2f(ml[e].x - M);
-        float4& a = (rot && s0 + e == 0) ? acc0 : acc;
+        const float w = exp2f(ml[e].x - st.M);
+        float4& a = (rot && s0 + e * WPH == 0) ? st.acc0 : st.acc;
         a.x += w * v[e].x;
         a.y += w * v[e].y;
         a.z += w * v[e].z;
         a.w += w * v[e].w;
-        lsum += w * ml[e].y;
+        st.l += w * ml[e].y;
       }
     }
   }
+  if constexpr (WPH > 1) {
+    s_st[warp][lane] = st;
+    __syncthreads();
+    if (wi != 0) return;
+#pragma unroll
+    for (int i = 1; i < WPH; ++i) merge_into(st, s_st[warp + i][lane]);
+  }
+  if (!active) return;
+  float4 acc = st.acc;
+  const float lsum = st.l;
   if (rot) {
     // the quantized part back to the original basis: acc . H over the warp's
     // 128 channels (lane L holds 4L..4L+3): butterflies of half-width 1 and 2
@@ -397,7 +425,7 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineParams p) {
       }
     }
     const float rs = (float)(1.0 / sqrt((double)D));
-    acc = make_float4(x[0] * rs + acc0.x, x[1] * rs + acc0.y, x[2] * rs + acc0.z, x[3] * rs + acc0.w);
+    acc = make_float4(x[0] * rs + st.acc0.x, x[1] * rs + st.acc0.y, x[2] * rs + st.acc0.z, x[3] * rs + st.acc0.w);
   }
   float r[4] = {0.f, 0.f, 0.f, 0.f};
   if (lsum > 0.f) {
@@ -466,12 +494,17 @@ cudaError_t launch_decode(const DecodeParams& p, int max_splits, cudaStream_t st
 
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream) {
   if (p.batch <= 0) return cudaSuccess;
+  // Warps per (sequence, query head): enough that each merges at most ~32
+  // slots (two rounds of loads), from the most slots a unit can use.
+  const int most = p.persistent ? p.max_unit_slots : p.slots;
+  const int wph = most <= 32 ? 1 : most <= 64 ? 2 : most <= 128 ? 4 : 8;
+  const int warps = wph > 4 ? wph : 4, heads = warps / wph;
   // Programmatic dependent launch: the combine grid may be scheduled while
   // the decode grid (which allows it at its start) is still running; each
   // combine CTA waits for the decode grid to complete before it reads.
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((p.num_q_heads + 3) / 4, p.batch);
-  cfg.blockDim = dim3(128);
+  cfg.gridDim = dim3((p.num_q_heads + heads - 1) / heads, p.batch);
+  cfg.blockDim = dim3(32 * warps);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -483,7 +516,12 @@ cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream) {
                          p.L.lens,       p.out_dtype,      p.num_q_heads,   p.L.num_kv_heads,
                          p.slots,        p.L.group_k,      p.blocks_per_split, p.persistent, p.L.hadamard,
                          p.q_heads,      p.q_rows};
-  return cudaLaunchKernelEx(&cfg, combine_kernel, cp);
+  switch (wph) {
+    case 1: return cudaLaunchKernelEx(&cfg, combine_kernel<1>, cp);
+    case 2: return cudaLaunchKernelEx(&cfg, combine_kernel<2>, cp);
+    case 4: return cudaLaunchKernelEx(&cfg, combine_kernel<4>, cp);
+    default: return cudaLaunchKernelEx(&cfg, combine_kernel<8>, cp);
+  }
 }
 
 }  // namespace kvq

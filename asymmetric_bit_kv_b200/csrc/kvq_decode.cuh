@@ -43,6 +43,7 @@ struct DecodeParams {
   int32_t total_blocks; // T, persistent mode: work items of all units
   int32_t num_ctas;     // persistent mode
   int32_t after_flush;  // persistent mode: launched after the flush kernel of a fused decode step
+  int32_t max_unit_slots;  // persistent mode: a bound on the slots any unit uses (sizes the combine)
   // Query rows. A unit (sequence b, KV head h) has num_q_heads / Hkv rows:
   // row j is query token t = j / (q_heads / Hkv) of this launch and head
   // h * (q_heads / Hkv) + j % (q_heads / Hkv), read from row

@@ -2,21 +2,35 @@
 
 One step = append one new token to every sequence of a batch (quantizing a
 G-token block whenever a ring fills) + decode attention for one query per
-sequence over the whole cache. The workload is the Llama-3-8B-shaped GQA
-layer: batch 32, 32 query / 8 KV heads, head_dim 128, context 8192, bf16
-keys N(0,1) x log-normal channel magnitudes and values N(0,1), keys 2-bit per
-channel in groups of 64 tokens, values 4-bit per token in groups of 64
-channels, residual window 128. `--workload kv1` runs the KV1 card's BQ2_0
-layout on the same shapes (2-bit keys and values per token over whole head
-vectors, Hadamard rotation, 4 exact sink tokens).
+sequence over the whole cache, in every layer of the workload. Workloads
+(`--workload`, synthetic and seeded, shapes of the models named):
+
+* llama3 (default, the headline): Llama-3-8B-shaped GQA layer, batch 32,
+  32 query / 8 KV heads, head_dim 128, context 8192, bf16 keys N(0,1) x
+  log-normal channel magnitudes, values N(0,1); keys 2-bit per channel in
+  groups of 64 tokens, values 4-bit per token in groups of 64 channels,
+  residual window 128.
+* tiny: 1 sequence, 8 heads (MHA), context 1024, fp16, K2/V2 in groups of
+  32, residual 32 (the oracle's small case).
+* llama2: Llama-2-7B-shaped MHA layer, batch 8, 32 heads, context 4096,
+  K2/V2 in groups of 32, residual 128; 256 steps by default, each timed as
+  its append and its attention separately.
+* long: one sequence of 131072 tokens, 32/8 heads, K2/V2 in groups of 128,
+  residual 128; plus a 4096-token prefill chunk appended to an empty
+  sequence in one call, timed on its own.
+* qwen3: Qwen3-8B-shaped 36 layers, 64 ragged sequences (context uniform in
+  [1024, 32768]), 32/8 heads, K4/V2 (layers 0-3 K8/V4) in groups of 64,
+  residual 64; paged block records; a step runs every layer.
+* kv1: the llama3 shapes with the KV1 card's BQ2_0 cache (2-bit keys and
+  values per token over whole head vectors, Hadamard rotation, 4 sinks).
 
 Timing: W warm-up steps, then exactly K steps between barriers and device
 synchronisations, timed with CUDA events on the launching stream; the job
-value is the max over ranks. Each step works on the next of several
-independent cache replicas, so every step streams a different cache (235 MB;
-151 MB for kv1: more than the 126 MB L2) and every replica's context grows only by K/replicas
-tokens. Multi-GPU runs (torchrun) give every rank its own replicas: weak
-scaling, no collective on the data path.
+value is the max over ranks. Steps cycle over independent cache replicas
+whose total size exceeds the 126 MB L2 many times over, so no step finds its
+cache in L2, and each replica grows by only K/replicas tokens. Multi-GPU
+runs (torchrun, or `--gpus N`, which launches them) give every rank its own
+replicas: weak scaling, no collective on the data path.
 
 `--impl reference` times the CPU oracle (the plain restatement of the method
 used by the tests) on the host cores instead, on a bounded sample of the same
@@ -40,28 +54,45 @@ sys.path.insert(0, ROOT)
 METRIC = "quantized-KV decode attention: KV tokens/s and achieved HBM GB/s vs B200 peak"
 UNIT = "KV tokens/s"
 
+# Per workload: cache replicas, default steps / warm-up, page size (0:
+# contiguous records), and what else is timed.
+SPECS = {
+    "llama3": dict(replicas=16, steps=2048, warmup=32, page_blocks=0),
+    "kv1": dict(replicas=16, steps=2048, warmup=32, page_blocks=0),
+    "tiny": dict(replicas=256, steps=2048, warmup=32, page_blocks=0),
+    "llama2": dict(replicas=16, steps=256, warmup=8, page_blocks=0, split_append=True),
+    "long": dict(replicas=16, steps=512, warmup=8, page_blocks=0, prefill_chunk=True),
+    "qwen3": dict(replicas=1, steps=16, warmup=3, page_blocks=16),
+}
+
 
 def _args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2048)
-    ap.add_argument("--warmup", type=int, default=32)
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default: the workload's)")
+    ap.add_argument("--warmup", type=int, default=None, help="warm-up steps (default: the workload's)")
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
-    ap.add_argument("--replicas", type=int, default=16)
+    ap.add_argument("--replicas", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="llama3", choices=["llama3", "kv1"],
-                    help="llama3: the headline KIVI layer (default); kv1: the same shapes with the KV1 card's BQ2_0 cache")
+    ap.add_argument("--workload", default="llama3", choices=sorted(SPECS))
     ap.add_argument("--query-tokens", type=int, default=1,
                     help="query tokens per sequence and step (> 1: append them, then kvq_decode_attention_multi)")
-    ap.add_argument("--page-blocks", type=int, default=0,
+    ap.add_argument("--page-blocks", type=int, default=None,
                     help="block records in pages of this many blocks drawn from a pool (0: contiguous)")
-    return ap.parse_args()
+    a = ap.parse_args()
+    spec = SPECS[a.workload]
+    a.steps = spec["steps"] if a.steps is None else a.steps
+    a.warmup = spec["warmup"] if a.warmup is None else a.warmup
+    a.replicas = spec["replicas"] if a.replicas is None else a.replicas
+    a.page_blocks = spec["page_blocks"] if a.page_blocks is None else a.page_blocks
+    return a
 
 
 def _bench_workload(name):
     from asymmetric_bit_kv_b200 import workloads as W
 
-    return W.llama3_8b_gqa() if name == "llama3" else W.kv1_bq2_gqa()
+    return {"llama3": W.llama3_8b_gqa, "kv1": W.kv1_bq2_gqa, "tiny": W.tiny_mha, "llama2": W.llama2_7b_mha,
+            "long": W.long_context_gqa, "qwen3": W.qwen3_8b_layers}[name]()
 
 
 def _layout(wl):
@@ -156,8 +187,17 @@ class ClockSampler:
 # CPU oracle baseline (host cores, spawned worker processes)
 # --------------------------------------------------------------------------
 
-def _oracle_worker(conn, unit, ctx, wname="llama3"):
-    """One unit of the workload -- one (sequence, KV head) with its 4 query
+def _oracle_unit(wname):
+    """(context, layer) of the oracle's unit of a workload: its (median)
+    context, in a layer of its most common bit widths."""
+    wl = _bench_workload(wname)
+    ctx = sorted(wl.context)[len(wl.context) // 2]
+    layer = 4 if wl.num_layers > 4 else 0
+    return ctx, layer
+
+
+def _oracle_worker(conn, unit, wname="llama3"):
+    """One unit of the workload -- one (sequence, KV head) with its query
     heads -- held in the oracle. Prefill is untimed; each 'step' command appends
     one token and runs decode attention, and replies with the tokens attended."""
     from threadpoolctl import threadpool_limits
@@ -167,16 +207,19 @@ def _oracle_worker(conn, unit, ctx, wname="llama3"):
 
     with threadpool_limits(1):
         wl = _bench_workload(wname)
+        ctx, layer = _oracle_unit(wname)
         sinks, k_axis, rot = _layout(wl)
         g = wl.num_q_heads // wl.num_kv_heads
         unit_wl = W.Workload(wl.name, 1, g, 1, wl.head_dim, [ctx], wl.k_bits, wl.v_bits, wl.group_k, wl.group_v,
-                             wl.residual, wl.kv_dtype, wl.key_dist, wl.value_std, wl.seed)
+                             wl.residual, wl.kv_dtype, wl.key_dist, wl.value_std, wl.seed,
+                             num_layers=wl.num_layers, outliers_per_head=wl.outliers_per_head,
+                             outlier_scale=wl.outlier_scale, outlier_channels=wl.outlier_channels)
         extra = 4096
-        k, v = W.generate_tokens(unit_wl, 0, [ctx + extra], seed_offset=7000 + unit)
+        k, v = W.generate_tokens(unit_wl, layer, [ctx + extra], seed_offset=7000 + unit)
         k = k.float().numpy()
         v = v.float().numpy()
-        c = O.SequenceCache(1, wl.head_dim, wl.k_bits[0], wl.v_bits[0], wl.group_k, wl.group_v, wl.residual,
-                            sinks=sinks, k_axis=k_axis, hadamard=bool(rot))
+        c = O.SequenceCache(1, wl.head_dim, wl.k_bits[layer], wl.v_bits[layer], wl.group_k, wl.group_v,
+                            wl.residual, sinks=sinks, k_axis=k_axis, hadamard=bool(rot))
         c.append(k[:ctx], v[:ctx])
         conn.send("ready")
         i = 0
@@ -184,7 +227,7 @@ def _oracle_worker(conn, unit, ctx, wname="llama3"):
             cmd = conn.recv()
             if cmd != "step":
                 break
-            q = W.generate_queries(unit_wl, 0, 1, step=i)[0].float().numpy()
+            q = W.generate_queries(unit_wl, layer, 1, step=i)[0].float().numpy()
             t = ctx + (i % extra)
             c.append(k[t:t + 1], v[t:t + 1])
             O.decode_attention(c, q, wl.softmax_scale)
@@ -196,29 +239,30 @@ def _oracle_worker(conn, unit, ctx, wname="llama3"):
 class OracleRunner:
     """`workers` spawned processes, one workload unit each, stepped together."""
 
-    def __init__(self, workers: int, ctx: int = 8192, wname: str = "llama3"):
+    def __init__(self, workers: int, wname: str = "llama3"):
         import multiprocessing as mp
 
         ctxm = mp.get_context("spawn")
         self.conns, self.procs = [], []
         for u in range(workers):
             a, b = ctxm.Pipe()
-            p = ctxm.Process(target=_oracle_worker, args=(b, u, ctx, wname), daemon=True)
+            p = ctxm.Process(target=_oracle_worker, args=(b, u, wname), daemon=True)
             p.start()
             self.conns.append(a)
             self.procs.append(p)
         for c in self.conns:
             assert c.recv() == "ready"
         self.workers = workers
-        self.ctx = ctx
+        self.wname = wname
+        self.hkv = _bench_workload(wname).num_kv_heads
 
     def step(self):
         t0 = time.perf_counter()
         for c in self.conns:
             c.send("step")
-        # a unit holds one of the workload's 8 KV heads: count KV tokens
-        # (all heads of a token) as unit tokens / 8
-        toks = sum(c.recv() for c in self.conns) / 8
+        # a unit holds one of the workload's KV heads: count KV tokens (all
+        # heads of a token) as unit tokens / Hkv
+        toks = sum(c.recv() for c in self.conns) / self.hkv
         return toks, time.perf_counter() - t0
 
     def close(self):
@@ -231,13 +275,24 @@ class OracleRunner:
             p.join(timeout=10)
 
     def describe(self, steps):
-        return (f"{self.workers} units of the workload in parallel, one (sequence, KV head) with its 4 query heads "
-                f"each (context {self.ctx}); a step = append one token + fp64 decode attention per unit; "
-                f"{steps} timed steps; KV tokens counted as unit tokens / 8 KV heads")
+        wl = _bench_workload(self.wname)
+        ctx, layer = _oracle_unit(self.wname)
+        g = wl.num_q_heads // wl.num_kv_heads
+        return (f"{self.workers} units of the workload in parallel, one (sequence, KV head) with its {g} query "
+                f"head(s) each (context {ctx}, layer {layer}'s bits); a step = append one token + fp64 decode "
+                f"attention per unit; {steps} timed steps; KV tokens counted as unit tokens / {self.hkv} KV heads")
 
 
-def cpu_oracle_baseline(steps: int = 100, warmup: int = 2, wname: str = "llama3"):
+def _oracle_steps(wname):
+    """Oracle steps of a bounded baseline sample (about 10-30 s of host work):
+    fewer for longer contexts."""
+    ctx, _ = _oracle_unit(wname)
+    return max(3, min(100, int(100 * 8192 / max(ctx, 1024))))
+
+
+def cpu_oracle_baseline(wname="llama3", steps=None, warmup=2):
     workers = max(1, min(os.cpu_count() or 1, 16))
+    steps = _oracle_steps(wname) if steps is None else steps
     run = OracleRunner(workers, wname=wname)
     try:
         for _ in range(warmup):
@@ -269,32 +324,38 @@ def cpu_oracle_baseline(steps: int = 100, warmup: int = 2, wname: str = "llama3"
 # the library arm
 # --------------------------------------------------------------------------
 
-def _cache_mb(wl):
-    """Quantized cache bytes of one replica (MB), from the record layout of
-    the method (codes + fp16 scale and zero point per group)."""
-    D, G, Gv = wl.head_dim, wl.group_k, wl.group_v
-    per_token_keys = _layout(wl)[1]
-    kgroups = D / Gv if per_token_keys else D / G
-    per_tok = wl.num_kv_heads * (D * (wl.k_bits[0] + wl.v_bits[0]) / 8 + 4 * kgroups + 4 * D / Gv)
-    return wl.batch * wl.context[0] * per_tok / 1e6
-
-
-def _workload_config(wl, replicas, world, mean_ctx=None):
+def _workload_config(wl, a, world, mean_ctx=None, cache_mb=None):
     """The `config` object of the JSON line (shared by both arms)."""
+    ctx = wl.context
     cfg = {
         "workload": wl.name,
-        "batch": wl.batch, "num_q_heads": wl.num_q_heads, "num_kv_heads": wl.num_kv_heads,
-        "head_dim": wl.head_dim, "context": wl.context[0], "k_bits": wl.k_bits[0], "v_bits": wl.v_bits[0],
+        "batch": wl.batch, "num_layers": wl.num_layers, "num_q_heads": wl.num_q_heads,
+        "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+        "context": ctx[0] if len(set(ctx)) == 1 else {"min": min(ctx), "max": max(ctx),
+                                                       "mean": sum(ctx) / len(ctx)},
+        "k_bits": wl.k_bits[0] if len(set(wl.k_bits)) == 1 else wl.k_bits,
+        "v_bits": wl.v_bits[0] if len(set(wl.v_bits)) == 1 else wl.v_bits,
         "group_k": wl.group_k, "group_v": wl.group_v, "residual": wl.residual,
         "sinks": _layout(wl)[0], "key_axis": "token" if _layout(wl)[1] else "channel", "hadamard": _layout(wl)[2],
-        "kv_dtype": "bf16", "out_dtype": "bf16",
-        "replicas": replicas,
-        "l2": f"inputs larger than L2: each step reads a different replica's ~{_cache_mb(wl):.0f} MB cache",
+        "kv_dtype": str(wl.kv_dtype).replace("torch.", ""), "out_dtype": str(wl.kv_dtype).replace("torch.", ""),
+        "replicas": a.replicas,
         "parallelism": f"dp{world} (independent replicas per rank)",
     }
+    if cache_mb is not None:
+        cfg["l2"] = (f"inputs larger than L2: each step reads a different replica's ~{cache_mb:.0f} MB cache "
+                     f"({a.replicas} replicas, {a.replicas * cache_mb:.0f} MB in all)")
+    if a.page_blocks:
+        cfg["page_blocks"] = a.page_blocks
+    if a.query_tokens > 1:
+        cfg["query_tokens"] = a.query_tokens
     if mean_ctx is not None:
         cfg["mean_context_timed"] = mean_ctx
     return cfg
+
+
+def _flushes(n, T, R, G):
+    """Blocks a ring of n tokens (R slots) flushes when T tokens arrive one by one."""
+    return 0 if n + T <= R else -(-(n + T - R) // G)
 
 
 def run_kvq(a):
@@ -310,68 +371,83 @@ def run_kvq(a):
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    spec = SPECS[a.workload]
     wl = _bench_workload(a.workload)
     sinks, k_axis, rot = _layout(wl)
-    # tensor-core layers take the new token inside the decode launch: per-channel
-    # keys without the rotation, or per-token keys over whole head vectors
-    fused = (k_axis == 0 and not rot) or (k_axis == 1 and wl.group_v == wl.head_dim)
-    B, Hq, Hkv, D = wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim
-    ctx = wl.context[0]
+    B, Hq, Hkv, D, NL = wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.num_layers
+    G, Rw = wl.group_k, wl.residual
+    ctx = list(wl.context)
     R = a.replicas
+    T = a.query_tokens  # query tokens per sequence and step (their keys and values are appended first)
+    split_append = spec.get("split_append", False) and T == 1
     steps_per_rep = math.ceil((a.warmup + 2 * a.steps) / R) + 2
-    cap = ctx + steps_per_rep * a.query_tokens + wl.group_k
-    cfg = CacheConfig(1, B, Hq, Hkv, D, cap, wl.group_k, wl.group_v, wl.residual, wl.kv_dtype, wl.k_bits, wl.v_bits,
-                      sink_tokens=sinks, k_axis=[k_axis], hadamard=rot, page_blocks=a.page_blocks,
-                      pool_pages=B * -(-(cap // wl.group_k) // a.page_blocks) if a.page_blocks else 0)
+    cap = max(ctx) + sinks + steps_per_rep * T + G
+    pool_pages = 0
+    if a.page_blocks:
+        pool_pages = sum(-(-((c + steps_per_rep * T + G) // G + 1) // a.page_blocks) for c in ctx) + B
+    cfg = CacheConfig(NL, B, Hq, Hkv, D, cap, G, wl.group_v, Rw, wl.kv_dtype, wl.k_bits, wl.v_bits,
+                      sink_tokens=sinks, k_axis=[k_axis] * NL, hadamard=rot, page_blocks=a.page_blocks,
+                      pool_pages=pool_pages)
     caches = []
     for r in range(R):
         c = KVCache(cfg, dev)
-        k, v = W.generate_tokens(wl, 0, [ctx] * B, device=dev, seed_offset=replica_seed(rank, r))
-        c.append(0, k, v, [ctx] * B)
-        del k, v
+        for layer in range(NL):
+            k, v = W.generate_tokens(wl, layer, ctx, device=dev, seed_offset=replica_seed(rank, r))
+            c.append(layer, k, v, ctx)
+            del k, v
         caches.append(c)
     torch.cuda.synchronize()
+    lib = caches[0].lib
     gen = torch.Generator(device=dev).manual_seed(12345 + rank)
     pool = 64  # distinct per-step inputs, reused round-robin
-    T = a.query_tokens  # query tokens per sequence and step (their keys and values are appended first)
     new_k = torch.randn(pool, B * T, Hkv, D, generator=gen, device=dev).to(wl.kv_dtype)
     new_v = torch.randn(pool, B * T, Hkv, D, generator=gen, device=dev).to(wl.kv_dtype)
     qs = torch.randn(pool, B * T, Hq, D, generator=gen, device=dev).to(wl.kv_dtype)
     out = torch.empty(B * T, Hq, D, dtype=wl.kv_dtype, device=dev)
     stream = torch.cuda.current_stream()
-    # per-step inputs as views made once, so that the timed loop only enqueues
-    views = [(new_k[j], new_v[j], qs[j]) for j in range(pool)]
-    # quantized bytes per token (all KV heads): the library's block record
-    # (codes, scales and zero points of G tokens of one KV head) / G
-    bytes_tok = Hkv * caches[0].layout(0).record_bytes / wl.group_k
+    oty = K.KVQ_BF16 if wl.kv_dtype == torch.bfloat16 else K.KVQ_F16
+    scale = float(wl.softmax_scale)
+    # quantized bytes per token (all KV heads) of each layer: the library's
+    # block record (codes, scales and zero points of G tokens of one KV head) / G
+    bytes_tok = [Hkv * caches[0].layout(layer).record_bytes / G for layer in range(NL)]
+    # tensor-core layers take the new token inside the decode launch:
+    # per-channel keys without the rotation, or per-token keys over whole head
+    # vectors, blocks of >= 64 tokens, 2-bit values in groups of >= 64
+    fused = G >= 64 and ((k_axis == 0 and not rot) or (k_axis == 1 and wl.group_v == D)) and \
+        (min(wl.v_bits) > 2 or wl.group_v >= 64)
 
-    G, Rw = wl.group_k, wl.residual
-
-    # The device-timed loop calls the C entry point kvq_decode_step (append
-    # one token per sequence + decode attention; the append rides inside the
-    # decode launch unless a ring must be flushed) with arguments prepared
+    # The device-timed loop calls the C entry points with arguments prepared
     # here, so that Python overhead per call stays far below the GPU time of a
     # step; the e2e leg below goes through the Python binding.
-    lib = caches[0].lib
-    c_step = lib.kvq_decode_step
-    c_append, c_multi = lib.kvq_append, lib.kvq_decode_attention_multi
+    c_step, c_append, c_decode, c_multi = (lib.kvq_decode_step, lib.kvq_append, lib.kvq_decode_attention,
+                                           lib.kvq_decode_attention_multi)
     t_lens = K.lens_array([T] * B)
     sh = stream.cuda_stream
     handles = [c.handle for c in caches]
-    ptrs = [(kk.data_ptr(), vv.data_ptr(), qq.data_ptr()) for kk, vv, qq in views]
-    optr, oty, scale = out.data_ptr(), 1, float(wl.softmax_scale)  # out dtype code 1 = bf16
+    ptrs = [(kk.data_ptr(), vv.data_ptr(), qq.data_ptr()) for kk, vv, qq in zip(new_k, new_v, qs)]
+    optr = out.data_ptr()
 
     def step(i, r, ev=None):
+        """One step on replica r: every layer; ev = (start, after append, end)
+        events (the middle one only with split_append)."""
         kp, vp, qp = ptrs[i % pool]
         h = handles[r]
         if ev is not None:
             ev[0].record(stream)
-        if T == 1:
-            st = c_step(h, 0, kp, vp, qp, optr, oty, scale, B, sh)
-        else:  # the T tokens' keys and values, then the T queries of every sequence
-            st = c_append(h, 0, kp, vp, t_lens, B, sh) or c_multi(h, 0, qp, optr, oty, scale, B, T, sh)
+        st = 0
+        for layer in range(NL):
+            if split_append:
+                st = st or c_append(h, layer, kp, vp, t_lens, B, sh)
+                if ev is not None and layer == NL - 1:
+                    ev[1].record(stream)
+                st = st or c_decode(h, layer, qp, optr, oty, scale, B, sh)
+            elif T == 1:
+                st = st or c_step(h, layer, kp, vp, qp, optr, oty, scale, B, sh)
+            else:  # the T tokens' keys and values, then the T queries of every sequence
+                st = st or c_append(h, layer, kp, vp, t_lens, B, sh) or c_multi(h, layer, qp, optr, oty, scale, B, T,
+                                                                               sh)
         if ev is not None:
-            ev[1].record(stream)
+            ev[2].record(stream)
         if st:
             raise RuntimeError(f"kvq call failed: {lib.kvq_last_error().decode()}")
 
@@ -382,45 +458,50 @@ def run_kvq(a):
         dist.barrier()
 
     # Per-step accounting, computed before the timed loop so that the loop only
-    # enqueues work: the (quantized, ring) lengths of every replica follow the
-    # flush rule (a token that finds a full ring first moves G ring tokens into
-    # the quantized cache), checked against the library's host mirror after.
-    lens = [[list(caches[r].lengths(0, b)) for b in range(B)] for r in range(R)]
-    plan = []  # (replica, launches, algorithmic bytes of the step, KV tokens attended)
+    # enqueues work: the (quantized, ring, pages) state of every replica follows
+    # the flush rule (a token that finds a full ring first moves G ring tokens
+    # into the quantized cache), checked against the library's host mirror after.
+    lens = [[[list(caches[r].lengths(layer, b)) for b in range(B)] for layer in range(NL)] for r in range(R)]
+    pages = [[[-(-(q // G) // a.page_blocks) if a.page_blocks else 0 for q, _ in row] for row in rep] for rep in lens]
+    plan = []  # (replica, launches, algorithmic bytes, KV tokens attended, any flush)
+    groups, t0, ngr = 0, 0, Hq // Hkv  # decode passes of a multi-token step (<= 8 query rows per KV head each)
+    while t0 < T:
+        tp = 1
+        while 2 * tp * ngr <= 8 and t0 + 2 * tp <= T:
+            tp *= 2
+        groups, t0 = groups + 1, t0 + tp
     for i in range(a.steps):
         r = (a.warmup + i) % R
-        # fused: decode + combine; a step that flushes a ring first runs the
-        # quantize and ring-write kernels (unfused: ring write, split kernel,
-        # combine, and the quantize kernel on a flush)
-        ab, tk = T * (2 * B * Hq * D * 2 + 2 * (2 * B * Hkv * D * 2)), 0  # q in, out; new k, v in and into the ring
-        ab += B * sinks * Hkv * D * 2 * 2  # the exact sink tokens
-        tk += B * T * sinks
+        ab = tk = launches = 0
         flush = False
-        for b in range(B):
-            qn, n = lens[r][b]
-            f = 0 if n + T <= Rw else -(-(n + T - Rw) // G)  # blocks the T appends flush
-            flush = flush or f > 0
-            qn, n = qn + f * G, n + T - f * G
-            lens[r][b] = [qn, n]
-            ab += qn * bytes_tok + n * Hkv * D * 2 * 2
-            tk += T * (qn + n) - T * (T - 1) // 2  # query t sees the tokens up to its own position
-        if T == 1:
-            # fused: prep (plan; on a flush step also the quantize CTAs),
-            # decode, combine; unfused: ring write (+ quantize on a flush),
-            # split kernel, combine
-            launches = 3 if fused else (3 + (1 if flush else 0))
-        else:
-            # append (ring write, + quantize on a flush), then decode + combine
-            # per group of query tokens (at most 8 query rows per KV head)
-            groups, t0, ngr = 0, 0, Hq // Hkv
-            while t0 < T:
-                tp = 1
-                while 2 * tp * ngr <= 8 and t0 + 2 * tp <= T:
-                    tp *= 2
-                groups, t0 = groups + 1, t0 + tp
-            launches = 1 + (1 if flush else 0) + 2 * groups
+        for layer in range(NL):
+            ab += T * (2 * B * Hq * D * 2 + 2 * (2 * B * Hkv * D * 2))  # q in, out; new k, v in and into the ring
+            ab += B * sinks * Hkv * D * 2 * 2  # the exact sink tokens
+            tk += B * T * sinks
+            lflush = new_pages = False
+            for b in range(B):
+                qn, n = lens[r][layer][b]
+                f = _flushes(n, T, Rw, G)
+                lflush = lflush or f > 0
+                qn, n = qn + f * G, n + T - f * G
+                lens[r][layer][b] = [qn, n]
+                if a.page_blocks:
+                    pg = -(-(qn // G) // a.page_blocks)
+                    new_pages = new_pages or pg > pages[r][layer][b]
+                    pages[r][layer][b] = pg
+                ab += qn * bytes_tok[layer] + n * Hkv * D * 2 * 2
+                tk += T * (qn + n) - T * (T - 1) // 2  # query t sees the tokens up to its own position
+            flush = flush or lflush
+            if T == 1 and fused and not split_append:
+                # flush kernel on a flushing step, page-table update when pages
+                # are taken, decode, combine
+                launches += 2 + (1 if lflush else 0) + (1 if new_pages else 0)
+            else:
+                # append (page-table update, quantize on a flush, ring write),
+                # then decode + combine per pass
+                launches += 1 + (1 if lflush else 0) + (1 if new_pages else 0) + 2 * groups
         plan.append((r, launches, ab, tk, flush))
-    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+    events = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(a.steps)]
     launches = sum(x[1] for x in plan)
     alg_total = float(sum(x[2] for x in plan))
     tok_total = sum(x[3] for x in plan)
@@ -443,22 +524,55 @@ def run_kvq(a):
         dist.barrier()
     clk = clocks.stop()
     for r in range(R):
-        for b in range(B):
-            assert tuple(lens[r][b]) == caches[r].lengths(0, b), "step accounting out of sync with the cache"
+        for layer in range(NL):
+            for b in range(B):
+                assert tuple(lens[r][layer][b]) == caches[r].lengths(layer, b), "step accounting out of sync"
     ms = e0.elapsed_time(e1)
-    call_ms = [x[0].elapsed_time(x[1]) for x in events]
+    call_ms = [x[0].elapsed_time(x[2]) for x in events]
+    app_ms = [x[0].elapsed_time(x[1]) for x in events] if split_append else [0.0]
     dec_ms = sum(call_ms)
     fl = [m for m, x in zip(call_ms, plan) if x[4]]
     nf = [m for m, x in zip(call_ms, plan) if not x[4]]
     fl_us = 1e3 * sum(fl) / len(fl) if fl else 0.0
     nf_us = 1e3 * sum(nf) / len(nf) if nf else 0.0
-    ms, dec_ms, fl_us, nf_us = cross_rank_max([ms, dec_ms, fl_us, nf_us], world, dev)
+    app_us = 1e3 * sum(app_ms) / len(app_ms)
+    ms, dec_ms, fl_us, nf_us, app_us = cross_rank_max([ms, dec_ms, fl_us, nf_us, app_us], world, dev)
     value = tok_total * world / (ms / 1e3)
     achieved_gbs = alg_total / (dec_ms / 1e3) / 1e9
 
+    # ---- a prefill chunk: one kvq_append of 4096 tokens to an empty sequence
+    prefill = None
+    if spec.get("prefill_chunk"):
+        chunk = wl.extra.get("prefill_chunk", 4096)
+        pc = CacheConfig(1, 1, Hq, Hkv, D, chunk + G, G, wl.group_v, Rw, wl.kv_dtype, wl.k_bits[:1], wl.v_bits[:1],
+                         sink_tokens=sinks, k_axis=[k_axis], hadamard=rot)
+        pcs = [KVCache(pc, dev) for _ in range(8)]
+        ck, cv = W.generate_tokens(wl, 0, [chunk], device=dev, seed_offset=99)
+        flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > L2, written before each run
+        pt = []
+        for rep in range(8 + 3):
+            c = pcs[rep % 8]
+            c.reset()
+            flush_buf.fill_(rep & 0xff)
+            pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            pa.record(stream)
+            c.append(0, ck, cv, [chunk])
+            pb.record(stream)
+            pt.append((pa, pb))
+        torch.cuda.synchronize()
+        us = sorted(x.elapsed_time(y) * 1e3 for x, y in pt[3:])
+        qb = pcs[0].lengths(0, 0)[0] // G
+        in_b = chunk * Hkv * D * 2 * 2
+        out_b = qb * G * bytes_tok[0] + (chunk - qb * G) * Hkv * D * 2 * 2
+        prefill = {"tokens": chunk, "us_median": us[len(us) // 2], "bytes_in": in_b, "bytes_out": int(out_b),
+                   "achieved_gbs": (in_b + out_b) / (us[len(us) // 2] * 1e-6) / 1e9,
+                   "what": "one kvq_append of the chunk to an empty sequence (quantize kernel + ring write), "
+                           "L2 flushed before each run"}
+        del pcs, flush_buf, ck, cv
+
     # ---- end to end through the public API with host buffers ----
     # each step's k, v and q sit back to back in one pinned host buffer and
-    # travel in one host-to-device copy
+    # travel in one host-to-device copy; the last layer's output comes back
     e2e_steps = min(a.steps, 512)
     nk, nq = B * T * Hkv * D, B * T * Hq * D
     hkvq = torch.empty(pool, 2 * nk + nq, dtype=wl.kv_dtype).pin_memory()
@@ -473,12 +587,13 @@ def run_kvq(a):
     tok_e2e = 0
     for i in range(e2e_steps):
         r = (a.warmup + a.steps + i) % R
-        for b in range(B):
-            qn, n = lens[r][b]
-            f = 0 if n + T <= Rw else -(-(n + T - Rw) // G)
-            qn, n = qn + f * G, n + T - f * G
-            lens[r][b] = [qn, n]
-            tok_e2e += T * (sinks + qn + n) - T * (T - 1) // 2
+        for layer in range(NL):
+            for b in range(B):
+                qn, n = lens[r][layer][b]
+                f = _flushes(n, T, Rw, G)
+                qn, n = qn + f * G, n + T - f * G
+                lens[r][layer][b] = [qn, n]
+                tok_e2e += T * (sinks + qn + n) - T * (T - 1) // 2
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -486,26 +601,38 @@ def run_kvq(a):
     f0.record(stream)
     for i in range(e2e_steps):
         r = (a.warmup + a.steps + i) % R
-        j = i % pool
-        dkvq.copy_(hkvq[j], non_blocking=True)
-        if T == 1:
-            caches[r].decode_step(0, dk, dv, dq, out, softmax_scale=wl.softmax_scale, stream=stream)
-            hout.copy_(out, non_blocking=True)
-        else:
-            caches[r].append(0, dk, dv, [T] * B, stream=stream)
-            o = caches[r].decode_attention_multi(0, dq.view(B, T, Hq, D), out_dtype=wl.kv_dtype,
-                                                 softmax_scale=wl.softmax_scale, stream=stream)
-            hout.copy_(o.view(B * T, Hq, D), non_blocking=True)
+        dkvq.copy_(hkvq[i % pool], non_blocking=True)
+        o = out
+        for layer in range(NL):
+            if T == 1:
+                caches[r].decode_step(layer, dk, dv, dq, out, softmax_scale=wl.softmax_scale, stream=stream)
+            else:
+                caches[r].append(layer, dk, dv, [T] * B, stream=stream)
+                o = caches[r].decode_attention_multi(layer, dq.view(B, T, Hq, D), out_dtype=wl.kv_dtype,
+                                                     softmax_scale=wl.softmax_scale, stream=stream)
+        hout.copy_(o.view(B * T, Hq, D), non_blocking=True)
     f1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1)
-    e2e_ms, = cross_rank_max([e2e_ms], world, dev)
+    e2e_ms, = cross_rank_max([f0.elapsed_time(f1)], world, dev)
     e2e_value = tok_e2e * world / (e2e_ms / 1e3)
 
     result = None
     if rank == 0:
         peak, peak_kind = _peaks()
-        traffic = _committed_traffic() if a.workload == "llama3" else None
+        cache_mb = sum(c * bytes_tok[layer] for layer in range(NL) for c in ctx) / 1e6
+        if T > 1:
+            kernel = (f"verify step: {T} tokens appended per sequence (ring write, quantize on a flush), then decode "
+                      "of their queries, causal among them (split-KV decode + combine per group of query tokens)")
+        elif split_append:
+            kernel = ("append (ring write; the quantize kernel when a ring fills), then the split-KV decode kernel "
+                      "and the log-sum-exp combine, per call")
+        elif fused:
+            kernel = ("decode step: one token appended per sequence inside the tensor-core split-KV decode kernel, "
+                      "+ log-sum-exp combine, per call (a step in which rings are full first runs the flush kernel "
+                      "that quantizes their oldest G tokens)")
+        else:
+            kernel = ("decode step: ring write (+ quantize when a ring fills), CUDA-core split-KV decode kernel and "
+                      "log-sum-exp combine, per call")
         result = {
             "metric": METRIC,
             "value": value,
@@ -517,23 +644,14 @@ def run_kvq(a):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "bf16",
-            "dtype_detail": ("bf16 keys, values, queries and outputs; quantizer in fp32; attention on fp16 "
-                             "tensor-core operands (codes exact, q*s and p*s as fp16 high and low parts) and "
-                             "bf16 ones for exact tokens, fp32 accumulation and softmax"),
-            "data": "synthetic (seeded; Llama-3-8B-shaped layer, no model weights)",
-            "config": dict(_workload_config(wl, R, world, tok_total / (a.steps * B * T)),
-                           **({"page_blocks": a.page_blocks} if a.page_blocks else {}),
-                           **({"query_tokens": T} if T > 1 else {})),
+            "dtype": str(wl.kv_dtype).replace("torch.", ""),
+            "dtype_detail": (f"{str(wl.kv_dtype).replace('torch.', '')} keys, values, queries and outputs; quantizer "
+                             "in fp32; attention on fp16 tensor-core operands (codes exact, q*s and p*s as fp16 high "
+                             "and low parts) or fp32 CUDA-core arithmetic, fp32 accumulation and softmax"),
+            "data": f"synthetic (seeded; {wl.name}, model-shaped, no model weights)",
+            "config": _workload_config(wl, a, world, tok_total / (a.steps * NL * B * T), cache_mb),
             "roofline": {
-                "kernel": (f"verify step: {T} tokens appended per sequence (ring write, quantize on a flush), then "
-                           "decode of their queries, causal among them (split-KV decode + combine per group of query "
-                           "tokens)") if T > 1 else
-                          ("decode step: one token appended per sequence inside the split-KV decode kernel, + log-sum-exp "
-                           "combine, per call (a step in which rings are full first runs the flush kernel that quantizes "
-                           "their oldest G tokens)") if fused else
-                          ("decode step: ring write, CUDA-core split-KV decode kernel and log-sum-exp combine, per call "
-                           "(a ring flush adds the quantize kernel)"),
+                "kernel": kernel,
                 "bound": "hbm",
                 "achieved": achieved_gbs,
                 "peak": peak,
@@ -541,14 +659,14 @@ def run_kvq(a):
                 "frac": achieved_gbs / peak,
                 "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
                 "frac_of_8tbs_nominal": achieved_gbs / 8000.0,
-                "traffic": traffic,
-                "decode_us_per_call": dec_ms / a.steps * 1e3,
+                "traffic": _committed_traffic(a.workload),
+                "step_call_us": dec_ms / a.steps * 1e3,
                 "flush_step_us": fl_us if fl else None,
                 "flush_steps": len(fl),
                 "nonflush_step_us": nf_us if nf else None,
                 "nonflush_steps": len(nf),
                 "host_enqueue_us_per_step": host_s / a.steps * 1e6,
-                "alg_bytes_per_call": alg_total / a.steps,
+                "alg_bytes_per_step": alg_total / a.steps,
             },
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": int((dk.numel() + dv.numel() + dq.numel()) * 2),
@@ -556,6 +674,11 @@ def run_kvq(a):
             "gpu_launches": launches,
             "clocks": clk,
         }
+        if split_append:
+            result["roofline"]["append_us_per_step"] = app_us
+            result["roofline"]["attention_us_per_step"] = dec_ms / a.steps * 1e3 - app_us
+        if prefill is not None:
+            result["prefill_chunk"] = prefill
     del caches
     if world > 1:
         dist.barrier()
@@ -576,16 +699,18 @@ def _kernel_source_hash():
     return h.hexdigest()
 
 
-def _committed_traffic():
-    """DRAM bytes (read + write) per decode launch from the committed ncu
-    capture, or None if there is none or the kernel sources changed since."""
+def _committed_traffic(workload="llama3"):
+    """DRAM bytes (read + write) per decode launch of a workload from the
+    committed ncu capture, or None if there is none or the kernel sources
+    changed since."""
     p = os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
         with open(p) as f:
             rec = json.load(f)
     except Exception:
         return None
-    if rec.get("source_sha256") != _kernel_source_hash():
+    rec = rec.get(workload)
+    if not rec or rec.get("source_sha256") != _kernel_source_hash():
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -600,7 +725,7 @@ def run_reference(a):
     wl = _bench_workload(wname)
     workers = max(1, min(os.cpu_count() or 1, 16))
     t_start = time.perf_counter()
-    run = OracleRunner(workers, wl.context[0], wname)
+    run = OracleRunner(workers, wname)
     try:
         for _ in range(a.warmup):
             run.step()
@@ -613,6 +738,7 @@ def run_reference(a):
         run.close()
     value = toks / secs
     base = {"value": value, "unit": UNIT, "cores": workers, "kind": "oracle", "sample": run.describe(a.steps)}
+    cfg_args = type("A", (), {"replicas": 1, "page_blocks": 0, "query_tokens": 1})()
     return {
         "impl": "reference",
         "metric": METRIC,
@@ -626,8 +752,8 @@ def run_reference(a):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f64",
-        "data": "synthetic (seeded; Llama-3-8B-shaped layer, no model weights)",
-        "config": dict(_workload_config(wl, 1, world), units_per_step=workers,
+        "data": f"synthetic (seeded; {wl.name}, model-shaped, no model weights)",
+        "config": dict(_workload_config(wl, cfg_args, world), units_per_step=workers,
                        l2="host run: one bounded sample of the workload per step"),
         "cpu_baseline": base,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -664,7 +790,7 @@ def main():
     rank, world, _ = _dist_env()
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline and a.query_tokens == 1:
-        cpu = cpu_oracle_baseline(wname=a.workload)   # spawned before any CUDA work in this process
+        cpu = cpu_oracle_baseline(a.workload)   # spawned before any CUDA work in this process
     res = run_kvq(a)
     if res is not None:
         res["cpu_baseline"] = cpu
