@@ -118,6 +118,31 @@ kvq_status validate_config(const kvq_config* c) {
 
 int residual_v_of(const kvq_config& c) { return c.residual_v > 0 ? c.residual_v : c.residual; }
 
+// Byte geometry of a layer's block records: runs of tiles of min(G, 64)
+// tokens, each tile part [kc | ksz | vc | vsz]; a block of several tiles with
+// per-channel keys stores its key scales once, before its tiles.
+struct RecordGeometry {
+  int32_t tile_tokens, tile_bytes, tile0_off, rec_ksz_off, kc_off, ksz_off, vc_off, vsz_off;
+  int64_t record_bytes;
+};
+RecordGeometry record_geometry(int G, int D, int kb, int vb, int gv, int k_axis) {
+  using kvq::round_up;
+  RecordGeometry g;
+  g.tile_tokens = std::min(G, 64);
+  const int nt = G / g.tile_tokens;
+  const bool shared_ksz = k_axis == 0 && nt > 1;
+  const int64_t ksz = k_axis == 1 ? kvq::ksz_token_bytes(g.tile_tokens, D, gv) : (shared_ksz ? 0 : kvq::ksz_bytes(D));
+  g.kc_off = 0;
+  g.ksz_off = (int32_t)kvq::kc_bytes(g.tile_tokens, D, kb);
+  g.vc_off = g.ksz_off + (int32_t)ksz;
+  g.vsz_off = g.vc_off + (int32_t)kvq::vc_bytes(g.tile_tokens, D, vb);
+  g.tile_bytes = (int32_t)round_up(g.vsz_off + kvq::vsz_bytes(g.tile_tokens, D, gv), 16);
+  g.rec_ksz_off = shared_ksz ? 0 : -1;
+  g.tile0_off = shared_ksz ? (int32_t)round_up(kvq::ksz_bytes(D), 16) : 0;
+  g.record_bytes = round_up(g.tile0_off + (int64_t)nt * g.tile_bytes, 16);
+  return g;
+}
+
 struct Plan {
   std::vector<int64_t> blocks_off, ring_k_off, ring_v_off, sink_k_off, sink_v_off, record_bytes, pt_off;
   int64_t max_blocks, lens_off, err_off, uslots_off, ws_o_off, ws_ml_off, total;
@@ -137,11 +162,7 @@ Plan make_plan(const kvq_config* c) {
   int64_t off = 0;
   for (int l = 0; l < c->num_layers; ++l) {
     const int kb = c->k_bits[l], vb = c->v_bits[l];
-    const bool per_token = c->k_axis && c->k_axis[l] == 1;
-    const int64_t ksz = per_token ? kvq::ksz_token_bytes(G, D, c->group_v) : kvq::ksz_bytes(D);
-    const int64_t rec = round_up(kvq::kc_bytes(G, D, kb) + ksz + kvq::vc_bytes(G, D, vb) +
-                                     kvq::vsz_bytes(G, D, c->group_v),
-                                 16);
+    const int64_t rec = record_geometry(G, D, kb, vb, c->group_v, c->k_axis ? c->k_axis[l] : 0).record_bytes;
     p.record_bytes.push_back(rec);
     p.blocks_off.push_back(off);
     off = round_up(off + records * rec, 256);
@@ -194,12 +215,17 @@ kvq::LayerView layer_view(const kvq_cache* c, int layer) {
   v.lens = reinterpret_cast<int32_t*>(c->arena + c->lens_off) + (int64_t)layer * cfg.max_batch * kvq::kLensStride;
   v.record_bytes = c->record_bytes[layer];
   v.max_blocks = c->max_blocks;
-  v.kc_off = 0;
-  v.ksz_off = (int32_t)kvq::kc_bytes(G, D, kb);
   v.k_axis = c->k_axis[layer];
   v.hadamard = cfg.hadamard;
-  v.vc_off = v.ksz_off + (int32_t)(v.k_axis == 1 ? kvq::ksz_token_bytes(G, D, cfg.group_v) : kvq::ksz_bytes(D));
-  v.vsz_off = v.vc_off + (int32_t)kvq::vc_bytes(G, D, vb);
+  const RecordGeometry rg = record_geometry(G, D, kb, vb, cfg.group_v, v.k_axis);
+  v.kc_off = rg.kc_off;
+  v.ksz_off = rg.ksz_off;
+  v.vc_off = rg.vc_off;
+  v.vsz_off = rg.vsz_off;
+  v.tile_tokens = rg.tile_tokens;
+  v.tile_bytes = rg.tile_bytes;
+  v.tile0_off = rg.tile0_off;
+  v.rec_ksz_off = rg.rec_ksz_off;
   v.k_bits = kb;
   v.v_bits = vb;
   v.num_kv_heads = cfg.num_kv_heads;
@@ -498,7 +524,7 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const 
     const int per_sm = kvq::mma_ctas_per_sm(L, mp, Hv);
     for (int b = 0; b < batch; ++b) {
       const size_t i = (size_t)layer * cfg.max_batch + b;
-      p.nblk[b] = c->q_len[i] / G;
+      p.nblk[b] = c->q_len[i] / L.tile_tokens;  // tile items of the quantized blocks
       p.nres[b] = c->n_len[i];
       p.nitem[b] = kvq::unit_items(p.nblk[b], p.nres[b], c->s_len[i]);
     }
@@ -924,6 +950,10 @@ kvq_status kvq_get_layout(const kvq_cache* c, int32_t layer, kvq_layout* out) {
   out->page_table = const_cast<int32_t*>(v.page_table);
   out->page_blocks = v.page_blocks;
   out->max_pages = v.max_pages;
+  out->tile_tokens = v.tile_tokens;
+  out->tile_bytes = v.tile_bytes;
+  out->tile0_offset = v.tile0_off;
+  out->rec_ksz_offset = v.rec_ksz_off;
   return KVQ_OK;
 }
 

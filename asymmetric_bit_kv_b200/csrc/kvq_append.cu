@@ -173,6 +173,19 @@ __device__ __forceinline__ int kc_index_p2(int d, int w, int lgW) {
   return d * W + ((((w >> 2) ^ sw)) << 2) + (w & 3);
 }
 
+// Where a block's parts go inside its record (the tile layout of
+// LayerView: tiles of 2^lgT tokens at tile0 + i * tile_bytes).
+struct RecOut {
+  uint8_t* rec;
+  int lgT, tile_bytes, tile0, kc_off, ksz_off, vc_off, vsz_off, rec_ksz;
+  __device__ __forceinline__ uint8_t* tile(int t) const { return rec + tile0 + (int64_t)(t >> lgT) * tile_bytes; }
+  __device__ __forceinline__ int local(int t) const { return t & ((1 << lgT) - 1); }
+};
+__device__ __forceinline__ RecOut rec_out(const LayerView& L, uint8_t* rec) {
+  return RecOut{rec,         __ffs(L.tile_tokens) - 1, L.tile_bytes, L.tile0_off, L.kc_off,
+                L.ksz_off,   L.vc_off,                 L.vsz_off,    L.rec_ksz_off};
+}
+
 // Groups of gv channels of staged rows [0, nt) (tokens t0 + row), BITS-wide
 // codes: one thread per output word (PER = 32/BITS channels); the gv/PER
 // threads of a group combine their min/max with xor shuffles. put_word(t, w,
@@ -203,13 +216,15 @@ __device__ __forceinline__ void quantize_token_groups(const uint8_t* rows, int t
   }
 }
 
-// Key codes packed along the token axis (kc layout) for channels [c0, c0+nc)
+// Key codes packed along the token axis (kc layout, per tile) for channels [c0, c0+nc)
 // and token words [w0, w0 + nw): thread item (channel d, word w) packs
 // tokens w*PER .. w*PER+PER-1 of channel d (staged row of token t at t - t0,
 // column d - sc0) with the fp32 (scale, zero, 1/scale) par(t, d).
 template <bool ROT, int KB, bool PT, class Par>
 __device__ __forceinline__ void pack_key_codes(const uint8_t* rows, int pitch, int t0, int sc0, int c0, int nc, int w0,
-                                               int nw, int lgW, int dt, uint32_t* kc, Par par) {
+                                               int nw, int dt, const RecOut& ro, Par par) {
+  constexpr int LGPER = KB == 2 ? 4 : KB == 4 ? 3 : 2;  // log2 of the tokens per word
+  const int lgWt = ro.lgT - LGPER;                        // log2 of the words per channel per tile
   constexpr int PER = 32 / KB;
   for (int item = threadIdx.x; item < nc * nw; item += kQuantThreads) {
     const int d = c0 + item % nc, w = w0 + item / nc;
@@ -229,7 +244,8 @@ __device__ __forceinline__ void pack_key_codes(const uint8_t* rows, int pitch, i
       const float4 pr = par(0, d);
       word = quant_word_rcp<KB, PER>(x, pr.y, pr.x, pr.z);
     }
-    kc[kc_index_p2(d, w, lgW)] = word;
+    uint8_t* tp = ro.tile(w << LGPER);
+    reinterpret_cast<uint32_t*>(tp + ro.kc_off)[kc_index_p2(d, w & ((1 << lgWt) - 1), lgWt)] = word;
   }
 }
 
@@ -238,9 +254,9 @@ __device__ __forceinline__ void pack_key_codes(const uint8_t* rows, int pitch, i
 // memory, then the codes.
 template <bool ROT, int KB>
 __device__ __forceinline__ void quantize_key_channels(const uint8_t* rows, const PartShape& s, int G, int dt,
-                                                      uint8_t* rec, const LayerView& L, float2* red, float4* kpar) {
+                                                      const RecOut& ro, float2* red, float4* kpar) {
   constexpr int PER = 32 / KB;
-  const int W = G / PER, lgW = __ffs(W) - 1;
+  const int W = G / PER;
   for (int item = threadIdx.x; item < s.nc * W; item += kQuantThreads) {
     const int dl = item % s.nc, w = item / s.nc;
     const int col = s.c0 + dl - s.sc0;
@@ -254,7 +270,7 @@ __device__ __forceinline__ void quantize_key_channels(const uint8_t* rows, const
     red[w * s.nc + dl] = make_float2(mn, mx);
   }
   __syncthreads();
-  __half2* ksz = reinterpret_cast<__half2*>(rec + L.ksz_off);
+  __half2* ksz = reinterpret_cast<__half2*>(ro.rec_ksz >= 0 ? ro.rec + ro.rec_ksz : ro.rec + ro.tile0 + ro.ksz_off);
   for (int dl = threadIdx.x; dl < s.nc; dl += kQuantThreads) {
     float mn = INFINITY, mx = -INFINITY;
     for (int w = 0; w < W; ++w) {
@@ -267,46 +283,46 @@ __device__ __forceinline__ void quantize_key_channels(const uint8_t* rows, const
     kpar[dl] = make_float4(gp.d, gp.m, __frcp_rn(gp.d), 0.f);
   }
   __syncthreads();
-  pack_key_codes<ROT, KB, false>(rows, s.snc, 0, s.sc0, s.c0, s.nc, 0, W, lgW, dt, reinterpret_cast<uint32_t*>(rec + L.kc_off),
-                          [&](int, int d) { return kpar[d - s.c0]; });
+  pack_key_codes<ROT, KB, false>(rows, s.snc, 0, s.sc0, s.c0, s.nc, 0, W, dt, ro,
+                                 [&](int, int d) { return kpar[d - s.c0]; });
 }
 
 // Keys per token over group_v channels (BQ2_0), tokens [t0, t0 + nt): the
 // token groups' scales and zero points, then the codes of those tokens
 // packed along the token axis.
 template <bool ROT, int KB>
-__device__ __forceinline__ void quantize_key_tokens(const uint8_t* rows, const PartShape& s, int G, int dt,
-                                                    uint8_t* rec, const LayerView& L, float4* kpar) {
+__device__ __forceinline__ void quantize_key_tokens(const uint8_t* rows, const PartShape& s, int dt, const RecOut& ro,
+                                                    int gv, float4* kpar) {
   constexpr int PER = 32 / KB;
-  const int ng = kHeadDim / L.group_v, gv = L.group_v;
-  __half2* ksz = reinterpret_cast<__half2*>(rec + L.ksz_off);
+  const int ng = kHeadDim / gv;
   quantize_token_groups<ROT, KB, false>(rows, s.t0, s.nt, gv, dt, [](int, int, uint32_t) {},
                                         [&](int t, int g, const GroupParams& gp) {
-                                          ksz[t * ng + g] = __halves2half2(gp.d16, gp.m16);
+                                          reinterpret_cast<__half2*>(ro.tile(t) + ro.ksz_off)[ro.local(t) * ng + g] =
+                                              __halves2half2(gp.d16, gp.m16);
                                           kpar[(t - s.t0) * ng + g] = make_float4(gp.d, gp.m, __frcp_rn(gp.d), 0.f);
                                         });
   __syncthreads();
-  const int W = G / PER, lgW = __ffs(W) - 1;
-  pack_key_codes<ROT, KB, true>(rows, kHeadDim, s.t0, 0, 0, kHeadDim, s.t0 / PER, s.nt / PER, lgW, dt,
-                          reinterpret_cast<uint32_t*>(rec + L.kc_off),
-                          [&](int t, int d) { return kpar[(t - s.t0) * ng + d / gv]; });
+  pack_key_codes<ROT, KB, true>(rows, kHeadDim, s.t0, 0, 0, kHeadDim, s.t0 / PER, s.nt / PER, dt, ro,
+                                [&](int t, int d) { return kpar[(t - s.t0) * ng + d / gv]; });
 }
 
 // Values per token over group_v channels (KIVI), tokens [t0, t0 + nt),
 // codes packed along head_dim.
 template <bool ROT, int KB, int VB>
-__device__ __forceinline__ void quantize_value_tokens(const uint8_t* rows, const PartShape& s, int G, int dt,
-                                                      uint8_t* rec, const LayerView& L) {
-  uint32_t* vc = reinterpret_cast<uint32_t*>(rec + L.vc_off);
-  __half* vsz = reinterpret_cast<__half*>(rec + L.vsz_off);
-  const int ng = kHeadDim / L.group_v;
+__device__ __forceinline__ void quantize_value_tokens(const uint8_t* rows, const PartShape& s, int dt, const RecOut& ro,
+                                                      int gv) {
+  const int ng = kHeadDim / gv, T = 1 << ro.lgT;
   constexpr int VW = kHeadDim * VB / 32;
-  quantize_token_groups<ROT, VB, true>(rows, s.t0, s.nt, L.group_v, dt,
-                                       [&](int t, int w, uint32_t word) { vc[vc_word_index(t, w, G, KB, VW)] = word; },
-                                       [&](int t, int g, const GroupParams& gp) {
-                                         vsz[vsz_half_index(t, g, G, KB, ng, false)] = gp.d16;
-                                         vsz[vsz_half_index(t, g, G, KB, ng, true)] = gp.m16;
-                                       });
+  quantize_token_groups<ROT, VB, true>(
+      rows, s.t0, s.nt, gv, dt,
+      [&](int t, int w, uint32_t word) {
+        reinterpret_cast<uint32_t*>(ro.tile(t) + ro.vc_off)[vc_word_index(ro.local(t), w, T, KB, VW)] = word;
+      },
+      [&](int t, int g, const GroupParams& gp) {
+        __half* vsz = reinterpret_cast<__half*>(ro.tile(t) + ro.vsz_off);
+        vsz[vsz_half_index(ro.local(t), g, T, KB, ng, false)] = gp.d16;
+        vsz[vsz_half_index(ro.local(t), g, T, KB, ng, true)] = gp.m16;
+      });
 }
 
 // One part CTA: stages its rows, then quantizes keys (record jk) or values
@@ -322,20 +338,20 @@ __device__ __forceinline__ void quantize_key_part(const LayerView& L, int b, int
   if constexpr (ROT) stage_rotated(src, s.t0, s.nt, dt, reinterpret_cast<float*>(smem));
   else stage_raw(src, s.t0, s.nt, s.sc0, s.snc, reinterpret_cast<uint16_t*>(smem));
   __syncthreads();
-  uint8_t* rec = record_ptr(L, b, h, jk);
+  const RecOut ro = rec_out(L, record_ptr(L, b, h, jk));
   float4* kpar = reinterpret_cast<float4*>(smem + sm.rows + sm.red);
-  if (L.k_axis == 0) quantize_key_channels<ROT, KB>(smem, s, G, dt, rec, L, reinterpret_cast<float2*>(smem + sm.rows), kpar);
-  else quantize_key_tokens<ROT, KB>(smem, s, G, dt, rec, L, kpar);
+  if (L.k_axis == 0) quantize_key_channels<ROT, KB>(smem, s, G, dt, ro, reinterpret_cast<float2*>(smem + sm.rows), kpar);
+  else quantize_key_tokens<ROT, KB>(smem, s, dt, ro, L.group_v, kpar);
 }
 
 template <bool ROT, int KB, int VB>
 __device__ __forceinline__ void quantize_value_part(const LayerView& L, int b, int h, int64_t jv, const BlockRows& src,
                                                     const PartShape& s, uint8_t* smem) {
-  const int G = L.group_k, dt = L.kv_dtype;
+  const int dt = L.kv_dtype;
   if constexpr (ROT) stage_rotated(src, s.t0, s.nt, dt, reinterpret_cast<float*>(smem));
   else stage_raw(src, s.t0, s.nt, 0, kHeadDim, reinterpret_cast<uint16_t*>(smem));
   __syncthreads();
-  quantize_value_tokens<ROT, KB, VB>(smem, s, G, dt, record_ptr(L, b, h, jv), L);
+  quantize_value_tokens<ROT, KB, VB>(smem, s, dt, rec_out(L, record_ptr(L, b, h, jv)), L.group_v);
 }
 
 // Part `part` of `parts` of the key block jk (key) or the value block jv of
@@ -508,25 +524,21 @@ __global__ void dequant_kernel(LayerView L, int seq, int sinks, int t0, int n, f
     const int t = tok % G;
     if (tok < Q) {
       const uint8_t* rec = record_ptr(L, seq, h, tok / G);
-      const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + L.kc_off);
       const int kper = 32 / kb;
-      const __half2 ksz = L.k_axis == 0
-                              ? reinterpret_cast<const __half2*>(rec + L.ksz_off)[d]
-                              // per-token keys: (scale, zero) per (token, channel group)
-                              : reinterpret_cast<const __half2*>(rec + L.ksz_off)[t * (D / L.group_v) + d / L.group_v];
-      const uint32_t kw = kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb);
+      const __half2 ksz = *reinterpret_cast<const __half2*>(rec + ksz_pair_byte(L, t, d));
+      const uint32_t kw = *reinterpret_cast<const uint32_t*>(rec + kc_word_byte(L, d, t / kper)) >> ((t % kper) * kb);
       k_out[o] = dequant_value(kw & ((1u << kb) - 1), __low2half(ksz), __high2half(ksz));
     } else {
       k_out[o] = load_kv(L.ring_k, (unit * L.residual + tok % L.residual) * D + d, L.kv_dtype);
     }
     if (tok < QV) {
       const uint8_t* rec = record_ptr(L, seq, h, tok / G);
-      const uint32_t* vc = reinterpret_cast<const uint32_t*>(rec + L.vc_off);
       const int vper = 32 / vb;
-      const uint32_t vq = (vc[vc_word_index(t, d / vper, G, kb, D / vper)] >> ((d % vper) * vb)) & ((1u << vb) - 1);
-      const __half* vsz = reinterpret_cast<const __half*>(rec + L.vsz_off);
-      const int ng = D / L.group_v, gg = d / L.group_v;
-      v_out[o] = dequant_value(vq, vsz[vsz_half_index(t, gg, G, kb, ng, false)], vsz[vsz_half_index(t, gg, G, kb, ng, true)]);
+      const uint32_t vq =
+          (*reinterpret_cast<const uint32_t*>(rec + vc_word_byte(L, t, d / vper)) >> ((d % vper) * vb)) & ((1u << vb) - 1);
+      const int gg = d / L.group_v;
+      v_out[o] = dequant_value(vq, *reinterpret_cast<const __half*>(rec + vsz_half_byte(L, t, gg, false)),
+                               *reinterpret_cast<const __half*>(rec + vsz_half_byte(L, t, gg, true)));
     } else {
       v_out[o] = load_kv(L.ring_v, (unit * L.residual_v + tok % L.residual_v) * D + d, L.kv_dtype);
     }

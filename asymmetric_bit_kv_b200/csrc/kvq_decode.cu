@@ -42,16 +42,18 @@ struct SoftmaxState {
   }
 };
 
-// Value of token t of a block record at this lane's channels lane + 32c,
+// Value of token tb of a block record at this lane's channels lane + 32c,
 // dequantized (x_hat = q*d + m, two roundings): the record's word placement
 // and its (scale, zero) order are resolved once per token, not per channel.
-__device__ __forceinline__ void token_values(const LayerView& L, const uint8_t* rec, int t, int lane,
+__device__ __forceinline__ void token_values(const LayerView& L, const uint8_t* rec, int tb, int lane,
                                              float (&vv)[4]) {
   constexpr int D = kHeadDim;
-  const int G = L.group_k, kb = L.k_bits, vb = L.v_bits, Gv = L.group_v;
+  const int G = L.tile_tokens, kb = L.k_bits, vb = L.v_bits, Gv = L.group_v;
   const int vper = 32 / vb, VW = D / vper, ng = D / Gv;
-  const uint32_t* vc = reinterpret_cast<const uint32_t*>(rec + L.vc_off);
-  const __half* vsz = reinterpret_cast<const __half*>(rec + L.vsz_off);
+  const uint8_t* tp = rec + tile_base(L, tb);  // the token's tile and its index there
+  const int t = tb % G;
+  const uint32_t* vc = reinterpret_cast<const uint32_t*>(tp + L.vc_off);
+  const __half* vsz = reinterpret_cast<const __half*>(tp + L.vsz_off);
   const int row = vc_row(t, G, kb);
   const int sw = VW >= 4 ? chunk_swizzle(row, VW / 4) : 0;
   // (scale, zero) of group gg at vsz[zi(gg)] / vsz[zi(gg) + zoff]
@@ -171,8 +173,6 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
         // keys or values of this block still exact, in their ring (never
         // with the rotation: a rotated cache has one residual length)
         const bool kq = j * G < Q, vq = j * G < QV;
-        const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + L.kc_off);
-        const int ng = D / Gv;
 #pragma unroll 1
         for (int t = warp; t < G; t += 4) {
           const int i = j * G + t;
@@ -181,9 +181,9 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
           for (int c = 0; c < 4; ++c) {
             const int d = lane + 32 * c;
             if (kq) {
-              const __half2 sz = L.k_axis == 1 ? reinterpret_cast<const __half2*>(rec + L.ksz_off)[t * ng + d / Gv]
-                                               : reinterpret_cast<const __half2*>(rec + L.ksz_off)[d];
-              const uint32_t kq2 = (kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb)) & kmask;
+              const __half2 sz = *reinterpret_cast<const __half2*>(rec + ksz_pair_byte(L, t, d));
+              const uint32_t kq2 =
+                  (*reinterpret_cast<const uint32_t*>(rec + kc_word_byte(L, d, t / kper)) >> ((t % kper) * kb)) & kmask;
               kv[c] = dequant_value(kq2, __low2half(sz), __high2half(sz));
             } else {
               kv[c] = load_kv(L.ring_k, (unit * R + i % R) * D + d, L.kv_dtype);
@@ -209,17 +209,19 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
       }
       if (L.k_axis == 1) {
         // per-token keys (BQ2_0): dequantize each key and dot it with q
-        const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + L.kc_off);
-        const __half2* ksz = reinterpret_cast<const __half2*>(rec + L.ksz_off);
-        const int ng = D / Gv;
+        const int ng = D / Gv, TT = L.tile_tokens;
 #pragma unroll 2
         for (int t = warp; t < G; t += 4) {
           float kv[4], vv[4];
+          const uint8_t* tp = rec + tile_base(L, t);
+          const uint32_t* kc = reinterpret_cast<const uint32_t*>(tp + L.kc_off);
+          const __half2* ksz = reinterpret_cast<const __half2*>(tp + L.ksz_off);
+          const int tl = t % TT;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const int d = lane + 32 * c;
-            const __half2 sz = ksz[t * ng + d / Gv];
-            const uint32_t kq = (kc[kc_word_index(d, t / kper, G / kper)] >> ((t % kper) * kb)) & kmask;
+            const __half2 sz = ksz[tl * ng + d / Gv];
+            const uint32_t kq = (kc[kc_word_index(d, tl / kper, TT / kper)] >> ((tl % kper) * kb)) & kmask;
             kv[c] = dequant_value(kq, __low2half(sz), __high2half(sz));
           }
           token_values(L, rec, t, lane, vv);
@@ -235,7 +237,7 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
       }
       {
         const int d = threadIdx.x;
-        const __half2 sz = reinterpret_cast<const __half2*>(rec + L.ksz_off)[d];
+        const __half2 sz = *reinterpret_cast<const __half2*>(rec + ksz_pair_byte(L, 0, d));
         const float sc = __low2float(sz), z = __high2float(sz);
 #pragma unroll
         for (int hh = 0; hh < NG; ++hh) {
@@ -248,14 +250,15 @@ __global__ void __launch_bounds__(128) decode_split_simple_kernel(DecodeParams p
       float bias[NG];
 #pragma unroll
       for (int hh = 0; hh < NG; ++hh) bias[hh] = sbias[0][hh] + sbias[1][hh] + sbias[2][hh] + sbias[3][hh];
-      const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + L.kc_off);
+      const int TT = L.tile_tokens;
       for (int t = warp; t < G; t += 4) {
         float kcode[4], vv[4];
-        const int kw = t / kper, ksh = (t % kper) * kb;
+        const uint32_t* kc = reinterpret_cast<const uint32_t*>(rec + tile_base(L, t) + L.kc_off);
+        const int tl = t % TT, kw = tl / kper, ksh = (tl % kper) * kb;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int d = lane + 32 * c;
-          kcode[c] = (float)((kc[kc_word_index(d, kw, G / kper)] >> ksh) & kmask);
+          kcode[c] = (float)((kc[kc_word_index(d, kw, TT / kper)] >> ksh) & kmask);
         }
         token_values(L, rec, t, lane, vv);
 #pragma unroll

@@ -63,23 +63,27 @@ bool mma_supported(const LayerView& L, int num_q_heads) {
   // kernel
   if (L.k_axis == 1 && L.group_v != kHeadDim) return false;
   if (L.hadamard && L.k_axis != 1) return false;
-  if (L.group_k < 64) return false;                   // tiles of 64 tokens
+  if (L.group_k < 64) return false;                   // tiles of 64 tokens (blocks of 128 are two of them)
   if (L.residual_v != L.residual) return false;       // one ring for keys and values
   if (L.v_bits == 2 && L.group_v < 64) return false;  // a 2-bit value chunk spans 64 channels
-  // two stages per warp must fit (8-bit keys in blocks of 128 tokens do not)
+  // two stages per warp must fit
   return make_mma_plan(L, num_q_heads).smem_bytes <= smem_limit();
 }
 
 MmaPlan make_mma_plan(const LayerView& L, int num_q_heads) {
   MmaPlan mp;
-  const int G = L.group_k, D = L.head_dim;
+  const int G = L.group_k;
   const int NG = num_q_heads / L.num_kv_heads;
-  const int ngrp = D / L.group_v;
   const int nkt = key_ntiles(L, num_q_heads);
-  mp.tx_bytes = L.vsz_off + G * ngrp * 4;  // kc | ksz | vc | vsz, one copy
+  // a stage holds one tile item as [kc | ksz | vc | vsz]: the record itself
+  // (one tile), or a tile part of a longer block (plus the block's
+  // per-channel key scales, when it stores them once for all its tiles)
+  const int NT = G / L.tile_tokens;
+  const int ksz_stage = L.rec_ksz_off >= 0 ? kHeadDim * 4 : L.vc_off - L.ksz_off;
   mp.kc_bytes = L.ksz_off;
-  mp.vc_soff = L.vc_off;
-  mp.vsz_soff = L.vsz_off;
+  mp.vc_soff = mp.kc_bytes + ksz_stage;
+  mp.vsz_soff = mp.vc_soff + (L.vsz_off - L.vc_off);
+  mp.tx_bytes = NT == 1 ? L.tile_bytes : (L.rec_ksz_off >= 0 ? kHeadDim * 4 : 0) + L.tile_bytes;
   const int ring_bytes = 2 * kResChunk * tc::kRowBytes;  // key and value rows of a ring chunk
   mp.stage_bytes = (int32_t)round_up(std::max(mp.tx_bytes, ring_bytes), 128);
   // per-consumer-warp scratch

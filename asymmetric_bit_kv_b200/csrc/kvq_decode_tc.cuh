@@ -709,7 +709,7 @@ __device__ __forceinline__ void store_new_token(const DecodeParams& p, int b, in
   const LayerView& L = p.L;
   const int i = p.nres[b] - 1;
   const int row = i % kResChunk;
-  const int slot = (nb * L.group_k + i) % L.residual;
+  const int slot = (nb * L.tile_tokens + i) % L.residual;
   const int64_t dst = (((int64_t)b * L.num_kv_heads + h) * L.residual + slot) * kRowBytes;
   reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(L.ring_k) + dst)[lane] =
       reinterpret_cast<const uint2*>(stage + row * kRowBytes)[lane];
@@ -717,9 +717,9 @@ __device__ __forceinline__ void store_new_token(const DecodeParams& p, int b, in
       reinterpret_cast<const uint2*>(stage + (kResChunk + row) * kRowBytes)[lane];
   if (h == 0 && lane == 0) {  // the step's lengths (a flush of this step moved G tokens to block nb - 1)
     int32_t* len = L.lens + (int64_t)b * kLensStride;
-    len[kLenQ] = nb * L.group_k;
+    len[kLenQ] = nb * L.tile_tokens;
     len[kLenN] = p.nres[b];
-    len[kLenQV] = nb * L.group_k;
+    len[kLenQV] = nb * L.tile_tokens;
   }
 }
 
@@ -749,19 +749,33 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, const MmaPlan&
     ++is.seq;
   }
   if (j < nb) {
+    // tile item j: tile j % NT of block j / NT (NT tiles per block)
+    const int NT = L.group_k / L.tile_tokens;
+    const int jb = j / NT, jt = j % NT;
     mbar_expect_tx(bar, mp.tx_bytes + (newq ? qbytes : 0u));
     const uint8_t* rec;
     if (L.page_table) {  // one page-table read per run of page_blocks blocks of the unit
-      const int run = j / L.page_blocks;
+      const int run = jb / L.page_blocks;
       if (newq || run != is.run) {
         is.run = run;
         is.page = __ldg(L.page_table + (int64_t)u.b * L.max_pages + run);
       }
-      rec = L.blocks + ((is.page * L.num_kv_heads + u.h) * L.page_blocks + j % L.page_blocks) * L.record_bytes;
+      rec = L.blocks + ((is.page * L.num_kv_heads + u.h) * L.page_blocks + jb % L.page_blocks) * L.record_bytes;
     } else {
-      rec = record_ptr(L, u.b, u.h, j);
+      rec = record_ptr(L, u.b, u.h, jb);
     }
-    bulk_g2s(dst, rec, mp.tx_bytes, bar);
+    if (NT == 1) {
+      bulk_g2s(dst, rec, mp.tx_bytes, bar);
+    } else {
+      const uint8_t* tp = rec + L.tile0_off + (int64_t)jt * L.tile_bytes;
+      if (L.rec_ksz_off >= 0) {  // the block's per-channel key scales, then the tile's codes and value scales
+        bulk_g2s(dst + mp.kc_bytes, rec + L.rec_ksz_off, kHeadDim * 4, bar);
+        bulk_g2s(dst, tp, mp.kc_bytes, bar);
+        bulk_g2s(dst + mp.vc_soff, tp + L.vc_off, L.tile_bytes - L.vc_off, bar);
+      } else {  // a tile part holds all it needs
+        bulk_g2s(dst, tp, L.tile_bytes, bar);
+      }
+    }
     if (j == nb - 1 && p.nres[u.b] > 0) {
       // the unit's ring chunks come next: bring its ring rows into L2 so that
       // those short items do not each wait a full HBM round trip
@@ -780,7 +794,7 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, const MmaPlan&
     if (sink) {
       row = ((int64_t)u.b * L.num_kv_heads + u.h) * KVQ_MAX_SINKS;
     } else {
-      const int slot = (nb * L.group_k + (j - nb) * kResChunk) % L.residual;
+      const int slot = (nb * L.tile_tokens + (j - nb) * kResChunk) % L.residual;
       row = ((int64_t)u.b * L.num_kv_heads + u.h) * L.residual + slot;
     }
     constexpr uint32_t bytes = kResChunk * kRowBytes;
@@ -832,7 +846,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
   const int Hkv = L.num_kv_heads;
   const int NG = p.num_q_heads / Hkv;  // query rows per unit
   const int ngr = p.q_heads / Hkv;      // query heads per KV head (rows per query token)
-  const int G = L.group_k;
+  const int G = L.tile_tokens;  // tokens of one work item's tile: the block, or 64 of a longer block
   const int rs = p.cta_start[c], re = p.cta_start[c + 1];
   const bool bf16 = L.kv_dtype == KVQ_BF16;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

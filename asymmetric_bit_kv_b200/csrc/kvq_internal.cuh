@@ -29,7 +29,12 @@ struct LayerView {
   int32_t* lens;          // [max_batch][kLensStride] length table (see kLensStride)
   int64_t record_bytes;
   int64_t max_blocks;
-  int32_t kc_off, ksz_off, vc_off, vsz_off;  // byte offsets inside a record
+  // A record is a run of tiles of tile_tokens = min(G, 64) tokens: tile part
+  // i at tile0_off + i * tile_bytes, laid out [kc | ksz | vc | vsz] with the
+  // byte offsets below; with several tiles and per-channel keys, the key
+  // scales are stored once, at rec_ksz_off (else rec_ksz_off = -1).
+  int32_t kc_off, ksz_off, vc_off, vsz_off;  // byte offsets inside a tile part
+  int32_t tile_tokens, tile_bytes, tile0_off, rec_ksz_off;
   int32_t k_bits, v_bits;
   int32_t num_kv_heads, head_dim, group_k, group_v, residual;
   int32_t residual_v;     // value ring slots (= residual unless the cache sets its own)
@@ -110,6 +115,30 @@ __host__ __device__ inline int vsz_half_index(int t, int gg, int G, int kb, int 
   const int r = col + 8 * (j & 1);  // its row in that M-tile
   const int entry = ((tile * 4 + mt) * 4 + ((r & 7) >> 1)) * ngrp + gg;
   return entry * 8 + (zero ? 4 : 0) + 2 * (r >> 3) + (r & 1);
+}
+
+// Byte offsets inside a record of token t's data (t < G, the block's own
+// token index): its tile part, the word of key codes holding it for channel
+// d (word w of a channel covers tokens w*32/k_bits ...), its key (scale,
+// zero) pair for channel d, its value word w and its value scale / zero.
+__host__ __device__ inline int64_t tile_base(const LayerView& L, int t) {
+  return L.tile0_off + (int64_t)(t / L.tile_tokens) * L.tile_bytes;
+}
+__host__ __device__ inline int64_t kc_word_byte(const LayerView& L, int d, int w) {
+  const int wt = L.tile_tokens * L.k_bits / 32;  // key words per channel per tile
+  return L.tile0_off + (int64_t)(w / wt) * L.tile_bytes + L.kc_off + 4 * (int64_t)kc_word_index(d, w % wt, wt);
+}
+__host__ __device__ inline int64_t ksz_pair_byte(const LayerView& L, int t, int d) {
+  if (L.k_axis == 0) return (L.rec_ksz_off >= 0 ? L.rec_ksz_off : L.tile0_off + L.ksz_off) + 4 * (int64_t)d;
+  return tile_base(L, t) + L.ksz_off + 4 * (int64_t)((t % L.tile_tokens) * (L.head_dim / L.group_v) + d / L.group_v);
+}
+__host__ __device__ inline int64_t vc_word_byte(const LayerView& L, int t, int w) {
+  return tile_base(L, t) + L.vc_off +
+         4 * (int64_t)vc_word_index(t % L.tile_tokens, w, L.tile_tokens, L.k_bits, L.head_dim * L.v_bits / 32);
+}
+__host__ __device__ inline int64_t vsz_half_byte(const LayerView& L, int t, int g, bool zero) {
+  return tile_base(L, t) + L.vsz_off +
+         2 * (int64_t)vsz_half_index(t % L.tile_tokens, g, L.tile_tokens, L.k_bits, L.head_dim / L.group_v, zero);
 }
 
 // Block record j of (sequence b, KV head h): contiguous per (b, h), or in a

@@ -73,6 +73,10 @@ class kvq_layout(ctypes.Structure):
         ("page_table", ctypes.c_void_p),
         ("page_blocks", ctypes.c_int32),
         ("max_pages", ctypes.c_int32),
+        ("tile_tokens", ctypes.c_int32),
+        ("tile_bytes", ctypes.c_int32),
+        ("tile0_offset", ctypes.c_int32),
+        ("rec_ksz_offset", ctypes.c_int32),
     ]
 
 

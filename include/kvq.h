@@ -129,29 +129,35 @@ typedef struct kvq_cache kvq_cache;
  * Block records: for sequence b, KV head h and key block j (positions
  * [j*G, (j+1)*G) of that sequence) the record starts at
  *   blocks + ((b * num_kv_heads + h) * max_blocks + j) * record_bytes
- * (a paged cache: see page_table below) and holds, at the given byte
- * offsets:
- *   kc  uint32 [D][W], W = G*k_bits/32: channel d's row holds W words; word
+ * (a paged cache: see page_table below). A record is a run of tiles of
+ * T = min(G, 64) tokens: tile i (tokens i*T ..) starts at tile0_offset +
+ * i*tile_bytes, and holds at the given byte offsets from its start
+ * (t below: the token's index inside the tile):
+ *   kc  uint32 [D][W], W = T*k_bits/32: channel d's row holds W words; word
  *       w packs the codes of tokens w*(32/k_bits) + i, i = 0.., code i at
  *       bits [i*k_bits, ...) (per-channel keys packed along the token axis);
- *   ksz half2 [D]: (scale d, zero point m) of each channel's key group;
+ *   ksz half2 [D]: (scale d, zero point m) of each channel's key group --
+ *       when G = 128 these pairs are stored once per record, at
+ *       rec_ksz_offset (a block has one key group per channel), and the tile
+ *       holds none (rec_ksz_offset = -1 otherwise);
  *   (k_axis 1: kc exactly as above, codes of each channel packed along the
- *   token axis; ksz half2 [G][D/group_v], (scale, zero point) per (token,
- *   channel group), row-major);
- *   vc  uint32 [G][V], V = D*v_bits/32: one row of V words per token; word w
+ *   token axis; ksz half2 [T][D/group_v], (scale, zero point) per (token,
+ *   channel group), row-major, in every tile);
+ *   vc  uint32 [T][V], V = D*v_bits/32: one row of V words per token; word w
  *       packs the codes of channels w*(32/v_bits) + i, code i at bits
  *       [i*v_bits, ...) (per-token values packed along head_dim);
  *   vsz fp16 scale and zero point of each (token, value group): for
- *       G < 64 the pairs [G][D/group_v] of (scale, zero point); for G >= 64
+ *       T < 64 the pairs [T][D/group_v] of (scale, zero point); for T = 64
  *       16-byte entries in the order the decode kernel reads them (see
  *       kvq_internal.cuh: vsz_half_index).
- * Placement inside kc and vc (so that one copy of a record is readable with
+ * Placement inside kc and vc (so that one copy of a tile is readable with
  * ldmatrix without shared-memory bank conflicts): in a row of n >= 2
  * 16-byte chunks (4 words each), chunk c of row r is stored at chunk
  * position c ^ s(r, n), with s(r, n) = r & 7 for n >= 8 and
  * (r / (8/n)) % n otherwise; rows of fewer than 4 words are not permuted.
- * Value rows are stored in token order t -> (t % c) * (G/c) + t / c, with
- * c = 16/k_bits. (kvq_internal.cuh: kc_word_index, vc_word_index.)
+ * Value rows are stored in token order t -> (t % c) * (T/c) + t / c, with
+ * c = 16/k_bits. (kvq_internal.cuh: kc_word_index, vc_word_index,
+ * kc_word_byte, ksz_pair_byte, vc_word_byte, vsz_half_byte.)
  * Rings: keys [max_batch][num_kv_heads][R][D] and values
  * [max_batch][num_kv_heads][RV][D] in kv_dtype (RV = residual_v, or R);
  * position i of a sequence whose key (value) is exact sits in slot i % R
@@ -164,7 +170,7 @@ typedef struct kvq_layout {
   void* blocks;
   int64_t record_bytes;
   int64_t max_blocks;
-  int64_t kc_offset, ksz_offset, vc_offset, vsz_offset;
+  int64_t kc_offset, ksz_offset, vc_offset, vsz_offset;  /* inside a tile */
   void* ring_k;
   void* ring_v;
   int32_t k_bits, v_bits;
@@ -177,6 +183,8 @@ typedef struct kvq_layout {
    * max_blocks is then the per-sequence capacity in blocks.               */
   void* page_table;
   int32_t page_blocks, max_pages;
+  /* tiles of a record (see above)                                          */
+  int32_t tile_tokens, tile_bytes, tile0_offset, rec_ksz_offset;
 } kvq_layout;
 
 /* Device bytes the arena must hold for cfg: all layers' block records and

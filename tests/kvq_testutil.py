@@ -150,26 +150,36 @@ class Twin:
         def part(off, nbytes, dtype, shape):
             return np.ascontiguousarray(raw[:, off:off + nbytes]).view(dtype).reshape((nblk,) + shape)
 
-        kcw = G * kb // 32
+        # a record is a run of tiles of TT tokens (tile i at tile0_offset +
+        # i * tile_bytes); per-channel key scales of a multi-tile record sit
+        # once at rec_ksz_offset
+        TT = lay.tile_tokens
+        kcw = TT * kb // 32
         vcw = D * vb // 32
         ng = D // Gv
-        vc = part(lay.vc_offset, G * vcw * 4, np.uint32, (G * vcw,))
-        vidx = np.array([[vc_word_index(t, w, G, kb, vcw) for w in range(vcw)] for t in range(G)])
-        # key codes: channel rows of words along the token axis, for both key axes
-        kc = part(lay.kc_offset, kcw * D * 4, np.uint32, (D * kcw,))
+        vidx = np.array([[vc_word_index(t, w, TT, kb, vcw) for w in range(vcw)] for t in range(TT)])
         kidx = np.array([[kc_word_index(d, w, kcw) for w in range(kcw)] for d in range(D)])
-        vsz = part(lay.vsz_offset, G * ng * 4, np.float16, (G * ng * 2,))
-        sidx = np.array([[[vsz_half_index(t, gg, G, kb, ng, z) for z in (False, True)] for gg in range(ng)]
-                         for t in range(G)])
-        if lay.k_axis == 1:  # per-token keys: (scale, zero) pairs [G][groups], row-major
-            ksz = part(lay.ksz_offset, G * ng * 4, np.float16, (G, ng, 2))
+        sidx = np.array([[[vsz_half_index(t, gg, TT, kb, ng, z) for z in (False, True)] for gg in range(ng)]
+                         for t in range(TT)])
+        kc, vc, vsz, ksz = [], [], [], []
+        for i in range(G // TT):
+            t0 = lay.tile0_offset + i * lay.tile_bytes
+            kc.append(part(t0 + lay.kc_offset, kcw * D * 4, np.uint32, (D * kcw,))[:, kidx])  # [n, D, kcw]
+            vc.append(part(t0 + lay.vc_offset, TT * vcw * 4, np.uint32, (TT * vcw,))[:, vidx])
+            vsz.append(part(t0 + lay.vsz_offset, TT * ng * 4, np.float16, (TT * ng * 2,))[:, sidx])
+            if lay.k_axis == 1:  # per-token keys: (scale, zero) pairs [TT][groups] in every tile
+                ksz.append(part(t0 + lay.ksz_offset, TT * ng * 4, np.float16, (TT, ng, 2)))
+        if lay.k_axis == 1:
+            ksz = np.concatenate(ksz, axis=1)
+        elif lay.rec_ksz_offset >= 0:
+            ksz = part(lay.rec_ksz_offset, D * 4, np.float16, (D, 2))
         else:
             ksz = part(lay.ksz_offset, D * 4, np.float16, (D, 2))
         return {
-            "kc": kc[:, kidx],
+            "kc": np.concatenate(kc, axis=2),
             "ksz": ksz,
-            "vc": vc[:, vidx],
-            "vsz": vsz[:, sidx],
+            "vc": np.concatenate(vc, axis=1),
+            "vsz": np.concatenate(vsz, axis=1),
         }
 
     def read_ring(self, layer: int, b: int):
