@@ -18,6 +18,8 @@
 // of a token, the min/max of a group combined with __shfl_xor. Codes use
 // IEEE-rounded fp32 arithmetic (__fsub_rn, __fdiv_rn, rintf), bit-exact with
 // the oracle.
+#include <algorithm>
+
 #include "kvq_append.cuh"
 #include "kvq_decode.cuh"
 
@@ -49,9 +51,12 @@ struct BlockRows {
 // One CTA quantizes one part of one tensor of a G-token block: per-channel
 // keys split by channels (the min/max of a channel runs over all G tokens),
 // values and per-token keys split by tokens. The fused step's flush uses
-// kStepParts parts per tensor (its grid is only batch x Hkv blocks); appends
-// use one.
-constexpr int kStepParts = 2;
+// kStepKeyParts + kStepValueParts CTAs per block (its grid is only batch x
+// Hkv blocks); appends use one per tensor.
+// (one key CTA and two value CTAs per block: 768 CTAs for 32 x 8 blocks, one
+// wave at the kernel's 6 CTAs per SM; two key parts, a second wave, measured
+// no faster)
+constexpr int kStepKeyParts = 1, kStepValueParts = 2;
 
 struct PartShape {
   bool key;
@@ -398,10 +403,11 @@ __global__ void __launch_bounds__(kQuantThreads, 6) quantize_blocks_kernel(Appen
   quantize_part<ROT>(L, b, h, key, 0, 1, (key ? p.q_old[b] : p.qv_old[b]) / G + j, src, smem_q);
 }
 
-// grid (batch * Hkv * 2 * kStepParts); block kQuantThreads. The flush of a
-// fused decode step: for (sequence, KV head) whose ring holds R tokens, the
-// oldest G ring tokens become the next block record (one ring shared by keys
-// and values); CTA x = ((b * Hkv + h) * 2 + tensor) * kStepParts + part. The
+// grid (batch * Hkv * (kStepKeyParts + kStepValueParts)); block
+// kQuantThreads. The flush of a fused decode step: for (sequence, KV head)
+// whose ring holds R tokens, the oldest G ring tokens become the next block
+// record (one ring shared by keys and values); CTA x of unit x / parts takes
+// key part x % parts if below kStepKeyParts, else a value part. The
 // decode launch that follows is its programmatic dependent and waits for it
 // (griddepcontrol.wait) before reading records; the decode kernel records
 // the new lengths.
@@ -410,9 +416,11 @@ __global__ void __launch_bounds__(kQuantThreads, 6) step_flush_kernel(FlushParam
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ __align__(16) uint8_t smem_q[];
   const LayerView& L = p.L;
-  const int part = blockIdx.x % kStepParts;
-  const bool key = ((blockIdx.x / kStepParts) & 1) == 0;
-  const int unit_i = blockIdx.x / (2 * kStepParts);
+  constexpr int parts = kStepKeyParts + kStepValueParts;
+  const int xp = blockIdx.x % parts;
+  const bool key = xp < kStepKeyParts;
+  const int part = key ? xp : xp - kStepKeyParts;
+  const int unit_i = blockIdx.x / parts;
   const int b = unit_i / L.num_kv_heads, h = unit_i % L.num_kv_heads;
   const int32_t* len = L.lens + (int64_t)b * kLensStride;
   const int q = len[kLenQ], n = len[kLenN];
@@ -420,18 +428,22 @@ __global__ void __launch_bounds__(kQuantThreads, 6) step_flush_kernel(FlushParam
   const int64_t unit = (int64_t)b * L.num_kv_heads + h;
   const BlockRows src{reinterpret_cast<const uint16_t*>(key ? L.ring_k : L.ring_v) + unit * L.residual * kHeadDim,
                       nullptr, 0, q, q + n, L.residual, L.num_kv_heads, h};
-  quantize_part<ROT>(L, b, h, key, part, kStepParts, q / L.group_k, src, smem_q);
+  quantize_part<ROT>(L, b, h, key, part, key ? kStepKeyParts : kStepValueParts, q / L.group_k, src, smem_q);
 }
 
 cudaError_t launch_step_flush(const FlushParams& p, cudaStream_t stream) {
   const LayerView& L = p.L;
   const bool rot = L.hadamard != 0;
-  const int smem = quant_smem_bytes(L.group_k, L.k_bits, L.group_v, L.k_axis, rot, kStepParts);
+  const int smem = std::max(
+      part_smem(part_shape(true, 0, kStepKeyParts, L.group_k, L.k_axis, rot), L.group_k, L.k_bits, L.group_v, L.k_axis,
+                rot).total,
+      part_smem(part_shape(false, 0, kStepValueParts, L.group_k, L.k_axis, rot), L.group_k, L.k_bits, L.group_v,
+                L.k_axis, rot).total);
   static uint64_t done_rot = 0, done_raw = 0;
   cudaError_t e = rot ? opt_in_max_smem(reinterpret_cast<const void*>(step_flush_kernel<true>), done_rot)
                       : opt_in_max_smem(reinterpret_cast<const void*>(step_flush_kernel<false>), done_raw);
   if (e != cudaSuccess) return e;
-  const int grid = p.ctas * 2 * kStepParts;
+  const int grid = p.ctas * (kStepKeyParts + kStepValueParts);
   if (rot) step_flush_kernel<true><<<grid, kQuantThreads, smem, stream>>>(p);
   else step_flush_kernel<false><<<grid, kQuantThreads, smem, stream>>>(p);
   return cudaGetLastError();
