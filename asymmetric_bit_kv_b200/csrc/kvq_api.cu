@@ -800,12 +800,15 @@ kvq_status kvq_decode_attention_multi(kvq_cache* c, int32_t layer, const void* q
                   n, num_tokens);
   }
   // groups of query tokens, at most 8 query rows per KV head per launch
+  // (2 where the tensor-core kernel of the layer takes no more)
   const int ngr = cfg.num_q_heads / cfg.num_kv_heads;
+  const kvq::LayerView lv = layer_view(c, layer);
+  const int max_rows = kvq::mma_supported(lv, cfg.num_q_heads) ? kvq::mma_max_rows(lv) : 8;
   const int64_t qrow = (int64_t)cfg.num_q_heads * cfg.head_dim;  // elements per query token of a sequence
   const int out_size = out_dtype == KVQ_F32 ? 4 : 2;
   for (int t0 = 0; t0 < num_tokens;) {
     int tp = 1;
-    while (2 * tp * ngr <= 8 && t0 + 2 * tp <= num_tokens) tp *= 2;
+    while (2 * tp * ngr <= max_rows && t0 + 2 * tp <= num_tokens) tp *= 2;
     const kvq::QueryGroup g{num_tokens * cfg.num_q_heads, tp, num_tokens - 1 - t0};
     s = kvq::enqueue_decode(c, layer, nullptr, nullptr, static_cast<const uint8_t*>(q) + t0 * qrow * 2,
                             static_cast<uint8_t*>(out) + t0 * qrow * out_size, out_dtype, softmax_scale, batch,
@@ -923,6 +926,18 @@ kvq_status kvq_device_errors(kvq_cache* c, int32_t* flags) {
   if (e == cudaSuccess && v != 0) e = cudaMemset(c->arena + c->err_off, 0, 4);
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
   *flags = v;
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_kernel(const kvq_cache* c, int32_t layer, int32_t rows, int32_t* kernel) {
+  g_last_error.clear();
+  kvq_status s = check_cache_layer(c, layer);
+  if (s != KVQ_OK) return s;
+  if (!kernel) return fail(KVQ_ERR_INVALID_ARG, "kernel is null");
+  if (rows < 1 || rows > 64) return fail(KVQ_ERR_INVALID_ARG, "rows_per_kv_head %d outside 1..64", rows);
+  const kvq::LayerView v = layer_view(c, layer);
+  if (!kvq::mma_supported(v, rows * c->cfg.num_kv_heads)) *kernel = KVQ_KERNEL_CUDA_CORE;
+  else *kernel = kvq::pair_layout(v.group_k, v.k_bits) ? KVQ_KERNEL_TENSOR_CORE_PAIR : KVQ_KERNEL_TENSOR_CORE;
   return KVQ_OK;
 }
 

@@ -172,6 +172,7 @@ __device__ __forceinline__ float staged(const uint8_t* rows, int pitch, int t, i
 // kc_word_index placement) with W = 2^lgW words per channel.
 __device__ __forceinline__ int kc_index_p2(int d, int w, int lgW) {
   const int W = 1 << lgW;
+  if (lgW == 1) return ((d & (kHeadDim / 2 - 1)) << 2) + ((d / (kHeadDim / 2)) << 1) + w;  // pair layout
   if (lgW < 2) return (d << lgW) + w;
   const int lgn = lgW - 2;  // 16-byte chunks per row: 2^lgn
   const int sw = lgn >= 3 ? (d & 7) : ((d >> (3 - lgn)) & ((1 << lgn) - 1));

@@ -58,7 +58,7 @@ __device__ __forceinline__ void token_values(const LayerView& L, const uint8_t* 
   const int sw = VW >= 4 ? chunk_swizzle(row, VW / 4) : 0;
   // (scale, zero) of group gg at vsz[zi(gg)] / vsz[zi(gg) + zoff]
   int zbase, zstride, zoff;
-  if (G < 64) {
+  if (!vsz_operand_order(G, kb)) {
     zbase = t * ng * 2;
     zstride = 2;
     zoff = 1;

@@ -121,6 +121,7 @@ struct MmaPlan {
 };
 
 bool mma_supported(const LayerView& L, int num_q_heads);
+int mma_max_rows(const LayerView& L);  // query rows per KV head one tensor-core launch takes
 MmaPlan make_mma_plan(const LayerView& L, int num_q_heads);
 int mma_ctas_per_sm(const LayerView& L, const MmaPlan& mp, int num_q_heads);
 cudaError_t launch_decode_mma(const DecodeParams& p, const MmaPlan& mp, cudaStream_t stream);

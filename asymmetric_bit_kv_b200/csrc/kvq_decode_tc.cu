@@ -19,14 +19,25 @@ KVQ_TC_DECL(4, 2)
 KVQ_TC_DECL(8, 1)
 KVQ_TC_DECL(8, 2)
 #undef KVQ_TC_DECL
+#define KVQ_PAIR_DECL(V)                                                                                   \
+  cudaError_t launch_pair_v##V(int ngrp, const DecodeParams& p, const MmaPlan& mp, cudaStream_t s);            \
+  const void* fn_pair_v##V(int ngrp);
+KVQ_PAIR_DECL(2)
+KVQ_PAIR_DECL(4)
+KVQ_PAIR_DECL(8)
+#undef KVQ_PAIR_DECL
 }  // namespace tc
 
 namespace {
 
 int key_ntiles(const LayerView& L, int num_q_heads) { return num_q_heads / L.num_kv_heads > 4 ? 2 : 1; }
 
+// 32-token blocks with 2-bit keys (the pair layout): decode_pair_kernel.
+bool pair_path(const LayerView& L) { return pair_layout(L.group_k, L.k_bits); }
+
 const void* instance_for(const LayerView& L, int num_q_heads) {
   const int vb = L.v_bits, ng = kHeadDim / L.group_v, nkt = key_ntiles(L, num_q_heads);
+  if (pair_path(L)) return vb == 2 ? tc::fn_pair_v2(ng) : vb == 4 ? tc::fn_pair_v4(ng) : tc::fn_pair_v8(ng);
 #define KVQ_TC_PICK(K, N) \
   if (L.k_bits == K && nkt == N) return tc::fn_tc_k##K##_##N(vb, ng, L.k_axis == 1);
   KVQ_TC_PICK(2, 1) KVQ_TC_PICK(2, 2) KVQ_TC_PICK(4, 1) KVQ_TC_PICK(4, 2) KVQ_TC_PICK(8, 1) KVQ_TC_PICK(8, 2)
@@ -58,13 +69,20 @@ int smem_limit() {
 
 bool mma_supported(const LayerView& L, int num_q_heads) {
   if (L.head_dim != kHeadDim) return false;
+  if (L.residual_v != L.residual) return false;  // one ring for keys and values
+  if (pair_path(L)) {
+    // per-channel keys, no rotation, at most two query rows per KV head
+    // (they share the B operand with the second channel set and the value
+    // groups)
+    if (L.k_axis != 0 || L.hadamard || num_q_heads > 2 * L.num_kv_heads) return false;
+    return make_mma_plan(L, num_q_heads).smem_bytes <= smem_limit();
+  }
   // per-token keys with one group per head vector (BQ2_0), with or without
   // the rotation; the rotation with per-channel keys runs on the CUDA-core
   // kernel
   if (L.k_axis == 1 && L.group_v != kHeadDim) return false;
   if (L.hadamard && L.k_axis != 1) return false;
   if (L.group_k < 64) return false;                   // tiles of 64 tokens (blocks of 128 are two of them)
-  if (L.residual_v != L.residual) return false;       // one ring for keys and values
   if (L.v_bits == 2 && L.group_v < 64) return false;  // a 2-bit value chunk spans 64 channels
   // two stages per warp must fit
   return make_mma_plan(L, num_q_heads).smem_bytes <= smem_limit();
@@ -152,9 +170,14 @@ int mma_ctas_per_sm(const LayerView& L, const MmaPlan& mp, int num_q_heads) {
   return n;
 }
 
+int mma_max_rows(const LayerView& L) { return pair_path(L) ? 2 : 8; }
+
 cudaError_t launch_decode_mma(const DecodeParams& p, const MmaPlan& mp, cudaStream_t stream) {
   const LayerView& L = p.L;
   const int vb = L.v_bits, ng = kHeadDim / L.group_v, nkt = key_ntiles(L, p.num_q_heads);
+  if (pair_path(L))
+    return vb == 2 ? tc::launch_pair_v2(ng, p, mp, stream)
+                   : vb == 4 ? tc::launch_pair_v4(ng, p, mp, stream) : tc::launch_pair_v8(ng, p, mp, stream);
 #define KVQ_TC_GO(K, N) \
   if (L.k_bits == K && nkt == N) return tc::launch_tc_k##K##_##N(vb, ng, L.k_axis == 1, p, mp, stream);
   KVQ_TC_GO(2, 1) KVQ_TC_GO(2, 2) KVQ_TC_GO(4, 1) KVQ_TC_GO(4, 2) KVQ_TC_GO(8, 1) KVQ_TC_GO(8, 2)

@@ -362,8 +362,10 @@ __device__ __forceinline__ float head_score(const float (&d)[NKT][4], int r, int
 // running maximum grows. GUARD: scores may be -inf (absent tokens), a whole
 // update may see none, and absent heads (valid false) are zeroed (ring
 // chunks); without it every score is finite, and absent heads just compute
-// finite values in columns that are never written (quantized tiles).
-template <int MTN, int HPL, int NGRP, bool GUARD>
+// finite values in columns that are never written (quantized tiles). OWN:
+// both output columns of a lane belong to the lane's own score head (the
+// pair kernel), so the lane rescales them by its own alpha.
+template <int MTN, int HPL, int NGRP, bool GUARD, bool OWN = false>
 __device__ __forceinline__ void softmax_update(float (&sc)[MTN][2 * HPL], SoftState<HPL>& st,
                                                const bool (&valid)[HPL], float (&O)[8][4], float (&Z)[NGRP][4],
                                                int lane) {
@@ -405,6 +407,8 @@ __device__ __forceinline__ void softmax_update(float (&sc)[MTN][2 * HPL], SoftSt
     if constexpr (HPL == 2) {
       a0 = a[0];
       a1 = a[1];
+    } else if constexpr (OWN) {
+      a0 = a1 = a[0];
     } else {
       const int t = lane & 3, base = lane & ~3;
       a0 = __shfl_sync(0xffffffffu, a[0], base + ((2 * t) & 3));

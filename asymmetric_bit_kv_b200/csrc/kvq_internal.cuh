@@ -68,7 +68,16 @@ __host__ __device__ inline int64_t vsz_bytes(int G, int D, int gv) { return (int
 //    sits in row (t % c) * (G / c) + t / c with c = 16 / k_bits, the number of
 //    tokens one 16-bit half of a key word holds (the tokens the decode kernel
 //    reads together for one n-tile are then 8 consecutive rows).
+//  * Pair layout (32-token blocks with 2-bit keys, W = 2 key words per
+//    channel): a channel row is 8 bytes, half of a 16-byte ldmatrix row, so
+//    channels d and d + 64 share 16-byte row d % 64 (d first); the decode
+//    kernel reads both halves with one ldmatrix and keeps them apart in the
+//    columns of its B operand. Token t = 8a + b (b < 8) of such a block
+//    sits in value row 16 * (b / 4) + 8 * ((b / 2) % 2) + 2a + b % 2: the
+//    16-token k-step b / 4 of its P.V product, at the row whose key score the
+//    decode kernel finds on M-tile row (a, b % 2) of key M-tile b / 2.
 // ---------------------------------------------------------------------------
+__host__ __device__ inline bool pair_layout(int G, int kb) { return G == 32 && kb == 2; }
 __host__ __device__ inline int chunk_swizzle(int row, int nchunks) {
   if (nchunks <= 1) return 0;
   if (nchunks >= 8) return row & 7;
@@ -77,12 +86,14 @@ __host__ __device__ inline int chunk_swizzle(int row, int nchunks) {
 // Index (in 32-bit words) of word w of channel d inside the key code array
 // of a record; W = G * k_bits / 32 words per channel.
 __host__ __device__ inline int kc_word_index(int d, int w, int W) {
+  if (W == 2) return (d % (kHeadDim / 2)) * 4 + (d / (kHeadDim / 2)) * 2 + w;  // pair layout
   if (W < 4) return d * W + w;
   const int c = w >> 2;
   return d * W + ((c ^ chunk_swizzle(d, W / 4)) << 2) + (w & 3);
 }
 // Row of token t (0 <= t < G) in the value code array of a record.
 __host__ __device__ inline int vc_row(int t, int G, int kb) {
+  if (pair_layout(G, kb)) return 16 * ((t >> 2) & 1) + 8 * ((t >> 1) & 1) + 2 * (t >> 3) + (t & 1);
   const int c = 16 / kb;
   return (t % c) * (G / c) + t / c;
 }
@@ -103,9 +114,17 @@ __host__ __device__ inline int vc_word_index(int t, int w, int G, int kb, int VW
 // record: a 64-token tile has four k-steps of 16 tokens, k-step mt row r
 // (0..15) being the token the key path puts on that row (the inverse of its
 // tile_token); entry ((tile*4 + mt)*4 + (r%8)/2, group) holds the scales of
-// rows 2q, 2q+1, 8+2q, 9+2q, then their zero points. Smaller blocks keep the
-// plain [G][groups] order of (scale, zero) pairs.
+// rows 2q, 2q+1, 8+2q, 9+2q, then their zero points. The pair layout keeps
+// the same entries for its two 16-token k-steps, k-step and row being
+// vc_row(t) / 16 and vc_row(t) % 16. Other blocks keep the plain [G][groups]
+// order of (scale, zero) pairs.
+__host__ __device__ inline bool vsz_operand_order(int G, int kb) { return G >= 64 || pair_layout(G, kb); }
 __host__ __device__ inline int vsz_half_index(int t, int gg, int G, int kb, int ngrp, bool zero) {
+  if (pair_layout(G, kb)) {
+    const int row = vc_row(t, G, kb), kst = row >> 4, r = row & 15;
+    const int entry = (kst * 4 + ((r & 7) >> 1)) * ngrp + gg;
+    return entry * 8 + (zero ? 4 : 0) + 2 * (r >> 3) + (r & 1);
+  }
   if (G < 64) return (t * ngrp + gg) * 2 + (zero ? 1 : 0);
   const int CPT16 = 16 / kb, TOKC = 128 / kb, JP = CPT16 / 2;
   const int tile = t / 64, tt = t % 64;

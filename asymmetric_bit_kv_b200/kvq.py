@@ -111,6 +111,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kvq_seq_lengths": (I32, [P, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32)]),
         "kvq_seq_sinks": (I32, [P, I32, I32, ctypes.POINTER(I32)]),
         "kvq_seq_value_lengths": (I32, [P, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32)]),
+        "kvq_decode_kernel": (I32, [P, I32, I32, ctypes.POINTER(I32)]),
         "kvq_status_string": (ctypes.c_char_p, [I32]),
         "kvq_last_error": (ctypes.c_char_p, []),
     }
@@ -333,6 +334,15 @@ class KVCache:
         _check(self.lib.kvq_seq_value_lengths(self.handle, layer, seq, ctypes.byref(q), ctypes.byref(n)),
                "kvq_seq_value_lengths")
         return q.value, n.value
+
+    def decode_kernel(self, layer: int, rows_per_kv_head: int | None = None) -> str:
+        """Decode kernel of a layer (kvq_decode_kernel): "cuda_core",
+        "tensor_core" or "tensor_core_pair"; rows_per_kv_head defaults to one
+        query token per sequence."""
+        rows = rows_per_kv_head or self.cfg.num_q_heads // self.cfg.num_kv_heads
+        k = ctypes.c_int32()
+        _check(self.lib.kvq_decode_kernel(self.handle, layer, rows, ctypes.byref(k)), "kvq_decode_kernel")
+        return ("cuda_core", "tensor_core", "tensor_core_pair")[k.value]
 
     def sinks(self, layer: int, seq: int) -> int:
         s = ctypes.c_int32()

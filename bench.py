@@ -24,8 +24,11 @@ sequence over the whole cache, in every layer of the workload. Workloads
 * kv1: the llama3 shapes with the KV1 card's BQ2_0 cache (2-bit keys and
   values per token over whole head vectors, Hadamard rotation, 4 sinks).
 
-Timing: W warm-up steps, then exactly K steps between barriers and device
-synchronisations, timed with CUDA events on the launching stream; the job
+Timing: one priming step per cache replica (after the prefill every ring is
+full, so a replica's first step flushes all of its sequences; the priming
+steps are timed and reported on their own), W warm-up steps, then exactly K
+steps between barriers and device synchronisations, timed with CUDA events
+on the launching stream; the job
 value is the max over ranks. Steps cycle over independent cache replicas
 whose total size exceeds the 126 MB L2 many times over, so no step finds its
 cache in L2, and each replica grows by only K/replicas tokens. Multi-GPU
@@ -380,7 +383,7 @@ def run_kvq(a):
     R = a.replicas
     T = a.query_tokens  # query tokens per sequence and step (their keys and values are appended first)
     split_append = spec.get("split_append", False) and T == 1
-    steps_per_rep = math.ceil((a.warmup + 2 * a.steps) / R) + 2
+    steps_per_rep = math.ceil((a.warmup + 2 * a.steps) / R) + 3  # + the priming step
     cap = max(ctx) + sinks + steps_per_rep * T + G
     pool_pages = 0
     if a.page_blocks:
@@ -410,11 +413,11 @@ def run_kvq(a):
     # quantized bytes per token (all KV heads) of each layer: the library's
     # block record (codes, scales and zero points of G tokens of one KV head) / G
     bytes_tok = [Hkv * caches[0].layout(layer).record_bytes / G for layer in range(NL)]
-    # tensor-core layers take the new token inside the decode launch:
-    # per-channel keys without the rotation, or per-token keys over whole head
-    # vectors, blocks of >= 64 tokens, 2-bit values in groups of >= 64
-    fused = G >= 64 and ((k_axis == 0 and not rot) or (k_axis == 1 and wl.group_v == D)) and \
-        (min(wl.v_bits) > 2 or wl.group_v >= 64)
+    # layers on a tensor-core kernel take the new token inside the decode
+    # launch (kvq_decode_step); the library says which kernel a layer runs
+    kernels = [caches[0].decode_kernel(layer) for layer in range(NL)]
+    fused = all(kn != "cuda_core" for kn in kernels)
+    max_rows = 2 if "tensor_core_pair" in kernels else 8  # query rows per KV head one decode pass takes
 
     # The device-timed loop calls the C entry points with arguments prepared
     # here, so that Python overhead per call stays far below the GPU time of a
@@ -451,8 +454,21 @@ def run_kvq(a):
         if st:
             raise RuntimeError(f"kvq call failed: {lib.kvq_last_error().decode()}")
 
+    # Priming: one step on every replica before the warm-up steps. After the
+    # prefill every sequence's ring is full (the context is a multiple of G),
+    # so the first step on a replica flushes every sequence; in steady state a
+    # sequence flushes once every G / T steps. Without priming a short run
+    # (fewer steps than replicas) would time almost only first-visit flushes.
+    # The priming steps are timed on their own and reported.
+    mirror0 = [[caches[r].lengths(layer, 0)[0] for layer in range(NL)] for r in range(R)]
+    prime_ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(R)]
+    for r in range(R):
+        step(r, r, prime_ev[r])
+    torch.cuda.synchronize()
+    prime_flush = [any(caches[r].lengths(layer, 0)[0] > mirror0[r][layer] for layer in range(NL)) for r in range(R)]
+    prime_ms = [e[0].elapsed_time(e[2]) for e in prime_ev]
     for i in range(a.warmup):
-        step(i, i % R)
+        step(R + i, i % R)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -467,7 +483,7 @@ def run_kvq(a):
     groups, t0, ngr = 0, 0, Hq // Hkv  # decode passes of a multi-token step (<= 8 query rows per KV head each)
     while t0 < T:
         tp = 1
-        while 2 * tp * ngr <= 8 and t0 + 2 * tp <= T:
+        while 2 * tp * ngr <= max_rows and t0 + 2 * tp <= T:
             tp *= 2
         groups, t0 = groups + 1, t0 + tp
     for i in range(a.steps):
@@ -515,8 +531,14 @@ def run_kvq(a):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     h0 = time.perf_counter()
     e0.record(stream)
+    # host cost of enqueueing a step: the first nburst steps (later ones also
+    # wait for room in the launch queue once the GPU falls behind)
+    nburst = min(a.steps, 32)
+    burst_s = 0.0
     for i in range(a.steps):
         step(a.warmup + i, plan[i][0], events[i])
+        if i + 1 == nburst:
+            burst_s = time.perf_counter() - h0
     e1.record(stream)
     host_s = time.perf_counter() - h0
     torch.cuda.synchronize()
@@ -665,7 +687,10 @@ def run_kvq(a):
                 "flush_steps": len(fl),
                 "nonflush_step_us": nf_us if nf else None,
                 "nonflush_steps": len(nf),
-                "host_enqueue_us_per_step": host_s / a.steps * 1e6,
+                "host_enqueue_us_per_step": burst_s / nburst * 1e6,
+                "host_loop_us_per_step": host_s / a.steps * 1e6,
+                "prime_step_us": 1e3 * sum(prime_ms) / len(prime_ms),
+                "prime_steps_flushing": sum(prime_flush),
                 "alg_bytes_per_step": alg_total / a.steps,
             },
             "e2e": {"value": e2e_value, "unit": UNIT,

@@ -147,16 +147,21 @@ typedef struct kvq_cache kvq_cache;
  *       packs the codes of channels w*(32/v_bits) + i, code i at bits
  *       [i*v_bits, ...) (per-token values packed along head_dim);
  *   vsz fp16 scale and zero point of each (token, value group): for
- *       T < 64 the pairs [T][D/group_v] of (scale, zero point); for T = 64
- *       16-byte entries in the order the decode kernel reads them (see
- *       kvq_internal.cuh: vsz_half_index).
+ *       T = 64, and for the pair layout below, 16-byte entries in the order
+ *       the decode kernel reads them (see kvq_internal.cuh:
+ *       vsz_half_index); otherwise the pairs [T][D/group_v] of (scale, zero
+ *       point).
  * Placement inside kc and vc (so that one copy of a tile is readable with
  * ldmatrix without shared-memory bank conflicts): in a row of n >= 2
  * 16-byte chunks (4 words each), chunk c of row r is stored at chunk
  * position c ^ s(r, n), with s(r, n) = r & 7 for n >= 8 and
  * (r / (8/n)) % n otherwise; rows of fewer than 4 words are not permuted.
  * Value rows are stored in token order t -> (t % c) * (T/c) + t / c, with
- * c = 16/k_bits. (kvq_internal.cuh: kc_word_index, vc_word_index,
+ * c = 16/k_bits. Pair layout (T = 32 with 2-bit keys, W = 2): the key rows
+ * of channels d and d + 64 (d < 64) share 16 bytes, words 4d, 4d+1 (channel
+ * d) and 4d+2, 4d+3 (channel d + 64); token t = 8a + b (b < 8) sits in value
+ * row 16*(b/4) + 8*((b/2) % 2) + 2a + b % 2.
+ * (kvq_internal.cuh: kc_word_index, vc_word_index,
  * kc_word_byte, ksz_pair_byte, vc_word_byte, vsz_half_byte.)
  * Rings: keys [max_batch][num_kv_heads][R][D] and values
  * [max_batch][num_kv_heads][RV][D] in kv_dtype (RV = residual_v, or R);
@@ -365,6 +370,21 @@ KVQ_API kvq_status kvq_seq_value_lengths(const kvq_cache* cache, int32_t layer, 
 /* Host mirror of a sequence's sink tokens, min(S, tokens appended). No
  * counterpart on the pages beyond the sinks themselves (KV1 card).         */
 KVQ_API kvq_status kvq_seq_sinks(const kvq_cache* cache, int32_t layer, int32_t seq, int32_t* sinks);
+
+/* Which decode kernel kvq_decode_attention runs for one layer when a KV
+ * head has rows_per_kv_head query rows (num_q_heads / num_kv_heads for one
+ * query token per sequence): the general CUDA-core split kernel, the
+ * tensor-core kernel (key blocks of 64 or more tokens), or its variant for
+ * 32-token blocks with 2-bit keys (at most two rows per KV head). The
+ * choice depends on the device's shared memory: call with the cache's
+ * device current. A test and tuning accessor; no counterpart on the pages. */
+typedef enum kvq_kernel {
+  KVQ_KERNEL_CUDA_CORE = 0,
+  KVQ_KERNEL_TENSOR_CORE = 1,
+  KVQ_KERNEL_TENSOR_CORE_PAIR = 2
+} kvq_kernel;
+KVQ_API kvq_status kvq_decode_kernel(const kvq_cache* cache, int32_t layer, int32_t rows_per_kv_head,
+                                     int32_t* kernel);
 
 /* Static description of a status code.                                     */
 KVQ_API const char* kvq_status_string(kvq_status status);

@@ -42,15 +42,29 @@ def chunk_swizzle(row: int, n: int) -> int:
     return (row // (8 // n)) % n
 
 
+def pair_layout(G: int, kb: int) -> bool:
+    """32-token blocks with 2-bit keys: channels d and d + 64 share a 16-byte key row."""
+    return G == 32 and kb == 2
+
+
+def vc_row(t: int, G: int, kb: int) -> int:
+    if pair_layout(G, kb):
+        a, b = divmod(t, 8)
+        return 16 * (b // 4) + 8 * ((b // 2) % 2) + 2 * a + b % 2
+    c = 16 // kb
+    return (t % c) * (G // c) + t // c
+
+
 def kc_word_index(d: int, w: int, W: int) -> int:
+    if W == 2:  # pair layout (head_dim 128)
+        return (d % 64) * 4 + (d // 64) * 2 + w
     if W < 4:
         return d * W + w
     return d * W + (((w >> 2) ^ chunk_swizzle(d, W // 4)) << 2) + (w & 3)
 
 
 def vc_word_index(t: int, w: int, G: int, kb: int, VW: int) -> int:
-    c = 16 // kb
-    r = (t % c) * (G // c) + t // c
+    r = vc_row(t, G, kb)
     if VW < 4:
         return r * VW + w
     return r * VW + (((w >> 2) ^ chunk_swizzle(r, VW // 4)) << 2) + (w & 3)
@@ -59,6 +73,10 @@ def vc_word_index(t: int, w: int, G: int, kb: int, VW: int) -> int:
 def vsz_half_index(t: int, gg: int, G: int, kb: int, ngrp: int, zero: bool) -> int:
     """Half position of the value scale (or zero point) of token t, group gg,
     in a record's vsz array (layout documented in kvq.h)."""
+    if pair_layout(G, kb):
+        kst, r = divmod(vc_row(t, G, kb), 16)
+        entry = (kst * 4 + ((r & 7) >> 1)) * ngrp + gg
+        return entry * 8 + (4 if zero else 0) + 2 * (r >> 3) + (r & 1)
     if G < 64:
         return (t * ngrp + gg) * 2 + (1 if zero else 0)
     cpt16, tokc = 16 // kb, 128 // kb
