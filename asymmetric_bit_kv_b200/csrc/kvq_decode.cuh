@@ -111,6 +111,7 @@ struct MmaPlan {
   int32_t vsz_soff;     // value scale/zero
   int32_t stage_bytes;
   int32_t nstages;      // stages per warp
+  int32_t lg_nt;        // log2 of the tile items per block record
   int32_t ws_soff;      // first consumer-warp scratch
   int32_t ws_bytes;     // bytes per consumer-warp scratch
   int32_t bfrag_off;    // scratch: key B fragments (q*s, fp16 high/low)

@@ -15,7 +15,7 @@
 //    The B operand has room for both because a KV head has at most two query
 //    rows here: column n is query row n / 4, channel set (n / 2) % 2, fp16
 //    high (n even) or low part of q*s. A token's score is then its set-A row
-//    in one lane plus its set-B row in another (two shuffles); M-tile jp of a
+//    in one lane plus its set-B row in another (one shuffle); M-tile jp of a
 //    block holds tokens 8a + 2jp + r (rows a and a + 8, a < 4).
 //  * Values. A value chunk of 2-bit codes spans 64 channels, two 32-channel
 //    groups, so one M-tile's rows need different scales. The B operand of
@@ -45,40 +45,61 @@ struct PairShape {
   static_assert(NGRP <= 4, "value groups are columns 0-3 of a query row");
 };
 
-// Key B fragments of one block, in registers: lane (g, t) holds column g
-// (query row g / 4, channel set (g / 2) % 2, high or low part) for k rows
-// 2t, 2t+1 (e = 0) and 8+2t, 9+2t (e = 1) of paired-row k-step kk: q*s of
-// channels 64*set + 16kk + 8e + 2t and the next. bias[r] = sum_d q_rd z_d
-// times score_scale. q*s of fp16 q (times q_prescale) and fp16 s has at most
-// 22 significant bits: the high part and the rounded remainder hold it.
-__device__ __forceinline__ void pair_prep(const uint8_t* stage, int kc_bytes, const uint32_t* qw, int NG, int lane,
+// The query words a lane needs for the key B fragments of every block of a
+// unit (loaded once per unit): lane (g, t) holds column g -- query row g / 4,
+// channel set (g / 2) % 2, high (g even) or low part -- for k rows 2t, 2t+1
+// (e = 0) and 8+2t, 9+2t (e = 1) of paired-row k-step kk, i.e. channels
+// 64*set + 16kk + 8e + 2t and the next (qk), and for the bias the channels
+// 2l, 2l+1 and 64+2l, 65+2l of lane l of both query rows (qb).
+struct PairQuery {
+  uint32_t qk[4][2];
+  uint32_t qb[2][2];
+};
+__device__ __forceinline__ void pair_query(const uint32_t* qw, int NG, int lane, PairQuery& pq) {
+  const int g = lane >> 2, t = lane & 3;
+  const int row = g >> 2, set = (g >> 1) & 1;
+  const bool present = row < NG;
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) pq.qk[kk][e] = present ? qw[q_word(row, 32 * set + 8 * kk + 4 * e + t)] : 0u;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    pq.qb[r][0] = r < NG ? qw[q_word(r, lane)] : 0u;
+    pq.qb[r][1] = r < NG ? qw[q_word(r, 32 + lane)] : 0u;
+  }
+}
+
+// Key B fragments of one block (registers, the columns of pair_query): q*s
+// of fp16 q (times q_prescale) and fp16 s has at most 22 significant bits,
+// so the high part and the rounded remainder hold it. bias[r] = sum_d q_rd
+// z_d times score_scale.
+__device__ __forceinline__ void pair_prep(const uint8_t* stage, int kc_bytes, const PairQuery& pq, int NG, int lane,
                                           float score_scale, uint32_t (&bq)[4][2], float (&bias)[2]) {
   const uint2* ksz2 = reinterpret_cast<const uint2*>(stage + kc_bytes);  // (s, z) of channels 2w, 2w+1
   const int g = lane >> 2, t = lane & 3;
-  const int row = g >> 2, set = (g >> 1) & 1;
-  const bool low = g & 1, present = row < NG;
+  const int set = (g >> 1) & 1;
+  const bool low = g & 1;
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const int w = 32 * set + 8 * kk + 4 * e + t;
-      const uint32_t q2 = present ? qw[q_word(row, w)] : 0u;
-      const uint2 sz = ksz2[w];
+      const uint2 sz = ksz2[32 * set + 8 * kk + 4 * e + t];
       const uint32_t s2 = __byte_perm(sz.x, sz.y, 0x5410);
-      const uint32_t hi = hmul2(q2, s2);
-      bq[kk][e] = low ? hfms2(q2, s2, hi) : hi;
+      const uint32_t hi = hmul2(pq.qk[kk][e], s2);
+      bq[kk][e] = low ? hfms2(pq.qk[kk][e], s2, hi) : hi;
     }
+  const uint2 sa = ksz2[lane], sb = ksz2[32 + lane];
+  bias[0] = bias[1] = 0.f;
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
-    float bp = 0.f;
-    if (r < NG) {  // channels 2l, 2l+1 and 64+2l, 65+2l of lane l
-      const uint2 sa = ksz2[lane], sb = ksz2[32 + lane];
-      bp = fma_q_z(qw[q_word(r, lane)], sa.x, sa.y, bp);
-      bp = fma_q_z(qw[q_word(r, 32 + lane)], sb.x, sb.y, bp);
-    }
+    if (r < NG) {  // warp-uniform
+      float bp = fma_q_z(pq.qb[r][0], sa.x, sa.y, 0.f);
+      bp = fma_q_z(pq.qb[r][1], sb.x, sb.y, bp);
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) bp += __shfl_xor_sync(0xffffffffu, bp, o);
-    bias[r] = bp * score_scale;
+      for (int o = 1; o < 32; o <<= 1) bp += __shfl_xor_sync(0xffffffffu, bp, o);
+      bias[r] = bp * score_scale;
+    }
   }
 }
 
@@ -197,12 +218,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_pair_kernel(DecodeParams p
   const bool valid[1] = {qrow < NG};
   const uint32_t ones[4] = {0x3c003c00u, 0x3c003c00u, 0x3c003c00u, 0x3c003c00u};  // fp16 1.0
   const int swv = chunk_swizzle(rr, S::NCH);
-  const int srcA = lane & ~1, srcB = ((lane | 1) + 16) & 31;  // set-A and set-B lanes of row g's token
+  // a token's set-A and set-B score rows meet in lanes (g < 4, t even) and
+  // (g >= 4, t odd), one xor-17 shuffle apart; both hold its full score
+  const bool score_lane = (g < 4) == ((t & 1) == 0);
   const int psrc = 4 * t + 2 * (g >> 2);                      // probabilities of B column g (query row g / 4)
   const bool pcol = (g >> 2) < NG;
   const int vgrp = min(g & 3, NGRP - 1);                      // value group of B column g
   uint2* bkw = reinterpret_cast<uint2*>(ws + mp.bfrag_off);
-  int qseq = -1;
+  int qslot = -1;  // query buffer of the current unit (matches IssueState::qslot)
+  int st = 0;      // stage of item n and its barrier phase parity
+  uint32_t ph = 0;
+  PairQuery pq;  // the unit's query words for the key B fragments
   UnitCursor u;
   int k = rs;
   while (k < re && !failed) {
@@ -219,16 +245,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_pair_kernel(DecodeParams p
     bool rq_ready = false;
     const int first = k + ((warp - (k - rs)) % kNC + kNC) % kNC;
     for (int kb = first; kb < hi; kb += kNC, ++n) {
-      const int st = n % SPW;
-      if (!mbar_wait(full + st, (n / SPW) & 1)) {
+      if (!mbar_wait(full + st, ph)) {
         failed = true;
         break;
       }
       const uint8_t* stage = stages + (size_t)st * mp.stage_bytes;
-      uint32_t* qw = reinterpret_cast<uint32_t*>(qbuf + (size_t)((qseq + (kb == first)) % SPW) * NG * kRowBytes);
+      if (kb == first) qslot = qslot + 1 == SPW ? 0 : qslot + 1;
+      uint32_t* qw = reinterpret_cast<uint32_t*>(qbuf + (size_t)qslot * NG * kRowBytes);
       if (kb == first) {
         // the unit's queries, to fp16 times q_prescale in the q_word order
-        ++qseq;
         uint32_t cv[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -245,13 +270,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_pair_kernel(DecodeParams p
           if (w < NG * (D / 2)) qw[q_word(w / (D / 2), w % (D / 2))] = cv[i];
         }
         __syncwarp();
+        pair_query(qw, NG, lane, pq);
       }
       const int j = kb - u.start;
       if (j < nb) {
         // ============ quantized block of 32 tokens
         uint32_t bq[4][2];
         float bias[2];
-        pair_prep(stage, mp.kc_bytes, qw, NG, lane, p.score_scale, bq, bias);
+        pair_prep(stage, mp.kc_bytes, pq, NG, lane, p.score_scale, bq, bias);
         const float bias_l = qrow ? bias[1] : bias[0];
         const uint32_t kc_s = smem_u32(stage);
         const uint32_t vc_s = smem_u32(stage + mp.vc_soff);
@@ -275,16 +301,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_pair_kernel(DecodeParams p
             }
           }
         }
-        // ---- a token's score: its set-A row plus its set-B row (rows g < 4
-        // of M-tile jp: tokens 8g + 2jp, 8g + 2jp + 1)
+        // ---- a token's score: its set-A row plus its set-B row (M-tile jp,
+        // rows g and g + 8: tokens 8(g % 4) + 2jp and 8(g % 4) + 2jp + 1)
         float sc[4][2];
 #pragma unroll
         for (int jp = 0; jp < 4; ++jp)
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
             const float x = Dk[jp][2 * r] + Dk[jp][2 * r + 1];
-            const float s = __shfl_sync(0xffffffffu, x, srcA) + __shfl_sync(0xffffffffu, x, srcB);
-            sc[jp][r] = g < 4 ? fmaf(s, p.score_scale * code_unscale<2>(2 * jp + r), bias_l) : -INFINITY;
+            const float s = x + __shfl_xor_sync(0xffffffffu, x, 17);
+            sc[jp][r] = score_lane ? fmaf(s, p.score_scale * code_unscale<2>(2 * jp + r), bias_l) : -INFINITY;
           }
         softmax_update<4, 1, 1, false, true>(sc, sst, valid, O, Z, lane);
         // ---- values: O += codes x (p * s), Z += ones x (p * z)
@@ -329,6 +355,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_pair_kernel(DecodeParams p
       if (lane == 0 && n + SPW < nmine) {
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         issue_item(p, mp, is, rs + warp + (n + SPW) * kNC, stages + (size_t)st * mp.stage_bytes, full + st, qbuf, NG);
+      }
+      if (++st == SPW) {
+        st = 0;
+        ph ^= 1u;
       }
     }
     if (failed) break;

@@ -97,6 +97,7 @@ MmaPlan make_mma_plan(const LayerView& L, int num_q_heads) {
   // (one tile), or a tile part of a longer block (plus the block's
   // per-channel key scales, when it stores them once for all its tiles)
   const int NT = G / L.tile_tokens;
+  mp.lg_nt = NT == 4 ? 2 : NT == 2 ? 1 : 0;  // G / tile_tokens: 1, 2 (or 4)
   const int ksz_stage = L.rec_ksz_off >= 0 ? kHeadDim * 4 : L.vc_off - L.ksz_off;
   mp.kc_bytes = L.ksz_off;
   mp.vc_soff = mp.kc_bytes + ksz_stage;

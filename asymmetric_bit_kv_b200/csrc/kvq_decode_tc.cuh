@@ -731,14 +731,16 @@ __device__ __forceinline__ void store_new_token(const DecodeParams& p, int b, in
 // item and the number of unit changes so far.
 struct IssueState {
   UnitCursor u;
-  int unit = -1, seq = -1;
+  int unit = -1;
+  int qslot = -1;         // query buffer of the unit (round robin over the nstages buffers)
+  int ring0 = 0;          // ring slot of the unit's first ring token
   int run = -1;           // paged cache: page-table entry (j / page_blocks) of the unit held in `page`
   int64_t page = 0;
 };
 
 // Issues the copy of work item k (a block record, or the key and value rows
 // of a ring chunk) into stage `dst`, completing on `bar`; on the first item
-// of a unit also the unit's queries, into query buffer seq % nstages.
+// of a unit also the unit's queries, into the next query buffer (qslot).
 __device__ __forceinline__ void issue_item(const DecodeParams& p, const MmaPlan& mp, IssueState& is, int k,
                                            uint8_t* dst, uint64_t* bar, uint8_t* qbuf, int NG) {
   const LayerView& L = p.L;
@@ -750,12 +752,12 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, const MmaPlan&
   const uint32_t qbytes = NG * kRowBytes;
   if (newq) {
     is.unit = unit;
-    ++is.seq;
+    is.qslot = is.qslot + 1 == mp.nstages ? 0 : is.qslot + 1;
+    is.ring0 = (nb * L.tile_tokens) % L.residual;
   }
   if (j < nb) {
-    // tile item j: tile j % NT of block j / NT (NT tiles per block)
-    const int NT = L.group_k / L.tile_tokens;
-    const int jb = j / NT, jt = j % NT;
+    // tile item j: tile j % NT of block j / NT (NT = 2^lg_nt tiles per block)
+    const int jb = j >> mp.lg_nt, jt = j & ((1 << mp.lg_nt) - 1);
     mbar_expect_tx(bar, mp.tx_bytes + (newq ? qbytes : 0u));
     const uint8_t* rec;
     if (L.page_table) {  // one page-table read per run of page_blocks blocks of the unit
@@ -768,7 +770,7 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, const MmaPlan&
     } else {
       rec = record_ptr(L, u.b, u.h, jb);
     }
-    if (NT == 1) {
+    if (mp.lg_nt == 0) {
       bulk_g2s(dst, rec, mp.tx_bytes, bar);
     } else {
       const uint8_t* tp = rec + L.tile0_off + (int64_t)jt * L.tile_bytes;
@@ -798,7 +800,8 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, const MmaPlan&
     if (sink) {
       row = ((int64_t)u.b * L.num_kv_heads + u.h) * KVQ_MAX_SINKS;
     } else {
-      const int slot = (nb * L.tile_tokens + (j - nb) * kResChunk) % L.residual;
+      int slot = is.ring0 + (j - nb) * kResChunk;  // (j - nb) * kResChunk < residual
+      if (slot >= L.residual) slot -= L.residual;
       row = ((int64_t)u.b * L.num_kv_heads + u.h) * L.residual + slot;
     }
     constexpr uint32_t bytes = kResChunk * kRowBytes;
@@ -829,7 +832,7 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, const MmaPlan&
   if (newq) {
     // the unit's query rows: ngr heads of each of the launch's query tokens
     const int ngr = p.q_heads / L.num_kv_heads;
-    uint8_t* qdst = qbuf + (size_t)(is.seq % mp.nstages) * qbytes;
+    uint8_t* qdst = qbuf + (size_t)is.qslot * qbytes;
     for (int t = 0; t < p.qtok; ++t)
       bulk_g2s(qdst + (size_t)t * ngr * kRowBytes,
                reinterpret_cast<const uint8_t*>(p.q) +
@@ -862,8 +865,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
   // otherwise)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   // this warp's items: rs + warp + n*kNC, n = 0, 1, ...; item n lands in the
-  // warp's own stage n % SPW, and the warp issues item n + SPW as soon as it
-  // is done with item n
+  // warp's own stage n % SPW (phase parity (n / SPW) & 1, both kept
+  // incrementally), and the warp issues item n + SPW as soon as it is done
+  // with item n
   const int SPW = mp.nstages;  // stages per warp
   uint8_t* stages = smem + (size_t)warp * SPW * mp.stage_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + mp.bar_off) + warp * SPW;
@@ -897,7 +901,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
     const uint2* bkr = reinterpret_cast<const uint2*>(ws + mp.bfrag_off);
     uint2* bkw = reinterpret_cast<uint2*>(ws + mp.bfrag_off);
     const float* biasr = reinterpret_cast<const float*>(ws + mp.bias_off);
-    int qseq = -1;  // unit changes seen by the consumer side (matches IssueState::seq)
+    int qslot = -1;  // query buffer of the current unit (matches IssueState::qslot)
+    int st = 0;      // stage of item n and its barrier phase parity
+    uint32_t ph = 0;
     const bool v0 = 2 * t < NG, v1 = 2 * t + 1 < NG;  // output columns (heads 2t, 2t+1) of this lane exist
     constexpr int HPL = heads_per_lane<NKT>();
     bool valid[HPL];  // score heads of this lane exist
@@ -930,17 +936,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
       // this warp's items of the unit: k' - rs = warp (mod kNC)
       const int first = k + ((warp - (k - rs)) % kNC + kNC) % kNC;
       for (int kb = first; kb < hi; kb += kNC, ++n) {
-        const int st = n % SPW;
-        if (!mbar_wait(full + st, (n / SPW) & 1)) {
+        if (!mbar_wait(full + st, ph)) {
           failed = true;
           break;
         }
         const uint8_t* stage = stages + (size_t)st * mp.stage_bytes;
-        uint32_t* qw = reinterpret_cast<uint32_t*>(qbuf + (size_t)((qseq + (kb == first)) % SPW) * NG * kRowBytes);
+        if (kb == first) qslot = qslot + 1 == SPW ? 0 : qslot + 1;
+        uint32_t* qw = reinterpret_cast<uint32_t*>(qbuf + (size_t)qslot * NG * kRowBytes);
         if (kb == first) {
           // the warp's first item of the unit brought its queries: to fp16
           // times q_prescale, in place
-          ++qseq;
           // (the permutation stays inside each head: four heads at a time)
           for (int h0 = 0; h0 < NG; h0 += 4) {
             uint32_t cv[8];
@@ -1127,6 +1132,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
         if (lane == 0 && n + SPW < nmine) {
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           issue_item(p, mp, is, rs + warp + (n + SPW) * kNC, stages + (size_t)st * mp.stage_bytes, full + st, qbuf, NG);
+        }
+        if (++st == SPW) {
+          st = 0;
+          ph ^= 1u;
         }
       }
       if (failed) break;

@@ -689,7 +689,7 @@ def run_kvq(a):
                 "nonflush_steps": len(nf),
                 "host_enqueue_us_per_step": burst_s / nburst * 1e6,
                 "host_loop_us_per_step": host_s / a.steps * 1e6,
-                "prime_step_us": 1e3 * sum(prime_ms) / len(prime_ms),
+                "prime_step_us": 1e3 * statistics.median(prime_ms),
                 "prime_steps_flushing": sum(prime_flush),
                 "alg_bytes_per_step": alg_total / a.steps,
             },
