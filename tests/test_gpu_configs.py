@@ -27,6 +27,13 @@ def _expected_lengths(L, R, G):
     return q, L - q
 
 
+# Largest errors of the fp32 decode outputs against the oracle, per workload
+# (max-abs, max-rel with rel = |a - b| / max(|b|, 0.2), the kernel that ran):
+# the margin to the 2e-3 / 1e-2 tolerance at full size, printed (and written
+# as JSON to $KVQ_ERROR_TABLE if set) by the last test of this file.
+ERRORS: dict = {}
+
+
 def _decode_and_check(tw: Twin, wl: W.Workload, layer: int, q: torch.Tensor, seqs, out_dtype=torch.float32):
     out = tw.gpu.decode_attention(layer, q.cuda(), out_dtype=out_dtype, softmax_scale=wl.softmax_scale)
     assert tw.gpu.device_errors() == 0
@@ -37,6 +44,14 @@ def _decode_and_check(tw: Twin, wl: W.Workload, layer: int, q: torch.Tensor, seq
         ref = tw.oracle_decode(layer, b, qn[b], wl.softmax_scale)
         if out_dtype == torch.float32:
             assert_attention_close(out[b], ref, f"layer {layer} seq {b}")
+            err = np.abs(out[b] - ref)
+            e = ERRORS.setdefault(wl.name, {"max_abs": 0.0, "max_rel": 0.0, "outputs": 0, "kernels": []})
+            e["max_abs"] = max(e["max_abs"], float(err.max()))
+            e["max_rel"] = max(e["max_rel"], float((err / np.maximum(np.abs(ref), 0.2)).max()))
+            e["outputs"] += int(err.size)
+            kern = tw.gpu.decode_kernel(layer)
+            if kern not in e["kernels"]:
+                e["kernels"].append(kern)
         else:
             assert np.all(np.abs(out[b] - ref) <= ulp(ref, out_dtype) / 2 + 2e-3)
     return out
@@ -141,3 +156,22 @@ def test_qwen3_36_layers_ragged_sampled():
         for b in (lo, hi):
             tw.check_codes(layer, b)
         _decode_and_check(tw, wl, layer, q, [lo, hi])
+
+
+def test_zz_error_table():
+    """The full-size error record of the tests above (run after them)."""
+    import json
+    import os
+
+    names = [f().name for f in (W.tiny_mha, W.llama2_7b_mha, W.llama3_8b_gqa, W.long_context_gqa, W.qwen3_8b_layers)]
+    for n in names:
+        if n in ERRORS:
+            e = ERRORS[n]
+            print(f"{n:48s} max_abs {e['max_abs']:.2e} (bound 2e-3)  max_rel {e['max_rel']:.2e} (bound 1e-2)  "
+                  f"outputs {e['outputs']}  kernels {','.join(e['kernels'])}")
+    path = os.environ.get("KVQ_ERROR_TABLE")
+    if path:
+        with open(path, "w") as f:
+            json.dump(ERRORS, f, indent=1)
+    if len(ERRORS) == len(names):  # the whole file ran: every workload has its record
+        assert all(ERRORS[n]["max_abs"] <= 2e-3 and ERRORS[n]["max_rel"] <= 1e-2 for n in names)
