@@ -391,11 +391,18 @@ __global__ void __launch_bounds__(32 * (WPH > 4 ? WPH : 4)) combine_kernel(Combi
     }
   }
   if constexpr (WPH > 1) {
+    // the head's warps merge their states pairwise in shared memory
     s_st[warp][lane] = st;
     __syncthreads();
-    if (wi != 0) return;
 #pragma unroll
-    for (int i = 1; i < WPH; ++i) merge_into(st, s_st[warp + i][lane]);
+    for (int half = WPH / 2; half >= 1; half >>= 1) {
+      if (wi < half) {
+        merge_into(st, s_st[warp + half][lane]);
+        if (half > 1) s_st[warp][lane] = st;
+      }
+      if (half > 1) __syncthreads();
+    }
+    if (wi != 0) return;
   }
   if (!active) return;
   float4 acc = st.acc;
@@ -497,10 +504,11 @@ cudaError_t launch_decode(const DecodeParams& p, int max_splits, cudaStream_t st
 
 cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream) {
   if (p.batch <= 0) return cudaSuccess;
-  // Warps per (sequence, query head): enough that each merges at most ~32
-  // slots (two rounds of loads), from the most slots a unit can use.
+  // Warps per (sequence, query head): enough that each merges at most 16
+  // slots (one round of loads), from the most slots a unit can use.
   const int most = p.persistent ? p.max_unit_slots : p.slots;
-  const int wph = most <= 32 ? 1 : most <= 64 ? 2 : most <= 128 ? 4 : 8;
+  int wph = 1;
+  while (wph < 32 && wph * 16 < most) wph *= 2;
   const int warps = wph > 4 ? wph : 4, heads = warps / wph;
   // Programmatic dependent launch: the combine grid may be scheduled while
   // the decode grid (which allows it at its start) is still running; each
@@ -523,7 +531,9 @@ cudaError_t launch_combine(const DecodeParams& p, cudaStream_t stream) {
     case 1: return cudaLaunchKernelEx(&cfg, combine_kernel<1>, cp);
     case 2: return cudaLaunchKernelEx(&cfg, combine_kernel<2>, cp);
     case 4: return cudaLaunchKernelEx(&cfg, combine_kernel<4>, cp);
-    default: return cudaLaunchKernelEx(&cfg, combine_kernel<8>, cp);
+    case 8: return cudaLaunchKernelEx(&cfg, combine_kernel<8>, cp);
+    case 16: return cudaLaunchKernelEx(&cfg, combine_kernel<16>, cp);
+    default: return cudaLaunchKernelEx(&cfg, combine_kernel<32>, cp);
   }
 }
 
