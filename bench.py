@@ -432,6 +432,12 @@ def run_kvq(a):
 
     lib_s = [0.0]  # host time inside the library's entry points (ctypes calls included)
 
+    def timed(fn, *args):
+        t = time.perf_counter()
+        st = fn(*args)
+        lib_s[0] += time.perf_counter() - t
+        return st
+
     def step(i, r, ev=None):
         """One step on replica r: every layer; ev = (start, after append, end)
         events (the middle one only with split_append)."""
@@ -440,19 +446,17 @@ def run_kvq(a):
         if ev is not None:
             ev[0].record(stream)
         st = 0
-        t_lib = time.perf_counter()
         for layer in range(NL):
             if split_append:
-                st = st or c_append(h, layer, kp, vp, t_lens, B, sh)
+                st = st or timed(c_append, h, layer, kp, vp, t_lens, B, sh)
                 if ev is not None and layer == NL - 1:
                     ev[1].record(stream)
-                st = st or c_decode(h, layer, qp, optr, oty, scale, B, sh)
+                st = st or timed(c_decode, h, layer, qp, optr, oty, scale, B, sh)
             elif T == 1:
-                st = st or c_step(h, layer, kp, vp, qp, optr, oty, scale, B, sh)
+                st = st or timed(c_step, h, layer, kp, vp, qp, optr, oty, scale, B, sh)
             else:  # the T tokens' keys and values, then the T queries of every sequence
-                st = st or c_append(h, layer, kp, vp, t_lens, B, sh) or c_multi(h, layer, qp, optr, oty, scale, B, T,
-                                                                               sh)
-        lib_s[0] += time.perf_counter() - t_lib
+                st = st or timed(c_append, h, layer, kp, vp, t_lens, B, sh) or \
+                    timed(c_multi, h, layer, qp, optr, oty, scale, B, T, sh)
         if ev is not None:
             ev[2].record(stream)
         if st:
@@ -535,9 +539,10 @@ def run_kvq(a):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     h0 = time.perf_counter()
     e0.record(stream)
-    # host cost of enqueueing a step: the first nburst steps (later ones also
-    # wait for room in the launch queue once the GPU falls behind)
-    nburst = min(a.steps, 32)
+    # host cost of enqueueing a step: the first nburst steps, about 64 library
+    # calls (later ones also wait for room in the launch queue once the GPU
+    # falls behind)
+    nburst = max(1, min(a.steps, 32, 64 // NL))
     burst_s = burst_lib_s = 0.0
     lib_s[0] = 0.0
     for i in range(a.steps):
