@@ -468,6 +468,10 @@ def run_kvq(a):
     # sequence flushes once every G / T steps. Without priming a short run
     # (fewer steps than replicas) would time almost only first-visit flushes.
     # The priming steps are timed on their own and reported.
+    # clocks are sampled from here on (priming, warm-up and the timed steps),
+    # so that no idle pause precedes the timed loop
+    clocks = ClockSampler(local)
+    clocks.start()
     mirror0 = [[caches[r].lengths(layer, 0)[0] for layer in range(NL)] for r in range(R)]
     prime_ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(R)]
     for r in range(R):
@@ -530,9 +534,6 @@ def run_kvq(a):
     alg_total = float(sum(x[2] for x in plan))
     tok_total = sum(x[3] for x in plan)
 
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.2)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
