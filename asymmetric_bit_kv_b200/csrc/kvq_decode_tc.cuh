@@ -853,7 +853,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
   const int Hkv = L.num_kv_heads;
   const int NG = p.num_q_heads / Hkv;  // query rows per unit
   const int ngr = p.q_heads / Hkv;      // query heads per KV head (rows per query token)
-  const int G = L.tile_tokens;  // tokens of one work item's tile: the block, or 64 of a longer block
+  // tokens of one work item's tile: the block, or 64 of a longer block (this
+  // kernel serves blocks of >= 64 tokens, so a tile is always 64 tokens)
+  constexpr int G = S::TT;
   const int rs = p.cta_start[c], re = p.cta_start[c + 1];
   const bool bf16 = L.kv_dtype == KVQ_BF16;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -892,7 +894,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
     }
     const int g = lane >> 2, t = lane & 3;
     const uint32_t ones[4] = {0x3c003c00u, 0x3c003c00u, 0x3c003c00u, 0x3c003c00u};  // fp16 1.0
-    const int kc_row = G * KB / 8;  // key code bytes per channel
+    constexpr int kc_row = G * KB / 8;  // key code bytes per channel of a tile
     const int mi = lane >> 3, rr = lane & 7;
     // ldmatrix rows of this lane: 8 consecutive rows, so the chunk swizzle of
     // the record layout depends on the lane's row index only
@@ -985,7 +987,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecodeParams p, 
           const uint32_t kc_s = smem_u32(stage);
           const uint32_t vc_s = smem_u32(stage + mp.vc_soff);
           const uint4* vsz4 = reinterpret_cast<const uint4*>(stage + mp.vsz_soff);
-          for (int tile = 0; tile < G / S::TT; ++tile) {
+#pragma unroll
+          for (int tile = 0; tile < G / S::TT; ++tile) {  // one tile per item
             // ---- scores: Dk[M-tile][n-tile] = codes x (q*s)
             float Dk[S::MT][NKT][4];
 #pragma unroll
