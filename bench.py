@@ -142,6 +142,47 @@ def _peaks():
 # clocks during the timed region
 # --------------------------------------------------------------------------
 
+class _Driver:
+    """The few CUDA driver calls of the end-to-end leg (asynchronous copies,
+    events and stream waits on raw handles), through ctypes: a microsecond or
+    two each, where torch's stream and event wrappers take several."""
+
+    def __init__(self):
+        import ctypes
+        c = ctypes.CDLL("libcuda.so.1")
+        P, U64, SZ, U = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_size_t, ctypes.c_uint
+        self._ct = ctypes
+        self._h2d, self._d2h = c.cuMemcpyHtoDAsync_v2, c.cuMemcpyDtoHAsync_v2
+        self._h2d.argtypes, self._d2h.argtypes = [U64, P, SZ, P], [P, U64, SZ, P]
+        self._rec, self._wait = c.cuEventRecord, c.cuStreamWaitEvent
+        self._rec.argtypes, self._wait.argtypes = [P, P], [P, P, U]
+        self._create, self._destroy = c.cuEventCreate, c.cuEventDestroy_v2
+        self._create.argtypes, self._destroy.argtypes = [ctypes.POINTER(P), U], [P]
+        for f in (self._h2d, self._d2h, self._rec, self._wait, self._create, self._destroy):
+            f.restype = ctypes.c_int
+
+    def event(self):
+        e = self._ct.c_void_p()
+        if self._create(self._ct.byref(e), 2):  # CU_EVENT_DISABLE_TIMING
+            raise RuntimeError("cuEventCreate failed")
+        return e.value
+
+    def destroy(self, e):
+        self._destroy(e)
+
+    def htod(self, dst, src, n, s):
+        return self._h2d(dst, src, n, s)
+
+    def dtoh(self, dst, src, n, s):
+        return self._d2h(dst, src, n, s)
+
+    def record(self, e, s):
+        return self._rec(e, s)
+
+    def wait(self, s, e):
+        return self._wait(s, e, 0)
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -156,6 +197,9 @@ class ClockSampler:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import atexit
+
+            atexit.register(lambda pr=self.proc: pr.poll() is None and pr.terminate())
         except Exception:
             self.proc = None
 
@@ -374,6 +418,11 @@ def run_kvq(a):
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    # clocks are sampled from here on (cache fill, priming, warm-up and the
+    # timed steps): nvidia-smi takes a while to start, and no idle pause
+    # precedes the timed loop
+    clocks = ClockSampler(local)
+    clocks.start()
     spec = SPECS[a.workload]
     wl = _bench_workload(a.workload)
     sinks, k_axis, rot = _layout(wl)
@@ -383,7 +432,9 @@ def run_kvq(a):
     R = a.replicas
     T = a.query_tokens  # query tokens per sequence and step (their keys and values are appended first)
     split_append = spec.get("split_append", False) and T == 1
-    steps_per_rep = math.ceil((a.warmup + 2 * a.steps) / R) + 3  # + the priming step
+    # steps per replica: priming, warm-up, the timed loop, the per-step pass
+    # (up to 256 steps) and the e2e leg (up to 512 steps)
+    steps_per_rep = math.ceil((a.warmup + a.steps + min(a.steps, 256) + min(a.steps, 512)) / R) + 3
     cap = max(ctx) + sinks + steps_per_rep * T + G
     pool_pages = 0
     if a.page_blocks:
@@ -468,10 +519,6 @@ def run_kvq(a):
     # sequence flushes once every G / T steps. Without priming a short run
     # (fewer steps than replicas) would time almost only first-visit flushes.
     # The priming steps are timed on their own and reported.
-    # clocks are sampled from here on (priming, warm-up and the timed steps),
-    # so that no idle pause precedes the timed loop
-    clocks = ClockSampler(local)
-    clocks.start()
     mirror0 = [[caches[r].lengths(layer, 0)[0] for layer in range(NL)] for r in range(R)]
     prime_ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(R)]
     for r in range(R):
@@ -491,49 +538,63 @@ def run_kvq(a):
     # into the quantized cache), checked against the library's host mirror after.
     lens = [[[list(caches[r].lengths(layer, b)) for b in range(B)] for layer in range(NL)] for r in range(R)]
     pages = [[[-(-(q // G) // a.page_blocks) if a.page_blocks else 0 for q, _ in row] for row in rep] for rep in lens]
-    plan = []  # (replica, launches, algorithmic bytes, KV tokens attended, any flush)
     groups, t0, ngr = 0, 0, Hq // Hkv  # decode passes of a multi-token step (<= 8 query rows per KV head each)
     while t0 < T:
         tp = 1
         while 2 * tp * ngr <= max_rows and t0 + 2 * tp <= T:
             tp *= 2
         groups, t0 = groups + 1, t0 + tp
-    for i in range(a.steps):
-        r = (a.warmup + i) % R
-        ab = tk = launches = 0
-        flush = False
-        for layer in range(NL):
-            ab += T * (2 * B * Hq * D * 2 + 2 * (2 * B * Hkv * D * 2))  # q in, out; new k, v in and into the ring
-            ab += B * sinks * Hkv * D * 2 * 2  # the exact sink tokens
-            tk += B * T * sinks
-            lflush = new_pages = False
-            for b in range(B):
-                qn, n = lens[r][layer][b]
-                f = _flushes(n, T, Rw, G)
-                lflush = lflush or f > 0
-                qn, n = qn + f * G, n + T - f * G
-                lens[r][layer][b] = [qn, n]
-                if a.page_blocks:
-                    pg = -(-(qn // G) // a.page_blocks)
-                    new_pages = new_pages or pg > pages[r][layer][b]
-                    pages[r][layer][b] = pg
-                ab += qn * bytes_tok[layer] + n * Hkv * D * 2 * 2
-                tk += T * (qn + n) - T * (T - 1) // 2  # query t sees the tokens up to its own position
-            flush = flush or lflush
-            if T == 1 and fused and not split_append:
-                # flush kernel on a flushing step, page-table update when pages
-                # are taken, decode, combine
-                launches += 2 + (1 if lflush else 0) + (1 if new_pages else 0)
-            else:
-                # append (page-table update, quantize on a flush, ring write),
-                # then decode + combine per pass
-                launches += 1 + (1 if lflush else 0) + (1 if new_pages else 0) + 2 * groups
-        plan.append((r, launches, ab, tk, flush))
-    events = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(a.steps)]
+
+    def make_plan(first, nsteps):
+        """(replica, launches, algorithmic bytes, KV tokens attended, any
+        flush) of steps first .. first + nsteps - 1, advancing lens/pages."""
+        plan = []
+        for i in range(first, first + nsteps):
+            r = i % R
+            ab = tk = launches = 0
+            flush = False
+            for layer in range(NL):
+                ab += T * (2 * B * Hq * D * 2 + 2 * (2 * B * Hkv * D * 2))  # q in, out; new k, v in and into the ring
+                ab += B * sinks * Hkv * D * 2 * 2  # the exact sink tokens
+                tk += B * T * sinks
+                lflush = new_pages = False
+                for b in range(B):
+                    qn, n = lens[r][layer][b]
+                    f = _flushes(n, T, Rw, G)
+                    lflush = lflush or f > 0
+                    qn, n = qn + f * G, n + T - f * G
+                    lens[r][layer][b] = [qn, n]
+                    if a.page_blocks:
+                        pg = -(-(qn // G) // a.page_blocks)
+                        new_pages = new_pages or pg > pages[r][layer][b]
+                        pages[r][layer][b] = pg
+                    ab += qn * bytes_tok[layer] + n * Hkv * D * 2 * 2
+                    tk += T * (qn + n) - T * (T - 1) // 2  # query t sees the tokens up to its own position
+                flush = flush or lflush
+                if T == 1 and fused and not split_append:
+                    # flush kernel on a flushing step, page-table update when pages
+                    # are taken, decode, combine
+                    launches += 2 + (1 if lflush else 0) + (1 if new_pages else 0)
+                else:
+                    # append (page-table update, quantize on a flush, ring write),
+                    # then decode + combine per pass
+                    launches += 1 + (1 if lflush else 0) + (1 if new_pages else 0) + 2 * groups
+            plan.append((r, launches, ab, tk, flush))
+        return plan
+
+    def check_mirror():
+        for r in range(R):
+            for layer in range(NL):
+                for b in range(B):
+                    assert tuple(lens[r][layer][b]) == caches[r].lengths(layer, b), "step accounting out of sync"
+
+    plan = make_plan(a.warmup, a.steps)
     launches = sum(x[1] for x in plan)
     alg_total = float(sum(x[2] for x in plan))
     tok_total = sum(x[3] for x in plan)
 
+    # The timed loop: exactly K steps between one pair of events (no event
+    # inside, so that nothing but the steps runs on the stream).
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -547,7 +608,7 @@ def run_kvq(a):
     burst_s = burst_lib_s = 0.0
     lib_s[0] = 0.0
     for i in range(a.steps):
-        step(a.warmup + i, plan[i][0], events[i])
+        step(a.warmup + i, plan[i][0])
         if i + 1 == nburst:
             burst_s = time.perf_counter() - h0
             burst_lib_s = lib_s[0]
@@ -557,22 +618,30 @@ def run_kvq(a):
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    for r in range(R):
-        for layer in range(NL):
-            for b in range(B):
-                assert tuple(lens[r][layer][b]) == caches[r].lengths(layer, b), "step accounting out of sync"
+    check_mirror()
     ms = e0.elapsed_time(e1)
+
+    # A second pass of up to 256 steps, each between its own events: how the
+    # step time splits into flush and non-flush steps (and append and
+    # attention with split_append). Not part of `value`.
+    n2 = min(a.steps, 256)
+    plan2 = make_plan(a.warmup + a.steps, n2)
+    events = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(n2)]
+    for i in range(n2):
+        step(a.warmup + a.steps + i, plan2[i][0], events[i])
+    torch.cuda.synchronize()
+    check_mirror()
     call_ms = [x[0].elapsed_time(x[2]) for x in events]
     app_ms = [x[0].elapsed_time(x[1]) for x in events] if split_append else [0.0]
-    dec_ms = sum(call_ms)
-    fl = [m for m, x in zip(call_ms, plan) if x[4]]
-    nf = [m for m, x in zip(call_ms, plan) if not x[4]]
+    fl = [m for m, x in zip(call_ms, plan2) if x[4]]
+    nf = [m for m, x in zip(call_ms, plan2) if not x[4]]
+    call_us = 1e3 * sum(call_ms) / len(call_ms)
     fl_us = 1e3 * sum(fl) / len(fl) if fl else 0.0
     nf_us = 1e3 * sum(nf) / len(nf) if nf else 0.0
     app_us = 1e3 * sum(app_ms) / len(app_ms)
-    ms, dec_ms, fl_us, nf_us, app_us = cross_rank_max([ms, dec_ms, fl_us, nf_us, app_us], world, dev)
+    ms, call_us, fl_us, nf_us, app_us = cross_rank_max([ms, call_us, fl_us, nf_us, app_us], world, dev)
     value = tok_total * world / (ms / 1e3)
-    achieved_gbs = alg_total / (dec_ms / 1e3) / 1e9
+    achieved_gbs = alg_total / (ms / 1e3) / 1e9
 
     # ---- a prefill chunk: one kvq_append of 4096 tokens to an empty sequence
     prefill = None
@@ -606,21 +675,23 @@ def run_kvq(a):
 
     # ---- end to end through the public API with host buffers ----
     # each step's k, v and q sit back to back in one pinned host buffer and
-    # travel in one host-to-device copy; the last layer's output comes back
+    # travel in one host-to-device copy; the last layer's output comes back.
+    # The copies run on their own stream, double-buffered, so that step i+1's
+    # inputs go up and step i's output comes down while the GPU computes
+    # (events order every reuse of a buffer); all of them lie inside the
+    # timed region.
     e2e_steps = min(a.steps, 512)
     nk, nq = B * T * Hkv * D, B * T * Hq * D
     hkvq = torch.empty(pool, 2 * nk + nq, dtype=wl.kv_dtype).pin_memory()
     hkvq[:, :nk].copy_(new_k.reshape(pool, nk).cpu())
     hkvq[:, nk:2 * nk].copy_(new_v.reshape(pool, nk).cpu())
     hkvq[:, 2 * nk:].copy_(qs.reshape(pool, nq).cpu())
-    hout = torch.empty(B * T, Hq, D, dtype=wl.kv_dtype).pin_memory()
-    dkvq = torch.empty(2 * nk + nq, dtype=wl.kv_dtype, device=dev)
-    dk = dkvq[:nk].view(B * T, Hkv, D)
-    dv = dkvq[nk:2 * nk].view(B * T, Hkv, D)
-    dq = dkvq[2 * nk:].view(B * T, Hq, D)
+    hout = torch.empty(2, B * T, Hq, D, dtype=wl.kv_dtype).pin_memory()
+    dkvq = [torch.empty(2 * nk + nq, dtype=wl.kv_dtype, device=dev) for _ in range(2)]
+    douts = [torch.empty(B * T, Hq, D, dtype=wl.kv_dtype, device=dev) for _ in range(2)]
     tok_e2e = 0
     for i in range(e2e_steps):
-        r = (a.warmup + a.steps + i) % R
+        r = (a.warmup + a.steps + n2 + i) % R
         for layer in range(NL):
             for b in range(B):
                 qn, n = lens[r][layer][b]
@@ -628,25 +699,57 @@ def run_kvq(a):
                 qn, n = qn + f * G, n + T - f * G
                 lens[r][layer][b] = [qn, n]
                 tok_e2e += T * (sinks + qn + n) - T * (T - 1) // 2
+    cstream = torch.cuda.Stream(device=dev)
+    drv = _Driver()
+    cs, ms_ = cstream.cuda_stream, stream.cuda_stream
+    ev_in = [drv.event() for _ in range(2)]    # inputs of the buffer landed
+    ev_used = [drv.event() for _ in range(2)]  # the step that read / wrote the buffer is done
+    ev_out = [drv.event() for _ in range(2)]   # its output copied to the host
+    ev_start = drv.event()
+    in_bytes = (2 * nk + nq) * 2
+    out_bytes = B * T * Hq * D * 2
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(stream)
+    rc = drv.record(ev_start, ms_) | drv.wait(cs, ev_start)
+
+    def upload(i):
+        j = i % 2
+        r_ = drv.wait(cs, ev_used[j]) if i >= 2 else 0
+        return r_ | drv.htod(dkvq[j].data_ptr(), hkvq[i % pool].data_ptr(), in_bytes, cs) | drv.record(ev_in[j], cs)
+
+    rc |= upload(0)
     for i in range(e2e_steps):
-        r = (a.warmup + a.steps + i) % R
-        dkvq.copy_(hkvq[i % pool], non_blocking=True)
-        o = out
+        j = i % 2
+        r = (a.warmup + a.steps + n2 + i) % R
+        if i + 1 < e2e_steps:
+            rc |= upload(i + 1)
+        rc |= drv.wait(ms_, ev_in[j])
+        if i >= 2:
+            rc |= drv.wait(ms_, ev_out[j])  # step i - 2's output has left douts[j]
+        dk = dkvq[j][:nk].view(B * T, Hkv, D)
+        dv = dkvq[j][nk:2 * nk].view(B * T, Hkv, D)
+        dq = dkvq[j][2 * nk:].view(B * T, Hq, D)
+        o = douts[j]
         for layer in range(NL):
             if T == 1:
-                caches[r].decode_step(layer, dk, dv, dq, out, softmax_scale=wl.softmax_scale, stream=stream)
+                caches[r].decode_step(layer, dk, dv, dq, douts[j], softmax_scale=wl.softmax_scale, stream=stream)
             else:
                 caches[r].append(layer, dk, dv, [T] * B, stream=stream)
                 o = caches[r].decode_attention_multi(layer, dq.view(B, T, Hq, D), out_dtype=wl.kv_dtype,
                                                      softmax_scale=wl.softmax_scale, stream=stream)
-        hout.copy_(o.view(B * T, Hq, D), non_blocking=True)
+                o.record_stream(cstream)  # allocated per call on `stream`, read by the copy stream
+        rc |= drv.record(ev_used[j], ms_) | drv.wait(cs, ev_used[j])
+        rc |= drv.dtoh(hout[j].data_ptr(), o.data_ptr(), out_bytes, cs) | drv.record(ev_out[j], cs)
+    stream.wait_stream(cstream)
     f1.record(stream)
     torch.cuda.synchronize()
+    if rc:
+        raise RuntimeError("a CUDA driver call of the end-to-end leg failed")
+    for e in ev_in + ev_used + ev_out + [ev_start]:
+        drv.destroy(e)
     e2e_ms, = cross_rank_max([f0.elapsed_time(f1)], world, dev)
     e2e_value = tok_e2e * world / (e2e_ms / 1e3)
 
@@ -659,14 +762,14 @@ def run_kvq(a):
                       "of their queries, causal among them (split-KV decode + combine per group of query tokens)")
         elif split_append:
             kernel = ("append (ring write; the quantize kernel when a ring fills), then the split-KV decode kernel "
-                      "and the log-sum-exp combine, per call")
+                      "and the log-sum-exp combine")
         elif fused:
             kernel = ("decode step: one token appended per sequence inside the tensor-core split-KV decode kernel, "
-                      "+ log-sum-exp combine, per call (a step in which rings are full first runs the flush kernel "
-                      "that quantizes their oldest G tokens)")
+                      "+ log-sum-exp combine (a step in which rings are full first runs the flush kernel that "
+                      "quantizes their oldest G tokens)")
         else:
             kernel = ("decode step: ring write (+ quantize when a ring fills), CUDA-core split-KV decode kernel and "
-                      "log-sum-exp combine, per call")
+                      "log-sum-exp combine")
         result = {
             "metric": METRIC,
             "value": value,
@@ -694,7 +797,11 @@ def run_kvq(a):
                 "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
                 "frac_of_8tbs_nominal": achieved_gbs / 8000.0,
                 "traffic": _committed_traffic(a.workload),
-                "step_call_us": dec_ms / a.steps * 1e3,
+                "timing": ("achieved = algorithmic bytes of the K timed steps / their device time (one event "
+                           "pair around the loop); step_call_us and the flush split come from a separate pass of "
+                           "up to 256 steps, each between its own events"),
+                "step_us": ms / a.steps * 1e3,
+                "step_call_us": call_us,
                 "flush_step_us": fl_us if fl else None,
                 "flush_steps": len(fl),
                 "nonflush_step_us": nf_us if nf else None,
@@ -708,13 +815,15 @@ def run_kvq(a):
             },
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": int((dk.numel() + dv.numel() + dq.numel()) * 2),
-                    "d2h_bytes_per_step": int(out.numel() * 2), "steps": e2e_steps},
+                    "d2h_bytes_per_step": int(out.numel() * 2), "steps": e2e_steps,
+                    "copies": "one pinned host-to-device and one device-to-host copy per step, on a copy stream "
+                              "overlapped with the previous and next steps"},
             "gpu_launches": launches,
             "clocks": clk,
         }
         if split_append:
             result["roofline"]["append_us_per_step"] = app_us
-            result["roofline"]["attention_us_per_step"] = dec_ms / a.steps * 1e3 - app_us
+            result["roofline"]["attention_us_per_step"] = call_us - app_us
         if prefill is not None:
             result["prefill_chunk"] = prefill
     del caches
