@@ -95,6 +95,23 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// The same copy with an L2 cache policy (createpolicy): block records are
+// read exactly once, so they are copied with an evict-first policy and do
+// not push out of L2 what is read again soon (the unit's ring rows
+// prefetched for its ring chunks, the split partials the combine reads).
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                              uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
 // L2 prefetch of a global range (16-byte multiple), no shared-memory target.
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
@@ -731,6 +748,7 @@ __device__ __forceinline__ void store_new_token(const DecodeParams& p, int b, in
 // item and the number of unit changes so far.
 struct IssueState {
   UnitCursor u;
+  uint64_t pol = evict_first_policy();  // L2 policy of the block-record copies
   int unit = -1;
   int qslot = -1;         // query buffer of the unit (round robin over the nstages buffers)
   int ring0 = 0;          // ring slot of the unit's first ring token
@@ -771,15 +789,15 @@ __device__ __forceinline__ void issue_item(const DecodeParams& p, const MmaPlan&
       rec = record_ptr(L, u.b, u.h, jb);
     }
     if (mp.lg_nt == 0) {
-      bulk_g2s(dst, rec, mp.tx_bytes, bar);
+      bulk_g2s_hint(dst, rec, mp.tx_bytes, bar, is.pol);
     } else {
       const uint8_t* tp = rec + L.tile0_off + (int64_t)jt * L.tile_bytes;
       if (L.rec_ksz_off >= 0) {  // the block's per-channel key scales, then the tile's codes and value scales
-        bulk_g2s(dst + mp.kc_bytes, rec + L.rec_ksz_off, kHeadDim * 4, bar);
-        bulk_g2s(dst, tp, mp.kc_bytes, bar);
-        bulk_g2s(dst + mp.vc_soff, tp + L.vc_off, L.tile_bytes - L.vc_off, bar);
+        bulk_g2s(dst + mp.kc_bytes, rec + L.rec_ksz_off, kHeadDim * 4, bar);  // read by both tiles
+        bulk_g2s_hint(dst, tp, mp.kc_bytes, bar, is.pol);
+        bulk_g2s_hint(dst + mp.vc_soff, tp + L.vc_off, L.tile_bytes - L.vc_off, bar, is.pol);
       } else {  // a tile part holds all it needs
-        bulk_g2s(dst, tp, L.tile_bytes, bar);
+        bulk_g2s_hint(dst, tp, L.tile_bytes, bar, is.pol);
       }
     }
     if (j == nb - 1 && p.nres[u.b] > 0) {
