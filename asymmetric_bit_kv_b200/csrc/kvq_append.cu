@@ -383,15 +383,17 @@ __device__ __forceinline__ void quantize_part(const LayerView& L, int b, int h, 
 
 cudaError_t opt_in_max_smem(const void* kernel, uint64_t& done_mask);
 
-// grid (max flush blocks * 2, batch, Hkv); block kQuantThreads; dynamic smem
-// quant_smem_bytes(..., 1). x = 2j + tensor: key block j of sequence b
-// covers positions q_old[b] + j*G .., value block j positions qv_old[b] +
-// j*G ..: ring tokens before the call's first new token, this call's input
-// after.
+// grid (max flush blocks * 2 * p.parts, batch, Hkv); block kQuantThreads;
+// dynamic smem quant_smem_bytes(..., p.parts). x = (2j + tensor) * parts +
+// part: key block j of sequence b covers positions q_old[b] + j*G .., value
+// block j positions qv_old[b] + j*G ..: ring tokens before the call's first
+// new token, this call's input after; part of parts: a slice of its
+// channels (per-channel keys) or tokens (otherwise).
 template <bool ROT>
 __global__ void __launch_bounds__(kQuantThreads, 6) quantize_blocks_kernel(AppendParams p) {
-  const int j = blockIdx.x >> 1, b = blockIdx.y, h = blockIdx.z;
-  const bool key = (blockIdx.x & 1) == 0;
+  const int part = blockIdx.x % p.parts, x = blockIdx.x / p.parts;
+  const int j = x >> 1, b = blockIdx.y, h = blockIdx.z;
+  const bool key = (x & 1) == 0;
   if (j >= (key ? p.flush[b] : p.flush_v[b])) return;
   extern __shared__ __align__(16) uint8_t smem_q[];
   const LayerView& L = p.L;
@@ -401,7 +403,7 @@ __global__ void __launch_bounds__(kQuantThreads, 6) quantize_blocks_kernel(Appen
   const BlockRows src{reinterpret_cast<const uint16_t*>(key ? L.ring_k : L.ring_v) + unit * R * kHeadDim,
                       reinterpret_cast<const uint16_t*>(key ? p.k_in : p.v_in), p.in_off[b],
                       (key ? p.q_old[b] : p.qv_old[b]) + j * G, p.len_old[b], R, L.num_kv_heads, h};
-  quantize_part<ROT>(L, b, h, key, 0, 1, (key ? p.q_old[b] : p.qv_old[b]) / G + j, src, smem_q);
+  quantize_part<ROT>(L, b, h, key, part, p.parts, (key ? p.q_old[b] : p.qv_old[b]) / G + j, src, smem_q);
 }
 
 // grid (batch * Hkv * (kStepKeyParts + kStepValueParts)); block
@@ -450,9 +452,9 @@ cudaError_t launch_step_flush(const FlushParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-// grid (batch, Hkv); copies this call's sink tokens to the sinks and its
-// tokens that stay exact into the key and value rings, and records the new
-// lengths.
+// grid (batch, Hkv, splits); copies this call's sink tokens to the sinks
+// and its tokens that stay exact into the key and value rings (CTA z a
+// slice of them), and records the new lengths.
 __global__ void ring_write_kernel(AppendParams p) {
   const int b = blockIdx.x, h = blockIdx.y;
   const LayerView& L = p.L;
@@ -465,7 +467,7 @@ __global__ void ring_write_kernel(AppendParams p) {
   const int ns = p.s_take[b];
   const int64_t unit = (int64_t)b * L.num_kv_heads + h;
   const int64_t sink_base = unit * KVQ_MAX_SINKS + p.s_old[b];
-  for (int idx = threadIdx.x; idx < ns * vec_per_tok; idx += blockDim.x) {
+  for (int idx = threadIdx.x; blockIdx.z == 0 && idx < ns * vec_per_tok; idx += blockDim.x) {
     const int i = idx / vec_per_tok, c = (idx % vec_per_tok) * 8;
     const int64_t row = (int64_t)p.in_off[b] - ns + i;
     const int64_t src = (row * L.num_kv_heads + h) * D + c;
@@ -479,12 +481,16 @@ __global__ void ring_write_kernel(AppendParams p) {
   // thread issues the loads of up to 4 chunks before their stores
   const int first_k = max(boundary, q_new), first_v = max(boundary, qv_new);
   const int first = min(first_k, first_v);
-  const int total = (end - first) * vec_per_tok;
+  // CTA z of gridDim.z takes its slice of the 16-byte chunks
+  const int all = (end - first) * vec_per_tok;
+  const int per = (all + gridDim.z - 1) / gridDim.z;
+  const int lo = blockIdx.z * per;
+  const int total = min(all, lo + per);
   const uint16_t* kin = reinterpret_cast<const uint16_t*>(p.k_in);
   const uint16_t* vin = reinterpret_cast<const uint16_t*>(p.v_in);
   uint16_t* rk = reinterpret_cast<uint16_t*>(L.ring_k);
   uint16_t* rv = reinterpret_cast<uint16_t*>(L.ring_v);
-  for (int base = threadIdx.x; base < total; base += 4 * blockDim.x) {
+  for (int base = lo + threadIdx.x; base < total; base += 4 * blockDim.x) {
     uint4 tk[4], tv[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -504,7 +510,7 @@ __global__ void ring_write_kernel(AppendParams p) {
       if (i >= first_v) *reinterpret_cast<uint4*>(rv + (unit * L.residual_v + i % L.residual_v) * D + c) = tv[u];
     }
   }
-  if (h == 0 && threadIdx.x == 0) {
+  if (h == 0 && blockIdx.z == 0 && threadIdx.x == 0) {
     int32_t* len = L.lens + (int64_t)b * kLensStride;
     len[kLenQ] = q_new;
     len[kLenN] = end - q_new;
@@ -575,27 +581,65 @@ cudaError_t opt_in_max_smem(const void* kernel, uint64_t& done_mask) {
   return e;
 }
 
-cudaError_t launch_quantize(const AppendParams& p, int max_flush, cudaStream_t stream) {
+// Streaming multiprocessors of the current device (0 if unknown).
+int device_sm_count() {
+  static int memo[64];  // per device, +1 (0: not queried yet)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  if (dev < 64 && memo[dev] > 0) return memo[dev] - 1;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  if (dev < 64) memo[dev] = n + 1;
+  return n;
+}
+
+cudaError_t launch_quantize(AppendParams& p, int max_flush, cudaStream_t stream) {
   const LayerView& L = p.L;
   const bool rot = L.hadamard != 0;
-  const int smem = quant_smem_bytes(L.group_k, L.k_bits, L.group_v, L.k_axis, rot, 1);
+  // A call that quantizes few blocks (a decode step's flush, a prefill
+  // chunk) splits each block and tensor into up to 4 parts -- channel slices
+  // for per-channel keys, token slices otherwise -- until the grid fills two
+  // waves of the kernel's 6 CTAs per SM; a CTA's time is its own latency
+  // (staging, then quantizing), so smaller parts finish sooner.
+  const int64_t ctas = 2LL * max_flush * p.batch * L.num_kv_heads;
+  const int64_t target = 12LL * std::max(1, device_sm_count());
+  // A part keeps at least 32 tokens or channels (a 32-token block split into
+  // 8-token slices measured slower than whole); per-token key slices then
+  // also hold whole code words (32 / k_bits tokens each).
+  const int most_parts = std::max(1, std::min(4, L.group_k / 32));
+  p.parts = 1;
+  while (p.parts < most_parts && ctas * p.parts < target) p.parts *= 2;
+  const int smem = quant_smem_bytes(L.group_k, L.k_bits, L.group_v, L.k_axis, rot, p.parts);
   static uint64_t done_rot = 0, done_raw = 0;
   cudaError_t e = rot ? opt_in_max_smem(reinterpret_cast<const void*>(quantize_blocks_kernel<true>), done_rot)
                       : opt_in_max_smem(reinterpret_cast<const void*>(quantize_blocks_kernel<false>), done_raw);
   if (e != cudaSuccess) return e;
-  dim3 grid(2 * max_flush, p.batch, L.num_kv_heads);
+  dim3 grid(2 * max_flush * p.parts, p.batch, L.num_kv_heads);
   if (rot) quantize_blocks_kernel<true><<<grid, kQuantThreads, smem, stream>>>(p);
   else quantize_blocks_kernel<false><<<grid, kQuantThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_append(const AppendParams& p, int max_flush, cudaStream_t stream) {
+cudaError_t launch_append(AppendParams& p, int max_flush, cudaStream_t stream) {
   const LayerView& L = p.L;
   if (max_flush > 0) {
     cudaError_t e = launch_quantize(p, max_flush, stream);
     if (e != cudaSuccess) return e;
   }
-  dim3 grid2(p.batch, L.num_kv_heads);
+  // one CTA per (sequence, KV head), or up to 4 splitting the tokens that
+  // stay exact when a call leaves many (a prefill: up to R per sequence), so
+  // that each thread has one round of loads
+  int most = 0;
+  for (int b = 0; b < p.batch; ++b) most = std::max(most, std::min(p.t_new[b], std::max(L.residual, L.residual_v)));
+  const int chunks = most * (kHeadDim / 8);
+  const int splits = std::max(1, std::min(4, (chunks + 4 * 256 - 1) / (4 * 256)));
+  dim3 grid2(p.batch, L.num_kv_heads, splits);
   ring_write_kernel<<<grid2, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }

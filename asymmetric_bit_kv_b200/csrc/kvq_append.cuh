@@ -16,6 +16,7 @@ struct AppendParams {
   const void* k_in;  // [sum t_new][Hkv][D], kv dtype
   const void* v_in;
   int32_t batch;
+  int32_t parts;                   // CTAs per block and tensor of the quantize kernel (set by launch_append)
   int32_t q_old[KVQ_MAX_BATCH];    // quantized keys before the call
   int32_t qv_old[KVQ_MAX_BATCH];   // quantized values before the call
   int32_t len_old[KVQ_MAX_BATCH];  // tokens before the call (quantized keys + key ring)
@@ -29,7 +30,8 @@ struct AppendParams {
 
 // Enqueues the quantize kernel (max_flush = the largest key or value block
 // count of any sequence; none if 0) and the ring / sink / length-table write.
-cudaError_t launch_append(const AppendParams& p, int max_flush, cudaStream_t stream);
+// p.parts is chosen here.
+cudaError_t launch_append(AppendParams& p, int max_flush, cudaStream_t stream);
 
 // Paged caches: page-table entries set by one launch (table[idx[i]] =
 // page[i]), enqueued before the append kernels that write the new pages.
