@@ -27,9 +27,53 @@ namespace kvq {
 
 namespace {
 
-__device__ __forceinline__ float bits_to_float(uint32_t v, int dtype) {
-  if (dtype == KVQ_BF16) return __uint_as_float(v << 16);
-  return __half2float(__ushort_as_half((unsigned short)v));
+// fp32 value (exact) of a 16-bit storage word of kv dtype DT, and of the low
+// and high element of a packed pair of them.
+template <int DT>
+__device__ __forceinline__ float f32_of(uint32_t v) {
+  if constexpr (DT == KVQ_BF16) return __uint_as_float(v << 16);
+  else return __half2float(__ushort_as_half((unsigned short)v));
+}
+template <int DT>
+__device__ __forceinline__ float f32_lo(uint32_t p) {
+  return f32_of<DT>(p & 0xffffu);
+}
+template <int DT>
+__device__ __forceinline__ float f32_hi(uint32_t p) {
+  if constexpr (DT == KVQ_BF16) return __uint_as_float(p & 0xffff0000u);
+  else return __half2float(__ushort_as_half((unsigned short)(p >> 16)));
+}
+
+// Elementwise min / max of two packed pairs of kv-dtype values. Min and max
+// are exact in any format, so these equal the fp32 min / max of the
+// conversions (up to the sign of a zero, on which no group parameter
+// depends: the zero point is min + 0, the scale a difference); one
+// instruction per two values.
+template <int DT>
+__device__ __forceinline__ uint32_t pair_min(uint32_t a, uint32_t b) {
+  uint32_t r;
+  if constexpr (DT == KVQ_BF16) {
+    const __nv_bfloat162 v = __hmin2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                                     *reinterpret_cast<const __nv_bfloat162*>(&b));
+    r = *reinterpret_cast<const uint32_t*>(&v);
+  } else {
+    const __half2 v = __hmin2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+    r = *reinterpret_cast<const uint32_t*>(&v);
+  }
+  return r;
+}
+template <int DT>
+__device__ __forceinline__ uint32_t pair_max(uint32_t a, uint32_t b) {
+  uint32_t r;
+  if constexpr (DT == KVQ_BF16) {
+    const __nv_bfloat162 v = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                                     *reinterpret_cast<const __nv_bfloat162*>(&b));
+    r = *reinterpret_cast<const uint32_t*>(&v);
+  } else {
+    const __half2 v = __hmax2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+    r = *reinterpret_cast<const uint32_t*>(&v);
+  }
+  return r;
 }
 
 // Where row t (0 <= t < G) of a block comes from: the ring (positions before
@@ -101,38 +145,59 @@ __host__ __device__ inline int quant_smem_bytes(int G, int kb, int gv, int k_axi
 }
 
 // Stages rows t0 .. t0+nt-1, channels c0 .. c0+nc-1 of a block as raw
-// 16-bit values ([nt][nc]) with 16-byte loads, two per thread in flight at
-// a time.
+// 16-bit values ([nt][nc]) with 16-byte loads. A row has nc/8 chunks (a
+// power of two, at most 16, dividing kQuantThreads): each thread keeps one
+// chunk column and walks the rows kQuantThreads/(nc/8) apart, four loads in
+// flight before their stores (no division per chunk).
 __device__ __forceinline__ void stage_raw(const BlockRows& src, int t0, int nt, int c0, int nc, uint16_t* dst) {
-  const int cpr = nc / 8;  // 16-byte chunks per staged row
-  const int n = nt * cpr;
-  for (int idx = threadIdx.x; idx < n; idx += 2 * kQuantThreads) {
-    const int i2 = idx + kQuantThreads;
-    const uint4 a = *reinterpret_cast<const uint4*>(src.row(t0 + idx / cpr) + c0 + (idx % cpr) * 8);
-    uint4 b2;
-    if (i2 < n) b2 = *reinterpret_cast<const uint4*>(src.row(t0 + i2 / cpr) + c0 + (i2 % cpr) * 8);
-    *reinterpret_cast<uint4*>(dst + (idx / cpr) * nc + (idx % cpr) * 8) = a;
-    if (i2 < n) *reinterpret_cast<uint4*>(dst + (i2 / cpr) * nc + (i2 % cpr) * 8) = b2;
+  const int lg = __ffs(nc >> 3) - 1;  // log2 of the chunks per row
+  const int col = (threadIdx.x & ((1 << lg) - 1)) * 8;
+  const int rstep = kQuantThreads >> lg;
+  for (int r = threadIdx.x >> lg; r < nt; r += 4 * rstep) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (r + u * rstep < nt) v[u] = *reinterpret_cast<const uint4*>(src.row(t0 + r + u * rstep) + c0 + col);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (r + u * rstep < nt) *reinterpret_cast<uint4*>(dst + (r + u * rstep) * nc + col) = v[u];
   }
 }
 
 // Stages rows t0 .. t0+nt-1 rotated (x . H, rotate_lane) as fp32 [nt][D]:
 // one warp per row.
-__device__ __forceinline__ void stage_rotated(const BlockRows& src, int t0, int nt, int dt, float* dst) {
+template <int DT>
+__device__ __forceinline__ void stage_rotated(const BlockRows& src, int t0, int nt, float* dst) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int t = warp; t < nt; t += kQuantThreads / 32) {
     const uint2 raw = *reinterpret_cast<const uint2*>(src.row(t0 + t) + 4 * lane);
-    float x[4] = {bits_to_float(raw.x & 0xffffu, dt), bits_to_float(raw.x >> 16, dt),
-                  bits_to_float(raw.y & 0xffffu, dt), bits_to_float(raw.y >> 16, dt)};
+    float x[4] = {f32_lo<DT>(raw.x), f32_hi<DT>(raw.x), f32_lo<DT>(raw.y), f32_hi<DT>(raw.y)};
     rotate_lane(x, lane);
     *reinterpret_cast<float4*>(dst + t * kHeadDim + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
   }
 }
 
+// Raw packed pairs of channels c .. c+N-1 (N >= 4) of staged 16-bit row t
+// (rows of `pitch` channels): N/2 words, 16-byte (N = 4: 8-byte) loads.
+template <int N>
+__device__ __forceinline__ void row_pairs(const uint8_t* rows, int pitch, int t, int c, uint32_t (&p)[N / 2]) {
+  const uint16_t* r = reinterpret_cast<const uint16_t*>(rows) + t * pitch + c;
+  if constexpr (N >= 8) {
+#pragma unroll
+    for (int i = 0; i < N / 8; ++i) {
+      const uint4 q = reinterpret_cast<const uint4*>(r)[i];
+      p[4 * i] = q.x, p[4 * i + 1] = q.y, p[4 * i + 2] = q.z, p[4 * i + 3] = q.w;
+    }
+  } else {
+    const uint2 q = *reinterpret_cast<const uint2*>(r);
+    p[0] = q.x, p[1] = q.y;
+  }
+}
+
 // Values x[0..N) of channels c .. c+N-1 of staged row t (rows of `pitch`
-// channels).
-template <bool ROT, int N>
-__device__ __forceinline__ void row_values(const uint8_t* rows, int pitch, int t, int c, int dt, float (&x)[N]) {
+// channels): fp32 rows when rotated, raw kv-dtype rows otherwise.
+template <bool ROT, int DT, int N>
+__device__ __forceinline__ void row_values(const uint8_t* rows, int pitch, int t, int c, float (&x)[N]) {
   if constexpr (ROT) {
     const float4* f = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(rows) + t * pitch + c);
 #pragma unroll
@@ -141,31 +206,18 @@ __device__ __forceinline__ void row_values(const uint8_t* rows, int pitch, int t
       x[4 * i] = q.x, x[4 * i + 1] = q.y, x[4 * i + 2] = q.z, x[4 * i + 3] = q.w;
     }
   } else {
-    const uint16_t* r = reinterpret_cast<const uint16_t*>(rows) + t * pitch + c;
-    if constexpr (N >= 8) {
+    uint32_t p[N / 2];
+    row_pairs<N>(rows, pitch, t, c, p);
 #pragma unroll
-      for (int i = 0; i < N / 8; ++i) {
-        const uint4 q = reinterpret_cast<const uint4*>(r)[i];
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          x[8 * i + 2 * e] = bits_to_float(w[e] & 0xffffu, dt);
-          x[8 * i + 2 * e + 1] = bits_to_float(w[e] >> 16, dt);
-        }
-      }
-    } else {
-      const uint2 q = *reinterpret_cast<const uint2*>(r);
-      x[0] = bits_to_float(q.x & 0xffffu, dt), x[1] = bits_to_float(q.x >> 16, dt);
-      x[2] = bits_to_float(q.y & 0xffffu, dt), x[3] = bits_to_float(q.y >> 16, dt);
-    }
+    for (int i = 0; i < N / 2; ++i) x[2 * i] = f32_lo<DT>(p[i]), x[2 * i + 1] = f32_hi<DT>(p[i]);
   }
 }
 
 // One staged value: row t, column c (rows of `pitch` channels).
-template <bool ROT>
-__device__ __forceinline__ float staged(const uint8_t* rows, int pitch, int t, int c, int dt) {
+template <bool ROT, int DT>
+__device__ __forceinline__ float staged(const uint8_t* rows, int pitch, int t, int c) {
   if constexpr (ROT) return reinterpret_cast<const float*>(rows)[t * pitch + c];
-  return bits_to_float(reinterpret_cast<const uint16_t*>(rows)[t * pitch + c], dt);
+  else return f32_of<DT>(reinterpret_cast<const uint16_t*>(rows)[t * pitch + c]);
 }
 
 // Word index of word w of channel d in a record's key code array (the
@@ -196,29 +248,54 @@ __device__ __forceinline__ RecOut rec_out(const LayerView& L, uint8_t* rec) {
 // codes: one thread per output word (PER = 32/BITS channels); the gv/PER
 // threads of a group combine their min/max with xor shuffles. put_word(t, w,
 // word) and put_sz(t, g, params) receive the results (t: token of the block).
-template <bool ROT, int BITS, bool CODES, class PutWord, class PutSz>
-__device__ __forceinline__ void quantize_token_groups(const uint8_t* rows, int t0, int nt, int gv, int dt,
-                                                      PutWord put_word, PutSz put_sz) {
+// Raw rows take their min/max on packed pairs and convert to fp32 only for
+// the codes.
+template <bool ROT, int DT, int BITS, bool CODES, class PutWord, class PutSz>
+__device__ __forceinline__ void quantize_token_groups(const uint8_t* rows, int t0, int nt, int gv, PutWord put_word,
+                                                      PutSz put_sz) {
   constexpr int PER = 32 / BITS;
   constexpr int WPT = kHeadDim / PER;  // words per row
   const int P = gv / PER;              // threads per group: a power of two, <= 32, dividing WPT
+  const int lgP = __ffs(P) - 1;
   for (int item = threadIdx.x; item < nt * WPT; item += kQuantThreads) {
     const int t = item / WPT, w = item % WPT;
-    float x[PER];
-    row_values<ROT, PER>(rows, kHeadDim, t, w * PER, dt, x);
-    float mn = x[0], mx = x[0];
+    float x[PER];        // rotated rows: the values
+    uint32_t pr[PER / 2];  // raw rows: the packed pairs
+    float mn, mx;
+    if constexpr (ROT) {
+      row_values<true, DT, PER>(rows, kHeadDim, t, w * PER, x);
+      mn = x[0], mx = x[0];
 #pragma unroll
-    for (int i = 1; i < PER; ++i) {
-      mn = fminf(mn, x[i]);
-      mx = fmaxf(mx, x[i]);
+      for (int i = 1; i < PER; ++i) {
+        mn = fminf(mn, x[i]);
+        mx = fmaxf(mx, x[i]);
+      }
+    } else {
+      row_pairs<PER>(rows, kHeadDim, t, w * PER, pr);
+      uint32_t lo = pr[0], hi = pr[0];
+#pragma unroll
+      for (int i = 1; i < PER / 2; ++i) {
+        lo = pair_min<DT>(lo, pr[i]);
+        hi = pair_max<DT>(hi, pr[i]);
+      }
+      mn = fminf(f32_lo<DT>(lo), f32_hi<DT>(lo));
+      mx = fmaxf(f32_lo<DT>(hi), f32_hi<DT>(hi));
     }
     for (int o = P / 2; o >= 1; o >>= 1) {
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
     const GroupParams gp = group_params(mn, mx, BITS);
-    if constexpr (CODES) put_word(t0 + t, w, quant_word_rcp<BITS, PER>(x, gp.m, gp.d, __frcp_rn(gp.d)));
-    if ((w % P) == 0) put_sz(t0 + t, w / P, gp);
+    if constexpr (CODES) {
+      const float r = __frcp_rn(gp.d);
+      uint32_t word;
+      if constexpr (ROT) word = quant_word_rcp<BITS, PER>(x, gp.m, gp.d, r);
+      else
+        word = quant_word_rcp_fn<BITS, PER>(
+            [&](int i) { return (i & 1) ? f32_hi<DT>(pr[i >> 1]) : f32_lo<DT>(pr[i >> 1]); }, gp.m, gp.d, r);
+      put_word(t0 + t, w, word);
+    }
+    if ((w & (P - 1)) == 0) put_sz(t0 + t, w >> lgP, gp);
   }
 }
 
@@ -226,17 +303,18 @@ __device__ __forceinline__ void quantize_token_groups(const uint8_t* rows, int t
 // and token words [w0, w0 + nw): thread item (channel d, word w) packs
 // tokens w*PER .. w*PER+PER-1 of channel d (staged row of token t at t - t0,
 // column d - sc0) with the fp32 (scale, zero, 1/scale) par(t, d).
-template <bool ROT, int KB, bool PT, class Par>
+template <bool ROT, int DT, int KB, bool PT, class Par>
 __device__ __forceinline__ void pack_key_codes(const uint8_t* rows, int pitch, int t0, int sc0, int c0, int nc, int w0,
-                                               int nw, int dt, const RecOut& ro, Par par) {
+                                               int nw, const RecOut& ro, Par par) {
   constexpr int LGPER = KB == 2 ? 4 : KB == 4 ? 3 : 2;  // log2 of the tokens per word
   const int lgWt = ro.lgT - LGPER;                        // log2 of the words per channel per tile
   constexpr int PER = 32 / KB;
+  const int lgnc = __ffs(nc) - 1;  // nc: a power of two
   for (int item = threadIdx.x; item < nc * nw; item += kQuantThreads) {
-    const int d = c0 + item % nc, w = w0 + item / nc;
+    const int d = c0 + (item & (nc - 1)), w = w0 + (item >> lgnc);
     float x[PER];
 #pragma unroll
-    for (int i = 0; i < PER; ++i) x[i] = staged<ROT>(rows, pitch, w * PER + i - t0, d - sc0, dt);
+    for (int i = 0; i < PER; ++i) x[i] = staged<ROT, DT>(rows, pitch, w * PER + i - t0, d - sc0);
     uint32_t word;
     if constexpr (PT) {  // per-token keys: each token has its own (scale, zero)
       word = 0;
@@ -256,24 +334,48 @@ __device__ __forceinline__ void pack_key_codes(const uint8_t* rows, int pitch, i
 }
 
 // Keys per channel (KIVI): channels [c0, c0 + nc) over all G tokens; the
-// min/max of every (channel, word-slice) item, combined through shared
-// memory, then the codes.
-template <bool ROT, int KB>
-__device__ __forceinline__ void quantize_key_channels(const uint8_t* rows, const PartShape& s, int G, int dt,
-                                                      const RecOut& ro, float2* red, float4* kpar) {
+// min/max of every (channels, token word) item, combined through shared
+// memory, then the codes (one channel and token word per thread item). Raw
+// rows hold exactly the part's channels (sc0 = c0, snc = nc): a min/max
+// item is a channel pair, one 32-bit word per staged row, reduced on packed
+// pairs. Rotated rows (fp32, all channels staged) take one channel per
+// item.
+template <bool ROT, int DT, int KB>
+__device__ __forceinline__ void quantize_key_channels(const uint8_t* rows, const PartShape& s, int G, const RecOut& ro,
+                                                      float2* red, float4* kpar) {
   constexpr int PER = 32 / KB;
+  constexpr int LGPER = KB == 2 ? 4 : KB == 4 ? 3 : 2;  // log2 of the tokens per word
   const int W = G / PER;
-  for (int item = threadIdx.x; item < s.nc * W; item += kQuantThreads) {
-    const int dl = item % s.nc, w = item / s.nc;
-    const int col = s.c0 + dl - s.sc0;
-    float mn = staged<ROT>(rows, s.snc, w * PER, col, dt), mx = mn;
+  const int np = s.nc / 2;  // channel pairs (raw rows: 32-bit words per staged row)
+  const int lgnc = __ffs(s.nc) - 1, lgnp = lgnc - 1;  // nc: a power of two
+  const uint32_t* r32 = reinterpret_cast<const uint32_t*>(rows);
+  if constexpr (ROT) {
+    for (int item = threadIdx.x; item < s.nc * W; item += kQuantThreads) {
+      const int dl = item & (s.nc - 1), w = item >> lgnc;
+      const int col = s.c0 + dl - s.sc0;
+      float mn = staged<ROT, DT>(rows, s.snc, w * PER, col), mx = mn;
 #pragma unroll 4
-    for (int i = 1; i < PER; ++i) {
-      const float x = staged<ROT>(rows, s.snc, w * PER + i, col, dt);
-      mn = fminf(mn, x);
-      mx = fmaxf(mx, x);
+      for (int i = 1; i < PER; ++i) {
+        const float x = staged<ROT, DT>(rows, s.snc, w * PER + i, col);
+        mn = fminf(mn, x);
+        mx = fmaxf(mx, x);
+      }
+      red[w * s.nc + dl] = make_float2(mn, mx);
     }
-    red[w * s.nc + dl] = make_float2(mn, mx);
+  } else {
+    for (int item = threadIdx.x; item < np * W; item += kQuantThreads) {
+      const int cp = item & (np - 1), w = item >> lgnp;
+      const uint32_t* col = r32 + w * PER * np + cp;
+      uint32_t lo = col[0], hi = lo;
+#pragma unroll
+      for (int i = 1; i < PER; ++i) {
+        const uint32_t v = col[i * np];
+        lo = pair_min<DT>(lo, v);
+        hi = pair_max<DT>(hi, v);
+      }
+      red[w * s.nc + 2 * cp] = make_float2(f32_lo<DT>(lo), f32_lo<DT>(hi));
+      red[w * s.nc + 2 * cp + 1] = make_float2(f32_hi<DT>(lo), f32_hi<DT>(hi));
+    }
   }
   __syncthreads();
   __half2* ksz = reinterpret_cast<__half2*>(ro.rec_ksz >= 0 ? ro.rec + ro.rec_ksz : ro.rec + ro.tile0 + ro.ksz_off);
@@ -289,38 +391,38 @@ __device__ __forceinline__ void quantize_key_channels(const uint8_t* rows, const
     kpar[dl] = make_float4(gp.d, gp.m, __frcp_rn(gp.d), 0.f);
   }
   __syncthreads();
-  pack_key_codes<ROT, KB, false>(rows, s.snc, 0, s.sc0, s.c0, s.nc, 0, W, dt, ro,
-                                 [&](int, int d) { return kpar[d - s.c0]; });
+  pack_key_codes<ROT, DT, KB, false>(rows, s.snc, 0, s.sc0, s.c0, s.nc, 0, W, ro,
+                                     [&](int, int d) { return kpar[d - s.c0]; });
 }
 
 // Keys per token over group_v channels (BQ2_0), tokens [t0, t0 + nt): the
 // token groups' scales and zero points, then the codes of those tokens
 // packed along the token axis.
-template <bool ROT, int KB>
-__device__ __forceinline__ void quantize_key_tokens(const uint8_t* rows, const PartShape& s, int dt, const RecOut& ro,
-                                                    int gv, float4* kpar) {
+template <bool ROT, int DT, int KB>
+__device__ __forceinline__ void quantize_key_tokens(const uint8_t* rows, const PartShape& s, const RecOut& ro, int gv,
+                                                    float4* kpar) {
   constexpr int PER = 32 / KB;
   const int ng = kHeadDim / gv;
-  quantize_token_groups<ROT, KB, false>(rows, s.t0, s.nt, gv, dt, [](int, int, uint32_t) {},
-                                        [&](int t, int g, const GroupParams& gp) {
-                                          reinterpret_cast<__half2*>(ro.tile(t) + ro.ksz_off)[ro.local(t) * ng + g] =
-                                              __halves2half2(gp.d16, gp.m16);
-                                          kpar[(t - s.t0) * ng + g] = make_float4(gp.d, gp.m, __frcp_rn(gp.d), 0.f);
-                                        });
+  quantize_token_groups<ROT, DT, KB, false>(rows, s.t0, s.nt, gv, [](int, int, uint32_t) {},
+                                            [&](int t, int g, const GroupParams& gp) {
+                                              reinterpret_cast<__half2*>(ro.tile(t) + ro.ksz_off)[ro.local(t) * ng + g] =
+                                                  __halves2half2(gp.d16, gp.m16);
+                                              kpar[(t - s.t0) * ng + g] = make_float4(gp.d, gp.m, __frcp_rn(gp.d), 0.f);
+                                            });
   __syncthreads();
-  pack_key_codes<ROT, KB, true>(rows, kHeadDim, s.t0, 0, 0, kHeadDim, s.t0 / PER, s.nt / PER, dt, ro,
-                                [&](int t, int d) { return kpar[(t - s.t0) * ng + d / gv]; });
+  pack_key_codes<ROT, DT, KB, true>(rows, kHeadDim, s.t0, 0, 0, kHeadDim, s.t0 / PER, s.nt / PER, ro,
+                                    [&](int t, int d) { return kpar[(t - s.t0) * ng + d / gv]; });
 }
 
 // Values per token over group_v channels (KIVI), tokens [t0, t0 + nt),
 // codes packed along head_dim.
-template <bool ROT, int KB, int VB>
-__device__ __forceinline__ void quantize_value_tokens(const uint8_t* rows, const PartShape& s, int dt, const RecOut& ro,
+template <bool ROT, int DT, int KB, int VB>
+__device__ __forceinline__ void quantize_value_tokens(const uint8_t* rows, const PartShape& s, const RecOut& ro,
                                                       int gv) {
   const int ng = kHeadDim / gv, T = 1 << ro.lgT;
   constexpr int VW = kHeadDim * VB / 32;
-  quantize_token_groups<ROT, VB, true>(
-      rows, s.t0, s.nt, gv, dt,
+  quantize_token_groups<ROT, DT, VB, true>(
+      rows, s.t0, s.nt, gv,
       [&](int t, int w, uint32_t word) {
         reinterpret_cast<uint32_t*>(ro.tile(t) + ro.vc_off)[vc_word_index(ro.local(t), w, T, KB, VW)] = word;
       },
@@ -335,48 +437,55 @@ __device__ __forceinline__ void quantize_value_tokens(const uint8_t* rows, const
 // (record jv). ROT: the rows are multiplied by the normalized Sylvester
 // Hadamard matrix first (rotate_lane: radix-2 butterflies of half-width 1,
 // 2, 4, ..., then one fp32 multiply by fp32(1/sqrt(D)); "KV1-1.2B" card,
-// BQ2_0).
-template <bool ROT, int KB>
+// BQ2_0). DT: the kv dtype of the rows.
+template <bool ROT, int DT, int KB>
 __device__ __forceinline__ void quantize_key_part(const LayerView& L, int b, int h, int64_t jk, const BlockRows& src,
                                                   const PartShape& s, uint8_t* smem) {
-  const int G = L.group_k, dt = L.kv_dtype;
+  const int G = L.group_k;
   const QuantSmem sm = part_smem(s, G, KB, L.group_v, L.k_axis, ROT);
-  if constexpr (ROT) stage_rotated(src, s.t0, s.nt, dt, reinterpret_cast<float*>(smem));
+  if constexpr (ROT) stage_rotated<DT>(src, s.t0, s.nt, reinterpret_cast<float*>(smem));
   else stage_raw(src, s.t0, s.nt, s.sc0, s.snc, reinterpret_cast<uint16_t*>(smem));
   __syncthreads();
   const RecOut ro = rec_out(L, record_ptr(L, b, h, jk));
   float4* kpar = reinterpret_cast<float4*>(smem + sm.rows + sm.red);
-  if (L.k_axis == 0) quantize_key_channels<ROT, KB>(smem, s, G, dt, ro, reinterpret_cast<float2*>(smem + sm.rows), kpar);
-  else quantize_key_tokens<ROT, KB>(smem, s, dt, ro, L.group_v, kpar);
+  if (L.k_axis == 0) quantize_key_channels<ROT, DT, KB>(smem, s, G, ro, reinterpret_cast<float2*>(smem + sm.rows), kpar);
+  else quantize_key_tokens<ROT, DT, KB>(smem, s, ro, L.group_v, kpar);
 }
 
-template <bool ROT, int KB, int VB>
+template <bool ROT, int DT, int KB, int VB>
 __device__ __forceinline__ void quantize_value_part(const LayerView& L, int b, int h, int64_t jv, const BlockRows& src,
                                                     const PartShape& s, uint8_t* smem) {
-  const int dt = L.kv_dtype;
-  if constexpr (ROT) stage_rotated(src, s.t0, s.nt, dt, reinterpret_cast<float*>(smem));
+  if constexpr (ROT) stage_rotated<DT>(src, s.t0, s.nt, reinterpret_cast<float*>(smem));
   else stage_raw(src, s.t0, s.nt, 0, kHeadDim, reinterpret_cast<uint16_t*>(smem));
   __syncthreads();
-  quantize_value_tokens<ROT, KB, VB>(smem, s, dt, rec_out(L, record_ptr(L, b, h, jv)), L.group_v);
+  quantize_value_tokens<ROT, DT, KB, VB>(smem, s, rec_out(L, record_ptr(L, b, h, jv)), L.group_v);
+}
+
+template <bool ROT, int DT>
+__device__ __forceinline__ void quantize_part_dt(const LayerView& L, int b, int h, bool key, const PartShape& s,
+                                                 int64_t j, const BlockRows& src, uint8_t* smem) {
+  if (key) {
+    if (L.k_bits == 2) quantize_key_part<ROT, DT, 2>(L, b, h, j, src, s, smem);
+    else if (L.k_bits == 4) quantize_key_part<ROT, DT, 4>(L, b, h, j, src, s, smem);
+    else quantize_key_part<ROT, DT, 8>(L, b, h, j, src, s, smem);
+    return;
+  }
+#define KVQ_VPART(K, V) \
+  if (L.k_bits == K && L.v_bits == V) return quantize_value_part<ROT, DT, K, V>(L, b, h, j, src, s, smem);
+  KVQ_VPART(2, 2) KVQ_VPART(2, 4) KVQ_VPART(2, 8) KVQ_VPART(4, 2) KVQ_VPART(4, 4) KVQ_VPART(4, 8)
+  KVQ_VPART(8, 2) KVQ_VPART(8, 4) KVQ_VPART(8, 8)
+#undef KVQ_VPART
 }
 
 // Part `part` of `parts` of the key block jk (key) or the value block jv of
 // (sequence b, KV head h), rows from src.
-template <bool ROT>
+// (The kernels are instantiated per kv dtype: one kernel holding both
+// dtypes' paths needed more than the 42 registers of 6 CTAs per SM.)
+template <bool ROT, int DT>
 __device__ __forceinline__ void quantize_part(const LayerView& L, int b, int h, bool key, int part, int parts,
                                               int64_t j, const BlockRows& src, uint8_t* smem) {
   const PartShape s = part_shape(key, part, parts, L.group_k, L.k_axis, ROT);
-  if (key) {
-    if (L.k_bits == 2) quantize_key_part<ROT, 2>(L, b, h, j, src, s, smem);
-    else if (L.k_bits == 4) quantize_key_part<ROT, 4>(L, b, h, j, src, s, smem);
-    else quantize_key_part<ROT, 8>(L, b, h, j, src, s, smem);
-    return;
-  }
-#define KVQ_VPART(K, V) \
-  if (L.k_bits == K && L.v_bits == V) return quantize_value_part<ROT, K, V>(L, b, h, j, src, s, smem);
-  KVQ_VPART(2, 2) KVQ_VPART(2, 4) KVQ_VPART(2, 8) KVQ_VPART(4, 2) KVQ_VPART(4, 4) KVQ_VPART(4, 8)
-  KVQ_VPART(8, 2) KVQ_VPART(8, 4) KVQ_VPART(8, 8)
-#undef KVQ_VPART
+  quantize_part_dt<ROT, DT>(L, b, h, key, s, j, src, smem);
 }
 
 }  // namespace
@@ -389,7 +498,7 @@ cudaError_t opt_in_max_smem(const void* kernel, uint64_t& done_mask);
 // block j positions qv_old[b] + j*G ..: ring tokens before the call's first
 // new token, this call's input after; part of parts: a slice of its
 // channels (per-channel keys) or tokens (otherwise).
-template <bool ROT>
+template <bool ROT, int DT>
 __global__ void __launch_bounds__(kQuantThreads, 6) quantize_blocks_kernel(AppendParams p) {
   const int part = blockIdx.x % p.parts, x = blockIdx.x / p.parts;
   const int j = x >> 1, b = blockIdx.y, h = blockIdx.z;
@@ -403,7 +512,7 @@ __global__ void __launch_bounds__(kQuantThreads, 6) quantize_blocks_kernel(Appen
   const BlockRows src{reinterpret_cast<const uint16_t*>(key ? L.ring_k : L.ring_v) + unit * R * kHeadDim,
                       reinterpret_cast<const uint16_t*>(key ? p.k_in : p.v_in), p.in_off[b],
                       (key ? p.q_old[b] : p.qv_old[b]) + j * G, p.len_old[b], R, L.num_kv_heads, h};
-  quantize_part<ROT>(L, b, h, key, part, p.parts, (key ? p.q_old[b] : p.qv_old[b]) / G + j, src, smem_q);
+  quantize_part<ROT, DT>(L, b, h, key, part, p.parts, (key ? p.q_old[b] : p.qv_old[b]) / G + j, src, smem_q);
 }
 
 // grid (batch * Hkv * (kStepKeyParts + kStepValueParts)); block
@@ -414,7 +523,7 @@ __global__ void __launch_bounds__(kQuantThreads, 6) quantize_blocks_kernel(Appen
 // decode launch that follows is its programmatic dependent and waits for it
 // (griddepcontrol.wait) before reading records; the decode kernel records
 // the new lengths.
-template <bool ROT>
+template <bool ROT, int DT>
 __global__ void __launch_bounds__(kQuantThreads, 6) step_flush_kernel(FlushParams p) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ __align__(16) uint8_t smem_q[];
@@ -431,7 +540,26 @@ __global__ void __launch_bounds__(kQuantThreads, 6) step_flush_kernel(FlushParam
   const int64_t unit = (int64_t)b * L.num_kv_heads + h;
   const BlockRows src{reinterpret_cast<const uint16_t*>(key ? L.ring_k : L.ring_v) + unit * L.residual * kHeadDim,
                       nullptr, 0, q, q + n, L.residual, L.num_kv_heads, h};
-  quantize_part<ROT>(L, b, h, key, part, key ? kStepKeyParts : kStepValueParts, q / L.group_k, src, smem_q);
+  quantize_part<ROT, DT>(L, b, h, key, part, key ? kStepKeyParts : kStepValueParts, q / L.group_k, src, smem_q);
+}
+
+// One instance of each quantize kernel per (rotation, kv dtype); the
+// shared-memory opt-in is recorded per instance and device.
+template <bool ROT, int DT>
+cudaError_t launch_flush_t(const FlushParams& p, int grid, int smem, cudaStream_t stream) {
+  static uint64_t done = 0;
+  const cudaError_t e = opt_in_max_smem(reinterpret_cast<const void*>(step_flush_kernel<ROT, DT>), done);
+  if (e != cudaSuccess) return e;
+  step_flush_kernel<ROT, DT><<<grid, kQuantThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+template <bool ROT, int DT>
+cudaError_t launch_quant_t(const AppendParams& p, dim3 grid, int smem, cudaStream_t stream) {
+  static uint64_t done = 0;
+  const cudaError_t e = opt_in_max_smem(reinterpret_cast<const void*>(quantize_blocks_kernel<ROT, DT>), done);
+  if (e != cudaSuccess) return e;
+  quantize_blocks_kernel<ROT, DT><<<grid, kQuantThreads, smem, stream>>>(p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_step_flush(const FlushParams& p, cudaStream_t stream) {
@@ -442,14 +570,10 @@ cudaError_t launch_step_flush(const FlushParams& p, cudaStream_t stream) {
                 rot).total,
       part_smem(part_shape(false, 0, kStepValueParts, L.group_k, L.k_axis, rot), L.group_k, L.k_bits, L.group_v,
                 L.k_axis, rot).total);
-  static uint64_t done_rot = 0, done_raw = 0;
-  cudaError_t e = rot ? opt_in_max_smem(reinterpret_cast<const void*>(step_flush_kernel<true>), done_rot)
-                      : opt_in_max_smem(reinterpret_cast<const void*>(step_flush_kernel<false>), done_raw);
-  if (e != cudaSuccess) return e;
   const int grid = p.ctas * (kStepKeyParts + kStepValueParts);
-  if (rot) step_flush_kernel<true><<<grid, kQuantThreads, smem, stream>>>(p);
-  else step_flush_kernel<false><<<grid, kQuantThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  const bool bf = L.kv_dtype == KVQ_BF16;
+  if (rot) return bf ? launch_flush_t<true, KVQ_BF16>(p, grid, smem, stream) : launch_flush_t<true, KVQ_F16>(p, grid, smem, stream);
+  return bf ? launch_flush_t<false, KVQ_BF16>(p, grid, smem, stream) : launch_flush_t<false, KVQ_F16>(p, grid, smem, stream);
 }
 
 // grid (batch, Hkv, splits); copies this call's sink tokens to the sinks
@@ -616,14 +740,10 @@ cudaError_t launch_quantize(AppendParams& p, int max_flush, cudaStream_t stream)
   p.parts = 1;
   while (p.parts < most_parts && ctas * p.parts < target) p.parts *= 2;
   const int smem = quant_smem_bytes(L.group_k, L.k_bits, L.group_v, L.k_axis, rot, p.parts);
-  static uint64_t done_rot = 0, done_raw = 0;
-  cudaError_t e = rot ? opt_in_max_smem(reinterpret_cast<const void*>(quantize_blocks_kernel<true>), done_rot)
-                      : opt_in_max_smem(reinterpret_cast<const void*>(quantize_blocks_kernel<false>), done_raw);
-  if (e != cudaSuccess) return e;
   dim3 grid(2 * max_flush * p.parts, p.batch, L.num_kv_heads);
-  if (rot) quantize_blocks_kernel<true><<<grid, kQuantThreads, smem, stream>>>(p);
-  else quantize_blocks_kernel<false><<<grid, kQuantThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  const bool bf = L.kv_dtype == KVQ_BF16;
+  if (rot) return bf ? launch_quant_t<true, KVQ_BF16>(p, grid, smem, stream) : launch_quant_t<true, KVQ_F16>(p, grid, smem, stream);
+  return bf ? launch_quant_t<false, KVQ_BF16>(p, grid, smem, stream) : launch_quant_t<false, KVQ_F16>(p, grid, smem, stream);
 }
 
 cudaError_t launch_append(AppendParams& p, int max_flush, cudaStream_t stream) {

@@ -273,31 +273,49 @@ __device__ __forceinline__ uint32_t quant_code_rcp(float x, float m, float d, fl
 // threshold, (qmax + 0.5) * 2^-21 >= |t| * 2^-21, serve every value: if any
 // value of the word falls within it of a half-integer, the whole word is
 // recomputed from the exact quotients.
+//
+// Packing: the bit pattern of tm is that of 1.5 * 2^23 (0x4B400000) plus the
+// code, so the word is the sum of the patterns, each shifted to its field
+// (one shift-add per code), minus the sum of the constant's shifted copies,
+// all modulo 2^32.
 template <int BITS, int N>
-__device__ __forceinline__ uint32_t quant_word_rcp(const float (&x)[N], float m, float d, float r) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+__host__ __device__ constexpr uint32_t round_bias() {
+  uint32_t s = 0;
+  for (int i = 0; i < N; ++i) s += 0x4B400000u << (i * BITS);
+  return s;
+}
+// x(i) gives value i of the word (an fp32 conversion of a staged value,
+// evaluated where it is used, so only the raw values stay in registers).
+template <int BITS, int N, class X>
+__device__ __forceinline__ uint32_t quant_word_rcp_fn(X x, float m, float d, float r) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23, bit pattern 0x4B400000
   constexpr int qmax = (1 << BITS) - 1;
   constexpr float lo = -0.49f, hi = (float)qmax + 0.49f;
   constexpr float near = 0.5f - ((float)qmax + 0.5f) * 0x1p-21f;  // |e| above this: within the window
-  uint32_t word = 0;
-  bool close = false;
+  uint32_t acc = 0;
+  float emax = 0.0f;  // the largest |e| of the word
 #pragma unroll
   for (int i = 0; i < N; ++i) {
-    const float t = fminf(fmaxf(__fmul_rn(__fsub_rn(x[i], m), r), lo), hi);
+    const float t = fminf(fmaxf(__fmul_rn(__fsub_rn(x(i), m), r), lo), hi);
     const float tm = __fadd_rn(t, kRound);
     const float e = __fsub_rn(t, __fsub_rn(tm, kRound));
-    close = close || fabsf(e) > near;
-    word |= (uint32_t)(__float_as_int(tm) - __float_as_int(kRound)) << (i * BITS);
+    emax = fmaxf(emax, fabsf(e));
+    acc += __float_as_uint(tm) << (i * BITS);
   }
-  if (close) {
+  uint32_t word = acc - round_bias<BITS, N>();
+  if (emax > near) {
     word = 0;
 #pragma unroll
     for (int i = 0; i < N; ++i) {
-      const float q = fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(x[i], m), d)), 0.0f), (float)qmax);  // ties to even
+      const float q = fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(x(i), m), d)), 0.0f), (float)qmax);  // ties to even
       word |= (uint32_t)q << (i * BITS);
     }
   }
   return word;
+}
+template <int BITS, int N>
+__device__ __forceinline__ uint32_t quant_word_rcp(const float (&x)[N], float m, float d, float r) {
+  return quant_word_rcp_fn<BITS, N>([&](int i) { return x[i]; }, m, d, r);
 }
 
 // x_hat = q * d + m with two roundings (no fused multiply-add).
