@@ -31,6 +31,7 @@ struct kvq_cache {
   int64_t uslots_off;             // int32 [max_batch][num_kv_heads] slots per unit (decode -> combine)
   int32_t slots;                  // partial slots per (sequence, query head)
   int32_t sm_count;
+  uint64_t launches = 0;          // kernels enqueued by calls on this cache (kvq_cache_kernel_launches)
   // host mirror [num_layers][max_batch]: quantized keys, key ring tokens,
   // sinks, quantized values (the value ring holds q_len + n_len - qv_len)
   std::vector<int32_t> q_len, n_len, s_len, qv_len;
@@ -284,11 +285,15 @@ kvq_status take_pages(kvq_cache* c, int layer, const int32_t* blocks_after, int 
       ++held[b];
       if (++u->n == kvq::kMaxPageUpdates) {
         e = kvq::launch_page_table_update(*u, stream);
+        if (e == cudaSuccess) ++c->launches;
         u->n = 0;
       }
     }
   }
-  if (e == cudaSuccess) e = kvq::launch_page_table_update(*u, stream);
+  if (e == cudaSuccess && u->n > 0) {
+    e = kvq::launch_page_table_update(*u, stream);
+    if (e == cudaSuccess) ++c->launches;
+  }
   delete u;
   if (e != cudaSuccess) return cuda_fail(e, "page-table update");
   return KVQ_OK;
@@ -356,6 +361,7 @@ kvq_status enqueue_append(kvq_cache* c, int layer, const void* k, const void* v,
   }
   cudaError_t e = kvq::launch_append(*p, max_flush, stream);
   if (e == cudaSuccess) {
+    c->launches += max_flush > 0 ? 2 : 1;  // the quantize kernel on a flush, the ring write
     for (int b = 0; b < batch; ++b) {
       const int qn = p->q_old[b] + p->flush[b] * G;
       const int end = p->len_old[b] + p->t_new[b];
@@ -534,6 +540,7 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const 
     plan_cta_starts(p, batch, cfg.num_kv_heads, (int64_t)std::max(1, c->sm_count) * per_sm, slot_cap);
     e = kvq::launch_decode_mma(p, mp, st);
     if (e == cudaSuccess) e = kvq::launch_combine(p, st);
+    if (e == cudaSuccess) c->launches += 2;  // the decode kernel and the combine
   } else {
     // Split plan (host mirror): blocks per split chosen to minimise (waves
     // of CTAs) x (blocks per CTA + a fixed per-CTA overhead), with at most
@@ -566,6 +573,7 @@ kvq_status enqueue_decode(kvq_cache* c, int32_t layer, const void* new_k, const 
     const int nsplits = (int)((max_blk + bps - 1) / bps);
     p.slots = slot_cap;
     e = kvq::launch_decode(p, nsplits, st);
+    if (e == cudaSuccess) c->launches += 2;  // the split kernel and the combine
   }
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return KVQ_OK;
@@ -885,6 +893,7 @@ kvq_status kvq_decode_step(kvq_cache* c, int32_t layer, const void* k, const voi
     fp.ctas = batch * cfg.num_kv_heads;
     const cudaError_t e = kvq::launch_step_flush(fp, st);
     if (e != cudaSuccess) s = cuda_fail(e, "flush launch");
+    else ++c->launches;
   }
   if (s == KVQ_OK)
     s = kvq::enqueue_decode(c, layer, k, v, q, out, out_dtype, softmax_scale, batch, stream, nullptr, nullptr, flush);
@@ -915,6 +924,7 @@ kvq_status kvq_dequant(kvq_cache* c, int32_t layer, int32_t seq, int32_t t0, int
   cudaError_t e = kvq::launch_dequant(layer_view(c, layer), seq, c->s_len[i], t0, t1, k_out, v_out,
                                       static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "dequant launch");
+  ++c->launches;
   return KVQ_OK;
 }
 
@@ -926,6 +936,13 @@ kvq_status kvq_device_errors(kvq_cache* c, int32_t* flags) {
   if (e == cudaSuccess && v != 0) e = cudaMemset(c->arena + c->err_off, 0, 4);
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
   *flags = v;
+  return KVQ_OK;
+}
+
+kvq_status kvq_cache_kernel_launches(const kvq_cache* c, uint64_t* count) {
+  g_last_error.clear();
+  if (!c || !count) return fail(KVQ_ERR_INVALID_ARG, "cache or count is null");
+  *count = c->launches;
   return KVQ_OK;
 }
 

@@ -344,7 +344,6 @@ template <bool ROT, int DT, int KB>
 __device__ __forceinline__ void quantize_key_channels(const uint8_t* rows, const PartShape& s, int G, const RecOut& ro,
                                                       float2* red, float4* kpar) {
   constexpr int PER = 32 / KB;
-  constexpr int LGPER = KB == 2 ? 4 : KB == 4 ? 3 : 2;  // log2 of the tokens per word
   const int W = G / PER;
   const int np = s.nc / 2;  // channel pairs (raw rows: 32-bit words per staged row)
   const int lgnc = __ffs(s.nc) - 1, lgnp = lgnc - 1;  // nc: a power of two

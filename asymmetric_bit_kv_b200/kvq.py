@@ -108,6 +108,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "kvq_dequant": (I32, [P, I32, I32, I32, I32, P, P, P]),
         "kvq_get_layout": (I32, [P, I32, ctypes.POINTER(kvq_layout)]),
         "kvq_device_errors": (I32, [P, ctypes.POINTER(I32)]),
+        "kvq_cache_kernel_launches": (I32, [P, ctypes.POINTER(ctypes.c_uint64)]),
         "kvq_seq_lengths": (I32, [P, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32)]),
         "kvq_seq_sinks": (I32, [P, I32, I32, ctypes.POINTER(I32)]),
         "kvq_seq_value_lengths": (I32, [P, I32, I32, ctypes.POINTER(I32), ctypes.POINTER(I32)]),
@@ -315,6 +316,12 @@ class KVCache:
         f = ctypes.c_int32()
         _check(self.lib.kvq_device_errors(self.handle, ctypes.byref(f)), "kvq_device_errors")
         return f.value
+
+    def kernel_launches(self) -> int:
+        """Kernels enqueued so far by calls on this cache (kvq_cache_kernel_launches)."""
+        n = ctypes.c_uint64()
+        _check(self.lib.kvq_cache_kernel_launches(self.handle, ctypes.byref(n)), "kvq_cache_kernel_launches")
+        return n.value
 
     def layout(self, layer: int) -> kvq_layout:
         lay = kvq_layout()

@@ -468,7 +468,6 @@ def run_kvq(a):
     # launch (kvq_decode_step); the library says which kernel a layer runs
     kernels = [caches[0].decode_kernel(layer) for layer in range(NL)]
     fused = all(kn != "cuda_core" for kn in kernels)
-    max_rows = 2 if "tensor_core_pair" in kernels else 8  # query rows per KV head one decode pass takes
 
     # The device-timed loop calls the C entry points with arguments prepared
     # here, so that Python overhead per call stays far below the GPU time of a
@@ -533,53 +532,34 @@ def run_kvq(a):
         dist.barrier()
 
     # Per-step accounting, computed before the timed loop so that the loop only
-    # enqueues work: the (quantized, ring, pages) state of every replica follows
+    # enqueues work: the (quantized, ring) state of every replica follows
     # the flush rule (a token that finds a full ring first moves G ring tokens
     # into the quantized cache), checked against the library's host mirror after.
     lens = [[[list(caches[r].lengths(layer, b)) for b in range(B)] for layer in range(NL)] for r in range(R)]
-    pages = [[[-(-(q // G) // a.page_blocks) if a.page_blocks else 0 for q, _ in row] for row in rep] for rep in lens]
-    groups, t0, ngr = 0, 0, Hq // Hkv  # decode passes of a multi-token step (<= 8 query rows per KV head each)
-    while t0 < T:
-        tp = 1
-        while 2 * tp * ngr <= max_rows and t0 + 2 * tp <= T:
-            tp *= 2
-        groups, t0 = groups + 1, t0 + tp
 
     def make_plan(first, nsteps):
-        """(replica, launches, algorithmic bytes, KV tokens attended, any
-        flush) of steps first .. first + nsteps - 1, advancing lens/pages."""
+        """(replica, algorithmic bytes, KV tokens attended, any flush) of
+        steps first .. first + nsteps - 1, advancing lens."""
         plan = []
         for i in range(first, first + nsteps):
             r = i % R
-            ab = tk = launches = 0
+            ab = tk = 0
             flush = False
             for layer in range(NL):
                 ab += T * (2 * B * Hq * D * 2 + 2 * (2 * B * Hkv * D * 2))  # q in, out; new k, v in and into the ring
                 ab += B * sinks * Hkv * D * 2 * 2  # the exact sink tokens
                 tk += B * T * sinks
-                lflush = new_pages = False
+                lflush = False
                 for b in range(B):
                     qn, n = lens[r][layer][b]
                     f = _flushes(n, T, Rw, G)
                     lflush = lflush or f > 0
                     qn, n = qn + f * G, n + T - f * G
                     lens[r][layer][b] = [qn, n]
-                    if a.page_blocks:
-                        pg = -(-(qn // G) // a.page_blocks)
-                        new_pages = new_pages or pg > pages[r][layer][b]
-                        pages[r][layer][b] = pg
                     ab += qn * bytes_tok[layer] + n * Hkv * D * 2 * 2
                     tk += T * (qn + n) - T * (T - 1) // 2  # query t sees the tokens up to its own position
                 flush = flush or lflush
-                if T == 1 and fused and not split_append:
-                    # flush kernel on a flushing step, page-table update when pages
-                    # are taken, decode, combine
-                    launches += 2 + (1 if lflush else 0) + (1 if new_pages else 0)
-                else:
-                    # append (page-table update, quantize on a flush, ring write),
-                    # then decode + combine per pass
-                    launches += 1 + (1 if lflush else 0) + (1 if new_pages else 0) + 2 * groups
-            plan.append((r, launches, ab, tk, flush))
+            plan.append((r, ab, tk, flush))
         return plan
 
     def check_mirror():
@@ -589,9 +569,8 @@ def run_kvq(a):
                     assert tuple(lens[r][layer][b]) == caches[r].lengths(layer, b), "step accounting out of sync"
 
     plan = make_plan(a.warmup, a.steps)
-    launches = sum(x[1] for x in plan)
-    alg_total = float(sum(x[2] for x in plan))
-    tok_total = sum(x[3] for x in plan)
+    alg_total = float(sum(x[1] for x in plan))
+    tok_total = sum(x[2] for x in plan)
 
     # The timed loop: exactly K steps between one pair of events (no event
     # inside, so that nothing but the steps runs on the stream).
@@ -599,6 +578,8 @@ def run_kvq(a):
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # kernels the timed steps enqueue, as the library counts them
+    launches0 = sum(c.kernel_launches() for c in caches)
     h0 = time.perf_counter()
     e0.record(stream)
     # host cost of enqueueing a step: the first nburst steps, about 64 library
@@ -614,6 +595,7 @@ def run_kvq(a):
             burst_lib_s = lib_s[0]
     e1.record(stream)
     host_s = time.perf_counter() - h0
+    launches = sum(c.kernel_launches() for c in caches) - launches0
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -633,8 +615,8 @@ def run_kvq(a):
     check_mirror()
     call_ms = [x[0].elapsed_time(x[2]) for x in events]
     app_ms = [x[0].elapsed_time(x[1]) for x in events] if split_append else [0.0]
-    fl = [m for m, x in zip(call_ms, plan2) if x[4]]
-    nf = [m for m, x in zip(call_ms, plan2) if not x[4]]
+    fl = [m for m, x in zip(call_ms, plan2) if x[3]]
+    nf = [m for m, x in zip(call_ms, plan2) if not x[3]]
     call_us = 1e3 * sum(call_ms) / len(call_ms)
     fl_us = 1e3 * sum(fl) / len(fl) if fl else 0.0
     nf_us = 1e3 * sum(nf) / len(nf) if nf else 0.0

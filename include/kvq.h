@@ -348,6 +348,16 @@ KVQ_API kvq_status kvq_dequant(kvq_cache* cache, int32_t layer, int32_t seq, int
  * this library.                                                           */
 KVQ_API kvq_status kvq_device_errors(kvq_cache* cache, int32_t* flags);
 
+/* Kernels enqueued so far by the calls on this cache, counted on the host
+ * when each call enqueues them: one per launch, whatever the kernel (append:
+ * ring write, plus the quantize kernel when a ring flushes, plus a page-table
+ * update when pages are taken; decode: the decode kernel and the combine
+ * kernel; a fused step's flush kernel on a step whose rings are full;
+ * dequant). For accounting, e.g. a benchmark that reads it
+ * around a timed region. No counterpart on the pages.
+ * - cache, count: non-null (else KVQ_ERR_INVALID_ARG). Host only.          */
+KVQ_API kvq_status kvq_cache_kernel_launches(const kvq_cache* cache, uint64_t* count);
+
 /* Layer layout (see kvq_layout): where the packed codes, scales and zero
  * points of the KV1-1.2B card's format (Quantization Format) and the
  * KIVI README's full-precision window live. For tests and tools that read

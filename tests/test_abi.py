@@ -90,6 +90,9 @@ def test_create_rejects_bad_arena_on_host():
     assert lib.kvq_cache_create(ctypes.byref(c), 0x1000000, n - 1, ctypes.byref(h)) == K.KVQ_ERR_WORKSPACE
     assert b"required" in lib.kvq_last_error()
     assert lib.kvq_append(None, 0, None, None, None, 0, None) == K.KVQ_ERR_INVALID_ARG
+    count = ctypes.c_uint64(7)
+    assert lib.kvq_cache_kernel_launches(None, ctypes.byref(count)) == K.KVQ_ERR_INVALID_ARG
+    assert count.value == 7
     assert lib.kvq_decode_attention(None, 0, None, None, 0, 1.0, 1, None) == K.KVQ_ERR_INVALID_ARG
 
 
