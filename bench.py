@@ -815,6 +815,12 @@ def run_kvq(a):
     return result
 
 
+# Sources a decode launch's DRAM traffic depends on: the decode kernels, the
+# record layout, the plan and launch code; not the quantize kernels
+# (kvq_append.*) nor the static-scratch entry point (kvq_noalloc.cu).
+_NOT_DECODE = ("kvq_append.cu", "kvq_append.cuh", "kvq_noalloc.cu")
+
+
 def _kernel_source_hash():
     import glob
     import hashlib
@@ -822,6 +828,8 @@ def _kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "asymmetric_bit_kv_b200", "csrc")
     for f in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
+        if os.path.basename(f) in _NOT_DECODE:
+            continue
         h.update(os.path.basename(f).encode())
         with open(f, "rb") as fh:
             h.update(fh.read())
