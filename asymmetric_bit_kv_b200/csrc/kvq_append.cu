@@ -460,31 +460,18 @@ __device__ __forceinline__ void quantize_value_part(const LayerView& L, int b, i
   quantize_value_tokens<ROT, DT, KB, VB>(smem, s, rec_out(L, record_ptr(L, b, h, jv)), L.group_v);
 }
 
-template <bool ROT, int DT>
-__device__ __forceinline__ void quantize_part_dt(const LayerView& L, int b, int h, bool key, const PartShape& s,
-                                                 int64_t j, const BlockRows& src, uint8_t* smem) {
-  if (key) {
-    if (L.k_bits == 2) quantize_key_part<ROT, DT, 2>(L, b, h, j, src, s, smem);
-    else if (L.k_bits == 4) quantize_key_part<ROT, DT, 4>(L, b, h, j, src, s, smem);
-    else quantize_key_part<ROT, DT, 8>(L, b, h, j, src, s, smem);
-    return;
-  }
-#define KVQ_VPART(K, V) \
-  if (L.k_bits == K && L.v_bits == V) return quantize_value_part<ROT, DT, K, V>(L, b, h, j, src, s, smem);
-  KVQ_VPART(2, 2) KVQ_VPART(2, 4) KVQ_VPART(2, 8) KVQ_VPART(4, 2) KVQ_VPART(4, 4) KVQ_VPART(4, 8)
-  KVQ_VPART(8, 2) KVQ_VPART(8, 4) KVQ_VPART(8, 8)
-#undef KVQ_VPART
-}
-
 // Part `part` of `parts` of the key block jk (key) or the value block jv of
-// (sequence b, KV head h), rows from src.
-// (The kernels are instantiated per kv dtype: one kernel holding both
-// dtypes' paths needed more than the 42 registers of 6 CTAs per SM.)
-template <bool ROT, int DT>
+// (sequence b, KV head h), rows from src. The kernels are instantiated per
+// rotation, kv dtype and bit widths: one kernel holding both dtypes' paths
+// needed more than the 42 registers of 6 CTAs per SM, and one holding every
+// bit-width pair spent its short flush launches waiting for instruction
+// fetch.
+template <bool ROT, int DT, int KB, int VB>
 __device__ __forceinline__ void quantize_part(const LayerView& L, int b, int h, bool key, int part, int parts,
                                               int64_t j, const BlockRows& src, uint8_t* smem) {
   const PartShape s = part_shape(key, part, parts, L.group_k, L.k_axis, ROT);
-  quantize_part_dt<ROT, DT>(L, b, h, key, s, j, src, smem);
+  if (key) quantize_key_part<ROT, DT, KB>(L, b, h, j, src, s, smem);
+  else quantize_value_part<ROT, DT, KB, VB>(L, b, h, j, src, s, smem);
 }
 
 }  // namespace
@@ -497,7 +484,7 @@ cudaError_t opt_in_max_smem(const void* kernel, uint64_t& done_mask);
 // block j positions qv_old[b] + j*G ..: ring tokens before the call's first
 // new token, this call's input after; part of parts: a slice of its
 // channels (per-channel keys) or tokens (otherwise).
-template <bool ROT, int DT>
+template <bool ROT, int DT, int KB, int VB>
 __global__ void __launch_bounds__(kQuantThreads, 6) quantize_blocks_kernel(AppendParams p) {
   const int part = blockIdx.x % p.parts, x = blockIdx.x / p.parts;
   const int j = x >> 1, b = blockIdx.y, h = blockIdx.z;
@@ -511,7 +498,8 @@ __global__ void __launch_bounds__(kQuantThreads, 6) quantize_blocks_kernel(Appen
   const BlockRows src{reinterpret_cast<const uint16_t*>(key ? L.ring_k : L.ring_v) + unit * R * kHeadDim,
                       reinterpret_cast<const uint16_t*>(key ? p.k_in : p.v_in), p.in_off[b],
                       (key ? p.q_old[b] : p.qv_old[b]) + j * G, p.len_old[b], R, L.num_kv_heads, h};
-  quantize_part<ROT, DT>(L, b, h, key, part, p.parts, (key ? p.q_old[b] : p.qv_old[b]) / G + j, src, smem_q);
+  quantize_part<ROT, DT, KB, VB>(L, b, h, key, part, p.parts, (key ? p.q_old[b] : p.qv_old[b]) / G + j, src,
+                                 smem_q);
 }
 
 // grid (batch * Hkv * (kStepKeyParts + kStepValueParts)); block
@@ -522,7 +510,7 @@ __global__ void __launch_bounds__(kQuantThreads, 6) quantize_blocks_kernel(Appen
 // decode launch that follows is its programmatic dependent and waits for it
 // (griddepcontrol.wait) before reading records; the decode kernel records
 // the new lengths.
-template <bool ROT, int DT>
+template <bool ROT, int DT, int KB, int VB>
 __global__ void __launch_bounds__(kQuantThreads, 6) step_flush_kernel(FlushParams p) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ __align__(16) uint8_t smem_q[];
@@ -539,27 +527,52 @@ __global__ void __launch_bounds__(kQuantThreads, 6) step_flush_kernel(FlushParam
   const int64_t unit = (int64_t)b * L.num_kv_heads + h;
   const BlockRows src{reinterpret_cast<const uint16_t*>(key ? L.ring_k : L.ring_v) + unit * L.residual * kHeadDim,
                       nullptr, 0, q, q + n, L.residual, L.num_kv_heads, h};
-  quantize_part<ROT, DT>(L, b, h, key, part, key ? kStepKeyParts : kStepValueParts, q / L.group_k, src, smem_q);
+  quantize_part<ROT, DT, KB, VB>(L, b, h, key, part, key ? kStepKeyParts : kStepValueParts, q / L.group_k, src,
+                                 smem_q);
 }
 
-// One instance of each quantize kernel per (rotation, kv dtype); the
-// shared-memory opt-in is recorded per instance and device.
-template <bool ROT, int DT>
+// One instance of each quantize kernel per (rotation, kv dtype, key bits,
+// value bits), chosen on the host; the shared-memory opt-in is recorded per
+// instance and device.
+template <bool ROT, int DT, int KB, int VB>
 cudaError_t launch_flush_t(const FlushParams& p, int grid, int smem, cudaStream_t stream) {
   static uint64_t done = 0;
-  const cudaError_t e = opt_in_max_smem(reinterpret_cast<const void*>(step_flush_kernel<ROT, DT>), done);
+  const cudaError_t e = opt_in_max_smem(reinterpret_cast<const void*>(step_flush_kernel<ROT, DT, KB, VB>), done);
   if (e != cudaSuccess) return e;
-  step_flush_kernel<ROT, DT><<<grid, kQuantThreads, smem, stream>>>(p);
+  step_flush_kernel<ROT, DT, KB, VB><<<grid, kQuantThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
-template <bool ROT, int DT>
+template <bool ROT, int DT, int KB, int VB>
 cudaError_t launch_quant_t(const AppendParams& p, dim3 grid, int smem, cudaStream_t stream) {
   static uint64_t done = 0;
-  const cudaError_t e = opt_in_max_smem(reinterpret_cast<const void*>(quantize_blocks_kernel<ROT, DT>), done);
+  const cudaError_t e = opt_in_max_smem(reinterpret_cast<const void*>(quantize_blocks_kernel<ROT, DT, KB, VB>), done);
   if (e != cudaSuccess) return e;
-  quantize_blocks_kernel<ROT, DT><<<grid, kQuantThreads, smem, stream>>>(p);
+  quantize_blocks_kernel<ROT, DT, KB, VB><<<grid, kQuantThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
+// Returns FN<rotation, dtype, key bits, value bits>(P, GRID, SMEM, STREAM)
+// for the layer of P (FN: launch_flush_t or launch_quant_t).
+#define KVQ_QUANT_DISPATCH(FN, P, GRID, SMEM, STREAM)                                           \
+  do {                                                                                          \
+    const LayerView& L_ = (P).L;                                                                \
+    const bool rot_ = L_.hadamard != 0, bf_ = L_.kv_dtype == KVQ_BF16;                          \
+    const int kb_ = L_.k_bits, vb_ = L_.v_bits;                                                 \
+    KVQ_QUANT_BITS(FN, true, KVQ_BF16, rot_ && bf_, P, GRID, SMEM, STREAM)                      \
+    KVQ_QUANT_BITS(FN, true, KVQ_F16, rot_ && !bf_, P, GRID, SMEM, STREAM)                      \
+    KVQ_QUANT_BITS(FN, false, KVQ_BF16, !rot_ && bf_, P, GRID, SMEM, STREAM)                    \
+    KVQ_QUANT_BITS(FN, false, KVQ_F16, !rot_ && !bf_, P, GRID, SMEM, STREAM)                    \
+    return cudaErrorInvalidValue;                                                               \
+  } while (0)
+#define KVQ_QUANT_ONE(FN, R, D, K, V, P, GRID, SMEM, STREAM) \
+  if (kb_ == K && vb_ == V) return FN<R, D, K, V>(P, GRID, SMEM, STREAM);
+#define KVQ_QUANT_BITS(FN, R, D, COND, P, GRID, SMEM, STREAM)                                                    \
+  if (COND) {                                                                                                    \
+    KVQ_QUANT_ONE(FN, R, D, 2, 2, P, GRID, SMEM, STREAM) KVQ_QUANT_ONE(FN, R, D, 2, 4, P, GRID, SMEM, STREAM)     \
+    KVQ_QUANT_ONE(FN, R, D, 2, 8, P, GRID, SMEM, STREAM) KVQ_QUANT_ONE(FN, R, D, 4, 2, P, GRID, SMEM, STREAM)     \
+    KVQ_QUANT_ONE(FN, R, D, 4, 4, P, GRID, SMEM, STREAM) KVQ_QUANT_ONE(FN, R, D, 4, 8, P, GRID, SMEM, STREAM)     \
+    KVQ_QUANT_ONE(FN, R, D, 8, 2, P, GRID, SMEM, STREAM) KVQ_QUANT_ONE(FN, R, D, 8, 4, P, GRID, SMEM, STREAM)     \
+    KVQ_QUANT_ONE(FN, R, D, 8, 8, P, GRID, SMEM, STREAM)                                                         \
+  }
 
 cudaError_t launch_step_flush(const FlushParams& p, cudaStream_t stream) {
   const LayerView& L = p.L;
@@ -570,9 +583,7 @@ cudaError_t launch_step_flush(const FlushParams& p, cudaStream_t stream) {
       part_smem(part_shape(false, 0, kStepValueParts, L.group_k, L.k_axis, rot), L.group_k, L.k_bits, L.group_v,
                 L.k_axis, rot).total);
   const int grid = p.ctas * (kStepKeyParts + kStepValueParts);
-  const bool bf = L.kv_dtype == KVQ_BF16;
-  if (rot) return bf ? launch_flush_t<true, KVQ_BF16>(p, grid, smem, stream) : launch_flush_t<true, KVQ_F16>(p, grid, smem, stream);
-  return bf ? launch_flush_t<false, KVQ_BF16>(p, grid, smem, stream) : launch_flush_t<false, KVQ_F16>(p, grid, smem, stream);
+  KVQ_QUANT_DISPATCH(launch_flush_t, p, grid, smem, stream);
 }
 
 // grid (batch, Hkv, splits); copies this call's sink tokens to the sinks
@@ -740,9 +751,7 @@ cudaError_t launch_quantize(AppendParams& p, int max_flush, cudaStream_t stream)
   while (p.parts < most_parts && ctas * p.parts < target) p.parts *= 2;
   const int smem = quant_smem_bytes(L.group_k, L.k_bits, L.group_v, L.k_axis, rot, p.parts);
   dim3 grid(2 * max_flush * p.parts, p.batch, L.num_kv_heads);
-  const bool bf = L.kv_dtype == KVQ_BF16;
-  if (rot) return bf ? launch_quant_t<true, KVQ_BF16>(p, grid, smem, stream) : launch_quant_t<true, KVQ_F16>(p, grid, smem, stream);
-  return bf ? launch_quant_t<false, KVQ_BF16>(p, grid, smem, stream) : launch_quant_t<false, KVQ_F16>(p, grid, smem, stream);
+  KVQ_QUANT_DISPATCH(launch_quant_t, p, grid, smem, stream);
 }
 
 cudaError_t launch_append(AppendParams& p, int max_flush, cudaStream_t stream) {
