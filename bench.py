@@ -800,7 +800,7 @@ def run_kvq(a):
                     "d2h_bytes_per_step": int(out.numel() * 2), "steps": e2e_steps,
                     "copies": "one pinned host-to-device and one device-to-host copy per step, on a copy stream "
                               "overlapped with the previous and next steps"},
-            "gpu_launches": launches,
+            "gpu_launches": launches * world,  # every rank runs the same steps: the whole job's kernels
             "clocks": clk,
         }
         if split_append:
