@@ -753,6 +753,9 @@ cudaError_t launch_quantize(AppendParams& p, int max_flush, cudaStream_t stream)
   dim3 grid(2 * max_flush * p.parts, p.batch, L.num_kv_heads);
   KVQ_QUANT_DISPATCH(launch_quant_t, p, grid, smem, stream);
 }
+#undef KVQ_QUANT_DISPATCH
+#undef KVQ_QUANT_BITS
+#undef KVQ_QUANT_ONE
 
 cudaError_t launch_append(AppendParams& p, int max_flush, cudaStream_t stream) {
   const LayerView& L = p.L;
