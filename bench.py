@@ -693,6 +693,9 @@ def run_kvq(a):
     ev_start = drv.event()
     in_bytes = (2 * nk + nq) * 2
     out_bytes = B * T * Hq * D * 2
+    # k, v and q views of each input buffer, made once
+    views = [(x[:nk].view(B * T, Hkv, D), x[nk:2 * nk].view(B * T, Hkv, D), x[2 * nk:].view(B * T, Hq, D),
+              x[2 * nk:].view(B, T, Hq, D)) for x in dkvq]
 
     def e2e_run(first, n):
         """Steps first .. first + n - 1 of the e2e sequence, copies included;
@@ -714,16 +717,14 @@ def run_kvq(a):
             rc |= drv.wait(ms_, ev_in[j])
             if i >= 2:
                 rc |= drv.wait(ms_, ev_out[j])  # step i - 2's output has left douts[j]
-            dk = dkvq[j][:nk].view(B * T, Hkv, D)
-            dv = dkvq[j][nk:2 * nk].view(B * T, Hkv, D)
-            dq = dkvq[j][2 * nk:].view(B * T, Hq, D)
+            dk, dv, dq, dq_t = views[j]
             o = douts[j]
             for layer in range(NL):
                 if T == 1:
-                    caches[r].decode_step(layer, dk, dv, dq, douts[j], softmax_scale=wl.softmax_scale, stream=stream)
+                    caches[r].decode_step(layer, dk, dv, dq, o, softmax_scale=wl.softmax_scale, stream=stream)
                 else:
                     caches[r].append(layer, dk, dv, [T] * B, stream=stream)
-                    o = caches[r].decode_attention_multi(layer, dq.view(B, T, Hq, D), out_dtype=wl.kv_dtype,
+                    o = caches[r].decode_attention_multi(layer, dq_t, out_dtype=wl.kv_dtype,
                                                          softmax_scale=wl.softmax_scale, stream=stream)
                     o.record_stream(cstream)  # allocated per call on `stream`, read by the copy stream
             rc |= drv.record(ev_used[j], ms_) | drv.wait(cs, ev_used[j])
